@@ -1,0 +1,81 @@
+"""A second, pure-Python reader of the NWB1 blob format (test helper).
+
+Written from the format statement alone, in a different language and style
+from the oracle's C++ decoder, so that the encoder is checked against the
+format and not only against its own decoder.  Slow; small blobs only."""
+import struct
+
+import numpy as np
+
+
+def parse(blob: bytes):
+    b = bytes(blob)
+    (magic, version, hdr, lmax, rows, cols, tile_rows, tile_cols, tiles_r, tiles_c,
+     filler, zero, lens_off, index_off, tiles_off, total, coded_bits) = struct.unpack_from(
+        "<IIIIQQIIQQIIQQQQQ", b, 0)
+    assert magic == 0x3142574E and version == 1 and hdr == 128, "header"
+    assert total == len(b), "total bytes"
+    lens = list(b[lens_off:lens_off + 256])
+    n_tiles = tiles_r * tiles_c
+    index = struct.unpack_from(f"<{n_tiles + 1}I", b, index_off)
+    return dict(lmax=lmax, rows=rows, cols=cols, tile_rows=tile_rows, tile_cols=tile_cols,
+                tiles_r=tiles_r, tiles_c=tiles_c, filler=filler, lens=lens,
+                index=index, tiles_off=tiles_off, total=total, coded_bits=coded_bits)
+
+
+def codebook(lens):
+    """{bitstring: symbol} by the canonical rule: sort by (length, symbol)."""
+    order = sorted((l, s) for s, l in enumerate(lens) if l)
+    book, value, prev = {}, None, None
+    for l, s in order:
+        value = 0 if value is None else (value + 1) << (l - prev)
+        prev = l
+        book[format(value, f"0{l}b")] = s
+    return book
+
+
+def sequence_bits(area: bytes) -> str:
+    """Bit i of the sequence is bit 31 - i % 32 of little-endian word i // 32."""
+    out = []
+    for w in struct.unpack(f"<{len(area) // 4}I", area):
+        out.append(format(w, "032b"))
+    return "".join(out)
+
+
+def decode(blob: bytes) -> np.ndarray:
+    h = parse(blob)
+    b = bytes(blob)
+    book = codebook(h["lens"])
+    rows, cols, tr, tc = h["rows"], h["cols"], h["tile_rows"], h["tile_cols"]
+    out = np.zeros((rows, cols), dtype=np.uint16)
+    per_lane = 2 * tr * (tc // 64)
+    for u in range(h["tiles_r"] * h["tiles_c"]):
+        i, j = u % h["tiles_r"], u // h["tiles_r"]
+        c0 = h["tiles_off"] + 16 * h["index"][u]
+        c1 = h["tiles_off"] + 16 * h["index"][u + 1]
+        raw = b[c0:c0 + tr * tc]
+        lane_len = b[c0 + tr * tc:c0 + tr * tc + 32]
+        bits = sequence_bits(b[c0 + tr * tc + 32:c1])
+        start = 0
+        for t in range(32):
+            s = bits[start:start + 8 * lane_len[t]]
+            start += 8 * lane_len[t]
+            p = 0
+            for k in range(per_lane):
+                q = p + 1
+                while s[p:q] not in book:
+                    q += 1
+                    assert q - p <= h["lmax"], "no code"
+                sym = book[s[p:q]]
+                p = q
+                rb = raw[(k // 16) * 512 + 16 * t + k % 16]
+                r = (k // 2) % 8
+                c = 64 * (k // 16) + 2 * t + k % 2
+                row, col = i * tr + r, j * tc + c
+                if row < rows and col < cols:
+                    out[row, col] = ((rb >> 7) << 15) | (sym << 7) | (rb & 0x7F)
+                else:
+                    assert sym == h["filler"] and rb == 0, "filler"
+            assert set(s[p:]) <= {"0"} and len(s) - p < 8, "lane padding"
+        assert set(bits[start:]) <= {"0"}, "area padding"
+    return out
