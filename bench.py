@@ -1,0 +1,437 @@
+#!/usr/bin/env python3
+"""Benchmark: fused decode-GEMV over losslessly compressed BF16 weights on B200.
+
+One step = one nwc_gemv call (the fused decode-GEMV, the hot path) on the
+workload's matrix at the headline batch, with x and y resident in HBM.  Steps
+rotate over enough compressed copies of the matrix that the weights never sit in
+L2 (126 MB), and are replayed from a CUDA graph so host launch overhead stays
+out of the device time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--batch B]
+    python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun, one rank per GPU) are
+independent replicas: every rank runs the same per-GPU work, with no collective
+on the data path (weak scaling); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("fused decode-GEMV µs/call, effective GB/s & % of B200 HBM peak; "
+          "compression ratio")
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_nwc_b200", "csrc", "kernels.cu")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="nwc", choices=["nwc", "reference"])
+    ap.add_argument("--workload", default="attn_4096_outliers")
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--graph-calls", type=int, default=0,
+                    help="calls per captured graph (0 = one pass over the rotating copies)")
+    ap.add_argument("--no-cublas", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    return ap.parse_args()
+
+
+def measured_peaks() -> tuple[dict, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    with open(KERNEL_SOURCE, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profile_traffic(workload: str, batch: int) -> float | None:
+    """Per-launch DRAM bytes of the GEMV kernel from a committed ncu summary,
+    if that summary was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        data = json.load(f)
+    entry = data.get(f"{workload}/b{batch}")
+    if not entry or entry.get("kernel_sha") != kernel_source_hash():
+        return None
+    return float(entry["dram_bytes_per_launch"])
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = f"/tmp/nwc_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self) -> dict:
+        if not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm, smax, power, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                    power.append(float(parts[3]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "power_w_max": max(power) if power else None, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def dist_setup(n_gpus: int):
+    import torch
+    rank, world = 0, 1
+    if n_gpus > 1 or "RANK" in os.environ:
+        import datetime
+
+        import torch.distributed as dist
+        rank = int(os.environ.get("RANK", 0))
+        world = int(os.environ.get("WORLD_SIZE", 1))
+        local = int(os.environ.get("LOCAL_RANK", rank))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def cpu_baseline(workload: str, batch: int, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands (decode + FP64 GEMV), single-threaded, on a
+    bounded sample: whole calls on the workload's first matrix until the budget
+    is spent.  Reported in the bench metric's unit (effective GB/s)."""
+    import oracle
+    from lossless_bf16_weight_nwc_b200 import synth
+    wl = synth.workload(workload)
+    spec = wl.matrices[0]
+    rows = spec.rows
+    # Bounded sample: at most 4096 rows of the matrix (all of it for the
+    # benchmark workloads of 4096 rows or fewer).
+    rows = min(rows, 4096)
+    w = synth.matrix(spec, wl.seed, 0, rows)
+    x = synth.activations(wl.seed, batch, spec.cols)
+    blob = oracle.encode(w)
+    calls, t0 = 0, time.perf_counter()
+    while True:
+        wd = oracle.decode(blob)
+        oracle.gemv(wd, x)
+        calls += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or calls >= 50:
+            break
+    per_call = el / calls
+    gbs = 2.0 * rows * spec.cols / per_call / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "us_per_call": per_call * 1e6,
+            "sample": f"{calls} whole oracle calls (decode of the blob + FP64 GEMV, batch {batch}) "
+                      f"on {rows}x{spec.cols} rows of '{workload}' matrix 0, single thread"}
+
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", 0))
+    if rank != 0:
+        return
+    base = cpu_baseline(args.workload, args.batch)
+    step_s = base["us_per_call"] / 1e6
+    from lossless_bf16_weight_nwc_b200 import synth
+    spec = synth.workload(args.workload).matrices[0]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": None, "warmup": None, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": args.batch,
+                   "matrix": f"{spec.rows}x{spec.cols}"},
+        "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample", "value", "unit")},
+        "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    import torch
+
+    from lossless_bf16_weight_nwc_b200 import _lib, synth
+    rank, world = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.workload(args.workload)
+    spec = wl.matrices[0]
+    batch = args.batch
+    w = synth.matrix(spec, wl.seed)
+    x_host = synth.activations(wl.seed, batch, spec.cols)
+    first = _lib.CompressedMatrix.compress(w, device=dev)
+    image_bytes = first.device_bytes
+    copies = max(2, int(np.ceil(2.2 * L2_BYTES / image_bytes)))
+    mats = [first] + [_lib.CompressedMatrix(first.image.clone(), None, spec.rows, spec.cols,
+                                            first.blob_bytes) for _ in range(copies - 1)]
+    for m in mats[1:]:
+        m.handle = _lib.nwc_handle_from_device(m.image, m.image.numel())
+    x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
+    y = torch.empty((batch, spec.rows), dtype=torch.float32, device=dev)
+    ws_bytes = _lib.nwc_gemv_workspace_size(first.handle, batch)
+    ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    launches_per_call = (batch + 7) // 8
+    stream = torch.cuda.Stream(device=dev)
+
+    def call(m, s):
+        _lib.nwc_gemv(m.handle, x, y, batch, ws, ws_bytes, s.cuda_stream)
+
+    # Warm-up (also configures kernel attributes before capture).
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            call(mats[i % copies], stream)
+    stream.synchronize()
+
+    calls_per_graph = args.graph_calls or copies
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(calls_per_graph):
+            call(mats[i % copies], stream)
+    # Per-launch durations: one graph with an event pair around every call.
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(copies)]
+    g_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ev, stream=stream):
+        for i in range(copies):
+            ev[i][0].record(stream)
+            call(mats[i], stream)
+            ev[i][1].record(stream)
+    replays = max(1, args.steps // calls_per_graph)
+    steps = replays * calls_per_graph
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            g.replay()
+    stream.synchronize()
+
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(replays):
+                g.replay()
+            t1.record(stream)
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    clock = clocks.summary()
+
+    # Average launch duration of the GEMV kernel (event pairs on its stream).
+    durs = []
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, 2000 // copies)):
+            g_ev.replay()
+            stream.synchronize()
+            durs += [a.elapsed_time(b) for a, b in ev]
+    kernel_ms = statistics.mean(durs) / launches_per_call
+    ms_per_step = elapsed_ms / steps
+
+    # Parity spot check of the timed configuration.
+    y_ref = None
+    if rank == 0:
+        import oracle
+        rows_chk = np.arange(0, spec.rows, max(1, spec.rows // 256))
+        y_ref = oracle.gemv(w, x_host)[:, rows_chk]
+        call(mats[0], torch.cuda.current_stream())
+        y_gpu = y.double().cpu().numpy()[:, rows_chk]
+        wf = synth.bf16_bits_to_float(w[rows_chk]).astype(np.float64)
+        xf = synth.bf16_bits_to_float(x_host).astype(np.float64)
+        bound = 1e-2 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1)) * 2.0 ** -8
+        parity_ok = bool((np.abs(y_gpu - y_ref) <= bound).all())
+    else:
+        parity_ok = True
+
+    weight_bytes = 2.0 * spec.rows * spec.cols
+    x_bytes, y_bytes = 2.0 * batch * spec.cols, 4.0 * batch * spec.rows
+    alg_bytes = image_bytes + x_bytes + y_bytes
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    eff_gbs = world * weight_bytes / (ms_per_step * 1e-3) / 1e9
+    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+    traffic = profile_traffic(args.workload, batch)
+
+    # End to end through the public API with host buffers: pinned x in, y out.
+    e2e = None
+    if args.e2e_steps > 0:
+        xh = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).pin_memory()
+        yh = torch.empty((batch, spec.rows), dtype=torch.float32).pin_memory()
+        xd = torch.empty_like(x)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(args.e2e_steps):
+                xd.copy_(xh, non_blocking=True)
+                _lib.nwc_gemv(mats[i % copies].handle, xd, y, batch, ws, ws_bytes,
+                              stream.cuda_stream)
+                yh.copy_(y, non_blocking=True)
+            e1.record(stream)
+        stream.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
+        e2e = {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "us_per_call": e2e_ms * 1e3, "h2d_bytes_per_step": int(x_bytes),
+               "d2h_bytes_per_step": int(y_bytes)}
+
+    # Uncompressed BF16 cuBLAS GEMV on the same shape and L2 policy, for context.
+    cublas = None
+    if not args.no_cublas:
+        wt = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).to(dev)
+        n_w = max(2, int(np.ceil(2.2 * L2_BYTES / (weight_bytes))))
+        wts = [wt] + [wt.clone() for _ in range(n_w - 1)]
+        yb = torch.empty((batch, spec.rows), dtype=torch.bfloat16, device=dev)
+        with torch.cuda.stream(stream):
+            for i in range(20):
+                torch.matmul(x, wts[i % n_w].t(), out=yb)
+        stream.synchronize()
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb, stream=stream):
+            for i in range(n_w):
+                torch.matmul(x, wts[i % n_w].t(), out=yb)
+        reps = max(1, 2000 // n_w)
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gb.replay()
+            c0.record(stream)
+            for _ in range(reps):
+                gb.replay()
+            c1.record(stream)
+        stream.synchronize()
+        cb_ms = c0.elapsed_time(c1) / (reps * n_w)
+        cublas = {"us_per_call": cb_ms * 1e3,
+                  "effective_gbs": weight_bytes / (cb_ms * 1e-3) / 1e9,
+                  "speedup_nwc_vs_cublas": cb_ms / ms_per_step}
+        del wts
+
+    line = {
+        "metric": METRIC,
+        "value": eff_gbs,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "matrix": f"{spec.rows}x{spec.cols}",
+                   "batch": batch, "values": spec.kind,
+                   "l2": f"inputs larger than L2: {copies} rotating compressed copies "
+                         f"({copies * image_bytes / 2**20:.0f} MiB)",
+                   "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
+        "us_per_call": ms_per_step * 1e3,
+        "compression_ratio": weight_bytes / image_bytes,
+        "compressed_bytes": image_bytes,
+        "pct_hbm_peak_compressed": 100.0 * (image_bytes / (kernel_ms * 1e-3) / 1e9) / hbm,
+        "pct_of_8tbs_compressed": 100.0 * (image_bytes / (kernel_ms * 1e-3) / 1e9) / 8000.0,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic,
+                     "peak_source": f"{peak_src} hbm_gbs (copy)",
+                     "kernel": "gemv_kernel", "kernel_us": kernel_ms * 1e3,
+                     "algorithmic_bytes_per_launch": alg_bytes},
+        "clocks": clock,
+        "e2e": e2e,
+        "gpu_launches": steps * launches_per_call,
+        "parity_spot_check": parity_ok,
+        "cublas_bf16": cublas,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, batch)
+        line["cpu_baseline"].pop("us_per_call", None)
+    if rank == 0:
+        print(json.dumps(line))
+    # Release graphs before the process group.
+    del g, g_ev
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,181 @@
+/*
+ * nwc.h — C ABI of libnwc: lossless BF16 weight compression with a fused
+ * decode-GEMV for NVIDIA B200 (sm_100a).
+ *
+ * The method, with the passages that define it:
+ *   - A BF16 weight (sign 1 | exponent 8 | fraction 7; "Efficient ML #1 — Deep
+ *     Learning Data Types", §4) is split into two byte planes.  The exponent byte
+ *     is entropy-coded and the sign+fraction byte is stored raw ("Unweight: how we
+ *     compressed an LLM 22% without sacrificing quality", section "Compressing BF16
+ *     Weights"; "NWC — Neural Weight Compression", "How it works > Byte planes").
+ *   - The code is one optimal prefix code per matrix, with lengths limited to lmax
+ *     (12 by default: the decoder peeks 12 bits, as in "NWC", "How it works >
+ *     Prefix code instead of rANS").
+ *   - The matrix is cut into independently decodable tiles of 8 rows x tile_cols
+ *     columns, with one bit stream per lane ("NWC", "How it works > Fused kernel").
+ *   - The GPU decodes the tiles in registers and shared memory inside the
+ *     matrix-vector kernel; no decompressed weight is written to device memory
+ *     ("NWC", "Fused kernel"; "Unweight", "Direct GPU Decompression").
+ *
+ * Conventions for every call:
+ *   - Matrices are row-major [rows x cols] = [out_features x in_features].  BF16
+ *     values are passed as their uint16_t bit patterns.
+ *   - The caller owns all device memory.  A handle owns only host metadata and
+ *     refers to the caller's device buffer, which must outlive it.  No call frees
+ *     caller memory, and no device call allocates.
+ *   - Device calls are asynchronous on the given stream (0 = legacy default
+ *     stream).  They do not synchronize, except where a call says it does.
+ *   - Arguments are validated on the host before anything is launched.  Invalid
+ *     input returns an error code and launches nothing.
+ *   - Errors found on the device (a corrupt tile, a bounded wait that gave up) set
+ *     bits in a device error word; nwc_get_device_error() reads and clears it.
+ *   - Thread safety: distinct handles may be used concurrently.  Calls that share
+ *     a handle or a workspace must be ordered by the caller.
+ */
+#ifndef NWC_H
+#define NWC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nwc_stream_t; /* same object as cudaStream_t */
+typedef struct nwc_plan_s* nwc_plan_t;     /* opaque, host only           */
+typedef struct nwc_handle_s* nwc_handle_t; /* opaque, host metadata only  */
+
+typedef enum {
+  NWC_OK = 0,
+  NWC_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad alignment, ...     */
+  NWC_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. tile geometry) */
+  NWC_ERR_CUDA = 3,           /* a CUDA runtime call failed                     */
+  NWC_ERR_CORRUPT = 4,        /* a blob or device image does not parse          */
+  NWC_ERR_NOMEM = 5,          /* host allocation failed, or buffer too small    */
+  NWC_ERR_DEVICE_TIMEOUT = 6, /* the device error word reported a timeout       */
+  NWC_ERR_DEVICE_CORRUPT = 7  /* the device error word reported corrupt data    */
+} nwc_status;
+
+/* Plan options.  Set struct_size = sizeof(nwc_opts); pass NULL for the defaults
+ * (lmax = 12, tile_rows = 8, tile_cols = 512, threads = 0 meaning all cores).
+ * lmax must be in [1, 12] and at least ceil(log2(distinct exponents)).
+ * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512. */
+typedef struct {
+  uint32_t struct_size;
+  uint32_t lmax;
+  uint32_t tile_rows;
+  uint32_t tile_cols;
+  uint32_t threads; /* host encoder threads; 0 = hardware concurrency */
+} nwc_opts;
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int nwc_version(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* nwc_status_string(nwc_status status);
+
+/* ---- Host encoder ------------------------------------------------------- */
+
+/* Histogram of the exponent bytes, the length-limited canonical code, and the
+ * exact compressed sizes.  w_host holds rows x cols BF16 patterns, row-major.
+ * It is read, not retained.  rows, cols >= 1.  On success *out_plan owns host
+ * memory; free it with nwc_plan_destroy.
+ * Errors: INVALID_ARG (null, sizes, options, > 64 GiB of tile data), NOMEM. */
+nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols,
+                    const nwc_opts* opts, nwc_plan_t* out_plan);
+
+/* Exact sizes for a plan.  *device_bytes is what nwc_compress needs in device
+ * memory: the serialisable blob plus a derived 16 KiB decode table, at a
+ * 256-byte aligned offset.  *host_blob_bytes is the size of the serialisable
+ * blob (nwc_compress_host).  Either pointer may be NULL. */
+nwc_status nwc_plan_size(nwc_plan_t plan, uint64_t* device_bytes,
+                         uint64_t* host_blob_bytes);
+
+/* Encode w_host (the same matrix given to nwc_plan) and upload it into the
+ * caller's device buffer d_buf (>= device_bytes, 256-byte aligned) on `stream`.
+ * The upload is asynchronous: w_host may be reused when the call returns,
+ * but d_buf must not be read before the stream reaches this point.  On success
+ * *out_handle refers to d_buf.
+ * Errors: INVALID_ARG (null, d_bytes too small, misaligned d_buf), NOMEM,
+ * CUDA. */
+nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf,
+                        uint64_t d_bytes, nwc_stream_t stream,
+                        nwc_handle_t* out_handle);
+
+/* Encode into a host buffer (>= host_blob_bytes).  The bytes are the
+ * serialisable "NWB1" blob. */
+nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob,
+                             uint64_t blob_bytes);
+
+/* Bytes of device memory needed to upload an existing blob (blob + table). */
+nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes,
+                                 uint64_t* device_bytes);
+
+/* Validate a host blob, upload it into d_buf, and build its decode table.  The
+ * call is synchronous: it returns after the copies finish.
+ * Errors: CORRUPT (header, code lengths or index do not parse), INVALID_ARG,
+ * CUDA. */
+nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
+                           uint64_t d_bytes, nwc_stream_t stream,
+                           nwc_handle_t* out_handle);
+
+/* Build a handle for a device buffer that already holds a device image (from
+ * nwc_compress or nwc_upload_blob, possibly copied elsewhere).  The call is
+ * synchronous: it reads the header, code lengths and index back to the host.
+ * Errors: CORRUPT, INVALID_ARG, CUDA. */
+nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes,
+                                  nwc_handle_t* out_handle);
+
+/* ---- Device kernels ---------------------------------------------------- */
+
+/* Bit-exact decompression ("NWC", "How it works > Dequantization and embedding
+ * lookup": the same decoder writes BF16).  d_w_out: device, rows x cols BF16,
+ * row-major, 4-byte aligned.  Asynchronous on `stream`.
+ * Errors: INVALID_ARG, CUDA (launch). */
+nwc_status nwc_decompress(nwc_handle_t handle, uint16_t* d_w_out, nwc_stream_t stream);
+
+/* Bytes of scratch that nwc_gemv needs for this handle and batch; 0 when the
+ * matrix has a single column tile.  The scratch holds one FP32 partial sum per
+ * (column tile, batch row, output row) plus one u32 counter per row tile; it
+ * makes the split-K reduction deterministic (fixed summation order). */
+nwc_status nwc_gemv_workspace_size(nwc_handle_t handle, int32_t batch,
+                                   uint64_t* bytes);
+
+/* y[b][n] = sum_k W[n][k] * x[b][k], for b < batch, n < rows, k < cols.
+ *   d_x: device, BF16 [batch x cols], row-major, 4-byte aligned, cols even.
+ *   d_y: device, FP32 [batch x rows], row-major (overwritten, not accumulated).
+ *   batch in [1, 64].
+ *   d_workspace: device, >= nwc_gemv_workspace_size bytes, 16-byte aligned,
+ *     zero-filled before its first use.  Every completed call leaves the counter
+ *     area zero again, so one workspace serves any number of ordered calls.  Two
+ *     calls that overlap on the GPU must not share a workspace.  It may be NULL
+ *     when the size is 0.
+ * Products and sums are in FP32; the result is the same bit pattern on every
+ * run.  Asynchronous on `stream`.
+ * Errors: INVALID_ARG (null, batch, alignment, odd cols, workspace too small),
+ * UNSUPPORTED, CUDA (launch). */
+nwc_status nwc_gemv(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
+                    int32_t batch, void* d_workspace, uint64_t workspace_bytes,
+                    nwc_stream_t stream);
+
+/* ---- Inspection, errors, teardown ------------------------------------- */
+
+/* Any pointer may be NULL.  *blob_bytes is the serialisable part; *device_bytes
+ * is the whole device image (blob + decode table). */
+nwc_status nwc_handle_info(nwc_handle_t handle, int64_t* rows, int64_t* cols,
+                           uint64_t* blob_bytes, uint64_t* device_bytes);
+
+/* Synchronizes `stream`, then reads and clears the device error word of the
+ * current device.  Returns OK, DEVICE_TIMEOUT or DEVICE_CORRUPT (timeout
+ * wins), or CUDA.  *word (optional) receives the raw bits. */
+nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word);
+
+/* Free host metadata.  NULL is accepted.  Device memory is never freed. */
+void nwc_plan_destroy(nwc_plan_t plan);
+void nwc_handle_destroy(nwc_handle_t handle);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NWC_H */

@@ -1,0 +1,278 @@
+"""ctypes binding of libnwc (include/nwc.h): argument marshalling only.
+
+Every function of the C ABI is exposed under the same name; each step of the
+path runs in libnwc's kernels.  PyTorch supplies device memory and streams.
+There is no fallback: if libnwc.so is missing or cannot be loaded, import of
+this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnwc.so")
+
+NWC_OK = 0
+STATUS = {0: "NWC_OK", 1: "NWC_ERR_INVALID_ARG", 2: "NWC_ERR_UNSUPPORTED", 3: "NWC_ERR_CUDA",
+          4: "NWC_ERR_CORRUPT", 5: "NWC_ERR_NOMEM", 6: "NWC_ERR_DEVICE_TIMEOUT",
+          7: "NWC_ERR_DEVICE_CORRUPT"}
+
+
+class NwcError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        super().__init__(f"{call} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+class nwc_opts(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("lmax", ctypes.c_uint32),
+                ("tile_rows", ctypes.c_uint32), ("tile_cols", ctypes.c_uint32),
+                ("threads", ctypes.c_uint32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libnwc.so not built ({LIB_PATH}); run "
+                           "`python -m lossless_bf16_weight_nwc_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    c = ctypes
+    vp, u64, i64, i32 = c.c_void_p, c.c_uint64, c.c_int64, c.c_int32
+    sig = {
+        "nwc_version": ([], c.c_int),
+        "nwc_status_string": ([c.c_int], c.c_char_p),
+        "nwc_plan": ([vp, i64, i64, c.POINTER(nwc_opts), c.POINTER(vp)], c.c_int),
+        "nwc_plan_size": ([vp, c.POINTER(u64), c.POINTER(u64)], c.c_int),
+        "nwc_compress": ([vp, vp, vp, u64, vp, c.POINTER(vp)], c.c_int),
+        "nwc_compress_host": ([vp, vp, vp, u64], c.c_int),
+        "nwc_blob_device_bytes": ([vp, u64, c.POINTER(u64)], c.c_int),
+        "nwc_upload_blob": ([vp, u64, vp, u64, vp, c.POINTER(vp)], c.c_int),
+        "nwc_handle_from_device": ([vp, u64, c.POINTER(vp)], c.c_int),
+        "nwc_decompress": ([vp, vp, vp], c.c_int),
+        "nwc_gemv_workspace_size": ([vp, i32, c.POINTER(u64)], c.c_int),
+        "nwc_gemv": ([vp, vp, vp, i32, vp, u64, vp], c.c_int),
+        "nwc_handle_info": ([vp, c.POINTER(i64), c.POINTER(i64), c.POINTER(u64),
+                             c.POINTER(u64)], c.c_int),
+        "nwc_get_device_error": ([vp, c.POINTER(c.c_uint32)], c.c_int),
+        "nwc_plan_destroy": ([vp], None),
+        "nwc_handle_destroy": ([vp], None),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+LIB = _load()
+EXPORTED = ("nwc_version", "nwc_status_string", "nwc_plan", "nwc_plan_size", "nwc_compress",
+            "nwc_compress_host", "nwc_blob_device_bytes", "nwc_upload_blob",
+            "nwc_handle_from_device", "nwc_decompress", "nwc_gemv_workspace_size", "nwc_gemv",
+            "nwc_handle_info", "nwc_get_device_error", "nwc_plan_destroy", "nwc_handle_destroy")
+
+
+def _check(status: int, call: str) -> None:
+    if status != NWC_OK:
+        raise NwcError(status, call)
+
+
+def _stream(stream) -> int | None:
+    """A torch.cuda.Stream, a raw handle, or None (the current torch stream)."""
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t) -> int:
+    return t.data_ptr() if hasattr(t, "data_ptr") else int(t)
+
+
+# ---- the C ABI, one Python function per entry point ------------------------
+
+def nwc_version() -> int:
+    return LIB.nwc_version()
+
+
+def nwc_plan(w_host: np.ndarray, lmax: int = 12, tile_cols: int = 512, threads: int = 0):
+    w = np.ascontiguousarray(w_host, dtype=np.uint16)
+    rows, cols = w.shape
+    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads)
+    plan = ctypes.c_void_p()
+    _check(LIB.nwc_plan(w.ctypes.data, rows, cols, ctypes.byref(opts), ctypes.byref(plan)),
+           "nwc_plan")
+    return plan
+
+
+def nwc_plan_size(plan) -> tuple[int, int]:
+    dev, host = ctypes.c_uint64(), ctypes.c_uint64()
+    _check(LIB.nwc_plan_size(plan, ctypes.byref(dev), ctypes.byref(host)), "nwc_plan_size")
+    return dev.value, host.value
+
+
+def nwc_compress(plan, w_host: np.ndarray, d_buf, d_bytes: int, stream=None):
+    w = np.ascontiguousarray(w_host, dtype=np.uint16)
+    h = ctypes.c_void_p()
+    _check(LIB.nwc_compress(plan, w.ctypes.data, _ptr(d_buf), d_bytes, _stream(stream),
+                            ctypes.byref(h)), "nwc_compress")
+    return h
+
+
+def nwc_compress_host(plan, w_host: np.ndarray) -> np.ndarray:
+    w = np.ascontiguousarray(w_host, dtype=np.uint16)
+    _, n = nwc_plan_size(plan)
+    blob = np.zeros(n, dtype=np.uint8)
+    _check(LIB.nwc_compress_host(plan, w.ctypes.data, blob.ctypes.data, n), "nwc_compress_host")
+    return blob
+
+
+def nwc_blob_device_bytes(blob: np.ndarray) -> int:
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    out = ctypes.c_uint64()
+    _check(LIB.nwc_blob_device_bytes(blob.ctypes.data, blob.size, ctypes.byref(out)),
+           "nwc_blob_device_bytes")
+    return out.value
+
+
+def nwc_upload_blob(blob: np.ndarray, d_buf, d_bytes: int, stream=None):
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    h = ctypes.c_void_p()
+    _check(LIB.nwc_upload_blob(blob.ctypes.data, blob.size, _ptr(d_buf), d_bytes,
+                               _stream(stream), ctypes.byref(h)), "nwc_upload_blob")
+    return h
+
+
+def nwc_handle_from_device(d_buf, d_bytes: int):
+    h = ctypes.c_void_p()
+    _check(LIB.nwc_handle_from_device(_ptr(d_buf), d_bytes, ctypes.byref(h)),
+           "nwc_handle_from_device")
+    return h
+
+
+def nwc_decompress(handle, d_w_out, stream=None) -> None:
+    _check(LIB.nwc_decompress(handle, _ptr(d_w_out), _stream(stream)), "nwc_decompress")
+
+
+def nwc_gemv_workspace_size(handle, batch: int) -> int:
+    out = ctypes.c_uint64()
+    _check(LIB.nwc_gemv_workspace_size(handle, batch, ctypes.byref(out)),
+           "nwc_gemv_workspace_size")
+    return out.value
+
+
+def nwc_gemv(handle, d_x, d_y, batch: int, d_workspace=None, workspace_bytes: int = 0,
+             stream=None) -> None:
+    ws = 0 if d_workspace is None else _ptr(d_workspace)
+    _check(LIB.nwc_gemv(handle, _ptr(d_x), _ptr(d_y), batch, ws, workspace_bytes,
+                        _stream(stream)), "nwc_gemv")
+
+
+def nwc_handle_info(handle) -> dict:
+    r, c = ctypes.c_int64(), ctypes.c_int64()
+    b, d = ctypes.c_uint64(), ctypes.c_uint64()
+    _check(LIB.nwc_handle_info(handle, ctypes.byref(r), ctypes.byref(c), ctypes.byref(b),
+                               ctypes.byref(d)), "nwc_handle_info")
+    return {"rows": r.value, "cols": c.value, "blob_bytes": b.value, "device_bytes": d.value}
+
+
+def nwc_get_device_error(stream=None) -> tuple[int, int]:
+    """(status, raw word); synchronizes the stream."""
+    w = ctypes.c_uint32()
+    st = LIB.nwc_get_device_error(_stream(stream), ctypes.byref(w))
+    return st, w.value
+
+
+def nwc_plan_destroy(plan) -> None:
+    LIB.nwc_plan_destroy(plan)
+
+
+def nwc_handle_destroy(handle) -> None:
+    LIB.nwc_handle_destroy(handle)
+
+
+# ---- convenience object over the same calls ---------------------------------
+
+class CompressedMatrix:
+    """A BF16 matrix held compressed in device memory that torch allocated.
+
+    Owns the device image (a uint8 CUDA tensor), the handle, and a GEMV
+    workspace that grows on demand.  Calls run on the current torch stream."""
+
+    def __init__(self, image, handle, rows: int, cols: int, blob_bytes: int):
+        self.image = image
+        self.handle = handle
+        self.rows, self.cols = rows, cols
+        self.blob_bytes = blob_bytes
+        self.device_bytes = image.numel()
+        self._ws = None
+
+    @classmethod
+    def compress(cls, w_host: np.ndarray, device="cuda", lmax: int = 12, tile_cols: int = 512,
+                 threads: int = 0, stream=None) -> "CompressedMatrix":
+        import torch
+        plan = nwc_plan(w_host, lmax=lmax, tile_cols=tile_cols, threads=threads)
+        try:
+            dev_bytes, blob_bytes = nwc_plan_size(plan)
+            image = torch.empty(dev_bytes, dtype=torch.uint8, device=device)
+            with torch.cuda.device(image.device):
+                h = nwc_compress(plan, w_host, image, dev_bytes, stream)
+        finally:
+            nwc_plan_destroy(plan)
+        return cls(image, h, w_host.shape[0], w_host.shape[1], blob_bytes)
+
+    @classmethod
+    def from_blob(cls, blob: np.ndarray, device="cuda", stream=None) -> "CompressedMatrix":
+        import torch
+        n = nwc_blob_device_bytes(blob)
+        image = torch.empty(n, dtype=torch.uint8, device=device)
+        with torch.cuda.device(image.device):
+            h = nwc_upload_blob(blob, image, n, stream)
+        info = nwc_handle_info(h)
+        return cls(image, h, info["rows"], info["cols"], info["blob_bytes"])
+
+    @property
+    def ratio(self) -> float:
+        """Uncompressed BF16 bytes / device bytes (blob + decode table)."""
+        return 2.0 * self.rows * self.cols / self.device_bytes
+
+    def workspace(self, batch: int):
+        import torch
+        need = nwc_gemv_workspace_size(self.handle, batch)
+        if need == 0:
+            return None, 0
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(need, dtype=torch.uint8, device=self.image.device)
+        return self._ws, self._ws.numel()
+
+    def decompress(self, out=None, stream=None):
+        import torch
+        if out is None:
+            out = torch.empty((self.rows, self.cols), dtype=torch.bfloat16,
+                              device=self.image.device)
+        nwc_decompress(self.handle, out, stream)
+        return out
+
+    def gemv(self, x, y=None, stream=None):
+        """y = x @ W^T for x BF16 [batch, cols] -> FP32 [batch, rows]."""
+        import torch
+        assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape[-1] == self.cols
+        xb = x.reshape(-1, self.cols)
+        batch = xb.shape[0]
+        if y is None:
+            y = torch.empty((batch, self.rows), dtype=torch.float32, device=x.device)
+        ws, ws_bytes = self.workspace(batch)
+        nwc_gemv(self.handle, xb, y, batch, ws, ws_bytes, stream)
+        return y
+
+    def close(self) -> None:
+        if self.handle is not None:
+            nwc_handle_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

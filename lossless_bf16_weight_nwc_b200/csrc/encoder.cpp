@@ -1,0 +1,412 @@
+// encoder.cpp — host encoder of libnwc (multi-threaded C++).
+//
+// Steps, in the pages' order:
+//  1. Byte planes: exponent byte s = bits 14..7 is coded, raw byte r = sign << 7
+//     | fraction is stored ("Unweight", "Compressing BF16 Weights"; "NWC", "How
+//     it works > Byte planes").
+//  2. Histogram of s over the matrix plus the filler positions of ragged tiles.
+//  3. Optimal code lengths limited to lmax (package-merge, Larmore & Hirschberg
+//     1990), assigned canonically.  Ties: leaves by (count, symbol); a leaf
+//     precedes a package of equal weight; codes in (length, symbol) order.  The
+//     filler is the most frequent exponent (smallest symbol on a tie).
+//  4. Tiles of 8 rows x tile_cols with one MSB-first bit stream per lane ("NWC",
+//     "How it works > Fused kernel"), an offset index, and the raw plane laid
+//     out so that one 128-bit load gives a lane 16 of its raw bytes.
+//  5. A 4096-entry decode table for the GPU ("NWC", "Prefix code instead of
+//     rANS": a 12-bit peek yields up to two complete codes).
+#include <algorithm>
+#include <cstring>
+#include <functional>
+#include <thread>
+#include <vector>
+
+#include "nwc_internal.h"
+
+namespace nwc {
+
+unsigned hardware_threads(uint32_t requested) {
+  if (requested) return requested;
+  unsigned n = std::thread::hardware_concurrency();
+  return n ? n : 1;
+}
+
+namespace {
+
+// Runs f(begin, end) over [0, n) split into `threads` contiguous parts.
+void parallel_for(int64_t n, unsigned threads, const std::function<void(int64_t, int64_t)>& f) {
+  if (n <= 0) return;
+  unsigned parts = (unsigned)std::min<int64_t>(threads, n);
+  if (parts <= 1) {
+    f(0, n);
+    return;
+  }
+  std::vector<std::thread> pool;
+  for (unsigned p = 0; p < parts; ++p) {
+    int64_t b = n * p / parts, e = n * (p + 1) / parts;
+    pool.emplace_back([&f, b, e] { f(b, e); });
+  }
+  for (auto& t : pool) t.join();
+}
+
+inline uint8_t exponent_byte(uint16_t w) { return (uint8_t)(w >> 7); }
+inline uint8_t raw_byte(uint16_t w) { return (uint8_t)(((w >> 8) & 0x80) | (w & 0x7F)); }
+
+// Symbol (exponent byte) of tile element (r, c); the filler outside the matrix.
+struct TileView {
+  const uint16_t* w;
+  int64_t rows, cols, row0, col0;
+  uint8_t filler;
+  inline bool inside(int r, int c) const { return row0 + r < rows && col0 + c < cols; }
+  inline uint16_t at(int r, int c) const { return w[(row0 + r) * cols + col0 + c]; }
+};
+
+// Bits of each lane's stream in tile u.
+void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t bits[kLanes]) {
+  const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
+  TileView v{w, p.rows, p.cols, i * kTileRows, j * (int64_t)p.tile_cols, (uint8_t)p.filler};
+  const int groups = (int)p.tile_cols / 64;
+  for (int t = 0; t < kLanes; ++t) bits[t] = 0;
+  for (int r = 0; r < kTileRows; ++r) {
+    for (int c = 0; c < (int)p.tile_cols; ++c) {
+      const int t = (c % 64) / 2;
+      const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
+      bits[t] += p.len[s];
+    }
+  }
+  (void)groups;
+}
+
+uint32_t stream_bytes_of(const uint32_t bits[kLanes]) {
+  uint32_t total = 0;
+  for (int t = 0; t < kLanes; ++t) total += (bits[t] + 7) / 8;
+  return total;
+}
+
+}  // namespace
+
+bool code_lengths(const uint64_t cnt[256], uint32_t lmax, uint8_t len[256]) {
+  // Package-merge over an arena of nodes: a node is a leaf (symbol) or a
+  // package of two earlier nodes.  The code length of a symbol is the number of
+  // times its leaf occurs below the 2n - 2 cheapest items of the last list.
+  struct Node {
+    uint64_t weight;
+    int32_t a, b;  // children; a < 0 encodes leaf symbol -a - 1
+  };
+  std::memset(len, 0, 256);
+  std::vector<int> syms;
+  for (int s = 0; s < 256; ++s)
+    if (cnt[s]) syms.push_back(s);
+  const size_t n = syms.size();
+  if (n == 0) return false;
+  if (n == 1) {
+    len[syms[0]] = 1;
+    return true;
+  }
+  if (lmax > 30 || n > (size_t(1) << lmax)) return false;
+  std::stable_sort(syms.begin(), syms.end(), [&](int x, int y) {
+    return cnt[x] != cnt[y] ? cnt[x] < cnt[y] : x < y;
+  });
+  std::vector<Node> arena;
+  std::vector<int32_t> leaves;
+  for (int s : syms) {
+    leaves.push_back((int32_t)arena.size());
+    arena.push_back({cnt[s], -s - 1, -1});
+  }
+  std::vector<int32_t> cur = leaves, next;
+  for (uint32_t level = lmax; level > 1; --level) {
+    next.clear();
+    size_t li = 0, pi = 0;
+    const size_t packages = cur.size() / 2;
+    // Merge leaves with packages of consecutive pairs of `cur`, creating each
+    // package node when it is taken.
+    std::vector<int32_t> pk(packages);
+    for (size_t q = 0; q < packages; ++q) {
+      pk[q] = (int32_t)arena.size();
+      arena.push_back({arena[cur[2 * q]].weight + arena[cur[2 * q + 1]].weight,
+                       cur[2 * q], cur[2 * q + 1]});
+    }
+    while (li < leaves.size() || pi < packages) {
+      if (pi >= packages ||
+          (li < leaves.size() && arena[leaves[li]].weight <= arena[pk[pi]].weight))
+        next.push_back(leaves[li++]);
+      else
+        next.push_back(pk[pi++]);
+    }
+    cur.swap(next);
+  }
+  if (cur.size() < 2 * n - 2) return false;
+  std::vector<int32_t> stack;
+  std::vector<uint32_t> uses(256, 0);
+  for (size_t q = 0; q < 2 * n - 2; ++q) {
+    stack.push_back(cur[q]);
+    while (!stack.empty()) {
+      const Node& nd = arena[stack.back()];
+      stack.pop_back();
+      if (nd.a < 0) {
+        uses[-nd.a - 1] += 1;
+      } else {
+        stack.push_back(nd.a);
+        stack.push_back(nd.b);
+      }
+    }
+  }
+  for (int s = 0; s < 256; ++s) len[s] = (uint8_t)uses[s];
+  return true;
+}
+
+void canonical_codes(const uint8_t len[256], uint32_t code[256]) {
+  // Count codes per length, then the first code of each length (shorter codes
+  // are prefixes of nothing longer), then hand out codes in symbol order.
+  uint32_t per_len[33] = {}, first[33] = {};
+  for (int s = 0; s < 256; ++s)
+    if (len[s]) per_len[len[s]] += 1;
+  uint32_t c = 0;
+  for (int l = 1; l <= 32; ++l) {
+    c = (c + per_len[l - 1]) << 1;
+    first[l] = c;
+  }
+  for (int s = 0; s < 256; ++s) code[s] = len[s] ? first[len[s]]++ : 0;
+}
+
+void build_decode_table(const uint8_t len[256], uint32_t table[kTableEntries]) {
+  uint32_t code[256];
+  canonical_codes(len, code);
+  // sym[l][v]: symbol with code v of length l, or -1.
+  std::vector<std::vector<int16_t>> sym(kPeekBits + 1);
+  for (int l = 1; l <= kPeekBits; ++l) sym[l].assign(size_t(1) << l, -1);
+  for (int s = 0; s < 256; ++s)
+    if (len[s] >= 1 && len[s] <= kPeekBits) sym[len[s]][code[s]] = (int16_t)s;
+  auto first_code = [&](uint32_t bits, int avail, int* s_out, int* l_out) {
+    for (int l = 1; l <= avail; ++l) {
+      const int s = sym[l][bits >> (kPeekBits - l)];
+      if (s >= 0) {
+        *s_out = s;
+        *l_out = l;
+        return true;
+      }
+    }
+    return false;
+  };
+  for (uint32_t v = 0; v < (uint32_t)kTableEntries; ++v) {
+    int s0, l0, s1, l1;
+    if (!first_code(v, kPeekBits, &s0, &l0)) {
+      table[v] = 2u | kEntryInvalid;  // consume two bits, emit exponent 0
+      continue;
+    }
+    const uint32_t rest = (v << l0) & (kTableEntries - 1);
+    uint32_t e = ((uint32_t)s0 << 7) | ((uint32_t)l0 << kEntryLen0Shift);
+    if (first_code(rest, kPeekBits - l0, &s1, &l1))
+      e |= (uint32_t)(l0 + l1) | ((uint32_t)s1 << 23);
+    else
+      e |= (uint32_t)l0 | kEntrySingle;
+    table[v] = e;
+  }
+}
+
+int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
+               uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* p) {
+  p->rows = rows;
+  p->cols = cols;
+  p->tile_rows = tile_rows;
+  p->tile_cols = tile_cols;
+  p->lmax = lmax;
+  p->threads = hardware_threads(threads);
+  p->tiles_r = (rows + kTileRows - 1) / kTileRows;
+  p->tiles_c = (cols + tile_cols - 1) / tile_cols;
+  p->tiles = p->tiles_r * p->tiles_c;
+
+  // Histogram, one partial per thread.
+  const unsigned nt = p->threads;
+  std::vector<std::vector<uint64_t>> part(nt, std::vector<uint64_t>(256, 0));
+  {
+    std::vector<std::thread> pool;
+    for (unsigned q = 0; q < nt; ++q) {
+      pool.emplace_back([&, q] {
+        const int64_t b = rows * q / nt, e = rows * (q + 1) / nt;
+        uint64_t* h = part[q].data();
+        for (int64_t r = b; r < e; ++r) {
+          const uint16_t* row = w + r * cols;
+          for (int64_t c = 0; c < cols; ++c) h[exponent_byte(row[c])] += 1;
+        }
+      });
+    }
+    for (auto& t : pool) t.join();
+  }
+  uint64_t cnt[256] = {};
+  for (unsigned q = 0; q < nt; ++q)
+    for (int s = 0; s < 256; ++s) cnt[s] += part[q][s];
+  uint32_t filler = 0;
+  for (uint32_t s = 1; s < 256; ++s)
+    if (cnt[s] > cnt[filler]) filler = s;
+  p->filler = filler;
+  cnt[filler] += (uint64_t)(p->tiles_r * kTileRows) * (uint64_t)(p->tiles_c * tile_cols) -
+                 (uint64_t)rows * (uint64_t)cols;
+  if (!code_lengths(cnt, lmax, p->len)) return -1;
+  canonical_codes(p->len, p->code);
+  p->coded_bits = 0;
+  for (int s = 0; s < 256; ++s) p->coded_bits += cnt[s] * p->len[s];
+
+  // Chunk sizes -> index.
+  std::vector<uint32_t> chunk16((size_t)p->tiles);
+  parallel_for(p->tiles, nt, [&](int64_t b, int64_t e) {
+    uint32_t bits[kLanes];
+    for (int64_t u = b; u < e; ++u) {
+      lane_bits(*p, w, u, bits);
+      const uint32_t bytes = raw_bytes(tile_cols) + kLanes + (uint32_t)round_up(stream_bytes_of(bits), 16);
+      chunk16[(size_t)u] = bytes / 16;
+    }
+  });
+  p->index.assign((size_t)p->tiles + 1, 0);
+  uint64_t acc = 0;
+  for (int64_t u = 0; u < p->tiles; ++u) {
+    p->index[(size_t)u] = (uint32_t)acc;
+    acc += chunk16[(size_t)u];
+    if (acc > 0xFFFFFFFFull) return -2;  // more than 64 GiB of tile data
+  }
+  p->index[(size_t)p->tiles] = (uint32_t)acc;
+  p->tiles_off = round_up(kIndexOffset + 4ull * (uint64_t)(p->tiles + 1), 256);
+  p->blob_bytes = p->tiles_off + 16ull * acc;
+  p->table_off = round_up(p->blob_bytes, 256);
+  p->device_bytes = p->table_off + kTableBytes;
+  return 0;
+}
+
+void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
+  BlobHeader h;
+  std::memset(&h, 0, sizeof(h));
+  h.magic = kMagic;
+  h.version = kVersion;
+  h.header_bytes = kHeaderBytes;
+  h.lmax = p.lmax;
+  h.rows = (uint64_t)p.rows;
+  h.cols = (uint64_t)p.cols;
+  h.tile_rows = kTileRows;
+  h.tile_cols = p.tile_cols;
+  h.tiles_r = (uint64_t)p.tiles_r;
+  h.tiles_c = (uint64_t)p.tiles_c;
+  h.filler = p.filler;
+  h.lens_off = kLensOffset;
+  h.index_off = kIndexOffset;
+  h.tiles_off = p.tiles_off;
+  h.total_bytes = p.blob_bytes;
+  h.coded_bits = p.coded_bits;
+  std::memset(blob, 0, p.tiles_off);
+  std::memcpy(blob, &h, sizeof(h));
+  std::memcpy(blob + kLensOffset, p.len, 256);
+  std::memcpy(blob + kIndexOffset, p.index.data(), 4 * p.index.size());
+
+  const uint32_t groups = p.tile_cols / 64;
+  const uint32_t raw_n = raw_bytes(p.tile_cols);
+  parallel_for(p.tiles, p.threads, [&](int64_t b, int64_t e) {
+    std::vector<uint8_t> seq;  // big-endian bytes of the stream run
+    for (int64_t u = b; u < e; ++u) {
+      const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
+      TileView v{w, p.rows, p.cols, i * kTileRows, j * (int64_t)p.tile_cols, (uint8_t)p.filler};
+      uint8_t* chunk = blob + p.tiles_off + 16ull * p.index[(size_t)u];
+      const uint32_t chunk_bytes = 16u * (p.index[(size_t)u + 1] - p.index[(size_t)u]);
+      const uint32_t area = chunk_bytes - raw_n - kLanes;
+      uint8_t* raw = chunk;
+      uint8_t* lane_len = chunk + raw_n;
+      uint8_t* words = chunk + raw_n + kLanes;
+      seq.assign(area, 0);
+      uint32_t out = 0;
+      for (int t = 0; t < kLanes; ++t) {
+        const uint32_t lane_start = out;
+        uint32_t accb = 0;  // pending bits, right-aligned
+        int nacc = 0;
+        for (uint32_t g = 0; g < groups; ++g) {
+          for (int r = 0; r < kTileRows; ++r) {
+            for (int hh = 0; hh < 2; ++hh) {
+              const int c = (int)(64 * g) + 2 * t + hh;
+              const int k = (int)(16 * g) + 2 * r + hh;
+              uint8_t s = v.filler, rb = 0;
+              if (v.inside(r, c)) {
+                const uint16_t x = v.at(r, c);
+                s = exponent_byte(x);
+                rb = raw_byte(x);
+              }
+              raw[(k / 16) * 512 + 16 * t + (k % 16)] = rb;
+              accb = (accb << p.len[s]) | p.code[s];
+              nacc += p.len[s];
+              while (nacc >= 8) {
+                seq[out++] = (uint8_t)(accb >> (nacc - 8));
+                nacc -= 8;
+              }
+              accb &= (1u << nacc) - 1u;
+            }
+          }
+        }
+        if (nacc > 0) seq[out++] = (uint8_t)(accb << (8 - nacc));
+        lane_len[t] = (uint8_t)(out - lane_start);
+      }
+      // Little-endian words with the earliest bit in bit 31.
+      for (uint32_t q = 0; q < area; q += 4) {
+        words[q + 0] = seq[q + 3];
+        words[q + 1] = seq[q + 2];
+        words[q + 2] = seq[q + 1];
+        words[q + 3] = seq[q + 0];
+      }
+    }
+  });
+}
+
+bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* hd,
+                const uint8_t** lens_out) {
+  if (!blob || head_bytes < kHeaderBytes + 256 || head_bytes > bytes) return false;
+  BlobHeader h;
+  std::memcpy(&h, blob, sizeof(h));
+  if (h.magic != kMagic || h.version != kVersion || h.header_bytes != kHeaderBytes) return false;
+  if (h.lmax < 1 || h.lmax > (uint32_t)kMaxLmax || h.tile_rows != (uint32_t)kTileRows) return false;
+  if (h.tile_cols < 64 || h.tile_cols > (uint32_t)kMaxTileCols || h.tile_cols % 64) return false;
+  if (h.rows < 1 || h.cols < 1 || h.rows > (1ull << 40) || h.cols > (1ull << 40)) return false;
+  if (h.tiles_r != (h.rows + 7) / 8 || h.tiles_c != (h.cols + h.tile_cols - 1) / h.tile_cols)
+    return false;
+  if (h.lens_off != kLensOffset || h.index_off != kIndexOffset || h.filler > 255) return false;
+  const uint64_t tiles = h.tiles_r * h.tiles_c;
+  if (h.tiles_off != round_up(kIndexOffset + 4 * (tiles + 1), 256)) return false;
+  if (h.total_bytes != bytes || h.tiles_off > head_bytes) return false;
+  const uint8_t* lens = blob + kLensOffset;
+  double kraft = 0;
+  for (int s = 0; s < 256; ++s) {
+    if (lens[s] > h.lmax) return false;
+    if (lens[s]) kraft += 1.0 / double(1u << lens[s]);
+  }
+  if (kraft > 1.0 || lens[h.filler] == 0) return false;
+  auto index_at = [&](uint64_t u) {
+    uint32_t v;
+    std::memcpy(&v, blob + kIndexOffset + 4 * u, 4);
+    return v;
+  };
+  const uint64_t max_chunk = max_chunk_bytes(h.tile_cols, h.lmax);
+  const uint64_t min_chunk = raw_bytes(h.tile_cols) + kLanes;
+  uint64_t largest = 0;
+  if (index_at(0) != 0) return false;
+  uint32_t prev = 0;
+  for (uint64_t u = 0; u < tiles; ++u) {
+    const uint32_t nxt = index_at(u + 1);
+    if (nxt < prev) return false;
+    const uint64_t c = 16ull * (uint64_t)(nxt - prev);
+    if (c < min_chunk || c > max_chunk) return false;
+    largest = std::max(largest, c);
+    prev = nxt;
+  }
+  if (h.tiles_off + 16ull * prev != bytes) return false;
+  hd->rows = (int64_t)h.rows;
+  hd->cols = (int64_t)h.cols;
+  hd->tile_cols = h.tile_cols;
+  hd->lmax = h.lmax;
+  hd->filler = h.filler;
+  hd->tiles_r = (int64_t)h.tiles_r;
+  hd->tiles_c = (int64_t)h.tiles_c;
+  hd->tiles = (int64_t)tiles;
+  hd->index_off = kIndexOffset;
+  hd->tiles_off = h.tiles_off;
+  hd->blob_bytes = bytes;
+  hd->table_off = round_up(bytes, 256);
+  hd->device_bytes = hd->table_off + kTableBytes;
+  hd->max_chunk = largest;
+  if (lens_out) *lens_out = lens;
+  return true;
+}
+
+}  // namespace nwc

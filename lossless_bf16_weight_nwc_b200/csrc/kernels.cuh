@@ -1,0 +1,47 @@
+// kernels.cuh — launch interface of the sm_100a kernels (host side).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace nwc {
+
+// Device error word bits (read and cleared by nwc_get_device_error).
+constexpr uint32_t kErrTimeout = 1u;   // a bounded mbarrier wait gave up
+constexpr uint32_t kErrCorrupt = 2u;   // a stream held no valid code
+
+struct TileParams {
+  const uint8_t* tiles;     // device: tile area of the blob
+  const uint32_t* index;    // device: chunk offsets (16-byte units), tiles + 1
+  const uint32_t* table;    // device: 4096-entry decode table
+  int64_t rows, cols;
+  int64_t tiles_r, tiles_c, n_tiles;
+  int32_t total_warps;      // warps sharing the tiles (contiguous ranges)
+  int32_t ring_bytes;       // per-warp staging ring in shared memory
+  // GEMV
+  const uint16_t* x;        // BF16 [batch x cols]
+  float* y;                 // FP32 [batch x rows]
+  int32_t batch;            // rows of x handled by this launch (<= 8)
+  float* partial;           // [tiles_c][batch][rows_pad] split-K partial sums
+  uint32_t* counters;       // [tiles_r] arrivals per row tile
+  int64_t rows_pad;         // 8 * tiles_r
+  // decompress
+  uint16_t* out;            // BF16 [rows x cols]
+};
+
+struct LaunchShape {
+  int ctas;
+  int warps_per_cta;
+  int ring_bytes;
+  size_t smem_bytes;
+};
+
+// Picks the grid for n_tiles tiles whose largest chunk is max_chunk bytes.
+LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, int sm_count);
+
+cudaError_t launch_gemv(const TileParams& p, int tile_cols, const LaunchShape& s,
+                        cudaStream_t stream);
+cudaError_t launch_decompress(const TileParams& p, int tile_cols, const LaunchShape& s,
+                              cudaStream_t stream);
+cudaError_t read_and_clear_error(uint32_t* word);
+
+}  // namespace nwc

@@ -1,0 +1,324 @@
+// nwc_api.cu — the C ABI declared in include/nwc.h.
+//
+// Host-side validation, plans and handles, device images, and kernel launches.
+// Every device call runs on the caller's stream and allocates no device memory.
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/nwc.h"
+#include "kernels.cuh"
+#include "nwc_internal.h"
+
+namespace {
+
+using nwc::round_up;
+
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {};
+std::mutex g_mu;
+
+nwc_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NWC_OK : NWC_ERR_CUDA; }
+
+// Number of SMs of the current device (cached).
+nwc_status current_device(int* dev, int* sms) {
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return NWC_ERR_CUDA;
+  if (*dev < 0 || *dev >= kMaxDevices) return NWC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sm_count[*dev]) {
+    int v = 0;
+    e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, *dev);
+    if (e != cudaSuccess) return NWC_ERR_CUDA;
+    g_sm_count[*dev] = v;
+  }
+  *sms = g_sm_count[*dev];
+  return NWC_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nwc::TileParams base_params(const nwc_handle_s& h) {
+  nwc::TileParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.tiles = h.d_base + h.tiles_off;
+  p.index = reinterpret_cast<const uint32_t*>(h.d_base + h.index_off);
+  p.table = reinterpret_cast<const uint32_t*>(h.d_base + h.table_off);
+  p.rows = h.rows;
+  p.cols = h.cols;
+  p.tiles_r = h.tiles_r;
+  p.tiles_c = h.tiles_c;
+  p.n_tiles = h.tiles;
+  p.rows_pad = 8 * h.tiles_r;
+  return p;
+}
+
+constexpr int kChunkBatch = 8;  // CUDA-core kernel handles up to 8 rows of x per pass
+
+uint64_t workspace_bytes_for(const nwc_handle_s& h, int32_t batch) {
+  if (h.tiles_c <= 1) return 0;
+  const int b = batch < kChunkBatch ? batch : kChunkBatch;
+  const uint64_t counters = round_up(4ull * (uint64_t)h.tiles_r, 256);
+  return counters + 4ull * (uint64_t)h.tiles_c * (uint64_t)b * (uint64_t)(8 * h.tiles_r);
+}
+
+nwc_status make_handle(const uint8_t* blob_host_header_region, uint64_t bytes, const void* d_buf,
+                       uint64_t d_bytes, nwc_handle_t* out, const uint8_t** lens) {
+  nwc_handle_s tmp;
+  if (!nwc::parse_blob(blob_host_header_region, bytes, bytes, &tmp, lens)) return NWC_ERR_CORRUPT;
+  if (d_bytes < tmp.device_bytes) return NWC_ERR_INVALID_ARG;
+  nwc_handle_s* h = new (std::nothrow) nwc_handle_s(tmp);
+  if (!h) return NWC_ERR_NOMEM;
+  h->d_base = static_cast<const uint8_t*>(d_buf);
+  h->d_bytes = d_bytes;
+  cudaGetDevice(&h->device);
+  *out = h;
+  return NWC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int nwc_version(void) { return 100; }
+
+const char* nwc_status_string(nwc_status s) {
+  switch (s) {
+    case NWC_OK: return "ok";
+    case NWC_ERR_INVALID_ARG: return "invalid argument";
+    case NWC_ERR_UNSUPPORTED: return "unsupported";
+    case NWC_ERR_CUDA: return "CUDA runtime error";
+    case NWC_ERR_CORRUPT: return "corrupt blob or device image";
+    case NWC_ERR_NOMEM: return "out of memory or buffer too small";
+    case NWC_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case NWC_ERR_DEVICE_CORRUPT: return "device found corrupt data";
+  }
+  return "unknown status";
+}
+
+nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nwc_opts* opts,
+                    nwc_plan_t* out_plan) {
+  if (!w_host || !out_plan || rows < 1 || cols < 1) return NWC_ERR_INVALID_ARG;
+  if (rows > (1ll << 40) || cols > (1ll << 40)) return NWC_ERR_INVALID_ARG;
+  *out_plan = nullptr;
+  uint32_t lmax = 12, tile_rows = 8, tile_cols = 512, threads = 0;
+  if (opts) {
+    if (opts->struct_size < sizeof(nwc_opts)) return NWC_ERR_INVALID_ARG;
+    lmax = opts->lmax;
+    tile_rows = opts->tile_rows;
+    tile_cols = opts->tile_cols;
+    threads = opts->threads;
+  }
+  if (lmax < 1 || lmax > (uint32_t)nwc::kMaxLmax) return NWC_ERR_INVALID_ARG;
+  if (tile_rows != 8) return NWC_ERR_UNSUPPORTED;
+  if (tile_cols != 64 && tile_cols != 128 && tile_cols != 256 && tile_cols != 512)
+    return NWC_ERR_UNSUPPORTED;
+  nwc_plan_s* p = new (std::nothrow) nwc_plan_s();
+  if (!p) return NWC_ERR_NOMEM;
+  int rc;
+  try {
+    rc = nwc::plan_build(w_host, rows, cols, tile_rows, tile_cols, lmax, threads, p);
+  } catch (const std::bad_alloc&) {
+    delete p;
+    return NWC_ERR_NOMEM;
+  }
+  if (rc != 0) {
+    delete p;
+    return NWC_ERR_INVALID_ARG;  // too many distinct exponents for lmax, or > 64 GiB
+  }
+  *out_plan = p;
+  return NWC_OK;
+}
+
+nwc_status nwc_plan_size(nwc_plan_t plan, uint64_t* device_bytes, uint64_t* host_blob_bytes) {
+  if (!plan) return NWC_ERR_INVALID_ARG;
+  if (device_bytes) *device_bytes = plan->device_bytes;
+  if (host_blob_bytes) *host_blob_bytes = plan->blob_bytes;
+  return NWC_OK;
+}
+
+nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob,
+                             uint64_t blob_bytes) {
+  if (!plan || !w_host || !blob || blob_bytes < plan->blob_bytes) return NWC_ERR_INVALID_ARG;
+  try {
+    nwc::encode_blob(*plan, w_host, static_cast<uint8_t*>(blob));
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
+  return NWC_OK;
+}
+
+nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, uint64_t d_bytes,
+                        nwc_stream_t stream, nwc_handle_t* out_handle) {
+  if (!plan || !w_host || !d_buf || !out_handle) return NWC_ERR_INVALID_ARG;
+  if (d_bytes < plan->device_bytes || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
+  *out_handle = nullptr;
+  uint8_t* img = static_cast<uint8_t*>(std::malloc(plan->device_bytes));
+  if (!img) return NWC_ERR_NOMEM;
+  try {
+    nwc::encode_blob(*plan, w_host, img);
+  } catch (const std::bad_alloc&) {
+    std::free(img);
+    return NWC_ERR_NOMEM;
+  }
+  std::memset(img + plan->blob_bytes, 0, plan->table_off - plan->blob_bytes);
+  nwc::build_decode_table(plan->len, reinterpret_cast<uint32_t*>(img + plan->table_off));
+  // From pageable memory the call returns once the bytes are staged, so the
+  // image can be freed right after.
+  cudaError_t e = cudaMemcpyAsync(d_buf, img, plan->device_bytes, cudaMemcpyHostToDevice,
+                                  reinterpret_cast<cudaStream_t>(stream));
+  nwc_status st = NWC_OK;
+  if (e != cudaSuccess) {
+    st = NWC_ERR_CUDA;
+  } else {
+    st = make_handle(img, plan->blob_bytes, d_buf, d_bytes, out_handle, nullptr);
+  }
+  std::free(img);
+  return st;
+}
+
+nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes, uint64_t* device_bytes) {
+  if (!blob || !device_bytes) return NWC_ERR_INVALID_ARG;
+  nwc_handle_s tmp;
+  if (!nwc::parse_blob(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &tmp, nullptr))
+    return NWC_ERR_CORRUPT;
+  *device_bytes = tmp.device_bytes;
+  return NWC_OK;
+}
+
+nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, uint64_t d_bytes,
+                           nwc_stream_t stream, nwc_handle_t* out_handle) {
+  if (!blob || !d_buf || !out_handle || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
+  *out_handle = nullptr;
+  const uint8_t* lens = nullptr;
+  nwc_handle_t h = nullptr;
+  nwc_status st = make_handle(static_cast<const uint8_t*>(blob), blob_bytes, d_buf, d_bytes, &h,
+                              &lens);
+  if (st != NWC_OK) return st;
+  std::vector<uint32_t> table(nwc::kTableEntries);
+  nwc::build_decode_table(lens, table.data());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(d_buf, blob, blob_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && h->table_off > blob_bytes)
+    e = cudaMemsetAsync(static_cast<uint8_t*>(d_buf) + blob_bytes, 0, h->table_off - blob_bytes, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(static_cast<uint8_t*>(d_buf) + h->table_off, table.data(),
+                        nwc::kTableBytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    delete h;
+    return NWC_ERR_CUDA;
+  }
+  *out_handle = h;
+  return NWC_OK;
+}
+
+nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes, nwc_handle_t* out_handle) {
+  if (!d_buf || !out_handle || d_bytes < nwc::kIndexOffset) return NWC_ERR_INVALID_ARG;
+  *out_handle = nullptr;
+  nwc::BlobHeader hd;
+  if (cudaMemcpy(&hd, d_buf, sizeof(hd), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return NWC_ERR_CUDA;
+  if (hd.magic != nwc::kMagic || hd.total_bytes > d_bytes || hd.tiles_off > hd.total_bytes ||
+      hd.tiles_off < nwc::kIndexOffset)
+    return NWC_ERR_CORRUPT;
+  // Header, lens and index; the tile area is not read back.
+  std::vector<uint8_t> head(hd.tiles_off);
+  if (cudaMemcpy(head.data(), d_buf, hd.tiles_off, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return NWC_ERR_CUDA;
+  nwc_handle_s tmp;
+  if (!nwc::parse_blob(head.data(), head.size(), hd.total_bytes, &tmp, nullptr))
+    return NWC_ERR_CORRUPT;
+  if (d_bytes < tmp.device_bytes) return NWC_ERR_INVALID_ARG;
+  nwc_handle_s* h = new (std::nothrow) nwc_handle_s(tmp);
+  if (!h) return NWC_ERR_NOMEM;
+  h->d_base = static_cast<const uint8_t*>(d_buf);
+  h->d_bytes = d_bytes;
+  cudaGetDevice(&h->device);
+  *out_handle = h;
+  return NWC_OK;
+}
+
+nwc_status nwc_decompress(nwc_handle_t h, uint16_t* d_w_out, nwc_stream_t stream) {
+  if (!h || !d_w_out || !aligned(d_w_out, 4)) return NWC_ERR_INVALID_ARG;
+  int dev, sms;
+  nwc_status st = current_device(&dev, &sms);
+  if (st != NWC_OK) return st;
+  nwc::TileParams p = base_params(*h);
+  p.out = d_w_out;
+  const nwc::LaunchShape s = nwc::launch_shape(h->tiles, h->max_chunk, sms);
+  p.total_warps = s.ctas * s.warps_per_cta < h->tiles ? s.ctas * s.warps_per_cta : (int32_t)h->tiles;
+  p.ring_bytes = s.ring_bytes;
+  return cuda_status(nwc::launch_decompress(p, (int)h->tile_cols, s,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nwc_status nwc_gemv_workspace_size(nwc_handle_t h, int32_t batch, uint64_t* bytes) {
+  if (!h || !bytes || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
+  *bytes = workspace_bytes_for(*h, batch);
+  return NWC_OK;
+}
+
+nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t batch,
+                    void* d_workspace, uint64_t workspace_bytes, nwc_stream_t stream) {
+  if (!h || !d_x || !d_y || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
+  if (!aligned(d_x, 4) || !aligned(d_y, 4) || (h->cols & 1)) return NWC_ERR_INVALID_ARG;
+  const uint64_t need = workspace_bytes_for(*h, batch);
+  if (need && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 16)))
+    return NWC_ERR_INVALID_ARG;
+  // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
+  if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
+  int dev, sms;
+  nwc_status st = current_device(&dev, &sms);
+  if (st != NWC_OK) return st;
+  nwc::TileParams p = base_params(*h);
+  const nwc::LaunchShape s = nwc::launch_shape(h->tiles, h->max_chunk, sms);
+  p.total_warps = s.ctas * s.warps_per_cta < h->tiles ? s.ctas * s.warps_per_cta : (int32_t)h->tiles;
+  p.ring_bytes = s.ring_bytes;
+  if (need) {
+    uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+    p.counters = reinterpret_cast<uint32_t*>(ws);
+    p.partial = reinterpret_cast<float*>(ws + round_up(4ull * (uint64_t)h->tiles_r, 256));
+  }
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  for (int32_t b0 = 0; b0 < batch; b0 += kChunkBatch) {
+    const int32_t nb = batch - b0 < kChunkBatch ? batch - b0 : kChunkBatch;
+    p.x = d_x + (int64_t)b0 * h->cols;
+    p.y = d_y + (int64_t)b0 * h->rows;
+    p.batch = nb;
+    cudaError_t e = nwc::launch_gemv(p, (int)h->tile_cols, s, cs);
+    if (e != cudaSuccess) return NWC_ERR_CUDA;
+  }
+  return NWC_OK;
+}
+
+nwc_status nwc_handle_info(nwc_handle_t h, int64_t* rows, int64_t* cols, uint64_t* blob_bytes,
+                           uint64_t* device_bytes) {
+  if (!h) return NWC_ERR_INVALID_ARG;
+  if (rows) *rows = h->rows;
+  if (cols) *cols = h->cols;
+  if (blob_bytes) *blob_bytes = h->blob_bytes;
+  if (device_bytes) *device_bytes = h->device_bytes;
+  return NWC_OK;
+}
+
+nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return NWC_ERR_CUDA;
+  uint32_t w = 0;
+  e = nwc::read_and_clear_error(&w);
+  if (e != cudaSuccess) return NWC_ERR_CUDA;
+  if (word) *word = w;
+  if (w & nwc::kErrTimeout) return NWC_ERR_DEVICE_TIMEOUT;
+  if (w & nwc::kErrCorrupt) return NWC_ERR_DEVICE_CORRUPT;
+  return NWC_OK;
+}
+
+void nwc_plan_destroy(nwc_plan_t plan) { delete plan; }
+void nwc_handle_destroy(nwc_handle_t h) { delete h; }
+
+}  // extern "C"

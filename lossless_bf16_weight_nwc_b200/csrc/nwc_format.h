@@ -1,0 +1,73 @@
+// nwc_format.h — layout of the "NWB1" blob and of the device image, as the
+// library reads and writes them (host and device code).
+//
+// Byte planes and code: "Unweight: how we compressed an LLM 22% without
+// sacrificing quality", section "Compressing BF16 Weights" (exponent bytes
+// entropy-coded, sign and mantissa kept); "NWC — Neural Weight Compression",
+// "How it works" (byte planes; a 12-bit table peek; blocks of 8 rows x 512
+// columns with one bit stream per lane).
+//
+// Blob: 128-byte header | lens u8[256] | index u32[tiles + 1] | tile chunks.
+// A chunk is raw u8[8 * tile_cols] | lane byte counts u8[32] | stream words.
+// Stream words are little-endian u32 whose bit 31 is the earliest bit; the 32
+// lane streams follow one another, each padded to a byte, the whole run padded
+// to 16 bytes.  Lane t's k-th symbol is the tile element (row (k/2) % 8,
+// column 64 (k/16) + 2t + k%2); its raw byte is at (k/16) * 512 + 16 t + k%16.
+// Tiles are stored column-block-major: u = j * tiles_r + i.
+//
+// Device image: blob | zero pad to 256 | decode table u32[4096].
+#pragma once
+#include <cstdint>
+
+namespace nwc {
+
+constexpr uint32_t kMagic = 0x3142574Eu;  // "NWB1"
+constexpr uint32_t kVersion = 1;
+constexpr uint32_t kHeaderBytes = 128;
+constexpr uint32_t kLensOffset = 128;
+constexpr uint32_t kIndexOffset = 384;
+constexpr int kLanes = 32;
+constexpr int kTileRows = 8;
+constexpr int kMaxTileCols = 512;
+constexpr int kMaxLmax = 12;
+constexpr int kPeekBits = 12;
+constexpr int kTableEntries = 1 << kPeekBits;
+constexpr uint32_t kTableBytes = kTableEntries * 4;
+
+// Decode-table entry for one 12-bit peek (most significant bit = next bit):
+//   bits  0..3   bits consumed by the step (both codes, or the first only)
+//   bits  7..14  first exponent byte  (its BF16 position in the low half)
+//   bits 15..18  length of the first code
+//   bit  19      the peek starts with no valid code (corrupt stream)
+//   bits 23..30  second exponent byte (its BF16 position in the high half)
+//   bit  31      the second code did not fit in the 12 bits
+// Bits 4..6 stay zero so that a running difference of entries tracks the
+// number of consumed bits in its low 7 bits.
+constexpr uint32_t kEntryConsumedMask = 0xFu;
+constexpr uint32_t kEntryExponentMask = 0x7F807F80u;
+constexpr uint32_t kEntryRawMask = 0x807F807Fu;  // complement of the above
+constexpr int kEntryLen0Shift = 15;
+constexpr uint32_t kEntryInvalid = 1u << 19;
+constexpr uint32_t kEntrySingle = 1u << 31;
+
+inline uint64_t round_up(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
+
+struct BlobHeader {
+  uint32_t magic, version, header_bytes, lmax;
+  uint64_t rows, cols;
+  uint32_t tile_rows, tile_cols;
+  uint64_t tiles_r, tiles_c;
+  uint32_t filler, zero;
+  uint64_t lens_off, index_off, tiles_off, total_bytes, coded_bits;
+  uint8_t pad[24];
+};
+static_assert(sizeof(BlobHeader) == 128, "header layout");
+
+// Bytes of one tile's raw plane and the worst-case chunk.
+constexpr uint32_t raw_bytes(uint32_t tile_cols) { return kTileRows * tile_cols; }
+constexpr uint32_t max_chunk_bytes(uint32_t tile_cols, uint32_t lmax) {
+  return raw_bytes(tile_cols) + kLanes +
+         (uint32_t)((kLanes * ((2 * kTileRows * (tile_cols / 64) * lmax + 7) / 8) + 15) / 16 * 16);
+}
+
+}  // namespace nwc

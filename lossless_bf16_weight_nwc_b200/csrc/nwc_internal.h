@@ -1,0 +1,52 @@
+// nwc_internal.h — host-side structures shared by the encoder and the C ABI.
+#pragma once
+#include <cstdint>
+#include <vector>
+
+#include "nwc_format.h"
+
+struct nwc_plan_s {
+  int64_t rows = 0, cols = 0;
+  uint32_t tile_rows = 8, tile_cols = 512, lmax = 12, threads = 0;
+  int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
+  uint8_t len[256] = {};
+  uint32_t code[256] = {};
+  uint32_t filler = 0;
+  uint64_t coded_bits = 0;
+  std::vector<uint32_t> index;  // tiles + 1 entries, 16-byte units
+  uint64_t tiles_off = 0;       // blob offset of the tile area
+  uint64_t blob_bytes = 0;      // serialisable blob
+  uint64_t table_off = 0;       // device-image offset of the decode table
+  uint64_t device_bytes = 0;    // blob + padding + decode table
+};
+
+struct nwc_handle_s {
+  const uint8_t* d_base = nullptr;  // caller's device buffer
+  uint64_t d_bytes = 0;
+  int64_t rows = 0, cols = 0;
+  uint32_t tile_cols = 512, lmax = 12, filler = 0;
+  int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
+  uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0;
+  uint64_t device_bytes = 0;
+  uint64_t max_chunk = 0;  // largest chunk in bytes
+  int device = 0;
+};
+
+namespace nwc {
+
+// Encoder steps (encoder.cpp).
+int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
+               uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* plan);
+void encode_blob(const nwc_plan_s& plan, const uint16_t* w, uint8_t* blob);
+bool code_lengths(const uint64_t cnt[256], uint32_t lmax, uint8_t len[256]);
+void canonical_codes(const uint8_t len[256], uint32_t code[256]);
+void build_decode_table(const uint8_t len[256], uint32_t table[kTableEntries]);
+// Parses and checks a blob's header, lens and index (the first head_bytes of a
+// blob of `bytes` bytes; head_bytes must reach the tile area); fills the
+// handle's geometry fields.  Returns false when the blob does not follow the
+// format.
+bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* h,
+                const uint8_t** lens_out);
+unsigned hardware_threads(uint32_t requested);
+
+}  // namespace nwc

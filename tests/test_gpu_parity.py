@@ -1,0 +1,201 @@
+"""GPU parity: the CUDA path (through the C ABI) against the oracle.
+
+* Decompression must be bit-exact (integer/bit work): equal to the oracle's
+  decode of the same matrix, for library-written and oracle-written blobs.
+* GEMV must meet the tolerance of the target statement, per output
+      |y_gpu - y_oracle| <= 1e-2 * ||W_n||_2 * ||x_b||_2 * 2^-8
+  and overall ||y_gpu - y_oracle||_2 / ||y_oracle||_2 <= 2e-3,
+  where y_oracle is the FP64 sum over the original BF16 weights.
+"""
+import numpy as np
+import pytest
+
+from lossless_bf16_weight_nwc_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from lossless_bf16_weight_nwc_b200 import build
+    build.build()
+    from lossless_bf16_weight_nwc_b200 import _lib
+    torch.cuda.set_device(0)
+    return _lib
+
+
+def to_bf16(a: np.ndarray):
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def bits(t) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def tolerance_check(y_gpu: np.ndarray, y_ref: np.ndarray, w: np.ndarray, x: np.ndarray):
+    wf = synth.bf16_bits_to_float(w).astype(np.float64)
+    xf = synth.bf16_bits_to_float(x).astype(np.float64)
+    bound = 1e-2 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1)) * 2.0 ** -8
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    worst = float((err / np.maximum(bound, 1e-300)).max())
+    assert (err <= bound).all(), f"per-output bound exceeded: worst ratio {worst:.3g}"
+    rel = np.linalg.norm(y_gpu - y_ref) / max(np.linalg.norm(y_ref), 1e-300)
+    assert rel <= 2e-3, rel
+    return worst, rel
+
+
+def no_device_error(lib):
+    st, word = lib.nwc_get_device_error()
+    assert st == 0, f"device error word {word:#x}"
+
+
+SHAPES = [((8, 512), 512), ((9, 513), 512), ((77, 1030), 512), ((1, 2), 512),
+          ((1000, 1026), 512), ((64, 4096), 512), ((129, 300), 256), ((40, 200), 128),
+          ((17, 130), 64), ((4100, 96), 512)]
+
+
+@pytest.mark.parametrize("shape,tile_cols", SHAPES)
+def test_decompress_bit_exact(lib, orc, shape, tile_cols):
+    spec = synth.MatrixSpec("w", shape[0], shape[1], "student_t5", 0.015, 1)
+    w = synth.matrix(spec, 5)
+    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols)
+    out = bits(m.decompress())
+    ref = orc.decode(orc.encode(w, tile_cols=tile_cols))
+    assert np.array_equal(ref, w)
+    assert np.array_equal(out, ref)
+    no_device_error(lib)
+
+
+def test_decompress_every_pattern(lib, orc):
+    w = np.arange(65536, dtype=np.uint16).reshape(256, 256)
+    for tile_cols, lmax in ((512, 12), (128, 8)):
+        m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
+        assert np.array_equal(bits(m.decompress()), w)
+    rng = np.random.default_rng(0)
+    shuffled = rng.permutation(w.reshape(-1)).reshape(128, 512)
+    m = lib.CompressedMatrix.compress(shuffled)
+    assert np.array_equal(bits(m.decompress()), shuffled)
+    no_device_error(lib)
+
+
+def test_gpu_decodes_oracle_blob(lib, orc):
+    spec = synth.MatrixSpec("w", 300, 2000, "normal_outliers", 1 / 64, 0)
+    w = synth.matrix(spec, 1)
+    blob = orc.encode(w)
+    m = lib.CompressedMatrix.from_blob(blob)
+    assert np.array_equal(bits(m.decompress()), w)
+    x = synth.activations(1, 2, spec.cols)
+    y = m.gemv(to_bf16(x)).cpu().numpy()
+    tolerance_check(y, orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("shape,tile_cols", SHAPES)
+@pytest.mark.parametrize("batch", [1, 3, 8])
+def test_gemv_parity_shapes(lib, orc, shape, tile_cols, batch):
+    if shape[1] % 2:
+        pytest.skip("nwc_gemv requires an even number of columns")
+    spec = synth.MatrixSpec("w", shape[0], shape[1], "normal", 0.02, 2)
+    w = synth.matrix(spec, 6)
+    x = synth.activations(6, batch, shape[1])
+    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols)
+    y = m.gemv(to_bf16(x)).cpu().numpy()
+    tolerance_check(y, orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
+@pytest.mark.parametrize("batch", [1, 2, 4, 5, 7, 8, 9, 16, 33, 64])
+def test_gemv_every_batch(lib, orc, batch):
+    spec = synth.MatrixSpec("w", 520, 2048, "normal_rowscale", 0.02, 3)
+    w = synth.matrix(spec, 4)
+    x = synth.activations(4, batch, spec.cols)
+    m = lib.CompressedMatrix.compress(w)
+    y = m.gemv(to_bf16(x)).cpu().numpy()
+    tolerance_check(y, orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
+def test_gemv_deterministic_and_workspace_reuse(lib, orc):
+    spec = synth.MatrixSpec("w", 2048, 4096, "normal", 0.02, 0)
+    w = synth.matrix(spec, 8)
+    x = synth.activations(8, 4, spec.cols)
+    m = lib.CompressedMatrix.compress(w)
+    xt = to_bf16(x)
+    first = m.gemv(xt).cpu().numpy()
+    for _ in range(20):
+        again = m.gemv(xt).cpu().numpy()
+        assert np.array_equal(first.view(np.uint32), again.view(np.uint32))
+    tolerance_check(first, orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
+def test_handle_from_device_image(lib, orc):
+    spec = synth.MatrixSpec("w", 96, 1536, "normal", 0.02, 0)
+    w = synth.matrix(spec, 2)
+    m = lib.CompressedMatrix.compress(w)
+    copy = m.image.clone()
+    h = lib.nwc_handle_from_device(copy, copy.numel())
+    out = torch.empty((96, 1536), dtype=torch.bfloat16, device="cuda")
+    lib.nwc_decompress(h, out)
+    assert np.array_equal(bits(out), w)
+    lib.nwc_handle_destroy(h)
+    no_device_error(lib)
+
+
+def test_invalid_arguments_rejected(lib):
+    w = synth.matrix(synth.MatrixSpec("w", 16, 1024, "normal", 0.02, 0), 0)
+    m = lib.CompressedMatrix.compress(w)
+    x = torch.zeros((1, 1024), dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros((1, 16), dtype=torch.float32, device="cuda")
+    with pytest.raises(lib.NwcError):
+        lib.nwc_gemv(m.handle, x, y, 0)
+    with pytest.raises(lib.NwcError):
+        lib.nwc_gemv(m.handle, x, y, 65)
+    with pytest.raises(lib.NwcError):            # workspace required (2 column tiles)
+        lib.nwc_gemv(m.handle, x, y, 1, None, 0)
+    with pytest.raises(lib.NwcError):            # misaligned x
+        lib.nwc_gemv(m.handle, x.data_ptr() + 2, y, 1, *m.workspace(1))
+    odd = lib.CompressedMatrix.compress(synth.matrix(synth.MatrixSpec("w", 4, 5, "normal", 0.02, 0), 0))
+    x5 = torch.zeros((1, 5), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lib.NwcError):            # odd column count
+        lib.nwc_gemv(odd.handle, x5, torch.zeros(4, device="cuda"), 1)
+    blob = np.zeros(1024, dtype=np.uint8)
+    with pytest.raises(lib.NwcError):
+        lib.CompressedMatrix.from_blob(blob)
+    no_device_error(lib)
+
+
+# ---- the benchmark workloads at full size ------------------------------------
+
+@pytest.mark.parametrize("name", ["single_1024", "attn_4096_outliers"])
+def test_workload_full_parity(lib, orc, name):
+    wl = synth.workload(name)
+    for spec in wl.matrices:
+        w = synth.matrix(spec, wl.seed)
+        m = lib.CompressedMatrix.compress(w)
+        assert np.array_equal(bits(m.decompress()), w)
+        assert m.ratio >= 1.25
+        for batch in wl.batches:
+            x = synth.activations(wl.seed, batch, spec.cols)
+            y = m.gemv(to_bf16(x)).cpu().numpy()
+            tolerance_check(y, orc.gemv(w, x), w, x)
+        m.close()
+    no_device_error(lib)
+
+
+def test_workload_mlp_pair_full(lib, orc):
+    wl = synth.workload("mlp_pair_t5")
+    for spec in wl.matrices:
+        w = synth.matrix(spec, wl.seed)
+        m = lib.CompressedMatrix.compress(w)
+        assert np.array_equal(bits(m.decompress()), w)
+        for batch in wl.batches:
+            x = synth.activations(wl.seed, batch, spec.cols)
+            y = m.gemv(to_bf16(x)).cpu().numpy()
+            tolerance_check(y, orc.gemv(w, x), w, x)
+        m.close()
+    no_device_error(lib)

@@ -1,0 +1,74 @@
+"""libnwc on the CPU: it loads, exports every symbol include/nwc.h declares, and
+its host encoder writes the same bytes as the oracle (no GPU calls here)."""
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT
+from lossless_bf16_weight_nwc_b200 import synth
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from lossless_bf16_weight_nwc_b200 import build
+    build.build()
+    from lossless_bf16_weight_nwc_b200 import _lib
+    return _lib
+
+
+def test_exports_every_declared_symbol(lib):
+    with open(f"{ROOT}/include/nwc.h") as f:
+        text = f.read()
+    declared = set(re.findall(r"\b(nwc_[a-z_]+)\s*\(", text))
+    assert len(declared) >= 16
+    for name in declared:
+        assert hasattr(lib.LIB, name), name
+    assert set(lib.EXPORTED) == declared
+
+
+def test_status_strings(lib):
+    for code in range(8):
+        assert lib.LIB.nwc_status_string(code)
+
+
+@pytest.mark.parametrize("shape,tile_cols,lmax", [((1024, 1024), 512, 12), ((9, 513), 512, 12),
+                                                  ((77, 1030), 256, 10), ((8, 64), 64, 8),
+                                                  ((333, 200), 128, 12), ((1, 1), 512, 12)])
+def test_host_encoder_byte_identical_to_oracle(lib, orc, shape, tile_cols, lmax):
+    spec = synth.MatrixSpec("w", shape[0], shape[1], "student_t5", 0.015, 3)
+    w = synth.matrix(spec, 7)
+    plan = lib.nwc_plan(w, lmax=lmax, tile_cols=tile_cols, threads=3)
+    try:
+        dev_bytes, blob_bytes = lib.nwc_plan_size(plan)
+        blob = lib.nwc_compress_host(plan, w)
+    finally:
+        lib.nwc_plan_destroy(plan)
+    ref = orc.encode(w, tile_cols=tile_cols, lmax=lmax)
+    assert blob.size == blob_bytes == ref.size
+    assert np.array_equal(blob, ref)
+    assert dev_bytes >= blob_bytes + 16384 and dev_bytes % 256 == 0
+    assert lib.nwc_blob_device_bytes(blob) == dev_bytes
+    assert np.array_equal(orc.decode(blob), w)
+
+
+def test_all_patterns_byte_identical(lib, orc):
+    w = np.arange(65536, dtype=np.uint16).reshape(256, 256)
+    plan = lib.nwc_plan(w, lmax=12)
+    blob = lib.nwc_compress_host(plan, w)
+    lib.nwc_plan_destroy(plan)
+    assert np.array_equal(blob, orc.encode(w))
+
+
+def test_host_validation(lib):
+    w = np.zeros((4, 4), dtype=np.uint16)
+    with pytest.raises(lib.NwcError):
+        lib.nwc_plan(w, tile_cols=100)
+    with pytest.raises(lib.NwcError):
+        lib.nwc_plan(w, lmax=13)
+    w = (np.arange(256, dtype=np.uint16) << 7).reshape(1, 256)
+    with pytest.raises(lib.NwcError):          # 256 exponents do not fit 7-bit codes
+        lib.nwc_plan(w, lmax=7)
+    bad = np.zeros(512, dtype=np.uint8)
+    with pytest.raises(lib.NwcError):
+        lib.nwc_blob_device_bytes(bad)
