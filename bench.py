@@ -269,15 +269,6 @@ def main():
     with torch.cuda.graph(g, stream=stream):
         for i in range(calls_per_graph):
             call(mats[i % copies], stream)
-    # Per-launch durations: one graph with an event pair around every call.
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(copies)]
-    g_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_ev, stream=stream):
-        for i in range(copies):
-            ev[i][0].record(stream)
-            call(mats[i], stream)
-            ev[i][1].record(stream)
     replays = max(1, args.steps // calls_per_graph)
     steps = replays * calls_per_graph
     with torch.cuda.stream(stream):
@@ -300,13 +291,22 @@ def main():
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
     clock = clocks.summary()
 
-    # Average launch duration of the GEMV kernel (event pairs on its stream).
+    # Average launch duration of the GEMV kernel: event pairs around direct
+    # launches on its stream, queued behind a GPU sleep so that the intervals
+    # hold the kernels only (not host submission gaps).
     durs = []
-    with torch.cuda.stream(stream):
-        for _ in range(max(3, 2000 // copies)):
-            g_ev.replay()
-            stream.synchronize()
-            durs += [a.elapsed_time(b) for a, b in ev]
+    n_timed = min(256, 8 * copies)
+    for _ in range(4):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_timed)]
+        with torch.cuda.stream(stream):
+            torch.cuda._sleep(100_000_000)
+            for i in range(n_timed):
+                ev[i][0].record(stream)
+                call(mats[i % copies], stream)
+                ev[i][1].record(stream)
+        stream.synchronize()
+        durs += [a.elapsed_time(b) for a, b in ev]
     kernel_ms = statistics.mean(durs) / launches_per_call
     ms_per_step = elapsed_ms / steps
 
@@ -427,7 +427,7 @@ def main():
     if rank == 0:
         print(json.dumps(line))
     # Release graphs before the process group.
-    del g, g_ev
+    del g
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -9,8 +9,9 @@
  *     compressed an LLM 22% without sacrificing quality", section "Compressing BF16
  *     Weights"; "NWC — Neural Weight Compression", "How it works > Byte planes").
  *   - The code is one optimal prefix code per matrix, with lengths limited to lmax
- *     (12 by default: the decoder peeks 12 bits, as in "NWC", "How it works >
- *     Prefix code instead of rANS").
+ *     (7 by default, so that one 14-bit table peek always holds two complete
+ *     codes, as the decoder in "NWC", "How it works > Prefix code instead of
+ *     rANS" does with its 12-bit peek).
  *   - The matrix is cut into independently decodable tiles of 8 rows x tile_cols
  *     columns, with one bit stream per lane ("NWC", "How it works > Fused kernel").
  *   - The GPU decodes the tiles in registers and shared memory inside the
@@ -58,8 +59,12 @@ typedef enum {
 } nwc_status;
 
 /* Plan options.  Set struct_size = sizeof(nwc_opts); pass NULL for the defaults
- * (lmax = 12, tile_rows = 8, tile_cols = 512, threads = 0 meaning all cores).
- * lmax must be in [1, 12] and at least ceil(log2(distinct exponents)).
+ * (lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0 meaning all cores).
+ * lmax: 0 = automatic (7, or the smallest limit that admits every distinct
+ * exponent when there are more than 128), else in [1, 12] and at least
+ * ceil(log2(distinct exponents)).  With lmax <= 7 the decoder peeks 14 bits and
+ * every peek holds two complete codes; with 8..12 it peeks 12 bits and takes a
+ * second lookup when a pair does not fit.
  * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512. */
 typedef struct {
   uint32_t struct_size;
@@ -86,9 +91,10 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols,
                     const nwc_opts* opts, nwc_plan_t* out_plan);
 
 /* Exact sizes for a plan.  *device_bytes is what nwc_compress needs in device
- * memory: the serialisable blob plus a derived 16 KiB decode table, at a
- * 256-byte aligned offset.  *host_blob_bytes is the size of the serialisable
- * blob (nwc_compress_host).  Either pointer may be NULL. */
+ * memory: the serialisable blob plus a derived decode table (64 KiB for
+ * lmax <= 7, else 16 KiB) at a 256-byte aligned offset.  *host_blob_bytes is
+ * the size of the serialisable blob (nwc_compress_host).  Either pointer may
+ * be NULL. */
 nwc_status nwc_plan_size(nwc_plan_t plan, uint64_t* device_bytes,
                          uint64_t* host_blob_bytes);
 

@@ -96,7 +96,7 @@ def nwc_version() -> int:
     return LIB.nwc_version()
 
 
-def nwc_plan(w_host: np.ndarray, lmax: int = 12, tile_cols: int = 512, threads: int = 0):
+def nwc_plan(w_host: np.ndarray, lmax: int = 0, tile_cols: int = 512, threads: int = 0):
     w = np.ascontiguousarray(w_host, dtype=np.uint16)
     rows, cols = w.shape
     opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads)
@@ -209,7 +209,7 @@ class CompressedMatrix:
         self._ws = None
 
     @classmethod
-    def compress(cls, w_host: np.ndarray, device="cuda", lmax: int = 12, tile_cols: int = 512,
+    def compress(cls, w_host: np.ndarray, device="cuda", lmax: int = 0, tile_cols: int = 512,
                  threads: int = 0, stream=None) -> "CompressedMatrix":
         import torch
         plan = nwc_plan(w_host, lmax=lmax, tile_cols=tile_cols, threads=threads)

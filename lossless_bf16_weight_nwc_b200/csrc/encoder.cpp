@@ -168,17 +168,19 @@ void canonical_codes(const uint8_t len[256], uint32_t code[256]) {
   for (int s = 0; s < 256; ++s) code[s] = len[s] ? first[len[s]]++ : 0;
 }
 
-void build_decode_table(const uint8_t len[256], uint32_t table[kTableEntries]) {
+void build_decode_table(const uint8_t len[256], uint32_t lmax, uint32_t* table) {
+  const int peek = peek_bits(lmax);
+  const uint32_t entries = table_entries(lmax);
   uint32_t code[256];
   canonical_codes(len, code);
   // sym[l][v]: symbol with code v of length l, or -1.
-  std::vector<std::vector<int16_t>> sym(kPeekBits + 1);
-  for (int l = 1; l <= kPeekBits; ++l) sym[l].assign(size_t(1) << l, -1);
+  std::vector<std::vector<int16_t>> sym(peek + 1);
+  for (int l = 1; l <= peek; ++l) sym[l].assign(size_t(1) << l, -1);
   for (int s = 0; s < 256; ++s)
-    if (len[s] >= 1 && len[s] <= kPeekBits) sym[len[s]][code[s]] = (int16_t)s;
+    if (len[s] >= 1 && len[s] <= peek) sym[len[s]][code[s]] = (int16_t)s;
   auto first_code = [&](uint32_t bits, int avail, int* s_out, int* l_out) {
     for (int l = 1; l <= avail; ++l) {
-      const int s = sym[l][bits >> (kPeekBits - l)];
+      const int s = sym[l][bits >> (peek - l)];
       if (s >= 0) {
         *s_out = s;
         *l_out = l;
@@ -187,15 +189,15 @@ void build_decode_table(const uint8_t len[256], uint32_t table[kTableEntries]) {
     }
     return false;
   };
-  for (uint32_t v = 0; v < (uint32_t)kTableEntries; ++v) {
+  for (uint32_t v = 0; v < entries; ++v) {
     int s0, l0, s1, l1;
-    if (!first_code(v, kPeekBits, &s0, &l0)) {
+    if (!first_code(v, peek, &s0, &l0)) {
       table[v] = 2u | kEntryInvalid;  // consume two bits, emit exponent 0
       continue;
     }
-    const uint32_t rest = (v << l0) & (kTableEntries - 1);
+    const uint32_t rest = (v << l0) & (entries - 1);
     uint32_t e = ((uint32_t)s0 << 7) | ((uint32_t)l0 << kEntryLen0Shift);
-    if (first_code(rest, kPeekBits - l0, &s1, &l1))
+    if (first_code(rest, peek - l0, &s1, &l1))
       e |= (uint32_t)(l0 + l1) | ((uint32_t)s1 << 23);
     else
       e |= (uint32_t)l0 | kEntrySingle;
@@ -241,6 +243,16 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   p->filler = filler;
   cnt[filler] += (uint64_t)(p->tiles_r * kTileRows) * (uint64_t)(p->tiles_c * tile_cols) -
                  (uint64_t)rows * (uint64_t)cols;
+  if (lmax == 0) {
+    // Automatic: 7 (two codes always fit the decoder's 14-bit peek) unless the
+    // matrix holds more than 128 distinct exponents; then the smallest limit
+    // that admits them all.
+    int distinct = 0;
+    for (int s = 0; s < 256; ++s) distinct += cnt[s] != 0;
+    lmax = 7;
+    while ((1 << lmax) < distinct) ++lmax;
+    p->lmax = lmax;
+  }
   if (!code_lengths(cnt, lmax, p->len)) return -1;
   canonical_codes(p->len, p->code);
   p->coded_bits = 0;
@@ -267,7 +279,7 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   p->tiles_off = round_up(kIndexOffset + 4ull * (uint64_t)(p->tiles + 1), 256);
   p->blob_bytes = p->tiles_off + 16ull * acc;
   p->table_off = round_up(p->blob_bytes, 256);
-  p->device_bytes = p->table_off + kTableBytes;
+  p->device_bytes = p->table_off + table_bytes(p->lmax);
   return 0;
 }
 
@@ -403,7 +415,7 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   hd->tiles_off = h.tiles_off;
   hd->blob_bytes = bytes;
   hd->table_off = round_up(bytes, 256);
-  hd->device_bytes = hd->table_off + kTableBytes;
+  hd->device_bytes = hd->table_off + table_bytes(h.lmax);
   hd->max_chunk = largest;
   if (lens_out) *lens_out = lens;
   return true;

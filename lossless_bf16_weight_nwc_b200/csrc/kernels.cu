@@ -2,24 +2,26 @@
 //
 // What runs where ("NWC — Neural Weight Compression", "How it works > Fused
 // kernel"; "Unweight", "Direct GPU Decompression"):
-//   * Each warp owns a contiguous range of tiles (8 rows x tile_cols), in the
-//     blob's column-block-major order, so it keeps one slice of x for long runs.
-//   * Lane 0 of the warp streams the tile chunks (raw plane + lane streams)
-//     from HBM into a per-warp shared-memory ring with cp.async.bulk (no
-//     multicast), each completion counted by an mbarrier.  Every wait is
-//     bounded: a wait that gives up sets the device error word and the warp
-//     drains its copies and stops.
-//   * Each lane decodes its own bit stream: a 64-bit window, a 12-bit peek into
-//     a 4096-entry table in shared memory that yields two exponent bytes at
-//     their BF16 positions ("NWC", "Prefix code instead of rANS"), a funnel
-//     shift by the consumed length, and a refill from shared memory every two
-//     steps.  A peek whose two codes do not fit in 12 bits takes a second
-//     lookup.
+//   * One persistent CTA per SM owns a contiguous range of tiles (8 rows x
+//     tile_cols), in the blob's column-block-major order.
+//   * A producer warp streams the tiles' chunks (raw plane + lane streams) from
+//     HBM into one CTA-wide shared-memory ring with cp.async.bulk (no
+//     multicast).  Each chunk lands in a slot with a "full" mbarrier (bytes
+//     counted) and is handed back through an "empty" mbarrier.  Every wait is
+//     bounded: a wait that gives up sets the device error word, and the
+//     producer drains its copies before leaving.
+//   * 16 consumer warps take the CTA's tiles round-robin.  Each lane decodes its
+//     own bit stream with a 64-bit window and a table peek.  With lmax <= 7 the
+//     peek is 14 bits and every entry holds two complete codes ("NWC", "Prefix
+//     code instead of rANS"), so a step is a lookup plus two funnel shifts.
+//     With lmax 8..12 the peek is 12 bits and a pair that does not fit takes a
+//     second lookup.  The window is refilled every two steps, without a branch.
 //   * BF16x2 reassembly is one byte permute of the raw plane and one bitwise
 //     select with the table entry; the weights never leave registers.
-//   * GEMV: FP32 FMAs into 8 row sums per batch row, a transposed warp-shuffle
-//     reduction per tile, and a split-K reduction in a fixed order through the
-//     workspace (the last warp to finish a row block sums the partials).
+//   * GEMV: FP32 accumulation of BF16 x BF16 products (fma.rn.f32.bf16) into 8
+//     row sums per batch row, a transposed warp-shuffle reduction per tile, and
+//     a split-K reduction in a fixed order through the workspace (the last of a
+//     row block's column tiles to finish sums the partials).
 //   * Decompress: the same decode, with a 32-bit store per weight pair, one
 //     128-byte line per warp store.
 #include <cuda_runtime.h>
@@ -35,11 +37,14 @@ __device__ unsigned int g_device_error;
 
 namespace {
 
-constexpr int kDepth = 4;                  // tiles in flight per warp
-constexpr uint32_t kWaitLimit = 1u << 22;  // bounded mbarrier polls
-constexpr int kMaxWarps = 16;
-constexpr int kRingSlack = 16;             // lanes may read a few words past a chunk
+constexpr int kConsumers = 16;                   // decoding warps per CTA
+constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
+constexpr int kSlots = 32;                       // tiles in flight or resident per CTA
+constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
+constexpr int kRingSlack = 16;                   // lanes may read a few words past a chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// ---- PTX helpers -----------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -52,6 +57,9 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
                : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -66,7 +74,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bulk copy global -> this CTA's shared memory, completion counted in bytes on
 // `bar`.  Plain (non-multicast) form.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
           smem_u32(dst)),
@@ -79,7 +88,6 @@ __device__ __forceinline__ void fence_barrier_init() {
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-
 // Polls `bar` for `parity` at most kWaitLimit times; on failure records a
 // timeout in the device error word.
 __device__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
@@ -89,30 +97,72 @@ __device__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+// Loads a word only when `need` is non-zero (predicated, no branch); else
+// returns 0.
+__device__ __forceinline__ uint32_t lds32_if(uint32_t addr, uint32_t need) {
+  uint32_t v = 0;
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p ld.shared.u32 %0, [%1];\n\t}"
+               : "+r"(v)
+               : "r"(addr), "r"(need));
+  return v;
+}
+// Low word of ({hi, lo} >> (n mod 32)).
+__device__ __forceinline__ uint32_t shr_wrap(uint32_t lo, uint32_t hi, uint32_t n) {
+  uint32_t r;
+  asm("shf.r.wrap.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(lo), "r"(hi), "r"(n));
+  return r;
+}
+// c + bf16(a half) * bf16(b half) in FP32; HI selects the upper halves.
+template <bool HI>
+__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
+  float d;
+  if (HI)
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+  else
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+  return d;
+}
 
-// Per-lane bit reader over the lane's stream in shared memory.  Invariant at
-// every refill point: at least 32 valid bits; one step consumes at most 12, so
-// two steps always have the 12 valid bits a peek needs.  The low 7 bits of
-// `nbacc` count valid bits; subtracting whole table entries keeps them exact
-// because entry bits 4..6 are zero and bits 0..3 hold the consumed count.
+// ---- bit reader --------------------------------------------------------------
+
+// Per-lane reader of the lane's stream in shared memory: a 64-bit window hi:lo
+// (next bit = bit 31 of hi) and a valid-bit count.  Invariant at each refill
+// point: at least 32 valid bits; a step consumes at most 14 bits, so the two
+// steps between refill points always have their peek bits.  The low 7 bits of
+// `nbacc` count valid bits; subtracting whole table entries keeps them exact,
+// since entry bits 4..6 are zero and bits 0..3 hold the consumed count.
 struct BitReader {
   uint32_t hi, lo, nbacc;
-  const uint32_t* wp;
+  uint32_t wp;  // shared-window address of the next stream word
 
-  __device__ __forceinline__ void init(const uint8_t* area, uint32_t start) {
-    wp = reinterpret_cast<const uint32_t*>(area) + (start >> 2);
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start) {
+    wp = area + (start & ~3u);
     const uint32_t sh = (start & 3u) * 8u;
-    const uint32_t w0 = wp[0], w1 = wp[1];
+    const uint32_t w0 = lds32(wp), w1 = lds32(wp + 4);
     hi = __funnelshift_l(w1, w0, sh);
     lo = w1 << sh;
     nbacc = 64u - sh;
-    wp += 2;
+    wp += 8;
   }
-  __device__ __forceinline__ uint32_t peek() const { return hi >> (32 - kPeekBits); }
-  // Consume the count held in bits 0..3 of e (upper bits are ignored by the
-  // funnel shifts, which use e & 31).
+  // Consumes the count in bits 0..3 of e (the funnel shifts use e & 31).
   __device__ __forceinline__ void consume_entry(uint32_t e) {
     hi = __funnelshift_l(lo, hi, e);
     lo = __funnelshift_l(0u, lo, e);
@@ -123,27 +173,35 @@ struct BitReader {
     lo = lo << n;
     nbacc -= n;
   }
+  // With fewer than 32 valid bits (bit 5 of the count clear; the count never
+  // reaches 64 at a refill point), append the next word right after the valid
+  // bits; the count becomes count | 32 either way.  No branch: the load is
+  // predicated and an empty word shifts in nothing.
   __device__ __forceinline__ void refill() {
-    const uint32_t nb = nbacc & 127u;
-    if (nb < 32u) {
-      const uint32_t w = *wp++;
-      const uint64_t win = ((uint64_t)hi << 32 | lo) | ((uint64_t)w << (32u - nb));
-      hi = (uint32_t)(win >> 32);
-      lo = (uint32_t)win;
-      nbacc += 32u;
-    }
+    const uint32_t need = (~nbacc) & 32u;
+    const uint32_t w = lds32_if(wp, need);
+    hi |= shr_wrap(w, 0u, nbacc);
+    lo |= shr_wrap(0u, w, nbacc);
+    wp += need >> 3;
+    nbacc |= 32u;
   }
 };
 
-// Decodes one step: two exponent bytes at their BF16 positions in a table
-// entry (bits 7..14 and 23..30).
-__device__ __forceinline__ uint32_t decode_pair(BitReader& br, const uint32_t* table) {
-  uint32_t e = table[br.peek()];
+// One step: a table entry holding two exponent bytes at their BF16 positions
+// (bits 7..14 and 23..30).  FAST: 14-bit peek, both codes always fit.
+template <bool FAST>
+__device__ __forceinline__ uint32_t decode_pair(BitReader& br, uint32_t table) {
+  if (FAST) {
+    const uint32_t e = lds32(table + ((br.hi >> 16) & 0xFFFCu));
+    br.consume_entry(e);
+    return e;
+  }
+  uint32_t e = lds32(table + ((br.hi >> 18) & 0x3FFCu));
   br.consume_entry(e);
-  if ((int32_t)e < 0) {
-    // The second code did not fit in the peek: look it up on its own.
+  if (__builtin_expect((int32_t)e < 0, 0)) {
+    // The second code did not fit in the 12-bit peek: look it up on its own.
     br.refill();
-    const uint32_t e2 = table[br.peek()];
+    const uint32_t e2 = lds32(table + ((br.hi >> 18) & 0x3FFCu));
     br.consume_bits((e2 >> kEntryLen0Shift) & 15u);
     e = (e & ~0x7F800000u) | ((e2 << 16) & 0x7F800000u) | (e2 & kEntryInvalid);
   }
@@ -157,115 +215,147 @@ __device__ __forceinline__ uint32_t raw_pair(const uint4& rv) {
   const uint32_t w = (R < 2) ? rv.x : (R < 4) ? rv.y : (R < 6) ? rv.z : rv.w;
   return __byte_perm(w, 0u, (R & 1) ? 0x3322u : 0x1100u);
 }
+__device__ __forceinline__ uint32_t raw_pair_r(const uint4& rv, int r) {
+  switch (r) {
+    case 0: return raw_pair<0>(rv);
+    case 1: return raw_pair<1>(rv);
+    case 2: return raw_pair<2>(rv);
+    case 3: return raw_pair<3>(rv);
+    case 4: return raw_pair<4>(rv);
+    case 5: return raw_pair<5>(rv);
+    case 6: return raw_pair<6>(rv);
+    default: return raw_pair<7>(rv);
+  }
+}
 
 __device__ __forceinline__ uint32_t assemble(uint32_t rawdup, uint32_t e) {
-  // Select sign+fraction from the raw bytes and the exponents from the entry.
+  // Sign+fraction from the raw bytes, exponents from the table entry.
   return (rawdup & kEntryRawMask) | (e & kEntryExponentMask);
 }
 
-// Lane-distributed per-warp staging pipeline (all lanes keep identical state;
-// lane 0 issues the copies; lane s < kDepth holds the ring position of slot s).
-struct Pipeline {
-  const uint8_t* tiles;
-  const uint32_t* index;
-  uint8_t* ring;
-  uint64_t* bars;
-  int64_t u0, n;          // this warp's tiles [u0, u0 + n)
-  int64_t issued, consumed;
-  uint32_t ring_bytes;
-  uint32_t vhead, vtail;  // virtual ring positions
-  uint32_t slot_vpos;     // lane s: virtual start of slot s
-  int64_t wb;             // index window base
-  uint32_t idx_a, idx_b;  // index[wb + lane], index[wb + 32 + lane]
-  int64_t n_index;        // entries in index (tiles + 1)
-  int lane;
+// Start of lane `lane`'s stream: prefix sum of the lane byte counts.
+__device__ __forceinline__ uint32_t lane_stream_start(uint32_t chunk, int raw, int lane) {
+  const uint32_t b4 = lds32(chunk + raw + (lane & ~3));
+  const uint32_t my_len = (b4 >> (8 * (lane & 3))) & 0xFFu;
+  uint32_t incl = my_len;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t v = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += v;
+  }
+  return incl - my_len;
+}
 
-  __device__ __forceinline__ uint32_t load_index(int64_t e) const {
-    return e < n_index ? __ldg(index + e) : 0u;
-  }
-  __device__ void init(const uint8_t* t, const uint32_t* ix, int64_t n_tiles, uint8_t* r,
-                       uint32_t rb, uint64_t* b, int64_t first, int64_t count, int ln) {
-    tiles = t;
-    index = ix;
-    ring = r;
-    ring_bytes = rb;
-    bars = b;
-    u0 = first;
-    n = count;
-    issued = consumed = 0;
-    vhead = vtail = 0;
-    slot_vpos = 0;
-    lane = ln;
-    n_index = n_tiles + 1;
-    wb = u0;
-    idx_a = load_index(wb + lane);
-    idx_b = load_index(wb + 32 + lane);
-  }
-  __device__ __forceinline__ uint32_t index_at(int64_t e) {
-    while (e - wb >= 64) {  // slide the window (uniform across the warp)
-      wb += 32;
-      idx_a = idx_b;
-      idx_b = load_index(wb + 32 + lane);
-    }
-    const int d = (int)(e - wb);
-    const uint32_t va = __shfl_sync(kFull, idx_a, d & 31);
-    const uint32_t vb = __shfl_sync(kFull, idx_b, d & 31);
-    return d < 32 ? va : vb;
-  }
-  // Issue copies while the ring has room and fewer than kDepth are in flight.
-  __device__ void issue() {
-    while (issued < n && issued - consumed < kDepth) {
-      const int64_t u = u0 + issued;
-      const uint32_t c0 = index_at(u), c1 = index_at(u + 1);
-      const uint32_t bytes = (c1 - c0) * 16u;
-      uint32_t p = vhead;
-      if (p % ring_bytes + bytes > ring_bytes) p = (p / ring_bytes + 1) * ring_bytes;
-      const bool empty = issued == consumed;
-      if (!empty && p + bytes - vtail > ring_bytes) break;
-      if (empty) vtail = p;
-      const int slot = (int)(issued % kDepth);
-      if (lane == slot) slot_vpos = p;
-      if (lane == 0) {
-        mbar_expect_tx(&bars[slot], bytes);
-        bulk_load(ring + p % ring_bytes, tiles + 16ull * c0, bytes, &bars[slot]);
-      }
-      vhead = p + bytes;
-      ++issued;
-    }
-  }
-  // Waits for tile `consumed`; returns its chunk or nullptr on timeout.
-  __device__ const uint8_t* wait_current() {
-    const int slot = (int)(consumed % kDepth);
-    const uint32_t parity = (uint32_t)((consumed / kDepth) & 1);
-    const bool ok = wait_bounded(&bars[slot], parity);
-    if (!__all_sync(kFull, ok)) return nullptr;
-    const uint32_t p = __shfl_sync(kFull, slot_vpos, slot);
-    return ring + p % ring_bytes;
-  }
-  __device__ void release_current() {
-    __syncwarp();
-    ++consumed;
-    if (issued > consumed)
-      vtail = __shfl_sync(kFull, slot_vpos, (int)(consumed % kDepth));
-    else
-      vtail = vhead;
-    if (lane == 0) fence_proxy_async();
-    __syncwarp();
-  }
-  // After a timeout: wait (bounded) for every copy still in flight.
-  __device__ void drain() {
-    for (int64_t c = consumed; c < issued; ++c)
-      wait_bounded(&bars[c % kDepth], (uint32_t)((c / kDepth) & 1));
-  }
+// ---- shared-memory layout and the producer ---------------------------------
+//
+// Tiles move in fixed batches of p.batch_tiles consecutive tiles (consecutive in
+// HBM too), one bulk copy per batch, so that each copy is large enough for the
+// copy engine to run at full bandwidth.  Batch k has a "full" barrier counting
+// its bytes; every tile has its own "empty" barrier, arrived at by the consumer
+// that decoded it.
+
+struct Smem {
+  uint64_t* table_bar;
+  uint64_t* full;    // per batch slot
+  uint64_t* empty;   // per tile slot
+  uint32_t* desc;    // per tile slot: ring offset of the tile's chunk
+  uint32_t* vstart;  // per tile slot: virtual ring position (producer)
+  uint8_t* ring;
 };
 
-// Shared-memory layout: decode table | table barrier | per-warp barriers |
-// per-warp rings.
-__host__ __device__ inline size_t ring_offset(int warps) {
-  return ((size_t)kTableBytes + 8 + (size_t)warps * kDepth * 8 + 15) / 16 * 16;
+__device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
+  Smem s;
+  s.table_bar = reinterpret_cast<uint64_t*>(smem + p.table_bytes);
+  s.full = s.table_bar + 1;
+  s.empty = s.full + kSlots;
+  s.desc = reinterpret_cast<uint32_t*>(s.empty + kSlots);
+  s.vstart = s.desc + kSlots;
+  s.ring = smem + p.ring_offset;
+  return s;
 }
-__host__ __device__ inline size_t smem_bytes_for(int warps, int ring_bytes) {
-  return ring_offset(warps) + (size_t)warps * (size_t)(ring_bytes + kRingSlack);
+
+// Streams tiles [first, first + n) into the ring, batch by batch; run by the
+// whole producer warp (uniform control flow), lane 0 issuing the copies.  The
+// chunk offsets come 32 at a time from one coalesced load.  A batch is
+// contiguous in the ring; ring space is reused once consumers release tiles.
+__device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, int64_t first, int n,
+                        int lane) {
+  if (lane == 0) {
+    mbar_expect_tx(s.table_bar, p.table_bytes);
+    bulk_load(smem, p.table, p.table_bytes, s.table_bar);
+  }
+  const int T = p.batch_tiles;
+  const uint32_t R = (uint32_t)p.ring_bytes;
+  uint32_t vhead = 0, vtail = 0;  // virtual ring positions
+  uint32_t phys = 0;              // vhead % R, kept incrementally
+  int q_tail = 0;                 // oldest tile whose release has not been seen
+  int wbase = 0;                  // index window: offsets of tiles wbase .. wbase + 63
+  uint32_t wa = lane <= n ? __ldg(p.index + first + lane) : 0u;
+  uint32_t wb = 32 + lane <= n ? __ldg(p.index + first + 32 + lane) : 0u;
+  auto offset_of = [&](int k) -> uint32_t {  // index[first + k], k in [wbase, wbase + 64)
+    const int d = k - wbase;
+    const uint32_t va = __shfl_sync(kFull, wa, d & 31);
+    const uint32_t vb = __shfl_sync(kFull, wb, d & 31);
+    return d < 32 ? va : vb;
+  };
+  bool ok = true;
+  int q0 = 0;
+  for (; q0 < n && ok; q0 += T) {
+    const int q1 = q0 + T < n ? q0 + T : n;
+    while (q1 - wbase >= 64) {  // slide the offset window (uniform)
+      wbase += 32;
+      wa = wb;
+      wb = wbase + 32 + lane <= n ? __ldg(p.index + first + wbase + 32 + lane) : 0u;
+    }
+    const uint32_t c0 = offset_of(q0), c1 = offset_of(q1);
+    const uint32_t bytes = (c1 - c0) * 16u;
+    uint32_t at = vhead, at_phys = phys;
+    if (at_phys + bytes > R) {  // a batch never wraps
+      at += R - at_phys;
+      at_phys = 0;
+    }
+    // Room: at most kSlots tiles resident, and the batch must not reach into
+    // bytes of unreleased tiles.
+    while (q_tail < q0 && (q1 - q_tail > kSlots || at + bytes - vtail > R)) {
+      if (!__all_sync(kFull, wait_bounded(&s.empty[q_tail % kSlots],
+                                          (uint32_t)((q_tail / kSlots) & 1)))) {
+        ok = false;
+        break;
+      }
+      ++q_tail;
+      vtail = q_tail < q0 ? s.vstart[q_tail % kSlots] : at;
+    }
+    if (!ok) break;
+    if (q_tail == q0) vtail = at;
+    // Per-tile ring offsets of the batch, then one copy for all of it.
+    const uint32_t off = (offset_of(lane < q1 - q0 ? q0 + lane : q0) - c0) * 16u;
+    if (lane < q1 - q0) {
+      s.vstart[(q0 + lane) % kSlots] = at + off;
+      s.desc[(q0 + lane) % kSlots] = at_phys + off;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      uint64_t* bar = &s.full[(q0 / T) % kSlots];
+      mbar_expect_tx(bar, bytes);  // arrive (release) + byte count
+      bulk_load(s.ring + at_phys, p.tiles + 16ull * c0, bytes, bar);
+    }
+    __syncwarp();
+    vhead = at + bytes;
+    phys = at_phys + bytes;
+  }
+  // Leave no copy in flight: wait for the last use of every batch slot issued.
+  const int batches = (q0 + T - 1) / T;  // batches [0, batches) were issued
+  if (lane == 0) {
+    for (int k = batches - 1; k >= 0 && k >= batches - kSlots; --k)
+      wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1));
+    wait_bounded(s.table_bar, 0);
+  }
+}
+
+// Consumer side: wait for tile q's batch; returns the chunk's ring offset.
+__device__ __forceinline__ bool wait_tile(const TileParams& p, const Smem& s, int q) {
+  const int k = q / p.batch_tiles;
+  return __all_sync(kFull, wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1)));
 }
 
 // Sums 8 per-lane row values over the 32 lanes.  On return every lane holds the
@@ -293,125 +383,109 @@ __device__ __forceinline__ float reduce_rows8(const float (&v)[8], int lane) {
   return c;
 }
 
-template <int CP, int B>
-struct GemvState {
-  float acc[8][B];
-  float xl[CP][B], xh[CP][B];  // x pairs of this lane's columns
-  int64_t xcol_block;          // column block whose x is loaded
-};
+__device__ __forceinline__ uint32_t load_x_pair(const uint16_t* x, int64_t cols, int64_t col) {
+  if (col + 1 < cols) return __ldg(reinterpret_cast<const uint32_t*>(x + col));
+  if (col < cols) return __ldg(x + col);
+  return 0u;
+}
 
-template <int CP, int B, bool RAGGED>
-__device__ __forceinline__ void decode_gemv_tile(const uint8_t* chunk, const uint32_t* table,
-                                                 int lane, GemvState<CP, B>& st) {
+// One tile of the GEMV: decode the lane's 16 * CP symbols, 8 rows per 64-column
+// group, and accumulate acc[r][b] += W[r][c] * x[b][c] in FP32.  The BF16 pair
+// of x for each group (columns col0 + 64 g + 2 lane, + 1) is read from L1 one
+// group ahead and serves the group's 8 rows.
+template <int CP, int B, bool FAST>
+__device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table, int lane,
+                                                 float (&acc)[8][B], const uint16_t* x,
+                                                 int64_t cols, int64_t col0) {
   constexpr int kRaw = CP * 512;
-  const uint32_t my_len = chunk[kRaw + lane];
-  uint32_t incl = my_len;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t v = __shfl_up_sync(kFull, incl, o);
-    if (lane >= o) incl += v;
-  }
   BitReader br;
-  br.init(chunk + kRaw + kLanes, incl - my_len);
+  br.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane));
+  uint32_t xn[B];
 #pragma unroll
+  for (int b = 0; b < B; ++b) xn[b] = load_x_pair(x + (int64_t)b * cols, cols, col0 + 2 * lane);
+#pragma unroll 1
   for (int g = 0; g < CP; ++g) {
-    const uint4 rv = *reinterpret_cast<const uint4*>(chunk + g * 512 + lane * 16);
+    const uint4 rv = lds128(chunk + g * 512 + lane * 16);
+    uint32_t xg[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) xg[b] = xn[b];
+    if (g + 1 < CP) {
+#pragma unroll
+      for (int b = 0; b < B; ++b)
+        xn[b] = load_x_pair(x + (int64_t)b * cols, cols, col0 + (g + 1) * 64 + 2 * lane);
+    }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const uint32_t e = decode_pair(br, table);
-      uint32_t rawdup;
-      switch (r) {
-        case 0: rawdup = raw_pair<0>(rv); break;
-        case 1: rawdup = raw_pair<1>(rv); break;
-        case 2: rawdup = raw_pair<2>(rv); break;
-        case 3: rawdup = raw_pair<3>(rv); break;
-        case 4: rawdup = raw_pair<4>(rv); break;
-        case 5: rawdup = raw_pair<5>(rv); break;
-        case 6: rawdup = raw_pair<6>(rv); break;
-        default: rawdup = raw_pair<7>(rv); break;
-      }
-      const uint32_t w = assemble(rawdup, e);
-      const float wl = bf16_lo(w), wh = bf16_hi(w);
+      const uint32_t e = decode_pair<FAST>(br, table);
+      const uint32_t w = assemble(raw_pair_r(rv, r), e);
 #pragma unroll
       for (int b = 0; b < B; ++b) {
-        st.acc[r][b] = fmaf(wl, st.xl[g][b], st.acc[r][b]);
-        st.acc[r][b] = fmaf(wh, st.xh[g][b], st.acc[r][b]);
+        acc[r][b] = fma_bf16<false>(w, xg[b], acc[r][b]);
+        acc[r][b] = fma_bf16<true>(w, xg[b], acc[r][b]);
       }
       if (r & 1) br.refill();
     }
   }
 }
 
-template <int CP, int B>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(TileParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
-  uint32_t* table = reinterpret_cast<uint32_t*>(smem);
-  uint64_t* table_bar = reinterpret_cast<uint64_t*>(smem + kTableBytes);
-  uint64_t* bars = table_bar + 1 + warp * kDepth;
-  uint8_t* ring = smem + ring_offset(warps) + (size_t)warp * (p.ring_bytes + kRingSlack);
+// Tile range of this CTA.
+__device__ __forceinline__ void cta_range(const TileParams& p, int64_t* first, int* n) {
+  const int64_t a = p.n_tiles * (int64_t)blockIdx.x / gridDim.x;
+  const int64_t b = p.n_tiles * (int64_t)(blockIdx.x + 1) / gridDim.x;
+  *first = a;
+  *n = (int)(b - a);
+}
 
-  if (threadIdx.x == 0) mbar_init(table_bar, 1);
-  if (lane == 0)
-    for (int d = 0; d < kDepth; ++d) mbar_init(&bars[d], 1);
+// Sets up barriers; returns false for the producer warp (its work is done) and
+// for consumers when the decode table never arrived.
+__device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const Smem& s,
+                                      int64_t first, int n) {
+  if (threadIdx.x == 0) {
+    mbar_init(s.table_bar, 1);
+    for (int k = 0; k < kSlots; ++k) {
+      mbar_init(&s.full[k], 1);
+      mbar_init(&s.empty[k], 1);
+    }
+  }
   fence_barrier_init();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_expect_tx(table_bar, kTableBytes);
-    bulk_load(table, p.table, kTableBytes, table_bar);
+  const int warp = threadIdx.x >> 5;
+  if (warp == kConsumers) {
+    produce(p, smem, s, first, n, threadIdx.x & 31);
+    return false;
   }
+  return __all_sync(kFull, wait_bounded(s.table_bar, 0));
+}
 
-  const int64_t gw = (int64_t)blockIdx.x * warps + warp;
-  const int64_t first = gw < p.total_warps ? p.n_tiles * gw / p.total_warps : 0;
-  const int64_t last = gw < p.total_warps ? p.n_tiles * (gw + 1) / p.total_warps : 0;
-  Pipeline pl;
-  pl.init(p.tiles, p.index, p.n_tiles, ring, (uint32_t)p.ring_bytes, bars, first, last - first,
-          lane);
-  pl.issue();
-  if (!__all_sync(kFull, wait_bounded(table_bar, 0))) {
-    if (threadIdx.x == 0) wait_bounded(table_bar, 0);
-    pl.drain();
-    return;
-  }
-
-  GemvState<CP, B> st;
-  st.xcol_block = -1;
+template <int CP, int B, bool FAST>
+__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(TileParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Smem s = carve(smem, p);
+  int64_t first;
+  int n;
+  cta_range(p, &first, &n);
+  if (!setup(p, smem, s, first, n)) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t table = smem_u32(smem);
+  const uint32_t ring = smem_u32(s.ring);
   const int64_t cols = p.cols;
-  for (int64_t c = 0; c < pl.n; ++c) {
-    const int64_t u = pl.u0 + c;
+  for (int q = warp; q < n; q += kConsumers) {
+    const int slot = q % kSlots;
+    if (!wait_tile(p, s, q)) return;
+    const uint32_t chunk = ring + s.desc[slot];
+    const int64_t u = first + q;
     const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
-    if (j != st.xcol_block) {  // load this lane's x pairs for column block j
-      st.xcol_block = j;
-#pragma unroll
-      for (int g = 0; g < CP; ++g) {
-        const int64_t col = j * (CP * 64) + g * 64 + 2 * lane;
-#pragma unroll
-        for (int b = 0; b < B; ++b) {
-          uint32_t xv = 0;
-          if (col + 1 < cols) {
-            xv = __ldg(reinterpret_cast<const uint32_t*>(p.x + (int64_t)b * cols + col));
-          } else if (col < cols) {
-            xv = __ldg(p.x + (int64_t)b * cols + col);
-          }
-          st.xl[g][b] = bf16_lo(xv);
-          st.xh[g][b] = bf16_hi(xv);
-        }
-      }
-    }
+    float acc[8][B];
 #pragma unroll
     for (int r = 0; r < 8; ++r)
 #pragma unroll
-      for (int b = 0; b < B; ++b) st.acc[r][b] = 0.f;
-
-    const uint8_t* chunk = pl.wait_current();
-    if (!chunk) {
-      pl.drain();
-      return;
+      for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
+    decode_gemv_tile<CP, B, FAST>(chunk, table, lane, acc, p.x, cols, j * (CP * 64));
+    __syncwarp();
+    if (lane == 0) {
+      fence_proxy_async();
+      mbar_arrive(&s.empty[slot]);
     }
-    decode_gemv_tile<CP, B, false>(chunk, table, lane, st);
-    pl.release_current();
-    pl.issue();
 
     // Row sums of this tile: lane L holds row L >> 2 for every batch row.
     float tot[B];
@@ -419,115 +493,96 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) gemv_kernel(TileParams p) {
     for (int b = 0; b < B; ++b) {
       float v[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) v[r] = st.acc[r][b];
+      for (int r = 0; r < 8; ++r) v[r] = acc[r][b];
       tot[b] = reduce_rows8(v, lane);
     }
-    const int r = lane >> 2;
-    const int64_t row = i * 8 + r;
-    if (p.tiles_c == 1) {
-      if ((lane & 3) == 0 && row < p.rows)
+    const int64_t row = i * 8 + (lane >> 2);
+    if ((lane & 3) == 0) {
+      if (p.tiles_c == 1) {
+        if (row < p.rows)
 #pragma unroll
-        for (int b = 0; b < B; ++b) p.y[(int64_t)b * p.rows + row] = tot[b];
-      continue;
+          for (int b = 0; b < B; ++b) p.y[(int64_t)b * p.rows + row] = tot[b];
+      } else {
+#pragma unroll
+        for (int b = 0; b < B; ++b)
+          __stcg(&p.partial[((int64_t)j * B + b) * p.rows_pad + row], tot[b]);
+      }
     }
-    if ((lane & 3) == 0)
-#pragma unroll
-      for (int b = 0; b < B; ++b)
-        p.partial[((int64_t)j * B + b) * p.rows_pad + row] = tot[b];
-    __threadfence();
-    __syncwarp();
-    uint32_t arrived = 0;
-    if (lane == 0) arrived = atomicAdd(&p.counters[i], 1u);
-    arrived = __shfl_sync(kFull, arrived, 0);
-    if (arrived == (uint32_t)(p.tiles_c - 1)) {
-      // Last arrival for row block i: sum the partials in column-block order.
-      __threadfence();
-      for (int q = lane; q < 8 * B; q += 32) {
-        const int b = q >> 3, rr = q & 7;
+  }
+  if (p.tiles_c == 1) return;
+  // Split-K, once per warp after all its tiles: publish (fence, then count the
+  // arrivals of all the warp's tiles at once); the last of a row block's
+  // tiles_c arrivals sums its partials in column-block order and writes y.
+  __threadfence();
+  __syncwarp();
+  for (int q0 = warp; q0 < n; q0 += 32 * kConsumers) {
+    const int q = q0 + lane * kConsumers;
+    uint32_t last = 0;
+    if (q < n) {
+      const int64_t i = (first + q) % p.tiles_r;
+      last = atomicAdd(&p.counters[i], 1u) == (uint32_t)(p.tiles_c - 1);
+    }
+    uint32_t mask = __ballot_sync(kFull, last);
+    if (mask) __threadfence();
+    while (mask) {
+      const int src = __ffs(mask) - 1;
+      mask &= mask - 1;
+      const int64_t i = (first + q0 + src * kConsumers) % p.tiles_r;
+      for (int qq = lane; qq < 8 * B; qq += 32) {
+        const int b = qq >> 3, rr = qq & 7;
         const int64_t orow = i * 8 + rr;
-        float s = 0.f;
-        for (int64_t jj = 0; jj < p.tiles_c; ++jj)
-          s += __ldcg(&p.partial[(jj * B + b) * p.rows_pad + orow]);
-        if (orow < p.rows) p.y[(int64_t)b * p.rows + orow] = s;
+        const float* part = p.partial + (int64_t)b * p.rows_pad + orow;
+        const int64_t stride = (int64_t)B * p.rows_pad;
+        float sum = 0.f;
+        int64_t jj = 0;
+        for (; jj + 8 <= p.tiles_c; jj += 8) {
+          float v[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) v[k] = __ldcg(part + (jj + k) * stride);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) sum += v[k];
+        }
+        for (; jj < p.tiles_c; ++jj) sum += __ldcg(part + jj * stride);
+        if (orow < p.rows) p.y[(int64_t)b * p.rows + orow] = sum;
       }
       if (lane == 0) p.counters[i] = 0u;
     }
   }
 }
 
-template <int CP>
-__global__ void __launch_bounds__(kMaxWarps * 32, 1) decompress_kernel(TileParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
+template <int CP, bool FAST>
+__global__ void __launch_bounds__(kThreads, 1) decompress_kernel(TileParams p) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const Smem s = carve(smem, p);
+  int64_t first;
+  int n;
+  cta_range(p, &first, &n);
+  if (!setup(p, smem, s, first, n)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
-  uint32_t* table = reinterpret_cast<uint32_t*>(smem);
-  uint64_t* table_bar = reinterpret_cast<uint64_t*>(smem + kTableBytes);
-  uint64_t* bars = table_bar + 1 + warp * kDepth;
-  uint8_t* ring = smem + ring_offset(warps) + (size_t)warp * (p.ring_bytes + kRingSlack);
-
-  if (threadIdx.x == 0) mbar_init(table_bar, 1);
-  if (lane == 0)
-    for (int d = 0; d < kDepth; ++d) mbar_init(&bars[d], 1);
-  fence_barrier_init();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_expect_tx(table_bar, kTableBytes);
-    bulk_load(table, p.table, kTableBytes, table_bar);
-  }
-  const int64_t gw = (int64_t)blockIdx.x * warps + warp;
-  const int64_t first = gw < p.total_warps ? p.n_tiles * gw / p.total_warps : 0;
-  const int64_t last = gw < p.total_warps ? p.n_tiles * (gw + 1) / p.total_warps : 0;
-  Pipeline pl;
-  pl.init(p.tiles, p.index, p.n_tiles, ring, (uint32_t)p.ring_bytes, bars, first, last - first,
-          lane);
-  pl.issue();
-  if (!__all_sync(kFull, wait_bounded(table_bar, 0))) {
-    if (threadIdx.x == 0) wait_bounded(table_bar, 0);
-    pl.drain();
-    return;
-  }
+  const uint32_t table = smem_u32(smem);
+  const uint32_t ring = smem_u32(s.ring);
   const int64_t cols = p.cols;
   const bool even_cols = (cols & 1) == 0;
-  uint32_t invalid = 0;
   constexpr int kRaw = CP * 512;
-  for (int64_t c = 0; c < pl.n; ++c) {
-    const int64_t u = pl.u0 + c;
+  uint32_t invalid = 0;
+  for (int q = warp; q < n; q += kConsumers) {
+    const int slot = q % kSlots;
+    if (!wait_tile(p, s, q)) return;
+    const uint32_t chunk = ring + s.desc[slot];
+    const int64_t u = first + q;
     const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
-    const uint8_t* chunk = pl.wait_current();
-    if (!chunk) {
-      pl.drain();
-      return;
-    }
-    const uint32_t my_len = chunk[kRaw + lane];
-    uint32_t incl = my_len;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t v = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += v;
-    }
     BitReader br;
-    br.init(chunk + kRaw + kLanes, incl - my_len);
+    br.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane));
     const bool full_tile = (i + 1) * 8 <= p.rows && (j + 1) * (CP * 64) <= cols && even_cols;
-#pragma unroll
+#pragma unroll 1
     for (int g = 0; g < CP; ++g) {
-      const uint4 rv = *reinterpret_cast<const uint4*>(chunk + g * 512 + lane * 16);
+      const uint4 rv = lds128(chunk + g * 512 + lane * 16);
       const int64_t col = j * (CP * 64) + g * 64 + 2 * lane;
 #pragma unroll
       for (int r = 0; r < 8; ++r) {
-        const uint32_t e = decode_pair(br, table);
+        const uint32_t e = decode_pair<FAST>(br, table);
         invalid |= e;
-        uint32_t rawdup;
-        switch (r) {
-          case 0: rawdup = raw_pair<0>(rv); break;
-          case 1: rawdup = raw_pair<1>(rv); break;
-          case 2: rawdup = raw_pair<2>(rv); break;
-          case 3: rawdup = raw_pair<3>(rv); break;
-          case 4: rawdup = raw_pair<4>(rv); break;
-          case 5: rawdup = raw_pair<5>(rv); break;
-          case 6: rawdup = raw_pair<6>(rv); break;
-          default: rawdup = raw_pair<7>(rv); break;
-        }
-        const uint32_t w = assemble(rawdup, e);
+        const uint32_t w = assemble(raw_pair_r(rv, r), e);
         const int64_t row = i * 8 + r;
         if (full_tile) {
           *reinterpret_cast<uint32_t*>(p.out + row * cols + col) = w;
@@ -538,8 +593,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) decompress_kernel(TileParam
         if (r & 1) br.refill();
       }
     }
-    pl.release_current();
-    pl.issue();
+    __syncwarp();
+    if (lane == 0) {
+      fence_proxy_async();
+      mbar_arrive(&s.empty[slot]);
+    }
   }
   if (__any_sync(kFull, invalid & kEntryInvalid) && lane == 0)
     atomicOr(&g_device_error, kErrCorrupt);
@@ -559,75 +617,91 @@ cudaError_t ensure_smem(Kernel k, size_t bytes, int (&configured)[64]) {
   return e;
 }
 
-template <int CP, int B>
-cudaError_t launch_gemv_cp_b(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+template <int CP, int B, bool FAST>
+cudaError_t launch_gemv_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(gemv_kernel<CP, B>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(gemv_kernel<CP, B, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  gemv_kernel<CP, B><<<s.ctas, s.warps_per_cta * 32, s.smem_bytes, stream>>>(p);
+  gemv_kernel<CP, B, FAST><<<s.ctas, kThreads, s.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
-template <int CP>
+template <int CP, bool FAST>
 cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   switch (p.batch) {
-    case 1: return launch_gemv_cp_b<CP, 1>(p, s, stream);
-    case 2: return launch_gemv_cp_b<CP, 2>(p, s, stream);
-    case 3: return launch_gemv_cp_b<CP, 3>(p, s, stream);
-    case 4: return launch_gemv_cp_b<CP, 4>(p, s, stream);
-    case 5: return launch_gemv_cp_b<CP, 5>(p, s, stream);
-    case 6: return launch_gemv_cp_b<CP, 6>(p, s, stream);
-    case 7: return launch_gemv_cp_b<CP, 7>(p, s, stream);
-    case 8: return launch_gemv_cp_b<CP, 8>(p, s, stream);
+    case 1: return launch_gemv_t<CP, 1, FAST>(p, s, stream);
+    case 2: return launch_gemv_t<CP, 2, FAST>(p, s, stream);
+    case 3: return launch_gemv_t<CP, 3, FAST>(p, s, stream);
+    case 4: return launch_gemv_t<CP, 4, FAST>(p, s, stream);
+    case 5: return launch_gemv_t<CP, 5, FAST>(p, s, stream);
+    case 6: return launch_gemv_t<CP, 6, FAST>(p, s, stream);
+    case 7: return launch_gemv_t<CP, 7, FAST>(p, s, stream);
+    case 8: return launch_gemv_t<CP, 8, FAST>(p, s, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int CP>
-cudaError_t launch_decompress_cp(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+template <int CP, bool FAST>
+cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(decompress_kernel<CP>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(decompress_kernel<CP, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  decompress_kernel<CP><<<s.ctas, s.warps_per_cta * 32, s.smem_bytes, stream>>>(p);
+  decompress_kernel<CP, FAST><<<s.ctas, kThreads, s.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, int sm_count) {
+LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_chunk,
+                         uint32_t table_bytes, int sm_count, size_t smem_limit) {
   LaunchShape s;
-  const int64_t target = (int64_t)sm_count * kMaxWarps;
-  const int64_t warps = n_tiles < target ? n_tiles : target;
-  int per_cta = (int)((warps + sm_count - 1) / sm_count);
-  if (per_cta < 1) per_cta = 1;
-  if (per_cta > kMaxWarps) per_cta = kMaxWarps;
-  s.warps_per_cta = per_cta;
-  s.ctas = (int)((warps + per_cta - 1) / per_cta);
-  // Room for one worst-case chunk and, typically, two ordinary ones.
-  const uint64_t ring = (max_chunk + 15) / 16 * 16;
-  s.ring_bytes = (int)(ring > 12288 ? ring : 12288);
-  s.smem_bytes = smem_bytes_for(per_cta, s.ring_bytes);
+  s.ctas = (int)(n_tiles < sm_count ? n_tiles : sm_count);
+  if (s.ctas < 1) s.ctas = 1;
+  s.table_bytes = table_bytes;
+  // table | table barrier | full[] | empty[] | desc[] | vstart[] | ring
+  const size_t head = (size_t)table_bytes + 8 + 2 * kSlots * 8 + 2 * kSlots * 4;
+  s.ring_offset = (head + 127) / 128 * 128;
+  const int64_t per_cta = (n_tiles + s.ctas - 1) / s.ctas;
+  // Tiles per bulk copy: enough for >= 16 KB of typical chunks, at most 8 and
+  // never more than a quarter of the slots.
+  int t = (int)((16384 + typical_chunk - 1) / (typical_chunk ? typical_chunk : 1));
+  if (t < 1) t = 1;
+  if (t > 8) t = 8;
+  s.batch_tiles = t;
+  // As much ring as the device allows, but no more than the CTA's tiles need.
+  size_t ring = smem_limit > s.ring_offset + kRingSlack + max_chunk
+                    ? smem_limit - s.ring_offset - kRingSlack
+                    : 0;
+  // A batch of worst-case chunks must fit, and the ring need not exceed the
+  // CTA's whole range.
+  const size_t batch_max = (size_t)s.batch_tiles * (size_t)max_chunk;
+  const size_t need = (size_t)per_cta * (size_t)max_chunk;
+  if (ring > need) ring = need;
+  ring = ring / 16 * 16;
+  if (ring < batch_max) ring = (batch_max + 15) / 16 * 16;
+  s.ring_bytes = (int)ring;
+  s.smem_bytes = s.ring_offset + ring + kRingSlack;
   return s;
 }
 
-cudaError_t launch_gemv(const TileParams& p, int tile_cols, const LaunchShape& s,
+cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const LaunchShape& s,
                         cudaStream_t stream) {
   switch (tile_cols) {
-    case 512: return launch_gemv_cp<8>(p, s, stream);
-    case 256: return launch_gemv_cp<4>(p, s, stream);
-    case 128: return launch_gemv_cp<2>(p, s, stream);
-    case 64: return launch_gemv_cp<1>(p, s, stream);
+    case 512: return fast ? launch_gemv_cp<8, true>(p, s, stream) : launch_gemv_cp<8, false>(p, s, stream);
+    case 256: return fast ? launch_gemv_cp<4, true>(p, s, stream) : launch_gemv_cp<4, false>(p, s, stream);
+    case 128: return fast ? launch_gemv_cp<2, true>(p, s, stream) : launch_gemv_cp<2, false>(p, s, stream);
+    case 64: return fast ? launch_gemv_cp<1, true>(p, s, stream) : launch_gemv_cp<1, false>(p, s, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_decompress(const TileParams& p, int tile_cols, const LaunchShape& s,
-                              cudaStream_t stream) {
+cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
+                              const LaunchShape& s, cudaStream_t stream) {
   switch (tile_cols) {
-    case 512: return launch_decompress_cp<8>(p, s, stream);
-    case 256: return launch_decompress_cp<4>(p, s, stream);
-    case 128: return launch_decompress_cp<2>(p, s, stream);
-    case 64: return launch_decompress_cp<1>(p, s, stream);
+    case 512: return fast ? launch_decompress_t<8, true>(p, s, stream) : launch_decompress_t<8, false>(p, s, stream);
+    case 256: return fast ? launch_decompress_t<4, true>(p, s, stream) : launch_decompress_t<4, false>(p, s, stream);
+    case 128: return fast ? launch_decompress_t<2, true>(p, s, stream) : launch_decompress_t<2, false>(p, s, stream);
+    case 64: return fast ? launch_decompress_t<1, true>(p, s, stream) : launch_decompress_t<1, false>(p, s, stream);
     default: return cudaErrorInvalidValue;
   }
 }

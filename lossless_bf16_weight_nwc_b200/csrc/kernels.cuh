@@ -12,11 +12,13 @@ constexpr uint32_t kErrCorrupt = 2u;   // a stream held no valid code
 struct TileParams {
   const uint8_t* tiles;     // device: tile area of the blob
   const uint32_t* index;    // device: chunk offsets (16-byte units), tiles + 1
-  const uint32_t* table;    // device: 4096-entry decode table
+  const uint32_t* table;    // device: decode table (table_bytes)
+  uint32_t table_bytes;     // 64 KiB (14-bit peek) or 16 KiB (12-bit peek)
+  uint32_t ring_offset;     // shared-memory offset of the staging ring
   int64_t rows, cols;
   int64_t tiles_r, tiles_c, n_tiles;
-  int32_t total_warps;      // warps sharing the tiles (contiguous ranges)
-  int32_t ring_bytes;       // per-warp staging ring in shared memory
+  int32_t ring_bytes;       // CTA staging ring in shared memory
+  int32_t batch_tiles;      // consecutive tiles moved by one bulk copy
   // GEMV
   const uint16_t* x;        // BF16 [batch x cols]
   float* y;                 // FP32 [batch x rows]
@@ -29,19 +31,25 @@ struct TileParams {
 };
 
 struct LaunchShape {
-  int ctas;
-  int warps_per_cta;
+  int ctas;             // one persistent CTA per SM (fewer for small matrices)
+  uint32_t table_bytes;
+  size_t ring_offset;
   int ring_bytes;
+  int batch_tiles;
   size_t smem_bytes;
 };
 
-// Picks the grid for n_tiles tiles whose largest chunk is max_chunk bytes.
-LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, int sm_count);
+// Grid and shared-memory layout for n_tiles tiles whose largest chunk is
+// max_chunk bytes (typical_chunk on average), within the device's per-block
+// shared-memory limit.
+LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_chunk,
+                         uint32_t table_bytes, int sm_count, size_t smem_limit);
 
-cudaError_t launch_gemv(const TileParams& p, int tile_cols, const LaunchShape& s,
+// fast: lmax <= 7 (14-bit peek, two codes per entry always).
+cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const LaunchShape& s,
                         cudaStream_t stream);
-cudaError_t launch_decompress(const TileParams& p, int tile_cols, const LaunchShape& s,
-                              cudaStream_t stream);
+cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
+                              const LaunchShape& s, cudaStream_t stream);
 cudaError_t read_and_clear_error(uint32_t* word);
 
 }  // namespace nwc

@@ -20,23 +20,40 @@ using nwc::round_up;
 
 constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {};
+int g_smem_optin[kMaxDevices] = {};
 std::mutex g_mu;
 
 nwc_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NWC_OK : NWC_ERR_CUDA; }
 
-// Number of SMs of the current device (cached).
-nwc_status current_device(int* dev, int* sms) {
+// SM count and per-block opt-in shared memory of the current device (cached).
+nwc_status current_device(int* dev, int* sms, size_t* smem) {
   cudaError_t e = cudaGetDevice(dev);
   if (e != cudaSuccess) return NWC_ERR_CUDA;
   if (*dev < 0 || *dev >= kMaxDevices) return NWC_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_mu);
   if (!g_sm_count[*dev]) {
-    int v = 0;
+    int v = 0, m = 0;
     e = cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, *dev);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&m, cudaDevAttrMaxSharedMemoryPerBlockOptin, *dev);
     if (e != cudaSuccess) return NWC_ERR_CUDA;
     g_sm_count[*dev] = v;
+    g_smem_optin[*dev] = m;
   }
   *sms = g_sm_count[*dev];
+  *smem = (size_t)g_smem_optin[*dev];
+  return NWC_OK;
+}
+
+// Launch geometry for a handle on the current device.
+nwc_status shape_for(const nwc_handle_s& h, nwc::LaunchShape* s) {
+  int dev, sms;
+  size_t smem;
+  nwc_status st = current_device(&dev, &sms, &smem);
+  if (st != NWC_OK) return st;
+  const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
+  *s = nwc::launch_shape(h.tiles, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms, smem);
+  if (s->smem_bytes > smem) return NWC_ERR_UNSUPPORTED;
   return NWC_OK;
 }
 
@@ -48,6 +65,7 @@ nwc::TileParams base_params(const nwc_handle_s& h) {
   p.tiles = h.d_base + h.tiles_off;
   p.index = reinterpret_cast<const uint32_t*>(h.d_base + h.index_off);
   p.table = reinterpret_cast<const uint32_t*>(h.d_base + h.table_off);
+  p.table_bytes = nwc::table_bytes(h.lmax);
   p.rows = h.rows;
   p.cols = h.cols;
   p.tiles_r = h.tiles_r;
@@ -105,7 +123,7 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
   if (!w_host || !out_plan || rows < 1 || cols < 1) return NWC_ERR_INVALID_ARG;
   if (rows > (1ll << 40) || cols > (1ll << 40)) return NWC_ERR_INVALID_ARG;
   *out_plan = nullptr;
-  uint32_t lmax = 12, tile_rows = 8, tile_cols = 512, threads = 0;
+  uint32_t lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0;
   if (opts) {
     if (opts->struct_size < sizeof(nwc_opts)) return NWC_ERR_INVALID_ARG;
     lmax = opts->lmax;
@@ -113,7 +131,7 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
     tile_cols = opts->tile_cols;
     threads = opts->threads;
   }
-  if (lmax < 1 || lmax > (uint32_t)nwc::kMaxLmax) return NWC_ERR_INVALID_ARG;
+  if (lmax > (uint32_t)nwc::kMaxLmax) return NWC_ERR_INVALID_ARG;
   if (tile_rows != 8) return NWC_ERR_UNSUPPORTED;
   if (tile_cols != 64 && tile_cols != 128 && tile_cols != 256 && tile_cols != 512)
     return NWC_ERR_UNSUPPORTED;
@@ -166,7 +184,7 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
     return NWC_ERR_NOMEM;
   }
   std::memset(img + plan->blob_bytes, 0, plan->table_off - plan->blob_bytes);
-  nwc::build_decode_table(plan->len, reinterpret_cast<uint32_t*>(img + plan->table_off));
+  nwc::build_decode_table(plan->len, plan->lmax, reinterpret_cast<uint32_t*>(img + plan->table_off));
   // From pageable memory the call returns once the bytes are staged, so the
   // image can be freed right after.
   cudaError_t e = cudaMemcpyAsync(d_buf, img, plan->device_bytes, cudaMemcpyHostToDevice,
@@ -199,15 +217,15 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, u
   nwc_status st = make_handle(static_cast<const uint8_t*>(blob), blob_bytes, d_buf, d_bytes, &h,
                               &lens);
   if (st != NWC_OK) return st;
-  std::vector<uint32_t> table(nwc::kTableEntries);
-  nwc::build_decode_table(lens, table.data());
+  std::vector<uint32_t> table(nwc::table_entries(h->lmax));
+  nwc::build_decode_table(lens, h->lmax, table.data());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(d_buf, blob, blob_bytes, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && h->table_off > blob_bytes)
     e = cudaMemsetAsync(static_cast<uint8_t*>(d_buf) + blob_bytes, 0, h->table_off - blob_bytes, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(static_cast<uint8_t*>(d_buf) + h->table_off, table.data(),
-                        nwc::kTableBytes, cudaMemcpyHostToDevice, s);
+                        nwc::table_bytes(h->lmax), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) {
     delete h;
@@ -245,15 +263,15 @@ nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes, nwc_handl
 
 nwc_status nwc_decompress(nwc_handle_t h, uint16_t* d_w_out, nwc_stream_t stream) {
   if (!h || !d_w_out || !aligned(d_w_out, 4)) return NWC_ERR_INVALID_ARG;
-  int dev, sms;
-  nwc_status st = current_device(&dev, &sms);
+  nwc::LaunchShape s;
+  nwc_status st = shape_for(*h, &s);
   if (st != NWC_OK) return st;
   nwc::TileParams p = base_params(*h);
   p.out = d_w_out;
-  const nwc::LaunchShape s = nwc::launch_shape(h->tiles, h->max_chunk, sms);
-  p.total_warps = s.ctas * s.warps_per_cta < h->tiles ? s.ctas * s.warps_per_cta : (int32_t)h->tiles;
+  p.ring_offset = (uint32_t)s.ring_offset;
   p.ring_bytes = s.ring_bytes;
-  return cuda_status(nwc::launch_decompress(p, (int)h->tile_cols, s,
+  p.batch_tiles = s.batch_tiles;
+  return cuda_status(nwc::launch_decompress(p, (int)h->tile_cols, h->lmax <= 7, s,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -272,13 +290,13 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
     return NWC_ERR_INVALID_ARG;
   // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
   if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
-  int dev, sms;
-  nwc_status st = current_device(&dev, &sms);
+  nwc::LaunchShape s;
+  nwc_status st = shape_for(*h, &s);
   if (st != NWC_OK) return st;
   nwc::TileParams p = base_params(*h);
-  const nwc::LaunchShape s = nwc::launch_shape(h->tiles, h->max_chunk, sms);
-  p.total_warps = s.ctas * s.warps_per_cta < h->tiles ? s.ctas * s.warps_per_cta : (int32_t)h->tiles;
+  p.ring_offset = (uint32_t)s.ring_offset;
   p.ring_bytes = s.ring_bytes;
+  p.batch_tiles = s.batch_tiles;
   if (need) {
     uint8_t* ws = static_cast<uint8_t*>(d_workspace);
     p.counters = reinterpret_cast<uint32_t*>(ws);
@@ -290,7 +308,7 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
     p.x = d_x + (int64_t)b0 * h->cols;
     p.y = d_y + (int64_t)b0 * h->rows;
     p.batch = nb;
-    cudaError_t e = nwc::launch_gemv(p, (int)h->tile_cols, s, cs);
+    cudaError_t e = nwc::launch_gemv(p, (int)h->tile_cols, h->lmax <= 7, s, cs);
     if (e != cudaSuccess) return NWC_ERR_CUDA;
   }
   return NWC_OK;

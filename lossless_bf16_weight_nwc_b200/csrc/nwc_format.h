@@ -15,7 +15,7 @@
 // column 64 (k/16) + 2t + k%2); its raw byte is at (k/16) * 512 + 16 t + k%16.
 // Tiles are stored column-block-major: u = j * tiles_r + i.
 //
-// Device image: blob | zero pad to 256 | decode table u32[4096].
+// Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)].
 #pragma once
 #include <cstdint>
 
@@ -30,17 +30,24 @@ constexpr int kLanes = 32;
 constexpr int kTileRows = 8;
 constexpr int kMaxTileCols = 512;
 constexpr int kMaxLmax = 12;
-constexpr int kPeekBits = 12;
-constexpr int kTableEntries = 1 << kPeekBits;
-constexpr uint32_t kTableBytes = kTableEntries * 4;
+constexpr int kMaxPeekBits = 14;
 
-// Decode-table entry for one 12-bit peek (most significant bit = next bit):
+// Width of the decoder's table peek for a length limit.  With lmax <= 7 the
+// peek is 14 bits, so every entry holds two complete codes and the decoder
+// never needs a second lookup ("NWC", "Prefix code instead of rANS": a table
+// peek yields two complete codes per step).  Longer codes use a 12-bit peek and
+// a second lookup when the pair does not fit.
+constexpr int peek_bits(uint32_t lmax) { return lmax <= 7 ? 14 : 12; }
+constexpr uint32_t table_entries(uint32_t lmax) { return 1u << peek_bits(lmax); }
+constexpr uint32_t table_bytes(uint32_t lmax) { return 4u * table_entries(lmax); }
+
+// Decode-table entry for one peek (most significant bit = next bit):
 //   bits  0..3   bits consumed by the step (both codes, or the first only)
 //   bits  7..14  first exponent byte  (its BF16 position in the low half)
 //   bits 15..18  length of the first code
 //   bit  19      the peek starts with no valid code (corrupt stream)
 //   bits 23..30  second exponent byte (its BF16 position in the high half)
-//   bit  31      the second code did not fit in the 12 bits
+//   bit  31      the second code did not fit in the peek (12-bit peek only)
 // Bits 4..6 stay zero so that a running difference of entries tracks the
 // number of consumed bits in its low 7 bits.
 constexpr uint32_t kEntryConsumedMask = 0xFu;

@@ -7,7 +7,7 @@
 
 struct nwc_plan_s {
   int64_t rows = 0, cols = 0;
-  uint32_t tile_rows = 8, tile_cols = 512, lmax = 12, threads = 0;
+  uint32_t tile_rows = 8, tile_cols = 512, lmax = 7, threads = 0;
   int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
   uint8_t len[256] = {};
   uint32_t code[256] = {};
@@ -24,7 +24,7 @@ struct nwc_handle_s {
   const uint8_t* d_base = nullptr;  // caller's device buffer
   uint64_t d_bytes = 0;
   int64_t rows = 0, cols = 0;
-  uint32_t tile_cols = 512, lmax = 12, filler = 0;
+  uint32_t tile_cols = 512, lmax = 7, filler = 0;
   int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
   uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0;
   uint64_t device_bytes = 0;
@@ -40,7 +40,8 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
 void encode_blob(const nwc_plan_s& plan, const uint16_t* w, uint8_t* blob);
 bool code_lengths(const uint64_t cnt[256], uint32_t lmax, uint8_t len[256]);
 void canonical_codes(const uint8_t len[256], uint32_t code[256]);
-void build_decode_table(const uint8_t len[256], uint32_t table[kTableEntries]);
+// Writes table_entries(lmax) entries.
+void build_decode_table(const uint8_t len[256], uint32_t lmax, uint32_t* table);
 // Parses and checks a blob's header, lens and index (the first head_bytes of a
 // blob of `bytes` bytes; head_bytes must reach the tile area); fills the
 // handle's geometry fields.  Returns false when the blob does not follow the

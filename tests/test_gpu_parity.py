@@ -58,13 +58,14 @@ SHAPES = [((8, 512), 512), ((9, 513), 512), ((77, 1030), 512), ((1, 2), 512),
           ((17, 130), 64), ((4100, 96), 512)]
 
 
+@pytest.mark.parametrize("lmax", [7, 12])
 @pytest.mark.parametrize("shape,tile_cols", SHAPES)
-def test_decompress_bit_exact(lib, orc, shape, tile_cols):
+def test_decompress_bit_exact(lib, orc, shape, tile_cols, lmax):
     spec = synth.MatrixSpec("w", shape[0], shape[1], "student_t5", 0.015, 1)
     w = synth.matrix(spec, 5)
-    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols)
+    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
     out = bits(m.decompress())
-    ref = orc.decode(orc.encode(w, tile_cols=tile_cols))
+    ref = orc.decode(orc.encode(w, tile_cols=tile_cols, lmax=lmax))
     assert np.array_equal(ref, w)
     assert np.array_equal(out, ref)
     no_device_error(lib)
@@ -72,7 +73,7 @@ def test_decompress_bit_exact(lib, orc, shape, tile_cols):
 
 def test_decompress_every_pattern(lib, orc):
     w = np.arange(65536, dtype=np.uint16).reshape(256, 256)
-    for tile_cols, lmax in ((512, 12), (128, 8)):
+    for tile_cols, lmax in ((512, 12), (128, 8), (256, 0)):
         m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
         assert np.array_equal(bits(m.decompress()), w)
     rng = np.random.default_rng(0)
@@ -82,10 +83,11 @@ def test_decompress_every_pattern(lib, orc):
     no_device_error(lib)
 
 
-def test_gpu_decodes_oracle_blob(lib, orc):
+@pytest.mark.parametrize("lmax", [7, 9, 12])
+def test_gpu_decodes_oracle_blob(lib, orc, lmax):
     spec = synth.MatrixSpec("w", 300, 2000, "normal_outliers", 1 / 64, 0)
     w = synth.matrix(spec, 1)
-    blob = orc.encode(w)
+    blob = orc.encode(w, lmax=lmax)
     m = lib.CompressedMatrix.from_blob(blob)
     assert np.array_equal(bits(m.decompress()), w)
     x = synth.activations(1, 2, spec.cols)
@@ -94,29 +96,47 @@ def test_gpu_decodes_oracle_blob(lib, orc):
     no_device_error(lib)
 
 
+@pytest.mark.parametrize("lmax", [0, 12])
 @pytest.mark.parametrize("shape,tile_cols", SHAPES)
 @pytest.mark.parametrize("batch", [1, 3, 8])
-def test_gemv_parity_shapes(lib, orc, shape, tile_cols, batch):
+def test_gemv_parity_shapes(lib, orc, shape, tile_cols, batch, lmax):
     if shape[1] % 2:
         pytest.skip("nwc_gemv requires an even number of columns")
     spec = synth.MatrixSpec("w", shape[0], shape[1], "normal", 0.02, 2)
     w = synth.matrix(spec, 6)
     x = synth.activations(6, batch, shape[1])
-    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols)
+    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
     y = m.gemv(to_bf16(x)).cpu().numpy()
     tolerance_check(y, orc.gemv(w, x), w, x)
     no_device_error(lib)
 
 
+@pytest.mark.parametrize("lmax", [0, 10])
 @pytest.mark.parametrize("batch", [1, 2, 4, 5, 7, 8, 9, 16, 33, 64])
-def test_gemv_every_batch(lib, orc, batch):
+def test_gemv_every_batch(lib, orc, batch, lmax):
     spec = synth.MatrixSpec("w", 520, 2048, "normal_rowscale", 0.02, 3)
     w = synth.matrix(spec, 4)
     x = synth.activations(4, batch, spec.cols)
-    m = lib.CompressedMatrix.compress(w)
+    m = lib.CompressedMatrix.compress(w, lmax=lmax)
     y = m.gemv(to_bf16(x)).cpu().numpy()
     tolerance_check(y, orc.gemv(w, x), w, x)
     no_device_error(lib)
+
+
+def test_auto_lmax_and_fast_path(lib, orc):
+    """Default plans use a 7-bit code limit (two codes per 14-bit peek) unless the
+    matrix holds more than 128 distinct exponents."""
+    w = synth.matrix(synth.MatrixSpec("w", 64, 1024, "normal", 0.02, 0), 3)
+    plan = lib.nwc_plan(w)
+    blob = lib.nwc_compress_host(plan, w)
+    lib.nwc_plan_destroy(plan)
+    assert int.from_bytes(blob[12:16].tobytes(), "little") == 7
+    assert np.array_equal(blob, orc.encode(w, lmax=7))
+    allp = np.arange(65536, dtype=np.uint16).reshape(128, 512)
+    plan = lib.nwc_plan(allp)
+    blob = lib.nwc_compress_host(plan, allp)
+    lib.nwc_plan_destroy(plan)
+    assert int.from_bytes(blob[12:16].tobytes(), "little") == 8
 
 
 def test_gemv_deterministic_and_workspace_reuse(lib, orc):
