@@ -37,9 +37,7 @@ __device__ unsigned int g_device_error;
 
 namespace {
 
-constexpr int kConsumers = 16;                   // decoding warps per CTA
-constexpr int kThreads = (kConsumers + 1) * 32;  // + one producer warp
-constexpr int kSlots = 32;                       // tiles in flight or resident per CTA
+constexpr int kSlots = 64;                       // tiles (and batches) in flight or resident per CTA
 constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
 constexpr int kRingSlack = 16;                   // lanes may read a few words past a chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -403,7 +401,8 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
   uint32_t xn[B];
 #pragma unroll
   for (int b = 0; b < B; ++b) xn[b] = load_x_pair(x + (int64_t)b * cols, cols, col0 + 2 * lane);
-#pragma unroll 1
+  constexpr int kGroupUnroll = B <= 4 ? 2 : 1;
+#pragma unroll kGroupUnroll
   for (int g = 0; g < CP; ++g) {
     const uint4 rv = lds128(chunk + g * 512 + lane * 16);
     uint32_t xg[B];
@@ -436,8 +435,9 @@ __device__ __forceinline__ void cta_range(const TileParams& p, int64_t* first, i
   *n = (int)(b - a);
 }
 
-// Sets up barriers; returns false for the producer warp (its work is done) and
-// for consumers when the decode table never arrived.
+// Sets up barriers; returns false for the producer warp (warp NC; its work is
+// done) and for consumers when the decode table never arrived.
+template <int NC>
 __device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const Smem& s,
                                       int64_t first, int n) {
   if (threadIdx.x == 0) {
@@ -450,31 +450,49 @@ __device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const 
   fence_barrier_init();
   __syncthreads();
   const int warp = threadIdx.x >> 5;
-  if (warp == kConsumers) {
+  if (warp == NC) {
     produce(p, smem, s, first, n, threadIdx.x & 31);
     return false;
   }
   return __all_sync(kFull, wait_bounded(s.table_bar, 0));
 }
 
-template <int CP, int B, bool FAST>
-__global__ void __launch_bounds__(kThreads, 1) gemv_kernel(TileParams p) {
+// Row block i and column block j of tile u = first + q, stepped by NC tiles.
+struct TilePos {
+  uint32_t i, j, tiles_r;
+  __device__ __forceinline__ void init(int64_t u, uint32_t tr) {
+    tiles_r = tr;
+    i = (uint32_t)(u % tr);
+    j = (uint32_t)(u / tr);
+  }
+  __device__ __forceinline__ void step(uint32_t by) {
+    i += by;
+    while (i >= tiles_r) {
+      i -= tiles_r;
+      ++j;
+    }
+  }
+};
+
+template <int NC, int CP, int B, bool FAST>
+__global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem s = carve(smem, p);
   int64_t first;
   int n;
   cta_range(p, &first, &n);
-  if (!setup(p, smem, s, first, n)) return;
+  if (!setup<NC>(p, smem, s, first, n)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
   const int64_t cols = p.cols;
-  for (int q = warp; q < n; q += kConsumers) {
+  TilePos pos;
+  pos.init(first + warp, (uint32_t)p.tiles_r);
+  for (int q = warp; q < n; q += NC, pos.step(NC)) {
     const int slot = q % kSlots;
     if (!wait_tile(p, s, q)) return;
     const uint32_t chunk = ring + s.desc[slot];
-    const int64_t u = first + q;
-    const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
+    const int64_t i = pos.i, j = pos.j;
     float acc[8][B];
 #pragma unroll
     for (int r = 0; r < 8; ++r)
@@ -515,11 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(TileParams p) {
   // tiles_c arrivals sums its partials in column-block order and writes y.
   __threadfence();
   __syncwarp();
-  for (int q0 = warp; q0 < n; q0 += 32 * kConsumers) {
-    const int q = q0 + lane * kConsumers;
+  for (int q0 = warp; q0 < n; q0 += 32 * NC) {
+    const int q = q0 + lane * NC;
     uint32_t last = 0;
     if (q < n) {
-      const int64_t i = (first + q) % p.tiles_r;
+      const uint32_t i = (uint32_t)(first + q) % (uint32_t)p.tiles_r;
       last = atomicAdd(&p.counters[i], 1u) == (uint32_t)(p.tiles_c - 1);
     }
     uint32_t mask = __ballot_sync(kFull, last);
@@ -527,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(TileParams p) {
     while (mask) {
       const int src = __ffs(mask) - 1;
       mask &= mask - 1;
-      const int64_t i = (first + q0 + src * kConsumers) % p.tiles_r;
+      const int64_t i = (uint32_t)(first + q0 + src * NC) % (uint32_t)p.tiles_r;
       for (int qq = lane; qq < 8 * B; qq += 32) {
         const int b = qq >> 3, rr = qq & 7;
         const int64_t orow = i * 8 + rr;
@@ -550,14 +568,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(TileParams p) {
   }
 }
 
-template <int CP, bool FAST>
-__global__ void __launch_bounds__(kThreads, 1) decompress_kernel(TileParams p) {
+template <int NC, int CP, bool FAST>
+__global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem s = carve(smem, p);
   int64_t first;
   int n;
   cta_range(p, &first, &n);
-  if (!setup(p, smem, s, first, n)) return;
+  if (!setup<NC>(p, smem, s, first, n)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
@@ -565,12 +583,13 @@ __global__ void __launch_bounds__(kThreads, 1) decompress_kernel(TileParams p) {
   const bool even_cols = (cols & 1) == 0;
   constexpr int kRaw = CP * 512;
   uint32_t invalid = 0;
-  for (int q = warp; q < n; q += kConsumers) {
+  TilePos pos;
+  pos.init(first + warp, (uint32_t)p.tiles_r);
+  for (int q = warp; q < n; q += NC, pos.step(NC)) {
     const int slot = q % kSlots;
     if (!wait_tile(p, s, q)) return;
     const uint32_t chunk = ring + s.desc[slot];
-    const int64_t u = first + q;
-    const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
+    const int64_t i = pos.i, j = pos.j;
     BitReader br;
     br.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane));
     const bool full_tile = (i + 1) * 8 <= p.rows && (j + 1) * (CP * 64) <= cols && even_cols;
@@ -617,12 +636,21 @@ cudaError_t ensure_smem(Kernel k, size_t bytes, int (&configured)[64]) {
   return e;
 }
 
+// Consumer warps per CTA: more warps hide the decoder's dependency chains, as
+// long as the batch's accumulators leave registers for them.
+// A CTA with W warps puts up to ceil(W / 4) on one SM sub-partition, whose
+// register file holds 16K registers: 25 warps leave 72 per thread, 17 leave 96,
+// 13 leave 128.
+template <int B>
+constexpr int consumers_for() { return B <= 2 ? 24 : (B <= 4 ? 16 : 12); }
+
 template <int CP, int B, bool FAST>
 cudaError_t launch_gemv_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+  constexpr int NC = consumers_for<B>();
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(gemv_kernel<CP, B, FAST>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(gemv_kernel<NC, CP, B, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  gemv_kernel<CP, B, FAST><<<s.ctas, kThreads, s.smem_bytes, stream>>>(p);
+  gemv_kernel<NC, CP, B, FAST><<<s.ctas, (NC + 1) * 32, s.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -643,10 +671,11 @@ cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream
 
 template <int CP, bool FAST>
 cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+  constexpr int NC = 24;
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(decompress_kernel<CP, FAST>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(decompress_kernel<NC, CP, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  decompress_kernel<CP, FAST><<<s.ctas, kThreads, s.smem_bytes, stream>>>(p);
+  decompress_kernel<NC, CP, FAST><<<s.ctas, (NC + 1) * 32, s.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
