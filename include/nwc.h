@@ -55,7 +55,8 @@ typedef enum {
   NWC_ERR_CORRUPT = 4,        /* a blob or device image does not parse          */
   NWC_ERR_NOMEM = 5,          /* host allocation failed, or buffer too small    */
   NWC_ERR_DEVICE_TIMEOUT = 6, /* the device error word reported a timeout       */
-  NWC_ERR_DEVICE_CORRUPT = 7  /* the device error word reported corrupt data    */
+  NWC_ERR_DEVICE_CORRUPT = 7, /* the device error word reported corrupt data    */
+  NWC_ERR_SCRATCH_LIMIT = 8   /* nwc_gemv_noalloc: scratch needed > the limit   */
 } nwc_status;
 
 /* Plan options.  Set struct_size = sizeof(nwc_opts); pass NULL for the defaults
@@ -164,6 +165,35 @@ nwc_status nwc_gemv_workspace_size(nwc_handle_t handle, int32_t batch,
 nwc_status nwc_gemv(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
                     int32_t batch, void* d_workspace, uint64_t workspace_bytes,
                     nwc_stream_t stream);
+
+/* GEMV for callers that cannot allocate device memory.  The pages describe
+ * no such call; it exists for integrations where the host application owns
+ * every device allocation and a library may not call cudaMalloc (inference
+ * servers with a fixed memory pool, plugins loaded into another framework),
+ * and for code that must not allocate while work is being recorded into a
+ * CUDA graph, since an allocation there breaks the recording.
+ *
+ * It computes exactly what nwc_gemv computes, with the same kernels, but takes
+ * its scratch (the split-K partial sums and arrival counters) from an array of
+ * NWC_NOALLOC_SCRATCH_BYTES bytes that the library defines as a static device
+ * variable.  Every GPU that loads the library holds that array until the
+ * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
+ * allocating library routine.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current, and caches it.  Make
+ *     that first call before any stream capture.
+ *   - Limit: when nwc_gemv_workspace_size(handle, batch) exceeds
+ *     NWC_NOALLOC_SCRATCH_BYTES the call returns NWC_ERR_SCRATCH_LIMIT and
+ *     launches nothing; use nwc_gemv with your own workspace instead.
+ *   - Sharing: every call uses the same array, which keeps the last call's
+ *     contents; each call first clears the counters it needs (an async memset
+ *     on `stream`).  Calls whose work overlaps on the GPU (different streams,
+ *     or different threads without ordering) race on the array and must not
+ *     be issued.
+ * Arguments and other errors as nwc_gemv. */
+#define NWC_NOALLOC_SCRATCH_BYTES (8u << 20)
+nwc_status nwc_gemv_noalloc(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
+                            int32_t batch, nwc_stream_t stream);
 
 /* ---- Inspection, errors, teardown ------------------------------------- */
 

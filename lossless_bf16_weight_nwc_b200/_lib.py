@@ -18,7 +18,9 @@ LIB_PATH = os.path.join(_PKG, "libnwc.so")
 NWC_OK = 0
 STATUS = {0: "NWC_OK", 1: "NWC_ERR_INVALID_ARG", 2: "NWC_ERR_UNSUPPORTED", 3: "NWC_ERR_CUDA",
           4: "NWC_ERR_CORRUPT", 5: "NWC_ERR_NOMEM", 6: "NWC_ERR_DEVICE_TIMEOUT",
-          7: "NWC_ERR_DEVICE_CORRUPT"}
+          7: "NWC_ERR_DEVICE_CORRUPT", 8: "NWC_ERR_SCRATCH_LIMIT"}
+NWC_ERR_SCRATCH_LIMIT = 8
+NWC_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class NwcError(RuntimeError):
@@ -53,6 +55,7 @@ def _load() -> ctypes.CDLL:
         "nwc_decompress": ([vp, vp, vp], c.c_int),
         "nwc_gemv_workspace_size": ([vp, i32, c.POINTER(u64)], c.c_int),
         "nwc_gemv": ([vp, vp, vp, i32, vp, u64, vp], c.c_int),
+        "nwc_gemv_noalloc": ([vp, vp, vp, i32, vp], c.c_int),
         "nwc_handle_info": ([vp, c.POINTER(i64), c.POINTER(i64), c.POINTER(u64),
                              c.POINTER(u64)], c.c_int),
         "nwc_get_device_error": ([vp, c.POINTER(c.c_uint32)], c.c_int),
@@ -70,6 +73,7 @@ LIB = _load()
 EXPORTED = ("nwc_version", "nwc_status_string", "nwc_plan", "nwc_plan_size", "nwc_compress",
             "nwc_compress_host", "nwc_blob_device_bytes", "nwc_upload_blob",
             "nwc_handle_from_device", "nwc_decompress", "nwc_gemv_workspace_size", "nwc_gemv",
+            "nwc_gemv_noalloc",
             "nwc_handle_info", "nwc_get_device_error", "nwc_plan_destroy", "nwc_handle_destroy")
 
 
@@ -167,6 +171,13 @@ def nwc_gemv(handle, d_x, d_y, batch: int, d_workspace=None, workspace_bytes: in
     ws = 0 if d_workspace is None else _ptr(d_workspace)
     _check(LIB.nwc_gemv(handle, _ptr(d_x), _ptr(d_y), batch, ws, workspace_bytes,
                         _stream(stream)), "nwc_gemv")
+
+
+def nwc_gemv_noalloc(handle, d_x, d_y, batch: int, stream=None) -> None:
+    """nwc_gemv with library-owned scratch, for callers that may not allocate
+    device memory (see include/nwc.h)."""
+    _check(LIB.nwc_gemv_noalloc(handle, _ptr(d_x), _ptr(d_y), batch, _stream(stream)),
+           "nwc_gemv_noalloc")
 
 
 def nwc_handle_info(handle) -> dict:

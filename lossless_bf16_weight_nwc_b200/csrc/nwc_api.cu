@@ -114,6 +114,7 @@ const char* nwc_status_string(nwc_status s) {
     case NWC_ERR_NOMEM: return "out of memory or buffer too small";
     case NWC_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case NWC_ERR_DEVICE_CORRUPT: return "device found corrupt data";
+    case NWC_ERR_SCRATCH_LIMIT: return "scratch needed exceeds the no-allocation limit";
   }
   return "unknown status";
 }
@@ -312,6 +313,46 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
     if (e != cudaSuccess) return NWC_ERR_CUDA;
   }
   return NWC_OK;
+}
+
+// Scratch of nwc_gemv_noalloc: a fixed array that lives as long as the module,
+// one copy per device.  Host code must not hand `g_noalloc_scratch` itself to a
+// kernel (on the host that name is a stand-in, not a device address); the
+// device address comes from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NWC_NOALLOC_SCRATCH_BYTES];
+static void* g_noalloc_addr[kMaxDevices] = {};
+
+static nwc_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return NWC_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr)
+      return NWC_ERR_CUDA;
+    g_noalloc_addr[dev] = addr;
+  }
+  *out = g_noalloc_addr[dev];
+  return NWC_OK;
+}
+
+nwc_status nwc_gemv_noalloc(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t batch,
+                            nwc_stream_t stream) {
+  if (!h || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
+  const uint64_t need = workspace_bytes_for(*h, batch);
+  if (need > NWC_NOALLOC_SCRATCH_BYTES) return NWC_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  if (need) {
+    nwc_status st = noalloc_scratch(&ws);
+    if (st != NWC_OK) return st;
+    // The array keeps the previous call's bytes: the arrival counters must
+    // start at zero, the partial sums are overwritten before they are read.
+    if (cudaMemsetAsync(ws, 0, 4ull * (uint64_t)h->tiles_r,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+      return NWC_ERR_CUDA;
+  }
+  return nwc_gemv(h, d_x, d_y, batch, ws, need, stream);
 }
 
 nwc_status nwc_handle_info(nwc_handle_t h, int64_t* rows, int64_t* cols, uint64_t* blob_bytes,

@@ -28,7 +28,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(8):
+    for code in range(9):
         assert lib.LIB.nwc_status_string(code)
 
 
