@@ -163,64 +163,90 @@ def barrier(world: int):
         dist.barrier()
 
 
-def max_over_ranks(v: float, world: int) -> float:
+def max_over_ranks(v: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's time: every rank contributes, all get the maximum."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    t = torch.tensor([v], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def cpu_baseline(workload: str, batch: int, budget_s: float = 12.0) -> dict:
-    """The oracle as it stands (decode + FP64 GEMV), single-threaded, on a
-    bounded sample: whole calls on the workload's first matrix until the budget
-    is spent.  Reported in the bench metric's unit (effective GB/s)."""
+def replica_value(weight_bytes: float, world: int, ms_per_step: float) -> float:
+    """Whole-job effective GB/s: every rank runs the same per-GPU work (weak
+    scaling, independent replicas), so the job moves world x weight_bytes per
+    step in the slowest rank's time."""
+    return world * weight_bytes / (ms_per_step * 1e-3) / 1e9
+
+
+def _oracle_sample(workload: str, batch: int, rows: int):
+    """A bounded sample of the workload for the oracle: the first `rows` rows of
+    its first matrix, encoded by the oracle, and the batch of activations."""
     import oracle
     from lossless_bf16_weight_nwc_b200 import synth
     wl = synth.workload(workload)
     spec = wl.matrices[0]
-    rows = spec.rows
-    # Bounded sample: at most 4096 rows of the matrix (all of it for the
-    # benchmark workloads of 4096 rows or fewer).
-    rows = min(rows, 4096)
+    rows = min(rows, spec.rows)
     w = synth.matrix(spec, wl.seed, 0, rows)
     x = synth.activations(wl.seed, batch, spec.cols)
-    blob = oracle.encode(w)
+    return oracle, oracle.encode(w), x, rows, spec.cols
+
+
+def cpu_baseline(workload: str, batch: int, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands (decode + FP64 GEMV), single-threaded, on a
+    bounded sample: whole calls on up to 4096 rows of the workload's first
+    matrix until the budget is spent, in the bench metric's unit."""
+    orc, blob, x, rows, cols = _oracle_sample(workload, batch, 4096)
     calls, t0 = 0, time.perf_counter()
     while True:
-        wd = oracle.decode(blob)
-        oracle.gemv(wd, x)
+        orc.gemv(orc.decode(blob), x)
         calls += 1
         el = time.perf_counter() - t0
         if el >= budget_s or calls >= 50:
             break
     per_call = el / calls
-    gbs = 2.0 * rows * spec.cols / per_call / 1e9
-    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "us_per_call": per_call * 1e6,
+    return {"value": 2.0 * rows * cols / per_call / 1e9, "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "us_per_call": per_call * 1e6,
             "sample": f"{calls} whole oracle calls (decode of the blob + FP64 GEMV, batch {batch}) "
-                      f"on {rows}x{spec.cols} rows of '{workload}' matrix 0, single thread"}
+                      f"on {rows}x{cols} rows of '{workload}' matrix 0, single thread"}
 
 
 def run_reference(args) -> None:
+    """The reference arm: the oracle on the host cores, rank 0 only.  Each step
+    is one oracle call (decode + FP64 GEMV) on a 256-row sample of the
+    workload's first matrix; at most as many of the --steps as fit in about a
+    minute are timed, after --warmup untimed calls."""
     rank = int(os.environ.get("RANK", 0))
     if rank != 0:
         return
-    base = cpu_baseline(args.workload, args.batch)
-    step_s = base["us_per_call"] / 1e6
-    from lossless_bf16_weight_nwc_b200 import synth
-    spec = synth.workload(args.workload).matrices[0]
+    orc, blob, x, rows, cols = _oracle_sample(args.workload, args.batch, 256)
+    for _ in range(max(args.warmup, 1)):
+        orc.gemv(orc.decode(blob), x)
+    t0 = time.perf_counter()
+    orc.gemv(orc.decode(blob), x)
+    est = time.perf_counter() - t0
+    steps = max(3, min(args.steps, int(60.0 / max(est, 1e-6))))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        orc.gemv(orc.decode(blob), x)
+    el = time.perf_counter() - t0
+    step_s = el / steps
+    value = 2.0 * rows * cols / step_s / 1e9
+    sample = (f"{steps} oracle calls (decode + FP64 GEMV, batch {args.batch}) on {rows}x{cols} "
+              f"rows of '{args.workload}' matrix 0, single thread, after {max(args.warmup, 1)} "
+              f"warm-up calls")
     line = {
-        "impl": "reference", "metric": METRIC, "value": base["value"], "unit": "GB/s",
-        "n_gpus": args.gpus, "steps": None, "warmup": None, "ms_per_step": step_s * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": max(args.warmup, 1),
+        "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "batch": args.batch,
-                   "matrix": f"{spec.rows}x{spec.cols}"},
-        "cpu_baseline": {k: base[k] for k in ("kind", "cores", "sample", "value", "unit")},
-        "e2e": {"value": base["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "matrix": f"{rows}x{cols} (sample)"},
+        "cpu_baseline": {"kind": "oracle", "cores": 1, "sample": sample, "value": value,
+                         "unit": "GB/s"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
@@ -330,7 +356,7 @@ def main():
     alg_bytes = image_bytes + x_bytes + y_bytes
     peaks, peak_src = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
-    eff_gbs = world * weight_bytes / (ms_per_step * 1e-3) / 1e9
+    eff_gbs = replica_value(weight_bytes, world, ms_per_step)
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
     traffic = profile_traffic(args.workload, batch)
 
