@@ -92,10 +92,12 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols,
                     const nwc_opts* opts, nwc_plan_t* out_plan);
 
 /* Exact sizes for a plan.  *device_bytes is what nwc_compress needs in device
- * memory: the serialisable blob plus a derived decode table (64 KiB for
- * lmax <= 7, else 16 KiB) at a 256-byte aligned offset.  *host_blob_bytes is
- * the size of the serialisable blob (nwc_compress_host).  Either pointer may
- * be NULL. */
+ * memory, the "device image": the serialisable blob, then at 256-byte aligned
+ * offsets a derived decode table (64 KiB for lmax <= 7, else 16 KiB) and the
+ * launch schedule (about 12 bytes per tile plus 5 KiB: which bytes each bulk
+ * copy of the kernels moves and where they land in shared memory, worked out
+ * on the host for the device that runs them).  *host_blob_bytes is the size of
+ * the serialisable blob (nwc_compress_host).  Either pointer may be NULL. */
 nwc_status nwc_plan_size(nwc_plan_t plan, uint64_t* device_bytes,
                          uint64_t* host_blob_bytes);
 
@@ -115,12 +117,14 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf,
 nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob,
                              uint64_t blob_bytes);
 
-/* Bytes of device memory needed to upload an existing blob (blob + table). */
+/* Bytes of device memory needed to upload an existing blob (the device image:
+ * blob + decode table + launch schedule). */
 nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes,
                                  uint64_t* device_bytes);
 
-/* Validate a host blob, upload it into d_buf, and build its decode table.  The
- * call is synchronous: it returns after the copies finish.
+/* Validate a host blob, upload it into d_buf, and build its decode table and
+ * launch schedule for the current device.  The call is synchronous: it returns
+ * after the copies finish.
  * Errors: CORRUPT (header, code lengths or index do not parse), INVALID_ARG,
  * CUDA. */
 nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
@@ -129,12 +133,19 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
 
 /* Build a handle for a device buffer that already holds a device image (from
  * nwc_compress or nwc_upload_blob, possibly copied elsewhere).  The call is
- * synchronous: it reads the header, code lengths and index back to the host.
+ * synchronous: it reads the header, code lengths and index back to the host,
+ * then rewrites the image's launch-schedule area for the current device (the
+ * blob and the decode table are not written).
  * Errors: CORRUPT, INVALID_ARG, CUDA. */
-nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes,
+nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
                                   nwc_handle_t* out_handle);
 
 /* ---- Device kernels ---------------------------------------------------- */
+
+/* nwc_decompress, nwc_gemv and nwc_gemv_noalloc launch one persistent CTA per
+ * SM (at most 256).  Should the current device's launch shape differ from the
+ * one the image's schedule was written for, the call first rewrites the
+ * schedule area on `stream` (a host-to-device copy, in stream order). */
 
 /* Bit-exact decompression ("NWC", "How it works > Dequantization and embedding
  * lookup": the same decoder writes BF16).  d_w_out: device, rows x cols BF16,
@@ -197,8 +208,34 @@ nwc_status nwc_gemv_noalloc(nwc_handle_t handle, const uint16_t* d_x, float* d_y
 
 /* ---- Inspection, errors, teardown ------------------------------------- */
 
+/* Launch shape and schedule the kernels would use for a blob on a device with
+ * sm_count SMs and smem_limit bytes of opt-in shared memory per block (B200:
+ * 148 and 232448).  Host only; touches no GPU.
+ *   info: set struct_size = sizeof(nwc_schedule_info).
+ *   cta_batch (optional, ctas + 1 entries): first batch of each CTA, and the
+ *     total number of batches at the end.  CTA c owns tiles
+ *     [tiles * c / ctas, tiles * (c + 1) / ctas) in blob order.
+ *   batch (optional, 4 * batches entries): per batch {tile-area offset in
+ *     16-byte units, bytes, offset in the CTA's ring, number of the CTA's
+ *     earlier batches that must be released before this one is issued}.
+ *   tile_ring (optional, tiles entries): ring offset of each tile's chunk.
+ * Query info first (arrays NULL) to size the arrays.
+ * Errors: INVALID_ARG, CORRUPT, UNSUPPORTED (shared memory too small). */
+typedef struct {
+  uint32_t struct_size;
+  int32_t ctas;        /* persistent CTAs                                  */
+  int32_t batch_tiles; /* consecutive tiles per bulk copy                  */
+  int32_t ring_bytes;  /* staging ring in shared memory, per CTA           */
+  int64_t tiles;       /* tiles of the matrix                              */
+  int64_t batches;     /* bulk copies over all CTAs                        */
+  uint64_t smem_bytes; /* dynamic shared memory per CTA                    */
+} nwc_schedule_info;
+nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
+                                 uint64_t smem_limit, nwc_schedule_info* info,
+                                 uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring);
+
 /* Any pointer may be NULL.  *blob_bytes is the serialisable part; *device_bytes
- * is the whole device image (blob + decode table). */
+ * is the whole device image (blob + decode table + launch schedule). */
 nwc_status nwc_handle_info(nwc_handle_t handle, int64_t* rows, int64_t* cols,
                            uint64_t* blob_bytes, uint64_t* device_bytes);
 

@@ -13,7 +13,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libnwc.so")
-SOURCES = ["kernels.cu", "nwc_api.cu", "encoder.cpp"]
+SOURCES = ["kernels.cu", "nwc_api.cu", "encoder.cpp", "schedule.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -279,7 +279,8 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   p->tiles_off = round_up(kIndexOffset + 4ull * (uint64_t)(p->tiles + 1), 256);
   p->blob_bytes = p->tiles_off + 16ull * acc;
   p->table_off = round_up(p->blob_bytes, 256);
-  p->device_bytes = p->table_off + table_bytes(p->lmax);
+  p->sched_off = round_up(p->table_off + table_bytes(p->lmax), 256);
+  p->device_bytes = p->sched_off + sched_bytes((uint64_t)p->tiles);
   return 0;
 }
 
@@ -412,10 +413,13 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   hd->tiles_c = (int64_t)h.tiles_c;
   hd->tiles = (int64_t)tiles;
   hd->index_off = kIndexOffset;
+  hd->index.resize((size_t)tiles + 1);
+  std::memcpy(hd->index.data(), blob + kIndexOffset, 4 * ((size_t)tiles + 1));
   hd->tiles_off = h.tiles_off;
   hd->blob_bytes = bytes;
   hd->table_off = round_up(bytes, 256);
-  hd->device_bytes = hd->table_off + table_bytes(h.lmax);
+  hd->sched_off = round_up(hd->table_off + table_bytes(h.lmax), 256);
+  hd->device_bytes = hd->sched_off + sched_bytes(tiles);
   hd->max_chunk = largest;
   if (lens_out) *lens_out = lens;
   return true;

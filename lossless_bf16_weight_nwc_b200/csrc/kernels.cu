@@ -37,7 +37,6 @@ __device__ unsigned int g_device_error;
 
 namespace {
 
-constexpr int kSlots = 64;                       // tiles (and batches) in flight or resident per CTA
 constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
 constexpr int kRingSlack = 16;                   // lanes may read a few words past a chunk
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -82,9 +81,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 // Polls `bar` for `parity` at most kWaitLimit times; on failure records a
 // timeout in the device error word.
@@ -246,18 +242,19 @@ __device__ __forceinline__ uint32_t lane_stream_start(uint32_t chunk, int raw, i
 
 // ---- shared-memory layout and the producer ---------------------------------
 //
-// Tiles move in fixed batches of p.batch_tiles consecutive tiles (consecutive in
-// HBM too), one bulk copy per batch, so that each copy is large enough for the
-// copy engine to run at full bandwidth.  Batch k has a "full" barrier counting
-// its bytes; every tile has its own "empty" barrier, arrived at by the consumer
-// that decoded it.
+// Tiles move in batches of p.batch_tiles consecutive tiles (consecutive in HBM
+// too), one bulk copy per batch, so that each copy is large enough for the copy
+// engine to run at full bandwidth.  Where each batch lands in the ring, and how
+// many earlier batches must have been released before it may be issued, is
+// fixed by the launch schedule that the host computed for this launch shape;
+// the producer only follows it.  Batch k of a CTA uses barrier slot k % kSlots:
+// a "full" barrier counting its bytes and an "empty" barrier that each of its
+// tiles' consumers arrives at once.
 
 struct Smem {
   uint64_t* table_bar;
-  uint64_t* full;    // per batch slot
-  uint64_t* empty;   // per tile slot
-  uint32_t* desc;    // per tile slot: ring offset of the tile's chunk
-  uint32_t* vstart;  // per tile slot: virtual ring position (producer)
+  uint64_t* full;    // per batch slot: bytes landed
+  uint64_t* empty;   // per batch slot: tiles released
   uint8_t* ring;
 };
 
@@ -266,93 +263,68 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
   s.table_bar = reinterpret_cast<uint64_t*>(smem + p.table_bytes);
   s.full = s.table_bar + 1;
   s.empty = s.full + kSlots;
-  s.desc = reinterpret_cast<uint32_t*>(s.empty + kSlots);
-  s.vstart = s.desc + kSlots;
   s.ring = smem + p.ring_offset;
   return s;
 }
 
-// Streams tiles [first, first + n) into the ring, batch by batch; run by the
-// whole producer warp (uniform control flow), lane 0 issuing the copies.  The
-// chunk offsets come 32 at a time from one coalesced load.  A batch is
-// contiguous in the ring; ring space is reused once consumers release tiles.
-__device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, int64_t first, int n,
-                        int lane) {
+// Issues the CTA's nb batches, descriptors desc[0 .. nb): {tile-area offset in
+// 16-byte units, bytes, ring offset, batches that must be released first}.
+// The whole warp runs the loop (the descriptors travel 32 at a time in its
+// registers, the next 32 loaded while the current ones are used); lane 0 waits
+// for releases and issues the copies.  The loop body is a handful of
+// instructions, so the copies go out as fast as the ring allows.
+__device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const uint4* desc,
+                        int nb, int lane) {
   if (lane == 0) {
     mbar_expect_tx(s.table_bar, p.table_bytes);
     bulk_load(smem, p.table, p.table_bytes, s.table_bar);
   }
-  const int T = p.batch_tiles;
-  const uint32_t R = (uint32_t)p.ring_bytes;
-  uint32_t vhead = 0, vtail = 0;  // virtual ring positions
-  uint32_t phys = 0;              // vhead % R, kept incrementally
-  int q_tail = 0;                 // oldest tile whose release has not been seen
-  int wbase = 0;                  // index window: offsets of tiles wbase .. wbase + 63
-  uint32_t wa = lane <= n ? __ldg(p.index + first + lane) : 0u;
-  uint32_t wb = 32 + lane <= n ? __ldg(p.index + first + 32 + lane) : 0u;
-  auto offset_of = [&](int k) -> uint32_t {  // index[first + k], k in [wbase, wbase + 64)
-    const int d = k - wbase;
-    const uint32_t va = __shfl_sync(kFull, wa, d & 31);
-    const uint32_t vb = __shfl_sync(kFull, wb, d & 31);
-    return d < 32 ? va : vb;
-  };
-  bool ok = true;
-  int q0 = 0;
-  for (; q0 < n && ok; q0 += T) {
-    const int q1 = q0 + T < n ? q0 + T : n;
-    while (q1 - wbase >= 64) {  // slide the offset window (uniform)
-      wbase += 32;
-      wa = wb;
-      wb = wbase + 32 + lane <= n ? __ldg(p.index + first + wbase + 32 + lane) : 0u;
+  const uint4 none = make_uint4(0u, 0u, 0u, 0u);
+  uint4 cur = lane < nb ? __ldg(desc + lane) : none;
+  uint4 nxt = 32 + lane < nb ? __ldg(desc + 32 + lane) : none;
+  uint32_t released = 0;  // batches whose release lane 0 has observed
+  int k = 0;
+  for (; k < nb; ++k) {
+    const int l = k & 31;
+    if (l == 0 && k) {
+      cur = nxt;
+      nxt = k + 32 + lane < nb ? __ldg(desc + k + 32 + lane) : none;
     }
-    const uint32_t c0 = offset_of(q0), c1 = offset_of(q1);
-    const uint32_t bytes = (c1 - c0) * 16u;
-    uint32_t at = vhead, at_phys = phys;
-    if (at_phys + bytes > R) {  // a batch never wraps
-      at += R - at_phys;
-      at_phys = 0;
-    }
-    // Room: at most kSlots tiles resident, and the batch must not reach into
-    // bytes of unreleased tiles.
-    while (q_tail < q0 && (q1 - q_tail > kSlots || at + bytes - vtail > R)) {
-      if (!__all_sync(kFull, wait_bounded(&s.empty[q_tail % kSlots],
-                                          (uint32_t)((q_tail / kSlots) & 1)))) {
-        ok = false;
-        break;
-      }
-      ++q_tail;
-      vtail = q_tail < q0 ? s.vstart[q_tail % kSlots] : at;
-    }
-    if (!ok) break;
-    if (q_tail == q0) vtail = at;
-    // Per-tile ring offsets of the batch, then one copy for all of it.
-    const uint32_t off = (offset_of(lane < q1 - q0 ? q0 + lane : q0) - c0) * 16u;
-    if (lane < q1 - q0) {
-      s.vstart[(q0 + lane) % kSlots] = at + off;
-      s.desc[(q0 + lane) % kSlots] = at_phys + off;
-    }
-    __syncwarp();
+    const uint32_t src = __shfl_sync(kFull, cur.x, l);
+    const uint32_t bytes = __shfl_sync(kFull, cur.y, l);
+    const uint32_t at = __shfl_sync(kFull, cur.z, l);
+    const uint32_t need = __shfl_sync(kFull, cur.w, l);
+    uint32_t ok = 1;
     if (lane == 0) {
-      uint64_t* bar = &s.full[(q0 / T) % kSlots];
-      mbar_expect_tx(bar, bytes);  // arrive (release) + byte count
-      bulk_load(s.ring + at_phys, p.tiles + 16ull * c0, bytes, bar);
+      for (; released < need; ++released) {
+        if (!wait_bounded(&s.empty[released % kSlots], (released / kSlots) & 1u)) {
+          ok = 0;
+          break;
+        }
+      }
+      if (ok) {
+        uint64_t* bar = &s.full[k % kSlots];
+        mbar_expect_tx(bar, bytes);  // arrive (release) + byte count
+        bulk_load(s.ring + at, p.tiles + 16ull * src, bytes, bar);
+      }
     }
-    __syncwarp();
-    vhead = at + bytes;
-    phys = at_phys + bytes;
+    if (!__shfl_sync(kFull, ok, 0)) break;
   }
-  // Leave no copy in flight: wait for the last use of every batch slot issued.
-  const int batches = (q0 + T - 1) / T;  // batches [0, batches) were issued
+  // Leave no copy in flight: batches [0, k) were issued, and those more than
+  // kSlots back have been released, hence landed.
   if (lane == 0) {
-    for (int k = batches - 1; k >= 0 && k >= batches - kSlots; --k)
-      wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1));
+    for (int j = k - 1; j >= 0 && j >= k - kSlots; --j)
+      wait_bounded(&s.full[j % kSlots], (uint32_t)((j / kSlots) & 1));
     wait_bounded(s.table_bar, 0);
   }
 }
 
-// Consumer side: wait for tile q's batch; returns the chunk's ring offset.
-__device__ __forceinline__ bool wait_tile(const TileParams& p, const Smem& s, int q) {
-  const int k = q / p.batch_tiles;
+// Consumer side: wait until tile q's batch k has landed.  The schedule keeps
+// fewer than kSlots - ceil(kMaxConsumers / batch_tiles) batches outstanding, so
+// by the time a consumer polls slot k % kSlots (after finishing its previous
+// tile, at most kMaxConsumers tiles back) the slot's previous batch k - kSlots
+// was released long ago: the parity it polls is batch k's.
+__device__ __forceinline__ bool wait_batch(const Smem& s, int k) {
   return __all_sync(kFull, wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1)));
 }
 
@@ -438,20 +410,20 @@ __device__ __forceinline__ void cta_range(const TileParams& p, int64_t* first, i
 // Sets up barriers; returns false for the producer warp (warp NC; its work is
 // done) and for consumers when the decode table never arrived.
 template <int NC>
-__device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const Smem& s,
-                                      int64_t first, int n) {
+__device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const Smem& s) {
   if (threadIdx.x == 0) {
     mbar_init(s.table_bar, 1);
     for (int k = 0; k < kSlots; ++k) {
       mbar_init(&s.full[k], 1);
-      mbar_init(&s.empty[k], 1);
+      mbar_init(&s.empty[k], (uint32_t)p.batch_tiles);
     }
   }
   fence_barrier_init();
   __syncthreads();
   const int warp = threadIdx.x >> 5;
   if (warp == NC) {
-    produce(p, smem, s, first, n, threadIdx.x & 31);
+    const uint32_t b0 = __ldg(p.sched_cta + blockIdx.x), b1 = __ldg(p.sched_cta + blockIdx.x + 1);
+    produce(p, smem, s, p.sched_batch + b0, (int)(b1 - b0), threadIdx.x & 31);
     return false;
   }
   return __all_sync(kFull, wait_bounded(s.table_bar, 0));
@@ -481,17 +453,20 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   int64_t first;
   int n;
   cta_range(p, &first, &n);
-  if (!setup<NC>(p, smem, s, first, n)) return;
+  if (!setup<NC>(p, smem, s)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
   const int64_t cols = p.cols;
+  const uint32_t* tile_ring = p.tile_ring + first;
+  uint32_t at_next = warp < n ? __ldg(tile_ring + warp) : 0u;
   TilePos pos;
   pos.init(first + warp, (uint32_t)p.tiles_r);
   for (int q = warp; q < n; q += NC, pos.step(NC)) {
-    const int slot = q % kSlots;
-    if (!wait_tile(p, s, q)) return;
-    const uint32_t chunk = ring + s.desc[slot];
+    const int k = q / p.batch_tiles;
+    const uint32_t chunk = ring + at_next;
+    if (q + NC < n) at_next = __ldg(tile_ring + q + NC);  // next tile's ring offset, early
+    if (!wait_batch(s, k)) return;
     const int64_t i = pos.i, j = pos.j;
     float acc[8][B];
 #pragma unroll
@@ -500,10 +475,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
       for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
     decode_gemv_tile<CP, B, FAST>(chunk, table, lane, acc, p.x, cols, j * (CP * 64));
     __syncwarp();
-    if (lane == 0) {
-      fence_proxy_async();
-      mbar_arrive(&s.empty[slot]);
-    }
+    if (lane == 0) mbar_arrive(&s.empty[k % kSlots]);  // release the tile's share of the batch
 
     // Row sums of this tile: lane L holds row L >> 2 for every batch row.
     float tot[B];
@@ -575,7 +547,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
   int64_t first;
   int n;
   cta_range(p, &first, &n);
-  if (!setup<NC>(p, smem, s, first, n)) return;
+  if (!setup<NC>(p, smem, s)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
@@ -583,12 +555,15 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
   const bool even_cols = (cols & 1) == 0;
   constexpr int kRaw = CP * 512;
   uint32_t invalid = 0;
+  const uint32_t* tile_ring = p.tile_ring + first;
+  uint32_t at_next = warp < n ? __ldg(tile_ring + warp) : 0u;
   TilePos pos;
   pos.init(first + warp, (uint32_t)p.tiles_r);
   for (int q = warp; q < n; q += NC, pos.step(NC)) {
-    const int slot = q % kSlots;
-    if (!wait_tile(p, s, q)) return;
-    const uint32_t chunk = ring + s.desc[slot];
+    const int k = q / p.batch_tiles;
+    const uint32_t chunk = ring + at_next;
+    if (q + NC < n) at_next = __ldg(tile_ring + q + NC);
+    if (!wait_batch(s, k)) return;
     const int64_t i = pos.i, j = pos.j;
     BitReader br;
     br.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane));
@@ -613,10 +588,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
       }
     }
     __syncwarp();
-    if (lane == 0) {
-      fence_proxy_async();
-      mbar_arrive(&s.empty[slot]);
-    }
+    if (lane == 0) mbar_arrive(&s.empty[k % kSlots]);  // release the tile's share of the batch
   }
   if (__any_sync(kFull, invalid & kEntryInvalid) && lane == 0)
     atomicOr(&g_device_error, kErrCorrupt);
@@ -647,6 +619,7 @@ constexpr int consumers_for() { return B <= 2 ? 24 : (B <= 4 ? 16 : 12); }
 template <int CP, int B, bool FAST>
 cudaError_t launch_gemv_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   constexpr int NC = consumers_for<B>();
+  static_assert(NC <= kMaxConsumers, "the launch schedule assumes at most kMaxConsumers");
   static int configured[64] = {};
   cudaError_t e = ensure_smem(gemv_kernel<NC, CP, B, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
@@ -672,6 +645,7 @@ cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream
 template <int CP, bool FAST>
 cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   constexpr int NC = 24;
+  static_assert(NC <= kMaxConsumers, "the launch schedule assumes at most kMaxConsumers");
   static int configured[64] = {};
   cudaError_t e = ensure_smem(decompress_kernel<NC, CP, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
@@ -684,25 +658,25 @@ cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaS
 LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_chunk,
                          uint32_t table_bytes, int sm_count, size_t smem_limit) {
   LaunchShape s;
-  s.ctas = (int)(n_tiles < sm_count ? n_tiles : sm_count);
-  if (s.ctas < 1) s.ctas = 1;
+  int64_t ctas = n_tiles < sm_count ? n_tiles : sm_count;
+  if (ctas > (int64_t)kMaxCtas) ctas = kMaxCtas;
+  s.ctas = ctas < 1 ? 1 : (int)ctas;
   s.table_bytes = table_bytes;
-  // table | table barrier | full[] | empty[] | desc[] | vstart[] | ring
-  const size_t head = (size_t)table_bytes + 8 + 2 * kSlots * 8 + 2 * kSlots * 4;
+  // table | table barrier | full[kSlots] | empty[kSlots] | ring
+  const size_t head = (size_t)table_bytes + 8 + 2 * kSlots * 8;
   s.ring_offset = (head + 127) / 128 * 128;
   const int64_t per_cta = (n_tiles + s.ctas - 1) / s.ctas;
-  // Tiles per bulk copy: enough for >= 16 KB of typical chunks, at most 8 and
-  // never more than a quarter of the slots.
+  // Tiles per bulk copy: enough for >= 16 KB of typical chunks, between 2 and 8
+  // (at least 2 keeps the schedule's batch count within its area).
   int t = (int)((16384 + typical_chunk - 1) / (typical_chunk ? typical_chunk : 1));
-  if (t < 1) t = 1;
+  if (t < 2) t = 2;
   if (t > 8) t = 8;
   s.batch_tiles = t;
-  // As much ring as the device allows, but no more than the CTA's tiles need.
+  // As much ring as the device allows, but no more than the CTA's tiles need;
+  // a batch of worst-case chunks must fit.
   size_t ring = smem_limit > s.ring_offset + kRingSlack + max_chunk
                     ? smem_limit - s.ring_offset - kRingSlack
                     : 0;
-  // A batch of worst-case chunks must fit, and the ring need not exceed the
-  // CTA's whole range.
   const size_t batch_max = (size_t)s.batch_tiles * (size_t)max_chunk;
   const size_t need = (size_t)per_cta * (size_t)max_chunk;
   if (ring > need) ring = need;

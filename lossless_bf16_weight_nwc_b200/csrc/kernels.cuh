@@ -5,13 +5,20 @@
 
 namespace nwc {
 
+// Barrier slots per CTA: batches in flight or resident at once are fewer.
+constexpr int kSlots = 64;
+// Most consumer warps any kernel runs; the launch schedule relies on it.
+constexpr int kMaxConsumers = 24;
+
 // Device error word bits (read and cleared by nwc_get_device_error).
 constexpr uint32_t kErrTimeout = 1u;   // a bounded mbarrier wait gave up
 constexpr uint32_t kErrCorrupt = 2u;   // a stream held no valid code
 
 struct TileParams {
   const uint8_t* tiles;     // device: tile area of the blob
-  const uint32_t* index;    // device: chunk offsets (16-byte units), tiles + 1
+  const uint32_t* sched_cta;   // device: first batch of each CTA, ctas + 1
+  const uint4* sched_batch;    // device: per batch {offset16, bytes, ring offset, need}
+  const uint32_t* tile_ring;   // device: per tile, ring offset of its chunk
   const uint32_t* table;    // device: decode table (table_bytes)
   uint32_t table_bytes;     // 64 KiB (14-bit peek) or 16 KiB (12-bit peek)
   uint32_t ring_offset;     // shared-memory offset of the staging ring
@@ -44,6 +51,16 @@ struct LaunchShape {
 // shared-memory limit.
 LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_chunk,
                          uint32_t table_bytes, int sm_count, size_t smem_limit);
+
+// Launch schedule for one shape (host): for every CTA (tiles [n c / C,
+// n (c + 1) / C)) its batches of batch_tiles consecutive tiles, each with its
+// tile-area offset (16-byte units), its bytes, its place in the ring (a batch
+// never wraps; space is reused first in, first out) and how many of the CTA's
+// earlier batches must have been released before it is issued (for room, and
+// to keep fewer than kSlots - ceil(kMaxConsumers / batch_tiles) outstanding).
+// `index` holds the tiles + 1 chunk offsets in 16-byte units; `out` receives
+// sched_bytes(n_tiles) bytes laid out as nwc_format.h describes.
+void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s, uint8_t* out);
 
 // fast: lmax <= 7 (14-bit peek, two codes per entry always).
 cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const LaunchShape& s,

@@ -45,16 +45,46 @@ nwc_status current_device(int* dev, int* sms, size_t* smem) {
   return NWC_OK;
 }
 
-// Launch geometry for a handle on the current device.
-nwc_status shape_for(const nwc_handle_s& h, nwc::LaunchShape* s) {
-  int dev, sms;
-  size_t smem;
-  nwc_status st = current_device(&dev, &sms, &smem);
-  if (st != NWC_OK) return st;
+// Launch geometry for a handle on a device with `sms` SMs and `smem` bytes of
+// opt-in shared memory per block.
+nwc_status shape_on(const nwc_handle_s& h, int sms, size_t smem, nwc::LaunchShape* s) {
   const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
   *s = nwc::launch_shape(h.tiles, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms, smem);
   if (s->smem_bytes > smem) return NWC_ERR_UNSUPPORTED;
   return NWC_OK;
+}
+
+bool same_shape(const nwc_handle_s& h, const nwc::LaunchShape& s) {
+  return h.sched_ctas == s.ctas && h.sched_ring == s.ring_bytes &&
+         h.sched_tiles_per_batch == s.batch_tiles;
+}
+
+// Writes the launch schedule for shape `s` into the device image on `stream`
+// (from pageable memory: the call returns once the bytes are staged).
+nwc_status write_schedule(nwc_handle_s* h, const nwc::LaunchShape& s, cudaStream_t stream) {
+  std::vector<uint8_t> sched(nwc::sched_bytes((uint64_t)h->tiles));
+  nwc::build_schedule(h->index.data(), h->tiles, s, sched.data());
+  if (cudaMemcpyAsync(h->d_base + h->sched_off, sched.data(), sched.size(),
+                      cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return NWC_ERR_CUDA;
+  h->sched_ctas = s.ctas;
+  h->sched_ring = s.ring_bytes;
+  h->sched_tiles_per_batch = s.batch_tiles;
+  return NWC_OK;
+}
+
+// Launch geometry on the current device; rewrites the image's schedule (in
+// stream order) when it was made for another shape.
+nwc_status shape_for(nwc_handle_s* h, nwc::LaunchShape* s, cudaStream_t stream) {
+  int dev, sms;
+  size_t smem;
+  nwc_status st = current_device(&dev, &sms, &smem);
+  if (st != NWC_OK) return st;
+  st = shape_on(*h, sms, smem, s);
+  if (st != NWC_OK) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!same_shape(*h, *s)) st = write_schedule(h, *s, stream);
+  return st;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -63,7 +93,10 @@ nwc::TileParams base_params(const nwc_handle_s& h) {
   nwc::TileParams p;
   std::memset(&p, 0, sizeof(p));
   p.tiles = h.d_base + h.tiles_off;
-  p.index = reinterpret_cast<const uint32_t*>(h.d_base + h.index_off);
+  const uint8_t* sched = h.d_base + h.sched_off;
+  p.sched_cta = reinterpret_cast<const uint32_t*>(sched);
+  p.sched_batch = reinterpret_cast<const uint4*>(sched + nwc::sched_batch_off());
+  p.tile_ring = reinterpret_cast<const uint32_t*>(sched + nwc::sched_tile_off((uint64_t)h.tiles));
   p.table = reinterpret_cast<const uint32_t*>(h.d_base + h.table_off);
   p.table_bytes = nwc::table_bytes(h.lmax);
   p.rows = h.rows;
@@ -84,17 +117,36 @@ uint64_t workspace_bytes_for(const nwc_handle_s& h, int32_t batch) {
   return counters + 4ull * (uint64_t)h.tiles_c * (uint64_t)b * (uint64_t)(8 * h.tiles_r);
 }
 
-nwc_status make_handle(const uint8_t* blob_host_header_region, uint64_t bytes, const void* d_buf,
+nwc_status make_handle(const uint8_t* blob_host_header_region, uint64_t bytes, void* d_buf,
                        uint64_t d_bytes, nwc_handle_t* out, const uint8_t** lens) {
   nwc_handle_s tmp;
   if (!nwc::parse_blob(blob_host_header_region, bytes, bytes, &tmp, lens)) return NWC_ERR_CORRUPT;
   if (d_bytes < tmp.device_bytes) return NWC_ERR_INVALID_ARG;
   nwc_handle_s* h = new (std::nothrow) nwc_handle_s(tmp);
   if (!h) return NWC_ERR_NOMEM;
-  h->d_base = static_cast<const uint8_t*>(d_buf);
+  h->d_base = static_cast<uint8_t*>(d_buf);
   h->d_bytes = d_bytes;
   cudaGetDevice(&h->device);
   *out = h;
+  return NWC_OK;
+}
+
+// Geometry and schedule of a new handle on the current device: writes the
+// schedule into `image` (a host copy of the device image) when given, else
+// into the device image on `stream`.
+nwc_status init_schedule(nwc_handle_s* h, uint8_t* image, cudaStream_t stream) {
+  int dev, sms;
+  size_t smem;
+  nwc_status st = current_device(&dev, &sms, &smem);
+  if (st != NWC_OK) return st;
+  nwc::LaunchShape s;
+  st = shape_on(*h, sms, smem, &s);
+  if (st != NWC_OK) return st;
+  if (!image) return write_schedule(h, s, stream);
+  nwc::build_schedule(h->index.data(), h->tiles, s, image + h->sched_off);
+  h->sched_ctas = s.ctas;
+  h->sched_ring = s.ring_bytes;
+  h->sched_tiles_per_batch = s.batch_tiles;
   return NWC_OK;
 }
 
@@ -186,18 +238,23 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
   }
   std::memset(img + plan->blob_bytes, 0, plan->table_off - plan->blob_bytes);
   nwc::build_decode_table(plan->len, plan->lmax, reinterpret_cast<uint32_t*>(img + plan->table_off));
+  const uint64_t table_end = plan->table_off + nwc::table_bytes(plan->lmax);
+  std::memset(img + table_end, 0, plan->sched_off - table_end);
+  nwc_handle_t h = nullptr;
+  nwc_status st = make_handle(img, plan->blob_bytes, d_buf, d_bytes, &h, nullptr);
+  if (st == NWC_OK) st = init_schedule(h, img, nullptr);
   // From pageable memory the call returns once the bytes are staged, so the
   // image can be freed right after.
-  cudaError_t e = cudaMemcpyAsync(d_buf, img, plan->device_bytes, cudaMemcpyHostToDevice,
-                                  reinterpret_cast<cudaStream_t>(stream));
-  nwc_status st = NWC_OK;
-  if (e != cudaSuccess) {
+  if (st == NWC_OK && cudaMemcpyAsync(d_buf, img, plan->device_bytes, cudaMemcpyHostToDevice,
+                                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     st = NWC_ERR_CUDA;
-  } else {
-    st = make_handle(img, plan->blob_bytes, d_buf, d_bytes, out_handle, nullptr);
-  }
   std::free(img);
-  return st;
+  if (st != NWC_OK) {
+    delete h;
+    return st;
+  }
+  *out_handle = h;
+  return NWC_OK;
 }
 
 nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes, uint64_t* device_bytes) {
@@ -227,7 +284,14 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, u
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(static_cast<uint8_t*>(d_buf) + h->table_off, table.data(),
                         nwc::table_bytes(h->lmax), cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) {
+    st = init_schedule(h, nullptr, s);
+    if (st != NWC_OK) {
+      delete h;
+      return st;
+    }
+    e = cudaStreamSynchronize(s);
+  }
   if (e != cudaSuccess) {
     delete h;
     return NWC_ERR_CUDA;
@@ -236,7 +300,7 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, u
   return NWC_OK;
 }
 
-nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes, nwc_handle_t* out_handle) {
+nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* out_handle) {
   if (!d_buf || !out_handle || d_bytes < nwc::kIndexOffset) return NWC_ERR_INVALID_ARG;
   *out_handle = nullptr;
   nwc::BlobHeader hd;
@@ -255,9 +319,15 @@ nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes, nwc_handl
   if (d_bytes < tmp.device_bytes) return NWC_ERR_INVALID_ARG;
   nwc_handle_s* h = new (std::nothrow) nwc_handle_s(tmp);
   if (!h) return NWC_ERR_NOMEM;
-  h->d_base = static_cast<const uint8_t*>(d_buf);
+  h->d_base = static_cast<uint8_t*>(d_buf);
   h->d_bytes = d_bytes;
   cudaGetDevice(&h->device);
+  nwc_status st = init_schedule(h, nullptr, nullptr);
+  if (st == NWC_OK && cudaStreamSynchronize(nullptr) != cudaSuccess) st = NWC_ERR_CUDA;
+  if (st != NWC_OK) {
+    delete h;
+    return st;
+  }
   *out_handle = h;
   return NWC_OK;
 }
@@ -265,7 +335,7 @@ nwc_status nwc_handle_from_device(const void* d_buf, uint64_t d_bytes, nwc_handl
 nwc_status nwc_decompress(nwc_handle_t h, uint16_t* d_w_out, nwc_stream_t stream) {
   if (!h || !d_w_out || !aligned(d_w_out, 4)) return NWC_ERR_INVALID_ARG;
   nwc::LaunchShape s;
-  nwc_status st = shape_for(*h, &s);
+  nwc_status st = shape_for(h, &s, reinterpret_cast<cudaStream_t>(stream));
   if (st != NWC_OK) return st;
   nwc::TileParams p = base_params(*h);
   p.out = d_w_out;
@@ -292,7 +362,7 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
   // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
   if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
   nwc::LaunchShape s;
-  nwc_status st = shape_for(*h, &s);
+  nwc_status st = shape_for(h, &s, reinterpret_cast<cudaStream_t>(stream));
   if (st != NWC_OK) return st;
   nwc::TileParams p = base_params(*h);
   p.ring_offset = (uint32_t)s.ring_offset;
@@ -374,6 +444,40 @@ nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word) {
   if (word) *word = w;
   if (w & nwc::kErrTimeout) return NWC_ERR_DEVICE_TIMEOUT;
   if (w & nwc::kErrCorrupt) return NWC_ERR_DEVICE_CORRUPT;
+  return NWC_OK;
+}
+
+nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
+                                 uint64_t smem_limit, nwc_schedule_info* info,
+                                 uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring) {
+  if (!blob || !info || info->struct_size < sizeof(nwc_schedule_info) || sm_count < 1)
+    return NWC_ERR_INVALID_ARG;
+  nwc_handle_s h;
+  if (!nwc::parse_blob(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &h, nullptr))
+    return NWC_ERR_CORRUPT;
+  nwc::LaunchShape s;
+  nwc_status st = shape_on(h, sm_count, (size_t)smem_limit, &s);
+  if (st != NWC_OK) return st;
+  std::vector<uint8_t> sched;
+  try {
+    sched.resize(nwc::sched_bytes((uint64_t)h.tiles));
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
+  nwc::build_schedule(h.index.data(), h.tiles, s, sched.data());
+  const uint32_t* cb = reinterpret_cast<const uint32_t*>(sched.data());
+  info->ctas = s.ctas;
+  info->batch_tiles = s.batch_tiles;
+  info->ring_bytes = s.ring_bytes;
+  info->tiles = h.tiles;
+  info->batches = cb[s.ctas];
+  info->smem_bytes = s.smem_bytes;
+  if (cta_batch) std::memcpy(cta_batch, cb, 4 * ((size_t)s.ctas + 1));
+  if (batch)
+    std::memcpy(batch, sched.data() + nwc::sched_batch_off(), 16 * (size_t)cb[s.ctas]);
+  if (tile_ring)
+    std::memcpy(tile_ring, sched.data() + nwc::sched_tile_off((uint64_t)h.tiles),
+                4 * (size_t)h.tiles);
   return NWC_OK;
 }
 

@@ -15,7 +15,15 @@
 // column 64 (k/16) + 2t + k%2); its raw byte is at (k/16) * 512 + 16 t + k%16.
 // Tiles are stored column-block-major: u = j * tiles_r + i.
 //
-// Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)].
+// Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)]
+// | zero pad to 256 | launch schedule (sched_bytes(tiles) bytes).  The launch
+// schedule is not part of the blob: the library writes it for the device that
+// runs the kernels (its SM count and shared memory), as
+//   u32 cta_batch[kMaxCtas + 1]   first batch of each CTA (padded to 16 bytes)
+//   u32x4 batch[sched_max_batches(tiles)]
+//        {tile-area offset in 16-byte units, bytes, ring offset, batches of
+//         the same CTA that must be released before this one is issued}
+//   u32 tile_ring[tiles]          ring offset of each tile's chunk
 #pragma once
 #include <cstdint>
 
@@ -57,7 +65,17 @@ constexpr int kEntryLen0Shift = 15;
 constexpr uint32_t kEntryInvalid = 1u << 19;
 constexpr uint32_t kEntrySingle = 1u << 31;
 
-inline uint64_t round_up(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
+constexpr uint64_t round_up(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
+
+// Launch-schedule area.  At most kMaxCtas persistent CTAs; every batch but a
+// CTA's last holds at least two tiles.
+constexpr uint32_t kMaxCtas = 256;
+constexpr uint64_t sched_max_batches(uint64_t tiles) { return (tiles + 1) / 2 + kMaxCtas; }
+constexpr uint64_t sched_batch_off() { return round_up(4ull * (kMaxCtas + 1), 16); }
+constexpr uint64_t sched_tile_off(uint64_t tiles) {
+  return sched_batch_off() + 16ull * sched_max_batches(tiles);
+}
+constexpr uint64_t sched_bytes(uint64_t tiles) { return round_up(sched_tile_off(tiles) + 4ull * tiles, 256); }
 
 struct BlobHeader {
   uint32_t magic, version, header_bytes, lmax;

@@ -17,19 +17,23 @@ struct nwc_plan_s {
   uint64_t tiles_off = 0;       // blob offset of the tile area
   uint64_t blob_bytes = 0;      // serialisable blob
   uint64_t table_off = 0;       // device-image offset of the decode table
-  uint64_t device_bytes = 0;    // blob + padding + decode table
+  uint64_t sched_off = 0;       // device-image offset of the launch schedule
+  uint64_t device_bytes = 0;    // blob + padding + decode table + schedule
 };
 
 struct nwc_handle_s {
-  const uint8_t* d_base = nullptr;  // caller's device buffer
+  uint8_t* d_base = nullptr;  // caller's device buffer
   uint64_t d_bytes = 0;
   int64_t rows = 0, cols = 0;
   uint32_t tile_cols = 512, lmax = 7, filler = 0;
   int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
-  uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0;
+  uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0, sched_off = 0;
   uint64_t device_bytes = 0;
   uint64_t max_chunk = 0;  // largest chunk in bytes
   int device = 0;
+  std::vector<uint32_t> index;  // chunk offsets (16-byte units), tiles + 1
+  // Shape the device image's launch schedule was written for (0: none yet).
+  int sched_ctas = 0, sched_ring = 0, sched_tiles_per_batch = 0;
 };
 
 namespace nwc {
