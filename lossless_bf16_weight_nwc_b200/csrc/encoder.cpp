@@ -64,16 +64,14 @@ struct TileView {
 void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t bits[kLanes]) {
   const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
   TileView v{w, p.rows, p.cols, i * kTileRows, j * (int64_t)p.tile_cols, (uint8_t)p.filler};
-  const int groups = (int)p.tile_cols / 64;
   for (int t = 0; t < kLanes; ++t) bits[t] = 0;
   for (int r = 0; r < kTileRows; ++r) {
     for (int c = 0; c < (int)p.tile_cols; ++c) {
-      const int t = (c % 64) / 2;
+      const int t = 4 * r + (c % 64) / 16;  // lane t = 4 r + q owns row r, columns 16 q .. of a group
       const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
       bits[t] += p.len[s];
     }
   }
-  (void)groups;
 }
 
 uint32_t stream_bytes_of(const uint32_t bits[kLanes]) {
@@ -327,26 +325,27 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
         const uint32_t lane_start = out;
         uint32_t accb = 0;  // pending bits, right-aligned
         int nacc = 0;
+        // Lane t = 4 r + q owns row r; group g gives it columns 64 g + 16 q ..
+        // 64 g + 16 q + 15, symbols 16 g .. 16 g + 15.
+        const int r = t / 4;
         for (uint32_t g = 0; g < groups; ++g) {
-          for (int r = 0; r < kTileRows; ++r) {
-            for (int hh = 0; hh < 2; ++hh) {
-              const int c = (int)(64 * g) + 2 * t + hh;
-              const int k = (int)(16 * g) + 2 * r + hh;
-              uint8_t s = v.filler, rb = 0;
-              if (v.inside(r, c)) {
-                const uint16_t x = v.at(r, c);
-                s = exponent_byte(x);
-                rb = raw_byte(x);
-              }
-              raw[(k / 16) * 512 + 16 * t + (k % 16)] = rb;
-              accb = (accb << p.len[s]) | p.code[s];
-              nacc += p.len[s];
-              while (nacc >= 8) {
-                seq[out++] = (uint8_t)(accb >> (nacc - 8));
-                nacc -= 8;
-              }
-              accb &= (1u << nacc) - 1u;
+          for (int kk = 0; kk < 16; ++kk) {
+            const int c = (int)(64 * g) + 16 * (t % 4) + kk;
+            const int k = (int)(16 * g) + kk;
+            uint8_t s = v.filler, rb = 0;
+            if (v.inside(r, c)) {
+              const uint16_t x = v.at(r, c);
+              s = exponent_byte(x);
+              rb = raw_byte(x);
             }
+            raw[(k / 16) * 512 + 16 * t + (k % 16)] = rb;
+            accb = (accb << p.len[s]) | p.code[s];
+            nacc += p.len[s];
+            while (nacc >= 8) {
+              seq[out++] = (uint8_t)(accb >> (nacc - 8));
+              nacc -= 8;
+            }
+            accb &= (1u << nacc) - 1u;
           }
         }
         if (nacc > 0) seq[out++] = (uint8_t)(accb << (8 - nacc));

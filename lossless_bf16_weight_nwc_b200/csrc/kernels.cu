@@ -38,7 +38,9 @@ __device__ unsigned int g_device_error;
 namespace {
 
 constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
-constexpr int kRingSlack = 16;                   // lanes may read a few words past a chunk
+constexpr int kRingSlack = 32;                   // lanes may read a few words past a chunk
+constexpr int kTablePieces = 8;                  // bulk copies that bring in the decode table
+constexpr int kXStageBytes = 8448;               // x columns staged per CTA (GEMV)
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---- PTX helpers -----------------------------------------------------------
@@ -96,6 +98,14 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -103,14 +113,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
                : "r"(addr));
   return v;
 }
-// Loads a word only when `need` is non-zero (predicated, no branch); else
-// returns 0.
-__device__ __forceinline__ uint32_t lds32_if(uint32_t addr, uint32_t need) {
-  uint32_t v = 0;
+// v = [addr] when `need` is non-zero, else v is left as it was (predicated
+// load, no branch).
+__device__ __forceinline__ void lds32_keep(uint32_t& v, uint32_t addr, uint32_t need) {
   asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %2, 0;\n\t@p ld.shared.u32 %0, [%1];\n\t}"
                : "+r"(v)
                : "r"(addr), "r"(need));
-  return v;
 }
 // Low word of ({hi, lo} >> (n mod 32)).
 __device__ __forceinline__ uint32_t shr_wrap(uint32_t lo, uint32_t hi, uint32_t n) {
@@ -118,21 +126,19 @@ __device__ __forceinline__ uint32_t shr_wrap(uint32_t lo, uint32_t hi, uint32_t 
   asm("shf.r.wrap.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(lo), "r"(hi), "r"(n));
   return r;
 }
-// c + bf16(a half) * bf16(b half) in FP32; HI selects the upper halves.
-template <bool HI>
-__device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
-  float d;
-  if (HI)
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}"
-        : "=f"(d)
-        : "r"(a), "r"(b), "f"(c));
-  else
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}"
-        : "=f"(d)
-        : "r"(a), "r"(b), "f"(c));
-  return d;
+// D += A B on the tensor cores, one warp: A is 16 x 16 BF16 (row-major
+// fragment a0..a3), B is 16 x 8 BF16 (column-major fragment b0, b1), D is
+// 16 x 8 FP32 (d0..d3).  Fragment of lane L (g = L / 4, c = L % 4):
+//   a0 = A[g][2c, 2c+1]   a1 = A[g+8][2c, 2c+1]   a2 = A[g][2c+8, 2c+9]   a3 = A[g+8][2c+8, 2c+9]
+//   b0 = B[2c, 2c+1][g]   b1 = B[2c+8, 2c+9][g]
+//   d0 = D[g][2c]   d1 = D[g][2c+1]   d2 = D[g+8][2c]   d3 = D[g+8][2c+1]
+// (the lower 16 bits of a register hold the first of its two elements).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // ---- bit reader --------------------------------------------------------------
@@ -145,16 +151,22 @@ __device__ __forceinline__ float fma_bf16(uint32_t a, uint32_t b, float c) {
 // since entry bits 4..6 are zero and bits 0..3 hold the consumed count.
 struct BitReader {
   uint32_t hi, lo, nbacc;
-  uint32_t wp;  // shared-window address of the next stream word
+  uint32_t nw;  // the stream word after the window, loaded ahead
+  uint32_t wp;  // shared-window address of the word after nw
 
-  __device__ __forceinline__ void init(uint32_t area, uint32_t start) {
-    wp = area + (start & ~3u);
+  uint32_t last;  // highest word address the reader may touch
+
+  // `limit`: end of the shared memory the reader may read (see PairReader).
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
+    last = limit - 4;
+    wp = min(area + (start & ~3u), last - 8);
     const uint32_t sh = (start & 3u) * 8u;
     const uint32_t w0 = lds32(wp), w1 = lds32(wp + 4);
+    nw = lds32(wp + 8);
     hi = __funnelshift_l(w1, w0, sh);
     lo = w1 << sh;
     nbacc = 64u - sh;
-    wp += 8;
+    wp += 12;
   }
   // Consumes the count in bits 0..3 of e (the funnel shifts use e & 31).
   __device__ __forceinline__ void consume_entry(uint32_t e) {
@@ -169,15 +181,18 @@ struct BitReader {
   }
   // With fewer than 32 valid bits (bit 5 of the count clear; the count never
   // reaches 64 at a refill point), append the next word right after the valid
-  // bits; the count becomes count | 32 either way.  No branch: the load is
-  // predicated and an empty word shifts in nothing.
+  // bits; the count becomes count | 32 either way.  No branch: an empty word
+  // shifts in nothing, and the word after it is fetched (predicated) only
+  // when this one was used, so the shared-memory load is off the decoder's
+  // dependency chain.
   __device__ __forceinline__ void refill() {
     const uint32_t need = (~nbacc) & 32u;
-    const uint32_t w = lds32_if(wp, need);
+    const uint32_t w = need ? nw : 0u;
     hi |= shr_wrap(w, 0u, nbacc);
     lo |= shr_wrap(0u, w, nbacc);
-    wp += need >> 3;
     nbacc |= 32u;
+    lds32_keep(nw, wp, need);
+    wp = min(wp + (need >> 3), last);
   }
 };
 
@@ -201,6 +216,77 @@ __device__ __forceinline__ uint32_t decode_pair(BitReader& br, uint32_t table) {
   }
   return e;
 }
+
+// Reader for the 14-bit peek (lmax <= 7), two steps at a time: two steps
+// consume at most 28 bits, so one 32-bit window taken before them holds both
+// peeks.  The stream is kept as three consecutive words a, b, c with p (< 32)
+// the offset of the next unread bit in a; after two steps the words move on by
+// one when p passed 32, and the word after c is fetched (predicated) at once,
+// two steps before it can be needed, so no shared-memory load of the stream
+// lies on the decoder's dependency chain.
+struct PairReader {
+  uint32_t a, b, c;  // stream words base, base + 1, base + 2
+  uint32_t p;        // next unread bit of a (0 = its bit 31)
+  uint32_t next;     // shared-window address of word base + 3
+
+  uint32_t last;     // highest word address the reader may touch
+
+  // `limit`: end of the shared memory the reader may read; a corrupt stream
+  // start or length can then misdecode but never read outside it.
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
+    last = limit - 4;
+    const uint32_t at = min(area + (start & ~3u), last - 8);
+    a = lds32(at);
+    b = lds32(at + 4);
+    c = lds32(at + 8);
+    next = at + 12;
+    p = (start & 3u) * 8u;
+  }
+  // Entries e0, e1 of the next two steps.
+  __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
+    const uint32_t w = __funnelshift_l(b, a, p);  // 32 bits from the next unread one
+    e0 = lds32(table + ((w >> 16) & 0xFFFCu));
+    const uint32_t w1 = __funnelshift_l(0u, w, e0);  // shift by e0's count (bits 0..3)
+    e1 = lds32(table + ((w1 >> 16) & 0xFFFCu));
+    // Bits 0..6 of e0 + e1 are the two counts' sum (bits 4..6 of an entry are
+    // zero), below 29, so q = p + both counts < 61.
+    const uint32_t q = (p + e0 + e1) & 0x7Fu;
+    const uint32_t adv = q & 32u;
+    a = adv ? b : a;
+    b = adv ? c : b;
+    lds32_keep(c, next, adv);
+    next = min(next + (adv >> 3), last);
+    p = q & 31u;
+  }
+};
+
+// Both readers behind one interface: two() yields the entries of the next two
+// steps.  FAST uses the window reader above; lmax 8..12 the bit buffer, whose
+// second lookup handles a pair that does not fit in the 12-bit peek.
+template <bool FAST>
+struct StreamDecoder;
+template <>
+struct StreamDecoder<true> {
+  PairReader r;
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
+    r.init(area, start, limit);
+  }
+  __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
+    r.two(table, e0, e1);
+  }
+};
+template <>
+struct StreamDecoder<false> {
+  BitReader br;
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
+    br.init(area, start, limit);
+  }
+  __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
+    e0 = decode_pair<false>(br, table);
+    e1 = decode_pair<false>(br, table);
+    br.refill();
+  }
+};
 
 // Raw bytes of step r (row r of a 64-column group) duplicated into both bytes
 // of each half: [r0, r0, r1, r1].
@@ -255,6 +341,7 @@ struct Smem {
   uint64_t* table_bar;
   uint64_t* full;    // per batch slot: bytes landed
   uint64_t* empty;   // per batch slot: tiles released
+  uint8_t* xstage;   // kXStageBytes: the CTA's columns of x (GEMV)
   uint8_t* ring;
 };
 
@@ -263,6 +350,7 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
   s.table_bar = reinterpret_cast<uint64_t*>(smem + p.table_bytes);
   s.full = s.table_bar + 1;
   s.empty = s.full + kSlots;
+  s.xstage = reinterpret_cast<uint8_t*>(s.empty + kSlots);
   s.ring = smem + p.ring_offset;
   return s;
 }
@@ -276,8 +364,14 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
 __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const uint4* desc,
                         int nb, int lane) {
   if (lane == 0) {
+    // The decode table in kTablePieces copies, each CTA starting at a different
+    // piece, so that the CTAs do not all ask the same L2 lines at once.
     mbar_expect_tx(s.table_bar, p.table_bytes);
-    bulk_load(smem, p.table, p.table_bytes, s.table_bar);
+    const uint32_t piece = p.table_bytes / kTablePieces;
+    for (int k = 0; k < kTablePieces; ++k) {
+      const uint32_t off = ((blockIdx.x + k) % kTablePieces) * piece;
+      bulk_load(smem + off, reinterpret_cast<const uint8_t*>(p.table) + off, piece, s.table_bar);
+    }
   }
   const uint4 none = make_uint4(0u, 0u, 0u, 0u);
   uint4 cur = lane < nb ? __ldg(desc + lane) : none;
@@ -319,82 +413,93 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
   }
 }
 
-// Consumer side: wait until tile q's batch k has landed.  The schedule keeps
-// fewer than kSlots - ceil(kMaxConsumers / batch_tiles) batches outstanding, so
-// by the time a consumer polls slot k % kSlots (after finishing its previous
-// tile, at most kMaxConsumers tiles back) the slot's previous batch k - kSlots
-// was released long ago: the parity it polls is batch k's.
+// Consumer side: wait until batch k has landed.  The schedule keeps fewer than
+// kSlots - ceil(kMaxLag / batch_tiles) batches outstanding, so by the time a
+// consumer polls slot k % kSlots (its last released tile at most kMaxLag tiles
+// back) the slot's previous batch k - kSlots was released long ago: the parity
+// it polls is batch k's.
 __device__ __forceinline__ bool wait_batch(const Smem& s, int k) {
   return __all_sync(kFull, wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1)));
 }
 
-// Sums 8 per-lane row values over the 32 lanes.  On return every lane holds the
-// total of row (lane >> 2).
-__device__ __forceinline__ float reduce_rows8(const float (&v)[8], int lane) {
-  float a[4], b[2];
-  const bool h16 = lane & 16, h8 = lane & 8, h4 = lane & 4;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float send = h16 ? v[i] : v[4 + i];
-    const float keep = h16 ? v[4 + i] : v[i];
-    a[i] = keep + __shfl_xor_sync(kFull, send, 16);
+// Four BF16 values x[col .. col + 3] of one row of x as two words, or zeros
+// where the row is absent or the columns lie past `cols` (cols is even, so a
+// word is wholly inside or outside).  Every lane loads from a valid address
+// and selects afterwards, so lanes never diverge.  vec (uniform): 8-byte
+// aligned and inside.
+__device__ __forceinline__ uint2 load_x4(const uint16_t* xrow, int64_t cols, int64_t col,
+                                         bool present, bool vec) {
+  uint2 v;
+  if (vec) {
+    v = __ldg(reinterpret_cast<const uint2*>(xrow + col));
+  } else {
+    const bool in0 = col < cols, in1 = col + 2 < cols;
+    v.x = __ldg(reinterpret_cast<const uint32_t*>(xrow + (in0 ? col : 0)));
+    v.y = __ldg(reinterpret_cast<const uint32_t*>(xrow + (in1 ? col + 2 : 0)));
+    v.x = in0 ? v.x : 0u;
+    v.y = in1 ? v.y : 0u;
   }
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const float send = h8 ? a[i] : a[2 + i];
-    const float keep = h8 ? a[2 + i] : a[i];
-    b[i] = keep + __shfl_xor_sync(kFull, send, 8);
-  }
-  const float send = h4 ? b[0] : b[1];
-  const float keep = h4 ? b[1] : b[0];
-  float c = keep + __shfl_xor_sync(kFull, send, 4);
-  c += __shfl_xor_sync(kFull, c, 2);
-  c += __shfl_xor_sync(kFull, c, 1);
-  return c;
+  v.x = present ? v.x : 0u;
+  v.y = present ? v.y : 0u;
+  return v;
 }
 
-__device__ __forceinline__ uint32_t load_x_pair(const uint16_t* x, int64_t cols, int64_t col) {
-  if (col + 1 < cols) return __ldg(reinterpret_cast<const uint32_t*>(x + col));
-  if (col < cols) return __ldg(x + col);
-  return 0u;
-}
-
-// One tile of the GEMV: decode the lane's 16 * CP symbols, 8 rows per 64-column
-// group, and accumulate acc[r][b] += W[r][c] * x[b][c] in FP32.  The BF16 pair
-// of x for each group (columns col0 + 64 g + 2 lane, + 1) is read from L1 one
-// group ahead and serves the group's 8 rows.
-template <int CP, int B, bool FAST>
-__device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table, int lane,
-                                                 float (&acc)[8][B], const uint16_t* x,
-                                                 int64_t cols, int64_t col0) {
+// A whole tile (8 rows x 64 CP columns at column col_tile) on the tensor cores.
+// Lane L = 4 g + c decodes row g, columns 64 m + 16 c .. + 15 of every group m.
+// In 16-column block s of a group the lane supplies W[row g][16 c + 4 s + 0..1]
+// and [.. + 2..3] as B = W^T (k x row), and x[batch g][the same columns] (and
+// batch g + 8 when WIDE) as A (batch x k), so D[batch][row] accumulates x W^T;
+// the k order inside a block is one column permutation for A and B alike, so
+// the sum is unchanged.  On return d[0..1] hold y[batch g][rows 2c, 2c + 1] of
+// the tile's contribution and d[2..3] the same for batch g + 8.  Each block's
+// x is read one block ahead: from shared memory (XSM: xs = the staged row 0 at
+// the tile's first column, rows xrow bytes apart) or else through L1.
+template <int CP, bool WIDE, bool FAST, bool XSM>
+__device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table, uint32_t limit,
+                                                 int lane, float (&d)[4], const TileParams& p,
+                                                 int64_t col_tile, bool xvec, uint32_t xs,
+                                                 uint32_t xrow) {
   constexpr int kRaw = CP * 512;
-  BitReader br;
-  br.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane));
-  uint32_t xn[B];
-#pragma unroll
-  for (int b = 0; b < B; ++b) xn[b] = load_x_pair(x + (int64_t)b * cols, cols, col0 + 2 * lane);
-  constexpr int kGroupUnroll = B <= 4 ? 2 : 1;
-#pragma unroll kGroupUnroll
-  for (int g = 0; g < CP; ++g) {
-    const uint4 rv = lds128(chunk + g * 512 + lane * 16);
-    uint32_t xg[B];
-#pragma unroll
-    for (int b = 0; b < B; ++b) xg[b] = xn[b];
-    if (g + 1 < CP) {
-#pragma unroll
-      for (int b = 0; b < B; ++b)
-        xn[b] = load_x_pair(x + (int64_t)b * cols, cols, col0 + (g + 1) * 64 + 2 * lane);
+  StreamDecoder<FAST> dec;
+  dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
+  const int g = lane >> 2, c = lane & 3;
+  const int64_t cols = p.cols;
+  // Rows past the batch read row 0 (a valid address) and are zeroed.
+  const bool has0 = g < p.batch, has1 = WIDE && g + 8 < p.batch;
+  const uint16_t* xr0 = p.x + (has0 ? (int64_t)g * cols : 0);
+  const uint16_t* xr1 = p.x + (has1 ? (int64_t)(g + 8) * cols : 0);
+  const uint32_t xs0 = xs + (has0 ? g * xrow : 0u) + 32u * c;
+  const uint32_t xs1 = xs + (has1 ? (g + 8) * xrow : 0u) + 32u * c;
+  const bool vec = xvec && col_tile + CP * 64 <= cols;  // whole tile inside and aligned
+  // x of the block at column offset o (from this lane's first column).
+  auto x_at = [&](const uint16_t* xr, uint32_t xsr, bool has, uint32_t o) -> uint2 {
+    if (XSM) {
+      uint2 v = lds64(xsr + 2 * o);
+      v.x = has ? v.x : 0u;
+      v.y = has ? v.y : 0u;
+      return v;
     }
+    return load_x4(xr, cols, col_tile + 16 * c + o, has, vec);
+  };
+  uint2 xa = x_at(xr0, xs0, has0, 0);
+  uint2 xb = WIDE ? x_at(xr1, xs1, has1, 0) : make_uint2(0u, 0u);
+#pragma unroll 1
+  for (int m = 0; m < CP; ++m) {
+    const uint4 rv = lds128(chunk + m * 512 + lane * 16);
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const uint32_t e = decode_pair<FAST>(br, table);
-      const uint32_t w = assemble(raw_pair_r(rv, r), e);
-#pragma unroll
-      for (int b = 0; b < B; ++b) {
-        acc[r][b] = fma_bf16<false>(w, xg[b], acc[r][b]);
-        acc[r][b] = fma_bf16<true>(w, xg[b], acc[r][b]);
+    for (int s = 0; s < 4; ++s) {
+      const uint2 xa_s = xa, xb_s = xb;
+      // Next block's x: + 4 columns, or the next group's first block.
+      const uint32_t no = s < 3 ? 64 * m + 4 * (s + 1) : 64 * (m + 1);
+      if (s < 3 || m + 1 < CP) {
+        xa = x_at(xr0, xs0, has0, no);
+        if (WIDE) xb = x_at(xr1, xs1, has1, no);
       }
-      if (r & 1) br.refill();
+      uint32_t e0, e1;
+      dec.two(table, e0, e1);
+      const uint32_t w0 = assemble(raw_pair_r(rv, 2 * s), e0);
+      const uint32_t w1 = assemble(raw_pair_r(rv, 2 * s + 1), e1);
+      mma_bf16_16816(d, xa_s.x, WIDE ? xb_s.x : 0u, xa_s.y, WIDE ? xb_s.y : 0u, w0, w1);
     }
   }
 }
@@ -407,8 +512,8 @@ __device__ __forceinline__ void cta_range(const TileParams& p, int64_t* first, i
   *n = (int)(b - a);
 }
 
-// Sets up barriers; returns false for the producer warp (warp NC; its work is
-// done) and for consumers when the decode table never arrived.
+// Sets up barriers and runs the producer warp (warp NC), for which it returns
+// false once its work is done.
 template <int NC>
 __device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const Smem& s) {
   if (threadIdx.x == 0) {
@@ -426,6 +531,11 @@ __device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const 
     produce(p, smem, s, p.sched_batch + b0, (int)(b1 - b0), threadIdx.x & 31);
     return false;
   }
+  return true;
+}
+
+// Consumers: wait for the decode table.
+__device__ __forceinline__ bool wait_table(const Smem& s) {
   return __all_sync(kFull, wait_bounded(s.table_bar, 0));
 }
 
@@ -446,7 +556,10 @@ struct TilePos {
   }
 };
 
-template <int NC, int CP, int B, bool FAST>
+// y[b][n] for up to 8 (16 when WIDE) rows b of x.  Consumer warp w takes
+// tiles w, w + NC, ...; each tile's partial sums go straight to y (one column
+// block) or to the workspace, reduced after all tiles in a fixed order.
+template <int NC, int CP, bool WIDE, bool FAST>
 __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem s = carve(smem, p);
@@ -455,9 +568,32 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   cta_range(p, &first, &n);
   if (!setup<NC>(p, smem, s)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
-  const int64_t cols = p.cols;
+  const uint32_t limit = ring + (uint32_t)p.ring_bytes + kRingSlack;  // end of the ring's slack
+  const int batch = p.batch;
+  const bool xvec = ((reinterpret_cast<uintptr_t>(p.x) & 7) == 0) && (p.cols % 4 == 0);
+  // The CTA's column blocks j0 .. j1 of x, staged in shared memory while the
+  // decode table is on its way, when they fit; else x is read through L1.
+  constexpr int kTileCols = CP * 64;
+  const int64_t j0 = first / p.tiles_r, j1 = (first + n - 1) / p.tiles_r;
+  const int64_t span = (j1 - j0 + 1) * kTileCols;        // columns staged
+  const uint32_t xrow = (uint32_t)(span * 2 + 16);       // bytes per row, padded
+  const bool xsmem = (uint64_t)batch * xrow <= (uint64_t)kXStageBytes;
+  if (xsmem) {
+    const uint32_t words = (uint32_t)(span / 2), total = (uint32_t)batch * words;
+    for (uint32_t t = threadIdx.x; t < total; t += NC * 32) {
+      const uint32_t b = t / words, w = t - b * words;
+      const int64_t col = j0 * kTileCols + 2 * (int64_t)w;
+      const uint32_t v =
+          col < p.cols ? __ldg(reinterpret_cast<const uint32_t*>(p.x + b * p.cols + col)) : 0u;
+      *reinterpret_cast<uint32_t*>(s.xstage + b * xrow + 4 * w) = v;
+    }
+    named_barrier_sync(1, NC * 32);  // consumers only
+  }
+  if (!wait_table(s)) return;
+  const uint32_t xst = smem_u32(s.xstage);
   const uint32_t* tile_ring = p.tile_ring + first;
   uint32_t at_next = warp < n ? __ldg(tile_ring + warp) : 0u;
   TilePos pos;
@@ -468,34 +604,28 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
     if (q + NC < n) at_next = __ldg(tile_ring + q + NC);  // next tile's ring offset, early
     if (!wait_batch(s, k)) return;
     const int64_t i = pos.i, j = pos.j;
-    float acc[8][B];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-      for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
-    decode_gemv_tile<CP, B, FAST>(chunk, table, lane, acc, p.x, cols, j * (CP * 64));
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    if (xsmem)
+      decode_gemv_tile<CP, WIDE, FAST, true>(chunk, table, limit, lane, d, p, j * kTileCols, xvec,
+                                             xst + (uint32_t)((j - j0) * kTileCols * 2), xrow);
+    else
+      decode_gemv_tile<CP, WIDE, FAST, false>(chunk, table, limit, lane, d, p, j * kTileCols, xvec,
+                                              0u, 0u);
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[k % kSlots]);  // release the tile's share of the batch
-
-    // Row sums of this tile: lane L holds row L >> 2 for every batch row.
-    float tot[B];
+    // Lane (g, c) holds rows 2c, 2c + 1 of the tile for batch rows g and g + 8.
+    const int64_t row = i * 8 + 2 * c;
 #pragma unroll
-    for (int b = 0; b < B; ++b) {
-      float v[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) v[r] = acc[r][b];
-      tot[b] = reduce_rows8(v, lane);
-    }
-    const int64_t row = i * 8 + (lane >> 2);
-    if ((lane & 3) == 0) {
+    for (int h = 0; h < (WIDE ? 2 : 1); ++h) {
+      const int b = g + 8 * h;
+      if (b >= batch) continue;
       if (p.tiles_c == 1) {
-        if (row < p.rows)
-#pragma unroll
-          for (int b = 0; b < B; ++b) p.y[(int64_t)b * p.rows + row] = tot[b];
+        float* yb = p.y + (int64_t)b * p.rows;
+        if (row < p.rows) yb[row] = d[2 * h];
+        if (row + 1 < p.rows) yb[row + 1] = d[2 * h + 1];
       } else {
-#pragma unroll
-        for (int b = 0; b < B; ++b)
-          __stcg(&p.partial[((int64_t)j * B + b) * p.rows_pad + row], tot[b]);
+        __stcg(reinterpret_cast<float2*>(p.partial + ((int64_t)j * batch + b) * p.rows_pad + row),
+               make_float2(d[2 * h], d[2 * h + 1]));
       }
     }
   }
@@ -518,19 +648,19 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
       const int src = __ffs(mask) - 1;
       mask &= mask - 1;
       const int64_t i = (uint32_t)(first + q0 + src * NC) % (uint32_t)p.tiles_r;
-      for (int qq = lane; qq < 8 * B; qq += 32) {
+      for (int qq = lane; qq < 8 * batch; qq += 32) {
         const int b = qq >> 3, rr = qq & 7;
         const int64_t orow = i * 8 + rr;
         const float* part = p.partial + (int64_t)b * p.rows_pad + orow;
-        const int64_t stride = (int64_t)B * p.rows_pad;
+        const int64_t stride = (int64_t)batch * p.rows_pad;
         float sum = 0.f;
         int64_t jj = 0;
         for (; jj + 8 <= p.tiles_c; jj += 8) {
           float v[8];
 #pragma unroll
-          for (int k = 0; k < 8; ++k) v[k] = __ldcg(part + (jj + k) * stride);
+          for (int u = 0; u < 8; ++u) v[u] = __ldcg(part + (jj + u) * stride);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) sum += v[k];
+          for (int u = 0; u < 8; ++u) sum += v[u];
         }
         for (; jj < p.tiles_c; ++jj) sum += __ldcg(part + jj * stride);
         if (orow < p.rows) p.y[(int64_t)b * p.rows + orow] = sum;
@@ -547,12 +677,14 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
   int64_t first;
   int n;
   cta_range(p, &first, &n);
-  if (!setup<NC>(p, smem, s)) return;
+  if (!setup<NC>(p, smem, s) || !wait_table(s)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
+  const uint32_t limit = ring + (uint32_t)p.ring_bytes + kRingSlack;  // end of the ring's slack
   const int64_t cols = p.cols;
-  const bool even_cols = (cols & 1) == 0;
+  // Rows start 16-byte aligned: 16 columns of a row go out as two 16-byte stores.
+  const bool vec = (cols % 8 == 0) && ((reinterpret_cast<uintptr_t>(p.out) & 15) == 0);
   constexpr int kRaw = CP * 512;
   uint32_t invalid = 0;
   const uint32_t* tile_ring = p.tile_ring + first;
@@ -565,26 +697,36 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     if (q + NC < n) at_next = __ldg(tile_ring + q + NC);
     if (!wait_batch(s, k)) return;
     const int64_t i = pos.i, j = pos.j;
-    BitReader br;
-    br.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane));
-    const bool full_tile = (i + 1) * 8 <= p.rows && (j + 1) * (CP * 64) <= cols && even_cols;
+    StreamDecoder<FAST> dec;
+    dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
+    // Lane L owns row L / 4 of the tile and 16 consecutive columns per group.
+    const int64_t row = i * 8 + (lane >> 2);
+    const bool row_in = row < p.rows;
+    uint16_t* orow = p.out + row * cols;
 #pragma unroll 1
     for (int g = 0; g < CP; ++g) {
       const uint4 rv = lds128(chunk + g * 512 + lane * 16);
-      const int64_t col = j * (CP * 64) + g * 64 + 2 * lane;
+      const int64_t col = j * (CP * 64) + g * 64 + 16 * (lane & 3);
+      uint32_t wv[8];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const uint32_t e = decode_pair<FAST>(br, table);
-        invalid |= e;
-        const uint32_t w = assemble(raw_pair_r(rv, r), e);
-        const int64_t row = i * 8 + r;
-        if (full_tile) {
-          *reinterpret_cast<uint32_t*>(p.out + row * cols + col) = w;
-        } else if (row < p.rows) {
-          if (col < cols) p.out[row * cols + col] = (uint16_t)w;
-          if (col + 1 < cols) p.out[row * cols + col + 1] = (uint16_t)(w >> 16);
+      for (int r = 0; r < 8; r += 2) {
+        uint32_t e0, e1;
+        dec.two(table, e0, e1);
+        invalid |= e0 | e1;
+        wv[r] = assemble(raw_pair_r(rv, r), e0);
+        wv[r + 1] = assemble(raw_pair_r(rv, r + 1), e1);
+      }
+      if (row_in && vec && col + 16 <= cols) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + col);
+        dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+      } else if (row_in) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          const int64_t c0 = col + 2 * r;
+          if (c0 < cols) orow[c0] = (uint16_t)wv[r];
+          if (c0 + 1 < cols) orow[c0 + 1] = (uint16_t)(wv[r] >> 16);
         }
-        if (r & 1) br.refill();
       }
     }
     __syncwarp();
@@ -608,48 +750,33 @@ cudaError_t ensure_smem(Kernel k, size_t bytes, int (&configured)[64]) {
   return e;
 }
 
-// Consumer warps per CTA: more warps hide the decoder's dependency chains, as
-// long as the batch's accumulators leave registers for them.
-// A CTA with W warps puts up to ceil(W / 4) on one SM sub-partition, whose
-// register file holds 16K registers: 25 warps leave 72 per thread, 17 leave 96,
-// 13 leave 128.
-template <int B>
-constexpr int consumers_for() { return B <= 2 ? 24 : (B <= 4 ? 16 : 12); }
+// Consumer warps per CTA: as many as the registers allow (25 warps leave 72
+// registers a thread); they hide the decoder's dependency chains.
+constexpr int kConsumers = 24;
+static_assert(kConsumers <= kMaxLag, "the launch schedule assumes a lag of at most kMaxLag");
 
-template <int CP, int B, bool FAST>
+template <int CP, bool WIDE, bool FAST>
 cudaError_t launch_gemv_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
-  constexpr int NC = consumers_for<B>();
-  static_assert(NC <= kMaxConsumers, "the launch schedule assumes at most kMaxConsumers");
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(gemv_kernel<NC, CP, B, FAST>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(gemv_kernel<kConsumers, CP, WIDE, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  gemv_kernel<NC, CP, B, FAST><<<s.ctas, (NC + 1) * 32, s.smem_bytes, stream>>>(p);
+  gemv_kernel<kConsumers, CP, WIDE, FAST><<<s.ctas, (kConsumers + 1) * 32, s.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
 template <int CP, bool FAST>
 cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
-  switch (p.batch) {
-    case 1: return launch_gemv_t<CP, 1, FAST>(p, s, stream);
-    case 2: return launch_gemv_t<CP, 2, FAST>(p, s, stream);
-    case 3: return launch_gemv_t<CP, 3, FAST>(p, s, stream);
-    case 4: return launch_gemv_t<CP, 4, FAST>(p, s, stream);
-    case 5: return launch_gemv_t<CP, 5, FAST>(p, s, stream);
-    case 6: return launch_gemv_t<CP, 6, FAST>(p, s, stream);
-    case 7: return launch_gemv_t<CP, 7, FAST>(p, s, stream);
-    case 8: return launch_gemv_t<CP, 8, FAST>(p, s, stream);
-    default: return cudaErrorInvalidValue;
-  }
+  if (p.batch < 1 || p.batch > kMaxPassRows) return cudaErrorInvalidValue;
+  return p.batch <= 8 ? launch_gemv_t<CP, false, FAST>(p, s, stream)
+                      : launch_gemv_t<CP, true, FAST>(p, s, stream);
 }
 
 template <int CP, bool FAST>
 cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
-  constexpr int NC = 24;
-  static_assert(NC <= kMaxConsumers, "the launch schedule assumes at most kMaxConsumers");
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(decompress_kernel<NC, CP, FAST>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(decompress_kernel<kConsumers, CP, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  decompress_kernel<NC, CP, FAST><<<s.ctas, (NC + 1) * 32, s.smem_bytes, stream>>>(p);
+  decompress_kernel<kConsumers, CP, FAST><<<s.ctas, (kConsumers + 1) * 32, s.smem_bytes, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -662,8 +789,8 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
   if (ctas > (int64_t)kMaxCtas) ctas = kMaxCtas;
   s.ctas = ctas < 1 ? 1 : (int)ctas;
   s.table_bytes = table_bytes;
-  // table | table barrier | full[kSlots] | empty[kSlots] | ring
-  const size_t head = (size_t)table_bytes + 8 + 2 * kSlots * 8;
+  // table | table barrier | full[kSlots] | empty[kSlots] | x stage | ring
+  const size_t head = (size_t)table_bytes + 8 + 2 * kSlots * 8 + kXStageBytes;
   s.ring_offset = (head + 127) / 128 * 128;
   const int64_t per_cta = (n_tiles + s.ctas - 1) / s.ctas;
   // Tiles per bulk copy: enough for >= 16 KB of typical chunks, between 2 and 8

@@ -7,8 +7,13 @@ namespace nwc {
 
 // Barrier slots per CTA: batches in flight or resident at once are fewer.
 constexpr int kSlots = 64;
-// Most consumer warps any kernel runs; the launch schedule relies on it.
-constexpr int kMaxConsumers = 24;
+// Most tiles a consumer warp's next wait can lie beyond the last tile it
+// released (its warps x tiles decoded at once, over all kernels); the launch
+// schedule relies on it.
+constexpr int kMaxLag = 48;
+
+// Rows of x one GEMV launch handles (one 16-row tensor-core operand).
+constexpr int kMaxPassRows = 16;
 
 // Device error word bits (read and cleared by nwc_get_device_error).
 constexpr uint32_t kErrTimeout = 1u;   // a bounded mbarrier wait gave up
@@ -29,7 +34,7 @@ struct TileParams {
   // GEMV
   const uint16_t* x;        // BF16 [batch x cols]
   float* y;                 // FP32 [batch x rows]
-  int32_t batch;            // rows of x handled by this launch (<= 8)
+  int32_t batch;            // rows of x handled by this launch (<= kMaxPassRows)
   float* partial;           // [tiles_c][batch][rows_pad] split-K partial sums
   uint32_t* counters;       // [tiles_r] arrivals per row tile
   int64_t rows_pad;         // 8 * tiles_r
@@ -57,7 +62,7 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
 // tile-area offset (16-byte units), its bytes, its place in the ring (a batch
 // never wraps; space is reused first in, first out) and how many of the CTA's
 // earlier batches must have been released before it is issued (for room, and
-// to keep fewer than kSlots - ceil(kMaxConsumers / batch_tiles) outstanding).
+// to keep fewer than kSlots - ceil(kMaxLag / batch_tiles) outstanding).
 // `index` holds the tiles + 1 chunk offsets in 16-byte units; `out` receives
 // sched_bytes(n_tiles) bytes laid out as nwc_format.h describes.
 void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s, uint8_t* out);

@@ -108,7 +108,7 @@ nwc::TileParams base_params(const nwc_handle_s& h) {
   return p;
 }
 
-constexpr int kChunkBatch = 8;  // CUDA-core kernel handles up to 8 rows of x per pass
+constexpr int kChunkBatch = nwc::kMaxPassRows;  // rows of x per kernel launch
 
 uint64_t workspace_bytes_for(const nwc_handle_s& h, int32_t batch) {
   if (h.tiles_c <= 1) return 0;

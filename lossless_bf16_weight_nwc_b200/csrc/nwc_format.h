@@ -11,8 +11,10 @@
 // A chunk is raw u8[8 * tile_cols] | lane byte counts u8[32] | stream words.
 // Stream words are little-endian u32 whose bit 31 is the earliest bit; the 32
 // lane streams follow one another, each padded to a byte, the whole run padded
-// to 16 bytes.  Lane t's k-th symbol is the tile element (row (k/2) % 8,
-// column 64 (k/16) + 2t + k%2); its raw byte is at (k/16) * 512 + 16 t + k%16.
+// to 16 bytes.  Lane t = 4g + c owns row g of the tile: its k-th symbol is the
+// element (row g, column 64 (k/16) + 16c + k%16), so a 64-column group gives the
+// lane 16 consecutive columns of its row; the raw byte is at
+// (k/16) * 512 + 16 t + k%16.
 // Tiles are stored column-block-major: u = j * tiles_r + i.
 //
 // Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)]

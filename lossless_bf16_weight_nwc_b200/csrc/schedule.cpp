@@ -23,8 +23,8 @@ void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s
   const int T = s.batch_tiles;
   const uint64_t R = (uint64_t)s.ring_bytes;
   // Outstanding (issued, not yet released) batches stay below kSlots minus the
-  // batches that a consumer warp can run ahead of the slowest one.
-  const int64_t max_outstanding = kSlots - (kMaxConsumers + T - 1) / T;
+  // batches that a consumer warp's next wait can lie beyond its last release.
+  const int64_t max_outstanding = kSlots - (kMaxLag + T - 1) / T;
   std::vector<uint64_t> vstart;  // virtual ring position of each batch of the CTA
   uint32_t g = 0;                // batches of the CTAs before this one
   for (int c = 0; c < s.ctas; ++c) {

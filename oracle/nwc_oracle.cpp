@@ -59,8 +59,9 @@
  *           whole sequence zero-padded to a multiple of 16 bytes and stored as
  *           little-endian 32-bit words in which bit i of the sequence is bit
  *           31 - (i mod 32) of word i / 32.
- *   Lane t's k-th symbol is the tile element at row r = (k / 2) mod 8 and
- *   column 64 * (k / 16) + 2 t + (k mod 2).
+ *   Lane t = 4 g + c (g = t / 4, c = t mod 4) owns row g of the tile: its k-th
+ *   symbol is the element at row g and column 64 * (k / 16) + 16 c + (k mod 16),
+ *   i.e. in every 64-column group the lane's 16 consecutive columns, in order.
  */
 #include "nwc_oracle.h"
 
@@ -94,11 +95,12 @@ uint64_t get_u64(const uint8_t* p) {
 uint64_t round_up(uint64_t v, uint64_t m) { return (v + m - 1) / m * m; }
 
 /* Tile element of lane t's k-th symbol ("NWC", "Fused kernel": each lane owns
- * one bit stream of the block; here a lane owns column pairs 2t, 2t+1 of every
- * 64-column group, all 8 rows). */
+ * one bit stream of the block; which elements it owns is not fixed there).
+ * Here lane t = 4 g + c owns row g and, in every 64-column group, the 16
+ * consecutive columns from 16 c on, taken in order. */
 void lane_symbol_position(int t, int k, int* r, int* c) {
-  *r = (k / 2) % 8;
-  *c = 64 * (k / 16) + 2 * t + (k % 2);
+  *r = t / 4;
+  *c = 64 * (k / 16) + 16 * (t % 4) + (k % 16);
 }
 int raw_position(int t, int k) { return (k / 16) * 512 + 16 * t + (k % 16); }
 

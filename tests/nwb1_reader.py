@@ -69,8 +69,8 @@ def decode(blob: bytes) -> np.ndarray:
                 sym = book[s[p:q]]
                 p = q
                 rb = raw[(k // 16) * 512 + 16 * t + k % 16]
-                r = (k // 2) % 8
-                c = 64 * (k // 16) + 2 * t + k % 2
+                r = t // 4
+                c = 64 * (k // 16) + 16 * (t % 4) + k % 16
                 row, col = i * tr + r, j * tc + c
                 if row < rows and col < cols:
                     out[row, col] = ((rb >> 7) << 15) | (sym << 7) | (rb & 0x7F)

@@ -92,8 +92,10 @@ def test_exact_size_invariant(orc, rows, cols, tile_cols):
             tile = padded[8 * i:8 * i + 8, tile_cols * j:tile_cols * (j + 1)]
             stream = 0
             for t in range(32):
-                cols_t = [64 * g + 2 * t + hh for g in range(tile_cols // 64) for hh in (0, 1)]
-                bits = int(lens[tile[:, cols_t]].sum())
+                # lane t = 4 g + c: row g, columns 64 m + 16 c .. + 15 of each group m
+                cols_t = [64 * m + 16 * (t % 4) + kk for m in range(tile_cols // 64)
+                          for kk in range(16)]
+                bits = int(lens[tile[t // 4, cols_t]].sum())
                 stream += -(-bits // 8)
             area += 8 * tile_cols + 32 + -(-stream // 16) * 16
     tiles_off = -(-(128 + 256 + 4 * (tiles_r * tiles_c + 1)) // 256) * 256

@@ -18,8 +18,9 @@ MUTANTS = [
      "for (size_t q = 0; q < 2 * n - 1; ++q)"),
     ("canonical step loses a bit", "next = (next + 1) << (l - prev_len);",
      "next = (next + 1) << (l > prev_len ? l - prev_len - 1 : 0);"),
-    ("lane owns a strided column", "*c = 64 * (k / 16) + 2 * t + (k % 2);",
-     "*c = 64 * (k / 16) + t + 32 * (k % 2);"),
+    ("lane owns strided columns", "*c = 64 * (k / 16) + 16 * (t % 4) + (k % 16);",
+     "*c = 64 * (k / 16) + 4 * (k % 16) + (t % 4);"),
+    ("lane row from the wrong bits", "*r = t / 4;", "*r = t % 8;"),
     ("raw plane lane-major", "int raw_position(int t, int k) { return (k / 16) * 512 + 16 * t + (k % 16); }",
      "int raw_position(int t, int k) { return (k / 16) * 512 + t + 32 * (k % 16); }"),
     ("filler is least frequent", "if (cnt[s] > cnt[best]) best = s;",

@@ -8,8 +8,9 @@ import pytest
 from lossless_bf16_weight_nwc_b200 import synth
 
 K_SLOTS = 64          # barrier slots per CTA (kernels.cuh)
-K_MAX_CONSUMERS = 24  # most consumer warps of any kernel (kernels.cuh)
+K_MAX_LAG = 48        # tiles a consumer's next wait may lie past its last release (kernels.cuh)
 K_MAX_CTAS = 256
+K_XSTAGE = 8448       # shared memory reserved for the CTA's columns of x (kernels.cu)
 B200_SMS, B200_SMEM = 148, 232448
 
 
@@ -46,7 +47,7 @@ def check_schedule(lib, blob, sms, smem):
     assert 2 <= T <= 8
     assert R % 16 == 0 and info["smem_bytes"] <= smem
     assert cta[0] == 0 and cta[C] == info["batches"] == len(bat)
-    max_out = K_SLOTS - -(-K_MAX_CONSUMERS // T)
+    max_out = K_SLOTS - -(-K_MAX_LAG // T)
     for c in range(C):
         first, last = n_tiles * c // C, n_tiles * (c + 1) // C
         b0, b1 = int(cta[c]), int(cta[c + 1])
@@ -96,8 +97,8 @@ def test_schedule_tight_ring_serialises(lib):
     T = info["batch_tiles"]
     index = index_of(blob)
     max_chunk = int(16 * np.diff(index).max())
-    ring_offset = -(-(16384 + 8 + 2 * K_SLOTS * 8) // 128) * 128
-    smem = ring_offset + T * max_chunk + 16 + 16
+    ring_offset = -(-(16384 + 8 + 2 * K_SLOTS * 8 + K_XSTAGE) // 128) * 128
+    smem = ring_offset + T * max_chunk + 32  # ring of one worst-case batch + read slack
     assert 2 * int(bat[:-1, 1].min()) > T * max_chunk + 16  # the last batch may be short
     info, _, bat, _ = lib.nwc_schedule_describe(blob, 1, smem)
     assert info["ring_bytes"] <= T * max_chunk + 16
