@@ -40,7 +40,8 @@ namespace {
 constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
 constexpr int kRingSlack = 32;                   // lanes may read a few words past a chunk
 constexpr int kTablePieces = 8;                  // bulk copies that bring in the decode table
-constexpr int kXStageBytes = 8448;               // x columns staged per CTA (GEMV)
+constexpr int kXStageBytes = 16640;              // x columns staged per CTA (GEMV)
+constexpr uint64_t kBatchTarget = 8192;          // bytes a bulk copy should move at least
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---- PTX helpers -----------------------------------------------------------
@@ -102,6 +103,15 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
+}
+// Programmatic dependent launch: let the next kernel on the stream start its
+// prologue now (its CTAs become resident as this grid's exit), and wait until
+// the previous kernel has completed and its writes are visible.
+__device__ __forceinline__ void allow_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void wait_prerequisites() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
@@ -345,12 +355,18 @@ struct Smem {
   uint8_t* ring;
 };
 
+// table | table barrier | full[kSlots] | empty[kSlots] | x stage (16-byte
+// aligned) | ring
+__host__ __device__ constexpr size_t xstage_offset(uint32_t table_bytes) {
+  return ((size_t)table_bytes + 8 + 2 * kSlots * 8 + 15) / 16 * 16;
+}
+
 __device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
   Smem s;
   s.table_bar = reinterpret_cast<uint64_t*>(smem + p.table_bytes);
   s.full = s.table_bar + 1;
   s.empty = s.full + kSlots;
-  s.xstage = reinterpret_cast<uint8_t*>(s.empty + kSlots);
+  s.xstage = smem + xstage_offset(p.table_bytes);
   s.ring = smem + p.ring_offset;
   return s;
 }
@@ -516,6 +532,7 @@ __device__ __forceinline__ void cta_range(const TileParams& p, int64_t* first, i
 // false once its work is done.
 template <int NC>
 __device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const Smem& s) {
+  allow_dependents();
   if (threadIdx.x == 0) {
     mbar_init(s.table_bar, 1);
     for (int k = 0; k < kSlots; ++k) {
@@ -581,14 +598,33 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   const int64_t span = (j1 - j0 + 1) * kTileCols;        // columns staged
   const uint32_t xrow = (uint32_t)(span * 2 + 16);       // bytes per row, padded
   const bool xsmem = (uint64_t)batch * xrow <= (uint64_t)kXStageBytes;
+  // x, y and the workspace may belong to the previous kernel on the stream; the
+  // producer only reads the device image, which no kernel writes.
+  wait_prerequisites();
   if (xsmem) {
-    const uint32_t words = (uint32_t)(span / 2), total = (uint32_t)batch * words;
-    for (uint32_t t = threadIdx.x; t < total; t += NC * 32) {
-      const uint32_t b = t / words, w = t - b * words;
-      const int64_t col = j0 * kTileCols + 2 * (int64_t)w;
-      const uint32_t v =
-          col < p.cols ? __ldg(reinterpret_cast<const uint32_t*>(p.x + b * p.cols + col)) : 0u;
-      *reinterpret_cast<uint32_t*>(s.xstage + b * xrow + 4 * w) = v;
+    // 16-byte pieces when rows of x start 16-byte aligned (a piece is then
+    // wholly inside or outside the matrix), else words; two loads in flight
+    // per thread before their stores.
+    if (((reinterpret_cast<uintptr_t>(p.x) & 15) == 0) && (p.cols % 8 == 0)) {
+      const uint32_t pieces = (uint32_t)(span / 8), total = (uint32_t)batch * pieces;
+#pragma unroll 2
+      for (uint32_t t = threadIdx.x; t < total; t += NC * 32) {
+        const uint32_t b = t / pieces, w = t - b * pieces;
+        const int64_t col = j0 * kTileCols + 8 * (int64_t)w;
+        const uint4 v = col < p.cols ? __ldg(reinterpret_cast<const uint4*>(p.x + b * p.cols + col))
+                                     : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(s.xstage + b * xrow + 16 * w) = v;
+      }
+    } else {
+      const uint32_t words = (uint32_t)(span / 2), total = (uint32_t)batch * words;
+#pragma unroll 2
+      for (uint32_t t = threadIdx.x; t < total; t += NC * 32) {
+        const uint32_t b = t / words, w = t - b * words;
+        const int64_t col = j0 * kTileCols + 2 * (int64_t)w;
+        const uint32_t v =
+            col < p.cols ? __ldg(reinterpret_cast<const uint32_t*>(p.x + b * p.cols + col)) : 0u;
+        *reinterpret_cast<uint32_t*>(s.xstage + b * xrow + 4 * w) = v;
+      }
     }
     named_barrier_sync(1, NC * 32);  // consumers only
   }
@@ -677,7 +713,9 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
   int64_t first;
   int n;
   cta_range(p, &first, &n);
-  if (!setup<NC>(p, smem, s) || !wait_table(s)) return;
+  if (!setup<NC>(p, smem, s)) return;
+  wait_prerequisites();  // the output may still be read by the previous kernel
+  if (!wait_table(s)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
@@ -755,13 +793,31 @@ cudaError_t ensure_smem(Kernel k, size_t bytes, int (&configured)[64]) {
 constexpr int kConsumers = 24;
 static_assert(kConsumers <= kMaxLag, "the launch schedule assumes a lag of at most kMaxLag");
 
+// One CTA per SM with programmatic stream serialization: the kernel may start
+// before the previous one on the stream ends; it waits for it (see
+// wait_prerequisites) before it touches anything that kernel could use.
+template <typename Kernel>
+cudaError_t launch_pdl(Kernel k, const LaunchShape& s, cudaStream_t stream, const TileParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)s.ctas);
+  cfg.blockDim = dim3((unsigned)((kConsumers + 1) * 32));
+  cfg.dynamicSmemBytes = s.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, p);
+}
+
+
 template <int CP, bool WIDE, bool FAST>
 cudaError_t launch_gemv_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   static int configured[64] = {};
   cudaError_t e = ensure_smem(gemv_kernel<kConsumers, CP, WIDE, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  gemv_kernel<kConsumers, CP, WIDE, FAST><<<s.ctas, (kConsumers + 1) * 32, s.smem_bytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(gemv_kernel<kConsumers, CP, WIDE, FAST>, s, stream, p);
 }
 
 template <int CP, bool FAST>
@@ -776,8 +832,7 @@ cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaS
   static int configured[64] = {};
   cudaError_t e = ensure_smem(decompress_kernel<kConsumers, CP, FAST>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  decompress_kernel<kConsumers, CP, FAST><<<s.ctas, (kConsumers + 1) * 32, s.smem_bytes, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decompress_kernel<kConsumers, CP, FAST>, s, stream, p);
 }
 
 }  // namespace
@@ -789,13 +844,13 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
   if (ctas > (int64_t)kMaxCtas) ctas = kMaxCtas;
   s.ctas = ctas < 1 ? 1 : (int)ctas;
   s.table_bytes = table_bytes;
-  // table | table barrier | full[kSlots] | empty[kSlots] | x stage | ring
-  const size_t head = (size_t)table_bytes + 8 + 2 * kSlots * 8 + kXStageBytes;
+  const size_t head = xstage_offset(table_bytes) + kXStageBytes;
   s.ring_offset = (head + 127) / 128 * 128;
   const int64_t per_cta = (n_tiles + s.ctas - 1) / s.ctas;
-  // Tiles per bulk copy: enough for >= 16 KB of typical chunks, between 2 and 8
-  // (at least 2 keeps the schedule's batch count within its area).
-  int t = (int)((16384 + typical_chunk - 1) / (typical_chunk ? typical_chunk : 1));
+  // Tiles per bulk copy: enough for kBatchTarget bytes of typical chunks,
+  // between 2 and 8 (at least 2 keeps the schedule's batch count within its
+  // area).
+  int t = (int)((kBatchTarget + typical_chunk - 1) / (typical_chunk ? typical_chunk : 1));
   if (t < 2) t = 2;
   if (t > 8) t = 8;
   s.batch_tiles = t;
