@@ -38,8 +38,11 @@ __device__ unsigned int g_device_error;
 namespace {
 
 constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
-constexpr int kRingSlack = 32;                   // lanes may read a few words past a chunk
+constexpr int kRingSlack = 256;                  // readers may run past a chunk (corrupt data)
 constexpr int kTablePieces = 8;                  // bulk copies that bring in the decode table
+constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
+constexpr uint32_t kPairReadSpan = 12 + 4 * kMaxPairSteps + 4;  // bytes one tile's reader may touch
+static_assert(kPairReadSpan <= kRingSlack, "a clamped reader must stay inside the ring slack");
 constexpr int kXStageBytes = 16640;              // x columns staged per CTA (GEMV)
 constexpr uint64_t kBatchTarget = 8192;          // bytes a bulk copy should move at least
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -236,16 +239,17 @@ __device__ __forceinline__ uint32_t decode_pair(BitReader& br, uint32_t table) {
 // lies on the decoder's dependency chain.
 struct PairReader {
   uint32_t a, b, c;  // stream words base, base + 1, base + 2
-  uint32_t p;        // next unread bit of a (0 = its bit 31)
+  uint32_t p;        // bits 0..4: next unread bit of a (0 = its bit 31); bit 5
+                     // clear between steps; higher bits are don't-care
   uint32_t next;     // shared-window address of word base + 3
 
-  uint32_t last;     // highest word address the reader may touch
-
-  // `limit`: end of the shared memory the reader may read; a corrupt stream
-  // start or length can then misdecode but never read outside it.
+  // A tile takes at most kMaxPairSteps calls of two(), each reading at most one
+  // word past the three it starts with, so the reader never touches more than
+  // kPairReadSpan bytes from its first word; `limit` (the end of the memory it
+  // may read) clamps that first word, so a corrupt stream start or length can
+  // misdecode but never read outside.
   __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
-    last = limit - 4;
-    const uint32_t at = min(area + (start & ~3u), last - 8);
+    const uint32_t at = min(area + (start & ~3u), limit - kPairReadSpan);
     a = lds32(at);
     b = lds32(at + 4);
     c = lds32(at + 8);
@@ -254,19 +258,20 @@ struct PairReader {
   }
   // Entries e0, e1 of the next two steps.
   __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
-    const uint32_t w = __funnelshift_l(b, a, p);  // 32 bits from the next unread one
+    const uint32_t w = __funnelshift_l(b, a, p);  // 32 bits from the next unread one (p & 31)
     e0 = lds32(table + ((w >> 16) & 0xFFFCu));
     const uint32_t w1 = __funnelshift_l(0u, w, e0);  // shift by e0's count (bits 0..3)
     e1 = lds32(table + ((w1 >> 16) & 0xFFFCu));
-    // Bits 0..6 of e0 + e1 are the two counts' sum (bits 4..6 of an entry are
-    // zero), below 29, so q = p + both counts < 61.
-    const uint32_t q = (p + e0 + e1) & 0x7Fu;
-    const uint32_t adv = q & 32u;
+    // Bits 0..6 of an entry are its count (bits 4..6 zero) and higher bits never
+    // carry into them, so bits 0..5 of p + e0 + e1 are the new offset (< 61):
+    // bit 5 says the window passed a word.
+    p += e0 + e1;
+    const uint32_t adv = p & 32u;
+    p ^= adv;
     a = adv ? b : a;
     b = adv ? c : b;
     lds32_keep(c, next, adv);
-    next = min(next + (adv >> 3), last);
-    p = q & 31u;
+    next += adv >> 3;
   }
 };
 
@@ -480,22 +485,19 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
   dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
   const int g = lane >> 2, c = lane & 3;
   const int64_t cols = p.cols;
-  // Rows past the batch read row 0 (a valid address) and are zeroed.
+  // Rows past the batch read row 0 (see x_at).
   const bool has0 = g < p.batch, has1 = WIDE && g + 8 < p.batch;
   const uint16_t* xr0 = p.x + (has0 ? (int64_t)g * cols : 0);
   const uint16_t* xr1 = p.x + (has1 ? (int64_t)(g + 8) * cols : 0);
   const uint32_t xs0 = xs + (has0 ? g * xrow : 0u) + 32u * c;
   const uint32_t xs1 = xs + (has1 ? (g + 8) * xrow : 0u) + 32u * c;
   const bool vec = xvec && col_tile + CP * 64 <= cols;  // whole tile inside and aligned
-  // x of the block at column offset o (from this lane's first column).
+  // x of the block at column offset o (from this lane's first column).  Lanes
+  // of batch rows past the batch read row 0 instead: they only feed rows of D
+  // that are never stored (row g of D depends on row g of A alone).
   auto x_at = [&](const uint16_t* xr, uint32_t xsr, bool has, uint32_t o) -> uint2 {
-    if (XSM) {
-      uint2 v = lds64(xsr + 2 * o);
-      v.x = has ? v.x : 0u;
-      v.y = has ? v.y : 0u;
-      return v;
-    }
-    return load_x4(xr, cols, col_tile + 16 * c + o, has, vec);
+    if (XSM) return lds64(xsr + 2 * o);
+    return load_x4(xr, cols, col_tile + 16 * c + o, true, vec);
   };
   uint2 xa = x_at(xr0, xs0, has0, 0);
   uint2 xb = WIDE ? x_at(xr1, xs1, has1, 0) : make_uint2(0u, 0u);
@@ -788,9 +790,9 @@ cudaError_t ensure_smem(Kernel k, size_t bytes, int (&configured)[64]) {
   return e;
 }
 
-// Consumer warps per CTA: as many as the registers allow (25 warps leave 72
+// Consumer warps per CTA: as many as the registers allow (32 warps leave 64
 // registers a thread); they hide the decoder's dependency chains.
-constexpr int kConsumers = 24;
+constexpr int kConsumers = 31;
 static_assert(kConsumers <= kMaxLag, "the launch schedule assumes a lag of at most kMaxLag");
 
 // One CTA per SM with programmatic stream serialization: the kernel may start
