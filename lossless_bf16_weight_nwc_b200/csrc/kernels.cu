@@ -239,8 +239,8 @@ __device__ __forceinline__ uint32_t decode_pair(BitReader& br, uint32_t table) {
 // lies on the decoder's dependency chain.
 struct PairReader {
   uint32_t a, b, c;  // stream words base, base + 1, base + 2
-  uint32_t p;        // bits 0..4: next unread bit of a (0 = its bit 31); bit 5
-                     // clear between steps; higher bits are don't-care
+  uint32_t p;        // bits 0..4: next unread bit of a (0 = its bit 31); higher
+                     // bits are don't-care
   uint32_t next;     // shared-window address of word base + 3
 
   // A tile takes at most kMaxPairSteps calls of two(), each reading at most one
@@ -259,19 +259,27 @@ struct PairReader {
   // Entries e0, e1 of the next two steps.
   __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
     const uint32_t w = __funnelshift_l(b, a, p);  // 32 bits from the next unread one (p & 31)
-    e0 = lds32(table + ((w >> 16) & 0xFFFCu));
+    e0 = lds32(table + ((w >> 18) << 2));
     const uint32_t w1 = __funnelshift_l(0u, w, e0);  // shift by e0's count (bits 0..3)
-    e1 = lds32(table + ((w1 >> 16) & 0xFFFCu));
+    e1 = lds32(table + ((w1 >> 18) << 2));
     // Bits 0..6 of an entry are its count (bits 4..6 zero) and higher bits never
-    // carry into them, so bits 0..5 of p + e0 + e1 are the new offset (< 61):
-    // bit 5 says the window passed a word.
-    p += e0 + e1;
-    const uint32_t adv = p & 32u;
-    p ^= adv;
-    a = adv ? b : a;
-    b = adv ? c : b;
-    lds32_keep(c, next, adv);
-    next += adv >> 3;
+    // carry into them, so bits 0..4 of p + e0 + e1 are the new offset; the two
+    // counts add less than 32, so the window passed a word exactly when bit 5
+    // flipped.
+    const uint32_t q = p + e0 + e1;
+    const uint32_t adv = (q ^ p) & 32u;
+    p = q;
+    advance(adv);
+  }
+  // When adv is non-zero: a, b, c move on by one word and the word after them
+  // is fetched.  One predicate covers the moves, the load and the address.
+  __device__ __forceinline__ void advance(uint32_t adv) {
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %4, 0;\n\t"
+        "@q mov.b32 %0, %1;\n\t@q mov.b32 %1, %2;\n\t"
+        "@q ld.shared.u32 %2, [%3];\n\t@q add.u32 %3, %3, 4;\n\t}"
+        : "+r"(a), "+r"(b), "+r"(c), "+r"(next)
+        : "r"(adv));
   }
 };
 
