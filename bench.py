@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--no-cublas", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--e2e-mode", default="host-y", choices=["copy", "host-y"],
+                    help="how y reaches the host in the end-to-end leg")
     return ap.parse_args()
 
 
@@ -369,19 +371,25 @@ def main():
         torch.cuda.synchronize()
         barrier(world)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # "copy": x and y move with cudaMemcpyAsync around the call; "host-y": the
+        # kernel stores y straight into the pinned (device-mapped) host buffer.
+        host_y = args.e2e_mode == "host-y"
         with torch.cuda.stream(stream):
             e0.record(stream)
             for i in range(args.e2e_steps):
                 xd.copy_(xh, non_blocking=True)
-                _lib.nwc_gemv(mats[i % copies].handle, xd, y, batch, ws, ws_bytes,
-                              stream.cuda_stream)
-                yh.copy_(y, non_blocking=True)
+                _lib.nwc_gemv(mats[i % copies].handle, xd, yh if host_y else y, batch, ws,
+                              ws_bytes, stream.cuda_stream)
+                if not host_y:
+                    yh.copy_(y, non_blocking=True)
             e1.record(stream)
         stream.synchronize()
         e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.e2e_steps
         e2e = {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                "us_per_call": e2e_ms * 1e3, "h2d_bytes_per_step": int(x_bytes),
-               "d2h_bytes_per_step": int(y_bytes)}
+               "d2h_bytes_per_step": int(y_bytes),
+               "transfers": ("x by cudaMemcpyAsync; y stored by the kernel into pinned host "
+                             "memory" if host_y else "x and y by cudaMemcpyAsync")}
 
     # Uncompressed BF16 cuBLAS GEMV on the same shape and L2 policy, for context.
     cublas = None

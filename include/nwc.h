@@ -162,7 +162,9 @@ nwc_status nwc_gemv_workspace_size(nwc_handle_t handle, int32_t batch,
 
 /* y[b][n] = sum_k W[n][k] * x[b][k], for b < batch, n < rows, k < cols.
  *   d_x: device, BF16 [batch x cols], row-major, 4-byte aligned, cols even.
- *   d_y: device, FP32 [batch x rows], row-major (overwritten, not accumulated).
+ *   d_y: FP32 [batch x rows], row-major (overwritten, not accumulated), in
+ *     device memory or in pinned host memory that the device can address (the
+ *     kernel then stores the result straight into host memory).
  *   batch in [1, 64].
  *   d_workspace: device, >= nwc_gemv_workspace_size bytes, 16-byte aligned,
  *     zero-filled before its first use.  Every completed call leaves the counter
