@@ -40,7 +40,8 @@ KERNEL_SOURCE = os.path.join(ROOT, "lossless_bf16_weight_nwc_b200", "csrc", "ker
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 20000 GEMV calls; 50 tokens for a stack)")
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", default="nwc", choices=["nwc", "reference"])
     ap.add_argument("--workload", default="attn_4096_outliers")
@@ -254,10 +255,215 @@ def run_reference(args) -> None:
     print(json.dumps(line))
 
 
+STACKS = ("qwen3_4b_stack", "llama31_8b_stack")
+
+
+def run_stack(args) -> None:
+    """Per-token sequence of a layer stack: every GEMV of every layer, then the
+    lm_head, captured as one CUDA graph; a step is one token.  Layer weights:
+    layer 0 of the workload, generated once, compressed once and held as two
+    device copies that alternate between layers (a layer is larger than L2, so
+    every read is cold); the lm_head is its first rows repeated (synth)."""
+    import torch
+
+    from lossless_bf16_weight_nwc_b200 import _lib, synth
+    rank, world = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl, layer0, head, n_layers = synth.stack_parts(args.workload)
+    batch = args.batch
+    steps = args.steps if args.steps is not None else 50
+    specs = layer0 + [head]
+    host_w = {}
+    comp = {}
+    for sp in specs:
+        host_w[sp.name] = synth.head_matrix(sp, wl.seed) if sp is head else synth.matrix(sp, wl.seed)
+        comp[sp.name] = _lib.CompressedMatrix.compress(host_w[sp.name], device=dev)
+    sets = [{sp.name: comp[sp.name] for sp in layer0}]
+    second = {}
+    for sp in layer0:
+        m0 = comp[sp.name]
+        m = _lib.CompressedMatrix(m0.image.clone(), None, sp.rows, sp.cols, m0.blob_bytes)
+        m.handle = _lib.nwc_handle_from_device(m.image, m.image.numel())
+        second[sp.name] = m
+    sets.append(second)
+    xs = {k: torch.from_numpy(synth.activations(wl.seed, batch, k).view(np.int16))
+          .view(torch.bfloat16).to(dev) for k in {sp.cols for sp in specs}}
+    ys = {n: torch.empty((batch, n), dtype=torch.float32, device=dev) for n in {sp.rows for sp in specs}}
+    wss = {}
+    for sp in specs:
+        nb = _lib.nwc_gemv_workspace_size(comp[sp.name].handle, batch)
+        wss[sp.name] = (torch.zeros(max(nb, 16), dtype=torch.uint8, device=dev), nb)
+    stream = torch.cuda.Stream(device=dev)
+    seq = [(sets[l % 2][sp.name], sp) for l in range(n_layers) for sp in layer0] + [(comp[head.name], head)]
+    launches = len(seq) * ((batch + 15) // 16)
+
+    def token(y_head=None):
+        for m, sp in seq:
+            ws, nb = wss[sp.name]
+            yt = y_head if (sp is head and y_head is not None) else ys[sp.rows]
+            _lib.nwc_gemv(m.handle, xs[sp.cols], yt, batch, ws, nb, stream.cuda_stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            token()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        token()
+    warm = max(args.warmup, 3)
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(steps):
+                g.replay()
+            t1.record(stream)
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms_per_token = max_over_ranks(t0.elapsed_time(t1), world) / steps
+
+    # Parity spot check: the lm_head and the first down projection, sampled rows.
+    parity_ok = True
+    if rank == 0:
+        import oracle
+        for sp in (head, layer0[-1]):
+            xh = synth.activations(wl.seed, batch, sp.cols)
+            comp[sp.name].gemv(torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).to(dev),
+                               y=ys[sp.rows])
+            idx = np.unique(np.linspace(0, sp.rows - 1, 256).astype(np.int64))
+            ref = oracle.gemv(host_w[sp.name][idx], xh)
+            got = ys[sp.rows].double().cpu().numpy()[:, idx]
+            wf = synth.bf16_bits_to_float(host_w[sp.name][idx]).astype(np.float64)
+            xf = synth.bf16_bits_to_float(xh).astype(np.float64)
+            bound = 1e-2 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1)) * 2.0 ** -8
+            parity_ok = parity_ok and bool((np.abs(got - ref) <= bound).all())
+
+    weight_bytes = sum(2.0 * sp.rows * sp.cols for _, sp in seq)
+    comp_bytes = sum(float(m.device_bytes) for m, _ in seq)
+    x_bytes = sum(2.0 * batch * sp.cols for _, sp in seq)
+    y_bytes = sum(4.0 * batch * sp.rows for _, sp in seq)
+    peaks, peak_src = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    alg = comp_bytes + x_bytes + y_bytes
+    achieved = alg / (ms_per_token * 1e-3) / 1e9
+
+    # End to end: the hidden-state x copied in from pinned memory and the logits
+    # stored by the lm_head kernel into pinned host memory, every token.
+    e2e = None
+    if args.e2e_steps > 0:
+        xh_pin = torch.from_numpy(synth.activations(wl.seed, batch, layer0[0].cols).view(np.int16)) \
+            .view(torch.bfloat16).pin_memory()
+        logits = torch.empty((batch, head.rows), dtype=torch.float32).pin_memory()
+        ge = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(ge, stream=stream):
+            xs[layer0[0].cols].copy_(xh_pin, non_blocking=True)
+            token(y_head=logits)
+        n_e2e = min(args.e2e_steps, steps)
+        with torch.cuda.stream(stream):
+            ge.replay()
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(n_e2e):
+                ge.replay()
+            e1.record(stream)
+        stream.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / n_e2e
+        e2e = {"value": world * weight_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "us_per_token": e2e_ms * 1e3,
+               "h2d_bytes_per_step": int(2 * batch * layer0[0].cols),
+               "d2h_bytes_per_step": int(4 * batch * head.rows),
+               "transfers": "hidden state by a captured copy from pinned memory; logits stored "
+                            "by the lm_head kernel into pinned host memory"}
+        del ge
+
+    cublas = None
+    if not args.no_cublas:
+        wts = {sp.name: torch.from_numpy(host_w[sp.name].view(np.int16)).view(torch.bfloat16).to(dev)
+               for sp in specs}
+        wts2 = {sp.name: wts[sp.name].clone() for sp in layer0}
+        xb = {k: v for k, v in xs.items()}
+        yb = {n: torch.empty((batch, n), dtype=torch.bfloat16, device=dev) for n in ys}
+        dense = [((wts if l % 2 == 0 else wts2)[sp.name], sp) for l in range(n_layers) for sp in layer0]
+        dense.append((wts[head.name], head))
+        with torch.cuda.stream(stream):
+            for wt, sp in dense:
+                torch.matmul(xb[sp.cols], wt.t(), out=yb[sp.rows])
+        stream.synchronize()
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb, stream=stream):
+            for wt, sp in dense:
+                torch.matmul(xb[sp.cols], wt.t(), out=yb[sp.rows])
+        reps = max(3, min(steps, 50))
+        c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gb.replay()
+            c0.record(stream)
+            for _ in range(reps):
+                gb.replay()
+            c1.record(stream)
+        stream.synchronize()
+        cb_ms = c0.elapsed_time(c1) / reps
+        cublas = {"us_per_token": cb_ms * 1e3, "effective_gbs": weight_bytes / (cb_ms * 1e-3) / 1e9,
+                  "speedup_nwc_vs_cublas": cb_ms / ms_per_token}
+        del gb, wts, wts2
+
+    line = {
+        "metric": METRIC, "value": replica_value(weight_bytes, world, ms_per_token), "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": ms_per_token,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "batch": batch, "step": f"one token: {len(seq)} GEMVs "
+                   f"({n_layers} layers x {len(layer0)} + lm_head), one CUDA graph",
+                   "weights": "layer 0 generated, two device copies alternating over the layers; "
+                              f"lm_head = its first {synth.HEAD_BLOCK_ROWS} rows repeated",
+                   "l2": "inputs larger than L2: every layer is larger than L2",
+                   "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
+        "us_per_token": ms_per_token * 1e3,
+        "tokens_per_s": 1e3 / ms_per_token,
+        "compression_ratio": weight_bytes / comp_bytes,
+        "compressed_bytes_per_token": comp_bytes,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs (copy)", "kernel": "gemv_kernel",
+                     "basis": "algorithmic bytes of the token's GEMVs / graph time per token",
+                     "tokens_per_s_ceiling_at_peak": hbm * 1e9 / alg},
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "gpu_launches": steps * launches,
+        "parity_spot_check": parity_ok,
+        "cublas_bf16": cublas,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.workload, batch)
+        line["cpu_baseline"].pop("us_per_call", None)
+    if rank == 0:
+        print(json.dumps(line))
+    del g
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     args = parse_args()
+    if args.steps is None and args.workload not in STACKS:
+        args.steps = 20000
     if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 50
         run_reference(args)
+        return
+    if args.workload in STACKS:
+        run_stack(args)
         return
     import torch
 

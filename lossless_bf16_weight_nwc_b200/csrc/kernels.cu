@@ -43,7 +43,7 @@ constexpr int kTablePieces = 8;                  // bulk copies that bring in th
 constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
 constexpr uint32_t kPairReadSpan = 12 + 4 * kMaxPairSteps + 4;  // bytes one tile's reader may touch
 static_assert(kPairReadSpan <= kRingSlack, "a clamped reader must stay inside the ring slack");
-constexpr int kXStageBytes = 16640;              // x columns staged per CTA (GEMV)
+constexpr int kXStageBytes = 33024;              // x columns staged per CTA (GEMV): 16 rows x 2 column blocks
 constexpr uint64_t kBatchTarget = 8192;          // bytes a bulk copy should move at least
 constexpr unsigned kFull = 0xFFFFFFFFu;
 

@@ -207,5 +207,28 @@ def workload(name: str) -> Workload:
     raise KeyError(name)
 
 
+# The stacks' per-token sequences reuse one generated layer for every layer
+# (a layer of either stack is larger than B200's L2, so each is read cold), and
+# build the lm_head from its first HEAD_BLOCK_ROWS rows repeated down the
+# matrix: full shapes at a fraction of the generation time.
+HEAD_BLOCK_ROWS = 16384
+
+
+def stack_parts(name: str):
+    """(workload, the 7 matrices of layer 0, the lm_head spec, number of layers)."""
+    wl = workload(name)
+    layer0 = [m for m in wl.matrices if m.name.startswith("layers.0.")]
+    head = [m for m in wl.matrices if m.name == "lm_head"][0]
+    layers = len({m.name.split(".")[1] for m in wl.matrices if m.name.startswith("layers.")})
+    return wl, layer0, head, layers
+
+
+def head_matrix(spec: MatrixSpec, seed: int) -> np.ndarray:
+    """The lm_head as its first HEAD_BLOCK_ROWS generated rows, repeated."""
+    block = matrix(spec, seed, 0, min(HEAD_BLOCK_ROWS, spec.rows))
+    reps = -(-spec.rows // block.shape[0])
+    return np.ascontiguousarray(np.tile(block, (reps, 1))[:spec.rows])
+
+
 WORKLOADS = ("single_1024", "attn_4096_outliers", "mlp_pair_t5", "qwen3_4b_stack",
              "llama31_8b_stack")

@@ -153,6 +153,21 @@ def test_gemv_deterministic_and_workspace_reuse(lib, orc):
     no_device_error(lib)
 
 
+def test_gemv_into_pinned_host_memory(lib, orc):
+    """y may be pinned host memory the device can address: the kernel stores the
+    result there directly."""
+    spec = synth.MatrixSpec("w", 1000, 2048, "normal", 0.02, 0)
+    w = synth.matrix(spec, 5)
+    x = synth.activations(5, 3, spec.cols)
+    m = lib.CompressedMatrix.compress(w)
+    yh = torch.full((3, spec.rows), float("nan"), dtype=torch.float32).pin_memory()
+    ws, nb = m.workspace(3)
+    lib.nwc_gemv(m.handle, to_bf16(x), yh, 3, ws, nb)
+    torch.cuda.synchronize()
+    tolerance_check(yh.numpy(), orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
 def test_handle_from_device_image(lib, orc):
     spec = synth.MatrixSpec("w", 96, 1536, "normal", 0.02, 0)
     w = synth.matrix(spec, 2)

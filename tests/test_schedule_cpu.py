@@ -10,7 +10,7 @@ from lossless_bf16_weight_nwc_b200 import synth
 K_SLOTS = 64          # barrier slots per CTA (kernels.cuh)
 K_MAX_LAG = 48        # tiles a consumer's next wait may lie past its last release (kernels.cuh)
 K_MAX_CTAS = 256
-K_XSTAGE = 16640      # shared memory reserved for the CTA's columns of x (kernels.cu)
+K_XSTAGE = 33024      # shared memory reserved for the CTA's columns of x (kernels.cu)
 K_RING_SLACK = 256    # shared memory after the ring that readers may touch (kernels.cu)
 B200_SMS, B200_SMEM = 148, 232448
 
