@@ -94,9 +94,9 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols,
 /* Exact sizes for a plan.  *device_bytes is what nwc_compress needs in device
  * memory, the "device image": the serialisable blob, then at 256-byte aligned
  * offsets a derived decode table (64 KiB for lmax <= 7, else 16 KiB) and the
- * launch schedule (about 12 bytes per tile plus 5 KiB: which bytes each bulk
- * copy of the kernels moves and where they land in shared memory, worked out
- * on the host for the device that runs them).  *host_blob_bytes is the size of
+ * launch schedules (two of about 12 bytes per tile plus 5 KiB each: which
+ * bytes each bulk copy of the kernels moves and where they land in shared
+ * memory, worked out on the host for the device that runs them).  *host_blob_bytes is the size of
  * the serialisable blob (nwc_compress_host).  Either pointer may be NULL. */
 nwc_status nwc_plan_size(nwc_plan_t plan, uint64_t* device_bytes,
                          uint64_t* host_blob_bytes);
@@ -144,8 +144,8 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
 
 /* nwc_decompress, nwc_gemv and nwc_gemv_noalloc launch one persistent CTA per
  * SM (at most 256).  Should the current device's launch shape differ from the
- * one the image's schedule was written for, the call first rewrites the
- * schedule area on `stream` (a host-to-device copy, in stream order). */
+ * one the image's schedule was written for, the call first rewrites that
+ * schedule on `stream` (a host-to-device copy, in stream order). */
 
 /* Bit-exact decompression ("NWC", "How it works > Dequantization and embedding
  * lookup": the same decoder writes BF16).  d_w_out: device, rows x cols BF16,
@@ -212,7 +212,11 @@ nwc_status nwc_gemv_noalloc(nwc_handle_t handle, const uint16_t* d_x, float* d_y
 
 /* Launch shape and schedule the kernels would use for a blob on a device with
  * sm_count SMs and smem_limit bytes of opt-in shared memory per block (B200:
- * 148 and 232448).  Host only; touches no GPU.
+ * 148 and 232448), for a launch handling rows_of_x rows of x (0 for
+ * decompression; nwc_gemv launches one kernel per 16 rows).  Launches of up to
+ * 4 rows reserve 8,448 bytes of shared memory for x, larger ones 33,024, so
+ * the two classes have different rings and schedules.  Host only; touches no
+ * GPU.
  *   info: set struct_size = sizeof(nwc_schedule_info).
  *   cta_batch (optional, ctas + 1 entries): first batch of each CTA, and the
  *     total number of batches at the end.  CTA c owns tiles
@@ -225,16 +229,18 @@ nwc_status nwc_gemv_noalloc(nwc_handle_t handle, const uint16_t* d_x, float* d_y
  * Errors: INVALID_ARG, CORRUPT, UNSUPPORTED (shared memory too small). */
 typedef struct {
   uint32_t struct_size;
-  int32_t ctas;        /* persistent CTAs                                  */
-  int32_t batch_tiles; /* consecutive tiles per bulk copy                  */
-  int32_t ring_bytes;  /* staging ring in shared memory, per CTA           */
-  int64_t tiles;       /* tiles of the matrix                              */
-  int64_t batches;     /* bulk copies over all CTAs                        */
-  uint64_t smem_bytes; /* dynamic shared memory per CTA                    */
+  int32_t ctas;          /* persistent CTAs                                  */
+  int32_t batch_tiles;   /* consecutive tiles per bulk copy                  */
+  int32_t ring_bytes;    /* staging ring in shared memory, per CTA           */
+  int64_t tiles;         /* tiles of the matrix                              */
+  int64_t batches;       /* bulk copies over all CTAs                        */
+  uint64_t smem_bytes;   /* dynamic shared memory per CTA                    */
+  uint32_t xstage_bytes; /* shared memory reserved for x, per CTA            */
 } nwc_schedule_info;
 nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
-                                 uint64_t smem_limit, nwc_schedule_info* info,
-                                 uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring);
+                                 uint64_t smem_limit, int32_t rows_of_x,
+                                 nwc_schedule_info* info, uint32_t* cta_batch,
+                                 uint32_t* batch, uint32_t* tile_ring);
 
 /* Any pointer may be NULL.  *blob_bytes is the serialisable part; *device_bytes
  * is the whole device image (blob + decode table + launch schedule). */

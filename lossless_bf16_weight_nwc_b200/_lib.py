@@ -33,7 +33,7 @@ class nwc_schedule_info(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("ctas", ctypes.c_int32),
                 ("batch_tiles", ctypes.c_int32), ("ring_bytes", ctypes.c_int32),
                 ("tiles", ctypes.c_int64), ("batches", ctypes.c_int64),
-                ("smem_bytes", ctypes.c_uint64)]
+                ("smem_bytes", ctypes.c_uint64), ("xstage_bytes", ctypes.c_uint32)]
 
 
 class nwc_opts(ctypes.Structure):
@@ -66,7 +66,8 @@ def _load() -> ctypes.CDLL:
         "nwc_handle_info": ([vp, c.POINTER(i64), c.POINTER(i64), c.POINTER(u64),
                              c.POINTER(u64)], c.c_int),
         "nwc_get_device_error": ([vp, c.POINTER(c.c_uint32)], c.c_int),
-        "nwc_schedule_describe": ([vp, u64, i32, u64, c.POINTER(nwc_schedule_info), vp, vp, vp],
+        "nwc_schedule_describe": ([vp, u64, i32, u64, i32, c.POINTER(nwc_schedule_info), vp, vp,
+                                   vp],
                                   c.c_int),
         "nwc_plan_destroy": ([vp], None),
         "nwc_handle_destroy": ([vp], None),
@@ -205,19 +206,20 @@ def nwc_get_device_error(stream=None) -> tuple[int, int]:
     return st, w.value
 
 
-def nwc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int = 232448):
-    """Launch shape and schedule for a blob on a device of the given size (host
-    only).  Returns (info dict, cta_batch [ctas + 1], batch [batches x 4],
-    tile_ring [tiles])."""
+def nwc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int = 232448,
+                          rows_of_x: int = 1):
+    """Launch shape and schedule for a blob on a device of the given size, for a
+    launch with rows_of_x rows of x (0: decompression); host only.  Returns
+    (info dict, cta_batch [ctas + 1], batch [batches x 4], tile_ring [tiles])."""
     blob = np.ascontiguousarray(blob, dtype=np.uint8)
     info = nwc_schedule_info(struct_size=ctypes.sizeof(nwc_schedule_info))
-    _check(LIB.nwc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit,
+    _check(LIB.nwc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit, rows_of_x,
                                      ctypes.byref(info), None, None, None),
            "nwc_schedule_describe")
     cta = np.zeros(info.ctas + 1, dtype=np.uint32)
     bat = np.zeros((info.batches, 4), dtype=np.uint32)
     ring = np.zeros(info.tiles, dtype=np.uint32)
-    _check(LIB.nwc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit,
+    _check(LIB.nwc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit, rows_of_x,
                                      ctypes.byref(info), cta.ctypes.data, bat.ctypes.data,
                                      ring.ctypes.data), "nwc_schedule_describe")
     d = {k: getattr(info, k) for k, _ in nwc_schedule_info._fields_ if k != "struct_size"}

@@ -43,7 +43,6 @@ constexpr int kTablePieces = 8;                  // bulk copies that bring in th
 constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
 constexpr uint32_t kPairReadSpan = 12 + 4 * kMaxPairSteps + 4;  // bytes one tile's reader may touch
 static_assert(kPairReadSpan <= kRingSlack, "a clamped reader must stay inside the ring slack");
-constexpr int kXStageBytes = 33024;              // x columns staged per CTA (GEMV): 16 rows x 2 column blocks
 constexpr uint64_t kBatchTarget = 8192;          // bytes a bulk copy should move at least
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -364,7 +363,7 @@ struct Smem {
   uint64_t* table_bar;
   uint64_t* full;    // per batch slot: bytes landed
   uint64_t* empty;   // per batch slot: tiles released
-  uint8_t* xstage;   // kXStageBytes: the CTA's columns of x (GEMV)
+  uint8_t* xstage;   // p.xstage_bytes: the CTA's columns of x (GEMV)
   uint8_t* ring;
 };
 
@@ -451,13 +450,12 @@ __device__ __forceinline__ bool wait_batch(const Smem& s, int k) {
   return __all_sync(kFull, wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1)));
 }
 
-// Four BF16 values x[col .. col + 3] of one row of x as two words, or zeros
-// where the row is absent or the columns lie past `cols` (cols is even, so a
-// word is wholly inside or outside).  Every lane loads from a valid address
-// and selects afterwards, so lanes never diverge.  vec (uniform): 8-byte
-// aligned and inside.
+// Four BF16 values x[col .. col + 3] of one row of x as two words, zeros where
+// the columns lie past `cols` (cols is even, so a word is wholly inside or
+// outside).  Every lane loads from a valid address and selects afterwards, so
+// lanes never diverge.  vec (uniform): 8-byte aligned and inside.
 __device__ __forceinline__ uint2 load_x4(const uint16_t* xrow, int64_t cols, int64_t col,
-                                         bool present, bool vec) {
+                                         bool vec) {
   uint2 v;
   if (vec) {
     v = __ldg(reinterpret_cast<const uint2*>(xrow + col));
@@ -468,8 +466,6 @@ __device__ __forceinline__ uint2 load_x4(const uint16_t* xrow, int64_t cols, int
     v.x = in0 ? v.x : 0u;
     v.y = in1 ? v.y : 0u;
   }
-  v.x = present ? v.x : 0u;
-  v.y = present ? v.y : 0u;
   return v;
 }
 
@@ -503,12 +499,12 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
   // x of the block at column offset o (from this lane's first column).  Lanes
   // of batch rows past the batch read row 0 instead: they only feed rows of D
   // that are never stored (row g of D depends on row g of A alone).
-  auto x_at = [&](const uint16_t* xr, uint32_t xsr, bool has, uint32_t o) -> uint2 {
+  auto x_at = [&](const uint16_t* xr, uint32_t xsr, uint32_t o) -> uint2 {
     if (XSM) return lds64(xsr + 2 * o);
-    return load_x4(xr, cols, col_tile + 16 * c + o, true, vec);
+    return load_x4(xr, cols, col_tile + 16 * c + o, vec);
   };
-  uint2 xa = x_at(xr0, xs0, has0, 0);
-  uint2 xb = WIDE ? x_at(xr1, xs1, has1, 0) : make_uint2(0u, 0u);
+  uint2 xa = x_at(xr0, xs0, 0);
+  uint2 xb = WIDE ? x_at(xr1, xs1, 0) : make_uint2(0u, 0u);
 #pragma unroll 1
   for (int m = 0; m < CP; ++m) {
     const uint4 rv = lds128(chunk + m * 512 + lane * 16);
@@ -518,8 +514,8 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
       // Next block's x: + 4 columns, or the next group's first block.
       const uint32_t no = s < 3 ? 64 * m + 4 * (s + 1) : 64 * (m + 1);
       if (s < 3 || m + 1 < CP) {
-        xa = x_at(xr0, xs0, has0, no);
-        if (WIDE) xb = x_at(xr1, xs1, has1, no);
+        xa = x_at(xr0, xs0, no);
+        if (WIDE) xb = x_at(xr1, xs1, no);
       }
       uint32_t e0, e1;
       dec.two(table, e0, e1);
@@ -607,7 +603,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   const int64_t j0 = first / p.tiles_r, j1 = (first + n - 1) / p.tiles_r;
   const int64_t span = (j1 - j0 + 1) * kTileCols;        // columns staged
   const uint32_t xrow = (uint32_t)(span * 2 + 16);       // bytes per row, padded
-  const bool xsmem = (uint64_t)batch * xrow <= (uint64_t)kXStageBytes;
+  const bool xsmem = (uint64_t)batch * xrow <= (uint64_t)p.xstage_bytes;
   // x, y and the workspace may belong to the previous kernel on the stream; the
   // producer only reads the device image, which no kernel writes.
   wait_prerequisites();
@@ -848,13 +844,15 @@ cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaS
 }  // namespace
 
 LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_chunk,
-                         uint32_t table_bytes, int sm_count, size_t smem_limit) {
+                         uint32_t table_bytes, int sm_count, size_t smem_limit,
+                         uint32_t xstage_bytes) {
   LaunchShape s;
+  s.xstage_bytes = xstage_bytes;
   int64_t ctas = n_tiles < sm_count ? n_tiles : sm_count;
   if (ctas > (int64_t)kMaxCtas) ctas = kMaxCtas;
   s.ctas = ctas < 1 ? 1 : (int)ctas;
   s.table_bytes = table_bytes;
-  const size_t head = xstage_offset(table_bytes) + kXStageBytes;
+  const size_t head = xstage_offset(table_bytes) + xstage_bytes;
   s.ring_offset = (head + 127) / 128 * 128;
   const int64_t per_cta = (n_tiles + s.ctas - 1) / s.ctas;
   // Tiles per bulk copy: enough for kBatchTarget bytes of typical chunks,

@@ -31,6 +31,7 @@ struct TileParams {
   int64_t tiles_r, tiles_c, n_tiles;
   int32_t ring_bytes;       // CTA staging ring in shared memory
   int32_t batch_tiles;      // consecutive tiles moved by one bulk copy
+  uint32_t xstage_bytes;    // shared memory reserved for x (GEMV)
   // GEMV
   const uint16_t* x;        // BF16 [batch x cols]
   float* y;                 // FP32 [batch x rows]
@@ -42,9 +43,17 @@ struct TileParams {
   uint16_t* out;            // BF16 [rows x cols]
 };
 
+// Shared memory that a CTA reserves for its columns of x, by x-stage class:
+// 4 rows (class 0: decompression and GEMV launches of up to 4 rows) or 16 rows
+// (class 1), over two column blocks of 512.  A smaller stage leaves a larger
+// ring.
+constexpr uint32_t kXStageBytes[2] = {8448, 33024};
+inline int stage_class(int rows_of_x) { return rows_of_x <= 4 ? 0 : 1; }
+
 struct LaunchShape {
   int ctas;             // one persistent CTA per SM (fewer for small matrices)
   uint32_t table_bytes;
+  uint32_t xstage_bytes;  // x stage reserved after the barriers
   size_t ring_offset;
   int ring_bytes;
   int batch_tiles;
@@ -55,7 +64,8 @@ struct LaunchShape {
 // max_chunk bytes (typical_chunk on average), within the device's per-block
 // shared-memory limit.
 LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_chunk,
-                         uint32_t table_bytes, int sm_count, size_t smem_limit);
+                         uint32_t table_bytes, int sm_count, size_t smem_limit,
+                         uint32_t xstage_bytes);
 
 // Launch schedule for one shape (host): for every CTA (tiles [n c / C,
 // n (c + 1) / C)) its batches of batch_tiles consecutive tiles, each with its
@@ -64,7 +74,7 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
 // earlier batches must have been released before it is issued (for room, and
 // to keep fewer than kSlots - ceil(kMaxLag / batch_tiles) outstanding).
 // `index` holds the tiles + 1 chunk offsets in 16-byte units; `out` receives
-// sched_bytes(n_tiles) bytes laid out as nwc_format.h describes.
+// sched_class_bytes(n_tiles) bytes (one class) laid out as nwc_format.h describes.
 void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s, uint8_t* out);
 
 // fast: lmax <= 7 (14-bit peek, two codes per entry always).

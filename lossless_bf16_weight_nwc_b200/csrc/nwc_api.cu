@@ -45,55 +45,65 @@ nwc_status current_device(int* dev, int* sms, size_t* smem) {
   return NWC_OK;
 }
 
-// Launch geometry for a handle on a device with `sms` SMs and `smem` bytes of
-// opt-in shared memory per block.
-nwc_status shape_on(const nwc_handle_s& h, int sms, size_t smem, nwc::LaunchShape* s) {
+// Launch geometry for a handle and x-stage class on a device with `sms` SMs
+// and `smem` bytes of opt-in shared memory per block.
+nwc_status shape_on(const nwc_handle_s& h, int sms, size_t smem, int cls, nwc::LaunchShape* s) {
   const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
-  *s = nwc::launch_shape(h.tiles, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms, smem);
+  *s = nwc::launch_shape(h.tiles, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms, smem,
+                         nwc::kXStageBytes[cls]);
   if (s->smem_bytes > smem) return NWC_ERR_UNSUPPORTED;
   return NWC_OK;
 }
 
-bool same_shape(const nwc_handle_s& h, const nwc::LaunchShape& s) {
-  return h.sched_ctas == s.ctas && h.sched_ring == s.ring_bytes &&
-         h.sched_tiles_per_batch == s.batch_tiles;
+bool same_shape(const nwc_handle_s& h, int cls, const nwc::LaunchShape& s) {
+  return h.sched_ctas[cls] == s.ctas && h.sched_ring[cls] == s.ring_bytes &&
+         h.sched_tiles_per_batch[cls] == s.batch_tiles;
 }
 
-// Writes the launch schedule for shape `s` into the device image on `stream`
-// (from pageable memory: the call returns once the bytes are staged).
-nwc_status write_schedule(nwc_handle_s* h, const nwc::LaunchShape& s, cudaStream_t stream) {
-  std::vector<uint8_t> sched(nwc::sched_bytes((uint64_t)h->tiles));
+void note_schedule(nwc_handle_s* h, int cls, const nwc::LaunchShape& s) {
+  h->sched_ctas[cls] = s.ctas;
+  h->sched_ring[cls] = s.ring_bytes;
+  h->sched_tiles_per_batch[cls] = s.batch_tiles;
+}
+
+uint64_t class_off(const nwc_handle_s& h, int cls) {
+  return h.sched_off + (uint64_t)cls * nwc::sched_class_bytes((uint64_t)h.tiles);
+}
+
+// Writes class cls's launch schedule for shape `s` into the device image on
+// `stream` (from pageable memory: the call returns once the bytes are staged).
+nwc_status write_schedule(nwc_handle_s* h, int cls, const nwc::LaunchShape& s,
+                          cudaStream_t stream) {
+  std::vector<uint8_t> sched(nwc::sched_class_bytes((uint64_t)h->tiles));
   nwc::build_schedule(h->index.data(), h->tiles, s, sched.data());
-  if (cudaMemcpyAsync(h->d_base + h->sched_off, sched.data(), sched.size(),
+  if (cudaMemcpyAsync(h->d_base + class_off(*h, cls), sched.data(), sched.size(),
                       cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return NWC_ERR_CUDA;
-  h->sched_ctas = s.ctas;
-  h->sched_ring = s.ring_bytes;
-  h->sched_tiles_per_batch = s.batch_tiles;
+  note_schedule(h, cls, s);
   return NWC_OK;
 }
 
-// Launch geometry on the current device; rewrites the image's schedule (in
-// stream order) when it was made for another shape.
-nwc_status shape_for(nwc_handle_s* h, nwc::LaunchShape* s, cudaStream_t stream) {
+// Launch geometry of class cls on the current device; rewrites that class's
+// schedule (in stream order) when it was made for another shape.
+nwc_status shape_for(nwc_handle_s* h, int cls, nwc::LaunchShape* s, cudaStream_t stream) {
   int dev, sms;
   size_t smem;
   nwc_status st = current_device(&dev, &sms, &smem);
   if (st != NWC_OK) return st;
-  st = shape_on(*h, sms, smem, s);
+  st = shape_on(*h, sms, smem, cls, s);
   if (st != NWC_OK) return st;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!same_shape(*h, *s)) st = write_schedule(h, *s, stream);
+  if (!same_shape(*h, cls, *s)) st = write_schedule(h, cls, *s, stream);
   return st;
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-nwc::TileParams base_params(const nwc_handle_s& h) {
+nwc::TileParams base_params(const nwc_handle_s& h, int cls, const nwc::LaunchShape& s) {
   nwc::TileParams p;
   std::memset(&p, 0, sizeof(p));
   p.tiles = h.d_base + h.tiles_off;
-  const uint8_t* sched = h.d_base + h.sched_off;
+  const uint8_t* sched = h.d_base + class_off(h, cls);
   p.sched_cta = reinterpret_cast<const uint32_t*>(sched);
   p.sched_batch = reinterpret_cast<const uint4*>(sched + nwc::sched_batch_off());
   p.tile_ring = reinterpret_cast<const uint32_t*>(sched + nwc::sched_tile_off((uint64_t)h.tiles));
@@ -105,6 +115,10 @@ nwc::TileParams base_params(const nwc_handle_s& h) {
   p.tiles_c = h.tiles_c;
   p.n_tiles = h.tiles;
   p.rows_pad = 8 * h.tiles_r;
+  p.ring_offset = (uint32_t)s.ring_offset;
+  p.ring_bytes = s.ring_bytes;
+  p.batch_tiles = s.batch_tiles;
+  p.xstage_bytes = s.xstage_bytes;
   return p;
 }
 
@@ -131,22 +145,26 @@ nwc_status make_handle(const uint8_t* blob_host_header_region, uint64_t bytes, v
   return NWC_OK;
 }
 
-// Geometry and schedule of a new handle on the current device: writes the
-// schedule into `image` (a host copy of the device image) when given, else
+// Geometry and schedules of a new handle on the current device: writes the
+// schedules into `image` (a host copy of the device image) when given, else
 // into the device image on `stream`.
 nwc_status init_schedule(nwc_handle_s* h, uint8_t* image, cudaStream_t stream) {
   int dev, sms;
   size_t smem;
   nwc_status st = current_device(&dev, &sms, &smem);
   if (st != NWC_OK) return st;
-  nwc::LaunchShape s;
-  st = shape_on(*h, sms, smem, &s);
-  if (st != NWC_OK) return st;
-  if (!image) return write_schedule(h, s, stream);
-  nwc::build_schedule(h->index.data(), h->tiles, s, image + h->sched_off);
-  h->sched_ctas = s.ctas;
-  h->sched_ring = s.ring_bytes;
-  h->sched_tiles_per_batch = s.batch_tiles;
+  for (int cls = 0; cls < nwc::kStageClasses; ++cls) {
+    nwc::LaunchShape s;
+    st = shape_on(*h, sms, smem, cls, &s);
+    if (st != NWC_OK) return st;
+    if (!image) {
+      st = write_schedule(h, cls, s, stream);
+      if (st != NWC_OK) return st;
+      continue;
+    }
+    nwc::build_schedule(h->index.data(), h->tiles, s, image + class_off(*h, cls));
+    note_schedule(h, cls, s);
+  }
   return NWC_OK;
 }
 
@@ -335,13 +353,10 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
 nwc_status nwc_decompress(nwc_handle_t h, uint16_t* d_w_out, nwc_stream_t stream) {
   if (!h || !d_w_out || !aligned(d_w_out, 4)) return NWC_ERR_INVALID_ARG;
   nwc::LaunchShape s;
-  nwc_status st = shape_for(h, &s, reinterpret_cast<cudaStream_t>(stream));
+  nwc_status st = shape_for(h, 0, &s, reinterpret_cast<cudaStream_t>(stream));
   if (st != NWC_OK) return st;
-  nwc::TileParams p = base_params(*h);
+  nwc::TileParams p = base_params(*h, 0, s);
   p.out = d_w_out;
-  p.ring_offset = (uint32_t)s.ring_offset;
-  p.ring_bytes = s.ring_bytes;
-  p.batch_tiles = s.batch_tiles;
   return cuda_status(nwc::launch_decompress(p, (int)h->tile_cols, h->lmax <= 7, s,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -361,21 +376,21 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
     return NWC_ERR_INVALID_ARG;
   // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
   if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
-  nwc::LaunchShape s;
-  nwc_status st = shape_for(h, &s, reinterpret_cast<cudaStream_t>(stream));
-  if (st != NWC_OK) return st;
-  nwc::TileParams p = base_params(*h);
-  p.ring_offset = (uint32_t)s.ring_offset;
-  p.ring_bytes = s.ring_bytes;
-  p.batch_tiles = s.batch_tiles;
-  if (need) {
-    uint8_t* ws = static_cast<uint8_t*>(d_workspace);
-    p.counters = reinterpret_cast<uint32_t*>(ws);
-    p.partial = reinterpret_cast<float*>(ws + round_up(4ull * (uint64_t)h->tiles_r, 256));
-  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   for (int32_t b0 = 0; b0 < batch; b0 += kChunkBatch) {
     const int32_t nb = batch - b0 < kChunkBatch ? batch - b0 : kChunkBatch;
+    // The x-stage class (and with it the schedule and ring) follows the rows
+    // of x this launch handles.
+    const int cls = nwc::stage_class(nb);
+    nwc::LaunchShape s;
+    nwc_status st = shape_for(h, cls, &s, cs);
+    if (st != NWC_OK) return st;
+    nwc::TileParams p = base_params(*h, cls, s);
+    if (need) {
+      uint8_t* ws = static_cast<uint8_t*>(d_workspace);
+      p.counters = reinterpret_cast<uint32_t*>(ws);
+      p.partial = reinterpret_cast<float*>(ws + round_up(4ull * (uint64_t)h->tiles_r, 256));
+    }
     p.x = d_x + (int64_t)b0 * h->cols;
     p.y = d_y + (int64_t)b0 * h->rows;
     p.batch = nb;
@@ -448,19 +463,21 @@ nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word) {
 }
 
 nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
-                                 uint64_t smem_limit, nwc_schedule_info* info,
+                                 uint64_t smem_limit, int32_t rows_of_x, nwc_schedule_info* info,
                                  uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring) {
-  if (!blob || !info || info->struct_size < sizeof(nwc_schedule_info) || sm_count < 1)
+  if (!blob || !info || info->struct_size < sizeof(nwc_schedule_info) || sm_count < 1 ||
+      rows_of_x < 0 || rows_of_x > nwc::kMaxPassRows)
     return NWC_ERR_INVALID_ARG;
   nwc_handle_s h;
   if (!nwc::parse_blob(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &h, nullptr))
     return NWC_ERR_CORRUPT;
+  const int cls = nwc::stage_class(rows_of_x);
   nwc::LaunchShape s;
-  nwc_status st = shape_on(h, sm_count, (size_t)smem_limit, &s);
+  nwc_status st = shape_on(h, sm_count, (size_t)smem_limit, cls, &s);
   if (st != NWC_OK) return st;
   std::vector<uint8_t> sched;
   try {
-    sched.resize(nwc::sched_bytes((uint64_t)h.tiles));
+    sched.resize(nwc::sched_class_bytes((uint64_t)h.tiles));
   } catch (const std::bad_alloc&) {
     return NWC_ERR_NOMEM;
   }
@@ -472,6 +489,7 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
   info->tiles = h.tiles;
   info->batches = cb[s.ctas];
   info->smem_bytes = s.smem_bytes;
+  info->xstage_bytes = s.xstage_bytes;
   if (cta_batch) std::memcpy(cta_batch, cb, 4 * ((size_t)s.ctas + 1));
   if (batch)
     std::memcpy(batch, sched.data() + nwc::sched_batch_off(), 16 * (size_t)cb[s.ctas]);

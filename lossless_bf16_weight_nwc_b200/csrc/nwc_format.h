@@ -18,9 +18,10 @@
 // Tiles are stored column-block-major: u = j * tiles_r + i.
 //
 // Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)]
-// | zero pad to 256 | launch schedule (sched_bytes(tiles) bytes).  The launch
-// schedule is not part of the blob: the library writes it for the device that
-// runs the kernels (its SM count and shared memory), as
+// | zero pad to 256 | launch schedules (sched_bytes(tiles) bytes: one per
+// x-stage class, each sched_class_bytes(tiles)).  They are not part of the
+// blob: the library writes them for the device that runs the kernels (its SM
+// count and shared memory), each as
 //   u32 cta_batch[kMaxCtas + 1]   first batch of each CTA (padded to 16 bytes)
 //   u32x4 batch[sched_max_batches(tiles)]
 //        {tile-area offset in 16-byte units, bytes, ring offset, batches of
@@ -77,7 +78,13 @@ constexpr uint64_t sched_batch_off() { return round_up(4ull * (kMaxCtas + 1), 16
 constexpr uint64_t sched_tile_off(uint64_t tiles) {
   return sched_batch_off() + 16ull * sched_max_batches(tiles);
 }
-constexpr uint64_t sched_bytes(uint64_t tiles) { return round_up(sched_tile_off(tiles) + 4ull * tiles, 256); }
+// One schedule per x-stage class (see kernels.cuh): class 0 for decompression
+// and GEMV launches of up to 4 rows of x, class 1 for 5 to 16 rows.
+constexpr int kStageClasses = 2;
+constexpr uint64_t sched_class_bytes(uint64_t tiles) {
+  return round_up(sched_tile_off(tiles) + 4ull * tiles, 256);
+}
+constexpr uint64_t sched_bytes(uint64_t tiles) { return kStageClasses * sched_class_bytes(tiles); }
 
 struct BlobHeader {
   uint32_t magic, version, header_bytes, lmax;

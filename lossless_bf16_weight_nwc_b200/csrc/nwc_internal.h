@@ -32,8 +32,10 @@ struct nwc_handle_s {
   uint64_t max_chunk = 0;  // largest chunk in bytes
   int device = 0;
   std::vector<uint32_t> index;  // chunk offsets (16-byte units), tiles + 1
-  // Shape the device image's launch schedule was written for (0: none yet).
-  int sched_ctas = 0, sched_ring = 0, sched_tiles_per_batch = 0;
+  // Shape each of the device image's launch schedules (one per x-stage
+  // class) was written for (0: none yet).
+  int sched_ctas[nwc::kStageClasses] = {}, sched_ring[nwc::kStageClasses] = {},
+      sched_tiles_per_batch[nwc::kStageClasses] = {};
 };
 
 namespace nwc {

@@ -16,7 +16,7 @@
 namespace nwc {
 
 void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s, uint8_t* out) {
-  std::memset(out, 0, sched_bytes((uint64_t)n_tiles));
+  std::memset(out, 0, sched_class_bytes((uint64_t)n_tiles));
   uint32_t* cta_batch = reinterpret_cast<uint32_t*>(out);
   uint32_t* batch = reinterpret_cast<uint32_t*>(out + sched_batch_off());
   uint32_t* tile_ring = reinterpret_cast<uint32_t*>(out + sched_tile_off((uint64_t)n_tiles));

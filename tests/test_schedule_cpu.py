@@ -10,7 +10,7 @@ from lossless_bf16_weight_nwc_b200 import synth
 K_SLOTS = 64          # barrier slots per CTA (kernels.cuh)
 K_MAX_LAG = 48        # tiles a consumer's next wait may lie past its last release (kernels.cuh)
 K_MAX_CTAS = 256
-K_XSTAGE = 33024      # shared memory reserved for the CTA's columns of x (kernels.cu)
+K_XSTAGE = {1: 8448, 16: 33024}  # shared memory for x by rows of x per launch (kernels.cuh)
 K_RING_SLACK = 256    # shared memory after the ring that readers may touch (kernels.cu)
 B200_SMS, B200_SMEM = 148, 232448
 
@@ -38,8 +38,8 @@ def index_of(blob):
     return np.frombuffer(blob[384:384 + 4 * (n + 1)].tobytes(), dtype=np.uint32).astype(np.int64)
 
 
-def check_schedule(lib, blob, sms, smem):
-    info, cta, bat, ring = lib.nwc_schedule_describe(blob, sms, smem)
+def check_schedule(lib, blob, sms, smem, rows_of_x=1):
+    info, cta, bat, ring = lib.nwc_schedule_describe(blob, sms, smem, rows_of_x)
     index = index_of(blob)
     n_tiles = len(index) - 1
     C, T, R = info["ctas"], info["batch_tiles"], info["ring_bytes"]
@@ -47,6 +47,7 @@ def check_schedule(lib, blob, sms, smem):
     assert C == min(n_tiles, sms, K_MAX_CTAS)
     assert 2 <= T <= 8
     assert R % 16 == 0 and info["smem_bytes"] <= smem
+    assert info["xstage_bytes"] == K_XSTAGE[1 if rows_of_x <= 4 else 16]
     assert cta[0] == 0 and cta[C] == info["batches"] == len(bat)
     max_out = K_SLOTS - -(-K_MAX_LAG // T)
     for c in range(C):
@@ -78,7 +79,20 @@ def check_schedule(lib, blob, sms, smem):
                                                  (14336, 512, 512), (77, 1030, 256),
                                                  (1000, 1026, 128), (4100, 96, 64), (8, 64, 64)])
 def test_schedule_invariants_b200(lib, rows, cols, tile_cols):
-    check_schedule(lib, blob_of(lib, rows, cols, tile_cols), B200_SMS, B200_SMEM)
+    blob = blob_of(lib, rows, cols, tile_cols)
+    for rows_of_x in (0, 1, 4, 5, 16):
+        check_schedule(lib, blob, B200_SMS, B200_SMEM, rows_of_x)
+
+
+def test_schedule_classes_differ_in_ring(lib):
+    """Launches of up to 4 rows of x reserve less shared memory for x, so their
+    ring is larger by up to the difference (a ring never exceeds what the CTA's
+    tiles need)."""
+    blob = blob_of(lib, 4096, 4096)
+    small, _, _, _ = lib.nwc_schedule_describe(blob, B200_SMS, B200_SMEM, 1)
+    large, _, _, _ = lib.nwc_schedule_describe(blob, B200_SMS, B200_SMEM, 16)
+    assert 0 < small["ring_bytes"] - large["ring_bytes"] <= K_XSTAGE[16] - K_XSTAGE[1]
+    assert small["smem_bytes"] <= large["smem_bytes"] <= B200_SMEM
 
 
 @pytest.mark.parametrize("sms,smem", [(1, B200_SMEM), (3, 100_000), (148, 120_000),
@@ -88,6 +102,8 @@ def test_schedule_invariants_other_devices(lib, sms, smem):
     # the CTA cap.
     blob = blob_of(lib, 2048, 2048, 512, lmax=12, kind="student_t5", seed=3)
     check_schedule(lib, blob, sms, smem)
+    if smem >= 100_000:
+        check_schedule(lib, blob, sms, smem, 16)
 
 
 def test_schedule_tight_ring_serialises(lib):
@@ -98,7 +114,7 @@ def test_schedule_tight_ring_serialises(lib):
     T = info["batch_tiles"]
     index = index_of(blob)
     max_chunk = int(16 * np.diff(index).max())
-    ring_offset = -(-(-(-(16384 + 8 + 2 * K_SLOTS * 8) // 16) * 16 + K_XSTAGE) // 128) * 128
+    ring_offset = -(-(-(-(16384 + 8 + 2 * K_SLOTS * 8) // 16) * 16 + K_XSTAGE[1]) // 128) * 128
     smem = ring_offset + T * max_chunk + K_RING_SLACK  # ring of one worst-case batch + read slack
     assert 2 * int(bat[:-1, 1].min()) > T * max_chunk + 16  # the last batch may be short
     info, _, bat, _ = lib.nwc_schedule_describe(blob, 1, smem)
@@ -113,5 +129,7 @@ def test_schedule_errors(lib):
         lib.nwc_schedule_describe(blob[:200], B200_SMS, B200_SMEM)
     with pytest.raises(lib.NwcError):
         lib.nwc_schedule_describe(blob, 0, B200_SMEM)
+    with pytest.raises(lib.NwcError):  # more rows than one launch takes
+        lib.nwc_schedule_describe(blob, B200_SMS, B200_SMEM, 17)
     with pytest.raises(lib.NwcError):  # a 64 KiB decode table alone does not fit
         lib.nwc_schedule_describe(blob, B200_SMS, 60_000)
