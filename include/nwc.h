@@ -153,6 +153,19 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
  * Errors: INVALID_ARG, CUDA (launch). */
 nwc_status nwc_decompress(nwc_handle_t handle, uint16_t* d_w_out, nwc_stream_t stream);
 
+/* Rows of W, bit-exact, straight from the compressed matrix: an embedding
+ * lookup, e.g. on a tied lm_head ("NWC", "How it works > Dequantization and
+ * embedding lookup").  out[i][k] = W[rows[i]][k] for i < n, k < cols.
+ *   d_rows: device, int32 [n], row ids in [0, rows), 4-byte aligned.
+ *   d_out: device, BF16 [n x cols] row-major, 2-byte aligned.
+ *   n in [1, 2^20].
+ * A row id out of range leaves its output row unwritten and sets a bit of the
+ * device error word (nwc_get_device_error then returns INVALID_ARG).  Only the
+ * tiles that hold the requested rows are read.  Asynchronous on `stream`.
+ * Errors: INVALID_ARG, CUDA (launch). */
+nwc_status nwc_gather_rows(nwc_handle_t handle, const int32_t* d_rows, int32_t n,
+                           uint16_t* d_out, nwc_stream_t stream);
+
 /* Bytes of scratch that nwc_gemv needs for this handle and batch; 0 when the
  * matrix has a single column tile.  The scratch holds one FP32 partial sum per
  * (column tile, batch row, output row) plus one u32 counter per row tile; it
@@ -248,8 +261,9 @@ nwc_status nwc_handle_info(nwc_handle_t handle, int64_t* rows, int64_t* cols,
                            uint64_t* blob_bytes, uint64_t* device_bytes);
 
 /* Synchronizes `stream`, then reads and clears the device error word of the
- * current device.  Returns OK, DEVICE_TIMEOUT or DEVICE_CORRUPT (timeout
- * wins), or CUDA.  *word (optional) receives the raw bits. */
+ * current device.  Returns OK, DEVICE_TIMEOUT, DEVICE_CORRUPT or INVALID_ARG
+ * (a gathered row id out of range), in that order of precedence, or CUDA.
+ * *word (optional) receives the raw bits. */
 nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word);
 
 /* Free host metadata.  NULL is accepted.  Device memory is never freed. */

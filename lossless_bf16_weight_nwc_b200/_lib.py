@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "nwc_upload_blob": ([vp, u64, vp, u64, vp, c.POINTER(vp)], c.c_int),
         "nwc_handle_from_device": ([vp, u64, c.POINTER(vp)], c.c_int),
         "nwc_decompress": ([vp, vp, vp], c.c_int),
+        "nwc_gather_rows": ([vp, vp, i32, vp, vp], c.c_int),
         "nwc_gemv_workspace_size": ([vp, i32, c.POINTER(u64)], c.c_int),
         "nwc_gemv": ([vp, vp, vp, i32, vp, u64, vp], c.c_int),
         "nwc_gemv_noalloc": ([vp, vp, vp, i32, vp], c.c_int),
@@ -82,7 +83,8 @@ def _load() -> ctypes.CDLL:
 LIB = _load()
 EXPORTED = ("nwc_version", "nwc_status_string", "nwc_plan", "nwc_plan_size", "nwc_compress",
             "nwc_compress_host", "nwc_blob_device_bytes", "nwc_upload_blob",
-            "nwc_handle_from_device", "nwc_decompress", "nwc_gemv_workspace_size", "nwc_gemv",
+            "nwc_handle_from_device", "nwc_decompress", "nwc_gather_rows",
+            "nwc_gemv_workspace_size", "nwc_gemv",
             "nwc_gemv_noalloc",
             "nwc_handle_info", "nwc_get_device_error", "nwc_schedule_describe",
             "nwc_plan_destroy", "nwc_handle_destroy")
@@ -168,6 +170,12 @@ def nwc_handle_from_device(d_buf, d_bytes: int):
 
 def nwc_decompress(handle, d_w_out, stream=None) -> None:
     _check(LIB.nwc_decompress(handle, _ptr(d_w_out), _stream(stream)), "nwc_decompress")
+
+
+def nwc_gather_rows(handle, d_rows, n: int, d_out, stream=None) -> None:
+    """out[i] = W[rows[i]] (BF16 bit patterns), decoded from the compressed matrix."""
+    _check(LIB.nwc_gather_rows(handle, _ptr(d_rows), n, _ptr(d_out), _stream(stream)),
+           "nwc_gather_rows")
 
 
 def nwc_gemv_workspace_size(handle, batch: int) -> int:
@@ -307,6 +315,14 @@ class CompressedMatrix:
         ws, ws_bytes = self.workspace(batch)
         nwc_gemv(self.handle, xb, y, batch, ws, ws_bytes, stream)
         return y
+
+    def gather_rows(self, rows, stream=None):
+        """BF16 rows W[rows] (torch.int32 ids on the device) -> [len(rows), cols]."""
+        import torch
+        rows = rows.to(torch.int32).contiguous()
+        out = torch.empty((rows.numel(), self.cols), dtype=torch.bfloat16, device=rows.device)
+        nwc_gather_rows(self.handle, rows, rows.numel(), out, stream)
+        return out
 
     def close(self) -> None:
         if self.handle is not None:

@@ -780,6 +780,61 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     atomicOr(&g_device_error, kErrCorrupt);
 }
 
+// Row gather ("NWC", "How it works > Dequantization and embedding lookup": the
+// same decoder serves row lookups): warp w writes output row w / tiles_c,
+// column block w % tiles_c.  Of the tile that holds the row, only the four
+// lanes that own that tile row decode (lane 4g + c owns row g), one code per
+// table lookup, reading the stream, the raw plane and the table through L1;
+// the other lanes leave.  Stream bytes past the chunk read as zero, so a corrupt
+// chunk can misdecode but never read outside it.
+__global__ void __launch_bounds__(256) gather_kernel(GatherParams p) {
+  const int64_t wg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wg >= (int64_t)p.n * p.tiles_c) return;
+  const int64_t i = wg / p.tiles_c, j = wg % p.tiles_c;
+  const int32_t row = __ldg(p.row_ids + i);
+  if (row < 0 || row >= p.rows) {
+    if (lane == 0 && j == 0) atomicOr(&g_device_error, kErrRange);
+    return;
+  }
+  if ((lane >> 2) != row % kTileRows) return;
+  const int c = lane & 3;
+  const int64_t u = j * p.tiles_r + row / kTileRows;
+  const uint32_t c0 = __ldg(p.index + u), c1 = __ldg(p.index + u + 1);
+  const uint8_t* chunk = p.tiles + 16ull * c0;
+  const uint32_t raw = (uint32_t)(kTileRows * p.tile_cols);
+  const uint32_t chunk_bytes = 16u * (c1 - c0);
+  const uint32_t area_bytes = chunk_bytes > raw + kLanes ? chunk_bytes - raw - kLanes : 0u;
+  const uint8_t* lens = chunk + raw;
+  const uint8_t* area = lens + kLanes;
+  uint32_t q = 0;  // next sequence byte of this lane's stream
+  for (int t = 0; t < lane; ++t) q += __ldg(lens + t);
+  // Sequence byte q sits in little-endian word q / 4 as its byte 3 - q % 4.
+  auto seq_byte = [&](uint32_t b) -> uint64_t {
+    return b < area_bytes ? (uint64_t)__ldg(area + ((b & ~3u) | (3u - (b & 3u)))) : 0ull;
+  };
+  uint64_t buf = 0;  // next bits, most significant first
+  int nbits = 0;
+  const int symbols = 16 * (p.tile_cols / 64);
+  uint16_t* orow = p.out + i * p.cols;
+  uint32_t bad = 0;
+  for (int k = 0; k < symbols; ++k) {
+    while (nbits < p.peek) {
+      buf |= seq_byte(q++) << (56 - nbits);
+      nbits += 8;
+    }
+    const uint32_t e = __ldg(p.table + (uint32_t)(buf >> (64 - p.peek)));
+    const uint32_t len = (e >> kEntryLen0Shift) & 15u, s = (e >> 7) & 0xFFu;
+    bad |= e & kEntryInvalid;
+    buf <<= (e & kEntryInvalid) ? 1u : len;  // an invalid prefix still moves on
+    nbits -= (e & kEntryInvalid) ? 1 : (int)len;
+    const uint32_t r = __ldg(chunk + (k / 16) * 512 + 16 * lane + (k % 16));
+    const int64_t col = j * p.tile_cols + 64 * (k / 16) + 16 * c + (k % 16);
+    if (col < p.cols) orow[col] = (uint16_t)(((r & 0x80u) << 8) | (s << 7) | (r & 0x7Fu));
+  }
+  if (bad) atomicOr(&g_device_error, kErrCorrupt);
+}
+
 // Raises a kernel's dynamic shared-memory limit on the current device once per
 // (kernel, device) to the largest size requested so far.
 template <typename Kernel>
@@ -897,6 +952,14 @@ cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
     case 64: return fast ? launch_decompress_t<1, true>(p, s, stream) : launch_decompress_t<1, false>(p, s, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_gather(const GatherParams& g, cudaStream_t stream) {
+  const int64_t warps = (int64_t)g.n * g.tiles_c;
+  const int64_t blocks = (warps + 7) / 8;
+  if (blocks < 1 || blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  gather_kernel<<<(unsigned)blocks, 256, 0, stream>>>(g);
+  return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_error(uint32_t* word) {

@@ -18,6 +18,7 @@ constexpr int kMaxPassRows = 16;
 // Device error word bits (read and cleared by nwc_get_device_error).
 constexpr uint32_t kErrTimeout = 1u;   // a bounded mbarrier wait gave up
 constexpr uint32_t kErrCorrupt = 2u;   // a stream held no valid code
+constexpr uint32_t kErrRange = 4u;     // a gathered row id was out of range
 
 struct TileParams {
   const uint8_t* tiles;     // device: tile area of the blob
@@ -82,6 +83,20 @@ cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const Lau
                         cudaStream_t stream);
 cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
                               const LaunchShape& s, cudaStream_t stream);
+// Row gather (embedding lookup) from the compressed matrix.
+struct GatherParams {
+  const uint8_t* tiles;     // device: tile area of the blob
+  const uint32_t* index;    // device: chunk offsets (16-byte units), tiles + 1
+  const uint32_t* table;    // device: decode table
+  int32_t peek;             // table peek width (12 or 14)
+  int32_t tile_cols;
+  int64_t rows, cols, tiles_r, tiles_c;
+  const int32_t* row_ids;   // device: n row ids
+  int32_t n;
+  uint16_t* out;            // device: BF16 [n x cols]
+};
+cudaError_t launch_gather(const GatherParams& g, cudaStream_t stream);
+
 cudaError_t read_and_clear_error(uint32_t* word);
 
 }  // namespace nwc

@@ -361,6 +361,28 @@ nwc_status nwc_decompress(nwc_handle_t h, uint16_t* d_w_out, nwc_stream_t stream
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uint16_t* d_out,
+                           nwc_stream_t stream) {
+  if (!h || !d_rows || !d_out || n < 1 || n > (1 << 20) || !aligned(d_rows, 4) ||
+      !aligned(d_out, 2))
+    return NWC_ERR_INVALID_ARG;
+  nwc::GatherParams g;
+  std::memset(&g, 0, sizeof(g));
+  g.tiles = h->d_base + h->tiles_off;
+  g.index = reinterpret_cast<const uint32_t*>(h->d_base + h->index_off);
+  g.table = reinterpret_cast<const uint32_t*>(h->d_base + h->table_off);
+  g.peek = nwc::peek_bits(h->lmax);
+  g.tile_cols = (int32_t)h->tile_cols;
+  g.rows = h->rows;
+  g.cols = h->cols;
+  g.tiles_r = h->tiles_r;
+  g.tiles_c = h->tiles_c;
+  g.row_ids = d_rows;
+  g.n = n;
+  g.out = d_out;
+  return cuda_status(nwc::launch_gather(g, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nwc_status nwc_gemv_workspace_size(nwc_handle_t h, int32_t batch, uint64_t* bytes) {
   if (!h || !bytes || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
   *bytes = workspace_bytes_for(*h, batch);
@@ -459,6 +481,7 @@ nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word) {
   if (word) *word = w;
   if (w & nwc::kErrTimeout) return NWC_ERR_DEVICE_TIMEOUT;
   if (w & nwc::kErrCorrupt) return NWC_ERR_DEVICE_CORRUPT;
+  if (w & nwc::kErrRange) return NWC_ERR_INVALID_ARG;
   return NWC_OK;
 }
 

@@ -168,6 +168,44 @@ def test_gemv_into_pinned_host_memory(lib, orc):
     no_device_error(lib)
 
 
+@pytest.mark.parametrize("lmax", [0, 12])
+@pytest.mark.parametrize("shape,tile_cols", [((77, 1030), 256), ((1000, 2048), 512), ((9, 64), 64),
+                                             ((4100, 96), 512)])
+def test_gather_rows(lib, shape, tile_cols, lmax):
+    """Embedding lookup from the compressed matrix: bit-exact rows."""
+    spec = synth.MatrixSpec("w", shape[0], shape[1], "student_t5", 0.015, 2)
+    w = synth.matrix(spec, 8)
+    m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
+    rng = np.random.default_rng(3)
+    ids = np.concatenate([[0, shape[0] - 1], rng.integers(0, shape[0], 37)]).astype(np.int32)
+    out = m.gather_rows(torch.from_numpy(ids).cuda())
+    assert np.array_equal(bits(out), w[ids])
+    no_device_error(lib)
+
+
+def test_gather_rows_every_pattern(lib):
+    """All 65,536 BF16 patterns (NaN payloads, infinities, zeros), which need
+    lmax 8 and the 12-bit table."""
+    w = np.arange(65536, dtype=np.uint16).reshape(256, 256)
+    m = lib.CompressedMatrix.compress(w)
+    ids = np.arange(255, -1, -1, dtype=np.int32)
+    assert np.array_equal(bits(m.gather_rows(torch.from_numpy(ids).cuda())), w[ids])
+    no_device_error(lib)
+
+
+def test_gather_rows_out_of_range(lib):
+    w = synth.matrix(synth.MatrixSpec("w", 24, 512, "normal", 0.02, 0), 1)
+    m = lib.CompressedMatrix.compress(w)
+    out = torch.zeros((2, 512), dtype=torch.int16, device="cuda")
+    ids = torch.tensor([5, 24], dtype=torch.int32, device="cuda")
+    lib.nwc_gather_rows(m.handle, ids, 2, out)
+    st, word = lib.nwc_get_device_error()
+    assert st == 1 and word & 4                     # INVALID_ARG: a row id out of range
+    assert np.array_equal(out[0].cpu().numpy().view(np.uint16), w[5])
+    assert not out[1].any()                         # left unwritten
+    no_device_error(lib)
+
+
 def test_handle_from_device_image(lib, orc):
     spec = synth.MatrixSpec("w", 96, 1536, "normal", 0.02, 0)
     w = synth.matrix(spec, 2)
