@@ -65,8 +65,16 @@ def measured_peaks() -> tuple[dict, str]:
 
 
 def kernel_source_hash() -> str:
-    with open(KERNEL_SOURCE, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the kernel source's code: '//' comments, trailing blanks and
+    empty lines are dropped, so that a comment edit keeps a capture valid while
+    any change to the code itself does not."""
+    lines = []
+    with open(KERNEL_SOURCE, encoding="utf-8") as f:
+        for line in f:
+            code = line.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
 def profile_traffic(workload: str, batch: int) -> float | None:

@@ -1,29 +1,32 @@
-// kernels.cu — sm_100a kernels: fused decode-GEMV and bit-exact decompress.
+// kernels.cu — sm_100a kernels: fused decode-GEMV, bit-exact decompress and
+// row gather.
 //
 // What runs where ("NWC — Neural Weight Compression", "How it works > Fused
 // kernel"; "Unweight", "Direct GPU Decompression"):
 //   * One persistent CTA per SM owns a contiguous range of tiles (8 rows x
 //     tile_cols), in the blob's column-block-major order.
-//   * A producer warp streams the tiles' chunks (raw plane + lane streams) from
-//     HBM into one CTA-wide shared-memory ring with cp.async.bulk (no
-//     multicast).  Each chunk lands in a slot with a "full" mbarrier (bytes
-//     counted) and is handed back through an "empty" mbarrier.  Every wait is
-//     bounded: a wait that gives up sets the device error word, and the
-//     producer drains its copies before leaving.
-//   * 16 consumer warps take the CTA's tiles round-robin.  Each lane decodes its
-//     own bit stream with a 64-bit window and a table peek.  With lmax <= 7 the
-//     peek is 14 bits and every entry holds two complete codes ("NWC", "Prefix
-//     code instead of rANS"), so a step is a lookup plus two funnel shifts.
-//     With lmax 8..12 the peek is 12 bits and a pair that does not fit takes a
-//     second lookup.  The window is refilled every two steps, without a branch.
+//   * A producer warp follows the launch schedule the host wrote into the
+//     device image: per batch of consecutive tiles it waits for the releases
+//     the schedule names and issues one cp.async.bulk (no multicast) into a
+//     CTA-wide shared-memory ring.  Each batch has a "full" mbarrier (bytes
+//     counted) and an "empty" one that its tiles' consumers arrive at.  Every
+//     wait is bounded: a wait that gives up sets the device error word, and the
+//     producer waits for its copies before leaving.
+//   * 31 consumer warps take the CTA's tiles round-robin.  Each lane decodes
+//     its own bit stream.  With lmax <= 7 the peek is 14 bits and every table
+//     entry holds two complete codes ("NWC", "Prefix code instead of rANS"), so
+//     two steps take one 32-bit window, two lookups and a predicated word
+//     rotation; lmax 8..12 uses a 12-bit peek with a second lookup for a pair
+//     that does not fit.
 //   * BF16x2 reassembly is one byte permute of the raw plane and one bitwise
 //     select with the table entry; the weights never leave registers.
-//   * GEMV: FP32 accumulation of BF16 x BF16 products (fma.rn.f32.bf16) into 8
-//     row sums per batch row, a transposed warp-shuffle reduction per tile, and
-//     a split-K reduction in a fixed order through the workspace (the last of a
-//     row block's column tiles to finish sums the partials).
-//   * Decompress: the same decode, with a 32-bit store per weight pair, one
-//     128-byte line per warp store.
+//   * GEMV: lane 4g + c owns row g of a tile, so two decoded pairs are the B
+//     operand of one m16n8k16 tensor-core step whose A operand is x (staged in
+//     shared memory); FP32 accumulation, then a split-K reduction in a fixed
+//     order through the workspace (the last of a row block's column tiles to
+//     finish sums the partials).  Launches use programmatic dependent launch.
+//   * Decompress: the same decode, two 16-byte stores per lane and group.
+//   * Row gather: the four lanes owning a requested row decode it from L1.
 #include <cuda_runtime.h>
 
 #include <cstdint>
