@@ -46,7 +46,7 @@ constexpr int kTablePieces = 8;                  // bulk copies that bring in th
 constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
 constexpr uint32_t kPairReadSpan = 12 + 4 * kMaxPairSteps + 4;  // bytes one tile's reader may touch
 static_assert(kPairReadSpan <= kRingSlack, "a clamped reader must stay inside the ring slack");
-constexpr uint64_t kBatchTarget = 8192;          // bytes a bulk copy should move at least
+constexpr uint64_t kBatchTarget = 12288;          // bytes a bulk copy should move at least
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
 // ---- PTX helpers -----------------------------------------------------------
@@ -508,7 +508,7 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
   };
   uint2 xa = x_at(xr0, xs0, 0);
   uint2 xb = WIDE ? x_at(xr1, xs1, 0) : make_uint2(0u, 0u);
-#pragma unroll 1
+#pragma unroll 2
   for (int m = 0; m < CP; ++m) {
     const uint4 rv = lds128(chunk + m * 512 + lane * 16);
 #pragma unroll
