@@ -110,7 +110,7 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   return v;
 }
 // Programmatic dependent launch: let the next kernel on the stream start its
-// prologue now (its CTAs become resident as this grid's exit), and wait until
+// prologue now (its CTAs become resident as this grid's CTAs exit), and wait until
 // the previous kernel has completed and its writes are visible.
 __device__ __forceinline__ void allow_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -158,12 +158,13 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
 
 // ---- bit reader --------------------------------------------------------------
 
-// Per-lane reader of the lane's stream in shared memory: a 64-bit window hi:lo
-// (next bit = bit 31 of hi) and a valid-bit count.  Invariant at each refill
-// point: at least 32 valid bits; a step consumes at most 14 bits, so the two
-// steps between refill points always have their peek bits.  The low 7 bits of
-// `nbacc` count valid bits; subtracting whole table entries keeps them exact,
-// since entry bits 4..6 are zero and bits 0..3 hold the consumed count.
+// Per-lane reader of the lane's stream in shared memory, used with the 12-bit
+// peek (lmax 8..12): a 64-bit window hi:lo (next bit = bit 31 of hi) and a
+// valid-bit count.  A refill point leaves at least 32 valid bits; a lookup
+// consumes at most 12, and a pair that does not fit refills before its second
+// lookup, so every lookup has its 12 peek bits.  The low 7 bits of `nbacc`
+// count valid bits; subtracting whole table entries keeps them exact, since
+// entry bits 4..6 are zero and bits 0..3 hold the consumed count.
 struct BitReader {
   uint32_t hi, lo, nbacc;
   uint32_t nw;  // the stream word after the window, loaded ahead
@@ -212,7 +213,9 @@ struct BitReader {
 };
 
 // One step: a table entry holding two exponent bytes at their BF16 positions
-// (bits 7..14 and 23..30).  FAST: 14-bit peek, both codes always fit.
+// (bits 7..14 and 23..30).  FAST: 14-bit peek, both codes always fit (the
+// kernels read that case with PairReader below); else 12-bit peek with a second
+// lookup for a pair that does not fit.
 template <bool FAST>
 __device__ __forceinline__ uint32_t decode_pair(BitReader& br, uint32_t table) {
   if (FAST) {
@@ -234,11 +237,11 @@ __device__ __forceinline__ uint32_t decode_pair(BitReader& br, uint32_t table) {
 
 // Reader for the 14-bit peek (lmax <= 7), two steps at a time: two steps
 // consume at most 28 bits, so one 32-bit window taken before them holds both
-// peeks.  The stream is kept as three consecutive words a, b, c with p (< 32)
-// the offset of the next unread bit in a; after two steps the words move on by
-// one when p passed 32, and the word after c is fetched (predicated) at once,
-// two steps before it can be needed, so no shared-memory load of the stream
-// lies on the decoder's dependency chain.
+// peeks.  The stream is kept as three consecutive words a, b, c with bits 0..4
+// of p the offset of the next unread bit in a; after two steps the words move
+// on by one when the offset passed 32, and the word after c is fetched
+// (predicated) at once, two steps before it can be needed, so no shared-memory
+// load of the stream lies on the decoder's dependency chain.
 struct PairReader {
   uint32_t a, b, c;  // stream words base, base + 1, base + 2
   uint32_t p;        // bits 0..4: next unread bit of a (0 = its bit 31); higher
@@ -313,8 +316,9 @@ struct StreamDecoder<false> {
   }
 };
 
-// Raw bytes of step r (row r of a 64-column group) duplicated into both bytes
-// of each half: [r0, r0, r1, r1].
+// Raw bytes of the lane's step r in a 64-column group (its symbols 2r and
+// 2r + 1, bytes 2r and 2r + 1 of the group's 16) duplicated into both bytes of
+// each half: [b1, b1, b0, b0] from high to low.
 template <int R>
 __device__ __forceinline__ uint32_t raw_pair(const uint4& rv) {
   const uint32_t w = (R < 2) ? rv.x : (R < 4) ? rv.y : (R < 6) ? rv.z : rv.w;
