@@ -145,7 +145,14 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
 /* nwc_decompress, nwc_gemv and nwc_gemv_noalloc launch one persistent CTA per
  * SM (at most 256).  Should the current device's launch shape differ from the
  * one the image's schedule was written for, the call first rewrites that
- * schedule on `stream` (a host-to-device copy, in stream order). */
+ * schedule on `stream` (a host-to-device copy, in stream order).
+ *
+ * They launch with programmatic stream serialization: a kernel may start while
+ * the previous kernel on the stream is still finishing.  Until that kernel has
+ * completed it reads only the device image (blob, decode table, schedule);
+ * x, y, the workspace and the output are touched only afterwards.  So the
+ * kernel launched just before such a call must not write the device image
+ * (stream order still holds for copies, memsets and events). */
 
 /* Bit-exact decompression ("NWC", "How it works > Dequantization and embedding
  * lookup": the same decoder writes BF16).  d_w_out: device, rows x cols BF16,
@@ -181,9 +188,10 @@ nwc_status nwc_gemv_workspace_size(nwc_handle_t handle, int32_t batch,
  *   batch in [1, 64].
  *   d_workspace: device, >= nwc_gemv_workspace_size bytes, 16-byte aligned,
  *     zero-filled before its first use.  Every completed call leaves the counter
- *     area zero again, so one workspace serves any number of ordered calls.  Two
- *     calls that overlap on the GPU must not share a workspace.  It may be NULL
- *     when the size is 0.
+ *     area zero again, so one workspace serves any number of ordered calls (a
+ *     call that ended with a device error may not: zero it again).  Two calls
+ *     that overlap on the GPU must not share a workspace.  It may be NULL when
+ *     the size is 0.
  * Products and sums are in FP32; the result is the same bit pattern on every
  * run.  Asynchronous on `stream`.
  * Errors: INVALID_ARG (null, batch, alignment, odd cols, workspace too small),
