@@ -374,6 +374,10 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   if (h.tiles_r != (h.rows + 7) / 8 || h.tiles_c != (h.cols + h.tile_cols - 1) / h.tile_cols)
     return false;
   if (h.lens_off != kLensOffset || h.index_off != kIndexOffset || h.filler > 255) return false;
+  // Every tile has a 4-byte index entry inside the head, which bounds the tile
+  // count before it is formed: no size computed from it below can wrap around.
+  const uint64_t max_tiles = head_bytes / 4;
+  if (h.tiles_r > max_tiles || h.tiles_c > max_tiles / h.tiles_r) return false;
   const uint64_t tiles = h.tiles_r * h.tiles_c;
   if (h.tiles_off != round_up(kIndexOffset + 4 * (tiles + 1), 256)) return false;
   if (h.total_bytes != bytes || h.tiles_off > head_bytes) return false;

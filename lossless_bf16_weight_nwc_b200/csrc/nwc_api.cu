@@ -8,6 +8,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 #include <vector>
 
 #include "../../include/nwc.h"
@@ -74,7 +75,12 @@ uint64_t class_off(const nwc_handle_s& h, int cls) {
 // `stream` (from pageable memory: the call returns once the bytes are staged).
 nwc_status write_schedule(nwc_handle_s* h, int cls, const nwc::LaunchShape& s,
                           cudaStream_t stream) {
-  std::vector<uint8_t> sched(nwc::sched_class_bytes((uint64_t)h->tiles));
+  std::vector<uint8_t> sched;
+  try {
+    sched.resize(nwc::sched_class_bytes((uint64_t)h->tiles));
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
   nwc::build_schedule(h->index.data(), h->tiles, s, sched.data());
   if (cudaMemcpyAsync(h->d_base + class_off(*h, cls), sched.data(), sched.size(),
                       cudaMemcpyHostToDevice, stream) != cudaSuccess)
@@ -98,6 +104,17 @@ nwc_status shape_for(nwc_handle_s* h, int cls, nwc::LaunchShape* s, cudaStream_t
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// parse_blob with host allocation failures (the index copy) reported as NOMEM:
+// no C++ exception leaves the C ABI.
+nwc_status parse(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* h,
+                 const uint8_t** lens) {
+  try {
+    return nwc::parse_blob(blob, head_bytes, bytes, h, lens) ? NWC_OK : NWC_ERR_CORRUPT;
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
+}
 
 nwc::TileParams base_params(const nwc_handle_s& h, int cls, const nwc::LaunchShape& s) {
   nwc::TileParams p;
@@ -134,9 +151,10 @@ uint64_t workspace_bytes_for(const nwc_handle_s& h, int32_t batch) {
 nwc_status make_handle(const uint8_t* blob_host_header_region, uint64_t bytes, void* d_buf,
                        uint64_t d_bytes, nwc_handle_t* out, const uint8_t** lens) {
   nwc_handle_s tmp;
-  if (!nwc::parse_blob(blob_host_header_region, bytes, bytes, &tmp, lens)) return NWC_ERR_CORRUPT;
+  const nwc_status st = parse(blob_host_header_region, bytes, bytes, &tmp, lens);
+  if (st != NWC_OK) return st;
   if (d_bytes < tmp.device_bytes) return NWC_ERR_INVALID_ARG;
-  nwc_handle_s* h = new (std::nothrow) nwc_handle_s(tmp);
+  nwc_handle_s* h = new (std::nothrow) nwc_handle_s(std::move(tmp));
   if (!h) return NWC_ERR_NOMEM;
   h->d_base = static_cast<uint8_t*>(d_buf);
   h->d_bytes = d_bytes;
@@ -278,8 +296,9 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
 nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes, uint64_t* device_bytes) {
   if (!blob || !device_bytes) return NWC_ERR_INVALID_ARG;
   nwc_handle_s tmp;
-  if (!nwc::parse_blob(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &tmp, nullptr))
-    return NWC_ERR_CORRUPT;
+  const nwc_status st = parse(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &tmp,
+                              nullptr);
+  if (st != NWC_OK) return st;
   *device_bytes = tmp.device_bytes;
   return NWC_OK;
 }
@@ -293,7 +312,13 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, u
   nwc_status st = make_handle(static_cast<const uint8_t*>(blob), blob_bytes, d_buf, d_bytes, &h,
                               &lens);
   if (st != NWC_OK) return st;
-  std::vector<uint32_t> table(nwc::table_entries(h->lmax));
+  std::vector<uint32_t> table;
+  try {
+    table.resize(nwc::table_entries(h->lmax));
+  } catch (const std::bad_alloc&) {
+    delete h;
+    return NWC_ERR_NOMEM;
+  }
   nwc::build_decode_table(lens, h->lmax, table.data());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(d_buf, blob, blob_bytes, cudaMemcpyHostToDevice, s);
@@ -328,19 +353,24 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
       hd.tiles_off < nwc::kIndexOffset)
     return NWC_ERR_CORRUPT;
   // Header, lens and index; the tile area is not read back.
-  std::vector<uint8_t> head(hd.tiles_off);
+  std::vector<uint8_t> head;
+  try {
+    head.resize(hd.tiles_off);
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
   if (cudaMemcpy(head.data(), d_buf, hd.tiles_off, cudaMemcpyDeviceToHost) != cudaSuccess)
     return NWC_ERR_CUDA;
   nwc_handle_s tmp;
-  if (!nwc::parse_blob(head.data(), head.size(), hd.total_bytes, &tmp, nullptr))
-    return NWC_ERR_CORRUPT;
+  nwc_status st = parse(head.data(), head.size(), hd.total_bytes, &tmp, nullptr);
+  if (st != NWC_OK) return st;
   if (d_bytes < tmp.device_bytes) return NWC_ERR_INVALID_ARG;
-  nwc_handle_s* h = new (std::nothrow) nwc_handle_s(tmp);
+  nwc_handle_s* h = new (std::nothrow) nwc_handle_s(std::move(tmp));
   if (!h) return NWC_ERR_NOMEM;
   h->d_base = static_cast<uint8_t*>(d_buf);
   h->d_bytes = d_bytes;
   cudaGetDevice(&h->device);
-  nwc_status st = init_schedule(h, nullptr, nullptr);
+  st = init_schedule(h, nullptr, nullptr);
   if (st == NWC_OK && cudaStreamSynchronize(nullptr) != cudaSuccess) st = NWC_ERR_CUDA;
   if (st != NWC_OK) {
     delete h;
@@ -492,11 +522,11 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
       rows_of_x < 0 || rows_of_x > nwc::kMaxPassRows)
     return NWC_ERR_INVALID_ARG;
   nwc_handle_s h;
-  if (!nwc::parse_blob(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &h, nullptr))
-    return NWC_ERR_CORRUPT;
+  nwc_status st = parse(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &h, nullptr);
+  if (st != NWC_OK) return st;
   const int cls = nwc::stage_class(rows_of_x);
   nwc::LaunchShape s;
-  nwc_status st = shape_on(h, sm_count, (size_t)smem_limit, cls, &s);
+  st = shape_on(h, sm_count, (size_t)smem_limit, cls, &s);
   if (st != NWC_OK) return st;
   std::vector<uint8_t> sched;
   try {
