@@ -244,6 +244,24 @@ def nwc_handle_destroy(handle) -> None:
 
 # ---- convenience object over the same calls ---------------------------------
 
+def _require(t, what: str, dtypes, shape, device, pinned_host_ok: bool = False) -> None:
+    """Host-side checks of a tensor handed to a kernel: a tensor on another
+    device, of another type or shape would otherwise be read or written out of
+    bounds on the GPU."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{what}: dtype {t.dtype}, expected one of {[str(d) for d in dtypes]}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{what}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{what}: must be contiguous")
+    if t.device != device and not (pinned_host_ok and t.device.type == "cpu" and t.is_pinned()):
+        where = f"{device} or pinned host memory" if pinned_host_ok else str(device)
+        raise ValueError(f"{what}: on {t.device}, expected {where}")
+
+
 class CompressedMatrix:
     """A BF16 matrix held compressed in device memory that torch allocated.
 
@@ -296,32 +314,55 @@ class CompressedMatrix:
             self._ws = torch.zeros(need, dtype=torch.uint8, device=self.image.device)
         return self._ws, self._ws.numel()
 
+    def _open(self) -> None:
+        if self.handle is None:
+            raise ValueError("the compressed matrix is closed")
+
     def decompress(self, out=None, stream=None):
+        """W as BF16 [rows, cols] (out may also be int16 or uint16: the bit patterns)."""
         import torch
+        self._open()
         if out is None:
             out = torch.empty((self.rows, self.cols), dtype=torch.bfloat16,
                               device=self.image.device)
+        _require(out, "out", (torch.bfloat16, torch.int16, torch.uint16), (self.rows, self.cols),
+                 self.image.device)
         nwc_decompress(self.handle, out, stream)
         return out
 
     def gemv(self, x, y=None, stream=None):
-        """y = x @ W^T for x BF16 [batch, cols] -> FP32 [batch, rows]."""
+        """y = x @ W^T for x BF16 [..., cols] on the matrix's device -> FP32
+        [batch, rows], batch = x.numel() // cols.  y, when given, is FP32
+        [batch, rows] on that device or in pinned host memory."""
         import torch
-        assert x.dtype == torch.bfloat16 and x.is_contiguous() and x.shape[-1] == self.cols
+        self._open()
+        if not isinstance(x, torch.Tensor) or x.dim() < 1 or x.shape[-1] != self.cols:
+            raise ValueError(f"x: expected a tensor [..., {self.cols}]")
         xb = x.reshape(-1, self.cols)
         batch = xb.shape[0]
+        if not 1 <= batch <= 64:
+            raise ValueError(f"x: {batch} rows; a call takes 1 to 64")
+        _require(xb, "x", (torch.bfloat16,), (batch, self.cols), self.image.device)
         if y is None:
-            y = torch.empty((batch, self.rows), dtype=torch.float32, device=x.device)
+            y = torch.empty((batch, self.rows), dtype=torch.float32, device=self.image.device)
+        _require(y, "y", (torch.float32,), (batch, self.rows), self.image.device,
+                 pinned_host_ok=True)
         ws, ws_bytes = self.workspace(batch)
         nwc_gemv(self.handle, xb, y, batch, ws, ws_bytes, stream)
         return y
 
     def gather_rows(self, rows, stream=None):
-        """BF16 rows W[rows] (torch.int32 ids on the device) -> [len(rows), cols]."""
+        """BF16 rows W[rows] -> [len(rows), cols]; integer ids, moved to the
+        matrix's device.  An id outside [0, rows) makes the kernel skip that row
+        and set the device error word (see nwc_get_device_error)."""
         import torch
-        rows = rows.to(torch.int32).contiguous()
-        out = torch.empty((rows.numel(), self.cols), dtype=torch.bfloat16, device=rows.device)
-        nwc_gather_rows(self.handle, rows, rows.numel(), out, stream)
+        self._open()
+        if not isinstance(rows, torch.Tensor) or rows.dtype.is_floating_point or rows.dim() != 1:
+            raise TypeError("rows: expected a 1-D integer tensor")
+        ids = rows.to(device=self.image.device, dtype=torch.int32).contiguous()
+        out = torch.empty((ids.numel(), self.cols), dtype=torch.bfloat16, device=self.image.device)
+        if ids.numel():
+            nwc_gather_rows(self.handle, ids, ids.numel(), out, stream)
         return out
 
     def close(self) -> None:

@@ -239,6 +239,11 @@ def test_invalid_arguments_rejected(lib):
     blob = np.zeros(1024, dtype=np.uint8)
     with pytest.raises(lib.NwcError):
         lib.CompressedMatrix.from_blob(blob)
+    with pytest.raises(ValueError):              # x in host memory never reaches a kernel
+        m.gemv(torch.zeros((1, 1024), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):              # nor a y smaller than the output
+        m.gemv(x, y=torch.zeros((1, 15), dtype=torch.float32, device="cuda"))
+    assert m.gather_rows(torch.tensor([3, 0])).shape == (2, 1024)  # host ids are moved
     no_device_error(lib)
 
 

@@ -72,3 +72,45 @@ def test_host_validation(lib):
     bad = np.zeros(512, dtype=np.uint8)
     with pytest.raises(lib.NwcError):
         lib.nwc_blob_device_bytes(bad)
+
+
+def test_compressed_matrix_checks_tensors_on_the_host(lib, monkeypatch):
+    """CompressedMatrix refuses tensors of the wrong type, shape or device before
+    any library call (the image lives on the meta device here, so a call that
+    got through would fail loudly)."""
+    torch = pytest.importorskip("torch")
+    monkeypatch.setattr(lib, "nwc_handle_destroy", lambda h: None)
+    rows, cols = 24, 40
+    m = lib.CompressedMatrix(torch.empty(256, dtype=torch.uint8, device="meta"), object(),
+                             rows, cols, 256)
+    meta = dict(device="meta")
+    with pytest.raises(TypeError):
+        m.gemv(torch.zeros((2, cols), dtype=torch.float32, **meta))
+    with pytest.raises(ValueError):
+        m.gemv(torch.zeros((2, cols + 1), dtype=torch.bfloat16, **meta))
+    with pytest.raises(ValueError):   # the host copy of x is not on the matrix's device
+        m.gemv(torch.zeros((2, cols), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):   # more rows of x than one call takes
+        m.gemv(torch.zeros((65, cols), dtype=torch.bfloat16, **meta))
+    x = torch.zeros((3, cols), dtype=torch.bfloat16, **meta)
+    with pytest.raises(ValueError):
+        m.gemv(x, y=torch.zeros((3, rows + 1), dtype=torch.float32, **meta))
+    with pytest.raises(TypeError):
+        m.gemv(x, y=torch.zeros((3, rows), dtype=torch.bfloat16, **meta))
+    with pytest.raises(ValueError):   # pageable host memory is not a valid y
+        m.gemv(x, y=torch.zeros((3, rows), dtype=torch.float32))
+    with pytest.raises(ValueError):
+        m.gemv(x, y=torch.zeros((rows, 3), dtype=torch.float32, **meta).t())
+    with pytest.raises(ValueError):
+        m.decompress(out=torch.empty((rows, cols + 1), dtype=torch.bfloat16, **meta))
+    with pytest.raises(ValueError):
+        m.decompress(out=torch.empty((rows, cols), dtype=torch.bfloat16))
+    with pytest.raises(TypeError):
+        m.decompress(out=torch.empty((rows, cols), dtype=torch.float16, **meta))
+    with pytest.raises(TypeError):
+        m.gather_rows(torch.zeros(3, dtype=torch.float32))
+    empty = m.gather_rows(torch.zeros(0, dtype=torch.int64))
+    assert empty.shape == (0, cols) and empty.dtype == torch.bfloat16
+    m.handle = None
+    with pytest.raises(ValueError):
+        m.gemv(x)
