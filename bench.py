@@ -533,9 +533,13 @@ def main():
     elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world)
     clock = clocks.summary()
 
-    # Average launch duration of the GEMV kernel: event pairs around direct
-    # launches on its stream, queued behind a GPU sleep so that the intervals
-    # hold the kernels only (not host submission gaps).
+    # The timed region holds GEMV launches only, so their average duration there
+    # is the region's event time over its launches (consecutive launches overlap
+    # their prologue with the previous tail).  For comparison, the duration of
+    # one launch on its own: event pairs around direct launches on the stream,
+    # queued behind a GPU sleep so that the intervals hold the kernels, not host
+    # submission gaps.
+    kernel_ms = elapsed_ms / (steps * launches_per_call)
     durs = []
     n_timed = min(256, 8 * copies)
     for _ in range(4):
@@ -549,7 +553,7 @@ def main():
                 ev[i][1].record(stream)
         stream.synchronize()
         durs += [a.elapsed_time(b) for a, b in ev]
-    kernel_ms = statistics.mean(durs) / launches_per_call
+    isolated_ms = statistics.mean(durs) / launches_per_call
     ms_per_step = elapsed_ms / steps
 
     # Parity spot check of the timed configuration.
@@ -662,6 +666,8 @@ def main():
                      "frac": achieved / hbm, "traffic": traffic,
                      "peak_source": f"{peak_src} hbm_gbs (copy)",
                      "kernel": "gemv_kernel", "kernel_us": kernel_ms * 1e3,
+                     "basis": "algorithmic bytes per launch / timed-region event time per launch",
+                     "isolated_launch_us": isolated_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg_bytes},
         "clocks": clock,
         "e2e": e2e,
