@@ -142,7 +142,11 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
 
 /* ---- Device kernels ---------------------------------------------------- */
 
-/* nwc_decompress, nwc_gemv and nwc_gemv_noalloc launch one persistent CTA per
+/* A handle belongs to the device that was current when it was made (the one
+ * holding its image); the calls below return INVALID_ARG when another device is
+ * current.
+ *
+ * nwc_decompress, nwc_gemv and nwc_gemv_noalloc launch one persistent CTA per
  * SM (at most 256).  Should the current device's launch shape differ from the
  * one the image's schedule was written for, the call first rewrites that
  * schedule on `stream` (a host-to-device copy, in stream order).

@@ -266,7 +266,8 @@ class CompressedMatrix:
     """A BF16 matrix held compressed in device memory that torch allocated.
 
     Owns the device image (a uint8 CUDA tensor), the handle, and a GEMV
-    workspace that grows on demand.  Calls run on the current torch stream."""
+    workspace that grows on demand.  Calls make the image's device current and
+    run on that device's current torch stream (or the stream given)."""
 
     def __init__(self, image, handle, rows: int, cols: int, blob_bytes: int):
         self.image = image
@@ -327,7 +328,8 @@ class CompressedMatrix:
                               device=self.image.device)
         _require(out, "out", (torch.bfloat16, torch.int16, torch.uint16), (self.rows, self.cols),
                  self.image.device)
-        nwc_decompress(self.handle, out, stream)
+        with torch.cuda.device(self.image.device):
+            nwc_decompress(self.handle, out, stream)
         return out
 
     def gemv(self, x, y=None, stream=None):
@@ -348,7 +350,8 @@ class CompressedMatrix:
         _require(y, "y", (torch.float32,), (batch, self.rows), self.image.device,
                  pinned_host_ok=True)
         ws, ws_bytes = self.workspace(batch)
-        nwc_gemv(self.handle, xb, y, batch, ws, ws_bytes, stream)
+        with torch.cuda.device(self.image.device):
+            nwc_gemv(self.handle, xb, y, batch, ws, ws_bytes, stream)
         return y
 
     def gather_rows(self, rows, stream=None):
@@ -362,7 +365,8 @@ class CompressedMatrix:
         ids = rows.to(device=self.image.device, dtype=torch.int32).contiguous()
         out = torch.empty((ids.numel(), self.cols), dtype=torch.bfloat16, device=self.image.device)
         if ids.numel():
-            nwc_gather_rows(self.handle, ids, ids.numel(), out, stream)
+            with torch.cuda.device(self.image.device):
+                nwc_gather_rows(self.handle, ids, ids.numel(), out, stream)
         return out
 
     def close(self) -> None:

@@ -89,13 +89,15 @@ nwc_status write_schedule(nwc_handle_s* h, int cls, const nwc::LaunchShape& s,
   return NWC_OK;
 }
 
-// Launch geometry of class cls on the current device; rewrites that class's
-// schedule (in stream order) when it was made for another shape.
+// Launch geometry of class cls on the current device, which must be the
+// handle's (the one current when it was made: its image lives there); rewrites
+// that class's schedule (in stream order) when it was made for another shape.
 nwc_status shape_for(nwc_handle_s* h, int cls, nwc::LaunchShape* s, cudaStream_t stream) {
   int dev, sms;
   size_t smem;
   nwc_status st = current_device(&dev, &sms, &smem);
   if (st != NWC_OK) return st;
+  if (dev != h->device) return NWC_ERR_INVALID_ARG;
   st = shape_on(*h, sms, smem, cls, s);
   if (st != NWC_OK) return st;
   std::lock_guard<std::mutex> lk(g_mu);
@@ -396,6 +398,9 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
   if (!h || !d_rows || !d_out || n < 1 || n > (1 << 20) || !aligned(d_rows, 4) ||
       !aligned(d_out, 2))
     return NWC_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;
+  if (dev != h->device) return NWC_ERR_INVALID_ARG;
   nwc::GatherParams g;
   std::memset(&g, 0, sizeof(g));
   g.tiles = h->d_base + h->tiles_off;
