@@ -118,15 +118,20 @@ nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob
                              uint64_t blob_bytes);
 
 /* Bytes of device memory needed to upload an existing blob (the device image:
- * blob + decode table + launch schedule). */
+ * blob + decode table + launch schedule).  Host only; the blob is checked as
+ * nwc_upload_blob checks it.
+ * Errors: INVALID_ARG (null), CORRUPT (the blob does not parse: a header field
+ * inconsistent with the others or with blob_bytes, code lengths over lmax or
+ * not a prefix code, an index that is not increasing or whose chunk sizes fall
+ * outside what the geometry allows), NOMEM (the host copy of the index). */
 nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes,
                                  uint64_t* device_bytes);
 
 /* Validate a host blob, upload it into d_buf, and build its decode table and
  * launch schedule for the current device.  The call is synchronous: it returns
  * after the copies finish.
- * Errors: CORRUPT (header, code lengths or index do not parse), INVALID_ARG,
- * CUDA. */
+ * Errors: CORRUPT (header, code lengths or index do not parse, as for
+ * nwc_blob_device_bytes), INVALID_ARG, NOMEM, CUDA. */
 nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
                            uint64_t d_bytes, nwc_stream_t stream,
                            nwc_handle_t* out_handle);
@@ -136,7 +141,7 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
  * synchronous: it reads the header, code lengths and index back to the host,
  * then rewrites the image's launch-schedule area for the current device (the
  * blob and the decode table are not written).
- * Errors: CORRUPT, INVALID_ARG, CUDA. */
+ * Errors: CORRUPT, INVALID_ARG, NOMEM, CUDA. */
 nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
                                   nwc_handle_t* out_handle);
 
