@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--e2e-mode", default="host-y", choices=["copy", "host-y"],
                     help="how y reaches the host in the end-to-end leg")
+    ap.add_argument("--fuse", action="store_true",
+                    help="stacks: q, k, v and gate, up each run as one stacked matrix")
     return ap.parse_args()
 
 
@@ -271,20 +273,29 @@ def run_stack(args) -> None:
     lm_head, captured as one CUDA graph; a step is one token.  Layer weights:
     layer 0 of the workload, generated once, compressed once and held as two
     device copies that alternate between layers (a layer is larger than L2, so
-    every read is cold); the lm_head is its first rows repeated (synth)."""
+    every read is cold); the lm_head is its first rows repeated (synth).  With
+    --fuse, the projections that read the same input (q, k, v; gate, up) are
+    one matrix each, their rows stacked, compressed under one code table and
+    multiplied in one call (the cuBLAS leg uses the same stacked shapes)."""
     import torch
 
     from lossless_bf16_weight_nwc_b200 import _lib, synth
     rank, world = dist_setup(args.gpus)
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl, layer0, head, n_layers = synth.stack_parts(args.workload)
+    wl, layer0_parts, head, n_layers = synth.stack_parts(args.workload)
+    units = (synth.fused_layer(layer0_parts) if args.fuse
+             else [(m.name.rsplit(".", 1)[-1], [m]) for m in layer0_parts])
+    layer0 = [synth.MatrixSpec(f"layers.0.{g}", sum(p.rows for p in ps), ps[0].cols, ps[0].kind,
+                               ps[0].std, ps[0].tensor) for g, ps in units]
+    parts_of = {sp.name: ps for sp, (_, ps) in zip(layer0, units)}
     batch = args.batch
     steps = args.steps if args.steps is not None else 50
     specs = layer0 + [head]
     host_w = {}
     comp = {}
     for sp in specs:
-        host_w[sp.name] = synth.head_matrix(sp, wl.seed) if sp is head else synth.matrix(sp, wl.seed)
+        host_w[sp.name] = (synth.head_matrix(sp, wl.seed) if sp is head
+                           else synth.stacked_matrix(parts_of[sp.name], wl.seed))
         comp[sp.name] = _lib.CompressedMatrix.compress(host_w[sp.name], device=dev)
     sets = [{sp.name: comp[sp.name] for sp in layer0}]
     second = {}
@@ -337,11 +348,12 @@ def run_stack(args) -> None:
     torch.cuda.synchronize()
     ms_per_token = max_over_ranks(t0.elapsed_time(t1), world) / steps
 
-    # Parity spot check: the lm_head and the first down projection, sampled rows.
+    # Parity spot check: the lm_head, the layer's first and last matrices
+    # (q or the stacked qkv; down), sampled rows.
     parity_ok = True
     if rank == 0:
         import oracle
-        for sp in (head, layer0[-1]):
+        for sp in (head, layer0[0], layer0[-1]):
             xh = synth.activations(wl.seed, batch, sp.cols)
             comp[sp.name].gemv(torch.from_numpy(xh.view(np.int16)).view(torch.bfloat16).to(dev),
                                y=ys[sp.rows])
@@ -431,6 +443,8 @@ def run_stack(args) -> None:
         "data": "synthetic",
         "config": {"workload": args.workload, "batch": batch, "step": f"one token: {len(seq)} GEMVs "
                    f"({n_layers} layers x {len(layer0)} + lm_head), one CUDA graph",
+                   "layer": [f"{g} {sp.rows}x{sp.cols}" for (g, _), sp in zip(units, layer0)],
+                   "fused": bool(args.fuse),
                    "weights": "layer 0 generated, two device copies alternating over the layers; "
                               f"lm_head = its first {synth.HEAD_BLOCK_ROWS} rows repeated",
                    "l2": "inputs larger than L2: every layer is larger than L2",

@@ -275,6 +275,7 @@ class CompressedMatrix:
         self.rows, self.cols = rows, cols
         self.blob_bytes = blob_bytes
         self.device_bytes = image.numel()
+        self.row_splits = [0, rows]  # first output row of each part, then rows
         self._ws = None
 
     @classmethod
@@ -290,6 +291,27 @@ class CompressedMatrix:
         finally:
             nwc_plan_destroy(plan)
         return cls(image, h, w_host.shape[0], w_host.shape[1], blob_bytes)
+
+    @classmethod
+    def compress_fused(cls, parts, device="cuda", lmax: int = 0, tile_cols: int = 512,
+                       threads: int = 0, stream=None) -> "CompressedMatrix":
+        """Projections that read the same input (q, k, v; gate, up) held as one
+        matrix: the parts' rows stacked in order under one code table, so that a
+        call is one launch ("NWC — Neural Weight Compression", "Install": fuse
+        before convert).  row_splits holds each part's first output row; split()
+        cuts a result into the parts' outputs."""
+        ws = [np.ascontiguousarray(p, dtype=np.uint16) for p in parts]
+        if not ws or any(w.ndim != 2 or w.shape[1] != ws[0].shape[1] for w in ws):
+            raise ValueError("parts: one or more 2-D matrices with the same number of columns")
+        m = cls.compress(np.concatenate(ws, axis=0), device=device, lmax=lmax,
+                         tile_cols=tile_cols, threads=threads, stream=stream)
+        m.row_splits = [int(v) for v in np.cumsum([0] + [w.shape[0] for w in ws])]
+        return m
+
+    def split(self, y):
+        """The parts' outputs: views of y's last dimension at row_splits."""
+        b = self.row_splits
+        return [y[..., b[i]:b[i + 1]] for i in range(len(b) - 1)]
 
     @classmethod
     def from_blob(cls, blob: np.ndarray, device="cuda", stream=None) -> "CompressedMatrix":

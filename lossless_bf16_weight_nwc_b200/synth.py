@@ -223,6 +223,41 @@ def stack_parts(name: str):
     return wl, layer0, head, layers
 
 
+# Projections of a layer that read the same input, run as one matrix whose rows
+# are the parts' rows in this order ("NWC — Neural Weight Compression",
+# "Install": fuse(model) before convert(model); "Run a model": --fusion).
+FUSED_GROUPS = (("qkv", ("q", "k", "v")), ("gate_up", ("gate", "up")))
+
+
+def fused_layer(layer: list[MatrixSpec]) -> list[tuple[str, list[MatrixSpec]]]:
+    """A layer's matrices as (name, parts) in layer order: each group of
+    FUSED_GROUPS present in the layer becomes one entry at the place of its first
+    part; every other matrix stands alone."""
+    by_short = {m.name.rsplit(".", 1)[-1]: m for m in layer}
+    group_of = {part: (g, parts) for g, parts in FUSED_GROUPS
+                if all(p in by_short for p in parts) for part in parts}
+    out, done = [], set()
+    for m in layer:
+        short = m.name.rsplit(".", 1)[-1]
+        if short not in group_of:
+            out.append((short, [m]))
+            continue
+        g, parts = group_of[short]
+        if g in done:
+            continue
+        members = [by_short[p] for p in parts]
+        if len({p.cols for p in members}) != 1:
+            raise ValueError(f"{g}: parts read inputs of different widths")
+        out.append((g, members))
+        done.add(g)
+    return out
+
+
+def stacked_matrix(parts: list[MatrixSpec], seed: int) -> np.ndarray:
+    """The parts' generated matrices with their rows stacked in order."""
+    return np.ascontiguousarray(np.concatenate([matrix(p, seed) for p in parts], axis=0))
+
+
 def head_matrix(spec: MatrixSpec, seed: int) -> np.ndarray:
     """The lm_head as its first HEAD_BLOCK_ROWS generated rows, repeated."""
     block = matrix(spec, seed, 0, min(HEAD_BLOCK_ROWS, spec.rows))

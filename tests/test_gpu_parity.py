@@ -153,6 +153,23 @@ def test_gemv_deterministic_and_workspace_reuse(lib, orc):
     no_device_error(lib)
 
 
+@pytest.mark.parametrize("batch", [1, 16])
+def test_fused_projections(lib, orc, batch):
+    """q, k, v stacked into one matrix (one code table, one call): each part's
+    slice of y meets the tolerance against that part alone."""
+    parts = [synth.MatrixSpec(f"layers.0.{n}", r, 1536, "normal", 0.02, t)
+             for t, (n, r) in enumerate((("q", 512), ("k", 128), ("v", 128)))]
+    ws = [synth.matrix(p, 9) for p in parts]
+    m = lib.CompressedMatrix.compress_fused(ws)
+    assert m.row_splits == [0, 512, 640, 768] and m.rows == 768
+    assert np.array_equal(bits(m.decompress()), np.concatenate(ws))
+    x = synth.activations(9, batch, 1536)
+    ys = m.split(m.gemv(to_bf16(x)))
+    for w, y in zip(ws, ys):
+        tolerance_check(y.cpu().numpy(), orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
 def test_gemv_into_pinned_host_memory(lib, orc):
     """y may be pinned host memory the device can address: the kernel stores the
     result there directly."""
