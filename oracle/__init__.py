@@ -73,6 +73,13 @@ def _declare(h: ctypes.CDLL) -> ctypes.CDLL:
     h.orc_decode_tiles.argtypes = [u8p, i64, i64, i64, u16p, i64]
     h.orc_gemv.argtypes = [u16p, i64, i64, u16p, c.c_int, i64, i64,
                            c.POINTER(c.c_double)]
+    h.orc_rank_table.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, u8p,
+                                 c.POINTER(c.c_int)]
+    h.orc_rank_blob_size.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int,
+                                     c.POINTER(i64)]
+    h.orc_rank_encode.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, u8p,
+                                  i64, c.POINTER(i64)]
+    h.orc_rank_decode.argtypes = [u8p, i64, u16p, i64]
     return h
 
 
@@ -237,3 +244,50 @@ def gemv(w: np.ndarray, x: np.ndarray, row_begin: int = 0,
     _check(lib().orc_gemv(_ptr(w, ctypes.c_uint16), rows, cols, _ptr(x, ctypes.c_uint16),
                           batch, row_begin, row_end, _ptr(y, ctypes.c_double)), "gemv")
     return y
+
+
+# ---- variant NWR1: the ranked unary code -----------------------------------
+
+def rank_table(w: np.ndarray, tile_cols: int = 512, ranks: int = 7,
+               tile_rows: int = 8) -> list[int]:
+    """The values of exponent bits 14..8 that get ranks, in rank order."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, cols = w.shape
+    table = np.zeros(7, dtype=np.uint8)
+    n = ctypes.c_int()
+    _check(lib().orc_rank_table(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows, tile_cols,
+                                ranks, _ptr(table, ctypes.c_uint8), ctypes.byref(n)),
+           "rank_table")
+    return [int(v) for v in table[:n.value]]
+
+
+def rank_encode(w: np.ndarray, tile_cols: int = 512, ranks: int = 7,
+                tile_rows: int = 8) -> np.ndarray:
+    """BF16 bit patterns [rows, cols] -> NWR1 blob (uint8 array)."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, cols = w.shape
+    size = ctypes.c_int64()
+    _check(lib().orc_rank_blob_size(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows,
+                                    tile_cols, ranks, ctypes.byref(size)), "rank_blob_size")
+    blob = np.zeros(size.value, dtype=np.uint8)
+    got = ctypes.c_int64()
+    _check(lib().orc_rank_encode(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows, tile_cols,
+                                 ranks, _ptr(blob, ctypes.c_uint8), blob.size,
+                                 ctypes.byref(got)), "rank_encode")
+    assert got.value == blob.size
+    return blob
+
+
+def rank_decode(blob: np.ndarray) -> np.ndarray:
+    """NWR1 blob -> BF16 bit patterns [rows, cols]."""
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    if blob.size < 32:
+        raise OracleError(ORC_E_CORRUPT, "rank_decode")
+    rows = int.from_bytes(blob[16:24].tobytes(), "little")
+    cols = int.from_bytes(blob[24:32].tobytes(), "little")
+    if not (1 <= rows <= 1 << 32 and 1 <= cols <= 1 << 32) or rows * cols > 1 << 34:
+        raise OracleError(ORC_E_CORRUPT, "rank_decode")
+    out = np.zeros((rows, cols), dtype=np.uint16)
+    _check(lib().orc_rank_decode(_ptr(blob, ctypes.c_uint8), blob.size,
+                                 _ptr(out, ctypes.c_uint16), out.size), "rank_decode")
+    return out

@@ -62,6 +62,36 @@
  *   Lane t = 4 g + c (g = t / 4, c = t mod 4) owns row g of the tile: its k-th
  *   symbol is the element at row g and column 64 * (k / 16) + 16 c + (k mod 16),
  *   i.e. in every 64-column group the lane's 16 consecutive columns, in order.
+ *
+ * Variant "NWR1", the ranked unary code ("NWC", "How it works > Prefix code
+ * instead of rANS": format v9 ranks the exponent by frequency and writes a
+ * unary rank code plus a raw sign bit, with an escape for rare values):
+ *
+ *  1. Planes of the literal byte split ("NWC", "How it works > Byte planes": the
+ *     byte holding the sign and the exponent is coded, the other byte stored):
+ *     the coded field e = exponent bits 14..8 (7 bits) with the sign bit 15
+ *     beside it; the raw byte is bits 7..0 (the exponent's lowest bit and the
+ *     fraction).
+ *  2. Ranks: the values of e ordered by count over the real weights and the
+ *     fillers, largest count first, smaller value first on a tie; the first
+ *     R = min(ranks, number of values present) of them get ranks 0 .. R - 1,
+ *     with ranks in 1..7 (a code then has at most 15 bits and a lane's stream
+ *     at most 240 bytes).
+ *  3. Code of a weight, most significant bit first: its sign bit; then, if its
+ *     e has rank r < R, r zero bits and a one bit; otherwise R zero bits and
+ *     the 7 bits of e (the escape).
+ *  4. Tiles, lanes, chunk layout, index and stream packing are those of NWB1;
+ *     the raw plane holds bits 7..0.  Filler positions hold sign 0, the rank-0
+ *     value of e and raw byte 0.
+ *
+ *   header differences from NWB1: magic 0x3152574E ("NWR1"); offset 12 holds
+ *   R; offset 56 the rank-0 value of e (the filler's); offset 96 the total
+ *   code bits; the 256 bytes at offset 128 hold the ranked values of e, rank
+ *   order, then zeros.
+ *
+ * Readings where the v9 passage is silent: the sign bit comes first, a rank is
+ * counted in zero bits ended by a one, the escape is the 7-bit field after R
+ * zero bits, R = 7 by default.
  */
 #include "nwc_oracle.h"
 
@@ -371,6 +401,261 @@ int decode_impl(const uint8_t* blob, int64_t size, int64_t u0, int64_t u1,
   return ORC_OK;
 }
 
+/* ---- Variant NWR1: the ranked unary code ---------------------------------- */
+
+const uint32_t kRankMagic = 0x3152574Eu;
+const int kMaxRanks = 7;
+
+/* Literal byte split: e = exponent bits 14..8, the sign bit 15, raw = bits 7..0. */
+void rank_split(uint16_t w, int* e, int* sign, uint8_t* raw) {
+  *e = (w >> 8) & 0x7F;
+  *sign = (w >> 15) & 1;
+  *raw = (uint8_t)(w & 0xFF);
+}
+
+uint16_t rank_join(int e, int sign, uint8_t raw) {
+  return (uint16_t)(((uint16_t)sign << 15) | ((uint16_t)e << 8) | raw);
+}
+
+/* Values of e by count (largest first, smaller value on a tie); at most
+ * `ranks` of those present.  Returns how many were ranked. */
+int rank_order(const uint64_t cnt[128], int ranks, uint8_t table[kMaxRanks]) {
+  std::vector<int> present;
+  for (int e = 0; e < 128; ++e)
+    if (cnt[e] > 0) present.push_back(e);
+  std::stable_sort(present.begin(), present.end(),
+                   [&](int a, int b) { return cnt[a] > cnt[b]; });
+  const int n = (int)std::min<size_t>(present.size(), (size_t)ranks);
+  for (int r = 0; r < n; ++r) table[r] = (uint8_t)present[(size_t)r];
+  return n;
+}
+
+/* Appends the code of one weight to a lane's bit list. */
+void rank_code_bits(int e, int sign, const uint8_t table[kMaxRanks], int ranks,
+                    std::vector<uint8_t>* bits) {
+  bits->push_back((uint8_t)sign);
+  int r = 0;
+  while (r < ranks && table[r] != e) ++r;
+  for (int z = 0; z < r; ++z) bits->push_back(0);
+  if (r < ranks) {
+    bits->push_back(1);
+  } else {
+    for (int b = 6; b >= 0; --b) bits->push_back((uint8_t)((e >> b) & 1));
+  }
+}
+
+int encode_rank_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                     int tile_cols, int ranks, uint8_t* blob, int64_t cap, int64_t* size) {
+  if (!w || rows < 1 || cols < 1 || !size) return ORC_E_ARG;
+  if (!geometry_ok(tile_rows, tile_cols, 12) || ranks < 1 || ranks > kMaxRanks)
+    return ORC_E_ARG;
+  const int64_t tiles_r = (rows + tile_rows - 1) / tile_rows;
+  const int64_t tiles_c = (cols + tile_cols - 1) / tile_cols;
+  const int64_t tiles = tiles_r * tiles_c;
+  const int lane_syms = 2 * tile_rows * (tile_cols / 64);
+  const int raw_bytes = tile_rows * tile_cols;
+
+  /* Counts of e over the real weights; the filler takes the most frequent
+   * value (smallest on a tie), then the fillers are counted. */
+  uint64_t cnt[128] = {};
+  for (int64_t q = 0; q < rows * cols; ++q) {
+    int e, sign;
+    uint8_t raw;
+    rank_split(w[q], &e, &sign, &raw);
+    cnt[e] += 1;
+  }
+  int filler = 0;
+  for (int e = 1; e < 128; ++e)
+    if (cnt[e] > cnt[filler]) filler = e;
+  cnt[filler] += (uint64_t)(tiles_r * tile_rows) * (uint64_t)(tiles_c * tile_cols) -
+                 (uint64_t)rows * (uint64_t)cols;
+  uint8_t table[kMaxRanks] = {};
+  const int R = rank_order(cnt, ranks, table);
+
+  const uint64_t table_off = kHeaderBytes;
+  const uint64_t index_off = table_off + 256;
+  const uint64_t tiles_off = round_up(index_off + 4 * (uint64_t)(tiles + 1), 256);
+  std::vector<uint32_t> index((size_t)tiles + 1);
+  uint64_t area = 0, code_bits = 0;
+  for (int64_t u = 0; u < tiles; ++u) {
+    const int64_t i = u % tiles_r, j = u / tiles_r;
+    std::vector<uint8_t> raw((size_t)raw_bytes, 0);
+    std::vector<uint8_t> seq;  /* one entry per bit */
+    uint8_t lane_bytes[kLanes];
+    for (int t = 0; t < kLanes; ++t) {
+      std::vector<uint8_t> lb;
+      for (int k = 0; k < lane_syms; ++k) {
+        int r, c;
+        lane_symbol_position(t, k, &r, &c);
+        const int64_t row = i * tile_rows + r, col = j * tile_cols + c;
+        int e = filler, sign = 0;
+        uint8_t rb = 0;
+        if (row < rows && col < cols) rank_split(w[row * cols + col], &e, &sign, &rb);
+        raw[(size_t)raw_position(t, k)] = rb;
+        rank_code_bits(e, sign, table, R, &lb);
+      }
+      code_bits += lb.size();
+      while (lb.size() % 8 != 0) lb.push_back(0);
+      lane_bytes[t] = (uint8_t)(lb.size() / 8);
+      seq.insert(seq.end(), lb.begin(), lb.end());
+    }
+    while (seq.size() % 128 != 0) seq.push_back(0);
+    std::vector<uint8_t> bits(seq.size() / 8, 0);
+    for (size_t b = 0; b < seq.size(); ++b) {
+      if (!seq[b]) continue;
+      const int bit = 31 - (int)(b % 32);
+      bits[(b / 32) * 4 + (size_t)(bit / 8)] |= (uint8_t)(1u << (bit % 8));
+    }
+    index[(size_t)u] = (uint32_t)(area / 16);
+    const uint64_t chunk = (uint64_t)raw_bytes + kLanes + bits.size();
+    if (blob) {
+      if ((int64_t)(tiles_off + area + chunk) > cap) return ORC_E_SPACE;
+      uint8_t* p = blob + tiles_off + area;
+      std::memcpy(p, raw.data(), raw.size());
+      std::memcpy(p + raw_bytes, lane_bytes, kLanes);
+      std::memcpy(p + raw_bytes + kLanes, bits.data(), bits.size());
+    }
+    area += chunk;
+    if (area / 16 > 0xFFFFFFFFull) return ORC_E_ARG;
+  }
+  index[(size_t)tiles] = (uint32_t)(area / 16);
+  const uint64_t total = tiles_off + area;
+  *size = (int64_t)total;
+  if (!blob) return ORC_OK;
+  if ((int64_t)total > cap) return ORC_E_SPACE;
+  std::memset(blob, 0, (size_t)tiles_off);
+  put_u32(blob + 0, kRankMagic);
+  put_u32(blob + 4, kVersion);
+  put_u32(blob + 8, kHeaderBytes);
+  put_u32(blob + 12, (uint32_t)R);
+  put_u64(blob + 16, (uint64_t)rows);
+  put_u64(blob + 24, (uint64_t)cols);
+  put_u32(blob + 32, (uint32_t)tile_rows);
+  put_u32(blob + 36, (uint32_t)tile_cols);
+  put_u64(blob + 40, (uint64_t)tiles_r);
+  put_u64(blob + 48, (uint64_t)tiles_c);
+  put_u32(blob + 56, (uint32_t)filler);
+  put_u64(blob + 64, table_off);
+  put_u64(blob + 72, index_off);
+  put_u64(blob + 80, tiles_off);
+  put_u64(blob + 88, total);
+  put_u64(blob + 96, code_bits);
+  std::memcpy(blob + table_off, table, (size_t)R);
+  for (int64_t u = 0; u <= tiles; ++u) put_u32(blob + index_off + 4 * u, index[(size_t)u]);
+  return ORC_OK;
+}
+
+int decode_rank_impl(const uint8_t* blob, int64_t size, uint16_t* out, int64_t cap_elems) {
+  if (!blob || size < kHeaderBytes + 256) return ORC_E_CORRUPT;
+  if (get_u32(blob) != kRankMagic || get_u32(blob + 4) != kVersion ||
+      get_u32(blob + 8) != (uint32_t)kHeaderBytes)
+    return ORC_E_CORRUPT;
+  const int R = (int)get_u32(blob + 12);
+  const int64_t rows = (int64_t)get_u64(blob + 16), cols = (int64_t)get_u64(blob + 24);
+  const int tile_rows = (int)get_u32(blob + 32), tile_cols = (int)get_u32(blob + 36);
+  const int64_t tiles_r = (int64_t)get_u64(blob + 40), tiles_c = (int64_t)get_u64(blob + 48);
+  const int filler = (int)get_u32(blob + 56);
+  const uint64_t table_off = get_u64(blob + 64), index_off = get_u64(blob + 72);
+  const uint64_t tiles_off = get_u64(blob + 80), total = get_u64(blob + 88);
+  if (rows < 1 || cols < 1 || !geometry_ok(tile_rows, tile_cols, 12)) return ORC_E_CORRUPT;
+  if (R < 1 || R > kMaxRanks) return ORC_E_CORRUPT;
+  if (tiles_r != (rows + tile_rows - 1) / tile_rows ||
+      tiles_c != (cols + tile_cols - 1) / tile_cols)
+    return ORC_E_CORRUPT;
+  const int64_t tiles = tiles_r * tiles_c;
+  if (table_off != (uint64_t)kHeaderBytes || index_off != table_off + 256 ||
+      tiles_off != round_up(index_off + 4 * (uint64_t)(tiles + 1), 256) ||
+      total != (uint64_t)size)
+    return ORC_E_CORRUPT;
+  /* The ranked values: distinct 7-bit values, then zeros; rank 0 is the filler's. */
+  uint8_t table[kMaxRanks] = {};
+  for (int r = 0; r < 256; ++r) {
+    const uint8_t v = blob[table_off + (uint64_t)r];
+    if (r >= R) {
+      if (v) return ORC_E_CORRUPT;
+      continue;
+    }
+    if (v > 127) return ORC_E_CORRUPT;
+    for (int q = 0; q < r; ++q)
+      if (table[q] == v) return ORC_E_CORRUPT;
+    table[r] = v;
+  }
+  if (filler != table[0]) return ORC_E_CORRUPT;
+  if (!out || cap_elems < rows * cols) return ORC_E_SPACE;
+
+  const int lane_syms = 2 * tile_rows * (tile_cols / 64);
+  const int raw_bytes = tile_rows * tile_cols;
+  const uint64_t area = (uint64_t)size - tiles_off;
+  for (int64_t u = 0; u < tiles; ++u) {
+    const uint64_t c0 = 16ull * get_u32(blob + index_off + 4 * u);
+    const uint64_t c1 = 16ull * get_u32(blob + index_off + 4 * (u + 1));
+    if (c1 < c0 || c1 > area || c1 - c0 < (uint64_t)raw_bytes + kLanes) return ORC_E_CORRUPT;
+    const uint8_t* chunk = blob + tiles_off + c0;
+    const uint8_t* raw = chunk;
+    const uint8_t* lane_bytes = chunk + raw_bytes;
+    const uint8_t* bits = chunk + raw_bytes + kLanes;
+    uint64_t stream_bytes = 0;
+    for (int t = 0; t < kLanes; ++t) stream_bytes += lane_bytes[t];
+    if (c1 - c0 != (uint64_t)raw_bytes + kLanes + round_up(stream_bytes, 16))
+      return ORC_E_CORRUPT;
+    auto bit_at = [&](uint64_t q) -> int {
+      const int b = 31 - (int)(q % 32);
+      return (bits[(q / 32) * 4 + (uint64_t)(b / 8)] >> (b % 8)) & 1;
+    };
+    const int64_t i = u % tiles_r, j = u / tiles_r;
+    uint64_t lane_start = 0;
+    for (int t = 0; t < kLanes; ++t) {
+      uint64_t pos = lane_start;
+      const uint64_t end = lane_start + 8ull * lane_bytes[t];
+      auto next = [&](int* bit) -> bool {
+        if (pos >= end) return false;
+        *bit = bit_at(pos++);
+        return true;
+      };
+      for (int k = 0; k < lane_syms; ++k) {
+        int sign, b, zeros = 0, e;
+        if (!next(&sign)) return ORC_E_CORRUPT;
+        bool ended = false;
+        while (zeros < R) {
+          if (!next(&b)) return ORC_E_CORRUPT;
+          if (b) {
+            ended = true;
+            break;
+          }
+          ++zeros;
+        }
+        if (ended) {
+          e = table[zeros];
+        } else {
+          e = 0;
+          for (int q = 0; q < 7; ++q) {
+            if (!next(&b)) return ORC_E_CORRUPT;
+            e = (e << 1) | b;
+          }
+          for (int q = 0; q < R; ++q)
+            if (table[q] == e) return ORC_E_CORRUPT; /* a ranked value is never escaped */
+        }
+        const uint8_t rb = raw[raw_position(t, k)];
+        int r, c;
+        lane_symbol_position(t, k, &r, &c);
+        const int64_t row = i * tile_rows + r, col = j * tile_cols + c;
+        if (row < rows && col < cols) {
+          out[row * cols + col] = rank_join(e, sign, rb);
+        } else if (sign != 0 || e != filler || rb != 0) {
+          return ORC_E_CORRUPT;
+        }
+      }
+      if (end - pos >= 8) return ORC_E_CORRUPT;
+      while (pos < end)
+        if (bit_at(pos++)) return ORC_E_CORRUPT;
+      lane_start = end;
+    }
+    for (uint64_t q = lane_start; q < 8 * round_up(stream_bytes, 16); ++q)
+      if (bit_at(q)) return ORC_E_CORRUPT;
+  }
+  return ORC_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -535,6 +820,35 @@ int orc_gemv(const uint16_t* w, int64_t rows, int64_t cols, const uint16_t* x,
     }
   }
   return ORC_OK;
+}
+
+int orc_rank_table(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                   int tile_cols, int ranks, uint8_t table[7], int* n) {
+  /* The ranked values and their number, read back from an encoded header. */
+  int64_t size = 0;
+  int rc = encode_rank_impl(w, rows, cols, tile_rows, tile_cols, ranks, nullptr, 0, &size);
+  if (rc != ORC_OK) return rc;
+  std::vector<uint8_t> blob((size_t)size);
+  rc = encode_rank_impl(w, rows, cols, tile_rows, tile_cols, ranks, blob.data(), size, &size);
+  if (rc != ORC_OK) return rc;
+  *n = (int)get_u32(blob.data() + 12);
+  std::memcpy(table, blob.data() + kHeaderBytes, 7);
+  return ORC_OK;
+}
+
+int orc_rank_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                       int tile_cols, int ranks, int64_t* size) {
+  return encode_rank_impl(w, rows, cols, tile_rows, tile_cols, ranks, nullptr, 0, size);
+}
+
+int orc_rank_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                    int tile_cols, int ranks, uint8_t* blob, int64_t cap, int64_t* size) {
+  if (!blob) return ORC_E_ARG;
+  return encode_rank_impl(w, rows, cols, tile_rows, tile_cols, ranks, blob, cap, size);
+}
+
+int orc_rank_decode(const uint8_t* blob, int64_t size, uint16_t* w_out, int64_t cap_elems) {
+  return decode_rank_impl(blob, size, w_out, cap_elems);
 }
 
 }  // extern "C"

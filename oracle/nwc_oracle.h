@@ -21,9 +21,9 @@
  *         "Fused kernel" (blocks of 8 rows x 512 columns, one bit stream per
  *         lane, padding for any shape).
  *
- * The format these functions write and read ("NWB1") is stated field by
- * field at the top of nwc_oracle.cpp.  Status codes: 0 = OK, negative =
- * error (see ORC_E_*).
+ * The formats these functions write and read ("NWB1", and the variant "NWR1"
+ * of [NWC]'s ranked unary code) are stated field by field at the top of
+ * nwc_oracle.cpp.  Status codes: 0 = OK, negative = error (see ORC_E_*).
  */
 #ifndef NWC_ORACLE_H
 #define NWC_ORACLE_H
@@ -78,6 +78,19 @@ int orc_decode_tiles(const uint8_t* blob, int64_t size, int64_t tile_begin,
  * row_end); x is BF16 [batch x cols]; y is FP64 [batch x rows]. */
 int orc_gemv(const uint16_t* w, int64_t rows, int64_t cols, const uint16_t* x,
              int batch, int64_t row_begin, int64_t row_end, double* y);
+
+/* Variant "NWR1" (stated at the top of nwc_oracle.cpp): [NWC] "Prefix code
+ * instead of rANS", format v9 — exponent bits 14..8 ranked by frequency in a
+ * unary code with the sign as a raw bit and an escape, bits 7..0 raw.  ranks
+ * in 1..7.  orc_rank_table gives the ranked values (rank order) and their
+ * number. */
+int orc_rank_table(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                   int tile_cols, int ranks, uint8_t table[7], int* n);
+int orc_rank_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                       int tile_cols, int ranks, int64_t* size);
+int orc_rank_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                    int tile_cols, int ranks, uint8_t* blob, int64_t cap, int64_t* size);
+int orc_rank_decode(const uint8_t* blob, int64_t size, uint16_t* w_out, int64_t cap_elems);
 
 #ifdef __cplusplus
 }
