@@ -59,13 +59,29 @@ typedef enum {
   NWC_ERR_SCRATCH_LIMIT = 8   /* nwc_gemv_noalloc: scratch needed > the limit   */
 } nwc_status;
 
+/* Exponent codes (nwc_opts.code). */
+typedef enum {
+  /* "NWB1": exponent bits 14..7 in a length-limited canonical prefix code;
+   * sign and fraction raw.  Every call of this library takes it. */
+  NWC_CODE_PREFIX = 0,
+  /* "NWR1": exponent bits 14..8 ranked by count in a unary code with the sign
+   * bit beside it and an escape ("NWC", "How it works > Prefix code instead of
+   * rANS", format v9); bits 7..0 raw.  Host encoder only for now: nwc_plan,
+   * nwc_plan_size (device_bytes = 0) and nwc_compress_host take it; the calls
+   * that need a device image return UNSUPPORTED. */
+  NWC_CODE_RANK = 1
+} nwc_code;
+
 /* Plan options.  Set struct_size = sizeof(nwc_opts); pass NULL for the defaults
- * (lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0 meaning all cores).
- * lmax: 0 = automatic (7, or the smallest limit that admits every distinct
- * exponent when there are more than 128), else in [1, 12] and at least
- * ceil(log2(distinct exponents)).  With lmax <= 7 the decoder peeks 14 bits and
- * every peek holds two complete codes; with 8..12 it peeks 12 bits and takes a
- * second lookup when a pair does not fit.
+ * (lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0 meaning all cores,
+ * code = NWC_CODE_PREFIX).  A struct_size that ends before `code` (the layout
+ * without it) means NWC_CODE_PREFIX.
+ * lmax, NWC_CODE_PREFIX: 0 = automatic (7, or the smallest limit that admits
+ * every distinct exponent when there are more than 128), else in [1, 12] and at
+ * least ceil(log2(distinct exponents)).  With lmax <= 7 the decoder peeks 14
+ * bits and every peek holds two complete codes; with 8..12 it peeks 12 bits and
+ * takes a second lookup when a pair does not fit.
+ * lmax, NWC_CODE_RANK: the number of ranks, 0 = 7, else in [1, 7].
  * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512. */
 typedef struct {
   uint32_t struct_size;
@@ -73,6 +89,7 @@ typedef struct {
   uint32_t tile_rows;
   uint32_t tile_cols;
   uint32_t threads; /* host encoder threads; 0 = hardware concurrency */
+  uint32_t code;    /* nwc_code */
 } nwc_opts;
 
 /* Library version: major * 10000 + minor * 100 + patch. */

@@ -36,10 +36,13 @@ class nwc_schedule_info(ctypes.Structure):
                 ("smem_bytes", ctypes.c_uint64), ("xstage_bytes", ctypes.c_uint32)]
 
 
+NWC_CODE_PREFIX, NWC_CODE_RANK = 0, 1
+
+
 class nwc_opts(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("lmax", ctypes.c_uint32),
                 ("tile_rows", ctypes.c_uint32), ("tile_cols", ctypes.c_uint32),
-                ("threads", ctypes.c_uint32)]
+                ("threads", ctypes.c_uint32), ("code", ctypes.c_uint32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -113,10 +116,13 @@ def nwc_version() -> int:
     return LIB.nwc_version()
 
 
-def nwc_plan(w_host: np.ndarray, lmax: int = 0, tile_cols: int = 512, threads: int = 0):
+def nwc_plan(w_host: np.ndarray, lmax: int = 0, tile_cols: int = 512, threads: int = 0,
+             code: int = NWC_CODE_PREFIX):
+    """code NWC_CODE_RANK: the ranked unary code, lmax = number of ranks (0 = 7);
+    host encoder only (nwc_compress_host)."""
     w = np.ascontiguousarray(w_host, dtype=np.uint16)
     rows, cols = w.shape
-    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads)
+    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads, code)
     plan = ctypes.c_void_p()
     _check(LIB.nwc_plan(w.ctypes.data, rows, cols, ctypes.byref(opts), ctypes.byref(plan)),
            "nwc_plan")

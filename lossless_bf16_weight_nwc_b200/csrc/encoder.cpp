@@ -14,6 +14,10 @@
 //     out so that one 128-bit load gives a lane 16 of its raw bytes.
 //  5. A 4096-entry decode table for the GPU ("NWC", "Prefix code instead of
 //     rANS": a 12-bit peek yields up to two complete codes).
+// The variant NWR1 (plan_build_rank) replaces steps 1-3 with the ranked unary
+// code of "NWC", "Prefix code instead of rANS" (format v9): exponent bits
+// 14..8 ranked by count, the sign bit raw in the stream, bits 7..0 raw; step 4
+// is shared.
 #include <algorithm>
 #include <cstring>
 #include <functional>
@@ -60,6 +64,37 @@ struct TileView {
   inline uint16_t at(int r, int c) const { return w[(row0 + r) * cols + col0 + c]; }
 };
 
+// NWR1's coded field: exponent bits 14..8.
+inline uint32_t rank_field(uint16_t w) { return (w >> 8) & 0x7Fu; }
+
+// Code bits (right-aligned), their number and the raw byte of tile element
+// (r, c) under the plan's code; positions outside the matrix hold the filler
+// with a zero raw byte (and, for NWR1, sign 0).
+inline void symbol_of(const nwc_plan_s& p, const TileView& v, int r, int c, uint32_t* code,
+                      int* len, uint8_t* raw) {
+  const bool in = v.inside(r, c);
+  const uint16_t x = in ? v.at(r, c) : 0;
+  *raw = 0;
+  if (p.code_kind == 0) {
+    uint8_t s = v.filler;
+    if (in) {
+      s = exponent_byte(x);
+      *raw = raw_byte(x);
+    }
+    *code = p.code[s];
+    *len = p.len[s];
+    return;
+  }
+  uint32_t e = p.filler, sign = 0;
+  if (in) {
+    e = rank_field(x);
+    sign = x >> 15;
+    *raw = (uint8_t)(x & 0xFF);
+  }
+  *code = (sign << p.rank_len[e]) | p.rank_code[e];
+  *len = p.rank_len[e] + 1;
+}
+
 // Bits of each lane's stream in tile u.
 void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t bits[kLanes]) {
   const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
@@ -68,8 +103,13 @@ void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t bits[
   for (int r = 0; r < kTileRows; ++r) {
     for (int c = 0; c < (int)p.tile_cols; ++c) {
       const int t = 4 * r + (c % 64) / 16;  // lane t = 4 r + q owns row r, columns 16 q .. of a group
-      const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
-      bits[t] += p.len[s];
+      if (p.code_kind == 0) {
+        const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
+        bits[t] += p.len[s];
+      } else {
+        const uint32_t e = v.inside(r, c) ? rank_field(v.at(r, c)) : p.filler;
+        bits[t] += p.rank_len[e] + 1u;
+      }
     }
   }
 }
@@ -203,6 +243,8 @@ void build_decode_table(const uint8_t len[256], uint32_t lmax, uint32_t* table) 
   }
 }
 
+int plan_tiles(const uint16_t* w, nwc_plan_s* p);
+
 int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
                uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* p) {
   p->rows = rows;
@@ -255,8 +297,85 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   canonical_codes(p->len, p->code);
   p->coded_bits = 0;
   for (int s = 0; s < 256; ++s) p->coded_bits += cnt[s] * p->len[s];
+  const int rc = plan_tiles(w, p);
+  if (rc != 0) return rc;
+  p->table_off = round_up(p->blob_bytes, 256);
+  p->sched_off = round_up(p->table_off + table_bytes(p->lmax), 256);
+  p->device_bytes = p->sched_off + sched_bytes((uint64_t)p->tiles);
+  return 0;
+}
 
-  // Chunk sizes -> index.
+int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_cols,
+                    uint32_t ranks, uint32_t threads, nwc_plan_s* p) {
+  if (ranks < 1 || ranks > (uint32_t)kMaxRanks) return -1;
+  p->code_kind = 1;
+  p->rows = rows;
+  p->cols = cols;
+  p->tile_rows = kTileRows;
+  p->tile_cols = tile_cols;
+  p->threads = hardware_threads(threads);
+  p->tiles_r = (rows + kTileRows - 1) / kTileRows;
+  p->tiles_c = (cols + tile_cols - 1) / tile_cols;
+  p->tiles = p->tiles_r * p->tiles_c;
+
+  // Counts of e over the real weights, one partial per thread.
+  const unsigned nt = p->threads;
+  std::vector<std::vector<uint64_t>> part(nt, std::vector<uint64_t>(128, 0));
+  {
+    std::vector<std::thread> pool;
+    for (unsigned q = 0; q < nt; ++q) {
+      pool.emplace_back([&, q] {
+        const int64_t b = rows * q / nt, e = rows * (q + 1) / nt;
+        uint64_t* h = part[q].data();
+        for (int64_t r = b; r < e; ++r) {
+          const uint16_t* row = w + r * cols;
+          for (int64_t c = 0; c < cols; ++c) h[rank_field(row[c])] += 1;
+        }
+      });
+    }
+    for (auto& t : pool) t.join();
+  }
+  uint64_t cnt[128] = {};
+  for (unsigned q = 0; q < nt; ++q)
+    for (int e = 0; e < 128; ++e) cnt[e] += part[q][e];
+  // The filler is the most frequent value (smallest on a tie), counted too.
+  uint32_t filler = 0;
+  for (uint32_t e = 1; e < 128; ++e)
+    if (cnt[e] > cnt[filler]) filler = e;
+  p->filler = filler;
+  cnt[filler] += (uint64_t)(p->tiles_r * kTileRows) * (uint64_t)(p->tiles_c * tile_cols) -
+                 (uint64_t)rows * (uint64_t)cols;
+  // Ranks by count, largest first, smaller value first on a tie.
+  std::vector<int> present;
+  for (int e = 0; e < 128; ++e)
+    if (cnt[e]) present.push_back(e);
+  std::stable_sort(present.begin(), present.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  p->ranks = (uint32_t)std::min<size_t>(present.size(), ranks);
+  p->lmax = p->ranks;
+  // Code after the sign bit: rank r -> r zeros and a one; escape -> R zeros and e.
+  for (int e = 0; e < 128; ++e) {
+    p->rank_len[e] = (uint8_t)(p->ranks + 7);
+    p->rank_code[e] = (uint32_t)e;
+  }
+  for (uint32_t r = 0; r < p->ranks; ++r) {
+    const int e = present[r];
+    p->rank_table[r] = (uint8_t)e;
+    p->rank_len[e] = (uint8_t)(r + 1);
+    p->rank_code[e] = 1;
+  }
+  p->coded_bits = 0;
+  for (int e = 0; e < 128; ++e) p->coded_bits += cnt[e] * (uint64_t)(p->rank_len[e] + 1);
+  const int rc = plan_tiles(w, p);
+  if (rc != 0) return rc;
+  // No kernel reads this code yet: there is no device image.
+  p->table_off = p->sched_off = p->device_bytes = 0;
+  return 0;
+}
+
+// Chunk sizes -> index, tile-area offset and blob size (either code).
+int plan_tiles(const uint16_t* w, nwc_plan_s* p) {
+  const unsigned nt = p->threads;
+  const uint32_t tile_cols = p->tile_cols;
   std::vector<uint32_t> chunk16((size_t)p->tiles);
   parallel_for(p->tiles, nt, [&](int64_t b, int64_t e) {
     uint32_t bits[kLanes];
@@ -276,16 +395,13 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   p->index[(size_t)p->tiles] = (uint32_t)acc;
   p->tiles_off = round_up(kIndexOffset + 4ull * (uint64_t)(p->tiles + 1), 256);
   p->blob_bytes = p->tiles_off + 16ull * acc;
-  p->table_off = round_up(p->blob_bytes, 256);
-  p->sched_off = round_up(p->table_off + table_bytes(p->lmax), 256);
-  p->device_bytes = p->sched_off + sched_bytes((uint64_t)p->tiles);
   return 0;
 }
 
 void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
   BlobHeader h;
   std::memset(&h, 0, sizeof(h));
-  h.magic = kMagic;
+  h.magic = p.code_kind == 0 ? kMagic : kRankMagic;
   h.version = kVersion;
   h.header_bytes = kHeaderBytes;
   h.lmax = p.lmax;
@@ -303,7 +419,10 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
   h.coded_bits = p.coded_bits;
   std::memset(blob, 0, p.tiles_off);
   std::memcpy(blob, &h, sizeof(h));
-  std::memcpy(blob + kLensOffset, p.len, 256);
+  if (p.code_kind == 0)
+    std::memcpy(blob + kLensOffset, p.len, 256);
+  else
+    std::memcpy(blob + kLensOffset, p.rank_table, p.ranks);
   std::memcpy(blob + kIndexOffset, p.index.data(), 4 * p.index.size());
 
   const uint32_t groups = p.tile_cols / 64;
@@ -332,15 +451,13 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
           for (int kk = 0; kk < 16; ++kk) {
             const int c = (int)(64 * g) + 16 * (t % 4) + kk;
             const int k = (int)(16 * g) + kk;
-            uint8_t s = v.filler, rb = 0;
-            if (v.inside(r, c)) {
-              const uint16_t x = v.at(r, c);
-              s = exponent_byte(x);
-              rb = raw_byte(x);
-            }
+            uint32_t code;
+            int len;
+            uint8_t rb;
+            symbol_of(p, v, r, c, &code, &len, &rb);
             raw[(k / 16) * 512 + 16 * t + (k % 16)] = rb;
-            accb = (accb << p.len[s]) | p.code[s];
-            nacc += p.len[s];
+            accb = (accb << len) | code;
+            nacc += len;
             while (nacc >= 8) {
               seq[out++] = (uint8_t)(accb >> (nacc - 8));
               nacc -= 8;

@@ -4,6 +4,7 @@
 // Every device call runs on the caller's stream and allocates no device memory.
 #include <cuda_runtime.h>
 
+#include <cstddef>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -111,6 +112,12 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // no C++ exception leaves the C ABI.
 nwc_status parse(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* h,
                  const uint8_t** lens) {
+  // An NWR1 blob (ranked unary code) is well defined but no kernel reads it yet.
+  if (blob && head_bytes >= 4) {
+    uint32_t magic;
+    std::memcpy(&magic, blob, 4);
+    if (magic == nwc::kRankMagic) return NWC_ERR_UNSUPPORTED;
+  }
   try {
     return nwc::parse_blob(blob, head_bytes, bytes, h, lens) ? NWC_OK : NWC_ERR_CORRUPT;
   } catch (const std::bad_alloc&) {
@@ -214,14 +221,17 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
   if (!w_host || !out_plan || rows < 1 || cols < 1) return NWC_ERR_INVALID_ARG;
   if (rows > (1ll << 40) || cols > (1ll << 40)) return NWC_ERR_INVALID_ARG;
   *out_plan = nullptr;
-  uint32_t lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0;
+  uint32_t lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0, code = NWC_CODE_PREFIX;
   if (opts) {
-    if (opts->struct_size < sizeof(nwc_opts)) return NWC_ERR_INVALID_ARG;
+    if (opts->struct_size < offsetof(nwc_opts, code)) return NWC_ERR_INVALID_ARG;
     lmax = opts->lmax;
     tile_rows = opts->tile_rows;
     tile_cols = opts->tile_cols;
     threads = opts->threads;
+    if (opts->struct_size >= sizeof(nwc_opts)) code = opts->code;
   }
+  if (code != NWC_CODE_PREFIX && code != NWC_CODE_RANK) return NWC_ERR_INVALID_ARG;
+  if (code == NWC_CODE_RANK && lmax > (uint32_t)nwc::kMaxRanks) return NWC_ERR_INVALID_ARG;
   if (lmax > (uint32_t)nwc::kMaxLmax) return NWC_ERR_INVALID_ARG;
   if (tile_rows != 8) return NWC_ERR_UNSUPPORTED;
   if (tile_cols != 64 && tile_cols != 128 && tile_cols != 256 && tile_cols != 512)
@@ -230,7 +240,10 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
   if (!p) return NWC_ERR_NOMEM;
   int rc;
   try {
-    rc = nwc::plan_build(w_host, rows, cols, tile_rows, tile_cols, lmax, threads, p);
+    rc = code == NWC_CODE_RANK
+             ? nwc::plan_build_rank(w_host, rows, cols, tile_cols, lmax ? lmax : nwc::kMaxRanks,
+                                    threads, p)
+             : nwc::plan_build(w_host, rows, cols, tile_rows, tile_cols, lmax, threads, p);
   } catch (const std::bad_alloc&) {
     delete p;
     return NWC_ERR_NOMEM;
@@ -264,8 +277,9 @@ nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob
 nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, uint64_t d_bytes,
                         nwc_stream_t stream, nwc_handle_t* out_handle) {
   if (!plan || !w_host || !d_buf || !out_handle) return NWC_ERR_INVALID_ARG;
-  if (d_bytes < plan->device_bytes || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
   *out_handle = nullptr;
+  if (plan->code_kind != NWC_CODE_PREFIX) return NWC_ERR_UNSUPPORTED;  // no kernel reads it yet
+  if (d_bytes < plan->device_bytes || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
   uint8_t* img = static_cast<uint8_t*>(std::malloc(plan->device_bytes));
   if (!img) return NWC_ERR_NOMEM;
   try {
@@ -351,6 +365,7 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
   nwc::BlobHeader hd;
   if (cudaMemcpy(&hd, d_buf, sizeof(hd), cudaMemcpyDeviceToHost) != cudaSuccess)
     return NWC_ERR_CUDA;
+  if (hd.magic == nwc::kRankMagic) return NWC_ERR_UNSUPPORTED;  // no kernel reads it yet
   if (hd.magic != nwc::kMagic || hd.total_bytes > d_bytes || hd.tiles_off > hd.total_bytes ||
       hd.tiles_off < nwc::kIndexOffset)
     return NWC_ERR_CORRUPT;

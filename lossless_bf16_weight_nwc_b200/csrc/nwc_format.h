@@ -33,6 +33,16 @@
 namespace nwc {
 
 constexpr uint32_t kMagic = 0x3142574Eu;  // "NWB1"
+// Variant "NWR1": the ranked unary code ("NWC", "How it works > Prefix code
+// instead of rANS", format v9).  The same header, index, chunk layout and
+// stream packing as NWB1, with: the coded field e = exponent bits 14..8 and the
+// sign bit, the raw byte = bits 7..0; the header's lmax field holds R, the
+// number of ranks (1..7); its 256-byte lens area holds the ranked values of e
+// (R bytes in rank order, then zeros); its filler field the rank-0 value.  A
+// weight's code is its sign bit, then r zeros and a one for rank r < R, else R
+// zeros and the 7 bits of e.  Host encoder only: no kernel reads it yet.
+constexpr uint32_t kRankMagic = 0x3152574Eu;  // "NWR1"
+constexpr int kMaxRanks = 7;
 constexpr uint32_t kVersion = 1;
 constexpr uint32_t kHeaderBytes = 128;
 constexpr uint32_t kLensOffset = 128;

@@ -13,6 +13,13 @@ struct nwc_plan_s {
   uint32_t code[256] = {};
   uint32_t filler = 0;
   uint64_t coded_bits = 0;
+  // Exponent code: 0 = canonical prefix code of bits 14..7 (NWB1), 1 = ranked
+  // unary code of bits 14..8 with the sign bit (NWR1).
+  uint32_t code_kind = 0;
+  uint32_t ranks = 0;                        // NWR1: R
+  uint8_t rank_table[nwc::kMaxRanks] = {};   // NWR1: ranked values of e
+  uint8_t rank_len[128] = {};                // NWR1: bits after the sign bit
+  uint32_t rank_code[128] = {};              // NWR1: those bits, right-aligned
   std::vector<uint32_t> index;  // tiles + 1 entries, 16-byte units
   uint64_t tiles_off = 0;       // blob offset of the tile area
   uint64_t blob_bytes = 0;      // serialisable blob
@@ -43,6 +50,10 @@ namespace nwc {
 // Encoder steps (encoder.cpp).
 int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
                uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* plan);
+// The ranked unary code (NWR1) with `ranks` ranks (1..7); the plan has no
+// device image (device_bytes = 0).
+int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_cols,
+                    uint32_t ranks, uint32_t threads, nwc_plan_s* plan);
 void encode_blob(const nwc_plan_s& plan, const uint16_t* w, uint8_t* blob);
 bool code_lengths(const uint64_t cnt[256], uint32_t lmax, uint8_t len[256]);
 void canonical_codes(const uint8_t len[256], uint32_t code[256]);

@@ -8,6 +8,8 @@ import pytest
 from conftest import ROOT
 from lossless_bf16_weight_nwc_b200 import synth
 
+UNSUPPORTED = 2  # NWC_ERR_UNSUPPORTED
+
 
 @pytest.fixture(scope="module")
 def lib():
@@ -114,3 +116,57 @@ def test_compressed_matrix_checks_tensors_on_the_host(lib, monkeypatch):
     m.handle = None
     with pytest.raises(ValueError):
         m.gemv(x)
+
+
+@pytest.mark.parametrize("shape,tile_cols,ranks", [((1024, 1024), 512, 0), ((9, 513), 512, 7),
+                                                   ((77, 1030), 256, 3), ((8, 64), 64, 1),
+                                                   ((333, 200), 128, 7), ((1, 1), 512, 0)])
+def test_rank_code_encoder_byte_identical_to_oracle(lib, orc, shape, tile_cols, ranks):
+    """The ranked unary code (NWR1): the library's multithreaded host encoder
+    writes the oracle's bytes."""
+    w = synth.matrix(synth.MatrixSpec("w", shape[0], shape[1], "student_t5", 0.015, 3), 11)
+    plan = lib.nwc_plan(w, lmax=ranks, tile_cols=tile_cols, threads=3, code=lib.NWC_CODE_RANK)
+    try:
+        dev_bytes, blob_bytes = lib.nwc_plan_size(plan)
+        blob = lib.nwc_compress_host(plan, w)
+    finally:
+        lib.nwc_plan_destroy(plan)
+    ref = orc.rank_encode(w, tile_cols=tile_cols, ranks=ranks or 7)
+    assert dev_bytes == 0 and blob.size == blob_bytes == ref.size
+    assert np.array_equal(blob, ref)
+    assert np.array_equal(orc.rank_decode(blob), w)
+
+
+def test_rank_code_all_patterns_and_device_calls_refused(lib, orc):
+    import ctypes
+    w = np.arange(65536, dtype=np.uint16).reshape(256, 256)
+    plan = lib.nwc_plan(w, code=lib.NWC_CODE_RANK)
+    blob = lib.nwc_compress_host(plan, w)
+    assert np.array_equal(blob, orc.rank_encode(w))
+    # No kernel reads this code yet: every call that needs a device image says so.
+    h = ctypes.c_void_p()
+    st = lib.LIB.nwc_compress(plan, w.ctypes.data, 1 << 20, 1 << 30, None, ctypes.byref(h))
+    assert st == UNSUPPORTED and not h.value
+    lib.nwc_plan_destroy(plan)
+    for call in (lambda: lib.nwc_blob_device_bytes(blob), lambda: lib.nwc_schedule_describe(blob)):
+        with pytest.raises(lib.NwcError) as e:
+            call()
+        assert e.value.status == UNSUPPORTED
+
+
+def test_plan_options_code_field(lib):
+    import ctypes
+    w = synth.matrix(synth.MatrixSpec("w", 16, 256, "normal", 0.02, 0), 1)
+    with pytest.raises(lib.NwcError):
+        lib.nwc_plan(w, code=2)
+    with pytest.raises(lib.NwcError):                   # at most 7 ranks
+        lib.nwc_plan(w, lmax=8, code=lib.NWC_CODE_RANK)
+    # The options layout without `code` still means the prefix code.
+    opts = lib.nwc_opts(20, 0, 8, 512, 1, 1)
+    plan = ctypes.c_void_p()
+    assert lib.LIB.nwc_plan(w.ctypes.data, 16, 256, ctypes.byref(opts), ctypes.byref(plan)) == 0
+    blob = lib.nwc_compress_host(plan, w)
+    lib.nwc_plan_destroy(plan)
+    assert int.from_bytes(blob[:4].tobytes(), "little") == 0x3142574E
+    opts = lib.nwc_opts(16, 0, 8, 512, 1, 0)            # too short for `threads`
+    assert lib.LIB.nwc_plan(w.ctypes.data, 16, 256, ctypes.byref(opts), ctypes.byref(plan)) == 1
