@@ -4,7 +4,9 @@ lm_head, compressed through the C ABI, decompressed bit-exact (checked on the
 device against the original), and multiplied at the stack's batch sizes.  y
 is compared with the oracle's FP64 sum on 256 sampled rows of each matrix
 (first and last row included), with the tolerance of tests/test_gpu_parity.py.
-The lm_head is its first rows repeated (synth.head_matrix), at full shape."""
+The lm_head is its first rows repeated (synth.head_matrix), at full shape.
+The stacked projections the per-token benchmark runs with --fuse (qkv,
+gate_up) are checked the same way, part by part."""
 import numpy as np
 import pytest
 
@@ -43,5 +45,24 @@ def test_stack_shapes_full_size(lib, orc, name):
             x = synth.activations(wl.seed, batch, spec.cols)
             y = m.gemv(to_bf16(x)).cpu().numpy()
             tolerance_check(y[:, idx], orc.gemv(w[idx], x), w[idx], x)
+        m.close()
+        no_device_error(lib)
+
+
+@pytest.mark.parametrize("name", ["qwen3_4b_stack", "llama31_8b_stack"])
+def test_stacked_projections_full_size(lib, orc, name):
+    wl, layer0, _, _ = synth.stack_parts(name)
+    for group, parts in synth.fused_layer(layer0):
+        if len(parts) == 1:
+            continue
+        ws = [synth.matrix(p, wl.seed) for p in parts]
+        m = lib.CompressedMatrix.compress_fused(ws)
+        assert m.ratio >= 1.25, (group, m.ratio)
+        for batch in wl.batches:
+            x = synth.activations(wl.seed, batch, parts[0].cols)
+            ys = m.split(m.gemv(to_bf16(x)))
+            for p, w, y in zip(parts, ws, ys):
+                idx = np.unique(np.linspace(0, p.rows - 1, 128).astype(np.int64))
+                tolerance_check(y.cpu().numpy()[:, idx], orc.gemv(w[idx], x), w[idx], x)
         m.close()
         no_device_error(lib)
