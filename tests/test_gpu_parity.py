@@ -170,6 +170,21 @@ def test_fused_projections(lib, orc, batch):
     no_device_error(lib)
 
 
+def test_autotune_picks_a_timed_candidate(lib, orc):
+    """The format autotuner times real candidates on the device; the format it
+    picks meets the tolerance."""
+    from lossless_bf16_weight_nwc_b200 import autotune
+    spec = synth.MatrixSpec("w", 1024, 4096, "normal", 0.02, 0)
+    w = synth.matrix(spec, 3)
+    choice = autotune.Tuner().tune(w, 1, candidates=[(512, 0), (256, 0)], reps=5)
+    assert (choice.tile_cols, choice.lmax) in {(512, 0), (256, 0)}
+    assert set(choice.timings) == {"512/0", "256/0"} and min(choice.timings.values()) > 0
+    m = lib.CompressedMatrix.compress(w, tile_cols=choice.tile_cols, lmax=choice.lmax)
+    x = synth.activations(3, 1, spec.cols)
+    tolerance_check(m.gemv(to_bf16(x)).cpu().numpy(), orc.gemv(w, x), w, x)
+    no_device_error(lib)
+
+
 def test_gemv_into_pinned_host_memory(lib, orc):
     """y may be pinned host memory the device can address: the kernel stores the
     result there directly."""
