@@ -11,7 +11,12 @@ numbers:
 * a frequency-ranked unary code of exponent bits 14..8 with the sign as a raw
   bit and an escape for rare values ("NWC", "How it works > Prefix code instead
   of rANS", format v9): rank r < R costs r + 1 bits, the escape R bits plus the
-  7-bit field.
+  7-bit field;
+* verbatim escape rows ("Unweight", "Compressing BF16 Weights": a run of 64
+  weights holding a rare exponent is stored whole): the 16 most frequent
+  exponents get an optimal code (12-bit limit), a run of 64 consecutive weights
+  of a matrix row that holds any other exponent costs 16 bits per weight, and
+  every run carries a 1-bit flag.
 
 `PYTHONPATH=. python tests/test_format_variants_cpu.py` prints the table."""
 import numpy as np
@@ -44,6 +49,32 @@ def unary_rank_cost(cnt, ranks: int, literal_bits: int) -> float:
     return float((p * np.where(r < ranks, r + 1, ranks + literal_bits)).sum())
 
 
+def escape_rows_cost(orc, w: np.ndarray, common: int = 16, run: int = 64) -> float:
+    """Bits per weight of the verbatim-escape-row layout (see the module text):
+    runs of `run` weights along a row, the `common` most frequent exponents
+    coded, any run holding another exponent stored as 16-bit words."""
+    e = ((w.astype(np.int64) >> 7) & 0xFF)
+    cnt = np.bincount(e.reshape(-1), minlength=256)
+    keep = np.zeros(256, dtype=bool)
+    keep[sorted(range(256), key=lambda v: (-cnt[v], v))[:common]] = True
+    rows, cols = e.shape
+    pad = (-cols) % run
+    runs = np.pad(e, ((0, 0), (0, pad)), constant_values=int(np.argmax(cnt))).reshape(rows, -1, run)
+    rare_run = (~keep[runs]).any(axis=2)
+    coded = np.zeros(256, dtype=np.int64)
+    for v in range(256):
+        if keep[v]:
+            coded[v] = int(np.count_nonzero(runs[~rare_run] == v))
+    lengths = np.zeros(256)
+    if coded.sum():
+        full = np.zeros(256, dtype=np.uint64)
+        full[:] = coded
+        lengths = orc.code_lengths(full, 12).astype(np.float64)
+    code_bits = float((coded * lengths).sum()) + 8.0 * coded.sum()
+    verbatim_bits = 16.0 * run * rare_run.sum()
+    return (code_bits + verbatim_bits + rare_run.size) / (rows * (cols + pad))
+
+
 def variant_costs(orc, name: str, rows: int = 2048) -> dict:
     wl = synth.workload(name)
     spec = wl.matrices[0]
@@ -59,6 +90,7 @@ def variant_costs(orc, name: str, rows: int = 2048) -> dict:
         "rank_unary_R15": 8 + 1 + unary_rank_cost(exp7, 15, 7),
         "rank_unary_R7": 8 + 1 + unary_rank_cost(exp7, 7, 7),
         "exp7_optimal": 8 + 1 + _code_cost(orc, exp7, 12),
+        "escape_rows_top16": escape_rows_cost(orc, w.reshape(min(spec.rows, rows), spec.cols)),
     }
 
 
@@ -87,12 +119,29 @@ def test_variant_costs(orc, name):
     assert c["rank_unary_R15"] <= c["rank_unary_R7"]
     assert abs(c["rank_unary_R15"] - c["exp7_optimal"]) < 0.005
     assert c["rank_unary_R7"] - c["exp7_optimal"] < 0.02
+    # Escape rows: never below the complete optimal code of the same byte split.
+    assert c["escape_rows_top16"] >= c["this_lmax12"] - 1e-9
+
+
+def test_escape_rows_closed_forms(orc):
+    # One exponent only: a 1-bit code, the raw byte and one flag bit per run.
+    w = np.full((2, 128), 0x3F80, dtype=np.uint16)
+    assert escape_rows_cost(orc, w) == pytest.approx(8 + 1 + 1 / 64)
+    # Row 0 starts with 16 other exponents (0x30..0x3f, once each) and row 1
+    # holds 0xfe once.  The common 16 are 0x7f and 0x30..0x3e (ties go to the
+    # smaller value), so 0x3f and 0xfe are rare: runs (0, 0..63) and
+    # (1, 0..63) are verbatim, the other two runs hold only 0x7f (1-bit code).
+    w2 = w.copy()
+    w2[0, :16] = (np.arange(0x30, 0x40, dtype=np.uint16) << 7)
+    w2[1, 5] = 0x7F00
+    expected = (128 * (8 + 1) + 128 * 16 + 4) / 256
+    assert escape_rows_cost(orc, w2) == pytest.approx(expected)
 
 
 if __name__ == "__main__":
     import oracle
     keys = ["entropy_exp8", "this_lmax12", "this_lmax7", "literal_lmax12", "exp7_optimal",
-            "rank_unary_R15", "rank_unary_R7"]
+            "rank_unary_R15", "rank_unary_R7", "escape_rows_top16"]
     print("| workload | " + " | ".join(keys) + " |")
     print("|---" * (len(keys) + 1) + "|")
     for n in NAMES:
