@@ -185,6 +185,20 @@ def test_autotune_picks_a_timed_candidate(lib, orc):
     no_device_error(lib)
 
 
+def test_sharded_matrix_single_process(lib, orc):
+    """A row-sharded matrix in one process (world 1, no collective) runs the
+    library on its one shard and meets the tolerance."""
+    from lossless_bf16_weight_nwc_b200 import sharded
+    spec = synth.MatrixSpec("w", 300, 1024, "normal", 0.02, 0)
+    w = synth.matrix(spec, 7)
+    m = sharded.ShardedMatrix.compress(w)
+    assert m.ranges == [(0, 300)] and m.local is not None
+    x = synth.activations(7, 2, spec.cols)
+    tolerance_check(m.gemv(to_bf16(x)).cpu().numpy(), orc.gemv(w, x), w, x)
+    m.close()
+    no_device_error(lib)
+
+
 def test_gemv_into_pinned_host_memory(lib, orc):
     """y may be pinned host memory the device can address: the kernel stores the
     result there directly."""
