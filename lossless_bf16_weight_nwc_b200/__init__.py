@@ -3,7 +3,8 @@
 The product is the C-ABI library libnwc.so (include/nwc.h); `_lib` binds it
 with ctypes (loaded on first use, and it raises if the library is missing).
 `synth` generates the seeded synthetic inputs; `autotune` picks a matrix's
-tile width and code limit by timing the library's GEMV on the device.
+tile width and code limit by timing the library's GEMV on the device;
+`sharded` splits a matrix by output rows over a process group.
 """
 import importlib
 
