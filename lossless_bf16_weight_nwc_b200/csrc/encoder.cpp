@@ -491,6 +491,7 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   if (h.tiles_r != (h.rows + 7) / 8 || h.tiles_c != (h.cols + h.tile_cols - 1) / h.tile_cols)
     return false;
   if (h.lens_off != kLensOffset || h.index_off != kIndexOffset || h.filler > 255) return false;
+  if (h.zero != 0) return false;  // one bit stream per lane (the streams field, S - 1)
   // Every tile has a 4-byte index entry inside the head, which bounds the tile
   // count before it is formed: no size computed from it below can wrap around.
   const uint64_t max_tiles = head_bytes / 4;

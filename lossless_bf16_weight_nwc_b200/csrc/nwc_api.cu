@@ -112,11 +112,14 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // no C++ exception leaves the C ABI.
 nwc_status parse(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* h,
                  const uint8_t** lens) {
-  // An NWR1 blob (ranked unary code) is well defined but no kernel reads it yet.
-  if (blob && head_bytes >= 4) {
-    uint32_t magic;
+  // Well-defined layouts that no kernel reads yet: an NWR1 blob (ranked unary
+  // code), and NWB1 with 2 or 4 bit streams per lane (header offset 60 = S - 1).
+  if (blob && head_bytes >= 64) {
+    uint32_t magic, streams_m1;
     std::memcpy(&magic, blob, 4);
+    std::memcpy(&streams_m1, blob + 60, 4);
     if (magic == nwc::kRankMagic) return NWC_ERR_UNSUPPORTED;
+    if (magic == nwc::kMagic && (streams_m1 == 1 || streams_m1 == 3)) return NWC_ERR_UNSUPPORTED;
   }
   try {
     return nwc::parse_blob(blob, head_bytes, bytes, h, lens) ? NWC_OK : NWC_ERR_CORRUPT;
@@ -366,6 +369,7 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
   if (cudaMemcpy(&hd, d_buf, sizeof(hd), cudaMemcpyDeviceToHost) != cudaSuccess)
     return NWC_ERR_CUDA;
   if (hd.magic == nwc::kRankMagic) return NWC_ERR_UNSUPPORTED;  // no kernel reads it yet
+  if (hd.magic == nwc::kMagic && (hd.zero == 1 || hd.zero == 3)) return NWC_ERR_UNSUPPORTED;
   if (hd.magic != nwc::kMagic || hd.total_bytes > d_bytes || hd.tiles_off > hd.total_bytes ||
       hd.tiles_off < nwc::kIndexOffset)
     return NWC_ERR_CORRUPT;

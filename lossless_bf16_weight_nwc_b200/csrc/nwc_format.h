@@ -16,6 +16,10 @@
 // lane 16 consecutive columns of its row; the raw byte is at
 // (k/16) * 512 + 16 t + k%16.
 // Tiles are stored column-block-major: u = j * tiles_r + i.
+// The header's u32 at offset 60 (`zero`) holds S - 1 for S bit streams per
+// lane; the kernels read S = 1 only, and the C ABI answers UNSUPPORTED for 2
+// or 4 (a layout the format defines for a decoder that follows several streams
+// per lane at once).
 //
 // Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)]
 // | zero pad to 256 | launch schedules (sched_bytes(tiles) bytes: one per

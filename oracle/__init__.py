@@ -68,6 +68,10 @@ def _declare(h: ctypes.CDLL) -> ctypes.CDLL:
                                 c.POINTER(i64)]
     h.orc_encode.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, u8p,
                              i64, c.POINTER(i64)]
+    h.orc_blob_size_streams.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, c.c_int,
+                                        c.POINTER(i64)]
+    h.orc_encode_streams.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, c.c_int, u8p,
+                                     i64, c.POINTER(i64)]
     h.orc_blob_info.argtypes = [u8p, i64, c.POINTER(i64), c.POINTER(i64)]
     h.orc_decode.argtypes = [u8p, i64, u16p, i64]
     h.orc_decode_tiles.argtypes = [u8p, i64, i64, i64, u16p, i64]
@@ -173,26 +177,37 @@ def canonical_codes(lengths) -> np.ndarray:
 
 
 def blob_size(w: np.ndarray, tile_cols: int = 512, lmax: int = 12,
-              tile_rows: int = 8) -> int:
+              tile_rows: int = 8, streams: int = 1) -> int:
     w = np.ascontiguousarray(w, dtype=np.uint16)
     rows, cols = w.shape
     size = ctypes.c_int64()
-    _check(lib().orc_blob_size(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows,
-                               tile_cols, lmax, ctypes.byref(size)), "blob_size")
+    if streams == 1:
+        rc = lib().orc_blob_size(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows,
+                                 tile_cols, lmax, ctypes.byref(size))
+    else:
+        rc = lib().orc_blob_size_streams(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows,
+                                         tile_cols, lmax, streams, ctypes.byref(size))
+    _check(rc, "blob_size")
     return size.value
 
 
 def encode(w: np.ndarray, tile_cols: int = 512, lmax: int = 12,
-           tile_rows: int = 8) -> np.ndarray:
-    """BF16 bit patterns [rows, cols] -> blob (uint8 array)."""
+           tile_rows: int = 8, streams: int = 1) -> np.ndarray:
+    """BF16 bit patterns [rows, cols] -> blob (uint8 array); `streams` bit
+    streams per lane and tile (1, 2 or 4)."""
     w = np.ascontiguousarray(w, dtype=np.uint16)
     rows, cols = w.shape
-    n = blob_size(w, tile_cols, lmax, tile_rows)
+    n = blob_size(w, tile_cols, lmax, tile_rows, streams)
     blob = np.zeros(n, dtype=np.uint8)
     size = ctypes.c_int64()
-    _check(lib().orc_encode(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows, tile_cols,
-                            lmax, _ptr(blob, ctypes.c_uint8), n, ctypes.byref(size)),
-           "encode")
+    if streams == 1:
+        rc = lib().orc_encode(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows, tile_cols,
+                              lmax, _ptr(blob, ctypes.c_uint8), n, ctypes.byref(size))
+    else:
+        rc = lib().orc_encode_streams(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows,
+                                      tile_cols, lmax, streams, _ptr(blob, ctypes.c_uint8), n,
+                                      ctypes.byref(size))
+    _check(rc, "encode")
     assert size.value == n
     return blob
 

@@ -63,6 +63,15 @@
  *   symbol is the element at row g and column 64 * (k / 16) + 16 c + (k mod 16),
  *   i.e. in every 64-column group the lane's 16 consecutive columns, in order.
  *
+ *   Streams per lane.  The header's u32 at offset 60 holds S - 1, S in {1, 2,
+ *   4} (0: one stream per lane, as above).  With S streams per lane a tile has
+ *   32 S streams, stream t S + j belonging to lane t and carrying the lane's
+ *   symbols k with (k / 2) mod S == j, in k order: consecutive symbol pairs
+ *   go to the lane's streams in turn, so a decoder can follow S independent
+ *   streams at once.  The lens array of a chunk then has 32 S entries, in
+ *   stream order, and the streams follow one another in that order.  This is
+ *   a B200 layout choice, not the pages' (they give one stream per lane).
+ *
  * Variant "NWR1", the ranked unary code ("NWC", "How it works > Prefix code
  * instead of rANS": format v9 ranks the exponent by frequency and writes a
  * unary rank code plus a raw sign bit, with an escape for rare values):
@@ -159,11 +168,19 @@ int filler_symbol(const uint64_t cnt[256]) {
   return best;
 }
 
+/* Sub-stream of lane t that carries its k-th symbol when each lane has
+ * `streams` streams: consecutive symbol pairs go to the lane's streams in
+ * turn (see "Streams per lane" in the format statement). */
+int stream_of(int t, int k, int streams) { return t * streams + (k / 2) % streams; }
+
 /* The encoder proper; blob == nullptr only measures. */
 int encode_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
-                int tile_cols, int lmax, uint8_t* blob, int64_t cap, int64_t* size) {
+                int tile_cols, int lmax, int streams, uint8_t* blob, int64_t cap,
+                int64_t* size) {
   if (!w || rows < 1 || cols < 1 || !size) return ORC_E_ARG;
   if (!geometry_ok(tile_rows, tile_cols, lmax)) return ORC_E_ARG;
+  if (streams != 1 && streams != 2 && streams != 4) return ORC_E_ARG;
+  const int nstreams = kLanes * streams;
 
   const int64_t tiles_r = (rows + tile_rows - 1) / tile_rows;
   const int64_t tiles_c = (cols + tile_cols - 1) / tile_cols;
@@ -201,7 +218,7 @@ int encode_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
     const int64_t i = u % tiles_r; /* row block */
     const int64_t j = u / tiles_r; /* column block */
     std::vector<uint8_t> raw((size_t)raw_bytes, 0);
-    std::vector<std::vector<uint8_t> > lane_bits(kLanes);  /* one entry per bit */
+    std::vector<std::vector<uint8_t> > lane_bits((size_t)nstreams);  /* one entry per bit */
     for (int t = 0; t < kLanes; ++t) {
       for (int k = 0; k < lane_syms; ++k) {
         int r, c;
@@ -212,17 +229,17 @@ int encode_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
         if (row < rows && col < cols) orc_plane_split(w[row * cols + col], &s, &rb);
         raw[(size_t)raw_position(t, k)] = rb;
         for (int b = len[s] - 1; b >= 0; --b)
-          lane_bits[(size_t)t].push_back((uint8_t)((code[s] >> b) & 1u));
+          lane_bits[(size_t)stream_of(t, k, streams)].push_back((uint8_t)((code[s] >> b) & 1u));
       }
     }
-    /* Concatenate the byte-padded lane streams. */
+    /* Concatenate the byte-padded streams, in stream order. */
     std::vector<uint8_t> seq;  /* one entry per bit */
-    uint8_t lane_bytes[kLanes];
-    for (int t = 0; t < kLanes; ++t) {
+    std::vector<uint8_t> lane_bytes((size_t)nstreams);
+    for (int t = 0; t < nstreams; ++t) {
       std::vector<uint8_t>& lb = lane_bits[(size_t)t];
       while (lb.size() % 8 != 0) lb.push_back(0);
       if (lb.size() / 8 > 255) return ORC_E_ARG; /* cannot happen for lmax <= 12 */
-      lane_bytes[t] = (uint8_t)(lb.size() / 8);
+      lane_bytes[(size_t)t] = (uint8_t)(lb.size() / 8);
       seq.insert(seq.end(), lb.begin(), lb.end());
     }
     while (seq.size() % 128 != 0) seq.push_back(0); /* 16 bytes */
@@ -236,7 +253,7 @@ int encode_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
     }
     chunk.clear();
     chunk.insert(chunk.end(), raw.begin(), raw.end());
-    chunk.insert(chunk.end(), lane_bytes, lane_bytes + kLanes);
+    chunk.insert(chunk.end(), lane_bytes.begin(), lane_bytes.end());
     chunk.insert(chunk.end(), bits.begin(), bits.end());
     index[(size_t)u] = (uint32_t)(area / 16);
     if (area / 16 > 0xFFFFFFFFull) return ORC_E_ARG;
@@ -265,6 +282,7 @@ int encode_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
   put_u64(blob + 40, (uint64_t)tiles_r);
   put_u64(blob + 48, (uint64_t)tiles_c);
   put_u32(blob + 56, (uint32_t)filler);
+  put_u32(blob + 60, (uint32_t)(streams - 1));
   put_u64(blob + 64, lens_off);
   put_u64(blob + 72, index_off);
   put_u64(blob + 80, tiles_off);
@@ -277,7 +295,7 @@ int encode_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
 
 struct Header {
   int64_t rows, cols, tiles_r, tiles_c;
-  int tile_rows, tile_cols, lmax, filler;
+  int tile_rows, tile_cols, lmax, filler, streams;
   uint64_t lens_off, index_off, tiles_off, total;
 };
 
@@ -294,6 +312,7 @@ int read_header(const uint8_t* blob, int64_t size, Header* h) {
   h->tiles_r = (int64_t)get_u64(blob + 40);
   h->tiles_c = (int64_t)get_u64(blob + 48);
   h->filler = (int)get_u32(blob + 56);
+  h->streams = (int)get_u32(blob + 60) + 1;
   h->lens_off = get_u64(blob + 64);
   h->index_off = get_u64(blob + 72);
   h->tiles_off = get_u64(blob + 80);
@@ -303,6 +322,7 @@ int read_header(const uint8_t* blob, int64_t size, Header* h) {
   if (h->tiles_r != (h->rows + h->tile_rows - 1) / h->tile_rows) return ORC_E_CORRUPT;
   if (h->tiles_c != (h->cols + h->tile_cols - 1) / h->tile_cols) return ORC_E_CORRUPT;
   if (h->filler < 0 || h->filler > 255) return ORC_E_CORRUPT;
+  if (h->streams != 1 && h->streams != 2 && h->streams != 4) return ORC_E_CORRUPT;
   const uint64_t tiles = (uint64_t)(h->tiles_r * h->tiles_c);
   if (h->lens_off != (uint64_t)kHeaderBytes || h->index_off != h->lens_off + 256)
     return ORC_E_CORRUPT;
@@ -348,13 +368,14 @@ int decode_impl(const uint8_t* blob, int64_t size, int64_t u0, int64_t u1,
     if (c1 < c0 || c1 > area) return ORC_E_CORRUPT;
     const uint8_t* chunk = blob + h.tiles_off + c0;
     const uint64_t chunk_bytes = c1 - c0;
-    if (chunk_bytes < (uint64_t)raw_bytes + kLanes) return ORC_E_CORRUPT;
+    const int nstreams = kLanes * h.streams;
+    if (chunk_bytes < (uint64_t)raw_bytes + nstreams) return ORC_E_CORRUPT;
     const uint8_t* raw = chunk;
     const uint8_t* lane_bytes = chunk + raw_bytes;
-    const uint8_t* bits = chunk + raw_bytes + kLanes;
+    const uint8_t* bits = chunk + raw_bytes + nstreams;
     uint64_t stream_bytes = 0;
-    for (int t = 0; t < kLanes; ++t) stream_bytes += lane_bytes[t];
-    if (chunk_bytes != (uint64_t)raw_bytes + kLanes + round_up(stream_bytes, 16))
+    for (int t = 0; t < nstreams; ++t) stream_bytes += lane_bytes[t];
+    if (chunk_bytes != (uint64_t)raw_bytes + nstreams + round_up(stream_bytes, 16))
       return ORC_E_CORRUPT;
     const uint64_t nbits = 8 * round_up(stream_bytes, 16);
     /* Bit i of the sequence is bit 31 - i % 32 of little-endian word i / 32. */
@@ -365,10 +386,14 @@ int decode_impl(const uint8_t* blob, int64_t size, int64_t u0, int64_t u1,
     };
     const int64_t i = u % h.tiles_r, j = u / h.tiles_r;
     uint64_t lane_start = 0;
-    for (int t = 0; t < kLanes; ++t) {
+    for (int sigma = 0; sigma < nstreams; ++sigma) {
+      /* Stream sigma belongs to lane t and carries the lane's symbols k with
+       * stream_of(t, k) == sigma, in k order. */
+      const int t = sigma / h.streams;
       uint64_t pos = lane_start;
-      const uint64_t end = lane_start + 8ull * lane_bytes[t];
+      const uint64_t end = lane_start + 8ull * lane_bytes[sigma];
       for (int k = 0; k < lane_syms; ++k) {
+        if (stream_of(t, k, h.streams) != sigma) continue;
         /* Read bits one at a time until they spell a code. */
         uint32_t v = 0;
         int l = 0, s = -1;
@@ -769,13 +794,25 @@ int orc_canonical_codes(const uint8_t len[256], uint32_t code[256]) {
 
 int orc_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
                   int tile_cols, int lmax, int64_t* size) {
-  return encode_impl(w, rows, cols, tile_rows, tile_cols, lmax, nullptr, 0, size);
+  return encode_impl(w, rows, cols, tile_rows, tile_cols, lmax, 1, nullptr, 0, size);
+}
+
+int orc_blob_size_streams(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                          int tile_cols, int lmax, int streams, int64_t* size) {
+  return encode_impl(w, rows, cols, tile_rows, tile_cols, lmax, streams, nullptr, 0, size);
+}
+
+int orc_encode_streams(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                       int tile_cols, int lmax, int streams, uint8_t* blob, int64_t cap,
+                       int64_t* size) {
+  if (!blob) return ORC_E_ARG;
+  return encode_impl(w, rows, cols, tile_rows, tile_cols, lmax, streams, blob, cap, size);
 }
 
 int orc_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
                int tile_cols, int lmax, uint8_t* blob, int64_t cap, int64_t* size) {
   if (!blob) return ORC_E_ARG;
-  return encode_impl(w, rows, cols, tile_rows, tile_cols, lmax, blob, cap, size);
+  return encode_impl(w, rows, cols, tile_rows, tile_cols, lmax, 1, blob, cap, size);
 }
 
 int orc_blob_info(const uint8_t* blob, int64_t size, int64_t* rows, int64_t* cols) {

@@ -63,6 +63,14 @@ int orc_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
 int orc_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
                int tile_cols, int lmax, uint8_t* blob, int64_t cap, int64_t* size);
 
+/* The same with `streams` (1, 2 or 4) bit streams per lane and tile (format
+ * statement, "Streams per lane"); streams = 1 gives the bytes above. */
+int orc_blob_size_streams(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                          int tile_cols, int lmax, int streams, int64_t* size);
+int orc_encode_streams(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                       int tile_cols, int lmax, int streams, uint8_t* blob, int64_t cap,
+                       int64_t* size);
+
 /* Read rows/cols from a blob header (validates the header). */
 int orc_blob_info(const uint8_t* blob, int64_t size, int64_t* rows, int64_t* cols);
 

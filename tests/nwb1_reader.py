@@ -1,4 +1,5 @@
-"""A second, pure-Python reader of the NWB1 blob format (test helper).
+"""A second, pure-Python reader of the NWB1 blob format (test helper), with 1,
+2 or 4 bit streams per lane.
 
 Written from the format statement alone, in a different language and style
 from the oracle's C++ decoder, so that the encoder is checked against the
@@ -15,12 +16,15 @@ def parse(blob: bytes):
         "<IIIIQQIIQQIIQQQQQ", b, 0)
     assert magic == 0x3142574E and version == 1 and hdr == 128, "header"
     assert total == len(b), "total bytes"
+    streams = zero + 1              # bit streams per lane and tile
+    assert streams in (1, 2, 4), "streams per lane"
     lens = list(b[lens_off:lens_off + 256])
     n_tiles = tiles_r * tiles_c
     index = struct.unpack_from(f"<{n_tiles + 1}I", b, index_off)
     return dict(lmax=lmax, rows=rows, cols=cols, tile_rows=tile_rows, tile_cols=tile_cols,
                 tiles_r=tiles_r, tiles_c=tiles_c, filler=filler, lens=lens,
-                index=index, tiles_off=tiles_off, total=total, coded_bits=coded_bits)
+                index=index, tiles_off=tiles_off, total=total, coded_bits=coded_bits,
+                streams=streams)
 
 
 def codebook(lens):
@@ -49,19 +53,23 @@ def decode(blob: bytes) -> np.ndarray:
     rows, cols, tr, tc = h["rows"], h["cols"], h["tile_rows"], h["tile_cols"]
     out = np.zeros((rows, cols), dtype=np.uint16)
     per_lane = 2 * tr * (tc // 64)
+    S = h["streams"]
+    n_streams = 32 * S
     for u in range(h["tiles_r"] * h["tiles_c"]):
         i, j = u % h["tiles_r"], u // h["tiles_r"]
         c0 = h["tiles_off"] + 16 * h["index"][u]
         c1 = h["tiles_off"] + 16 * h["index"][u + 1]
         raw = b[c0:c0 + tr * tc]
-        lane_len = b[c0 + tr * tc:c0 + tr * tc + 32]
-        bits = sequence_bits(b[c0 + tr * tc + 32:c1])
+        lane_len = b[c0 + tr * tc:c0 + tr * tc + n_streams]
+        bits = sequence_bits(b[c0 + tr * tc + n_streams:c1])
         start = 0
-        for t in range(32):
-            s = bits[start:start + 8 * lane_len[t]]
-            start += 8 * lane_len[t]
+        for sigma in range(n_streams):
+            # Stream sigma: lane sigma // S, the lane's symbol pairs q with q % S == sigma % S.
+            t = sigma // S
+            s = bits[start:start + 8 * lane_len[sigma]]
+            start += 8 * lane_len[sigma]
             p = 0
-            for k in range(per_lane):
+            for k in [k for k in range(per_lane) if (k // 2) % S == sigma % S]:
                 q = p + 1
                 while s[p:q] not in book:
                     q += 1

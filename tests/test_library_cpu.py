@@ -170,3 +170,18 @@ def test_plan_options_code_field(lib):
     assert int.from_bytes(blob[:4].tobytes(), "little") == 0x3142574E
     opts = lib.nwc_opts(16, 0, 8, 512, 1, 0)            # too short for `threads`
     assert lib.LIB.nwc_plan(w.ctypes.data, 16, 256, ctypes.byref(opts), ctypes.byref(plan)) == 1
+
+
+def test_multi_stream_blobs_refused_until_a_kernel_reads_them(lib, orc):
+    """The format defines 2 or 4 bit streams per lane; no kernel reads them yet."""
+    w = synth.matrix(synth.MatrixSpec("w", 40, 600, "normal", 0.02, 0), 2)
+    for streams in (2, 4):
+        blob = orc.encode(w, tile_cols=128, streams=streams)
+        with pytest.raises(lib.NwcError) as e:
+            lib.nwc_blob_device_bytes(blob)
+        assert e.value.status == UNSUPPORTED
+    bad = orc.encode(w, tile_cols=128).copy()
+    bad[60] = 2                                          # S = 3 is not a layout
+    with pytest.raises(lib.NwcError) as e:
+        lib.nwc_blob_device_bytes(bad)
+    assert e.value.status == 4                           # NWC_ERR_CORRUPT
