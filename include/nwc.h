@@ -82,7 +82,12 @@ typedef enum {
  * bits and every peek holds two complete codes; with 8..12 it peeks 12 bits and
  * takes a second lookup when a pair does not fit.
  * lmax, NWC_CODE_RANK: the number of ranks, 0 = 7, else in [1, 7].
- * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512. */
+ * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512.
+ * streams (a struct_size that ends before it means 1): bit streams per lane
+ * and tile, each lane's symbol pairs dealt to its streams in turn (header
+ * offset 60 holds streams - 1).  2 and 4 are a host-encoder-only layout for
+ * now, with the prefix code only: nwc_plan_size reports device_bytes = 0 and
+ * the calls that need a device image return UNSUPPORTED. */
 typedef struct {
   uint32_t struct_size;
   uint32_t lmax;
@@ -90,6 +95,7 @@ typedef struct {
   uint32_t tile_cols;
   uint32_t threads; /* host encoder threads; 0 = hardware concurrency */
   uint32_t code;    /* nwc_code */
+  uint32_t streams; /* bit streams per lane and tile: 0 or 1, 2, 4 (see below) */
 } nwc_opts;
 
 /* Library version: major * 10000 + minor * 100 + patch. */

@@ -42,7 +42,8 @@ NWC_CODE_PREFIX, NWC_CODE_RANK = 0, 1
 class nwc_opts(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("lmax", ctypes.c_uint32),
                 ("tile_rows", ctypes.c_uint32), ("tile_cols", ctypes.c_uint32),
-                ("threads", ctypes.c_uint32), ("code", ctypes.c_uint32)]
+                ("threads", ctypes.c_uint32), ("code", ctypes.c_uint32),
+                ("streams", ctypes.c_uint32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -117,12 +118,13 @@ def nwc_version() -> int:
 
 
 def nwc_plan(w_host: np.ndarray, lmax: int = 0, tile_cols: int = 512, threads: int = 0,
-             code: int = NWC_CODE_PREFIX):
+             code: int = NWC_CODE_PREFIX, streams: int = 1):
     """code NWC_CODE_RANK: the ranked unary code, lmax = number of ranks (0 = 7);
-    host encoder only (nwc_compress_host)."""
+    streams 2 or 4: bit streams per lane.  Both host encoder only for now
+    (nwc_compress_host)."""
     w = np.ascontiguousarray(w_host, dtype=np.uint16)
     rows, cols = w.shape
-    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads, code)
+    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads, code, streams)
     plan = ctypes.c_void_p()
     _check(LIB.nwc_plan(w.ctypes.data, rows, cols, ctypes.byref(opts), ctypes.byref(plan)),
            "nwc_plan")

@@ -95,28 +95,35 @@ inline void symbol_of(const nwc_plan_s& p, const TileView& v, int r, int c, uint
   *len = p.rank_len[e] + 1;
 }
 
-// Bits of each lane's stream in tile u.
-void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t bits[kLanes]) {
+// Stream of lane t that carries the lane's k-th symbol when each lane has S
+// streams: consecutive symbol pairs go to the lane's streams in turn.
+inline int stream_of(int t, int k, int S) { return t * S + (k / 2) % S; }
+
+// Bits of each stream in tile u (kLanes * p.streams entries).
+void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t* bits) {
   const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
   TileView v{w, p.rows, p.cols, i * kTileRows, j * (int64_t)p.tile_cols, (uint8_t)p.filler};
-  for (int t = 0; t < kLanes; ++t) bits[t] = 0;
+  const int S = (int)p.streams;
+  for (int t = 0; t < kLanes * S; ++t) bits[t] = 0;
   for (int r = 0; r < kTileRows; ++r) {
     for (int c = 0; c < (int)p.tile_cols; ++c) {
       const int t = 4 * r + (c % 64) / 16;  // lane t = 4 r + q owns row r, columns 16 q .. of a group
+      const int k = 16 * (c / 64) + c % 16;  // the lane's symbol index
+      const int sigma = stream_of(t, k, S);
       if (p.code_kind == 0) {
         const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
-        bits[t] += p.len[s];
+        bits[sigma] += p.len[s];
       } else {
         const uint32_t e = v.inside(r, c) ? rank_field(v.at(r, c)) : p.filler;
-        bits[t] += p.rank_len[e] + 1u;
+        bits[sigma] += p.rank_len[e] + 1u;
       }
     }
   }
 }
 
-uint32_t stream_bytes_of(const uint32_t bits[kLanes]) {
+uint32_t stream_bytes_of(const uint32_t* bits, int n) {
   uint32_t total = 0;
-  for (int t = 0; t < kLanes; ++t) total += (bits[t] + 7) / 8;
+  for (int t = 0; t < n; ++t) total += (bits[t] + 7) / 8;
   return total;
 }
 
@@ -246,7 +253,10 @@ void build_decode_table(const uint8_t len[256], uint32_t lmax, uint32_t* table) 
 int plan_tiles(const uint16_t* w, nwc_plan_s* p);
 
 int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
-               uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* p) {
+               uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* p,
+               uint32_t streams) {
+  if (streams != 1 && streams != 2 && streams != 4) return -1;
+  p->streams = streams;
   p->rows = rows;
   p->cols = cols;
   p->tile_rows = tile_rows;
@@ -299,6 +309,10 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   for (int s = 0; s < 256; ++s) p->coded_bits += cnt[s] * p->len[s];
   const int rc = plan_tiles(w, p);
   if (rc != 0) return rc;
+  if (p->streams != 1) {  // no kernel reads several streams per lane yet
+    p->table_off = p->sched_off = p->device_bytes = 0;
+    return 0;
+  }
   p->table_off = round_up(p->blob_bytes, 256);
   p->sched_off = round_up(p->table_off + table_bytes(p->lmax), 256);
   p->device_bytes = p->sched_off + sched_bytes((uint64_t)p->tiles);
@@ -377,11 +391,13 @@ int plan_tiles(const uint16_t* w, nwc_plan_s* p) {
   const unsigned nt = p->threads;
   const uint32_t tile_cols = p->tile_cols;
   std::vector<uint32_t> chunk16((size_t)p->tiles);
+  const int n = kLanes * (int)p->streams;
   parallel_for(p->tiles, nt, [&](int64_t b, int64_t e) {
-    uint32_t bits[kLanes];
+    uint32_t bits[kLanes * kMaxStreams];
     for (int64_t u = b; u < e; ++u) {
       lane_bits(*p, w, u, bits);
-      const uint32_t bytes = raw_bytes(tile_cols) + kLanes + (uint32_t)round_up(stream_bytes_of(bits), 16);
+      const uint32_t bytes =
+          raw_bytes(tile_cols) + n + (uint32_t)round_up(stream_bytes_of(bits, n), 16);
       chunk16[(size_t)u] = bytes / 16;
     }
   });
@@ -412,6 +428,7 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
   h.tiles_r = (uint64_t)p.tiles_r;
   h.tiles_c = (uint64_t)p.tiles_c;
   h.filler = p.filler;
+  h.zero = p.streams - 1;  // streams per lane, S - 1
   h.lens_off = kLensOffset;
   h.index_off = kIndexOffset;
   h.tiles_off = p.tiles_off;
@@ -427,6 +444,8 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
 
   const uint32_t groups = p.tile_cols / 64;
   const uint32_t raw_n = raw_bytes(p.tile_cols);
+  const int S = (int)p.streams;
+  const uint32_t nstreams = kLanes * (uint32_t)S;
   parallel_for(p.tiles, p.threads, [&](int64_t b, int64_t e) {
     std::vector<uint8_t> seq;  // big-endian bytes of the stream run
     for (int64_t u = b; u < e; ++u) {
@@ -434,23 +453,26 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
       TileView v{w, p.rows, p.cols, i * kTileRows, j * (int64_t)p.tile_cols, (uint8_t)p.filler};
       uint8_t* chunk = blob + p.tiles_off + 16ull * p.index[(size_t)u];
       const uint32_t chunk_bytes = 16u * (p.index[(size_t)u + 1] - p.index[(size_t)u]);
-      const uint32_t area = chunk_bytes - raw_n - kLanes;
+      const uint32_t area = chunk_bytes - raw_n - nstreams;
       uint8_t* raw = chunk;
       uint8_t* lane_len = chunk + raw_n;
-      uint8_t* words = chunk + raw_n + kLanes;
+      uint8_t* words = chunk + raw_n + nstreams;
       seq.assign(area, 0);
       uint32_t out = 0;
-      for (int t = 0; t < kLanes; ++t) {
+      for (int sigma = 0; sigma < (int)nstreams; ++sigma) {
         const uint32_t lane_start = out;
         uint32_t accb = 0;  // pending bits, right-aligned
         int nacc = 0;
-        // Lane t = 4 r + q owns row r; group g gives it columns 64 g + 16 q ..
-        // 64 g + 16 q + 15, symbols 16 g .. 16 g + 15.
+        // Stream sigma belongs to lane t = sigma / S = 4 r + q, which owns row
+        // r; group g gives it columns 64 g + 16 q .. 64 g + 16 q + 15, symbols
+        // 16 g .. 16 g + 15, of which this stream takes those of its pairs.
+        const int t = sigma / S;
         const int r = t / 4;
         for (uint32_t g = 0; g < groups; ++g) {
           for (int kk = 0; kk < 16; ++kk) {
             const int c = (int)(64 * g) + 16 * (t % 4) + kk;
             const int k = (int)(16 * g) + kk;
+            if (stream_of(t, k, S) != sigma) continue;
             uint32_t code;
             int len;
             uint8_t rb;
@@ -466,7 +488,7 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
           }
         }
         if (nacc > 0) seq[out++] = (uint8_t)(accb << (8 - nacc));
-        lane_len[t] = (uint8_t)(out - lane_start);
+        lane_len[sigma] = (uint8_t)(out - lane_start);
       }
       // Little-endian words with the earliest bit in bit 31.
       for (uint32_t q = 0; q < area; q += 4) {

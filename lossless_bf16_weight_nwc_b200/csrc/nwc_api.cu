@@ -225,15 +225,19 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
   if (rows > (1ll << 40) || cols > (1ll << 40)) return NWC_ERR_INVALID_ARG;
   *out_plan = nullptr;
   uint32_t lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0, code = NWC_CODE_PREFIX;
+  uint32_t streams = 1;
   if (opts) {
     if (opts->struct_size < offsetof(nwc_opts, code)) return NWC_ERR_INVALID_ARG;
     lmax = opts->lmax;
     tile_rows = opts->tile_rows;
     tile_cols = opts->tile_cols;
     threads = opts->threads;
-    if (opts->struct_size >= sizeof(nwc_opts)) code = opts->code;
+    if (opts->struct_size >= offsetof(nwc_opts, streams)) code = opts->code;
+    if (opts->struct_size >= sizeof(nwc_opts) && opts->streams) streams = opts->streams;
   }
   if (code != NWC_CODE_PREFIX && code != NWC_CODE_RANK) return NWC_ERR_INVALID_ARG;
+  if (streams != 1 && streams != 2 && streams != 4) return NWC_ERR_INVALID_ARG;
+  if (code == NWC_CODE_RANK && streams != 1) return NWC_ERR_UNSUPPORTED;
   if (code == NWC_CODE_RANK && lmax > (uint32_t)nwc::kMaxRanks) return NWC_ERR_INVALID_ARG;
   if (lmax > (uint32_t)nwc::kMaxLmax) return NWC_ERR_INVALID_ARG;
   if (tile_rows != 8) return NWC_ERR_UNSUPPORTED;
@@ -246,7 +250,8 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
     rc = code == NWC_CODE_RANK
              ? nwc::plan_build_rank(w_host, rows, cols, tile_cols, lmax ? lmax : nwc::kMaxRanks,
                                     threads, p)
-             : nwc::plan_build(w_host, rows, cols, tile_rows, tile_cols, lmax, threads, p);
+             : nwc::plan_build(w_host, rows, cols, tile_rows, tile_cols, lmax, threads, p,
+                               streams);
   } catch (const std::bad_alloc&) {
     delete p;
     return NWC_ERR_NOMEM;
@@ -281,7 +286,8 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
                         nwc_stream_t stream, nwc_handle_t* out_handle) {
   if (!plan || !w_host || !d_buf || !out_handle) return NWC_ERR_INVALID_ARG;
   *out_handle = nullptr;
-  if (plan->code_kind != NWC_CODE_PREFIX) return NWC_ERR_UNSUPPORTED;  // no kernel reads it yet
+  // No kernel reads these layouts yet.
+  if (plan->code_kind != NWC_CODE_PREFIX || plan->streams != 1) return NWC_ERR_UNSUPPORTED;
   if (d_bytes < plan->device_bytes || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
   uint8_t* img = static_cast<uint8_t*>(std::malloc(plan->device_bytes));
   if (!img) return NWC_ERR_NOMEM;

@@ -56,6 +56,7 @@ constexpr int kTileRows = 8;
 constexpr int kMaxTileCols = 512;
 constexpr int kMaxLmax = 12;
 constexpr int kMaxPeekBits = 14;
+constexpr int kMaxStreams = 4;  // bit streams per lane and tile: 1, 2 or 4
 
 // Width of the decoder's table peek for a length limit.  With lmax <= 7 the
 // peek is 14 bits, so every entry holds two complete codes and the decoder

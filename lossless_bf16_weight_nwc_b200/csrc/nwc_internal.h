@@ -16,6 +16,7 @@ struct nwc_plan_s {
   // Exponent code: 0 = canonical prefix code of bits 14..7 (NWB1), 1 = ranked
   // unary code of bits 14..8 with the sign bit (NWR1).
   uint32_t code_kind = 0;
+  uint32_t streams = 1;                      // bit streams per lane and tile (1, 2, 4)
   uint32_t ranks = 0;                        // NWR1: R
   uint8_t rank_table[nwc::kMaxRanks] = {};   // NWR1: ranked values of e
   uint8_t rank_len[128] = {};                // NWR1: bits after the sign bit
@@ -48,8 +49,11 @@ struct nwc_handle_s {
 namespace nwc {
 
 // Encoder steps (encoder.cpp).
+// streams: bit streams per lane and tile (1, 2 or 4); only 1 has a device
+// image (device_bytes = 0 otherwise).
 int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
-               uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* plan);
+               uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* plan,
+               uint32_t streams = 1);
 // The ranked unary code (NWR1) with `ranks` ranks (1..7); the plan has no
 // device image (device_bytes = 0).
 int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_cols,

@@ -185,3 +185,24 @@ def test_multi_stream_blobs_refused_until_a_kernel_reads_them(lib, orc):
     with pytest.raises(lib.NwcError) as e:
         lib.nwc_blob_device_bytes(bad)
     assert e.value.status == 4                           # NWC_ERR_CORRUPT
+
+
+def test_streams_per_lane_encoder_and_refusals(lib, orc):
+    import ctypes
+    w = synth.matrix(synth.MatrixSpec("w", 40, 600, "normal", 0.02, 0), 2)
+    for streams in (2, 4):
+        plan = lib.nwc_plan(w, tile_cols=128, streams=streams)
+        dev_bytes, _ = lib.nwc_plan_size(plan)
+        blob = lib.nwc_compress_host(plan, w)
+        assert dev_bytes == 0 and np.array_equal(blob, orc.encode(w, tile_cols=128, lmax=7,
+                                                                  streams=streams))
+        h = ctypes.c_void_p()
+        st = lib.LIB.nwc_compress(plan, w.ctypes.data, 1 << 20, 1 << 30, None, ctypes.byref(h))
+        assert st == UNSUPPORTED and not h.value
+        lib.nwc_plan_destroy(plan)
+    with pytest.raises(lib.NwcError) as e:
+        lib.nwc_plan(w, streams=3)
+    assert e.value.status == 1                         # NWC_ERR_INVALID_ARG
+    with pytest.raises(lib.NwcError) as e:
+        lib.nwc_plan(w, streams=2, code=lib.NWC_CODE_RANK)
+    assert e.value.status == UNSUPPORTED
