@@ -29,9 +29,11 @@
  *   - Arguments are validated on the host before anything is launched.  Invalid
  *     input returns an error code and launches nothing.
  *   - Errors found on the device (a corrupt tile, a bounded wait that gave up) set
- *     bits in a device error word; nwc_get_device_error() reads and clears it.
- *   - Thread safety: distinct handles may be used concurrently.  Calls that share
- *     a handle or a workspace must be ordered by the caller.
+ *     bits in the handle's error word, which lives in its device image;
+ *     nwc_get_device_error() reads and clears it.
+ *   - Thread safety: distinct handles may be used concurrently.  Device calls on
+ *     one handle write its image's scratch area, so they must be ordered by the
+ *     caller (one stream, or events between streams).
  */
 #ifndef NWC_H
 #define NWC_H
@@ -107,7 +109,11 @@ const char* nwc_status_string(nwc_status status);
 /* ---- Host encoder ------------------------------------------------------- */
 
 /* Histogram of the exponent bytes, the length-limited canonical code, and the
- * exact compressed sizes.  w_host holds rows x cols BF16 patterns, row-major.
+ * exact compressed sizes ("Unweight", "Compressing BF16 Weights": the exponent
+ * byte is Huffman-coded from its histogram, sign and mantissa kept; "NWC",
+ * "How it works > Prefix code instead of rANS": one code table per matrix,
+ * decoded by a fixed-width table peek).  w_host holds rows x cols BF16
+ * patterns, row-major.
  * It is read, not retained.  rows, cols >= 1.  On success *out_plan owns host
  * memory; free it with nwc_plan_destroy.
  * Errors: INVALID_ARG (null, sizes, options, > 64 GiB of tile data), NOMEM. */
@@ -116,16 +122,24 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols,
 
 /* Exact sizes for a plan.  *device_bytes is what nwc_compress needs in device
  * memory, the "device image": the serialisable blob, then at 256-byte aligned
- * offsets a derived decode table (64 KiB for lmax <= 7, else 16 KiB) and the
- * launch schedules (two of about 12 bytes per tile plus 5 KiB each: which
- * bytes each bulk copy of the kernels moves and where they land in shared
- * memory, worked out on the host for the device that runs them).  *host_blob_bytes is the size of
- * the serialisable blob (nwc_compress_host).  Either pointer may be NULL. */
+ * offsets a derived decode table (64 KiB for lmax <= 7, else 16 KiB), the
+ * launch schedules (which bytes each bulk copy of the kernels moves and where
+ * they land in shared memory, worked out on the host for the device that runs
+ * them), and a scratch area that the kernels write: the handle's error word,
+ * split-K arrival counters (4 bytes per 8 rows) and partial sums (for a matrix
+ * of more than one column tile: 4 bytes x 16 rows of x x rows x column tiles,
+ * about 9 % of the compressed size at 512-column tiles, or 1 MiB if that is
+ * larger).  *host_blob_bytes is the size of the serialisable blob
+ * (nwc_compress_host).  Either pointer may be NULL. */
 nwc_status nwc_plan_size(nwc_plan_t plan, uint64_t* device_bytes,
                          uint64_t* host_blob_bytes);
 
 /* Encode w_host (the same matrix given to nwc_plan) and upload it into the
- * caller's device buffer d_buf (>= device_bytes, 256-byte aligned) on `stream`.
+ * caller's device buffer d_buf (>= device_bytes, 256-byte aligned) on `stream`
+ * ("NWC", "How it works > Byte planes" and "> Fused kernel": byte planes in
+ * independently decodable blocks of 8 rows x 512 columns, one bit stream per
+ * lane).  Only the blob, table, schedules and the start of the scratch area
+ * are copied; the partial sums need no initial value.
  * The upload is asynchronous: w_host may be reused when the call returns,
  * but d_buf must not be read before the stream reaches this point.  On success
  * *out_handle refers to d_buf.
@@ -205,32 +219,34 @@ nwc_status nwc_decompress(nwc_handle_t handle, uint16_t* d_w_out, nwc_stream_t s
 nwc_status nwc_gather_rows(nwc_handle_t handle, const int32_t* d_rows, int32_t n,
                            uint16_t* d_out, nwc_stream_t stream);
 
-/* Bytes of scratch that nwc_gemv needs for this handle and batch; 0 when the
- * matrix has a single column tile.  The scratch holds one FP32 partial sum per
- * (column tile, batch row, output row) plus one u32 counter per row tile; it
- * makes the split-K reduction deterministic (fixed summation order). */
-nwc_status nwc_gemv_workspace_size(nwc_handle_t handle, int32_t batch,
-                                   uint64_t* bytes);
+/* Bytes of split-K scratch one GEMV call of `batch` rows uses: u32 arrival
+ * counters (one per 8 rows, padded to 256 bytes) and one FP32 partial sum per
+ * (column tile, row of x in a launch, output row); 0 when the matrix has a
+ * single column tile.  nwc_gemv takes them from the device image's scratch
+ * area, nwc_gemv_noalloc from the library's static array.  The partials make
+ * the reduction deterministic (fixed summation order). */
+nwc_status nwc_gemv_scratch_bytes(nwc_handle_t handle, int32_t batch, uint64_t* bytes);
 
-/* y[b][n] = sum_k W[n][k] * x[b][k], for b < batch, n < rows, k < cols.
+/* The fused decode-GEMV ("NWC", "How it works > Fused kernel": the matrix-vector
+ * kernel decodes the compressed blocks itself and keeps partial sums per
+ * (row, column block); "Unweight", "Direct GPU Decompression": weights are
+ * decompressed in shared memory and fed to the tensor cores, never written
+ * back): y[b][n] = sum_k W[n][k] * x[b][k], for b < batch, n < rows, k < cols.
  *   d_x: device, BF16 [batch x cols], row-major, 4-byte aligned, cols even.
  *   d_y: FP32 [batch x rows], row-major (overwritten, not accumulated), in
  *     device memory or in pinned host memory that the device can address (the
  *     kernel then stores the result straight into host memory).
  *   batch in [1, 64].
- *   d_workspace: device, >= nwc_gemv_workspace_size bytes, 16-byte aligned,
- *     zero-filled before its first use.  Every completed call leaves the counter
- *     area zero again, so one workspace serves any number of ordered calls (a
- *     call that ended with a device error may not: zero it again).  Two calls
- *     that overlap on the GPU must not share a workspace.  It may be NULL when
- *     the size is 0.
+ * The caller passes no workspace: the split-K partial sums and counters live
+ * in the scratch area of the handle's device image, so calls on one handle
+ * must be ordered (a completed call leaves the counters zero again;
+ * nwc_get_device_error clears them after a call that ended with an error).
  * Products and sums are in FP32; the result is the same bit pattern on every
- * run.  Asynchronous on `stream`.
- * Errors: INVALID_ARG (null, batch, alignment, odd cols, workspace too small),
- * UNSUPPORTED, CUDA (launch). */
+ * run.  Asynchronous on `stream`; allocates nothing.
+ * Errors: INVALID_ARG (null, batch, alignment, odd cols, another device
+ * current), UNSUPPORTED, CUDA (launch). */
 nwc_status nwc_gemv(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
-                    int32_t batch, void* d_workspace, uint64_t workspace_bytes,
-                    nwc_stream_t stream);
+                    int32_t batch, nwc_stream_t stream);
 
 /* GEMV for callers that cannot allocate device memory.  The pages describe
  * no such call; it exists for integrations where the host application owns
@@ -242,21 +258,23 @@ nwc_status nwc_gemv(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
  * It computes exactly what nwc_gemv computes, with the same kernels, but takes
  * its scratch (the split-K partial sums and arrival counters) from an array of
  * NWC_NOALLOC_SCRATCH_BYTES bytes that the library defines as a static device
- * variable.  Every GPU that loads the library holds that array until the
+ * variable instead of the device image's scratch area (the handle's error word
+ * stays in the image).  Every GPU that loads the library holds that array until the
  * process exits.  The call allocates nothing: no cudaMalloc, no cudaFree, no
  * allocating library routine.
  *   - Set-up: the first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current, and caches it.  Make
  *     that first call before any stream capture.
- *   - Limit: when nwc_gemv_workspace_size(handle, batch) exceeds
+ *   - Limit: when nwc_gemv_scratch_bytes(handle, batch) exceeds
  *     NWC_NOALLOC_SCRATCH_BYTES the call returns NWC_ERR_SCRATCH_LIMIT and
- *     launches nothing; use nwc_gemv with your own workspace instead.
+ *     launches nothing; use nwc_gemv instead.
  *   - Sharing: every call uses the same array, which keeps the last call's
  *     contents; each call first clears the counters it needs (an async memset
  *     on `stream`).  Calls whose work overlaps on the GPU (different streams,
  *     or different threads without ordering) race on the array and must not
  *     be issued.
- * Arguments and other errors as nwc_gemv. */
+ * Arguments and other errors as nwc_gemv; every argument is checked before
+ * anything is enqueued. */
 #define NWC_NOALLOC_SCRATCH_BYTES (8u << 20)
 nwc_status nwc_gemv_noalloc(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
                             int32_t batch, nwc_stream_t stream);
@@ -295,16 +313,28 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
                                  nwc_schedule_info* info, uint32_t* cta_batch,
                                  uint32_t* batch, uint32_t* tile_ring);
 
-/* Any pointer may be NULL.  *blob_bytes is the serialisable part; *device_bytes
- * is the whole device image (blob + decode table + launch schedule). */
+/* Any pointer may be NULL.  *blob_bytes is the serialisable part;
+ * *compressed_bytes is what holds the matrix (blob, decode table and launch
+ * schedules: the offset of the scratch area); *device_bytes is the whole device
+ * image (compressed bytes + scratch area). */
 nwc_status nwc_handle_info(nwc_handle_t handle, int64_t* rows, int64_t* cols,
-                           uint64_t* blob_bytes, uint64_t* device_bytes);
+                           uint64_t* blob_bytes, uint64_t* device_bytes,
+                           uint64_t* compressed_bytes);
 
-/* Synchronizes `stream`, then reads and clears the device error word of the
- * current device.  Returns OK, DEVICE_TIMEOUT, DEVICE_CORRUPT or INVALID_ARG
- * (a gathered row id out of range), in that order of precedence, or CUDA.
- * *word (optional) receives the raw bits. */
-nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word);
+/* Reads the handle's device error word in order on `stream` (which it then
+ * synchronizes) and clears it, together with the split-K arrival counters, when
+ * it is non-zero.  Only this handle's kernels set it.  Returns OK,
+ * DEVICE_TIMEOUT, DEVICE_CORRUPT or INVALID_ARG (a gathered row id out of
+ * range), in that order of precedence, or CUDA.  *word (optional) receives the
+ * raw bits: 1 a bounded wait gave up, 2 corrupt stream, 4 row id out of range. */
+nwc_status nwc_get_device_error(nwc_handle_t handle, nwc_stream_t stream, uint32_t* word);
+
+/* Test and diagnostic use only: the number of polls after which a kernel's
+ * bounded wait on an mbarrier gives up (sets error bit 1 and returns) for
+ * launches made after this call, process-wide; 0 restores the default
+ * (2^22 polls).  A small limit makes a wait that would otherwise only be slow
+ * give up, so ordinary callers never set it. */
+void nwc_test_set_wait_limit(uint32_t polls);
 
 /* Free host metadata.  NULL is accepted.  Device memory is never freed. */
 void nwc_plan_destroy(nwc_plan_t plan);

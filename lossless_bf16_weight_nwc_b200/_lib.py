@@ -65,12 +65,13 @@ def _load() -> ctypes.CDLL:
         "nwc_handle_from_device": ([vp, u64, c.POINTER(vp)], c.c_int),
         "nwc_decompress": ([vp, vp, vp], c.c_int),
         "nwc_gather_rows": ([vp, vp, i32, vp, vp], c.c_int),
-        "nwc_gemv_workspace_size": ([vp, i32, c.POINTER(u64)], c.c_int),
-        "nwc_gemv": ([vp, vp, vp, i32, vp, u64, vp], c.c_int),
+        "nwc_gemv_scratch_bytes": ([vp, i32, c.POINTER(u64)], c.c_int),
+        "nwc_gemv": ([vp, vp, vp, i32, vp], c.c_int),
         "nwc_gemv_noalloc": ([vp, vp, vp, i32, vp], c.c_int),
         "nwc_handle_info": ([vp, c.POINTER(i64), c.POINTER(i64), c.POINTER(u64),
-                             c.POINTER(u64)], c.c_int),
-        "nwc_get_device_error": ([vp, c.POINTER(c.c_uint32)], c.c_int),
+                             c.POINTER(u64), c.POINTER(u64)], c.c_int),
+        "nwc_get_device_error": ([vp, vp, c.POINTER(c.c_uint32)], c.c_int),
+        "nwc_test_set_wait_limit": ([c.c_uint32], None),
         "nwc_schedule_describe": ([vp, u64, i32, u64, i32, c.POINTER(nwc_schedule_info), vp, vp,
                                    vp],
                                   c.c_int),
@@ -88,9 +89,10 @@ LIB = _load()
 EXPORTED = ("nwc_version", "nwc_status_string", "nwc_plan", "nwc_plan_size", "nwc_compress",
             "nwc_compress_host", "nwc_blob_device_bytes", "nwc_upload_blob",
             "nwc_handle_from_device", "nwc_decompress", "nwc_gather_rows",
-            "nwc_gemv_workspace_size", "nwc_gemv",
+            "nwc_gemv_scratch_bytes", "nwc_gemv",
             "nwc_gemv_noalloc",
-            "nwc_handle_info", "nwc_get_device_error", "nwc_schedule_describe",
+            "nwc_handle_info", "nwc_get_device_error", "nwc_test_set_wait_limit",
+            "nwc_schedule_describe",
             "nwc_plan_destroy", "nwc_handle_destroy")
 
 
@@ -186,18 +188,14 @@ def nwc_gather_rows(handle, d_rows, n: int, d_out, stream=None) -> None:
            "nwc_gather_rows")
 
 
-def nwc_gemv_workspace_size(handle, batch: int) -> int:
+def nwc_gemv_scratch_bytes(handle, batch: int) -> int:
     out = ctypes.c_uint64()
-    _check(LIB.nwc_gemv_workspace_size(handle, batch, ctypes.byref(out)),
-           "nwc_gemv_workspace_size")
+    _check(LIB.nwc_gemv_scratch_bytes(handle, batch, ctypes.byref(out)), "nwc_gemv_scratch_bytes")
     return out.value
 
 
-def nwc_gemv(handle, d_x, d_y, batch: int, d_workspace=None, workspace_bytes: int = 0,
-             stream=None) -> None:
-    ws = 0 if d_workspace is None else _ptr(d_workspace)
-    _check(LIB.nwc_gemv(handle, _ptr(d_x), _ptr(d_y), batch, ws, workspace_bytes,
-                        _stream(stream)), "nwc_gemv")
+def nwc_gemv(handle, d_x, d_y, batch: int, stream=None) -> None:
+    _check(LIB.nwc_gemv(handle, _ptr(d_x), _ptr(d_y), batch, _stream(stream)), "nwc_gemv")
 
 
 def nwc_gemv_noalloc(handle, d_x, d_y, batch: int, stream=None) -> None:
@@ -209,17 +207,24 @@ def nwc_gemv_noalloc(handle, d_x, d_y, batch: int, stream=None) -> None:
 
 def nwc_handle_info(handle) -> dict:
     r, c = ctypes.c_int64(), ctypes.c_int64()
-    b, d = ctypes.c_uint64(), ctypes.c_uint64()
+    b, d, k = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
     _check(LIB.nwc_handle_info(handle, ctypes.byref(r), ctypes.byref(c), ctypes.byref(b),
-                               ctypes.byref(d)), "nwc_handle_info")
-    return {"rows": r.value, "cols": c.value, "blob_bytes": b.value, "device_bytes": d.value}
+                               ctypes.byref(d), ctypes.byref(k)), "nwc_handle_info")
+    return {"rows": r.value, "cols": c.value, "blob_bytes": b.value, "device_bytes": d.value,
+            "compressed_bytes": k.value}
 
 
-def nwc_get_device_error(stream=None) -> tuple[int, int]:
-    """(status, raw word); synchronizes the stream."""
+def nwc_get_device_error(handle, stream=None) -> tuple[int, int]:
+    """(status, raw word) of the handle's device error word, read and cleared in
+    order on the stream, which it synchronizes."""
     w = ctypes.c_uint32()
-    st = LIB.nwc_get_device_error(_stream(stream), ctypes.byref(w))
+    st = LIB.nwc_get_device_error(handle, _stream(stream), ctypes.byref(w))
     return st, w.value
+
+
+def nwc_test_set_wait_limit(polls: int) -> None:
+    """Test use only: polls before a kernel's bounded wait gives up (0 = default)."""
+    LIB.nwc_test_set_wait_limit(polls)
 
 
 def nwc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int = 232448,
@@ -273,9 +278,10 @@ def _require(t, what: str, dtypes, shape, device, pinned_host_ok: bool = False) 
 class CompressedMatrix:
     """A BF16 matrix held compressed in device memory that torch allocated.
 
-    Owns the device image (a uint8 CUDA tensor), the handle, and a GEMV
-    workspace that grows on demand.  Calls make the image's device current and
-    run on that device's current torch stream (or the stream given)."""
+    Owns the device image (a uint8 CUDA tensor, which also holds the GEMV's
+    scratch) and the handle.  Calls make the image's device current and run on
+    that device's current torch stream (or the stream given); calls on one
+    matrix must be ordered."""
 
     def __init__(self, image, handle, rows: int, cols: int, blob_bytes: int):
         self.image = image
@@ -284,7 +290,6 @@ class CompressedMatrix:
         self.blob_bytes = blob_bytes
         self.device_bytes = image.numel()
         self.row_splits = [0, rows]  # first output row of each part, then rows
-        self._ws = None
 
     @classmethod
     def compress(cls, w_host: np.ndarray, device="cuda", lmax: int = 0, tile_cols: int = 512,
@@ -333,17 +338,19 @@ class CompressedMatrix:
 
     @property
     def ratio(self) -> float:
-        """Uncompressed BF16 bytes / device bytes (blob + decode table)."""
-        return 2.0 * self.rows * self.cols / self.device_bytes
+        """Uncompressed BF16 bytes / compressed bytes (blob, decode table and
+        launch schedules: the device image without its scratch area)."""
+        return 2.0 * self.rows * self.cols / self.compressed_bytes
 
-    def workspace(self, batch: int):
+    @property
+    def compressed_bytes(self) -> int:
+        return nwc_handle_info(self.handle)["compressed_bytes"]
+
+    def device_error(self, stream=None) -> tuple[int, int]:
+        """(status, raw word) of this matrix's device error word (read and cleared)."""
         import torch
-        need = nwc_gemv_workspace_size(self.handle, batch)
-        if need == 0:
-            return None, 0
-        if self._ws is None or self._ws.numel() < need:
-            self._ws = torch.zeros(need, dtype=torch.uint8, device=self.image.device)
-        return self._ws, self._ws.numel()
+        with torch.cuda.device(self.image.device):
+            return nwc_get_device_error(self.handle, stream)
 
     def _open(self) -> None:
         if self.handle is None:
@@ -379,9 +386,8 @@ class CompressedMatrix:
             y = torch.empty((batch, self.rows), dtype=torch.float32, device=self.image.device)
         _require(y, "y", (torch.float32,), (batch, self.rows), self.image.device,
                  pinned_host_ok=True)
-        ws, ws_bytes = self.workspace(batch)
         with torch.cuda.device(self.image.device):
-            nwc_gemv(self.handle, xb, y, batch, ws, ws_bytes, stream)
+            nwc_gemv(self.handle, xb, y, batch, stream)
         return y
 
     def gather_rows(self, rows, stream=None):

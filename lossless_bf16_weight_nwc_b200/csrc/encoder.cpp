@@ -310,12 +310,15 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   const int rc = plan_tiles(w, p);
   if (rc != 0) return rc;
   if (p->streams != 1) {  // no kernel reads several streams per lane yet
-    p->table_off = p->sched_off = p->device_bytes = 0;
+    p->table_off = p->sched_off = p->scratch_off = p->device_bytes = 0;
     return 0;
   }
-  p->table_off = round_up(p->blob_bytes, 256);
-  p->sched_off = round_up(p->table_off + table_bytes(p->lmax), 256);
-  p->device_bytes = p->sched_off + sched_bytes((uint64_t)p->tiles);
+  const ImageLayout L =
+      image_layout(p->blob_bytes, p->lmax, (uint64_t)p->tiles_r, (uint64_t)p->tiles_c);
+  p->table_off = L.table_off;
+  p->sched_off = L.sched_off;
+  p->scratch_off = L.scratch_off;
+  p->device_bytes = L.device_bytes;
   return 0;
 }
 
@@ -382,7 +385,7 @@ int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile
   const int rc = plan_tiles(w, p);
   if (rc != 0) return rc;
   // No kernel reads this code yet: there is no device image.
-  p->table_off = p->sched_off = p->device_bytes = 0;
+  p->table_off = p->sched_off = p->scratch_off = p->device_bytes = 0;
   return 0;
 }
 
@@ -560,9 +563,11 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   std::memcpy(hd->index.data(), blob + kIndexOffset, 4 * ((size_t)tiles + 1));
   hd->tiles_off = h.tiles_off;
   hd->blob_bytes = bytes;
-  hd->table_off = round_up(bytes, 256);
-  hd->sched_off = round_up(hd->table_off + table_bytes(h.lmax), 256);
-  hd->device_bytes = hd->sched_off + sched_bytes(tiles);
+  const ImageLayout L = image_layout(bytes, h.lmax, h.tiles_r, h.tiles_c);
+  hd->table_off = L.table_off;
+  hd->sched_off = L.sched_off;
+  hd->scratch_off = L.scratch_off;
+  hd->device_bytes = L.device_bytes;
   hd->max_chunk = largest;
   if (lens_out) *lens_out = lens;
   return true;

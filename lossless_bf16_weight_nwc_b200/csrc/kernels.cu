@@ -36,11 +36,8 @@
 
 namespace nwc {
 
-__device__ unsigned int g_device_error;
-
 namespace {
 
-constexpr uint32_t kWaitLimit = 1u << 22;        // bounded mbarrier polls
 constexpr int kRingSlack = 256;                  // readers may run past a chunk (corrupt data)
 constexpr int kTablePieces = 8;                  // bulk copies that bring in the decode table
 constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
@@ -90,12 +87,20 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
-// Polls `bar` for `parity` at most kWaitLimit times; on failure records a
-// timeout in the device error word.
-__device__ bool wait_bounded(uint64_t* bar, uint32_t parity) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it)
+// Where a bounded wait reports giving up, and after how many polls.
+struct WaitCtl {
+  uint32_t* err;
+  uint32_t limit;
+};
+__device__ __forceinline__ WaitCtl wait_ctl(const TileParams& p) {
+  return WaitCtl{p.err, p.wait_limit ? p.wait_limit : kDefaultWaitLimit};
+}
+// Polls `bar` for `parity` at most w.limit times; on failure records a
+// timeout in the handle's error word.
+__device__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
+  for (uint32_t it = 0; it < w.limit; ++it)
     if (mbar_try_wait(bar, parity)) return true;
-  atomicOr(&g_device_error, kErrTimeout);
+  atomicOr(w.err, kErrTimeout);
   return false;
 }
 
@@ -408,6 +413,7 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
       bulk_load(smem + off, reinterpret_cast<const uint8_t*>(p.table) + off, piece, s.table_bar);
     }
   }
+  const WaitCtl wc = wait_ctl(p);
   const uint4 none = make_uint4(0u, 0u, 0u, 0u);
   uint4 cur = lane < nb ? __ldg(desc + lane) : none;
   uint4 nxt = 32 + lane < nb ? __ldg(desc + 32 + lane) : none;
@@ -426,7 +432,7 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
     uint32_t ok = 1;
     if (lane == 0) {
       for (; released < need; ++released) {
-        if (!wait_bounded(&s.empty[released % kSlots], (released / kSlots) & 1u)) {
+        if (!wait_bounded(&s.empty[released % kSlots], (released / kSlots) & 1u, wc)) {
           ok = 0;
           break;
         }
@@ -443,8 +449,8 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
   // kSlots back have been released, hence landed.
   if (lane == 0) {
     for (int j = k - 1; j >= 0 && j >= k - kSlots; --j)
-      wait_bounded(&s.full[j % kSlots], (uint32_t)((j / kSlots) & 1));
-    wait_bounded(s.table_bar, 0);
+      wait_bounded(&s.full[j % kSlots], (uint32_t)((j / kSlots) & 1), wc);
+    wait_bounded(s.table_bar, 0, wc);
   }
 }
 
@@ -453,8 +459,8 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
 // consumer polls slot k % kSlots (its last released tile at most kMaxLag tiles
 // back) the slot's previous batch k - kSlots was released long ago: the parity
 // it polls is batch k's.
-__device__ __forceinline__ bool wait_batch(const Smem& s, int k) {
-  return __all_sync(kFull, wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1)));
+__device__ __forceinline__ bool wait_batch(const Smem& s, int k, const WaitCtl& wc) {
+  return __all_sync(kFull, wait_bounded(&s.full[k % kSlots], (uint32_t)((k / kSlots) & 1), wc));
 }
 
 // Four BF16 values x[col .. col + 3] of one row of x as two words, zeros where
@@ -565,8 +571,8 @@ __device__ __forceinline__ bool setup(const TileParams& p, uint8_t* smem, const 
 }
 
 // Consumers: wait for the decode table.
-__device__ __forceinline__ bool wait_table(const Smem& s) {
-  return __all_sync(kFull, wait_bounded(s.table_bar, 0));
+__device__ __forceinline__ bool wait_table(const Smem& s, const WaitCtl& wc) {
+  return __all_sync(kFull, wait_bounded(s.table_bar, 0, wc));
 }
 
 // Row block i and column block j of tile u = first + q, stepped by NC tiles.
@@ -597,6 +603,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   int n;
   cta_range(p, &first, &n);
   if (!setup<NC>(p, smem, s)) return;
+  const WaitCtl wc = wait_ctl(p);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
   const uint32_t table = smem_u32(smem);
@@ -641,7 +648,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
     }
     named_barrier_sync(1, NC * 32);  // consumers only
   }
-  if (!wait_table(s)) return;
+  if (!wait_table(s, wc)) return;
   const uint32_t xst = smem_u32(s.xstage);
   const uint32_t* tile_ring = p.tile_ring + first;
   uint32_t at_next = warp < n ? __ldg(tile_ring + warp) : 0u;
@@ -651,7 +658,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
     const int k = q / p.batch_tiles;
     const uint32_t chunk = ring + at_next;
     if (q + NC < n) at_next = __ldg(tile_ring + q + NC);  // next tile's ring offset, early
-    if (!wait_batch(s, k)) return;
+    if (!wait_batch(s, k, wc)) return;
     const int64_t i = pos.i, j = pos.j;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     if (xsmem)
@@ -728,7 +735,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
   cta_range(p, &first, &n);
   if (!setup<NC>(p, smem, s)) return;
   wait_prerequisites();  // the output may still be read by the previous kernel
-  if (!wait_table(s)) return;
+  const WaitCtl wc = wait_ctl(p);
+  if (!wait_table(s, wc)) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
@@ -746,7 +754,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     const int k = q / p.batch_tiles;
     const uint32_t chunk = ring + at_next;
     if (q + NC < n) at_next = __ldg(tile_ring + q + NC);
-    if (!wait_batch(s, k)) return;
+    if (!wait_batch(s, k, wc)) return;
     const int64_t i = pos.i, j = pos.j;
     StreamDecoder<FAST> dec;
     dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
@@ -784,7 +792,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     if (lane == 0) mbar_arrive(&s.empty[k % kSlots]);  // release the tile's share of the batch
   }
   if (__any_sync(kFull, invalid & kEntryInvalid) && lane == 0)
-    atomicOr(&g_device_error, kErrCorrupt);
+    atomicOr(p.err, kErrCorrupt);
 }
 
 // Row gather ("NWC", "How it works > Dequantization and embedding lookup": the
@@ -801,7 +809,7 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherParams p) {
   const int64_t i = wg / p.tiles_c, j = wg % p.tiles_c;
   const int32_t row = __ldg(p.row_ids + i);
   if (row < 0 || row >= p.rows) {
-    if (lane == 0 && j == 0) atomicOr(&g_device_error, kErrRange);
+    if (lane == 0 && j == 0) atomicOr(p.err, kErrRange);
     return;
   }
   if ((lane >> 2) != row % kTileRows) return;
@@ -839,7 +847,7 @@ __global__ void __launch_bounds__(256) gather_kernel(GatherParams p) {
     const int64_t col = j * p.tile_cols + 64 * (k / 16) + 16 * c + (k % 16);
     if (col < p.cols) orow[col] = (uint16_t)(((r & 0x80u) << 8) | (s << 7) | (r & 0x7Fu));
   }
-  if (bad) atomicOr(&g_device_error, kErrCorrupt);
+  if (bad) atomicOr(p.err, kErrCorrupt);
 }
 
 // Raises a kernel's dynamic shared-memory limit on the current device once per
@@ -967,13 +975,6 @@ cudaError_t launch_gather(const GatherParams& g, cudaStream_t stream) {
   if (blocks < 1 || blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
   gather_kernel<<<(unsigned)blocks, 256, 0, stream>>>(g);
   return cudaGetLastError();
-}
-
-cudaError_t read_and_clear_error(uint32_t* word) {
-  uint32_t zero = 0;
-  cudaError_t e = cudaMemcpyFromSymbol(word, g_device_error, sizeof(uint32_t));
-  if (e != cudaSuccess) return e;
-  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(uint32_t));
 }
 
 }  // namespace nwc

@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "nwc_format.h"
+
 namespace nwc {
 
 // Barrier slots per CTA: batches in flight or resident at once are fewer.
@@ -12,13 +14,15 @@ constexpr int kSlots = 64;
 // schedule relies on it.
 constexpr int kMaxLag = 48;
 
-// Rows of x one GEMV launch handles (one 16-row tensor-core operand).
-constexpr int kMaxPassRows = 16;
-
-// Device error word bits (read and cleared by nwc_get_device_error).
+// Device error word bits (the first word of a device image's scratch area;
+// read and cleared by nwc_get_device_error).
 constexpr uint32_t kErrTimeout = 1u;   // a bounded mbarrier wait gave up
 constexpr uint32_t kErrCorrupt = 2u;   // a stream held no valid code
 constexpr uint32_t kErrRange = 4u;     // a gathered row id was out of range
+
+// Polls of a bounded mbarrier wait before it gives up (TileParams.wait_limit
+// 0 means this).
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 
 struct TileParams {
   const uint8_t* tiles;     // device: tile area of the blob
@@ -42,6 +46,8 @@ struct TileParams {
   int64_t rows_pad;         // 8 * tiles_r
   // decompress
   uint16_t* out;            // BF16 [rows x cols]
+  uint32_t* err;            // device: the handle's error word
+  uint32_t wait_limit;      // polls before a bounded wait gives up (0: default)
 };
 
 // Shared memory that a CTA reserves for its columns of x, by x-stage class:
@@ -94,9 +100,8 @@ struct GatherParams {
   const int32_t* row_ids;   // device: n row ids
   int32_t n;
   uint16_t* out;            // device: BF16 [n x cols]
+  uint32_t* err;            // device: the handle's error word
 };
 cudaError_t launch_gather(const GatherParams& g, cudaStream_t stream);
-
-cudaError_t read_and_clear_error(uint32_t* word);
 
 }  // namespace nwc

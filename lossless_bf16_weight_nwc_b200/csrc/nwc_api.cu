@@ -6,6 +6,7 @@
 
 #include <cstddef>
 #include <cstdlib>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -24,6 +25,9 @@ constexpr int kMaxDevices = 64;
 int g_sm_count[kMaxDevices] = {};
 int g_smem_optin[kMaxDevices] = {};
 std::mutex g_mu;
+// Polls before a bounded wait in a kernel gives up; 0 = the kernels' default.
+// Set only by nwc_test_set_wait_limit.
+std::atomic<uint32_t> g_wait_limit{0};
 
 nwc_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NWC_OK : NWC_ERR_CUDA; }
 
@@ -128,6 +132,10 @@ nwc_status parse(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_h
   }
 }
 
+uint32_t* error_word(const nwc_handle_s& h) {
+  return reinterpret_cast<uint32_t*>(h.d_base + h.scratch_off);
+}
+
 nwc::TileParams base_params(const nwc_handle_s& h, int cls, const nwc::LaunchShape& s) {
   nwc::TileParams p;
   std::memset(&p, 0, sizeof(p));
@@ -148,16 +156,26 @@ nwc::TileParams base_params(const nwc_handle_s& h, int cls, const nwc::LaunchSha
   p.ring_bytes = s.ring_bytes;
   p.batch_tiles = s.batch_tiles;
   p.xstage_bytes = s.xstage_bytes;
+  p.err = error_word(h);
+  p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
   return p;
 }
 
 constexpr int kChunkBatch = nwc::kMaxPassRows;  // rows of x per kernel launch
 
-uint64_t workspace_bytes_for(const nwc_handle_s& h, int32_t batch) {
+// Split-K scratch one GEMV call of `batch` rows uses: the arrival counters
+// (padded to 256 bytes) and the partial sums of one launch.
+uint64_t scratch_bytes_for(const nwc_handle_s& h, int32_t batch) {
   if (h.tiles_c <= 1) return 0;
   const int b = batch < kChunkBatch ? batch : kChunkBatch;
-  const uint64_t counters = round_up(4ull * (uint64_t)h.tiles_r, 256);
-  return counters + 4ull * (uint64_t)h.tiles_c * (uint64_t)b * (uint64_t)(8 * h.tiles_r);
+  return round_up(4ull * (uint64_t)h.tiles_r, 256) +
+         nwc::split_partial_bytes((uint64_t)h.tiles_r, (uint64_t)h.tiles_c, (uint64_t)b);
+}
+
+// Zeroes the error word and the arrival counters of a handle's scratch area.
+cudaError_t clear_scratch(const nwc_handle_s& h, cudaStream_t stream) {
+  return cudaMemsetAsync(h.d_base + h.scratch_off, 0,
+                         nwc::scratch_partial_off((uint64_t)h.tiles_r), stream);
 }
 
 nwc_status make_handle(const uint8_t* blob_host_header_region, uint64_t bytes, void* d_buf,
@@ -289,7 +307,8 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
   // No kernel reads these layouts yet.
   if (plan->code_kind != NWC_CODE_PREFIX || plan->streams != 1) return NWC_ERR_UNSUPPORTED;
   if (d_bytes < plan->device_bytes || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
-  uint8_t* img = static_cast<uint8_t*>(std::malloc(plan->device_bytes));
+  uint8_t* img = static_cast<uint8_t*>(std::malloc(
+      plan->scratch_off + nwc::scratch_partial_off((uint64_t)plan->tiles_r)));
   if (!img) return NWC_ERR_NOMEM;
   try {
     nwc::encode_blob(*plan, w_host, img);
@@ -301,12 +320,17 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
   nwc::build_decode_table(plan->len, plan->lmax, reinterpret_cast<uint32_t*>(img + plan->table_off));
   const uint64_t table_end = plan->table_off + nwc::table_bytes(plan->lmax);
   std::memset(img + table_end, 0, plan->sched_off - table_end);
+  // The scratch area starts with the error word and the arrival counters,
+  // which must be zero; the partial sums are written before they are read.
+  const uint64_t scratch_head = nwc::scratch_partial_off((uint64_t)plan->tiles_r);
+  std::memset(img + plan->scratch_off, 0, scratch_head);
+  const uint64_t upload = plan->scratch_off + scratch_head;
   nwc_handle_t h = nullptr;
   nwc_status st = make_handle(img, plan->blob_bytes, d_buf, d_bytes, &h, nullptr);
   if (st == NWC_OK) st = init_schedule(h, img, nullptr);
   // From pageable memory the call returns once the bytes are staged, so the
   // image can be freed right after.
-  if (st == NWC_OK && cudaMemcpyAsync(d_buf, img, plan->device_bytes, cudaMemcpyHostToDevice,
+  if (st == NWC_OK && cudaMemcpyAsync(d_buf, img, upload, cudaMemcpyHostToDevice,
                                       reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     st = NWC_ERR_CUDA;
   std::free(img);
@@ -352,6 +376,7 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, u
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(static_cast<uint8_t*>(d_buf) + h->table_off, table.data(),
                         nwc::table_bytes(h->lmax), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = clear_scratch(*h, s);
   if (e == cudaSuccess) {
     st = init_schedule(h, nullptr, s);
     if (st != NWC_OK) {
@@ -398,6 +423,7 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
   h->d_bytes = d_bytes;
   cudaGetDevice(&h->device);
   st = init_schedule(h, nullptr, nullptr);
+  if (st == NWC_OK && clear_scratch(*h, nullptr) != cudaSuccess) st = NWC_ERR_CUDA;
   if (st == NWC_OK && cudaStreamSynchronize(nullptr) != cudaSuccess) st = NWC_ERR_CUDA;
   if (st != NWC_OK) {
     delete h;
@@ -440,25 +466,38 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
   g.row_ids = d_rows;
   g.n = n;
   g.out = d_out;
+  g.err = error_word(*h);
   return cuda_status(nwc::launch_gather(g, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-nwc_status nwc_gemv_workspace_size(nwc_handle_t h, int32_t batch, uint64_t* bytes) {
+nwc_status nwc_gemv_scratch_bytes(nwc_handle_t h, int32_t batch, uint64_t* bytes) {
   if (!h || !bytes || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
-  *bytes = workspace_bytes_for(*h, batch);
+  *bytes = scratch_bytes_for(*h, batch);
   return NWC_OK;
 }
 
-nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t batch,
-                    void* d_workspace, uint64_t workspace_bytes, nwc_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the GEMV entry points, done before anything is enqueued.
+nwc_status gemv_check(const nwc_handle_s* h, const uint16_t* d_x, const float* d_y,
+                      int32_t batch) {
   if (!h || !d_x || !d_y || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
   if (!aligned(d_x, 4) || !aligned(d_y, 4) || (h->cols & 1)) return NWC_ERR_INVALID_ARG;
-  const uint64_t need = workspace_bytes_for(*h, batch);
-  if (need && (!d_workspace || workspace_bytes < need || !aligned(d_workspace, 16)))
-    return NWC_ERR_INVALID_ARG;
   // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
   if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
-  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;
+  if (dev != h->device) return NWC_ERR_INVALID_ARG;
+  return NWC_OK;
+}
+
+// The GEMV launches, with split-K scratch at `counters` (u32 [tiles_r], zero
+// on entry and left zero) and `partial` (scratch_bytes_for bytes less the
+// counters' 256-byte-padded area).
+nwc_status gemv_run(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t batch,
+                    uint32_t* counters, float* partial, cudaStream_t cs) {
   for (int32_t b0 = 0; b0 < batch; b0 += kChunkBatch) {
     const int32_t nb = batch - b0 < kChunkBatch ? batch - b0 : kChunkBatch;
     // The x-stage class (and with it the schedule and ring) follows the rows
@@ -468,11 +507,8 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
     nwc_status st = shape_for(h, cls, &s, cs);
     if (st != NWC_OK) return st;
     nwc::TileParams p = base_params(*h, cls, s);
-    if (need) {
-      uint8_t* ws = static_cast<uint8_t*>(d_workspace);
-      p.counters = reinterpret_cast<uint32_t*>(ws);
-      p.partial = reinterpret_cast<float*>(ws + round_up(4ull * (uint64_t)h->tiles_r, 256));
-    }
+    p.counters = counters;
+    p.partial = partial;
     p.x = d_x + (int64_t)b0 * h->cols;
     p.y = d_y + (int64_t)b0 * h->rows;
     p.batch = nb;
@@ -486,10 +522,10 @@ nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t bat
 // one copy per device.  Host code must not hand `g_noalloc_scratch` itself to a
 // kernel (on the host that name is a stand-in, not a device address); the
 // device address comes from cudaGetSymbolAddress, looked up once per device.
-static __device__ __align__(256) unsigned char g_noalloc_scratch[NWC_NOALLOC_SCRATCH_BYTES];
-static void* g_noalloc_addr[kMaxDevices] = {};
+__device__ __align__(256) unsigned char g_noalloc_scratch[NWC_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_addr[kMaxDevices] = {};
 
-static nwc_status noalloc_scratch(void** out) {
+nwc_status noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return NWC_ERR_UNSUPPORTED;
@@ -504,45 +540,78 @@ static nwc_status noalloc_scratch(void** out) {
   return NWC_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+nwc_status nwc_gemv(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t batch,
+                    nwc_stream_t stream) {
+  nwc_status st = gemv_check(h, d_x, d_y, batch);
+  if (st != NWC_OK) return st;
+  uint8_t* scratch = h->d_base + h->scratch_off;
+  return gemv_run(h, d_x, d_y, batch,
+                  reinterpret_cast<uint32_t*>(scratch + nwc::kScratchCountersOff),
+                  reinterpret_cast<float*>(scratch + nwc::scratch_partial_off((uint64_t)h->tiles_r)),
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
 nwc_status nwc_gemv_noalloc(nwc_handle_t h, const uint16_t* d_x, float* d_y, int32_t batch,
                             nwc_stream_t stream) {
-  if (!h || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
-  const uint64_t need = workspace_bytes_for(*h, batch);
+  // Every argument is checked before the shared array is touched, so a
+  // rejected call enqueues nothing.
+  nwc_status st = gemv_check(h, d_x, d_y, batch);
+  if (st != NWC_OK) return st;
+  const uint64_t need = scratch_bytes_for(*h, batch);
   if (need > NWC_NOALLOC_SCRATCH_BYTES) return NWC_ERR_SCRATCH_LIMIT;
-  void* ws = nullptr;
+  uint8_t* ws = nullptr;
   if (need) {
-    nwc_status st = noalloc_scratch(&ws);
+    void* addr = nullptr;
+    st = noalloc_scratch(&addr);
     if (st != NWC_OK) return st;
+    ws = static_cast<uint8_t*>(addr);
     // The array keeps the previous call's bytes: the arrival counters must
     // start at zero, the partial sums are overwritten before they are read.
     if (cudaMemsetAsync(ws, 0, 4ull * (uint64_t)h->tiles_r,
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
       return NWC_ERR_CUDA;
   }
-  return nwc_gemv(h, d_x, d_y, batch, ws, need, stream);
+  return gemv_run(h, d_x, d_y, batch, reinterpret_cast<uint32_t*>(ws),
+                  ws ? reinterpret_cast<float*>(ws + round_up(4ull * (uint64_t)h->tiles_r, 256))
+                     : nullptr,
+                  reinterpret_cast<cudaStream_t>(stream));
 }
 
 nwc_status nwc_handle_info(nwc_handle_t h, int64_t* rows, int64_t* cols, uint64_t* blob_bytes,
-                           uint64_t* device_bytes) {
+                           uint64_t* device_bytes, uint64_t* compressed_bytes) {
   if (!h) return NWC_ERR_INVALID_ARG;
   if (rows) *rows = h->rows;
   if (cols) *cols = h->cols;
   if (blob_bytes) *blob_bytes = h->blob_bytes;
   if (device_bytes) *device_bytes = h->device_bytes;
+  if (compressed_bytes) *compressed_bytes = h->scratch_off;
   return NWC_OK;
 }
 
-nwc_status nwc_get_device_error(nwc_stream_t stream, uint32_t* word) {
-  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return NWC_ERR_CUDA;
+nwc_status nwc_get_device_error(nwc_handle_t h, nwc_stream_t stream, uint32_t* word) {
+  if (!h) return NWC_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint32_t w = 0;
-  e = nwc::read_and_clear_error(&w);
+  cudaError_t e = cudaMemcpyAsync(&w, error_word(*h), sizeof(w), cudaMemcpyDeviceToHost, cs);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(cs);
   if (e != cudaSuccess) return NWC_ERR_CUDA;
+  // A kernel that gave up may have left arrival counters behind: clear them
+  // with the word so that the next call starts from zero.
+  if (w && (clear_scratch(*h, cs) != cudaSuccess || cudaStreamSynchronize(cs) != cudaSuccess))
+    return NWC_ERR_CUDA;
   if (word) *word = w;
   if (w & nwc::kErrTimeout) return NWC_ERR_DEVICE_TIMEOUT;
   if (w & nwc::kErrCorrupt) return NWC_ERR_DEVICE_CORRUPT;
   if (w & nwc::kErrRange) return NWC_ERR_INVALID_ARG;
   return NWC_OK;
+}
+
+void nwc_test_set_wait_limit(uint32_t polls) {
+  g_wait_limit.store(polls, std::memory_order_relaxed);
 }
 
 nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,

@@ -23,9 +23,11 @@
 //
 // Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)]
 // | zero pad to 256 | launch schedules (sched_bytes(tiles) bytes: one per
-// x-stage class, each sched_class_bytes(tiles)).  They are not part of the
-// blob: the library writes them for the device that runs the kernels (its SM
-// count and shared memory), each as
+// x-stage class, each sched_class_bytes(tiles)) | scratch (scratch_bytes:
+// the error word, the split-K arrival counters and partial sums that the
+// kernels write).  None of it is part of the blob: the library writes the
+// table and schedules for the device that runs the kernels (its SM count and
+// shared memory), each schedule as
 //   u32 cta_batch[kMaxCtas + 1]   first batch of each CTA (padded to 16 bytes)
 //   u32x4 batch[sched_max_batches(tiles)]
 //        {tile-area offset in 16-byte units, bytes, ring offset, batches of
@@ -100,6 +102,48 @@ constexpr uint64_t sched_class_bytes(uint64_t tiles) {
   return round_up(sched_tile_off(tiles) + 4ull * tiles, 256);
 }
 constexpr uint64_t sched_bytes(uint64_t tiles) { return kStageClasses * sched_class_bytes(tiles); }
+
+// Rows of x one launch of the CUDA-core GEMV kernel handles (one 16-row
+// tensor-core operand of mma.sync); larger batches run as several launches.
+constexpr int kMaxPassRows = 16;
+// Rows of x the tensor-core (tcgen05) kernel handles in one launch.
+constexpr int kMaxTcRows = 64;
+
+// Scratch area of the device image, written by the kernels of the handle
+// (calls on one handle must therefore be ordered):
+//   u32 error word (kErr* bits) | pad to 256
+//   u32 arrival counters [tiles_r] | pad to 256
+//   FP32 partial sums: the split-K partials of one CUDA-core launch
+//   [tiles_c][kMaxPassRows][8 tiles_r], or the tensor-core kernel's partial row
+//   tiles at CTA boundaries [2 kMaxCtas][8][kMaxTcRows], whichever is larger;
+//   none when the matrix has one column tile.
+constexpr uint64_t kScratchCountersOff = 256;
+constexpr uint64_t scratch_partial_off(uint64_t tiles_r) {
+  return kScratchCountersOff + round_up(4ull * tiles_r, 256);
+}
+constexpr uint64_t split_partial_bytes(uint64_t tiles_r, uint64_t tiles_c, uint64_t rows_of_x) {
+  return tiles_c <= 1 ? 0 : 4ull * tiles_c * rows_of_x * 8ull * tiles_r;
+}
+constexpr uint64_t tc_partial_bytes(uint64_t tiles_c) {
+  return tiles_c <= 1 ? 0 : 4ull * 2ull * kMaxCtas * 8ull * (uint64_t)kMaxTcRows;
+}
+constexpr uint64_t scratch_bytes(uint64_t tiles_r, uint64_t tiles_c) {
+  const uint64_t a = split_partial_bytes(tiles_r, tiles_c, kMaxPassRows), b = tc_partial_bytes(tiles_c);
+  return round_up(scratch_partial_off(tiles_r) + (a > b ? a : b), 256);
+}
+
+// Offsets of the device image's derived parts after a blob of blob_bytes.
+struct ImageLayout {
+  uint64_t table_off, sched_off, scratch_off, device_bytes;
+};
+constexpr ImageLayout image_layout(uint64_t blob_bytes, uint32_t lmax, uint64_t tiles_r,
+                                   uint64_t tiles_c) {
+  const uint64_t table_off = round_up(blob_bytes, 256);
+  const uint64_t sched_off = round_up(table_off + table_bytes(lmax), 256);
+  const uint64_t scratch_off = round_up(sched_off + sched_bytes(tiles_r * tiles_c), 256);
+  return ImageLayout{table_off, sched_off, scratch_off,
+                     scratch_off + scratch_bytes(tiles_r, tiles_c)};
+}
 
 struct BlobHeader {
   uint32_t magic, version, header_bytes, lmax;

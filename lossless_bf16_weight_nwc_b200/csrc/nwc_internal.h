@@ -26,7 +26,8 @@ struct nwc_plan_s {
   uint64_t blob_bytes = 0;      // serialisable blob
   uint64_t table_off = 0;       // device-image offset of the decode table
   uint64_t sched_off = 0;       // device-image offset of the launch schedule
-  uint64_t device_bytes = 0;    // blob + padding + decode table + schedule
+  uint64_t scratch_off = 0;     // device-image offset of the scratch area
+  uint64_t device_bytes = 0;    // blob + padding + decode table + schedules + scratch
 };
 
 struct nwc_handle_s {
@@ -35,7 +36,8 @@ struct nwc_handle_s {
   int64_t rows = 0, cols = 0;
   uint32_t tile_cols = 512, lmax = 7, filler = 0;
   int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
-  uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0, sched_off = 0;
+  uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0, sched_off = 0,
+           scratch_off = 0;
   uint64_t device_bytes = 0;
   uint64_t max_chunk = 0;  // largest chunk in bytes
   int device = 0;

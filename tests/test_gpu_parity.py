@@ -48,9 +48,11 @@ def tolerance_check(y_gpu: np.ndarray, y_ref: np.ndarray, w: np.ndarray, x: np.n
     return worst, rel
 
 
-def no_device_error(lib):
-    st, word = lib.nwc_get_device_error()
-    assert st == 0, f"device error word {word:#x}"
+def no_device_error(lib, *mats):
+    """Each matrix's (or raw handle's) device error word is clear."""
+    for m in mats:
+        st, word = m.device_error() if hasattr(m, "device_error") else lib.nwc_get_device_error(m)
+        assert st == 0, f"device error word {word:#x}"
 
 
 SHAPES = [((8, 512), 512), ((9, 513), 512), ((77, 1030), 512), ((1, 2), 512),
@@ -68,7 +70,7 @@ def test_decompress_bit_exact(lib, orc, shape, tile_cols, lmax):
     ref = orc.decode(orc.encode(w, tile_cols=tile_cols, lmax=lmax))
     assert np.array_equal(ref, w)
     assert np.array_equal(out, ref)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_decompress_every_pattern(lib, orc):
@@ -76,11 +78,12 @@ def test_decompress_every_pattern(lib, orc):
     for tile_cols, lmax in ((512, 12), (128, 8), (256, 0)):
         m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
         assert np.array_equal(bits(m.decompress()), w)
+        no_device_error(lib, m)
     rng = np.random.default_rng(0)
     shuffled = rng.permutation(w.reshape(-1)).reshape(128, 512)
     m = lib.CompressedMatrix.compress(shuffled)
     assert np.array_equal(bits(m.decompress()), shuffled)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 @pytest.mark.parametrize("lmax", [7, 9, 12])
@@ -93,7 +96,7 @@ def test_gpu_decodes_oracle_blob(lib, orc, lmax):
     x = synth.activations(1, 2, spec.cols)
     y = m.gemv(to_bf16(x)).cpu().numpy()
     tolerance_check(y, orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 @pytest.mark.parametrize("lmax", [0, 12])
@@ -108,7 +111,7 @@ def test_gemv_parity_shapes(lib, orc, shape, tile_cols, batch, lmax):
     m = lib.CompressedMatrix.compress(w, tile_cols=tile_cols, lmax=lmax)
     y = m.gemv(to_bf16(x)).cpu().numpy()
     tolerance_check(y, orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 @pytest.mark.parametrize("lmax", [0, 10])
@@ -120,7 +123,7 @@ def test_gemv_every_batch(lib, orc, batch, lmax):
     m = lib.CompressedMatrix.compress(w, lmax=lmax)
     y = m.gemv(to_bf16(x)).cpu().numpy()
     tolerance_check(y, orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_auto_lmax_and_fast_path(lib, orc):
@@ -139,7 +142,7 @@ def test_auto_lmax_and_fast_path(lib, orc):
     assert int.from_bytes(blob[12:16].tobytes(), "little") == 8
 
 
-def test_gemv_deterministic_and_workspace_reuse(lib, orc):
+def test_gemv_deterministic_and_scratch_reuse(lib, orc):
     spec = synth.MatrixSpec("w", 2048, 4096, "normal", 0.02, 0)
     w = synth.matrix(spec, 8)
     x = synth.activations(8, 4, spec.cols)
@@ -150,7 +153,7 @@ def test_gemv_deterministic_and_workspace_reuse(lib, orc):
         again = m.gemv(xt).cpu().numpy()
         assert np.array_equal(first.view(np.uint32), again.view(np.uint32))
     tolerance_check(first, orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 @pytest.mark.parametrize("batch", [1, 16])
@@ -167,7 +170,7 @@ def test_fused_projections(lib, orc, batch):
     ys = m.split(m.gemv(to_bf16(x)))
     for w, y in zip(ws, ys):
         tolerance_check(y.cpu().numpy(), orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_autotune_picks_a_timed_candidate(lib, orc):
@@ -182,7 +185,7 @@ def test_autotune_picks_a_timed_candidate(lib, orc):
     m = lib.CompressedMatrix.compress(w, tile_cols=choice.tile_cols, lmax=choice.lmax)
     x = synth.activations(3, 1, spec.cols)
     tolerance_check(m.gemv(to_bf16(x)).cpu().numpy(), orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_sharded_matrix_single_process(lib, orc):
@@ -195,8 +198,8 @@ def test_sharded_matrix_single_process(lib, orc):
     assert m.ranges == [(0, 300)] and m.local is not None
     x = synth.activations(7, 2, spec.cols)
     tolerance_check(m.gemv(to_bf16(x)).cpu().numpy(), orc.gemv(w, x), w, x)
+    no_device_error(lib, m.local)
     m.close()
-    no_device_error(lib)
 
 
 def test_gemv_into_pinned_host_memory(lib, orc):
@@ -207,11 +210,10 @@ def test_gemv_into_pinned_host_memory(lib, orc):
     x = synth.activations(5, 3, spec.cols)
     m = lib.CompressedMatrix.compress(w)
     yh = torch.full((3, spec.rows), float("nan"), dtype=torch.float32).pin_memory()
-    ws, nb = m.workspace(3)
-    lib.nwc_gemv(m.handle, to_bf16(x), yh, 3, ws, nb)
+    lib.nwc_gemv(m.handle, to_bf16(x), yh, 3)
     torch.cuda.synchronize()
     tolerance_check(yh.numpy(), orc.gemv(w, x), w, x)
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 @pytest.mark.parametrize("lmax", [0, 12])
@@ -226,7 +228,7 @@ def test_gather_rows(lib, shape, tile_cols, lmax):
     ids = np.concatenate([[0, shape[0] - 1], rng.integers(0, shape[0], 37)]).astype(np.int32)
     out = m.gather_rows(torch.from_numpy(ids).cuda())
     assert np.array_equal(bits(out), w[ids])
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_gather_rows_every_pattern(lib):
@@ -236,7 +238,7 @@ def test_gather_rows_every_pattern(lib):
     m = lib.CompressedMatrix.compress(w)
     ids = np.arange(255, -1, -1, dtype=np.int32)
     assert np.array_equal(bits(m.gather_rows(torch.from_numpy(ids).cuda())), w[ids])
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_gather_rows_out_of_range(lib):
@@ -245,11 +247,11 @@ def test_gather_rows_out_of_range(lib):
     out = torch.zeros((2, 512), dtype=torch.int16, device="cuda")
     ids = torch.tensor([5, 24], dtype=torch.int32, device="cuda")
     lib.nwc_gather_rows(m.handle, ids, 2, out)
-    st, word = lib.nwc_get_device_error()
+    st, word = m.device_error()
     assert st == 1 and word & 4                     # INVALID_ARG: a row id out of range
     assert np.array_equal(out[0].cpu().numpy().view(np.uint16), w[5])
     assert not out[1].any()                         # left unwritten
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 def test_handle_from_device_image(lib, orc):
@@ -261,8 +263,8 @@ def test_handle_from_device_image(lib, orc):
     out = torch.empty((96, 1536), dtype=torch.bfloat16, device="cuda")
     lib.nwc_decompress(h, out)
     assert np.array_equal(bits(out), w)
+    no_device_error(lib, h, m)
     lib.nwc_handle_destroy(h)
-    no_device_error(lib)
 
 
 def test_invalid_arguments_rejected(lib):
@@ -274,10 +276,8 @@ def test_invalid_arguments_rejected(lib):
         lib.nwc_gemv(m.handle, x, y, 0)
     with pytest.raises(lib.NwcError):
         lib.nwc_gemv(m.handle, x, y, 65)
-    with pytest.raises(lib.NwcError):            # workspace required (2 column tiles)
-        lib.nwc_gemv(m.handle, x, y, 1, None, 0)
     with pytest.raises(lib.NwcError):            # misaligned x
-        lib.nwc_gemv(m.handle, x.data_ptr() + 2, y, 1, *m.workspace(1))
+        lib.nwc_gemv(m.handle, x.data_ptr() + 2, y, 1)
     odd = lib.CompressedMatrix.compress(synth.matrix(synth.MatrixSpec("w", 4, 5, "normal", 0.02, 0), 0))
     x5 = torch.zeros((1, 5), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lib.NwcError):            # odd column count
@@ -290,7 +290,7 @@ def test_invalid_arguments_rejected(lib):
     with pytest.raises(ValueError):              # nor a y smaller than the output
         m.gemv(x, y=torch.zeros((1, 15), dtype=torch.float32, device="cuda"))
     assert m.gather_rows(torch.tensor([3, 0])).shape == (2, 1024)  # host ids are moved
-    no_device_error(lib)
+    no_device_error(lib, m)
 
 
 # ---- the benchmark workloads at full size ------------------------------------
@@ -307,8 +307,8 @@ def test_workload_full_parity(lib, orc, name):
             x = synth.activations(wl.seed, batch, spec.cols)
             y = m.gemv(to_bf16(x)).cpu().numpy()
             tolerance_check(y, orc.gemv(w, x), w, x)
+        no_device_error(lib, m)
         m.close()
-    no_device_error(lib)
 
 
 def test_workload_mlp_pair_full(lib, orc):
@@ -321,5 +321,5 @@ def test_workload_mlp_pair_full(lib, orc):
             x = synth.activations(wl.seed, batch, spec.cols)
             y = m.gemv(to_bf16(x)).cpu().numpy()
             tolerance_check(y, orc.gemv(w, x), w, x)
+        no_device_error(lib, m)
         m.close()
-    no_device_error(lib)

@@ -45,8 +45,8 @@ def test_stack_shapes_full_size(lib, orc, name):
             x = synth.activations(wl.seed, batch, spec.cols)
             y = m.gemv(to_bf16(x)).cpu().numpy()
             tolerance_check(y[:, idx], orc.gemv(w[idx], x), w[idx], x)
+        no_device_error(lib, m)
         m.close()
-        no_device_error(lib)
 
 
 @pytest.mark.parametrize("name", ["qwen3_4b_stack", "llama31_8b_stack"])
@@ -64,5 +64,5 @@ def test_stacked_projections_full_size(lib, orc, name):
             for p, w, y in zip(parts, ws, ys):
                 idx = np.unique(np.linspace(0, p.rows - 1, 128).astype(np.int64))
                 tolerance_check(y.cpu().numpy()[:, idx], orc.gemv(w[idx], x), w[idx], x)
+        no_device_error(lib, m)
         m.close()
-        no_device_error(lib)
