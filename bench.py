@@ -59,6 +59,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--e2e-mode", default="host-y", choices=["copy", "host-y"],
                     help="how y reaches the host in the end-to-end leg")
+    ap.add_argument("--report", action="store_true",
+                    help="the five configurations as a markdown table (not the headline line)")
+    ap.add_argument("--report-json", default=None, help="with --report: every line, to this file")
     ap.add_argument("--fuse", action="store_true",
                     help="stacks: q, k, v and gate, up each run as one stacked matrix")
     return ap.parse_args()
@@ -342,7 +345,10 @@ def run_stack(args) -> None:
     ys = {n: torch.empty((batch, n), dtype=torch.float32, device=dev) for n in {sp.rows for sp in specs}}
     stream = torch.cuda.Stream(device=dev)
     seq = [(sets[l % 2][sp.name], sp) for l in range(n_layers) for sp in layer0] + [(comp[head.name], head)]
-    launches = len(seq) * ((batch + 15) // 16)
+    paths = [_lib.nwc_gemv_path(m.handle, xs[sp.cols], batch) for m, sp in seq]
+    launches = sum(n for n, _ in paths)
+    kernel = "gemv_tc_kernel" if all(tc for _, tc in paths) else \
+        "gemv_kernel" if not any(tc for _, tc in paths) else "gemv_kernel+gemv_tc_kernel"
 
     def token(y_head=None):
         for m, sp in seq:
@@ -483,42 +489,26 @@ def run_stack(args) -> None:
         "footprint_ratio": weight_bytes / image_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": None,
-                     "peak_source": f"{peak_src} hbm_gbs (copy)", "kernel": "gemv_kernel",
+                     "peak_source": f"{peak_src} hbm_gbs (copy)", "kernel": kernel,
                      "basis": "algorithmic bytes of the token's GEMVs / graph time per token",
                      "tokens_per_s_ceiling_at_peak": hbm * 1e9 / alg},
         "clocks": clocks.summary(),
         "e2e": e2e,
         "gpu_launches": steps * launches,
+        "kernel_path": kernel,
         "parity_spot_check": parity_ok,
         "cublas_bf16": cublas,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, batch)
         line["cpu_baseline"].pop("us_per_call", None)
-    if rank == 0:
-        print(json.dumps(line))
     del g
-    if world > 1:
-        import torch.distributed as dist
-        dist.destroy_process_group()
+    return line if rank == 0 else None
 
 
-def main():
-    args = parse_args()
-    if args.steps is None and args.workload not in STACKS:
-        args.steps = 20000
-    if args.warmup is None and args.workload not in STACKS:
-        args.warmup = 200
-    if args.impl == "reference":
-        if args.steps is None:
-            args.steps = 50
-        if args.warmup is None:
-            args.warmup = 3
-        run_reference(args)
-        return
-    if args.workload in STACKS:
-        run_stack(args)
-        return
+def run_matrix(args):
+    """One matrix of the workload: a step is one nwc_gemv call, rotating over
+    enough compressed copies that the weights never sit in L2."""
     import torch
 
     from lossless_bf16_weight_nwc_b200 import _lib, synth
@@ -539,7 +529,8 @@ def main():
         m.handle = _lib.nwc_handle_from_device(m.image, m.image.numel())
     x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
     y = torch.empty((batch, spec.rows), dtype=torch.float32, device=dev)
-    launches_per_call = (batch + 15) // 16  # rows of x per kernel launch: 16
+    launches_per_call, on_tc = _lib.nwc_gemv_path(first.handle, x, batch)
+    kernel = "gemv_tc_kernel" if on_tc else "gemv_kernel"
     stream = torch.cuda.Stream(device=dev)
 
     def call(m, s):
@@ -717,26 +708,90 @@ def main():
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
                      "peak_source": f"{peak_src} hbm_gbs (copy)",
-                     "kernel": "gemv_kernel", "kernel_us": kernel_ms * 1e3,
+                     "kernel": kernel, "kernel_us": kernel_ms * 1e3,
                      "basis": "algorithmic bytes per launch / timed-region event time per launch",
                      "isolated_launch_us": isolated_ms * 1e3,
                      "algorithmic_bytes_per_launch": alg_bytes},
         "clocks": clock,
         "e2e": e2e,
         "gpu_launches": steps * launches_per_call,
+        "kernel_path": kernel,
         "parity_spot_check": parity_ok,
         "cublas_bf16": cublas,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.workload, batch)
         line["cpu_baseline"].pop("us_per_call", None)
-    if rank == 0:
-        print(json.dumps(line))
     # Release graphs before the process group.
     del g, g_rest
-    if world > 1:
+    return line if rank == 0 else None
+
+
+def main():
+    args = parse_args()
+    if args.steps is None and args.workload not in STACKS:
+        args.steps = 20000
+    if args.warmup is None and args.workload not in STACKS:
+        args.warmup = 200
+    if args.impl == "reference":
+        if args.steps is None:
+            args.steps = 50
+        if args.warmup is None:
+            args.warmup = 3
+        run_reference(args)
+        return
+    if args.report:
+        run_report(args)
+        return
+    line = run_stack(args) if args.workload in STACKS else run_matrix(args)
+    if line is not None:
+        print(json.dumps(line))
+    if int(os.environ.get("WORLD_SIZE", 1)) > 1:
         import torch.distributed as dist
-        dist.destroy_process_group()
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def run_report(args) -> None:
+    """The five benchmark configurations in one run, as a markdown table
+    (and every configuration's JSON line in --report-json when given): per
+    call or per token, effective and compressed GB/s, fraction of the HBM
+    peak, compression ratio, the uncompressed cuBLAS time and the kernel
+    path."""
+    rows = [("single_1024", 1), ("attn_4096_outliers", 1), ("attn_4096_outliers", 4),
+            ("mlp_pair_t5", 1), ("mlp_pair_t5", 2), ("mlp_pair_t5", 8),
+            ("qwen3_4b_stack", 1), ("llama31_8b_stack", 1), ("llama31_8b_stack", 16),
+            ("llama31_8b_stack", 64)]
+    lines = []
+    for workload, batch in rows:
+        a = argparse.Namespace(**vars(args))
+        a.workload, a.batch, a.report = workload, batch, False
+        a.no_cpu_baseline = True
+        a.e2e_steps = 0
+        stack = workload in STACKS
+        a.steps = args.steps if args.steps is not None else (10 if stack else 4000)
+        a.warmup = 3 if stack else 50
+        line = run_stack(a) if stack else run_matrix(a)
+        lines.append(line)
+        print(f"{workload} b{batch}: {line['ms_per_step'] * 1e3:.2f} us", file=sys.stderr, flush=True)
+    print("| workload | batch | µs per step | effective GB/s | compressed GB/s | fraction of HBM "
+          "peak | ratio | cuBLAS BF16 µs | kernel |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for (workload, batch), line in zip(rows, lines):
+        rf = line["roofline"]
+        comp = line.get("compressed_bytes") or line.get("compressed_bytes_per_token")
+        us = line["ms_per_step"] * 1e3
+        cb = line.get("cublas_bf16") or {}
+        cb_us = cb.get("us_per_call") or cb.get("us_per_token")
+        print(f"| {workload} | {batch} | {us:.2f} | {line['value']:.0f} | "
+              f"{comp / (us * 1e-6) / 1e9:.0f} | {rf['frac']:.3f} ({rf['peak_source']}) | "
+              f"{line['compression_ratio']:.3f} | {cb_us:.2f} | {line.get('kernel_path')} |")
+    if args.report_json:
+        with open(args.report_json, "w") as f:
+            for line in lines:
+                f.write(json.dumps(line) + "\n")
+
+
 
 
 if __name__ == "__main__":

@@ -232,7 +232,8 @@ nwc_status nwc_gemv_scratch_bytes(nwc_handle_t handle, int32_t batch, uint64_t* 
  * (row, column block); "Unweight", "Direct GPU Decompression": weights are
  * decompressed in shared memory and fed to the tensor cores, never written
  * back): y[b][n] = sum_k W[n][k] * x[b][k], for b < batch, n < rows, k < cols.
- *   d_x: device, BF16 [batch x cols], row-major, 4-byte aligned, cols even.
+ *   d_x: device, BF16 [batch x cols], row-major, 4-byte aligned (2-byte when
+ *     cols is odd).
  *   d_y: FP32 [batch x rows], row-major (overwritten, not accumulated), in
  *     device memory or in pinned host memory that the device can address (the
  *     kernel then stores the result straight into host memory).
@@ -243,10 +244,30 @@ nwc_status nwc_gemv_scratch_bytes(nwc_handle_t handle, int32_t batch, uint64_t* 
  * nwc_get_device_error clears them after a call that ended with an error).
  * Products and sums are in FP32; the result is the same bit pattern on every
  * run.  Asynchronous on `stream`; allocates nothing.
- * Errors: INVALID_ARG (null, batch, alignment, odd cols, another device
- * current), UNSUPPORTED, CUDA (launch). */
+ * Errors: INVALID_ARG (null, batch, alignment, another device current),
+ * UNSUPPORTED, CUDA (launch). */
 nwc_status nwc_gemv(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
                     int32_t batch, nwc_stream_t stream);
+
+/* Two kernels compute nwc_gemv.  The CUDA-core kernel multiplies the decoded
+ * weights in registers (mma.sync) and handles up to 16 rows of x per launch,
+ * decoding the matrix again for every 16 rows.  The tensor-core kernel decodes
+ * each tile once into shared memory and multiplies it with every row of x
+ * (up to 64) on the tcgen05 tensor cores, accumulating in TMEM ("Unweight",
+ * "Direct GPU Decompression": decompress into shared memory, then the tensor
+ * cores).  A GEMV takes the tensor-core kernel when batch >= the handle's
+ * threshold (16 by default), cols is a multiple of 8, d_x is 16-byte aligned
+ * and the kernel's shared-memory layout fits the device.
+ * nwc_gemv_set_tc_min_batch sets the threshold: 1..64, or 0 for never.
+ * Errors: INVALID_ARG. */
+nwc_status nwc_gemv_set_tc_min_batch(nwc_handle_t handle, int32_t min_batch);
+
+/* Which kernel a GEMV of `batch` rows with this d_x would take, without
+ * launching: *launches (optional) kernel launches, *tensor_cores (optional) 1
+ * for the tensor-core kernel, else 0.  Host only.
+ * Errors: INVALID_ARG. */
+nwc_status nwc_gemv_path(nwc_handle_t handle, const uint16_t* d_x, int32_t batch,
+                         int32_t* launches, int32_t* tensor_cores);
 
 /* GEMV for callers that cannot allocate device memory.  The pages describe
  * no such call; it exists for integrations where the host application owns
@@ -312,6 +333,30 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
                                  uint64_t smem_limit, int32_t rows_of_x,
                                  nwc_schedule_info* info, uint32_t* cta_batch,
                                  uint32_t* batch, uint32_t* tile_ring);
+
+/* The tensor-core kernel's launch shape and schedule for a blob on a device
+ * of sm_count SMs and smem_limit bytes of opt-in shared memory per block.
+ * Host only; touches no GPU.  CTA c owns the tiles [tiles c / ctas,
+ * tiles (c + 1) / ctas) of the row-major tile order v = i tiles_c + j, in
+ * M-groups of `rows` row tiles; `teams` teams of `rows` decode warps take the
+ * column blocks j = t, t + teams, ... of a group.
+ *   cta_batch (optional, ctas + 1 entries), batch (optional, 4 * batches):
+ *     as nwc_schedule_describe.
+ *   tile_ring, tile_batch (optional, tiles entries each), indexed by blob tile
+ *     u = j tiles_r + i: the tile's ring offset, and the CTA's batch that
+ *     brings it with, in bits 28..31, the extra releases its consumer adds
+ *     (batch_tiles minus the tiles of that batch, on its first tile).
+ * Errors: INVALID_ARG, CORRUPT, UNSUPPORTED (no layout fits). */
+typedef struct {
+  uint32_t struct_size;
+  int32_t ctas, rows, teams, batch_tiles, ring_bytes;
+  int64_t tiles, batches;
+  uint64_t smem_bytes, a_offset, b_offset, ring_offset;
+} nwc_tc_schedule_info;
+nwc_status nwc_tc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
+                                    uint64_t smem_limit, nwc_tc_schedule_info* info,
+                                    uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring,
+                                    uint32_t* tile_batch);
 
 /* Any pointer may be NULL.  *blob_bytes is the serialisable part;
  * *compressed_bytes is what holds the matrix (blob, decode table and launch

@@ -36,6 +36,15 @@ class nwc_schedule_info(ctypes.Structure):
                 ("smem_bytes", ctypes.c_uint64), ("xstage_bytes", ctypes.c_uint32)]
 
 
+class nwc_tc_schedule_info(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("ctas", ctypes.c_int32),
+                ("rows", ctypes.c_int32), ("teams", ctypes.c_int32),
+                ("batch_tiles", ctypes.c_int32), ("ring_bytes", ctypes.c_int32),
+                ("tiles", ctypes.c_int64), ("batches", ctypes.c_int64),
+                ("smem_bytes", ctypes.c_uint64), ("a_offset", ctypes.c_uint64),
+                ("b_offset", ctypes.c_uint64), ("ring_offset", ctypes.c_uint64)]
+
+
 NWC_CODE_PREFIX, NWC_CODE_RANK = 0, 1
 
 
@@ -68,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "nwc_gemv_scratch_bytes": ([vp, i32, c.POINTER(u64)], c.c_int),
         "nwc_gemv": ([vp, vp, vp, i32, vp], c.c_int),
         "nwc_gemv_noalloc": ([vp, vp, vp, i32, vp], c.c_int),
+        "nwc_gemv_set_tc_min_batch": ([vp, i32], c.c_int),
+        "nwc_gemv_path": ([vp, vp, i32, c.POINTER(i32), c.POINTER(i32)], c.c_int),
         "nwc_handle_info": ([vp, c.POINTER(i64), c.POINTER(i64), c.POINTER(u64),
                              c.POINTER(u64), c.POINTER(u64)], c.c_int),
         "nwc_get_device_error": ([vp, vp, c.POINTER(c.c_uint32)], c.c_int),
@@ -75,6 +86,8 @@ def _load() -> ctypes.CDLL:
         "nwc_schedule_describe": ([vp, u64, i32, u64, i32, c.POINTER(nwc_schedule_info), vp, vp,
                                    vp],
                                   c.c_int),
+        "nwc_tc_schedule_describe": ([vp, u64, i32, u64, c.POINTER(nwc_tc_schedule_info), vp, vp,
+                                      vp, vp], c.c_int),
         "nwc_plan_destroy": ([vp], None),
         "nwc_handle_destroy": ([vp], None),
     }
@@ -90,9 +103,9 @@ EXPORTED = ("nwc_version", "nwc_status_string", "nwc_plan", "nwc_plan_size", "nw
             "nwc_compress_host", "nwc_blob_device_bytes", "nwc_upload_blob",
             "nwc_handle_from_device", "nwc_decompress", "nwc_gather_rows",
             "nwc_gemv_scratch_bytes", "nwc_gemv",
-            "nwc_gemv_noalloc",
+            "nwc_gemv_noalloc", "nwc_gemv_set_tc_min_batch", "nwc_gemv_path",
             "nwc_handle_info", "nwc_get_device_error", "nwc_test_set_wait_limit",
-            "nwc_schedule_describe",
+            "nwc_schedule_describe", "nwc_tc_schedule_describe",
             "nwc_plan_destroy", "nwc_handle_destroy")
 
 
@@ -198,6 +211,19 @@ def nwc_gemv(handle, d_x, d_y, batch: int, stream=None) -> None:
     _check(LIB.nwc_gemv(handle, _ptr(d_x), _ptr(d_y), batch, _stream(stream)), "nwc_gemv")
 
 
+def nwc_gemv_set_tc_min_batch(handle, min_batch: int) -> None:
+    """Batches >= min_batch take the tensor-core kernel (0: never)."""
+    _check(LIB.nwc_gemv_set_tc_min_batch(handle, min_batch), "nwc_gemv_set_tc_min_batch")
+
+
+def nwc_gemv_path(handle, d_x, batch: int) -> tuple[int, bool]:
+    """(kernel launches, tensor-core kernel?) of a GEMV of `batch` rows with d_x."""
+    n, tc = ctypes.c_int32(), ctypes.c_int32()
+    _check(LIB.nwc_gemv_path(handle, _ptr(d_x), batch, ctypes.byref(n), ctypes.byref(tc)),
+           "nwc_gemv_path")
+    return n.value, bool(tc.value)
+
+
 def nwc_gemv_noalloc(handle, d_x, d_y, batch: int, stream=None) -> None:
     """nwc_gemv with library-owned scratch, for callers that may not allocate
     device memory (see include/nwc.h)."""
@@ -245,6 +271,27 @@ def nwc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int
                                      ring.ctypes.data), "nwc_schedule_describe")
     d = {k: getattr(info, k) for k, _ in nwc_schedule_info._fields_ if k != "struct_size"}
     return d, cta, bat, ring
+
+
+def nwc_tc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int = 232448):
+    """The tensor-core kernel's launch shape and schedule for a blob on a
+    device of the given size; host only.  Returns (info dict, cta_batch
+    [ctas + 1], batch [batches x 4], tile_ring [tiles], tile_batch [tiles])."""
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    info = nwc_tc_schedule_info(struct_size=ctypes.sizeof(nwc_tc_schedule_info))
+    _check(LIB.nwc_tc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit,
+                                        ctypes.byref(info), None, None, None, None),
+           "nwc_tc_schedule_describe")
+    cta = np.zeros(info.ctas + 1, dtype=np.uint32)
+    bat = np.zeros((info.batches, 4), dtype=np.uint32)
+    ring = np.zeros(info.tiles, dtype=np.uint32)
+    tb = np.zeros(info.tiles, dtype=np.uint32)
+    _check(LIB.nwc_tc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit,
+                                        ctypes.byref(info), cta.ctypes.data, bat.ctypes.data,
+                                        ring.ctypes.data, tb.ctypes.data),
+           "nwc_tc_schedule_describe")
+    d = {k: getattr(info, k) for k, _ in nwc_tc_schedule_info._fields_ if k != "struct_size"}
+    return d, cta, bat, ring, tb
 
 
 def nwc_plan_destroy(plan) -> None:

@@ -95,6 +95,12 @@ struct WaitCtl {
 __device__ __forceinline__ WaitCtl wait_ctl(const TileParams& p) {
   return WaitCtl{p.err, p.wait_limit ? p.wait_limit : kDefaultWaitLimit};
 }
+// Waits for a CTA's own copies and MMAs in flight before it leaves: never
+// shorter than the default, whatever limit a test set, so that no CTA exits
+// while a copy into its shared memory is still running.
+__device__ __forceinline__ WaitCtl drain_ctl(const TileParams& p) {
+  return WaitCtl{p.err, p.wait_limit > kDefaultWaitLimit ? p.wait_limit : kDefaultWaitLimit};
+}
 // Polls `bar` for `parity` at most w.limit times; on failure records a
 // timeout in the handle's error word.
 __device__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
@@ -402,7 +408,7 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
 // for releases and issues the copies.  The loop body is a handful of
 // instructions, so the copies go out as fast as the ring allows.
 __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const uint4* desc,
-                        int nb, int lane) {
+                        int nb, int lane, volatile uint32_t* issued = nullptr) {
   if (lane == 0) {
     // The decode table in kTablePieces copies, each CTA starting at a different
     // piece, so that the CTAs do not all ask the same L2 lines at once.
@@ -441,6 +447,7 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
         uint64_t* bar = &s.full[k % kSlots];
         mbar_expect_tx(bar, bytes);  // arrive (release) + byte count
         bulk_load(s.ring + at, p.tiles + 16ull * src, bytes, bar);
+        if (issued) *issued = (uint32_t)(k + 1);
       }
     }
     if (!__shfl_sync(kFull, ok, 0)) break;
@@ -448,9 +455,10 @@ __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const
   // Leave no copy in flight: batches [0, k) were issued, and those more than
   // kSlots back have been released, hence landed.
   if (lane == 0) {
+    const WaitCtl dc = drain_ctl(p);
     for (int j = k - 1; j >= 0 && j >= k - kSlots; --j)
-      wait_bounded(&s.full[j % kSlots], (uint32_t)((j / kSlots) & 1), wc);
-    wait_bounded(s.table_bar, 0, wc);
+      wait_bounded(&s.full[j % kSlots], (uint32_t)((j / kSlots) & 1), dc);
+    wait_bounded(s.table_bar, 0, dc);
   }
 }
 
@@ -464,14 +472,29 @@ __device__ __forceinline__ bool wait_batch(const Smem& s, int k, const WaitCtl& 
 }
 
 // Four BF16 values x[col .. col + 3] of one row of x as two words, zeros where
-// the columns lie past `cols` (cols is even, so a word is wholly inside or
-// outside).  Every lane loads from a valid address and selects afterwards, so
-// lanes never diverge.  vec (uniform): 8-byte aligned and inside.
+// the columns lie past `cols` (for an even cols a word is wholly inside or
+// outside; an odd cols is read element by element).  Every lane loads from a
+// valid address and selects afterwards, so lanes never diverge.  vec
+// (uniform): 8-byte aligned and inside.
+__device__ __forceinline__ uint32_t ldg_u16(const uint16_t* p) {
+  return (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(p));
+}
+// x[col] and x[col + 1] of a row as one word, zeros past `cols`, any
+// alignment (rows of an odd number of columns start on 2-byte boundaries).
+__device__ __forceinline__ uint32_t load_x2_any(const uint16_t* xrow, int64_t cols, int64_t col) {
+  const uint32_t lo = col < cols ? ldg_u16(xrow + col) : 0u;
+  const uint32_t hi = col + 1 < cols ? ldg_u16(xrow + col + 1) : 0u;
+  return lo | (hi << 16);
+}
+
 __device__ __forceinline__ uint2 load_x4(const uint16_t* xrow, int64_t cols, int64_t col,
                                          bool vec) {
   uint2 v;
   if (vec) {
     v = __ldg(reinterpret_cast<const uint2*>(xrow + col));
+  } else if (cols & 1) {
+    v.x = load_x2_any(xrow, cols, col);
+    v.y = load_x2_any(xrow, cols, col + 2);
   } else {
     const bool in0 = col < cols, in1 = col + 2 < cols;
     v.x = __ldg(reinterpret_cast<const uint32_t*>(xrow + (in0 ? col : 0)));
@@ -637,12 +660,15 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
       }
     } else {
       const uint32_t words = (uint32_t)(span / 2), total = (uint32_t)batch * words;
+      const bool odd = (p.cols & 1) != 0;  // rows start on 2-byte boundaries
 #pragma unroll 2
       for (uint32_t t = threadIdx.x; t < total; t += NC * 32) {
         const uint32_t b = t / words, w = t - b * words;
         const int64_t col = j0 * kTileCols + 2 * (int64_t)w;
+        const uint16_t* xr = p.x + b * p.cols;
         const uint32_t v =
-            col < p.cols ? __ldg(reinterpret_cast<const uint32_t*>(p.x + b * p.cols + col)) : 0u;
+            odd ? load_x2_any(xr, p.cols, col)
+                : (col < p.cols ? __ldg(reinterpret_cast<const uint32_t*>(xr + col)) : 0u);
         *reinterpret_cast<uint32_t*>(s.xstage + b * xrow + 4 * w) = v;
       }
     }
@@ -796,58 +822,588 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
 }
 
 // Row gather ("NWC", "How it works > Dequantization and embedding lookup": the
-// same decoder serves row lookups): warp w writes output row w / tiles_c,
-// column block w % tiles_c.  Of the tile that holds the row, only the four
-// lanes that own that tile row decode (lane 4g + c owns row g), one code per
-// table lookup, reading the stream, the raw plane and the table through L1;
-// the other lanes leave.  Stream bytes past the chunk read as zero, so a corrupt
-// chunk can misdecode but never read outside it.
-__global__ void __launch_bounds__(256) gather_kernel(GatherParams p) {
-  const int64_t wg = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (wg >= (int64_t)p.n * p.tiles_c) return;
-  const int64_t i = wg / p.tiles_c, j = wg % p.tiles_c;
-  const int32_t row = __ldg(p.row_ids + i);
-  if (row < 0 || row >= p.rows) {
-    if (lane == 0 && j == 0) atomicOr(p.err, kErrRange);
+// same decoder serves row lookups).  Persistent CTAs take the requested rows in
+// turn; each first copies the decode table into shared memory.  For a row, warp
+// w takes column blocks w, w + warps, ...: it stages the tile's lane lengths
+// and bit streams in shared memory with coalesced 16-byte loads, finds every
+// lane's stream start by a warp prefix sum, and the four lanes that own the
+// row's tile row (lane 4g + c owns row g) decode it with the GEMV's reader,
+// taking the raw plane straight from global memory.  Only the tiles of the
+// requested rows are read.
+constexpr int kGatherWarps = 8;
+
+template <int CP, bool FAST>
+__global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams p) {
+  extern __shared__ __align__(16) uint8_t gsm[];
+  constexpr int kRaw = CP * 512;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (uint32_t o = 16 * threadIdx.x; o < p.table_bytes; o += 16 * blockDim.x)
+    *reinterpret_cast<uint4*>(gsm + o) =
+        __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.table) + o));
+  __syncthreads();
+  const uint32_t table = smem_u32(gsm);
+  uint8_t* stage = gsm + p.table_bytes + (size_t)warp * p.stage_bytes;
+  const uint32_t sbase = smem_u32(stage);
+  const uint32_t limit = sbase + p.stage_bytes;
+  const int g = lane >> 2, c = lane & 3;
+  const bool vec = (p.cols % 8 == 0) && ((reinterpret_cast<uintptr_t>(p.out) & 15) == 0);
+  uint32_t invalid = 0;
+  for (int64_t i = blockIdx.x; i < p.n; i += gridDim.x) {
+    const int32_t row = __ldg(p.row_ids + i);
+    if (row < 0 || row >= p.rows) {
+      if (threadIdx.x == 0) atomicOr(p.err, kErrRange);
+      continue;
+    }
+    uint16_t* orow = p.out + i * p.cols;
+    for (int64_t j = warp; j < p.tiles_c; j += kGatherWarps) {
+      const int64_t u = j * p.tiles_r + row / kTileRows;
+      const uint32_t c0 = __ldg(p.index + u), c1 = __ldg(p.index + u + 1);
+      const uint8_t* chunk = p.tiles + 16ull * c0;
+      // Lane lengths and streams: the chunk after its raw plane, clamped to the
+      // stage (a corrupt index can misdecode but not overrun it).
+      uint32_t bytes = 16u * (c1 - c0) > (uint32_t)kRaw ? 16u * (c1 - c0) - (uint32_t)kRaw : 0u;
+      if (bytes > p.stage_bytes - kRingSlack) bytes = p.stage_bytes - kRingSlack;
+      __syncwarp();
+      for (uint32_t o = 16 * lane; o < bytes; o += 16 * 32)
+        *reinterpret_cast<uint4*>(stage + o) = __ldg(reinterpret_cast<const uint4*>(chunk + kRaw + o));
+      __syncwarp();
+      const uint32_t start = lane_stream_start(sbase, 0, lane);
+      if (g != row % kTileRows) continue;
+      StreamDecoder<FAST> dec;
+      dec.init(sbase + kLanes, start, limit);
+      uint4 rv = __ldg(reinterpret_cast<const uint4*>(chunk + lane * 16));
+#pragma unroll 1
+      for (int m = 0; m < CP; ++m) {
+        const uint4 cur = rv;
+        if (m + 1 < CP) rv = __ldg(reinterpret_cast<const uint4*>(chunk + (m + 1) * 512 + lane * 16));
+        uint32_t wv[8];
+#pragma unroll
+        for (int r = 0; r < 8; r += 2) {
+          uint32_t e0, e1;
+          dec.two(table, e0, e1);
+          invalid |= e0 | e1;
+          wv[r] = assemble(raw_pair_r(cur, r), e0);
+          wv[r + 1] = assemble(raw_pair_r(cur, r + 1), e1);
+        }
+        const int64_t col = j * (CP * 64) + m * 64 + 16 * c;
+        if (vec && col + 16 <= p.cols) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + col);
+          dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+        } else {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            const int64_t c2 = col + 2 * r;
+            if (c2 < p.cols) orow[c2] = (uint16_t)wv[r];
+            if (c2 + 1 < p.cols) orow[c2 + 1] = (uint16_t)(wv[r] >> 16);
+          }
+        }
+      }
+    }
+  }
+  if (invalid & kEntryInvalid) atomicOr(p.err, kErrCorrupt);
+}
+
+// ---- tensor-core path: decode once into shared memory, tcgen05 MMA ---------
+//
+// "Unweight", "Direct GPU Decompression": the compressed weights are
+// decompressed into shared memory and fed straight to the tensor cores.  Here
+// the decoded tile chunks are the A operand (M = 128 rows of W, K-major, 128-
+// byte swizzle) of tcgen05.mma kind::f16 with BF16 inputs and FP32
+// accumulation in TMEM; B is x (N = rows of x padded to 16, 32 or 64), brought
+// in by TMA with the same swizzle.  Each weight is decoded once for every row
+// of x.
+
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Shared-memory matrix descriptor of a K-major operand with 128-byte swizzle:
+// rows of 128 bytes (64 BF16 of K), 8-row atoms of 1024 bytes one after the
+// other (stride 1024), atoms 1024-byte aligned; the leading offset is unused
+// for this layout.  A start 32 bytes further selects the next 16 columns.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// Instruction descriptor of kind::f16: D FP32, A and B BF16, both K-major,
+// shape M x N (K = 16).
+__device__ __forceinline__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+         ((uint32_t)(m >> 4) << 24);
+}
+// D[tmem] (+)= A B, issued by one thread.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// `bar` completes one phase when every tcgen05 operation this thread issued
+// before has completed.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+// 2-D TMA load (tile mode, no multicast) of the box at (c0, c1) into `dst`.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t c0,
+                                            int32_t c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], "
+      "[%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                       uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
+}
+// NCOL consecutive TMEM columns of the warp's 32 lanes: lane l gets the row
+// (lane base + l), v[k] = column (col + k), as FP32.
+template <int NCOL>
+__device__ __forceinline__ void tmem_load(uint32_t taddr, float (&v)[NCOL]);
+template <>
+__device__ __forceinline__ void tmem_load<4>(uint32_t taddr, float (&v)[4]) {
+  uint32_t r[4];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 4; ++k) v[k] = __uint_as_float(r[k]);
+}
+template <>
+__device__ __forceinline__ void tmem_load<8>(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                 "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(r[k]);
+}
+template <>
+__device__ __forceinline__ void tmem_load<16>(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
+}
+
+// Barriers and flags of the tensor-core kernel (at p.tc_bar_off).
+struct TcBars {
+  uint64_t* xfull;    // [team][2]: x chunk of the stage landed (TMA bytes)
+  uint64_t* sfull;    // [team][2]: the team's R decode warps wrote the A stage
+  uint64_t* sempty;   // [team][2]: the MMAs that read the stage completed
+  uint64_t* accfull;  // [team]: the team's accumulator holds its M-group sum
+  uint64_t* accempty; // every decode warp has read the accumulators
+  uint32_t* tmem;     // TMEM base address (tcgen05.alloc writes it)
+  volatile uint32_t* abort;   // a wait gave up: leave
+  volatile uint32_t* issued;  // batches the producer has issued so far
+};
+__device__ __forceinline__ TcBars tc_bars(uint8_t* smem, const TileParams& p) {
+  TcBars b;
+  b.xfull = reinterpret_cast<uint64_t*>(smem + p.tc_bar_off);
+  b.sfull = b.xfull + 2 * kTcMaxTeams;
+  b.sempty = b.sfull + 2 * kTcMaxTeams;
+  b.accfull = b.sempty + 2 * kTcMaxTeams;
+  b.accempty = b.accfull + kTcMaxTeams;
+  b.tmem = reinterpret_cast<uint32_t*>(b.accempty + 1);
+  b.abort = b.tmem + 1;
+  b.issued = b.tmem + 2;
+  return b;
+}
+static_assert(8 * (7 * kTcMaxTeams + 1) + 12 <= (int)kTcBarBytes, "tensor-core barrier area");
+
+// A consumer polls batch k's slot only once the producer has issued batch k:
+// the schedule keeps fewer than kSlots batches outstanding, so the slot's
+// previous batch (k - kSlots) has landed by then and the parity it polls is
+// batch k's, however far this warp's tiles lie apart (the row-panel order can
+// put them far apart).
+__device__ __forceinline__ bool wait_issued(const TcBars& tb, uint32_t k, const WaitCtl& w) {
+  for (uint32_t it = 0; it < w.limit; ++it) {
+    if (*tb.issued > k) return true;
+    if (*tb.abort) break;
+    __nanosleep(32);
+  }
+  atomicOr(w.err, kErrTimeout);
+  return false;
+}
+
+// Tiles of this CTA in the row-major tile order, and the row tiles they touch.
+struct TcWork {
+  int64_t a, b;   // linear range [a, b) of v = i tiles_c + j
+  int64_t i0, i1; // first and last row tile touched
+  int groups;     // M-groups of R row tiles
+};
+__device__ __forceinline__ TcWork tc_work(const TileParams& p) {
+  TcWork w;
+  w.a = p.n_tiles * (int64_t)blockIdx.x / gridDim.x;
+  w.b = p.n_tiles * (int64_t)(blockIdx.x + 1) / gridDim.x;
+  w.i0 = w.a / p.tiles_c;
+  w.i1 = (w.b - 1) / p.tiles_c;
+  w.groups = (int)((w.i1 - w.i0 + p.tc_rows) / p.tc_rows);
+  return w;
+}
+// CTA that owns linear tile v (the largest c with floor(T c / C) <= v).
+__device__ __forceinline__ int64_t tc_cta_of(int64_t v, int64_t tiles, int64_t ctas) {
+  return ((v + 1) * ctas - 1) / tiles;
+}
+
+// Accumulator columns (N / 4) a decode warp reads back: the sum of the teams'
+// accumulators for the warp's lane quarter q = warp % 4 and column quarter
+// warp / 4, and its store to y or, for a row tile shared with other CTAs, to
+// this CTA's boundary slot.
+template <int NQ>
+__device__ __forceinline__ void tc_epilogue(const TileParams& p, const TcWork& wk, uint32_t tmem,
+                                            int warp, int lane, int64_t ig, int rg) {
+  const int q = warp & 3, kq = warp >> 2;
+  float acc[NQ];
+#pragma unroll
+  for (int u = 0; u < NQ; ++u) acc[u] = 0.f;
+  const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kq * NQ);
+  for (int t = 0; t < p.tc_teams; ++t) {
+    float v[NQ];
+    tmem_load<NQ>(base + (uint32_t)(t * p.tc_n), v);
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) acc[u] += v[u];
+  }
+  const int mrow = 32 * q + lane, rr = mrow >> 3;
+  if (rr >= rg) return;
+  const int64_t i = ig + rr, orow = 8 * i + (lane & 7);
+  if (orow >= p.rows) return;
+  const bool full = i * p.tiles_c >= wk.a && (i + 1) * p.tiles_c <= wk.b;
+  float* slot = p.partial + (int64_t)(2 * blockIdx.x + (i == wk.i0 ? 0 : 1)) * 8 * kMaxTcRows;
+#pragma unroll
+  for (int u = 0; u < NQ; ++u) {
+    const int bc = kq * NQ + u;
+    if (bc >= p.batch) break;
+    if (full)
+      p.y[(int64_t)bc * p.rows + orow] = acc[u];
+    else
+      __stcg(slot + bc * 8 + (lane & 7), acc[u]);
+  }
+}
+
+// The last CTA to deliver its part of a row tile shared by several CTAs sums
+// the parts in CTA order and writes y.  One warp.
+__device__ void tc_boundary(const TileParams& p, int64_t i, int lane) {
+  const int64_t ctas = gridDim.x;
+  const int64_t c_lo = tc_cta_of(i * p.tiles_c, p.n_tiles, ctas);
+  const int64_t c_hi = tc_cta_of((i + 1) * p.tiles_c - 1, p.n_tiles, ctas);
+  uint32_t last = 0;
+  if (lane == 0) {
+    __threadfence();
+    last = atomicAdd(&p.counters[i], 1u) == (uint32_t)(c_hi - c_lo);
+  }
+  if (!__shfl_sync(kFull, last, 0)) return;
+  __threadfence();
+  for (int idx = lane; idx < 8 * p.batch; idx += 32) {
+    const int bc = idx >> 3, r = idx & 7;
+    const int64_t orow = 8 * i + r;
+    float sum = 0.f;
+    for (int64_t c = c_lo; c <= c_hi; ++c) {
+      const int64_t first_row = (p.n_tiles * c / ctas) / p.tiles_c;
+      const float* slot = p.partial + (2 * c + (i == first_row ? 0 : 1)) * 8 * kMaxTcRows;
+      sum += __ldcg(slot + bc * 8 + r);
+    }
+    if (orow < p.rows) p.y[(int64_t)bc * p.rows + orow] = sum;
+  }
+  if (lane == 0) p.counters[i] = 0u;
+}
+
+// Decode warps (0 .. 15): warp w < teams R is slot r = w % R of team t = w / R.
+template <int CP, bool FAST>
+__device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, const TcBars& tb,
+                          const TcWork& wk, int warp, int lane) {
+  constexpr int kRaw = CP * 512;
+  const WaitCtl wc = wait_ctl(p);
+  const int R = p.tc_rows, TT = p.tc_teams;
+  const bool decoder = warp < TT * R;
+  const int t = warp / R, r = warp % R;
+  const int g = lane >> 2, c = lane & 3;
+  const uint32_t table = smem_u32(smem);
+  const uint32_t ring = smem_u32(s.ring);
+  const uint32_t limit = ring + (uint32_t)p.ring_bytes + kRingSlack;
+  const uint32_t a_area = smem_u32(smem + p.tc_a_off);
+  const int64_t nj = decoder ? (p.tiles_c - t + TT - 1) / TT : 0;
+  const uint32_t chunk_lo = ((uint32_t)(2 * c) ^ (uint32_t)g) << 4;
+  const uint32_t chunk_hi = ((uint32_t)(2 * c + 1) ^ (uint32_t)g) << 4;
+  uint32_t seq = 0;
+  bool ok = true;
+  for (int gi = 0; gi < wk.groups && ok; ++gi) {
+    const int64_t ig = wk.i0 + (int64_t)gi * R;
+    const int rg = (int)min((int64_t)R, wk.i1 + 1 - ig);
+    const int64_t i = ig + r;
+    for (int64_t jj = 0; jj < nj && ok; ++jj) {
+      const int64_t j = t + jj * TT;
+      const int64_t v = i * p.tiles_c + j;
+      const bool present = r < rg && v >= wk.a && v < wk.b;
+      StreamDecoder<FAST> dec;
+      uint32_t chunk = 0, bw = 0;
+      if (present) {
+        const int64_t u = j * p.tiles_r + i;
+        bw = __ldg(p.tile_batch + u);
+        chunk = ring + __ldg(p.tile_ring + u);
+        if (!wait_issued(tb, bw & 0x0FFFFFFFu, wc) || !wait_batch(s, (int)(bw & 0x0FFFFFFFu), wc)) {
+          ok = false;
+          break;
+        }
+        dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
+      }
+      for (int m = 0; m < CP; ++m, ++seq) {
+        const uint32_t st = seq & 1u, use = seq >> 1;
+        if (use > 0 &&
+            !__all_sync(kFull, wait_bounded(&tb.sempty[2 * t + st], (use - 1) & 1u, wc))) {
+          ok = false;
+          break;
+        }
+        const uint32_t arow =
+            a_area + ((uint32_t)(2 * t + (int)st) * (uint32_t)R + (uint32_t)r) * kTcStageA +
+            (uint32_t)g * 128u;
+        if (present) {
+          const uint4 rv = lds128(chunk + m * 512 + lane * 16);
+          uint32_t wv[8];
+#pragma unroll
+          for (int k = 0; k < 8; k += 2) {
+            uint32_t e0, e1;
+            dec.two(table, e0, e1);
+            wv[k] = assemble(raw_pair_r(rv, k), e0);
+            wv[k + 1] = assemble(raw_pair_r(rv, k + 1), e1);
+          }
+          sts128(arow + chunk_lo, wv[0], wv[1], wv[2], wv[3]);
+          sts128(arow + chunk_hi, wv[4], wv[5], wv[6], wv[7]);
+        } else if (r < rg) {
+          // A row tile of the group outside this CTA's range for this column
+          // block: zeros, so its accumulator rows get nothing from it.
+          sts128(arow + chunk_lo, 0u, 0u, 0u, 0u);
+          sts128(arow + chunk_hi, 0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tb.sfull[2 * t + st]);
+      }
+      if (present && ok) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_n(&s.empty[(bw & 0x0FFFFFFFu) % kSlots], 1u + (bw >> 28));
+      }
+    }
+    if (!ok) break;
+    // Epilogue of the group, by all 16 decode warps.
+    for (int tt = 0; tt < TT && ok; ++tt)
+      ok = __all_sync(kFull, wait_bounded(&tb.accfull[tt], (uint32_t)gi & 1u, wc));
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t tmem = *tb.tmem;
+    switch (p.tc_n) {
+      case 16: tc_epilogue<4>(p, wk, tmem, warp, lane, ig, rg); break;
+      case 32: tc_epilogue<8>(p, wk, tmem, warp, lane, ig, rg); break;
+      default: tc_epilogue<16>(p, wk, tmem, warp, lane, ig, rg); break;
+    }
+    tc_fence_before();
+    __threadfence();  // this warp's y and slot stores, before the arrival below
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tb.accempty);
+    // Row tiles shared with other CTAs (at most the first and the last of the
+    // range): once every decode warp has stored its part (accempty completes
+    // this group's phase after all 16 arrivals), warp 0 delivers them.
+    if (warp == 0 && p.tiles_c > 1) {
+      ok = __all_sync(kFull, wait_bounded(tb.accempty, (uint32_t)gi & 1u, wc));
+      if (!ok) break;
+      auto shared_row = [&](int64_t ii) {
+        return ii >= ig && ii < ig + rg &&
+               !(ii * p.tiles_c >= wk.a && (ii + 1) * p.tiles_c <= wk.b);
+      };
+      if (shared_row(wk.i0)) tc_boundary(p, wk.i0, lane);
+      if (wk.i1 != wk.i0 && shared_row(wk.i1)) tc_boundary(p, wk.i1, lane);
+    }
+  }
+  if (!ok && lane == 0) *tb.abort = 1u;
+}
+
+// The MMA warp: lane 0 loads x (TMA) into each team's B stage, issues the four
+// K = 16 MMAs of every chunk once the team's decode warps have written it, and
+// commits their completion to the stage's barrier (and at the end of an
+// M-group to the team's accumulator barrier).  It serves the teams in turn
+// without blocking on any of them.
+template <int CP>
+__device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* smem,
+                       const TcBars& tb, const TcWork& wk) {
+  const WaitCtl wc = wait_ctl(p);
+  const int R = p.tc_rows, TT = p.tc_teams, N = p.tc_n;
+  const uint32_t a_area = smem_u32(smem + p.tc_a_off), b_area = smem_u32(smem + p.tc_b_off);
+  const uint32_t idesc = umma_idesc_bf16(128, N);
+  const uint32_t tmem = *tb.tmem;
+  uint32_t nx[kTcMaxTeams], nm[kTcMaxTeams], per_group[kTcMaxTeams], total[kTcMaxTeams];
+  for (int t = 0; t < TT; ++t) {
+    per_group[t] = (uint32_t)((p.tiles_c - t + TT - 1) / TT) * CP;
+    total[t] = (uint32_t)wk.groups * per_group[t];
+    nx[t] = nm[t] = 0;
+  }
+  wait_prerequisites();  // x may be written by the previous kernel on the stream
+  uint32_t idle = 0;
+  for (;;) {
+    bool done = true, moved = false;
+    for (int t = 0; t < TT; ++t) {
+      if (nm[t] >= total[t]) continue;
+      done = false;
+      // x of chunk nx[t]: its stage is free once the MMAs two chunks back are done.
+      if (nx[t] < total[t] && nx[t] < nm[t] + 2) {
+        const uint32_t sx = nx[t] & 1u, use = nx[t] >> 1;
+        if (use == 0 || mbar_test_wait(&tb.sempty[2 * t + sx], (use - 1) & 1u)) {
+          const uint32_t within = nx[t] % per_group[t];
+          const int64_t j = t + (int64_t)(within / CP) * TT;
+          const int m = (int)(within % CP);
+          mbar_expect_tx(&tb.xfull[2 * t + sx], (uint32_t)N * 128u);
+          tma_load_2d(b_area + (uint32_t)(2 * t + (int)sx) * kTcStageB, tmap,
+                      (int32_t)(j * CP * 64 + m * 64), 0, &tb.xfull[2 * t + sx]);
+          ++nx[t];
+          moved = true;
+        }
+      }
+      // MMAs of chunk nm[t].
+      if (nm[t] < nx[t]) {
+        const uint32_t sm = nm[t] & 1u, ph = (nm[t] >> 1) & 1u;
+        const uint32_t within = nm[t] % per_group[t], gi = nm[t] / per_group[t];
+        if (mbar_test_wait(&tb.xfull[2 * t + sm], ph) && mbar_test_wait(&tb.sfull[2 * t + sm], ph) &&
+            (within != 0 || gi == 0 || mbar_test_wait(tb.accempty, (gi - 1) & 1u))) {
+          tc_fence_after();
+          const uint32_t a0 = a_area + (uint32_t)(2 * t + (int)sm) * (uint32_t)R * kTcStageA;
+          const uint32_t b0 = b_area + (uint32_t)(2 * t + (int)sm) * kTcStageB;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            umma_bf16(tmem + (uint32_t)(t * N), umma_desc_sw128(a0 + 32u * k),
+                      umma_desc_sw128(b0 + 32u * k), idesc, (within == 0 && k == 0) ? 0u : 1u);
+          umma_commit(&tb.sempty[2 * t + sm]);
+          if (within + 1 == per_group[t]) umma_commit(&tb.accfull[t]);
+          ++nm[t];
+          moved = true;
+        }
+      }
+    }
+    if (done) break;
+    if (moved) {
+      idle = 0;
+    } else if (++idle >= wc.limit || *tb.abort) {
+      atomicOr(wc.err, kErrTimeout);
+      *tb.abort = 1u;
+      break;
+    }
+  }
+  // Leave nothing in flight: x loads issued but not consumed, and the MMAs.
+  const WaitCtl dc = drain_ctl(p);
+  for (int t = 0; t < TT; ++t) {
+    for (uint32_t k = nm[t]; k < nx[t]; ++k)
+      wait_bounded(&tb.xfull[2 * t + (int)(k & 1u)], (k >> 1) & 1u, dc);
+    if (nm[t] > 0)
+      wait_bounded(&tb.sempty[2 * t + (int)((nm[t] - 1) & 1u)], ((nm[t] - 1) >> 1) & 1u, dc);
+  }
+}
+
+// y[b][n] for up to kMaxTcRows rows b of x, every weight decoded once.
+// Warps 0..15 decode into the A stages and read the accumulators back, warp 16
+// allocates TMEM and issues x loads and MMAs, warp 17 moves the compressed
+// tiles into the ring (the same producer as the other kernels).
+template <int CP, bool FAST>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemv_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap) {
+  extern __shared__ __align__(1024) uint8_t smem_tc[];
+  uint8_t* smem = smem_tc;
+  allow_dependents();
+  if (smem_u32(smem) & 1023u) {  // the swizzled stages need 1024-byte alignment
+    if (threadIdx.x == 0) atomicOr(p.err, kErrLayout);
     return;
   }
-  if ((lane >> 2) != row % kTileRows) return;
-  const int c = lane & 3;
-  const int64_t u = j * p.tiles_r + row / kTileRows;
-  const uint32_t c0 = __ldg(p.index + u), c1 = __ldg(p.index + u + 1);
-  const uint8_t* chunk = p.tiles + 16ull * c0;
-  const uint32_t raw = (uint32_t)(kTileRows * p.tile_cols);
-  const uint32_t chunk_bytes = 16u * (c1 - c0);
-  const uint32_t area_bytes = chunk_bytes > raw + kLanes ? chunk_bytes - raw - kLanes : 0u;
-  const uint8_t* lens = chunk + raw;
-  const uint8_t* area = lens + kLanes;
-  uint32_t q = 0;  // next sequence byte of this lane's stream
-  for (int t = 0; t < lane; ++t) q += __ldg(lens + t);
-  // Sequence byte q sits in little-endian word q / 4 as its byte 3 - q % 4.
-  auto seq_byte = [&](uint32_t b) -> uint64_t {
-    return b < area_bytes ? (uint64_t)__ldg(area + ((b & ~3u) | (3u - (b & 3u)))) : 0ull;
-  };
-  uint64_t buf = 0;  // next bits, most significant first
-  int nbits = 0;
-  const int symbols = 16 * (p.tile_cols / 64);
-  uint16_t* orow = p.out + i * p.cols;
-  uint32_t bad = 0;
-  for (int k = 0; k < symbols; ++k) {
-    while (nbits < p.peek) {
-      buf |= seq_byte(q++) << (56 - nbits);
-      nbits += 8;
+  const Smem s = carve(smem, p);
+  const TcBars tb = tc_bars(smem, p);
+  const TcWork wk = tc_work(p);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(s.table_bar, 1);
+    for (int k = 0; k < kSlots; ++k) {
+      mbar_init(&s.full[k], 1);
+      mbar_init(&s.empty[k], (uint32_t)p.batch_tiles);
     }
-    const uint32_t e = __ldg(p.table + (uint32_t)(buf >> (64 - p.peek)));
-    const uint32_t len = (e >> kEntryLen0Shift) & 15u, s = (e >> 7) & 0xFFu;
-    bad |= e & kEntryInvalid;
-    buf <<= (e & kEntryInvalid) ? 1u : len;  // an invalid prefix still moves on
-    nbits -= (e & kEntryInvalid) ? 1 : (int)len;
-    const uint32_t r = __ldg(chunk + (k / 16) * 512 + 16 * lane + (k % 16));
-    const int64_t col = j * p.tile_cols + 64 * (k / 16) + 16 * c + (k % 16);
-    if (col < p.cols) orow[col] = (uint16_t)(((r & 0x80u) << 8) | (s << 7) | (r & 0x7Fu));
+    for (int k = 0; k < 2 * kTcMaxTeams; ++k) {
+      mbar_init(&tb.xfull[k], 1);
+      mbar_init(&tb.sfull[k], (uint32_t)p.tc_rows);
+      mbar_init(&tb.sempty[k], 1);
+    }
+    for (int k = 0; k < kTcMaxTeams; ++k) mbar_init(&tb.accfull[k], 1);
+    mbar_init(tb.accempty, kTcDecodeWarps);
+    *tb.abort = 0u;
+    *tb.issued = 0u;
   }
-  if (bad) atomicOr(p.err, kErrCorrupt);
+  if (warp == kTcMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tb.tmem)),
+                 "r"(p.tc_tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_barrier_init();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kTcProducerWarp) {
+    const uint32_t b0 = __ldg(p.sched_cta + blockIdx.x), b1 = __ldg(p.sched_cta + blockIdx.x + 1);
+    produce(p, smem, s, p.sched_batch + b0, (int)(b1 - b0), lane, tb.issued);
+    return;
+  }
+  if (warp < kTcDecodeWarps) {
+    wait_prerequisites();  // y and the scratch may belong to the previous kernel
+    const WaitCtl wc = wait_ctl(p);
+    if (wait_table(s, wc)) {
+      tc_decode<CP, FAST>(p, smem, s, tb, wk, warp, lane);
+    } else if (lane == 0) {
+      *tb.abort = 1u;
+    }
+    __syncwarp();
+  } else if (lane == 0) {
+    tc_mma<CP>(p, &tmap, smem, tb, wk);
+  }
+  __syncwarp();
+  // Teardown: every decode warp and the MMA warp, then TMEM goes back.
+  tc_fence_before();
+  named_barrier_sync(3, (kTcDecodeWarps + 1) * 32);
+  if (warp == kTcMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*tb.tmem),
+                 "r"(p.tc_tmem_cols)
+                 : "memory");
+  }
 }
 
 // Raises a kernel's dynamic shared-memory limit on the current device once per
@@ -901,6 +1457,25 @@ cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream
   if (p.batch < 1 || p.batch > kMaxPassRows) return cudaErrorInvalidValue;
   return p.batch <= 8 ? launch_gemv_t<CP, false, FAST>(p, s, stream)
                       : launch_gemv_t<CP, true, FAST>(p, s, stream);
+}
+
+template <int CP, bool FAST>
+cudaError_t launch_gemv_tc_t(const TileParams& p, const CUtensorMap& tmap, const LaunchShape& s,
+                             cudaStream_t stream) {
+  static int configured[64] = {};
+  cudaError_t e = ensure_smem(gemv_tc_kernel<CP, FAST>, s.smem_bytes, configured);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)s.ctas);
+  cfg.blockDim = dim3((unsigned)kTcThreads);
+  cfg.dynamicSmemBytes = s.smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<CP, FAST>, p, tmap);
 }
 
 template <int CP, bool FAST>
@@ -969,12 +1544,108 @@ cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
   }
 }
 
-cudaError_t launch_gather(const GatherParams& g, cudaStream_t stream) {
-  const int64_t warps = (int64_t)g.n * g.tiles_c;
-  const int64_t blocks = (warps + 7) / 8;
-  if (blocks < 1 || blocks > 0x7FFFFFFF) return cudaErrorInvalidValue;
-  gather_kernel<<<(unsigned)blocks, 256, 0, stream>>>(g);
+bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_chunk, uint64_t typical_chunk,
+              uint32_t table_bytes, int sm_count, size_t smem_limit, TcShape* out) {
+  const int64_t tiles = tiles_r * tiles_c;
+  int64_t ctas = tiles < sm_count ? tiles : sm_count;
+  if (ctas > (int64_t)kMaxCtas) ctas = kMaxCtas;
+  if (ctas < 1) ctas = 1;
+  const int64_t per_cta = (tiles + ctas - 1) / ctas;
+  // Row tiles a CTA touches: its tiles span at most this many rows.
+  int64_t rows_max = (per_cta + tiles_c - 1) / tiles_c + 1;
+  if (rows_max > tiles_r) rows_max = tiles_r;
+  if (rows_max > 16) rows_max = 16;
+  int bt = (int)((kBatchTarget + typical_chunk - 1) / (typical_chunk ? typical_chunk : 1));
+  if (bt < 2) bt = 2;
+  if (bt > 8) bt = 8;
+  const uint32_t bar_off = (uint32_t)xstage_offset(table_bytes);
+  bool found = false;
+  TcShape best{};
+  int64_t best_rounds = 0, best_ring = 0;
+  for (int R = (int)rows_max; R >= 1; --R) {
+    int tmax = 16 / R;
+    if (tmax > tiles_c) tmax = (int)tiles_c;
+    if (tmax > kTcMaxTeams) tmax = kTcMaxTeams;
+    for (int TT = tmax; TT >= 1; --TT) {
+      const uint32_t a_off = (bar_off + kTcBarBytes + 1023u) / 1024u * 1024u;
+      const uint32_t b_off = a_off + (uint32_t)(2 * TT * R) * kTcStageA;
+      const size_t head = b_off + (size_t)(2 * TT) * kTcStageB;
+      const size_t ring_offset = (head + 127) / 128 * 128;
+      if (smem_limit < ring_offset + kRingSlack) continue;
+      size_t ring = smem_limit - ring_offset - kRingSlack;
+      const size_t cap = (size_t)per_cta * (size_t)max_chunk;
+      if (ring > cap) ring = cap;
+      ring = ring / 16 * 16;
+      // A team's run of R tiles plus two copies of worst-case chunks (no more
+      // than the CTA's tiles), and the last A stage's 16 KiB operand window,
+      // must fit.
+      int64_t need_tiles = (int64_t)R + 2 * bt;
+      if (need_tiles > per_cta) need_tiles = per_cta;
+      if (ring < (size_t)need_tiles * (size_t)max_chunk) continue;
+      if (ring_offset + ring + kRingSlack < (size_t)a_off + (size_t)(2 * TT * R - 1) * kTcStageA + 16384)
+        continue;
+      // Tile decodes on a decode warp's critical path: M-groups of the CTA's
+      // rows times rounds of column blocks per group.
+      const int64_t rounds = (rows_max + R - 1) / R * ((tiles_c + TT - 1) / TT);
+      if (!found || rounds < best_rounds || (rounds == best_rounds && (int64_t)ring > best_ring)) {
+        found = true;
+        best_rounds = rounds;
+        best_ring = (int64_t)ring;
+        best.rows = R;
+        best.teams = TT;
+        best.bar_off = bar_off;
+        best.a_off = a_off;
+        best.b_off = b_off;
+        best.s.ctas = (int)ctas;
+        best.s.table_bytes = table_bytes;
+        best.s.xstage_bytes = (uint32_t)(head - bar_off);
+        best.s.ring_offset = ring_offset;
+        best.s.ring_bytes = (int)ring;
+        best.s.batch_tiles = bt;
+        best.s.smem_bytes = ring_offset + ring + kRingSlack;
+      }
+    }
+  }
+  if (found) *out = best;
+  return found;
+}
+
+cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols, bool fast,
+                           const TcShape& s, cudaStream_t stream) {
+  if (p.batch < 1 || p.batch > kMaxTcRows || p.tc_teams < 1 || p.tc_teams > kTcMaxTeams ||
+      p.tc_rows < 1 || p.tc_rows * p.tc_teams > kTcDecodeWarps)
+    return cudaErrorInvalidValue;
+  switch (tile_cols) {
+    case 512: return fast ? launch_gemv_tc_t<8, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<8, false>(p, tmap, s.s, stream);
+    case 256: return fast ? launch_gemv_tc_t<4, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<4, false>(p, tmap, s.s, stream);
+    case 128: return fast ? launch_gemv_tc_t<2, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<2, false>(p, tmap, s.s, stream);
+    case 64: return fast ? launch_gemv_tc_t<1, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<1, false>(p, tmap, s.s, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <int CP, bool FAST>
+cudaError_t launch_gather_t(const GatherParams& g, int ctas, size_t smem, cudaStream_t stream) {
+  static int configured[64] = {};
+  cudaError_t e = ensure_smem(gather_kernel<CP, FAST>, smem, configured);
+  if (e != cudaSuccess) return e;
+  gather_kernel<CP, FAST><<<(unsigned)ctas, kGatherWarps * 32, smem, stream>>>(g);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const GatherParams& g, int sm_count, cudaStream_t stream) {
+  if (g.n < 1) return cudaErrorInvalidValue;
+  const int64_t want = 2 * (int64_t)(sm_count > 0 ? sm_count : 1);
+  const int ctas = (int)(g.n < want ? g.n : want);
+  const size_t smem = (size_t)g.table_bytes + (size_t)kGatherWarps * g.stage_bytes;
+  const bool fast = g.peek == 14;
+  switch (g.tile_cols) {
+    case 512: return fast ? launch_gather_t<8, true>(g, ctas, smem, stream) : launch_gather_t<8, false>(g, ctas, smem, stream);
+    case 256: return fast ? launch_gather_t<4, true>(g, ctas, smem, stream) : launch_gather_t<4, false>(g, ctas, smem, stream);
+    case 128: return fast ? launch_gather_t<2, true>(g, ctas, smem, stream) : launch_gather_t<2, false>(g, ctas, smem, stream);
+    case 64: return fast ? launch_gather_t<1, true>(g, ctas, smem, stream) : launch_gather_t<1, false>(g, ctas, smem, stream);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace nwc

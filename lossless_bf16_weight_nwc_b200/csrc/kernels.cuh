@@ -1,5 +1,6 @@
 // kernels.cuh — launch interface of the sm_100a kernels (host side).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -19,6 +20,7 @@ constexpr int kMaxLag = 48;
 constexpr uint32_t kErrTimeout = 1u;   // a bounded mbarrier wait gave up
 constexpr uint32_t kErrCorrupt = 2u;   // a stream held no valid code
 constexpr uint32_t kErrRange = 4u;     // a gathered row id was out of range
+constexpr uint32_t kErrLayout = 8u;    // shared memory not aligned as a kernel needs
 
 // Polls of a bounded mbarrier wait before it gives up (TileParams.wait_limit
 // 0 means this).
@@ -48,6 +50,13 @@ struct TileParams {
   uint16_t* out;            // BF16 [rows x cols]
   uint32_t* err;            // device: the handle's error word
   uint32_t wait_limit;      // polls before a bounded wait gives up (0: default)
+  // tensor-core kernel
+  const uint32_t* tile_batch;  // device: per tile, its batch | extra releases << 28
+  int32_t tc_rows;          // R: row tiles per M-group (rows of the MMA / 8)
+  int32_t tc_teams;         // teams of R decode warps, each on its own column blocks
+  int32_t tc_n;             // accumulator columns: rows of x padded to 16, 32 or 64
+  uint32_t tc_tmem_cols;    // TMEM columns allocated (power of two >= 32)
+  uint32_t tc_bar_off, tc_a_off, tc_b_off;  // shared-memory offsets
 };
 
 // Shared memory that a CTA reserves for its columns of x, by x-stage class:
@@ -87,6 +96,47 @@ void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s
 // fast: lmax <= 7 (14-bit peek, two codes per entry always).
 cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const LaunchShape& s,
                         cudaStream_t stream);
+
+// ---- tensor-core (tcgen05) GEMV: decode once, multiply every row of x -----
+//
+// CTA c owns the tiles [T c / C, T (c + 1) / C) of the ROW-major tile order
+// v = i tiles_c + j (T tiles, C CTAs), so it owns whole row tiles except at
+// most one partial row tile at each end, and sums over K on chip.  Its row
+// tiles form M-groups of R (the MMA's M = 128 rows holds up to 16 row tiles);
+// `teams` teams of R decode warps take the column blocks j = t, t + teams, ...
+// of a group, each team accumulating into its own TMEM accumulator.
+constexpr int kTcDecodeWarps = 16;
+constexpr int kTcMmaWarp = 16;       // TMEM allocation, x loads (TMA), MMA issue
+constexpr int kTcProducerWarp = 17;  // bulk copies of the compressed tiles
+constexpr int kTcThreads = 18 * 32;
+constexpr uint32_t kTcBarBytes = 1024;                 // barriers, TMEM address, flags
+constexpr uint32_t kTcStageA = 1024;                   // one row tile: 8 x 64 BF16
+constexpr uint32_t kTcStageB = (uint32_t)kMaxTcRows * 128;  // 64 rows of x x 64 BF16
+constexpr int kTcMaxTeams = 8;                         // 8 accumulators of 64 columns
+
+struct TcShape {
+  LaunchShape s;       // grid, ring and copies; s.xstage_bytes spans barriers, A and B
+  int rows;            // R
+  int teams;
+  uint32_t bar_off, a_off, b_off;  // shared-memory offsets
+};
+// Chooses R and the team count for a matrix of tiles_r x tiles_c tiles on a
+// device of sm_count SMs and smem_limit bytes of shared memory per block: the
+// fewest tile decodes on a decode warp's path (M-groups of the rows a CTA
+// touches x rounds of column blocks per group), then the largest ring, with
+// room in the ring
+// for a team's tiles plus two copies of worst-case chunks (so that a team never
+// waits for a tile that cannot be issued).  Returns false when nothing fits.
+bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_chunk, uint64_t typical_chunk,
+              uint32_t table_bytes, int sm_count, size_t smem_limit, TcShape* out);
+// The tensor-core kernel's schedule (layout in nwc_format.h) for shape s;
+// `out` receives sched_tc_bytes(tiles) bytes.
+void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c, const TcShape& s,
+                       uint8_t* out);
+// tmap: the TMA descriptor of x (BF16 [rows of x][cols], box 64 columns x
+// tc_n rows, 128-byte swizzle).
+cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols,
+                           bool fast, const TcShape& s, cudaStream_t stream);
 cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
                               const LaunchShape& s, cudaStream_t stream);
 // Row gather (embedding lookup) from the compressed matrix.
@@ -94,6 +144,8 @@ struct GatherParams {
   const uint8_t* tiles;     // device: tile area of the blob
   const uint32_t* index;    // device: chunk offsets (16-byte units), tiles + 1
   const uint32_t* table;    // device: decode table
+  uint32_t table_bytes;
+  uint32_t stage_bytes;     // per warp: a tile's lane lengths and streams + slack
   int32_t peek;             // table peek width (12 or 14)
   int32_t tile_cols;
   int64_t rows, cols, tiles_r, tiles_c;
@@ -102,6 +154,6 @@ struct GatherParams {
   uint16_t* out;            // device: BF16 [n x cols]
   uint32_t* err;            // device: the handle's error word
 };
-cudaError_t launch_gather(const GatherParams& g, cudaStream_t stream);
+cudaError_t launch_gather(const GatherParams& g, int sm_count, cudaStream_t stream);
 
 }  // namespace nwc

@@ -2,6 +2,8 @@
 //
 // Host-side validation, plans and handles, device images, and kernel launches.
 // Every device call runs on the caller's stream and allocates no device memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -94,6 +96,54 @@ nwc_status write_schedule(nwc_handle_s* h, int cls, const nwc::LaunchShape& s,
   return NWC_OK;
 }
 
+uint64_t tc_class_off(const nwc_handle_s& h) {
+  return h.sched_off + (uint64_t)nwc::kStageClasses * nwc::sched_class_bytes((uint64_t)h.tiles);
+}
+
+// Tensor-core launch shape for a handle on a device of `sms` SMs and `smem`
+// bytes of opt-in shared memory per block; false when it does not fit.
+bool tc_shape_on(const nwc_handle_s& h, int sms, size_t smem, nwc::TcShape* ts) {
+  const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
+  return nwc::tc_shape(h.tiles_r, h.tiles_c, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms,
+                       smem, ts);
+}
+
+bool same_tc_shape(const nwc_handle_s& h, const nwc::TcShape& t) {
+  return h.tc_rows == t.rows && h.tc_teams == t.teams && h.tc_ctas == t.s.ctas &&
+         h.tc_ring == t.s.ring_bytes && h.tc_bt == t.s.batch_tiles;
+}
+
+void note_tc_schedule(nwc_handle_s* h, const nwc::TcShape& t) {
+  h->tc_rows = t.rows;
+  h->tc_teams = t.teams;
+  h->tc_ctas = t.s.ctas;
+  h->tc_ring = t.s.ring_bytes;
+  h->tc_bt = t.s.batch_tiles;
+}
+
+// Writes the tensor-core schedule for shape t into the device image on
+// `stream`, or into `image` (a host copy of the device image) when given.
+nwc_status write_tc_schedule(nwc_handle_s* h, const nwc::TcShape& t, uint8_t* image,
+                             cudaStream_t stream) {
+  if (image) {
+    nwc::build_tc_schedule(h->index.data(), h->tiles_r, h->tiles_c, t, image + tc_class_off(*h));
+    note_tc_schedule(h, t);
+    return NWC_OK;
+  }
+  std::vector<uint8_t> sched;
+  try {
+    sched.resize(nwc::sched_tc_bytes((uint64_t)h->tiles));
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
+  nwc::build_tc_schedule(h->index.data(), h->tiles_r, h->tiles_c, t, sched.data());
+  if (cudaMemcpyAsync(h->d_base + tc_class_off(*h), sched.data(), sched.size(),
+                      cudaMemcpyHostToDevice, stream) != cudaSuccess)
+    return NWC_ERR_CUDA;
+  note_tc_schedule(h, t);
+  return NWC_OK;
+}
+
 // Launch geometry of class cls on the current device, which must be the
 // handle's (the one current when it was made: its image lives there); rewrites
 // that class's schedule (in stream order) when it was made for another shape.
@@ -165,11 +215,13 @@ constexpr int kChunkBatch = nwc::kMaxPassRows;  // rows of x per kernel launch
 
 // Split-K scratch one GEMV call of `batch` rows uses: the arrival counters
 // (padded to 256 bytes) and the partial sums of one launch.
-uint64_t scratch_bytes_for(const nwc_handle_s& h, int32_t batch) {
+uint64_t scratch_bytes_for(const nwc_handle_s& h, int32_t batch, bool tensor_cores) {
   if (h.tiles_c <= 1) return 0;
   const int b = batch < kChunkBatch ? batch : kChunkBatch;
   return round_up(4ull * (uint64_t)h.tiles_r, 256) +
-         nwc::split_partial_bytes((uint64_t)h.tiles_r, (uint64_t)h.tiles_c, (uint64_t)b);
+         (tensor_cores ? nwc::tc_partial_bytes((uint64_t)h.tiles_c)
+                       : nwc::split_partial_bytes((uint64_t)h.tiles_r, (uint64_t)h.tiles_c,
+                                                  (uint64_t)b));
 }
 
 // Zeroes the error word and the arrival counters of a handle's scratch area.
@@ -213,6 +265,8 @@ nwc_status init_schedule(nwc_handle_s* h, uint8_t* image, cudaStream_t stream) {
     nwc::build_schedule(h->index.data(), h->tiles, s, image + class_off(*h, cls));
     note_schedule(h, cls, s);
   }
+  nwc::TcShape ts;
+  if (tc_shape_on(*h, sms, smem, &ts)) return write_tc_schedule(h, ts, image, stream);
   return NWC_OK;
 }
 
@@ -449,14 +503,22 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
   if (!h || !d_rows || !d_out || n < 1 || n > (1 << 20) || !aligned(d_rows, 4) ||
       !aligned(d_out, 2))
     return NWC_ERR_INVALID_ARG;
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;
+  int dev = -1, sms = 0;
+  size_t smem = 0;
+  nwc_status st = current_device(&dev, &sms, &smem);
+  if (st != NWC_OK) return st;
   if (dev != h->device) return NWC_ERR_INVALID_ARG;
   nwc::GatherParams g;
   std::memset(&g, 0, sizeof(g));
   g.tiles = h->d_base + h->tiles_off;
   g.index = reinterpret_cast<const uint32_t*>(h->d_base + h->index_off);
   g.table = reinterpret_cast<const uint32_t*>(h->d_base + h->table_off);
+  g.table_bytes = nwc::table_bytes(h->lmax);
+  // Lane lengths and the longest streams a tile can hold, plus the readers'
+  // slack.
+  g.stage_bytes = (uint32_t)(nwc::max_chunk_bytes(h->tile_cols, h->lmax) -
+                             nwc::raw_bytes(h->tile_cols) + 256);
+  if ((size_t)g.table_bytes + 8ull * g.stage_bytes > smem) return NWC_ERR_UNSUPPORTED;
   g.peek = nwc::peek_bits(h->lmax);
   g.tile_cols = (int32_t)h->tile_cols;
   g.rows = h->rows;
@@ -467,12 +529,13 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
   g.n = n;
   g.out = d_out;
   g.err = error_word(*h);
-  return cuda_status(nwc::launch_gather(g, reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(nwc::launch_gather(g, sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 nwc_status nwc_gemv_scratch_bytes(nwc_handle_t h, int32_t batch, uint64_t* bytes) {
   if (!h || !bytes || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
-  *bytes = scratch_bytes_for(*h, batch);
+  *bytes = scratch_bytes_for(*h, batch, batch >= h->tc_min_batch && h->tc_min_batch > 0 &&
+                                              h->tc_rows > 0 && (h->cols % 8) == 0);
   return NWC_OK;
 }
 
@@ -484,7 +547,8 @@ namespace {
 nwc_status gemv_check(const nwc_handle_s* h, const uint16_t* d_x, const float* d_y,
                       int32_t batch) {
   if (!h || !d_x || !d_y || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
-  if (!aligned(d_x, 4) || !aligned(d_y, 4) || (h->cols & 1)) return NWC_ERR_INVALID_ARG;
+  // x is read in BF16 pairs (4-byte words) unless cols is odd.
+  if (!aligned(d_x, (h->cols & 1) ? 2 : 4) || !aligned(d_y, 4)) return NWC_ERR_INVALID_ARG;
   // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
   if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
   int dev = -1;
@@ -493,11 +557,107 @@ nwc_status gemv_check(const nwc_handle_s* h, const uint16_t* d_x, const float* d
   return NWC_OK;
 }
 
+// cuTensorMapEncodeTiled from the driver, looked up once.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// Accumulator columns of the tensor-core kernel for `batch` rows of x.
+int tc_columns(int32_t batch) { return batch <= 16 ? 16 : batch <= 32 ? 32 : 64; }
+
+// Whether a GEMV of `batch` rows takes the tensor-core kernel: at or above the
+// handle's threshold, when its shape fits this device and x can be read by TMA
+// (16-byte aligned rows).
+bool use_tensor_cores(const nwc_handle_s& h, const uint16_t* d_x, int32_t batch) {
+  return h.tc_min_batch > 0 && batch >= h.tc_min_batch && batch <= nwc::kMaxTcRows &&
+         h.tc_rows > 0 && (h.cols % 8) == 0 && aligned(d_x, 16);
+}
+
+// The tensor-core launch: one kernel for up to 64 rows of x, every weight
+// decoded once.
+nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t batch,
+                       uint32_t* counters, float* partial, cudaStream_t cs) {
+  int dev, sms;
+  size_t smem;
+  nwc_status st = current_device(&dev, &sms, &smem);
+  if (st != NWC_OK) return st;
+  nwc::TcShape ts;
+  if (!tc_shape_on(*h, sms, smem, &ts)) return NWC_ERR_UNSUPPORTED;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!same_tc_shape(*h, ts)) {
+      st = write_tc_schedule(h, ts, nullptr, cs);
+      if (st != NWC_OK) return st;
+    }
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (!encode) return NWC_ERR_UNSUPPORTED;
+  const int n = tc_columns(batch);
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)h->cols, (cuuint64_t)batch};
+  const cuuint64_t strides[1] = {(cuuint64_t)h->cols * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)n};
+  const cuuint32_t elem[2] = {1, 1};
+  if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(d_x), dims, strides,
+             box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return NWC_ERR_UNSUPPORTED;
+  nwc::TileParams p;
+  std::memset(&p, 0, sizeof(p));
+  const uint8_t* sched = h->d_base + tc_class_off(*h);
+  p.tiles = h->d_base + h->tiles_off;
+  p.sched_cta = reinterpret_cast<const uint32_t*>(sched);
+  p.sched_batch = reinterpret_cast<const uint4*>(sched + nwc::sched_batch_off());
+  p.tile_ring = reinterpret_cast<const uint32_t*>(sched + nwc::sched_tc_ring_off((uint64_t)h->tiles));
+  p.tile_batch =
+      reinterpret_cast<const uint32_t*>(sched + nwc::sched_tc_tbatch_off((uint64_t)h->tiles));
+  p.table = reinterpret_cast<const uint32_t*>(h->d_base + h->table_off);
+  p.table_bytes = nwc::table_bytes(h->lmax);
+  p.rows = h->rows;
+  p.cols = h->cols;
+  p.tiles_r = h->tiles_r;
+  p.tiles_c = h->tiles_c;
+  p.n_tiles = h->tiles;
+  p.rows_pad = 8 * h->tiles_r;
+  p.ring_offset = (uint32_t)ts.s.ring_offset;
+  p.ring_bytes = ts.s.ring_bytes;
+  p.batch_tiles = ts.s.batch_tiles;
+  p.xstage_bytes = ts.s.xstage_bytes;
+  p.err = error_word(*h);
+  p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  p.x = d_x;
+  p.y = d_y;
+  p.batch = batch;
+  p.counters = counters;
+  p.partial = partial;
+  p.tc_rows = ts.rows;
+  p.tc_teams = ts.teams;
+  p.tc_n = n;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(ts.teams * n)) cols <<= 1;
+  p.tc_tmem_cols = cols;
+  p.tc_bar_off = ts.bar_off;
+  p.tc_a_off = ts.a_off;
+  p.tc_b_off = ts.b_off;
+  return cuda_status(nwc::launch_gemv_tc(p, tmap, (int)h->tile_cols, h->lmax <= 7, ts, cs));
+}
+
 // The GEMV launches, with split-K scratch at `counters` (u32 [tiles_r], zero
 // on entry and left zero) and `partial` (scratch_bytes_for bytes less the
 // counters' 256-byte-padded area).
 nwc_status gemv_run(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t batch,
                     uint32_t* counters, float* partial, cudaStream_t cs) {
+  if (use_tensor_cores(*h, d_x, batch)) return gemv_run_tc(h, d_x, d_y, batch, counters, partial, cs);
   for (int32_t b0 = 0; b0 < batch; b0 += kChunkBatch) {
     const int32_t nb = batch - b0 < kChunkBatch ? batch - b0 : kChunkBatch;
     // The x-stage class (and with it the schedule and ring) follows the rows
@@ -561,7 +721,7 @@ nwc_status nwc_gemv_noalloc(nwc_handle_t h, const uint16_t* d_x, float* d_y, int
   // rejected call enqueues nothing.
   nwc_status st = gemv_check(h, d_x, d_y, batch);
   if (st != NWC_OK) return st;
-  const uint64_t need = scratch_bytes_for(*h, batch);
+  const uint64_t need = scratch_bytes_for(*h, batch, use_tensor_cores(*h, d_x, batch));
   if (need > NWC_NOALLOC_SCRATCH_BYTES) return NWC_ERR_SCRATCH_LIMIT;
   uint8_t* ws = nullptr;
   if (need) {
@@ -607,6 +767,22 @@ nwc_status nwc_get_device_error(nwc_handle_t h, nwc_stream_t stream, uint32_t* w
   if (w & nwc::kErrTimeout) return NWC_ERR_DEVICE_TIMEOUT;
   if (w & nwc::kErrCorrupt) return NWC_ERR_DEVICE_CORRUPT;
   if (w & nwc::kErrRange) return NWC_ERR_INVALID_ARG;
+  if (w & nwc::kErrLayout) return NWC_ERR_UNSUPPORTED;
+  return NWC_OK;
+}
+
+nwc_status nwc_gemv_set_tc_min_batch(nwc_handle_t h, int32_t min_batch) {
+  if (!h || min_batch < 0 || min_batch > nwc::kMaxTcRows) return NWC_ERR_INVALID_ARG;
+  h->tc_min_batch = min_batch;
+  return NWC_OK;
+}
+
+nwc_status nwc_gemv_path(nwc_handle_t h, const uint16_t* d_x, int32_t batch, int32_t* launches,
+                         int32_t* tensor_cores) {
+  if (!h || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
+  const bool tc = use_tensor_cores(*h, d_x, batch);
+  if (launches) *launches = tc ? 1 : (batch + kChunkBatch - 1) / kChunkBatch;
+  if (tensor_cores) *tensor_cores = tc ? 1 : 0;
   return NWC_OK;
 }
 
@@ -648,6 +824,45 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
   if (tile_ring)
     std::memcpy(tile_ring, sched.data() + nwc::sched_tile_off((uint64_t)h.tiles),
                 4 * (size_t)h.tiles);
+  return NWC_OK;
+}
+
+nwc_status nwc_tc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
+                                    uint64_t smem_limit, nwc_tc_schedule_info* info,
+                                    uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring,
+                                    uint32_t* tile_batch) {
+  if (!blob || !info || info->struct_size < sizeof(nwc_tc_schedule_info) || sm_count < 1)
+    return NWC_ERR_INVALID_ARG;
+  nwc_handle_s h;
+  nwc_status st = parse(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &h, nullptr);
+  if (st != NWC_OK) return st;
+  nwc::TcShape ts;
+  if (!tc_shape_on(h, sm_count, (size_t)smem_limit, &ts)) return NWC_ERR_UNSUPPORTED;
+  std::vector<uint8_t> sched;
+  try {
+    sched.resize(nwc::sched_tc_bytes((uint64_t)h.tiles));
+  } catch (const std::bad_alloc&) {
+    return NWC_ERR_NOMEM;
+  }
+  nwc::build_tc_schedule(h.index.data(), h.tiles_r, h.tiles_c, ts, sched.data());
+  const uint32_t* cb = reinterpret_cast<const uint32_t*>(sched.data());
+  info->ctas = ts.s.ctas;
+  info->rows = ts.rows;
+  info->teams = ts.teams;
+  info->batch_tiles = ts.s.batch_tiles;
+  info->ring_bytes = ts.s.ring_bytes;
+  info->tiles = h.tiles;
+  info->batches = cb[ts.s.ctas];
+  info->smem_bytes = ts.s.smem_bytes;
+  info->a_offset = ts.a_off;
+  info->b_offset = ts.b_off;
+  info->ring_offset = ts.s.ring_offset;
+  const uint64_t tiles = (uint64_t)h.tiles;
+  if (cta_batch) std::memcpy(cta_batch, cb, 4 * ((size_t)ts.s.ctas + 1));
+  if (batch) std::memcpy(batch, sched.data() + nwc::sched_batch_off(), 16 * (size_t)cb[ts.s.ctas]);
+  if (tile_ring) std::memcpy(tile_ring, sched.data() + nwc::sched_tc_ring_off(tiles), 4 * tiles);
+  if (tile_batch)
+    std::memcpy(tile_batch, sched.data() + nwc::sched_tc_tbatch_off(tiles), 4 * tiles);
   return NWC_OK;
 }
 

@@ -101,7 +101,24 @@ constexpr int kStageClasses = 2;
 constexpr uint64_t sched_class_bytes(uint64_t tiles) {
   return round_up(sched_tile_off(tiles) + 4ull * tiles, 256);
 }
-constexpr uint64_t sched_bytes(uint64_t tiles) { return kStageClasses * sched_class_bytes(tiles); }
+// The tensor-core kernel's schedule follows the class schedules.  Its CTAs
+// take their tiles in another order (row panels, see kernels.cuh), so a copy
+// may move a single tile; it adds, per tile, the batch that brings it:
+//   u32 cta_batch[kMaxCtas + 1] | u32x4 batch[tiles + kMaxCtas]
+//   | u32 tile_ring[tiles] | u32 tile_batch[tiles]
+// tile_batch = batch index | (extra releases << 28): a batch of fewer tiles
+// than the launch's batch_tiles has its first tile release it once more for
+// each missing one.  Arrays are indexed by blob tile u = j tiles_r + i.
+constexpr uint64_t sched_tc_ring_off(uint64_t tiles) {
+  return sched_batch_off() + 16ull * (tiles + kMaxCtas);
+}
+constexpr uint64_t sched_tc_tbatch_off(uint64_t tiles) { return sched_tc_ring_off(tiles) + 4ull * tiles; }
+constexpr uint64_t sched_tc_bytes(uint64_t tiles) {
+  return round_up(sched_tc_tbatch_off(tiles) + 4ull * tiles, 256);
+}
+constexpr uint64_t sched_bytes(uint64_t tiles) {
+  return kStageClasses * sched_class_bytes(tiles) + sched_tc_bytes(tiles);
+}
 
 // Rows of x one launch of the CUDA-core GEMV kernel handles (one 16-row
 // tensor-core operand of mma.sync); larger batches run as several launches.

@@ -103,8 +103,6 @@ def test_gpu_decodes_oracle_blob(lib, orc, lmax):
 @pytest.mark.parametrize("shape,tile_cols", SHAPES)
 @pytest.mark.parametrize("batch", [1, 3, 8])
 def test_gemv_parity_shapes(lib, orc, shape, tile_cols, batch, lmax):
-    if shape[1] % 2:
-        pytest.skip("nwc_gemv requires an even number of columns")
     spec = synth.MatrixSpec("w", shape[0], shape[1], "normal", 0.02, 2)
     w = synth.matrix(spec, 6)
     x = synth.activations(6, batch, shape[1])
@@ -202,6 +200,21 @@ def test_sharded_matrix_single_process(lib, orc):
     m.close()
 
 
+@pytest.mark.parametrize("batch", [1, 2, 5, 16, 40])
+@pytest.mark.parametrize("cols", [1, 3, 513, 1025, 4097])
+def test_gemv_odd_columns(lib, orc, cols, batch):
+    """An odd number of columns: x rows start on 2-byte boundaries, read one
+    element at a time; staged in shared memory or read directly."""
+    spec = synth.MatrixSpec("w", 300, cols, "normal", 0.02, 1)
+    w = synth.matrix(spec, 3)
+    x = synth.activations(3, batch, cols)
+    m = lib.CompressedMatrix.compress(w)
+    xt = to_bf16(x)
+    assert lib.nwc_gemv_path(m.handle, xt, batch)[1] is False
+    tolerance_check(m.gemv(xt).cpu().numpy(), orc.gemv(w, x), w, x)
+    no_device_error(lib, m)
+
+
 def test_gemv_into_pinned_host_memory(lib, orc):
     """y may be pinned host memory the device can address: the kernel stores the
     result there directly."""
@@ -279,9 +292,9 @@ def test_invalid_arguments_rejected(lib):
     with pytest.raises(lib.NwcError):            # misaligned x
         lib.nwc_gemv(m.handle, x.data_ptr() + 2, y, 1)
     odd = lib.CompressedMatrix.compress(synth.matrix(synth.MatrixSpec("w", 4, 5, "normal", 0.02, 0), 0))
-    x5 = torch.zeros((1, 5), dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(lib.NwcError):            # odd column count
-        lib.nwc_gemv(odd.handle, x5, torch.zeros(4, device="cuda"), 1)
+    x5 = torch.zeros((2, 5), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lib.NwcError):            # x of an odd-width matrix on an odd address
+        lib.nwc_gemv(odd.handle, x5.data_ptr() + 1, torch.zeros(4, device="cuda"), 1)
     blob = np.zeros(1024, dtype=np.uint8)
     with pytest.raises(lib.NwcError):
         lib.CompressedMatrix.from_blob(blob)
