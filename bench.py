@@ -59,6 +59,14 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--e2e-mode", default="host-y", choices=["copy", "host-y"],
                     help="how y reaches the host in the end-to-end leg")
+    ap.add_argument("--streams", type=int, default=1, choices=[1, 2],
+                    help="bit streams per lane and tile of the compressed matrices")
+    ap.add_argument("--code", default="prefix", choices=["prefix", "rank"],
+                    help="exponent code: the length-limited prefix code (NWB1) or the ranked "
+                         "unary code (NWR1, 7 ranks)")
+    ap.add_argument("--tc-min-batch", type=int, default=None,
+                    help="smallest batch that takes the tensor-core kernel (default: the "
+                         "library's, 16; 0 = never)")
     ap.add_argument("--report", action="store_true",
                     help="the five configurations as a markdown table (not the headline line)")
     ap.add_argument("--report-json", default=None, help="with --report: every line, to this file")
@@ -301,6 +309,7 @@ def run_reference(args) -> None:
 
 
 STACKS = ("qwen3_4b_stack", "llama31_8b_stack")
+CODES = {"prefix": 0, "rank": 1}    # nwc_opts.code
 
 
 def run_stack(args) -> None:
@@ -331,7 +340,9 @@ def run_stack(args) -> None:
     for sp in specs:
         host_w[sp.name] = (synth.head_matrix(sp, wl.seed) if sp is head
                            else synth.stacked_matrix(parts_of[sp.name], wl.seed))
-        comp[sp.name] = _lib.CompressedMatrix.compress(host_w[sp.name], device=dev)
+        comp[sp.name] = _lib.CompressedMatrix.compress(host_w[sp.name], device=dev,
+                                                       streams=args.streams,
+                                                       code=CODES[args.code])
     sets = [{sp.name: comp[sp.name] for sp in layer0}]
     second = {}
     for sp in layer0:
@@ -340,6 +351,9 @@ def run_stack(args) -> None:
         m.handle = _lib.nwc_handle_from_device(m.image, m.image.numel())
         second[sp.name] = m
     sets.append(second)
+    if args.tc_min_batch is not None:
+        for m in list(comp.values()) + list(second.values()):
+            _lib.nwc_gemv_set_tc_min_batch(m.handle, args.tc_min_batch)
     xs = {k: torch.from_numpy(synth.activations(wl.seed, batch, k).view(np.int16))
           .view(torch.bfloat16).to(dev) for k in {sp.cols for sp in specs}}
     ys = {n: torch.empty((batch, n), dtype=torch.float32, device=dev) for n in {sp.rows for sp in specs}}
@@ -476,7 +490,8 @@ def run_stack(args) -> None:
         "config": {"workload": args.workload, "batch": batch, "step": f"one token: {len(seq)} GEMVs "
                    f"({n_layers} layers x {len(layer0)} + lm_head), one CUDA graph",
                    "layer": [f"{g} {sp.rows}x{sp.cols}" for (g, _), sp in zip(units, layer0)],
-                   "fused": bool(args.fuse),
+                   "fused": bool(args.fuse), "streams_per_lane": args.streams,
+                   "code": args.code,
                    "weights": "layer 0 generated, two device copies alternating over the layers; "
                               f"lm_head = its first {synth.HEAD_BLOCK_ROWS} rows repeated",
                    "l2": "inputs larger than L2: every layer is larger than L2",
@@ -519,7 +534,8 @@ def run_matrix(args):
     batch = args.batch
     w = synth.matrix(spec, wl.seed)
     x_host = synth.activations(wl.seed, batch, spec.cols)
-    first = _lib.CompressedMatrix.compress(w, device=dev)
+    first = _lib.CompressedMatrix.compress(w, device=dev, streams=args.streams,
+                                           code=CODES[args.code])
     image_bytes = first.compressed_bytes   # blob, table and schedules (no scratch)
     copies = max(2, int(np.ceil(2.2 * L2_BYTES / image_bytes)))
     copies = min(copies, args.steps) if args.steps >= 2 else copies
@@ -527,6 +543,9 @@ def run_matrix(args):
                                             first.blob_bytes) for _ in range(copies - 1)]
     for m in mats[1:]:
         m.handle = _lib.nwc_handle_from_device(m.image, m.image.numel())
+    if args.tc_min_batch is not None:
+        for m in mats:
+            _lib.nwc_gemv_set_tc_min_batch(m.handle, args.tc_min_batch)
     x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
     y = torch.empty((batch, spec.rows), dtype=torch.float32, device=dev)
     launches_per_call, on_tc = _lib.nwc_gemv_path(first.handle, x, batch)
@@ -695,7 +714,8 @@ def run_matrix(args):
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "matrix": f"{spec.rows}x{spec.cols}",
-                   "batch": batch, "values": spec.kind,
+                   "batch": batch, "values": spec.kind, "streams_per_lane": args.streams,
+                   "code": args.code,
                    "l2": f"inputs larger than L2: {copies} rotating compressed copies "
                          f"({copies * image_bytes / 2**20:.0f} MiB)",
                    "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},

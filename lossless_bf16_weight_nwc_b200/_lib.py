@@ -135,8 +135,8 @@ def nwc_version() -> int:
 def nwc_plan(w_host: np.ndarray, lmax: int = 0, tile_cols: int = 512, threads: int = 0,
              code: int = NWC_CODE_PREFIX, streams: int = 1):
     """code NWC_CODE_RANK: the ranked unary code, lmax = number of ranks (0 = 7);
-    streams 2 or 4: bit streams per lane.  Both host encoder only for now
-    (nwc_compress_host)."""
+    streams 2 or 4: bit streams per lane (the kernels read 1 and 2; 4 is host
+    encoder only, nwc_compress_host)."""
     w = np.ascontiguousarray(w_host, dtype=np.uint16)
     rows, cols = w.shape
     opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads, code, streams)
@@ -340,9 +340,14 @@ class CompressedMatrix:
 
     @classmethod
     def compress(cls, w_host: np.ndarray, device="cuda", lmax: int = 0, tile_cols: int = 512,
-                 threads: int = 0, stream=None) -> "CompressedMatrix":
+                 threads: int = 0, stream=None, streams: int = 1,
+                 code: int = NWC_CODE_PREFIX) -> "CompressedMatrix":
+        """streams: bit streams per lane and tile (1 or 2; with 2 a lane's
+        decoder follows two independent streams).  code NWC_CODE_RANK: the
+        ranked unary code, lmax = its number of ranks (0 = 7)."""
         import torch
-        plan = nwc_plan(w_host, lmax=lmax, tile_cols=tile_cols, threads=threads)
+        plan = nwc_plan(w_host, lmax=lmax, tile_cols=tile_cols, threads=threads, streams=streams,
+                        code=code)
         try:
             dev_bytes, blob_bytes = nwc_plan_size(plan)
             image = torch.empty(dev_bytes, dtype=torch.uint8, device=device)
@@ -354,7 +359,7 @@ class CompressedMatrix:
 
     @classmethod
     def compress_fused(cls, parts, device="cuda", lmax: int = 0, tile_cols: int = 512,
-                       threads: int = 0, stream=None) -> "CompressedMatrix":
+                       threads: int = 0, stream=None, streams: int = 1) -> "CompressedMatrix":
         """Projections that read the same input (q, k, v; gate, up) held as one
         matrix: the parts' rows stacked in order under one code table, so that a
         call is one launch ("NWC — Neural Weight Compression", "Install": fuse
@@ -364,7 +369,7 @@ class CompressedMatrix:
         if not ws or any(w.ndim != 2 or w.shape[1] != ws[0].shape[1] for w in ws):
             raise ValueError("parts: one or more 2-D matrices with the same number of columns")
         m = cls.compress(np.concatenate(ws, axis=0), device=device, lmax=lmax,
-                         tile_cols=tile_cols, threads=threads, stream=stream)
+                         tile_cols=tile_cols, threads=threads, stream=stream, streams=streams)
         m.row_splits = [int(v) for v in np.cumsum([0] + [w.shape[0] for w in ws])]
         return m
 

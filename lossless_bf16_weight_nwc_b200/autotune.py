@@ -1,17 +1,27 @@
-"""Per-shape choice of the compressed format by measurement.
+"""Per-shape choice of the GEMV strategy by measurement.
 
 "Unweight: how we compressed an LLM 22% without sacrificing quality", section
 "Direct GPU Decompression": the execution strategy depends on the weight
 matrix and the batch size, and an autotuner picks the fastest one for each
-workload.  Here the strategies are the format's tile width (64, 128, 256 or
-512 columns: how many tiles, and so how the persistent CTAs and the split-K
-reduction divide a matrix) and its code limit (7 bits, whose 14-bit peek always
-holds two codes, or a longer limit).  Both are fixed when a matrix is
-compressed, so `tune` compresses the matrix once per candidate, times its GEMV
-at the given batch on the current device with CUDA events, and returns the
-fastest.  Choices are remembered per (device, rows, cols, batch), the
-quantities they depend on (the values move the compressed size by a few per
-cent at most).
+workload.  Here a strategy is
+
+* the format, fixed when a matrix is compressed: the tile width (64, 128, 256
+  or 512 columns: how many tiles, and so how the persistent CTAs divide a
+  matrix), the code limit (7 bits, whose 14-bit table peek always holds two
+  codes, or a longer limit), the bit streams per lane (1, or 2 so that a lane
+  follows two independent decode chains) and the exponent code (the
+  length-limited prefix code, or the table-free ranked unary code);
+* the kernel, chosen per call: the CUDA-core kernel (mma.sync on the decoded
+  registers, up to 16 rows of x per launch, the matrix decoded again for every
+  16 rows) or the tensor-core kernel (tcgen05, each weight decoded once into
+  shared memory for up to 64 rows of x).
+
+`tune` compresses the matrix once per format, times its GEMV at the given batch
+under each kernel on the current device with CUDA events behind an L2 flush,
+and returns the fastest.  Choices are remembered per (device, rows, cols,
+batch), the quantities they depend on (the values move the compressed size by
+a few per cent at most).  `apply` sets a compressed matrix's kernel threshold
+from a choice.
 
 Every timed call runs the library's kernels; this module only chooses among
 them.
@@ -21,41 +31,88 @@ from __future__ import annotations
 import dataclasses
 import json
 import os
-from typing import Callable, Iterable, Sequence
+from typing import Callable, Iterable
 
 import numpy as np
 
-# (tile_cols, lmax): lmax 0 is the library's automatic limit (7 unless the
-# matrix holds more than 128 distinct exponents).
-DEFAULT_CANDIDATES: tuple[tuple[int, int], ...] = ((512, 0), (256, 0), (128, 0), (512, 12))
 TILE_COLS = (64, 128, 256, 512)
+CODES = ("prefix", "rank")
+KERNELS = ("cuda", "tensor")
+
+
+@dataclasses.dataclass(frozen=True)
+class Strategy:
+    tile_cols: int = 512
+    lmax: int = 0          # prefix: 0 = automatic (7 unless > 128 exponents); rank: ranks (0 = 7)
+    streams: int = 1
+    code: str = "prefix"
+    kernel: str = "cuda"
+
+    @property
+    def key(self) -> str:
+        return f"{self.tile_cols}/{self.lmax}/{self.streams}/{self.code}/{self.kernel}"
+
+    @property
+    def format(self) -> tuple:
+        return (self.tile_cols, self.lmax, self.streams, self.code)
+
+
+def default_candidates(batch: int) -> list[Strategy]:
+    """The formats worth comparing, each under the kernels that suit the batch
+    (the tensor-core kernel for any batch; the CUDA-core one up to 16 rows of x
+    per launch, so for larger batches only as a baseline)."""
+    formats = [(512, 0, 1, "prefix"), (512, 0, 2, "prefix"), (256, 0, 1, "prefix"),
+               (512, 12, 1, "prefix"), (512, 0, 1, "rank")]
+    kernels = ("cuda", "tensor") if batch >= 8 else ("cuda",)
+    return [Strategy(*f, kernel=k) for f in formats for k in kernels]
 
 
 @dataclasses.dataclass(frozen=True)
 class Choice:
-    tile_cols: int
-    lmax: int
+    strategy: Strategy
     us_per_call: float
-    timings: dict  # "tile_cols/lmax" -> microseconds per call
+    timings: dict  # Strategy.key -> microseconds per call
+
+    def to_json(self) -> dict:
+        return {"strategy": dataclasses.asdict(self.strategy), "us_per_call": self.us_per_call,
+                "timings": self.timings}
+
+    @classmethod
+    def from_json(cls, d: dict) -> "Choice":
+        return cls(Strategy(**d["strategy"]), float(d["us_per_call"]), dict(d["timings"]))
 
 
 def _key(device_name: str, rows: int, cols: int, batch: int) -> str:
     return f"{device_name}|{rows}x{cols}|b{batch}"
 
 
-def validate_candidates(candidates: Iterable[Sequence[int]]) -> list[tuple[int, int]]:
+def validate_candidates(candidates: Iterable[Strategy]) -> list[Strategy]:
     out = []
-    for cand in candidates:
-        tile_cols, lmax = int(cand[0]), int(cand[1])
-        if tile_cols not in TILE_COLS:
-            raise ValueError(f"tile_cols {tile_cols}: one of {TILE_COLS}")
-        if not 0 <= lmax <= 12:
-            raise ValueError(f"lmax {lmax}: 0 (automatic) or 1..12")
-        if (tile_cols, lmax) not in out:
-            out.append((tile_cols, lmax))
+    for s in candidates:
+        if not isinstance(s, Strategy):
+            raise TypeError(f"{s!r}: expected a Strategy")
+        if s.tile_cols not in TILE_COLS:
+            raise ValueError(f"tile_cols {s.tile_cols}: one of {TILE_COLS}")
+        if s.code not in CODES:
+            raise ValueError(f"code {s.code!r}: one of {CODES}")
+        if s.kernel not in KERNELS:
+            raise ValueError(f"kernel {s.kernel!r}: one of {KERNELS}")
+        if s.streams not in (1, 2) or (s.code == "rank" and s.streams != 1):
+            raise ValueError(f"streams {s.streams}: 1 or 2 (1 for the rank code)")
+        if not 0 <= s.lmax <= (7 if s.code == "rank" else 12):
+            raise ValueError(f"lmax {s.lmax}: 0 (automatic) or 1..12 (ranks: 1..7)")
+        if s not in out:
+            out.append(s)
     if not out:
         raise ValueError("no candidates")
     return out
+
+
+def apply(m, strategy: Strategy) -> None:
+    """Make a compressed matrix's GEMVs take the strategy's kernel: the
+    tensor-core kernel for every batch, or never."""
+    from ._lib import nwc_gemv_set_tc_min_batch
+    nwc_gemv_set_tc_min_batch(m.handle, 1 if strategy.kernel == "tensor" else 0)
 
 
 def time_gemv(m, x, reps: int = 50, flush_bytes: int = 256 << 20) -> float:
@@ -85,10 +142,12 @@ class Tuner:
     def __init__(self, path: str | None = None,
                  compress: Callable | None = None, timer: Callable | None = None,
                  device_name: Callable[[], str] | None = None,
-                 activations: Callable[[int, int], object] | None = None):
-        """compress(w, tile_cols, lmax), timer(matrix, x, reps) -> microseconds,
-        device_name() and activations(batch, cols) default to the library, CUDA
-        events, the current CUDA device and seeded BF16 activations on it."""
+                 activations: Callable[[int, int], object] | None = None,
+                 set_kernel: Callable | None = None):
+        """compress(w, strategy) -> matrix, timer(matrix, x, reps) ->
+        microseconds, set_kernel(matrix, strategy), device_name() and
+        activations(batch, cols) default to the library, CUDA events, the
+        current CUDA device and seeded BF16 activations on it."""
         self.path = path
         self.cache: dict[str, dict] = {}
         if path and os.path.exists(path):
@@ -98,6 +157,7 @@ class Tuner:
         self._timer = timer
         self._device_name = device_name
         self._make_x = activations
+        self._set_kernel = set_kernel
 
     def _name(self) -> str:
         if self._device_name is not None:
@@ -107,9 +167,9 @@ class Tuner:
 
     def lookup(self, rows: int, cols: int, batch: int) -> Choice | None:
         hit = self.cache.get(_key(self._name(), rows, cols, batch))
-        return None if hit is None else Choice(**hit)
+        return None if hit is None else Choice.from_json(hit)
 
-    def tune(self, w_host: np.ndarray, batch: int, candidates=DEFAULT_CANDIDATES,
+    def tune(self, w_host: np.ndarray, batch: int, candidates: Iterable[Strategy] | None = None,
              reps: int = 50, retune: bool = False) -> Choice:
         """The fastest candidate for this matrix shape and batch on the current
         device (from the cache unless retune)."""
@@ -121,31 +181,39 @@ class Tuner:
         rows, cols = w_host.shape
         key = _key(self._name(), rows, cols, batch)
         if not retune and key in self.cache:
-            return Choice(**self.cache[key])
-        cands = validate_candidates(candidates)
+            return Choice.from_json(self.cache[key])
+        cands = validate_candidates(default_candidates(batch) if candidates is None
+                                    else candidates)
         compress = self._compress or self._compress_default
         timer = self._timer or time_gemv
+        set_kernel = self._set_kernel or apply
         x = self._activations(batch, cols)
         timings, refused = {}, {}
-        for tile_cols, lmax in cands:
+        formats: dict[tuple, list[Strategy]] = {}
+        for s in cands:
+            formats.setdefault(s.format, []).append(s)
+        for fmt, strategies in formats.items():
             try:
-                m = compress(w_host, tile_cols=tile_cols, lmax=lmax)
+                m = compress(w_host, strategies[0])
             except RuntimeError as e:  # e.g. a code limit too short for the matrix
-                refused[f"{tile_cols}/{lmax}"] = str(e)
+                for s in strategies:
+                    refused[s.key] = str(e)
                 continue
             try:
-                timings[f"{tile_cols}/{lmax}"] = float(timer(m, x, reps))
+                for s in strategies:
+                    set_kernel(m, s)
+                    timings[s.key] = float(timer(m, x, reps))
             finally:
                 close = getattr(m, "close", None)
                 if close:
                     close()
         if not timings:
             raise RuntimeError(f"no candidate could be compressed: {refused}")
-        timed = [c for c in cands if f"{c[0]}/{c[1]}" in timings]
-        # Fastest; on a tie the wider tile, then the automatic code limit.
-        best = min(timed, key=lambda c: (timings[f"{c[0]}/{c[1]}"], -c[0], c[1]))
-        choice = Choice(best[0], best[1], timings[f"{best[0]}/{best[1]}"], timings)
-        self.cache[key] = dataclasses.asdict(choice)
+        timed = [s for s in cands if s.key in timings]
+        # Fastest; on a tie the earlier candidate (the simpler format first).
+        best = min(timed, key=lambda s: (timings[s.key], timed.index(s)))
+        choice = Choice(best, timings[best.key], timings)
+        self.cache[key] = choice.to_json()
         if self.path:
             with open(self.path, "w") as f:
                 json.dump(self.cache, f, indent=1, sort_keys=True)
@@ -160,6 +228,45 @@ class Tuner:
         return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).cuda()
 
     @staticmethod
-    def _compress_default(w_host, tile_cols, lmax):
-        from ._lib import CompressedMatrix
-        return CompressedMatrix.compress(w_host, tile_cols=tile_cols, lmax=lmax)
+    def _compress_default(w_host, s: Strategy):
+        from ._lib import NWC_CODE_PREFIX, NWC_CODE_RANK, CompressedMatrix
+        return CompressedMatrix.compress(w_host, tile_cols=s.tile_cols, lmax=s.lmax,
+                                         streams=s.streams,
+                                         code=NWC_CODE_RANK if s.code == "rank" else NWC_CODE_PREFIX)
+
+
+def sweep(workloads, batches, path: str, reps: int = 30) -> dict:
+    """Tunes every distinct matrix shape of the given workloads (synthetic
+    weights of the workload's distribution) at each batch; returns and saves
+    the cache."""
+    from . import synth
+    tuner = Tuner(path)
+    for name in workloads:
+        if name in ("qwen3_4b_stack", "llama31_8b_stack"):
+            wl, layer0, head, _ = synth.stack_parts(name)
+            specs = layer0 + [head]
+        else:
+            wl = synth.workload(name)
+            head, specs = None, list(wl.matrices)
+        seen = set()
+        for spec in specs:
+            if (spec.rows, spec.cols) in seen:
+                continue
+            seen.add((spec.rows, spec.cols))
+            w = synth.head_matrix(spec, wl.seed) if spec is head else synth.matrix(spec, wl.seed)
+            for batch in batches:
+                c = tuner.tune(w, batch, reps=reps)
+                print(f"{name} {spec.rows}x{spec.cols} b{batch}: {c.strategy.key} "
+                      f"{c.us_per_call:.2f} us", flush=True)
+    return tuner.cache
+
+
+if __name__ == "__main__":
+    import argparse
+    ap = argparse.ArgumentParser(description="tune the GEMV strategy per matrix shape and batch")
+    ap.add_argument("--workloads", nargs="+", default=["qwen3_4b_stack", "llama31_8b_stack"])
+    ap.add_argument("--batches", nargs="+", type=int, default=[1, 16, 64])
+    ap.add_argument("--out", required=True, help="the JSON cache to write (and extend)")
+    ap.add_argument("--reps", type=int, default=30)
+    a = ap.parse_args()
+    sweep(a.workloads, a.batches, a.out, a.reps)

@@ -309,7 +309,7 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   for (int s = 0; s < 256; ++s) p->coded_bits += cnt[s] * p->len[s];
   const int rc = plan_tiles(w, p);
   if (rc != 0) return rc;
-  if (p->streams != 1) {  // no kernel reads several streams per lane yet
+  if (p->streams > kMaxDeviceStreams) {  // no kernel reads four streams per lane
     p->table_off = p->sched_off = p->scratch_off = p->device_bytes = 0;
     return 0;
   }
@@ -384,9 +384,21 @@ int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile
   for (int e = 0; e < 128; ++e) p->coded_bits += cnt[e] * (uint64_t)(p->rank_len[e] + 1);
   const int rc = plan_tiles(w, p);
   if (rc != 0) return rc;
-  // No kernel reads this code yet: there is no device image.
-  p->table_off = p->sched_off = p->scratch_off = p->device_bytes = 0;
+  const ImageLayout L =
+      image_layout(p->blob_bytes, p->lmax, (uint64_t)p->tiles_r, (uint64_t)p->tiles_c, true);
+  p->table_off = L.table_off;
+  p->sched_off = L.sched_off;
+  p->scratch_off = L.scratch_off;
+  p->device_bytes = L.device_bytes;
   return 0;
+}
+
+void build_rank_table(const uint8_t* ranked, uint32_t ranks, uint32_t* out) {
+  std::memset(out, 0, kRankTableBytes);
+  uint8_t bytes[8] = {};
+  for (uint32_t r = 0; r < ranks && r < (uint32_t)kMaxRanks; ++r) bytes[r] = ranked[r];
+  std::memcpy(out, bytes, 8);
+  out[2] = ranks;
 }
 
 // Chunk sizes -> index, tile-area offset and blob size (either code).
@@ -509,14 +521,20 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   if (!blob || head_bytes < kHeaderBytes + 256 || head_bytes > bytes) return false;
   BlobHeader h;
   std::memcpy(&h, blob, sizeof(h));
-  if (h.magic != kMagic || h.version != kVersion || h.header_bytes != kHeaderBytes) return false;
-  if (h.lmax < 1 || h.lmax > (uint32_t)kMaxLmax || h.tile_rows != (uint32_t)kTileRows) return false;
+  const bool rank = h.magic == kRankMagic;
+  if ((h.magic != kMagic && !rank) || h.version != kVersion || h.header_bytes != kHeaderBytes)
+    return false;
+  const uint32_t lmax_cap = rank ? (uint32_t)kMaxRanks : (uint32_t)kMaxLmax;
+  if (h.lmax < 1 || h.lmax > lmax_cap || h.tile_rows != (uint32_t)kTileRows) return false;
   if (h.tile_cols < 64 || h.tile_cols > (uint32_t)kMaxTileCols || h.tile_cols % 64) return false;
   if (h.rows < 1 || h.cols < 1 || h.rows > (1ull << 40) || h.cols > (1ull << 40)) return false;
   if (h.tiles_r != (h.rows + 7) / 8 || h.tiles_c != (h.cols + h.tile_cols - 1) / h.tile_cols)
     return false;
   if (h.lens_off != kLensOffset || h.index_off != kIndexOffset || h.filler > 255) return false;
-  if (h.zero != 0) return false;  // one bit stream per lane (the streams field, S - 1)
+  // The streams field holds S - 1 for S bit streams per lane (1 or 2 here;
+  // the ranked unary code has one).
+  if (h.zero + 1 > (rank ? 1u : kMaxDeviceStreams)) return false;
+  const uint32_t S = h.zero + 1;
   // Every tile has a 4-byte index entry inside the head, which bounds the tile
   // count before it is formed: no size computed from it below can wrap around.
   const uint64_t max_tiles = head_bytes / 4;
@@ -525,19 +543,35 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   if (h.tiles_off != round_up(kIndexOffset + 4 * (tiles + 1), 256)) return false;
   if (h.total_bytes != bytes || h.tiles_off > head_bytes) return false;
   const uint8_t* lens = blob + kLensOffset;
-  double kraft = 0;
-  for (int s = 0; s < 256; ++s) {
-    if (lens[s] > h.lmax) return false;
-    if (lens[s]) kraft += 1.0 / double(1u << lens[s]);
+  if (rank) {
+    // R distinct values of the 7-bit field in rank order, then zeros; rank 0
+    // is the filler's.
+    bool seen[128] = {};
+    for (uint32_t r = 0; r < 256; ++r) {
+      if (r >= h.lmax) {
+        if (lens[r]) return false;
+        continue;
+      }
+      if (lens[r] > 127 || seen[lens[r]]) return false;
+      seen[lens[r]] = true;
+    }
+    if (h.filler != lens[0]) return false;
+  } else {
+    double kraft = 0;
+    for (int s = 0; s < 256; ++s) {
+      if (lens[s] > h.lmax) return false;
+      if (lens[s]) kraft += 1.0 / double(1u << lens[s]);
+    }
+    if (kraft > 1.0 || lens[h.filler] == 0) return false;
   }
-  if (kraft > 1.0 || lens[h.filler] == 0) return false;
   auto index_at = [&](uint64_t u) {
     uint32_t v;
     std::memcpy(&v, blob + kIndexOffset + 4 * u, 4);
     return v;
   };
-  const uint64_t max_chunk = max_chunk_bytes(h.tile_cols, h.lmax);
-  const uint64_t min_chunk = raw_bytes(h.tile_cols) + kLanes;
+  const uint64_t max_chunk =
+      rank ? max_rank_chunk_bytes(h.tile_cols, h.lmax) : max_chunk_bytes(h.tile_cols, h.lmax, S);
+  const uint64_t min_chunk = raw_bytes(h.tile_cols) + kLanes * S;
   uint64_t largest = 0;
   if (index_at(0) != 0) return false;
   uint32_t prev = 0;
@@ -554,6 +588,8 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   hd->cols = (int64_t)h.cols;
   hd->tile_cols = h.tile_cols;
   hd->lmax = h.lmax;
+  hd->streams = S;
+  hd->code_kind = rank ? 1u : 0u;
   hd->filler = h.filler;
   hd->tiles_r = (int64_t)h.tiles_r;
   hd->tiles_c = (int64_t)h.tiles_c;
@@ -563,7 +599,7 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   std::memcpy(hd->index.data(), blob + kIndexOffset, 4 * ((size_t)tiles + 1));
   hd->tiles_off = h.tiles_off;
   hd->blob_bytes = bytes;
-  const ImageLayout L = image_layout(bytes, h.lmax, h.tiles_r, h.tiles_c);
+  const ImageLayout L = image_layout(bytes, h.lmax, h.tiles_r, h.tiles_c, rank);
   hd->table_off = L.table_off;
   hd->sched_off = L.sched_off;
   hd->scratch_off = L.scratch_off;

@@ -38,11 +38,14 @@ namespace nwc {
 
 namespace {
 
-constexpr int kRingSlack = 256;                  // readers may run past a chunk (corrupt data)
+constexpr int kRingSlack = 512;                  // readers may run past a chunk (corrupt data)
 constexpr int kTablePieces = 8;                  // bulk copies that bring in the decode table
 constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
 constexpr uint32_t kPairReadSpan = 12 + 4 * kMaxPairSteps + 4;  // bytes one tile's reader may touch
 static_assert(kPairReadSpan <= kRingSlack, "a clamped reader must stay inside the ring slack");
+// The rank reader advances at most one word per pair (64 pairs per tile).
+constexpr uint32_t kRankReadSpan = 12 + 4 * 2 * kMaxPairSteps + 4;
+static_assert(kRankReadSpan <= kRingSlack, "a clamped rank reader must stay inside the slack");
 constexpr uint64_t kBatchTarget = 12288;          // bytes a bulk copy should move at least
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -299,15 +302,70 @@ struct PairReader {
   }
 };
 
-// Both readers behind one interface: two() yields the entries of the next two
-// steps.  FAST uses the window reader above; lmax 8..12 the bit buffer, whose
-// second lookup handles a pair that does not fit in the 12-bit peek.
-template <bool FAST>
+// Reader of the ranked unary code (variant NWR1; "NWC", "How it works > Prefix
+// code instead of rANS", format v9): a weight's code is its sign bit, then r
+// zeros and a one for rank r < R, else R zeros and the 7-bit field e (exponent
+// bits 14..8).  A code has at most 1 + R + 7 <= 15 bits, so one 32-bit window
+// always holds a pair of codes; the words move as in PairReader, one step
+// (pair) at a time.  No table: the R ranked values sit in two registers and a
+// rank picks its byte with one byte permute.  A step's entry carries the two
+// weights' high bytes (sign and e) at bits 8..15 and 24..31.
+struct RankReader {
+  uint32_t a, b, c, p, next;
+  uint32_t rank_lo, rank_hi, R;
+
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit,
+                                       uint32_t table) {
+    const uint32_t at = min(area + (start & ~3u), limit - kRankReadSpan);
+    a = lds32(at);
+    b = lds32(at + 4);
+    c = lds32(at + 8);
+    next = at + 12;
+    p = (start & 3u) * 8u;
+    rank_lo = lds32(table);
+    rank_hi = lds32(table + 4);
+    R = lds32(table + 8);
+  }
+  // High byte (sign << 7 | e) of the code at the top of t, and its length.
+  __device__ __forceinline__ uint32_t code(uint32_t t, uint32_t& len) const {
+    const uint32_t u = t << 1;
+    const uint32_t z = __clz(u);  // zeros after the sign bit (32 when none is one)
+    const bool ranked = z < R;
+    const uint32_t e = ranked ? (__byte_perm(rank_lo, rank_hi, z) & 0xFFu) : ((u << R) >> 25);
+    len = ranked ? z + 2u : R + 8u;
+    return ((t >> 31) << 7) | e;
+  }
+  __device__ __forceinline__ uint32_t step() {
+    const uint32_t w = __funnelshift_l(b, a, p);
+    uint32_t l0, l1;
+    const uint32_t h0 = code(w, l0);
+    const uint32_t h1 = code(w << l0, l1);
+    // The pair took at most 30 bits: a word was passed exactly when bit 5 of
+    // the offset flipped.
+    const uint32_t q = p + l0 + l1;
+    const uint32_t adv = (q ^ p) & 32u;
+    p = q;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %4, 0;\n\t"
+        "@q mov.b32 %0, %1;\n\t@q mov.b32 %1, %2;\n\t"
+        "@q ld.shared.u32 %2, [%3];\n\t@q add.u32 %3, %3, 4;\n\t}"
+        : "+r"(a), "+r"(b), "+r"(c), "+r"(next)
+        : "r"(adv));
+    return (h0 << 8) | (h1 << 24);
+  }
+};
+
+// The readers behind one interface: two() yields the entries of the next two
+// steps.  kCode14 uses the window reader, kCode12 the bit buffer (whose second
+// lookup handles a pair that does not fit in the 12-bit peek), kCodeRank the
+// rank reader.
+template <int CODE>
 struct StreamDecoder;
 template <>
-struct StreamDecoder<true> {
+struct StreamDecoder<kCode14> {
   PairReader r;
-  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit,
+                                       uint32_t) {
     r.init(area, start, limit);
   }
   __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
@@ -315,15 +373,28 @@ struct StreamDecoder<true> {
   }
 };
 template <>
-struct StreamDecoder<false> {
+struct StreamDecoder<kCode12> {
   BitReader br;
-  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit) {
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit,
+                                       uint32_t) {
     br.init(area, start, limit);
   }
   __device__ __forceinline__ void two(uint32_t table, uint32_t& e0, uint32_t& e1) {
     e0 = decode_pair<false>(br, table);
     e1 = decode_pair<false>(br, table);
     br.refill();
+  }
+};
+template <>
+struct StreamDecoder<kCodeRank> {
+  RankReader r;
+  __device__ __forceinline__ void init(uint32_t area, uint32_t start, uint32_t limit,
+                                       uint32_t table) {
+    r.init(area, start, limit, table);
+  }
+  __device__ __forceinline__ void two(uint32_t, uint32_t& e0, uint32_t& e1) {
+    e0 = r.step();
+    e1 = r.step();
   }
 };
 
@@ -348,9 +419,16 @@ __device__ __forceinline__ uint32_t raw_pair_r(const uint4& rv, int r) {
   }
 }
 
+template <int CODE>
 __device__ __forceinline__ uint32_t assemble(uint32_t rawdup, uint32_t e) {
-  // Sign+fraction from the raw bytes, exponents from the table entry.
-  return (rawdup & kEntryRawMask) | (e & kEntryExponentMask);
+  if constexpr (CODE == kCodeRank) {
+    // The raw bytes are the low bytes (exponent bit 7 and the fraction); the
+    // entry holds the high bytes (sign and exponent bits 14..8).
+    return (rawdup & 0x00FF00FFu) | e;
+  } else {
+    // Sign+fraction from the raw bytes, exponents from the table entry.
+    return (rawdup & kEntryRawMask) | (e & kEntryExponentMask);
+  }
 }
 
 // Start of lane `lane`'s stream: prefix sum of the lane byte counts.
@@ -365,6 +443,60 @@ __device__ __forceinline__ uint32_t lane_stream_start(uint32_t chunk, int raw, i
   }
   return incl - my_len;
 }
+
+// Stream starts of lane `lane` with S bit streams per lane (S = 2: the lengths
+// of streams 2t and 2t + 1 are bytes 2t and 2t + 1 of the length array).
+template <int S>
+__device__ __forceinline__ void lane_stream_starts(uint32_t chunk, int raw, int lane,
+                                                   uint32_t (&start)[S]) {
+  if constexpr (S == 1) {
+    start[0] = lane_stream_start(chunk, raw, lane);
+  } else {
+    const uint32_t w = lds32(chunk + raw + ((2 * lane) & ~3));
+    const uint32_t b = w >> (8 * ((2 * lane) & 3));
+    const uint32_t len0 = b & 0xFFu, len1 = (b >> 8) & 0xFFu;
+    const uint32_t mine = len0 + len1;
+    uint32_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += v;
+    }
+    start[0] = incl - mine;
+    start[1] = start[0] + len0;
+  }
+}
+
+// A lane's decoder over its S bit streams: quad() yields the table entries of
+// the lane's next four symbol pairs in order.  With S = 2 the pairs alternate
+// between the streams, so the two streams' dependency chains interleave.
+template <int CODE, int S>
+struct LaneDecoder;
+template <int CODE>
+struct LaneDecoder<CODE, 1> {
+  StreamDecoder<CODE> d;
+  __device__ __forceinline__ void init(uint32_t area, const uint32_t (&start)[1], uint32_t limit,
+                                       uint32_t table) {
+    d.init(area, start[0], limit, table);
+  }
+  __device__ __forceinline__ void quad(uint32_t table, uint32_t (&e)[4]) {
+    d.two(table, e[0], e[1]);
+    d.two(table, e[2], e[3]);
+  }
+};
+template <int CODE>
+struct LaneDecoder<CODE, 2> {
+  StreamDecoder<CODE> d0, d1;
+  __device__ __forceinline__ void init(uint32_t area, const uint32_t (&start)[2], uint32_t limit,
+                                       uint32_t table) {
+    d0.init(area, start[0], limit, table);
+    d1.init(area, start[1], limit, table);
+  }
+  __device__ __forceinline__ void quad(uint32_t table, uint32_t (&e)[4]) {
+    d0.two(table, e[0], e[2]);
+    d1.two(table, e[1], e[3]);
+  }
+};
 
 // ---- shared-memory layout and the producer ---------------------------------
 //
@@ -515,14 +647,18 @@ __device__ __forceinline__ uint2 load_x4(const uint16_t* xrow, int64_t cols, int
 // the tile's contribution and d[2..3] the same for batch g + 8.  Each block's
 // x is read one block ahead: from shared memory (XSM: xs = the staged row 0 at
 // the tile's first column, rows xrow bytes apart) or else through L1.
-template <int CP, bool WIDE, bool FAST, bool XSM>
+template <int CP, bool WIDE, int CODE, int S, bool XSM>
 __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table, uint32_t limit,
                                                  int lane, float (&d)[4], const TileParams& p,
                                                  int64_t col_tile, bool xvec, uint32_t xs,
                                                  uint32_t xrow) {
   constexpr int kRaw = CP * 512;
-  StreamDecoder<FAST> dec;
-  dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
+  LaneDecoder<CODE, S> dec;
+  {
+    uint32_t start[S];
+    lane_stream_starts<S>(chunk, kRaw, lane, start);
+    dec.init(chunk + kRaw + kLanes * S, start, limit, table);
+  }
   const int g = lane >> 2, c = lane & 3;
   const int64_t cols = p.cols;
   // Rows past the batch read row 0 (see x_at).
@@ -545,19 +681,23 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
   for (int m = 0; m < CP; ++m) {
     const uint4 rv = lds128(chunk + m * 512 + lane * 16);
 #pragma unroll
-    for (int s = 0; s < 4; ++s) {
-      const uint2 xa_s = xa, xb_s = xb;
-      // Next block's x: + 4 columns, or the next group's first block.
-      const uint32_t no = s < 3 ? 64 * m + 4 * (s + 1) : 64 * (m + 1);
-      if (s < 3 || m + 1 < CP) {
-        xa = x_at(xr0, xs0, no);
-        if (WIDE) xb = x_at(xr1, xs1, no);
+    for (int s2 = 0; s2 < 4; s2 += 2) {
+      uint32_t e[4];
+      dec.quad(table, e);  // pairs 2 s2 .. 2 s2 + 3: blocks s2 and s2 + 1
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int s = s2 + h;
+        const uint2 xa_s = xa, xb_s = xb;
+        // Next block's x: + 4 columns, or the next group's first block.
+        const uint32_t no = s < 3 ? 64 * m + 4 * (s + 1) : 64 * (m + 1);
+        if (s < 3 || m + 1 < CP) {
+          xa = x_at(xr0, xs0, no);
+          if (WIDE) xb = x_at(xr1, xs1, no);
+        }
+        const uint32_t w0 = assemble<CODE>(raw_pair_r(rv, 2 * s), e[2 * h]);
+        const uint32_t w1 = assemble<CODE>(raw_pair_r(rv, 2 * s + 1), e[2 * h + 1]);
+        mma_bf16_16816(d, xa_s.x, WIDE ? xb_s.x : 0u, xa_s.y, WIDE ? xb_s.y : 0u, w0, w1);
       }
-      uint32_t e0, e1;
-      dec.two(table, e0, e1);
-      const uint32_t w0 = assemble(raw_pair_r(rv, 2 * s), e0);
-      const uint32_t w1 = assemble(raw_pair_r(rv, 2 * s + 1), e1);
-      mma_bf16_16816(d, xa_s.x, WIDE ? xb_s.x : 0u, xa_s.y, WIDE ? xb_s.y : 0u, w0, w1);
     }
   }
 }
@@ -618,7 +758,7 @@ struct TilePos {
 // y[b][n] for up to 8 (16 when WIDE) rows b of x.  Consumer warp w takes
 // tiles w, w + NC, ...; each tile's partial sums go straight to y (one column
 // block) or to the workspace, reduced after all tiles in a fixed order.
-template <int NC, int CP, bool WIDE, bool FAST>
+template <int NC, int CP, bool WIDE, int CODE, int S>
 __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem s = carve(smem, p);
@@ -688,11 +828,12 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
     const int64_t i = pos.i, j = pos.j;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     if (xsmem)
-      decode_gemv_tile<CP, WIDE, FAST, true>(chunk, table, limit, lane, d, p, j * kTileCols, xvec,
-                                             xst + (uint32_t)((j - j0) * kTileCols * 2), xrow);
+      decode_gemv_tile<CP, WIDE, CODE, S, true>(chunk, table, limit, lane, d, p, j * kTileCols,
+                                                xvec, xst + (uint32_t)((j - j0) * kTileCols * 2),
+                                                xrow);
     else
-      decode_gemv_tile<CP, WIDE, FAST, false>(chunk, table, limit, lane, d, p, j * kTileCols, xvec,
-                                              0u, 0u);
+      decode_gemv_tile<CP, WIDE, CODE, S, false>(chunk, table, limit, lane, d, p, j * kTileCols,
+                                                 xvec, 0u, 0u);
     __syncwarp();
     if (lane == 0) mbar_arrive(&s.empty[k % kSlots]);  // release the tile's share of the batch
     // Lane (g, c) holds rows 2c, 2c + 1 of the tile for batch rows g and g + 8.
@@ -752,7 +893,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) gemv_kernel(TileParams p) {
   }
 }
 
-template <int NC, int CP, bool FAST>
+template <int NC, int CP, int CODE, int S>
 __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const Smem s = carve(smem, p);
@@ -782,8 +923,12 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     if (q + NC < n) at_next = __ldg(tile_ring + q + NC);
     if (!wait_batch(s, k, wc)) return;
     const int64_t i = pos.i, j = pos.j;
-    StreamDecoder<FAST> dec;
-    dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
+    LaneDecoder<CODE, S> dec;
+    {
+      uint32_t start[S];
+      lane_stream_starts<S>(chunk, kRaw, lane, start);
+      dec.init(chunk + kRaw + kLanes * S, start, limit, table);
+    }
     // Lane L owns row L / 4 of the tile and 16 consecutive columns per group.
     const int64_t row = i * 8 + (lane >> 2);
     const bool row_in = row < p.rows;
@@ -794,12 +939,14 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
       const int64_t col = j * (CP * 64) + g * 64 + 16 * (lane & 3);
       uint32_t wv[8];
 #pragma unroll
-      for (int r = 0; r < 8; r += 2) {
-        uint32_t e0, e1;
-        dec.two(table, e0, e1);
-        invalid |= e0 | e1;
-        wv[r] = assemble(raw_pair_r(rv, r), e0);
-        wv[r + 1] = assemble(raw_pair_r(rv, r + 1), e1);
+      for (int r = 0; r < 8; r += 4) {
+        uint32_t e[4];
+        dec.quad(table, e);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          invalid |= e[k];
+          wv[r + k] = assemble<CODE>(raw_pair_r(rv, r + k), e[k]);
+        }
       }
       if (row_in && vec && col + 16 <= cols) {
         uint4* dst = reinterpret_cast<uint4*>(orow + col);
@@ -832,7 +979,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
 // requested rows are read.
 constexpr int kGatherWarps = 8;
 
-template <int CP, bool FAST>
+template <int CP, int CODE, int S>
 __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams p) {
   extern __shared__ __align__(16) uint8_t gsm[];
   constexpr int kRaw = CP * 512;
@@ -867,10 +1014,11 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
       for (uint32_t o = 16 * lane; o < bytes; o += 16 * 32)
         *reinterpret_cast<uint4*>(stage + o) = __ldg(reinterpret_cast<const uint4*>(chunk + kRaw + o));
       __syncwarp();
-      const uint32_t start = lane_stream_start(sbase, 0, lane);
+      uint32_t start[S];
+      lane_stream_starts<S>(sbase, 0, lane, start);
       if (g != row % kTileRows) continue;
-      StreamDecoder<FAST> dec;
-      dec.init(sbase + kLanes, start, limit);
+      LaneDecoder<CODE, S> dec;
+      dec.init(sbase + kLanes * S, start, limit, table);
       uint4 rv = __ldg(reinterpret_cast<const uint4*>(chunk + lane * 16));
 #pragma unroll 1
       for (int m = 0; m < CP; ++m) {
@@ -878,12 +1026,14 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
         if (m + 1 < CP) rv = __ldg(reinterpret_cast<const uint4*>(chunk + (m + 1) * 512 + lane * 16));
         uint32_t wv[8];
 #pragma unroll
-        for (int r = 0; r < 8; r += 2) {
-          uint32_t e0, e1;
-          dec.two(table, e0, e1);
-          invalid |= e0 | e1;
-          wv[r] = assemble(raw_pair_r(cur, r), e0);
-          wv[r + 1] = assemble(raw_pair_r(cur, r + 1), e1);
+        for (int r = 0; r < 8; r += 4) {
+          uint32_t e[4];
+          dec.quad(table, e);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            invalid |= e[k];
+            wv[r + k] = assemble<CODE>(raw_pair_r(cur, r + k), e[k]);
+          }
         }
         const int64_t col = j * (CP * 64) + m * 64 + 16 * c;
         if (vec && col + 16 <= p.cols) {
@@ -1146,7 +1296,7 @@ __device__ void tc_boundary(const TileParams& p, int64_t i, int lane) {
 }
 
 // Decode warps (0 .. 15): warp w < teams R is slot r = w % R of team t = w / R.
-template <int CP, bool FAST>
+template <int CP, int CODE, int S>
 __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, const TcBars& tb,
                           const TcWork& wk, int warp, int lane) {
   constexpr int kRaw = CP * 512;
@@ -1172,7 +1322,7 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
       const int64_t j = t + jj * TT;
       const int64_t v = i * p.tiles_c + j;
       const bool present = r < rg && v >= wk.a && v < wk.b;
-      StreamDecoder<FAST> dec;
+      LaneDecoder<CODE, S> dec;
       uint32_t chunk = 0, bw = 0;
       if (present) {
         const int64_t u = j * p.tiles_r + i;
@@ -1182,7 +1332,9 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
           ok = false;
           break;
         }
-        dec.init(chunk + kRaw + kLanes, lane_stream_start(chunk, kRaw, lane), limit);
+        uint32_t start[S];
+        lane_stream_starts<S>(chunk, kRaw, lane, start);
+        dec.init(chunk + kRaw + kLanes * S, start, limit, table);
       }
       for (int m = 0; m < CP; ++m, ++seq) {
         const uint32_t st = seq & 1u, use = seq >> 1;
@@ -1198,11 +1350,11 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
           const uint4 rv = lds128(chunk + m * 512 + lane * 16);
           uint32_t wv[8];
 #pragma unroll
-          for (int k = 0; k < 8; k += 2) {
-            uint32_t e0, e1;
-            dec.two(table, e0, e1);
-            wv[k] = assemble(raw_pair_r(rv, k), e0);
-            wv[k + 1] = assemble(raw_pair_r(rv, k + 1), e1);
+          for (int k = 0; k < 8; k += 4) {
+            uint32_t e[4];
+            dec.quad(table, e);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) wv[k + q] = assemble<CODE>(raw_pair_r(rv, k + q), e[q]);
           }
           sts128(arow + chunk_lo, wv[0], wv[1], wv[2], wv[3]);
           sts128(arow + chunk_hi, wv[4], wv[5], wv[6], wv[7]);
@@ -1267,48 +1419,61 @@ __device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* sm
   const uint32_t a_area = smem_u32(smem + p.tc_a_off), b_area = smem_u32(smem + p.tc_b_off);
   const uint32_t idesc = umma_idesc_bf16(128, N);
   const uint32_t tmem = *tb.tmem;
-  uint32_t nx[kTcMaxTeams], nm[kTcMaxTeams], per_group[kTcMaxTeams], total[kTcMaxTeams];
-  for (int t = 0; t < TT; ++t) {
-    per_group[t] = (uint32_t)((p.tiles_c - t + TT - 1) / TT) * CP;
+  // Per team, in registers (the team loops are unrolled to kTcMaxTeams):
+  // chunks whose x was fetched (nx) and that were multiplied (nm), out of
+  // total; the within-group index of the next chunk to fetch (xw) and to
+  // multiply (mw), and the group of the latter (mg).  No divisions: CP is a
+  // power of two and the indices advance by one.
+  uint32_t nx[kTcMaxTeams], nm[kTcMaxTeams], total[kTcMaxTeams], per_group[kTcMaxTeams];
+  uint32_t xw[kTcMaxTeams], mw[kTcMaxTeams], mg[kTcMaxTeams];
+#pragma unroll
+  for (int t = 0; t < kTcMaxTeams; ++t) {
+    per_group[t] = t < TT ? (uint32_t)((p.tiles_c - t + TT - 1) / TT) * CP : 0u;
     total[t] = (uint32_t)wk.groups * per_group[t];
-    nx[t] = nm[t] = 0;
+    nx[t] = nm[t] = xw[t] = mw[t] = mg[t] = 0;
   }
   wait_prerequisites();  // x may be written by the previous kernel on the stream
   uint32_t idle = 0;
   for (;;) {
     bool done = true, moved = false;
-    for (int t = 0; t < TT; ++t) {
+#pragma unroll
+    for (int t = 0; t < kTcMaxTeams; ++t) {
       if (nm[t] >= total[t]) continue;
       done = false;
       // x of chunk nx[t]: its stage is free once the MMAs two chunks back are done.
       if (nx[t] < total[t] && nx[t] < nm[t] + 2) {
         const uint32_t sx = nx[t] & 1u, use = nx[t] >> 1;
         if (use == 0 || mbar_test_wait(&tb.sempty[2 * t + sx], (use - 1) & 1u)) {
-          const uint32_t within = nx[t] % per_group[t];
-          const int64_t j = t + (int64_t)(within / CP) * TT;
-          const int m = (int)(within % CP);
+          const int64_t j = t + (int64_t)(xw[t] / CP) * TT;
+          const int m = (int)(xw[t] % CP);
           mbar_expect_tx(&tb.xfull[2 * t + sx], (uint32_t)N * 128u);
           tma_load_2d(b_area + (uint32_t)(2 * t + (int)sx) * kTcStageB, tmap,
                       (int32_t)(j * CP * 64 + m * 64), 0, &tb.xfull[2 * t + sx]);
           ++nx[t];
+          xw[t] = xw[t] + 1 == per_group[t] ? 0u : xw[t] + 1;
           moved = true;
         }
       }
       // MMAs of chunk nm[t].
       if (nm[t] < nx[t]) {
         const uint32_t sm = nm[t] & 1u, ph = (nm[t] >> 1) & 1u;
-        const uint32_t within = nm[t] % per_group[t], gi = nm[t] / per_group[t];
         if (mbar_test_wait(&tb.xfull[2 * t + sm], ph) && mbar_test_wait(&tb.sfull[2 * t + sm], ph) &&
-            (within != 0 || gi == 0 || mbar_test_wait(tb.accempty, (gi - 1) & 1u))) {
+            (mw[t] != 0 || mg[t] == 0 || mbar_test_wait(tb.accempty, (mg[t] - 1) & 1u))) {
           tc_fence_after();
           const uint32_t a0 = a_area + (uint32_t)(2 * t + (int)sm) * (uint32_t)R * kTcStageA;
           const uint32_t b0 = b_area + (uint32_t)(2 * t + (int)sm) * kTcStageB;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_bf16(tmem + (uint32_t)(t * N), umma_desc_sw128(a0 + 32u * k),
-                      umma_desc_sw128(b0 + 32u * k), idesc, (within == 0 && k == 0) ? 0u : 1u);
+                      umma_desc_sw128(b0 + 32u * k), idesc, (mw[t] == 0 && k == 0) ? 0u : 1u);
           umma_commit(&tb.sempty[2 * t + sm]);
-          if (within + 1 == per_group[t]) umma_commit(&tb.accfull[t]);
+          if (mw[t] + 1 == per_group[t]) {
+            umma_commit(&tb.accfull[t]);
+            mw[t] = 0;
+            ++mg[t];
+          } else {
+            ++mw[t];
+          }
           ++nm[t];
           moved = true;
         }
@@ -1325,7 +1490,8 @@ __device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* sm
   }
   // Leave nothing in flight: x loads issued but not consumed, and the MMAs.
   const WaitCtl dc = drain_ctl(p);
-  for (int t = 0; t < TT; ++t) {
+#pragma unroll
+  for (int t = 0; t < kTcMaxTeams; ++t) {
     for (uint32_t k = nm[t]; k < nx[t]; ++k)
       wait_bounded(&tb.xfull[2 * t + (int)(k & 1u)], (k >> 1) & 1u, dc);
     if (nm[t] > 0)
@@ -1337,7 +1503,7 @@ __device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* sm
 // Warps 0..15 decode into the A stages and read the accumulators back, warp 16
 // allocates TMEM and issues x loads and MMAs, warp 17 moves the compressed
 // tiles into the ring (the same producer as the other kernels).
-template <int CP, bool FAST>
+template <int CP, int CODE, int S>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemv_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap) {
   extern __shared__ __align__(1024) uint8_t smem_tc[];
@@ -1386,7 +1552,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     wait_prerequisites();  // y and the scratch may belong to the previous kernel
     const WaitCtl wc = wait_ctl(p);
     if (wait_table(s, wc)) {
-      tc_decode<CP, FAST>(p, smem, s, tb, wk, warp, lane);
+      tc_decode<CP, CODE, S>(p, smem, s, tb, wk, warp, lane);
     } else if (lane == 0) {
       *tb.abort = 1u;
     }
@@ -1444,26 +1610,37 @@ cudaError_t launch_pdl(Kernel k, const LaunchShape& s, cudaStream_t stream, cons
 }
 
 
-template <int CP, bool WIDE, bool FAST>
+template <int CP, bool WIDE, int CODE, int S>
 cudaError_t launch_gemv_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(gemv_kernel<kConsumers, CP, WIDE, FAST>, s.smem_bytes, configured);
+  cudaError_t e =
+      ensure_smem(gemv_kernel<kConsumers, CP, WIDE, CODE, S>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  return launch_pdl(gemv_kernel<kConsumers, CP, WIDE, FAST>, s, stream, p);
+  return launch_pdl(gemv_kernel<kConsumers, CP, WIDE, CODE, S>, s, stream, p);
 }
 
-template <int CP, bool FAST>
-cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+template <int CP, int CODE, int S>
+cudaError_t launch_gemv_s(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   if (p.batch < 1 || p.batch > kMaxPassRows) return cudaErrorInvalidValue;
-  return p.batch <= 8 ? launch_gemv_t<CP, false, FAST>(p, s, stream)
-                      : launch_gemv_t<CP, true, FAST>(p, s, stream);
+  return p.batch <= 8 ? launch_gemv_t<CP, false, CODE, S>(p, s, stream)
+                      : launch_gemv_t<CP, true, CODE, S>(p, s, stream);
 }
 
-template <int CP, bool FAST>
-cudaError_t launch_gemv_tc_t(const TileParams& p, const CUtensorMap& tmap, const LaunchShape& s,
+template <int CP, int CODE>
+cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+  if constexpr (CODE == kCodeRank) {
+    return launch_gemv_s<CP, CODE, 1>(p, s, stream);
+  } else {
+    return p.streams == 2 ? launch_gemv_s<CP, CODE, 2>(p, s, stream)
+                          : launch_gemv_s<CP, CODE, 1>(p, s, stream);
+  }
+}
+
+template <int CP, int CODE, int S>
+cudaError_t launch_gemv_tc_s(const TileParams& p, const CUtensorMap& tmap, const LaunchShape& s,
                              cudaStream_t stream) {
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(gemv_tc_kernel<CP, FAST>, s.smem_bytes, configured);
+  cudaError_t e = ensure_smem(gemv_tc_kernel<CP, CODE, S>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)s.ctas);
@@ -1475,15 +1652,37 @@ cudaError_t launch_gemv_tc_t(const TileParams& p, const CUtensorMap& tmap, const
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<CP, FAST>, p, tmap);
+  return cudaLaunchKernelEx(&cfg, gemv_tc_kernel<CP, CODE, S>, p, tmap);
 }
 
-template <int CP, bool FAST>
-cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+template <int CP, int CODE>
+cudaError_t launch_gemv_tc_t(const TileParams& p, const CUtensorMap& tmap, const LaunchShape& s,
+                             cudaStream_t stream) {
+  if constexpr (CODE == kCodeRank) {
+    return launch_gemv_tc_s<CP, CODE, 1>(p, tmap, s, stream);
+  } else {
+    return p.streams == 2 ? launch_gemv_tc_s<CP, CODE, 2>(p, tmap, s, stream)
+                          : launch_gemv_tc_s<CP, CODE, 1>(p, tmap, s, stream);
+  }
+}
+
+template <int CP, int CODE, int S>
+cudaError_t launch_decompress_s(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(decompress_kernel<kConsumers, CP, FAST>, s.smem_bytes, configured);
+  cudaError_t e =
+      ensure_smem(decompress_kernel<kConsumers, CP, CODE, S>, s.smem_bytes, configured);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decompress_kernel<kConsumers, CP, FAST>, s, stream, p);
+  return launch_pdl(decompress_kernel<kConsumers, CP, CODE, S>, s, stream, p);
+}
+
+template <int CP, int CODE>
+cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
+  if constexpr (CODE == kCodeRank) {
+    return launch_decompress_s<CP, CODE, 1>(p, s, stream);
+  } else {
+    return p.streams == 2 ? launch_decompress_s<CP, CODE, 2>(p, s, stream)
+                          : launch_decompress_s<CP, CODE, 1>(p, s, stream);
+  }
 }
 
 }  // namespace
@@ -1522,24 +1721,24 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
   return s;
 }
 
-cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const LaunchShape& s,
+cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const LaunchShape& s,
                         cudaStream_t stream) {
   switch (tile_cols) {
-    case 512: return fast ? launch_gemv_cp<8, true>(p, s, stream) : launch_gemv_cp<8, false>(p, s, stream);
-    case 256: return fast ? launch_gemv_cp<4, true>(p, s, stream) : launch_gemv_cp<4, false>(p, s, stream);
-    case 128: return fast ? launch_gemv_cp<2, true>(p, s, stream) : launch_gemv_cp<2, false>(p, s, stream);
-    case 64: return fast ? launch_gemv_cp<1, true>(p, s, stream) : launch_gemv_cp<1, false>(p, s, stream);
+    case 512: return code == kCodeRank ? launch_gemv_cp<8, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<8, kCode14>(p, s, stream) : launch_gemv_cp<8, kCode12>(p, s, stream);
+    case 256: return code == kCodeRank ? launch_gemv_cp<4, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<4, kCode14>(p, s, stream) : launch_gemv_cp<4, kCode12>(p, s, stream);
+    case 128: return code == kCodeRank ? launch_gemv_cp<2, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<2, kCode14>(p, s, stream) : launch_gemv_cp<2, kCode12>(p, s, stream);
+    case 64: return code == kCodeRank ? launch_gemv_cp<1, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<1, kCode14>(p, s, stream) : launch_gemv_cp<1, kCode12>(p, s, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
+cudaError_t launch_decompress(const TileParams& p, int tile_cols, int code,
                               const LaunchShape& s, cudaStream_t stream) {
   switch (tile_cols) {
-    case 512: return fast ? launch_decompress_t<8, true>(p, s, stream) : launch_decompress_t<8, false>(p, s, stream);
-    case 256: return fast ? launch_decompress_t<4, true>(p, s, stream) : launch_decompress_t<4, false>(p, s, stream);
-    case 128: return fast ? launch_decompress_t<2, true>(p, s, stream) : launch_decompress_t<2, false>(p, s, stream);
-    case 64: return fast ? launch_decompress_t<1, true>(p, s, stream) : launch_decompress_t<1, false>(p, s, stream);
+    case 512: return code == kCodeRank ? launch_decompress_t<8, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<8, kCode14>(p, s, stream) : launch_decompress_t<8, kCode12>(p, s, stream);
+    case 256: return code == kCodeRank ? launch_decompress_t<4, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<4, kCode14>(p, s, stream) : launch_decompress_t<4, kCode12>(p, s, stream);
+    case 128: return code == kCodeRank ? launch_decompress_t<2, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<2, kCode14>(p, s, stream) : launch_decompress_t<2, kCode12>(p, s, stream);
+    case 64: return code == kCodeRank ? launch_decompress_t<1, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<1, kCode14>(p, s, stream) : launch_decompress_t<1, kCode12>(p, s, stream);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1610,27 +1809,37 @@ bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_chunk, uint64_t typ
   return found;
 }
 
-cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols, bool fast,
+cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols, int code,
                            const TcShape& s, cudaStream_t stream) {
   if (p.batch < 1 || p.batch > kMaxTcRows || p.tc_teams < 1 || p.tc_teams > kTcMaxTeams ||
       p.tc_rows < 1 || p.tc_rows * p.tc_teams > kTcDecodeWarps)
     return cudaErrorInvalidValue;
   switch (tile_cols) {
-    case 512: return fast ? launch_gemv_tc_t<8, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<8, false>(p, tmap, s.s, stream);
-    case 256: return fast ? launch_gemv_tc_t<4, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<4, false>(p, tmap, s.s, stream);
-    case 128: return fast ? launch_gemv_tc_t<2, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<2, false>(p, tmap, s.s, stream);
-    case 64: return fast ? launch_gemv_tc_t<1, true>(p, tmap, s.s, stream) : launch_gemv_tc_t<1, false>(p, tmap, s.s, stream);
+    case 512: return code == kCodeRank ? launch_gemv_tc_t<8, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<8, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<8, kCode12>(p, tmap, s.s, stream);
+    case 256: return code == kCodeRank ? launch_gemv_tc_t<4, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<4, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<4, kCode12>(p, tmap, s.s, stream);
+    case 128: return code == kCodeRank ? launch_gemv_tc_t<2, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<2, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<2, kCode12>(p, tmap, s.s, stream);
+    case 64: return code == kCodeRank ? launch_gemv_tc_t<1, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<1, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<1, kCode12>(p, tmap, s.s, stream);
     default: return cudaErrorInvalidValue;
   }
 }
 
-template <int CP, bool FAST>
-cudaError_t launch_gather_t(const GatherParams& g, int ctas, size_t smem, cudaStream_t stream) {
+template <int CP, int CODE, int S>
+cudaError_t launch_gather_s(const GatherParams& g, int ctas, size_t smem, cudaStream_t stream) {
   static int configured[64] = {};
-  cudaError_t e = ensure_smem(gather_kernel<CP, FAST>, smem, configured);
+  cudaError_t e = ensure_smem(gather_kernel<CP, CODE, S>, smem, configured);
   if (e != cudaSuccess) return e;
-  gather_kernel<CP, FAST><<<(unsigned)ctas, kGatherWarps * 32, smem, stream>>>(g);
+  gather_kernel<CP, CODE, S><<<(unsigned)ctas, kGatherWarps * 32, smem, stream>>>(g);
   return cudaGetLastError();
+}
+
+template <int CP, int CODE>
+cudaError_t launch_gather_t(const GatherParams& g, int ctas, size_t smem, cudaStream_t stream) {
+  if constexpr (CODE == kCodeRank) {
+    return launch_gather_s<CP, CODE, 1>(g, ctas, smem, stream);
+  } else {
+    return g.streams == 2 ? launch_gather_s<CP, CODE, 2>(g, ctas, smem, stream)
+                          : launch_gather_s<CP, CODE, 1>(g, ctas, smem, stream);
+  }
 }
 
 cudaError_t launch_gather(const GatherParams& g, int sm_count, cudaStream_t stream) {
@@ -1638,12 +1847,12 @@ cudaError_t launch_gather(const GatherParams& g, int sm_count, cudaStream_t stre
   const int64_t want = 2 * (int64_t)(sm_count > 0 ? sm_count : 1);
   const int ctas = (int)(g.n < want ? g.n : want);
   const size_t smem = (size_t)g.table_bytes + (size_t)kGatherWarps * g.stage_bytes;
-  const bool fast = g.peek == 14;
+  const int code = g.code;
   switch (g.tile_cols) {
-    case 512: return fast ? launch_gather_t<8, true>(g, ctas, smem, stream) : launch_gather_t<8, false>(g, ctas, smem, stream);
-    case 256: return fast ? launch_gather_t<4, true>(g, ctas, smem, stream) : launch_gather_t<4, false>(g, ctas, smem, stream);
-    case 128: return fast ? launch_gather_t<2, true>(g, ctas, smem, stream) : launch_gather_t<2, false>(g, ctas, smem, stream);
-    case 64: return fast ? launch_gather_t<1, true>(g, ctas, smem, stream) : launch_gather_t<1, false>(g, ctas, smem, stream);
+    case 512: return code == kCodeRank ? launch_gather_t<8, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<8, kCode14>(g, ctas, smem, stream) : launch_gather_t<8, kCode12>(g, ctas, smem, stream);
+    case 256: return code == kCodeRank ? launch_gather_t<4, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<4, kCode14>(g, ctas, smem, stream) : launch_gather_t<4, kCode12>(g, ctas, smem, stream);
+    case 128: return code == kCodeRank ? launch_gather_t<2, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<2, kCode14>(g, ctas, smem, stream) : launch_gather_t<2, kCode12>(g, ctas, smem, stream);
+    case 64: return code == kCodeRank ? launch_gather_t<1, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<1, kCode14>(g, ctas, smem, stream) : launch_gather_t<1, kCode12>(g, ctas, smem, stream);
     default: return cudaErrorInvalidValue;
   }
 }

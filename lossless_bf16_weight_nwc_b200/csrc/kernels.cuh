@@ -26,6 +26,10 @@ constexpr uint32_t kErrLayout = 8u;    // shared memory not aligned as a kernel 
 // 0 means this).
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 
+// The exponent code a kernel reads: the prefix code through a 12-bit or a
+// 14-bit table peek, or the ranked unary code (variant NWR1, no table).
+constexpr int kCode12 = 0, kCode14 = 1, kCodeRank = 2;
+
 struct TileParams {
   const uint8_t* tiles;     // device: tile area of the blob
   const uint32_t* sched_cta;   // device: first batch of each CTA, ctas + 1
@@ -50,6 +54,7 @@ struct TileParams {
   uint16_t* out;            // BF16 [rows x cols]
   uint32_t* err;            // device: the handle's error word
   uint32_t wait_limit;      // polls before a bounded wait gives up (0: default)
+  int32_t streams;          // bit streams per lane and tile (1 or 2)
   // tensor-core kernel
   const uint32_t* tile_batch;  // device: per tile, its batch | extra releases << 28
   int32_t tc_rows;          // R: row tiles per M-group (rows of the MMA / 8)
@@ -93,8 +98,9 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
 // sched_class_bytes(n_tiles) bytes (one class) laid out as nwc_format.h describes.
 void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s, uint8_t* out);
 
-// fast: lmax <= 7 (14-bit peek, two codes per entry always).
-cudaError_t launch_gemv(const TileParams& p, int tile_cols, bool fast, const LaunchShape& s,
+// code: kCode12, kCode14 (lmax <= 7: two codes per table entry always) or
+// kCodeRank.
+cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const LaunchShape& s,
                         cudaStream_t stream);
 
 // ---- tensor-core (tcgen05) GEMV: decode once, multiply every row of x -----
@@ -136,8 +142,8 @@ void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c, 
 // tmap: the TMA descriptor of x (BF16 [rows of x][cols], box 64 columns x
 // tc_n rows, 128-byte swizzle).
 cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols,
-                           bool fast, const TcShape& s, cudaStream_t stream);
-cudaError_t launch_decompress(const TileParams& p, int tile_cols, bool fast,
+                           int code, const TcShape& s, cudaStream_t stream);
+cudaError_t launch_decompress(const TileParams& p, int tile_cols, int code,
                               const LaunchShape& s, cudaStream_t stream);
 // Row gather (embedding lookup) from the compressed matrix.
 struct GatherParams {
@@ -146,6 +152,8 @@ struct GatherParams {
   const uint32_t* table;    // device: decode table
   uint32_t table_bytes;
   uint32_t stage_bytes;     // per warp: a tile's lane lengths and streams + slack
+  int32_t streams;          // bit streams per lane and tile (1 or 2)
+  int32_t code;             // kCode12, kCode14 or kCodeRank
   int32_t peek;             // table peek width (12 or 14)
   int32_t tile_cols;
   int64_t rows, cols, tiles_r, tiles_c;

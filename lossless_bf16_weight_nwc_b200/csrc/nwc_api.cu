@@ -53,11 +53,19 @@ nwc_status current_device(int* dev, int* sms, size_t* smem) {
   return NWC_OK;
 }
 
+// The code kind the kernels read for a handle, and the table bytes a CTA loads.
+int code_of(const nwc_handle_s& h) {
+  return h.code_kind == 1 ? nwc::kCodeRank : h.lmax <= 7 ? nwc::kCode14 : nwc::kCode12;
+}
+uint32_t table_bytes_of(const nwc_handle_s& h) {
+  return nwc::device_table_bytes(h.lmax, h.code_kind == 1);
+}
+
 // Launch geometry for a handle and x-stage class on a device with `sms` SMs
 // and `smem` bytes of opt-in shared memory per block.
 nwc_status shape_on(const nwc_handle_s& h, int sms, size_t smem, int cls, nwc::LaunchShape* s) {
   const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
-  *s = nwc::launch_shape(h.tiles, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms, smem,
+  *s = nwc::launch_shape(h.tiles, h.max_chunk, typical, table_bytes_of(h), sms, smem,
                          nwc::kXStageBytes[cls]);
   if (s->smem_bytes > smem) return NWC_ERR_UNSUPPORTED;
   return NWC_OK;
@@ -104,8 +112,8 @@ uint64_t tc_class_off(const nwc_handle_s& h) {
 // bytes of opt-in shared memory per block; false when it does not fit.
 bool tc_shape_on(const nwc_handle_s& h, int sms, size_t smem, nwc::TcShape* ts) {
   const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
-  return nwc::tc_shape(h.tiles_r, h.tiles_c, h.max_chunk, typical, nwc::table_bytes(h.lmax), sms,
-                       smem, ts);
+  return nwc::tc_shape(h.tiles_r, h.tiles_c, h.max_chunk, typical, table_bytes_of(h), sms, smem,
+                       ts);
 }
 
 bool same_tc_shape(const nwc_handle_s& h, const nwc::TcShape& t) {
@@ -166,14 +174,13 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // no C++ exception leaves the C ABI.
 nwc_status parse(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* h,
                  const uint8_t** lens) {
-  // Well-defined layouts that no kernel reads yet: an NWR1 blob (ranked unary
-  // code), and NWB1 with 2 or 4 bit streams per lane (header offset 60 = S - 1).
+  // A well-defined layout that no kernel reads: NWB1 with 4 bit streams per
+  // lane (header offset 60 = S - 1).
   if (blob && head_bytes >= 64) {
     uint32_t magic, streams_m1;
     std::memcpy(&magic, blob, 4);
     std::memcpy(&streams_m1, blob + 60, 4);
-    if (magic == nwc::kRankMagic) return NWC_ERR_UNSUPPORTED;
-    if (magic == nwc::kMagic && (streams_m1 == 1 || streams_m1 == 3)) return NWC_ERR_UNSUPPORTED;
+    if (magic == nwc::kMagic && streams_m1 == 3) return NWC_ERR_UNSUPPORTED;
   }
   try {
     return nwc::parse_blob(blob, head_bytes, bytes, h, lens) ? NWC_OK : NWC_ERR_CORRUPT;
@@ -195,7 +202,7 @@ nwc::TileParams base_params(const nwc_handle_s& h, int cls, const nwc::LaunchSha
   p.sched_batch = reinterpret_cast<const uint4*>(sched + nwc::sched_batch_off());
   p.tile_ring = reinterpret_cast<const uint32_t*>(sched + nwc::sched_tile_off((uint64_t)h.tiles));
   p.table = reinterpret_cast<const uint32_t*>(h.d_base + h.table_off);
-  p.table_bytes = nwc::table_bytes(h.lmax);
+  p.table_bytes = table_bytes_of(h);
   p.rows = h.rows;
   p.cols = h.cols;
   p.tiles_r = h.tiles_r;
@@ -208,6 +215,7 @@ nwc::TileParams base_params(const nwc_handle_s& h, int cls, const nwc::LaunchSha
   p.xstage_bytes = s.xstage_bytes;
   p.err = error_word(h);
   p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  p.streams = (int32_t)h.streams;
   return p;
 }
 
@@ -359,7 +367,8 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
   if (!plan || !w_host || !d_buf || !out_handle) return NWC_ERR_INVALID_ARG;
   *out_handle = nullptr;
   // No kernel reads these layouts yet.
-  if (plan->code_kind != NWC_CODE_PREFIX || plan->streams != 1) return NWC_ERR_UNSUPPORTED;
+  if (plan->streams > nwc::kMaxDeviceStreams || plan->device_bytes == 0)
+    return NWC_ERR_UNSUPPORTED;
   if (d_bytes < plan->device_bytes || !aligned(d_buf, 256)) return NWC_ERR_INVALID_ARG;
   uint8_t* img = static_cast<uint8_t*>(std::malloc(
       plan->scratch_off + nwc::scratch_partial_off((uint64_t)plan->tiles_r)));
@@ -371,8 +380,14 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf, ui
     return NWC_ERR_NOMEM;
   }
   std::memset(img + plan->blob_bytes, 0, plan->table_off - plan->blob_bytes);
-  nwc::build_decode_table(plan->len, plan->lmax, reinterpret_cast<uint32_t*>(img + plan->table_off));
-  const uint64_t table_end = plan->table_off + nwc::table_bytes(plan->lmax);
+  if (plan->code_kind == NWC_CODE_RANK)
+    nwc::build_rank_table(plan->rank_table, plan->ranks,
+                          reinterpret_cast<uint32_t*>(img + plan->table_off));
+  else
+    nwc::build_decode_table(plan->len, plan->lmax,
+                            reinterpret_cast<uint32_t*>(img + plan->table_off));
+  const uint64_t table_end =
+      plan->table_off + nwc::device_table_bytes(plan->lmax, plan->code_kind == NWC_CODE_RANK);
   std::memset(img + table_end, 0, plan->sched_off - table_end);
   // The scratch area starts with the error word and the arrival counters,
   // which must be zero; the partial sums are written before they are read.
@@ -417,19 +432,22 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf, u
   if (st != NWC_OK) return st;
   std::vector<uint32_t> table;
   try {
-    table.resize(nwc::table_entries(h->lmax));
+    table.resize(table_bytes_of(*h) / 4);
   } catch (const std::bad_alloc&) {
     delete h;
     return NWC_ERR_NOMEM;
   }
-  nwc::build_decode_table(lens, h->lmax, table.data());
+  if (h->code_kind == 1)
+    nwc::build_rank_table(lens, h->lmax, table.data());
+  else
+    nwc::build_decode_table(lens, h->lmax, table.data());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemcpyAsync(d_buf, blob, blob_bytes, cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess && h->table_off > blob_bytes)
     e = cudaMemsetAsync(static_cast<uint8_t*>(d_buf) + blob_bytes, 0, h->table_off - blob_bytes, s);
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(static_cast<uint8_t*>(d_buf) + h->table_off, table.data(),
-                        nwc::table_bytes(h->lmax), cudaMemcpyHostToDevice, s);
+                        table_bytes_of(*h), cudaMemcpyHostToDevice, s);
   if (e == cudaSuccess) e = clear_scratch(*h, s);
   if (e == cudaSuccess) {
     st = init_schedule(h, nullptr, s);
@@ -453,9 +471,9 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
   nwc::BlobHeader hd;
   if (cudaMemcpy(&hd, d_buf, sizeof(hd), cudaMemcpyDeviceToHost) != cudaSuccess)
     return NWC_ERR_CUDA;
-  if (hd.magic == nwc::kRankMagic) return NWC_ERR_UNSUPPORTED;  // no kernel reads it yet
-  if (hd.magic == nwc::kMagic && (hd.zero == 1 || hd.zero == 3)) return NWC_ERR_UNSUPPORTED;
-  if (hd.magic != nwc::kMagic || hd.total_bytes > d_bytes || hd.tiles_off > hd.total_bytes ||
+  if (hd.magic == nwc::kMagic && hd.zero == 3) return NWC_ERR_UNSUPPORTED;
+  if ((hd.magic != nwc::kMagic && hd.magic != nwc::kRankMagic) || hd.total_bytes > d_bytes ||
+      hd.tiles_off > hd.total_bytes ||
       hd.tiles_off < nwc::kIndexOffset)
     return NWC_ERR_CORRUPT;
   // Header, lens and index; the tile area is not read back.
@@ -494,7 +512,7 @@ nwc_status nwc_decompress(nwc_handle_t h, uint16_t* d_w_out, nwc_stream_t stream
   if (st != NWC_OK) return st;
   nwc::TileParams p = base_params(*h, 0, s);
   p.out = d_w_out;
-  return cuda_status(nwc::launch_decompress(p, (int)h->tile_cols, h->lmax <= 7, s,
+  return cuda_status(nwc::launch_decompress(p, (int)h->tile_cols, code_of(*h), s,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -513,13 +531,17 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
   g.tiles = h->d_base + h->tiles_off;
   g.index = reinterpret_cast<const uint32_t*>(h->d_base + h->index_off);
   g.table = reinterpret_cast<const uint32_t*>(h->d_base + h->table_off);
-  g.table_bytes = nwc::table_bytes(h->lmax);
+  g.table_bytes = table_bytes_of(*h);
   // Lane lengths and the longest streams a tile can hold, plus the readers'
   // slack.
-  g.stage_bytes = (uint32_t)(nwc::max_chunk_bytes(h->tile_cols, h->lmax) -
-                             nwc::raw_bytes(h->tile_cols) + 256);
+  const uint32_t max_chunk = h->code_kind == 1
+                                 ? nwc::max_rank_chunk_bytes(h->tile_cols, h->lmax)
+                                 : nwc::max_chunk_bytes(h->tile_cols, h->lmax, h->streams);
+  g.stage_bytes = max_chunk - nwc::raw_bytes(h->tile_cols) + 512;
   if ((size_t)g.table_bytes + 8ull * g.stage_bytes > smem) return NWC_ERR_UNSUPPORTED;
   g.peek = nwc::peek_bits(h->lmax);
+  g.streams = (int32_t)h->streams;
+  g.code = code_of(*h);
   g.tile_cols = (int32_t)h->tile_cols;
   g.rows = h->rows;
   g.cols = h->cols;
@@ -549,8 +571,10 @@ nwc_status gemv_check(const nwc_handle_s* h, const uint16_t* d_x, const float* d
   if (!h || !d_x || !d_y || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
   // x is read in BF16 pairs (4-byte words) unless cols is odd.
   if (!aligned(d_x, (h->cols & 1) ? 2 : 4) || !aligned(d_y, 4)) return NWC_ERR_INVALID_ARG;
-  // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0.
-  if (h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0) return NWC_ERR_UNSUPPORTED;
+  // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0
+  // (the ranked code's filler, e with raw byte 0, is always finite).
+  if (h->code_kind == 0 && h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0)
+    return NWC_ERR_UNSUPPORTED;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;
   if (dev != h->device) return NWC_ERR_INVALID_ARG;
@@ -622,7 +646,7 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
   p.tile_batch =
       reinterpret_cast<const uint32_t*>(sched + nwc::sched_tc_tbatch_off((uint64_t)h->tiles));
   p.table = reinterpret_cast<const uint32_t*>(h->d_base + h->table_off);
-  p.table_bytes = nwc::table_bytes(h->lmax);
+  p.table_bytes = table_bytes_of(*h);
   p.rows = h->rows;
   p.cols = h->cols;
   p.tiles_r = h->tiles_r;
@@ -635,6 +659,7 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
   p.xstage_bytes = ts.s.xstage_bytes;
   p.err = error_word(*h);
   p.wait_limit = g_wait_limit.load(std::memory_order_relaxed);
+  p.streams = (int32_t)h->streams;
   p.x = d_x;
   p.y = d_y;
   p.batch = batch;
@@ -649,7 +674,7 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
   p.tc_bar_off = ts.bar_off;
   p.tc_a_off = ts.a_off;
   p.tc_b_off = ts.b_off;
-  return cuda_status(nwc::launch_gemv_tc(p, tmap, (int)h->tile_cols, h->lmax <= 7, ts, cs));
+  return cuda_status(nwc::launch_gemv_tc(p, tmap, (int)h->tile_cols, code_of(*h), ts, cs));
 }
 
 // The GEMV launches, with split-K scratch at `counters` (u32 [tiles_r], zero
@@ -672,7 +697,7 @@ nwc_status gemv_run(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t ba
     p.x = d_x + (int64_t)b0 * h->cols;
     p.y = d_y + (int64_t)b0 * h->rows;
     p.batch = nb;
-    cudaError_t e = nwc::launch_gemv(p, (int)h->tile_cols, h->lmax <= 7, s, cs);
+    cudaError_t e = nwc::launch_gemv(p, (int)h->tile_cols, code_of(*h), s, cs);
     if (e != cudaSuccess) return NWC_ERR_CUDA;
   }
   return NWC_OK;

@@ -17,9 +17,10 @@
 // (k/16) * 512 + 16 t + k%16.
 // Tiles are stored column-block-major: u = j * tiles_r + i.
 // The header's u32 at offset 60 (`zero`) holds S - 1 for S bit streams per
-// lane; the kernels read S = 1 only, and the C ABI answers UNSUPPORTED for 2
-// or 4 (a layout the format defines for a decoder that follows several streams
-// per lane at once).
+// lane: a lane's symbol pairs go to its S streams in turn, the chunk's length
+// array has 32 S entries (lane-major) and the streams follow in that order.
+// The kernels read S = 1 and 2 (a decoder follows both streams of a lane at
+// once); the C ABI answers UNSUPPORTED for 4.
 //
 // Device image: blob | zero pad to 256 | decode table u32[table_entries(lmax)]
 // | zero pad to 256 | launch schedules (sched_bytes(tiles) bytes: one per
@@ -68,6 +69,13 @@ constexpr int kMaxStreams = 4;  // bit streams per lane and tile: 1, 2 or 4
 constexpr int peek_bits(uint32_t lmax) { return lmax <= 7 ? 14 : 12; }
 constexpr uint32_t table_entries(uint32_t lmax) { return 1u << peek_bits(lmax); }
 constexpr uint32_t table_bytes(uint32_t lmax) { return 4u * table_entries(lmax); }
+// The ranked unary code needs no decode table; its device image holds, in the
+// table's place, u32[4] = {ranked values 0..3 (bytes), values 4..6, R, 0},
+// padded to 256 bytes.
+constexpr uint32_t kRankTableBytes = 256;
+constexpr uint32_t device_table_bytes(uint32_t lmax, bool rank) {
+  return rank ? kRankTableBytes : table_bytes(lmax);
+}
 
 // Decode-table entry for one peek (most significant bit = next bit):
 //   bits  0..3   bits consumed by the step (both codes, or the first only)
@@ -154,9 +162,9 @@ struct ImageLayout {
   uint64_t table_off, sched_off, scratch_off, device_bytes;
 };
 constexpr ImageLayout image_layout(uint64_t blob_bytes, uint32_t lmax, uint64_t tiles_r,
-                                   uint64_t tiles_c) {
+                                   uint64_t tiles_c, bool rank = false) {
   const uint64_t table_off = round_up(blob_bytes, 256);
-  const uint64_t sched_off = round_up(table_off + table_bytes(lmax), 256);
+  const uint64_t sched_off = round_up(table_off + device_table_bytes(lmax, rank), 256);
   const uint64_t scratch_off = round_up(sched_off + sched_bytes(tiles_r * tiles_c), 256);
   return ImageLayout{table_off, sched_off, scratch_off,
                      scratch_off + scratch_bytes(tiles_r, tiles_c)};
@@ -173,11 +181,25 @@ struct BlobHeader {
 };
 static_assert(sizeof(BlobHeader) == 128, "header layout");
 
-// Bytes of one tile's raw plane and the worst-case chunk.
+// Bytes of one tile's raw plane and the worst-case chunk with S bit streams
+// per lane (each holding 16 (tile_cols / 64) / S symbols of at most lmax bits,
+// padded to a byte).
 constexpr uint32_t raw_bytes(uint32_t tile_cols) { return kTileRows * tile_cols; }
-constexpr uint32_t max_chunk_bytes(uint32_t tile_cols, uint32_t lmax) {
+constexpr uint32_t max_chunk_bytes(uint32_t tile_cols, uint32_t lmax, uint32_t streams = 1) {
+  return raw_bytes(tile_cols) + kLanes * streams +
+         (uint32_t)((kLanes * streams *
+                         ((2 * kTileRows * (tile_cols / 64) / streams * lmax + 7) / 8) +
+                     15) /
+                    16 * 16);
+}
+// Bit streams per lane that the kernels read (1 or 2).
+constexpr uint32_t kMaxDeviceStreams = 2;
+// Worst-case chunk of the ranked unary code with R ranks (one stream per
+// lane): a code has at most 1 + R + 7 bits.
+constexpr uint32_t max_rank_chunk_bytes(uint32_t tile_cols, uint32_t ranks) {
   return raw_bytes(tile_cols) + kLanes +
-         (uint32_t)((kLanes * ((2 * kTileRows * (tile_cols / 64) * lmax + 7) / 8) + 15) / 16 * 16);
+         (uint32_t)((kLanes * ((2 * kTileRows * (tile_cols / 64) * (ranks + 8) + 7) / 8) + 15) /
+                    16 * 16);
 }
 
 }  // namespace nwc

@@ -35,6 +35,8 @@ struct nwc_handle_s {
   uint64_t d_bytes = 0;
   int64_t rows = 0, cols = 0;
   uint32_t tile_cols = 512, lmax = 7, filler = 0;
+  uint32_t streams = 1;    // bit streams per lane and tile (1 or 2)
+  uint32_t code_kind = 0;  // 0: prefix code (NWB1), 1: ranked unary code (NWR1)
   int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
   uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0, sched_off = 0,
            scratch_off = 0;
@@ -69,6 +71,9 @@ bool code_lengths(const uint64_t cnt[256], uint32_t lmax, uint8_t len[256]);
 void canonical_codes(const uint8_t len[256], uint32_t code[256]);
 // Writes table_entries(lmax) entries.
 void build_decode_table(const uint8_t len[256], uint32_t lmax, uint32_t* table);
+// The device image's table area of a ranked unary code (kRankTableBytes):
+// u32[4] = {ranked values 0..3, values 4..6, R, 0}, then zeros.
+void build_rank_table(const uint8_t* ranked, uint32_t ranks, uint32_t* out);
 // Parses and checks a blob's header, lens and index (the first head_bytes of a
 // blob of `bytes` bytes; head_bytes must reach the tile area); fills the
 // handle's geometry fields.  Returns false when the blob does not follow the

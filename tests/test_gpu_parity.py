@@ -172,17 +172,25 @@ def test_fused_projections(lib, orc, batch):
 
 
 def test_autotune_picks_a_timed_candidate(lib, orc):
-    """The format autotuner times real candidates on the device; the format it
-    picks meets the tolerance."""
+    """The strategy autotuner times real candidates on the device (two formats,
+    both kernels); the strategy it picks, applied, meets the tolerance."""
     from lossless_bf16_weight_nwc_b200 import autotune
+    from lossless_bf16_weight_nwc_b200.autotune import Strategy
     spec = synth.MatrixSpec("w", 1024, 4096, "normal", 0.02, 0)
     w = synth.matrix(spec, 3)
-    choice = autotune.Tuner().tune(w, 1, candidates=[(512, 0), (256, 0)], reps=5)
-    assert (choice.tile_cols, choice.lmax) in {(512, 0), (256, 0)}
-    assert set(choice.timings) == {"512/0", "256/0"} and min(choice.timings.values()) > 0
-    m = lib.CompressedMatrix.compress(w, tile_cols=choice.tile_cols, lmax=choice.lmax)
-    x = synth.activations(3, 1, spec.cols)
-    tolerance_check(m.gemv(to_bf16(x)).cpu().numpy(), orc.gemv(w, x), w, x)
+    cands = [Strategy(512, 0, 1, "prefix", "cuda"), Strategy(512, 0, 1, "prefix", "tensor"),
+             Strategy(256, 0, 2, "prefix", "cuda"), Strategy(512, 0, 1, "rank", "tensor")]
+    choice = autotune.Tuner().tune(w, 16, candidates=cands, reps=5)
+    assert choice.strategy in cands
+    assert set(choice.timings) == {c.key for c in cands} and min(choice.timings.values()) > 0
+    s = choice.strategy
+    m = lib.CompressedMatrix.compress(w, tile_cols=s.tile_cols, lmax=s.lmax, streams=s.streams,
+                                      code=lib.NWC_CODE_RANK if s.code == "rank" else 0)
+    autotune.apply(m, s)
+    x = synth.activations(3, 16, spec.cols)
+    xt = to_bf16(x)
+    assert lib.nwc_gemv_path(m.handle, xt, 16)[1] == (s.kernel == "tensor")
+    tolerance_check(m.gemv(xt).cpu().numpy(), orc.gemv(w, x), w, x)
     no_device_error(lib, m)
 
 

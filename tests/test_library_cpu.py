@@ -132,26 +132,30 @@ def test_rank_code_encoder_byte_identical_to_oracle(lib, orc, shape, tile_cols, 
     finally:
         lib.nwc_plan_destroy(plan)
     ref = orc.rank_encode(w, tile_cols=tile_cols, ranks=ranks or 7)
-    assert dev_bytes == 0 and blob.size == blob_bytes == ref.size
+    assert blob.size == blob_bytes == ref.size
     assert np.array_equal(blob, ref)
     assert np.array_equal(orc.rank_decode(blob), w)
+    # The device image: the blob, the 256-byte rank table, schedules, scratch.
+    assert dev_bytes == lib.nwc_blob_device_bytes(blob) > blob.size
 
 
-def test_rank_code_all_patterns_and_device_calls_refused(lib, orc):
-    import ctypes
+def test_rank_code_all_patterns_and_device_image(lib, orc):
     w = np.arange(65536, dtype=np.uint16).reshape(256, 256)
     plan = lib.nwc_plan(w, code=lib.NWC_CODE_RANK)
     blob = lib.nwc_compress_host(plan, w)
-    assert np.array_equal(blob, orc.rank_encode(w))
-    # No kernel reads this code yet: every call that needs a device image says so.
-    h = ctypes.c_void_p()
-    st = lib.LIB.nwc_compress(plan, w.ctypes.data, 1 << 20, 1 << 30, None, ctypes.byref(h))
-    assert st == UNSUPPORTED and not h.value
+    dev_bytes, _ = lib.nwc_plan_size(plan)
     lib.nwc_plan_destroy(plan)
-    for call in (lambda: lib.nwc_blob_device_bytes(blob), lambda: lib.nwc_schedule_describe(blob)):
+    assert np.array_equal(blob, orc.rank_encode(w))
+    assert lib.nwc_blob_device_bytes(blob) == dev_bytes
+    info, _, _, ring = lib.nwc_schedule_describe(blob)
+    assert info["tiles"] == len(ring) == 32
+    # A broken rank table is refused: a repeated ranked value, a value past 127.
+    for at, v in ((129, blob[128]), (128, 200)):
+        bad = blob.copy()
+        bad[at] = v
         with pytest.raises(lib.NwcError) as e:
-            call()
-        assert e.value.status == UNSUPPORTED
+            lib.nwc_blob_device_bytes(bad)
+        assert e.value.status == 4                    # NWC_ERR_CORRUPT
 
 
 def test_plan_options_code_field(lib):
@@ -172,14 +176,15 @@ def test_plan_options_code_field(lib):
     assert lib.LIB.nwc_plan(w.ctypes.data, 16, 256, ctypes.byref(opts), ctypes.byref(plan)) == 1
 
 
-def test_multi_stream_blobs_refused_until_a_kernel_reads_them(lib, orc):
-    """The format defines 2 or 4 bit streams per lane; no kernel reads them yet."""
+def test_four_stream_blobs_refused(lib, orc):
+    """The format defines 1, 2 or 4 bit streams per lane; the kernels read 1 and
+    2, so a device image exists for those and a 4-stream blob is refused."""
     w = synth.matrix(synth.MatrixSpec("w", 40, 600, "normal", 0.02, 0), 2)
-    for streams in (2, 4):
-        blob = orc.encode(w, tile_cols=128, streams=streams)
-        with pytest.raises(lib.NwcError) as e:
-            lib.nwc_blob_device_bytes(blob)
-        assert e.value.status == UNSUPPORTED
+    assert lib.nwc_blob_device_bytes(orc.encode(w, tile_cols=128, streams=2)) > 0
+    blob = orc.encode(w, tile_cols=128, streams=4)
+    with pytest.raises(lib.NwcError) as e:
+        lib.nwc_blob_device_bytes(blob)
+    assert e.value.status == UNSUPPORTED
     bad = orc.encode(w, tile_cols=128).copy()
     bad[60] = 2                                          # S = 3 is not a layout
     with pytest.raises(lib.NwcError) as e:
@@ -194,11 +199,15 @@ def test_streams_per_lane_encoder_and_refusals(lib, orc):
         plan = lib.nwc_plan(w, tile_cols=128, streams=streams)
         dev_bytes, _ = lib.nwc_plan_size(plan)
         blob = lib.nwc_compress_host(plan, w)
-        assert dev_bytes == 0 and np.array_equal(blob, orc.encode(w, tile_cols=128, lmax=7,
-                                                                  streams=streams))
-        h = ctypes.c_void_p()
-        st = lib.LIB.nwc_compress(plan, w.ctypes.data, 1 << 20, 1 << 30, None, ctypes.byref(h))
-        assert st == UNSUPPORTED and not h.value
+        assert np.array_equal(blob, orc.encode(w, tile_cols=128, lmax=7, streams=streams))
+        if streams == 2:
+            assert dev_bytes == lib.nwc_blob_device_bytes(blob) > blob.size
+        else:
+            assert dev_bytes == 0
+            h = ctypes.c_void_p()
+            st = lib.LIB.nwc_compress(plan, w.ctypes.data, 1 << 20, 1 << 30, None,
+                                      ctypes.byref(h))
+            assert st == UNSUPPORTED and not h.value
         lib.nwc_plan_destroy(plan)
     with pytest.raises(lib.NwcError) as e:
         lib.nwc_plan(w, streams=3)

@@ -11,7 +11,7 @@ K_SLOTS = 64          # barrier slots per CTA (kernels.cuh)
 K_MAX_LAG = 48        # tiles a consumer's next wait may lie past its last release (kernels.cuh)
 K_MAX_CTAS = 256
 K_XSTAGE = {1: 8448, 16: 33024}  # shared memory for x by rows of x per launch (kernels.cuh)
-K_RING_SLACK = 256    # shared memory after the ring that readers may touch (kernels.cu)
+K_RING_SLACK = 512    # shared memory after the ring that readers may touch (kernels.cu)
 B200_SMS, B200_SMEM = 148, 232448
 
 
