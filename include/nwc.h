@@ -334,29 +334,34 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
                                  nwc_schedule_info* info, uint32_t* cta_batch,
                                  uint32_t* batch, uint32_t* tile_ring);
 
-/* The tensor-core kernel's launch shape and schedule for a blob on a device
- * of sm_count SMs and smem_limit bytes of opt-in shared memory per block.
- * Host only; touches no GPU.  CTA c owns the tiles [tiles c / ctas,
- * tiles (c + 1) / ctas) of the row-major tile order v = i tiles_c + j, in
- * M-groups of `rows` row tiles; `teams` teams of `rows` decode warps take the
- * column blocks j = t, t + teams, ... of a group.
+/* The tensor-core kernel's launch shape and schedule for a blob, a GEMV of
+ * rows_of_x rows (1..64; the accumulator has 16, 32 or 64 columns, and each
+ * width has its own shape) on a device of sm_count SMs and smem_limit bytes of
+ * opt-in shared memory per block.  Host only; touches no GPU.  K is split
+ * into `ksplit` column ranges and the row tiles into ctas / ksplit row ranges
+ * (range k of n parts of m items: [m k / n, m (k + 1) / n)); CTA
+ * c = rs ksplit + ks owns row range rs x column range ks, in M-groups of
+ * `rows` row tiles; `teams` teams of `rows` decode warps take the column
+ * blocks j_lo + t, j_lo + t + teams, ... of a group.  Each copy moves one
+ * tile's lane lengths and streams (batch_tiles = 1); the raw plane is read
+ * from global memory.
  *   cta_batch (optional, ctas + 1 entries), batch (optional, 4 * batches):
  *     as nwc_schedule_describe.
  *   tile_ring, tile_batch (optional, tiles entries each), indexed by blob tile
- *     u = j tiles_r + i: the tile's ring offset, and the CTA's batch that
- *     brings it with, in bits 28..31, the extra releases its consumer adds
- *     (batch_tiles minus the tiles of that batch, on its first tile).
+ *     u = j tiles_r + i: the ring offset of the tile's streams, and the CTA's
+ *     copy that brings them.
  * Errors: INVALID_ARG, CORRUPT, UNSUPPORTED (no layout fits). */
 typedef struct {
   uint32_t struct_size;
-  int32_t ctas, rows, teams, batch_tiles, ring_bytes;
+  int32_t ctas, rows, teams, batch_tiles, ring_bytes, n, x_stages;
   int64_t tiles, batches;
   uint64_t smem_bytes, a_offset, b_offset, ring_offset;
+  int32_t ksplit;
 } nwc_tc_schedule_info;
 nwc_status nwc_tc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
-                                    uint64_t smem_limit, nwc_tc_schedule_info* info,
-                                    uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring,
-                                    uint32_t* tile_batch);
+                                    uint64_t smem_limit, int32_t rows_of_x,
+                                    nwc_tc_schedule_info* info, uint32_t* cta_batch,
+                                    uint32_t* batch, uint32_t* tile_ring, uint32_t* tile_batch);
 
 /* Any pointer may be NULL.  *blob_bytes is the serialisable part;
  * *compressed_bytes is what holds the matrix (blob, decode table and launch

@@ -40,9 +40,11 @@ class nwc_tc_schedule_info(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("ctas", ctypes.c_int32),
                 ("rows", ctypes.c_int32), ("teams", ctypes.c_int32),
                 ("batch_tiles", ctypes.c_int32), ("ring_bytes", ctypes.c_int32),
+                ("n", ctypes.c_int32), ("x_stages", ctypes.c_int32),
                 ("tiles", ctypes.c_int64), ("batches", ctypes.c_int64),
                 ("smem_bytes", ctypes.c_uint64), ("a_offset", ctypes.c_uint64),
-                ("b_offset", ctypes.c_uint64), ("ring_offset", ctypes.c_uint64)]
+                ("b_offset", ctypes.c_uint64), ("ring_offset", ctypes.c_uint64),
+                ("ksplit", ctypes.c_int32)]
 
 
 NWC_CODE_PREFIX, NWC_CODE_RANK = 0, 1
@@ -86,8 +88,8 @@ def _load() -> ctypes.CDLL:
         "nwc_schedule_describe": ([vp, u64, i32, u64, i32, c.POINTER(nwc_schedule_info), vp, vp,
                                    vp],
                                   c.c_int),
-        "nwc_tc_schedule_describe": ([vp, u64, i32, u64, c.POINTER(nwc_tc_schedule_info), vp, vp,
-                                      vp, vp], c.c_int),
+        "nwc_tc_schedule_describe": ([vp, u64, i32, u64, i32, c.POINTER(nwc_tc_schedule_info), vp,
+                                      vp, vp, vp], c.c_int),
         "nwc_plan_destroy": ([vp], None),
         "nwc_handle_destroy": ([vp], None),
     }
@@ -273,22 +275,24 @@ def nwc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int
     return d, cta, bat, ring
 
 
-def nwc_tc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int = 232448):
-    """The tensor-core kernel's launch shape and schedule for a blob on a
-    device of the given size; host only.  Returns (info dict, cta_batch
-    [ctas + 1], batch [batches x 4], tile_ring [tiles], tile_batch [tiles])."""
+def nwc_tc_schedule_describe(blob: np.ndarray, sm_count: int = 148, smem_limit: int = 232448,
+                             rows_of_x: int = 64):
+    """The tensor-core kernel's launch shape and schedule for a blob and a GEMV
+    of rows_of_x rows on a device of the given size; host only.  Returns (info
+    dict, cta_batch [ctas + 1], batch [batches x 4], tile_ring [tiles],
+    tile_batch [tiles])."""
     blob = np.ascontiguousarray(blob, dtype=np.uint8)
     info = nwc_tc_schedule_info(struct_size=ctypes.sizeof(nwc_tc_schedule_info))
     _check(LIB.nwc_tc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit,
-                                        ctypes.byref(info), None, None, None, None),
+                                        rows_of_x, ctypes.byref(info), None, None, None, None),
            "nwc_tc_schedule_describe")
     cta = np.zeros(info.ctas + 1, dtype=np.uint32)
     bat = np.zeros((info.batches, 4), dtype=np.uint32)
     ring = np.zeros(info.tiles, dtype=np.uint32)
     tb = np.zeros(info.tiles, dtype=np.uint32)
     _check(LIB.nwc_tc_schedule_describe(blob.ctypes.data, blob.size, sm_count, smem_limit,
-                                        ctypes.byref(info), cta.ctypes.data, bat.ctypes.data,
-                                        ring.ctypes.data, tb.ctypes.data),
+                                        rows_of_x, ctypes.byref(info), cta.ctypes.data,
+                                        bat.ctypes.data, ring.ctypes.data, tb.ctypes.data),
            "nwc_tc_schedule_describe")
     d = {k: getattr(info, k) for k, _ in nwc_tc_schedule_info._fields_ if k != "struct_size"}
     return d, cta, bat, ring, tb

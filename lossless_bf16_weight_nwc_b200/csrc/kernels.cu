@@ -1075,10 +1075,6 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t n) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(n)
-               : "memory");
-}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -1173,16 +1169,18 @@ __device__ __forceinline__ void tmem_load<16>(uint32_t taddr, float (&v)[16]) {
   for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-// Barriers and flags of the tensor-core kernel (at p.tc_bar_off).
+// Barriers, the MMA warp's state and flags of the tensor-core kernel (at
+// p.tc_bar_off).
 struct TcBars {
   uint64_t* xfull;    // [team][2]: x chunk of the stage landed (TMA bytes)
   uint64_t* sfull;    // [team][2]: the team's R decode warps wrote the A stage
   uint64_t* sempty;   // [team][2]: the MMAs that read the stage completed
   uint64_t* accfull;  // [team]: the team's accumulator holds its M-group sum
-  uint64_t* accempty; // every decode warp has read the accumulators
+  uint64_t* accempty; // the epilogue warps have read the accumulators
   uint32_t* tmem;     // TMEM base address (tcgen05.alloc writes it)
   volatile uint32_t* abort;   // a wait gave up: leave
   volatile uint32_t* issued;  // batches the producer has issued so far
+  uint32_t* mma;      // [7][team]: the MMA warp's counters (see tc_mma)
 };
 __device__ __forceinline__ TcBars tc_bars(uint8_t* smem, const TileParams& p) {
   TcBars b;
@@ -1194,9 +1192,11 @@ __device__ __forceinline__ TcBars tc_bars(uint8_t* smem, const TileParams& p) {
   b.tmem = reinterpret_cast<uint32_t*>(b.accempty + 1);
   b.abort = b.tmem + 1;
   b.issued = b.tmem + 2;
+  b.mma = b.tmem + 4;
   return b;
 }
-static_assert(8 * (7 * kTcMaxTeams + 1) + 12 <= (int)kTcBarBytes, "tensor-core barrier area");
+static_assert(8 * (7 * kTcMaxTeams + 1) + 16 + 4 * 7 * kTcMaxTeams <= (int)kTcBarBytes,
+              "tensor-core barrier area");
 
 // A consumer polls batch k's slot only once the producer has issued batch k:
 // the schedule keeps fewer than kSlots batches outstanding, so the slot's
@@ -1213,30 +1213,38 @@ __device__ __forceinline__ bool wait_issued(const TcBars& tb, uint32_t k, const 
   return false;
 }
 
-// Tiles of this CTA in the row-major tile order, and the row tiles they touch.
+// The rectangle of tiles this CTA owns: row tiles [i_lo, i_hi) x column
+// blocks [j_lo, j_hi), column range ks of the K split.
 struct TcWork {
-  int64_t a, b;   // linear range [a, b) of v = i tiles_c + j
-  int64_t i0, i1; // first and last row tile touched
+  int64_t i_lo, i_hi, j_lo, j_hi;
+  int ks;         // this CTA's column range
   int groups;     // M-groups of R row tiles
+  int teams;      // teams with at least one column block (min(TT, j_hi - j_lo))
 };
 __device__ __forceinline__ TcWork tc_work(const TileParams& p) {
   TcWork w;
-  w.a = p.n_tiles * (int64_t)blockIdx.x / gridDim.x;
-  w.b = p.n_tiles * (int64_t)(blockIdx.x + 1) / gridDim.x;
-  w.i0 = w.a / p.tiles_c;
-  w.i1 = (w.b - 1) / p.tiles_c;
-  w.groups = (int)((w.i1 - w.i0 + p.tc_rows) / p.tc_rows);
+  const int64_t ks = blockIdx.x % p.tc_ksplit, rs = blockIdx.x / p.tc_ksplit;
+  const int64_t row_ranges = gridDim.x / p.tc_ksplit;
+  w.i_lo = p.tiles_r * rs / row_ranges;
+  w.i_hi = p.tiles_r * (rs + 1) / row_ranges;
+  w.j_lo = p.tiles_c * ks / p.tc_ksplit;
+  w.j_hi = p.tiles_c * (ks + 1) / p.tc_ksplit;
+  w.ks = (int)ks;
+  w.groups = (int)((w.i_hi - w.i_lo + p.tc_rows - 1) / p.tc_rows);
+  const int64_t cols = w.j_hi - w.j_lo;
+  w.teams = (int)(cols < p.tc_teams ? cols : p.tc_teams);
   return w;
 }
-// CTA that owns linear tile v (the largest c with floor(T c / C) <= v).
-__device__ __forceinline__ int64_t tc_cta_of(int64_t v, int64_t tiles, int64_t ctas) {
-  return ((v + 1) * ctas - 1) / tiles;
+// Slot of the scratch that holds column range ks's sums of row tile i:
+// [kMaxTcRows][8] floats.
+__device__ __forceinline__ float* tc_slot(const TileParams& p, int ks, int64_t i) {
+  return p.partial + ((int64_t)ks * p.tiles_r + i) * (8 * kMaxTcRows);
 }
 
-// Accumulator columns (N / 4) a decode warp reads back: the sum of the teams'
-// accumulators for the warp's lane quarter q = warp % 4 and column quarter
-// warp / 4, and its store to y or, for a row tile shared with other CTAs, to
-// this CTA's boundary slot.
+// Accumulator columns (N / 4) an epilogue warp reads back: the sum of the
+// teams' accumulators for the warp's lane quarter q = warp % 4 and column
+// quarter warp / 4, and its store to y or, when K is split, to the slot of
+// this CTA's column range.
 template <int NQ>
 __device__ __forceinline__ void tc_epilogue(const TileParams& p, const TcWork& wk, uint32_t tmem,
                                             int warp, int lane, int64_t ig, int rg) {
@@ -1245,7 +1253,7 @@ __device__ __forceinline__ void tc_epilogue(const TileParams& p, const TcWork& w
 #pragma unroll
   for (int u = 0; u < NQ; ++u) acc[u] = 0.f;
   const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kq * NQ);
-  for (int t = 0; t < p.tc_teams; ++t) {
+  for (int t = 0; t < wk.teams; ++t) {
     float v[NQ];
     tmem_load<NQ>(base + (uint32_t)(t * p.tc_n), v);
 #pragma unroll
@@ -1254,30 +1262,32 @@ __device__ __forceinline__ void tc_epilogue(const TileParams& p, const TcWork& w
   const int mrow = 32 * q + lane, rr = mrow >> 3;
   if (rr >= rg) return;
   const int64_t i = ig + rr, orow = 8 * i + (lane & 7);
-  if (orow >= p.rows) return;
-  const bool full = i * p.tiles_c >= wk.a && (i + 1) * p.tiles_c <= wk.b;
-  float* slot = p.partial + (int64_t)(2 * blockIdx.x + (i == wk.i0 ? 0 : 1)) * 8 * kMaxTcRows;
+  if (p.tc_ksplit == 1) {
+    if (orow >= p.rows) return;
 #pragma unroll
-  for (int u = 0; u < NQ; ++u) {
-    const int bc = kq * NQ + u;
-    if (bc >= p.batch) break;
-    if (full)
+    for (int u = 0; u < NQ; ++u) {
+      const int bc = kq * NQ + u;
+      if (bc >= p.batch) break;
       p.y[(int64_t)bc * p.rows + orow] = acc[u];
-    else
+    }
+  } else {
+    float* slot = tc_slot(p, wk.ks, i);
+#pragma unroll
+    for (int u = 0; u < NQ; ++u) {
+      const int bc = kq * NQ + u;
+      if (bc >= p.batch) break;
       __stcg(slot + bc * 8 + (lane & 7), acc[u]);
+    }
   }
 }
 
-// The last CTA to deliver its part of a row tile shared by several CTAs sums
-// the parts in CTA order and writes y.  One warp.
-__device__ void tc_boundary(const TileParams& p, int64_t i, int lane) {
-  const int64_t ctas = gridDim.x;
-  const int64_t c_lo = tc_cta_of(i * p.tiles_c, p.n_tiles, ctas);
-  const int64_t c_hi = tc_cta_of((i + 1) * p.tiles_c - 1, p.n_tiles, ctas);
+// Row tile i when K is split: the last of the ksplit CTAs to deliver its slot
+// adds the slots in column-range order and writes y.  One warp.
+__device__ void tc_reduce(const TileParams& p, int64_t i, int lane) {
   uint32_t last = 0;
   if (lane == 0) {
     __threadfence();
-    last = atomicAdd(&p.counters[i], 1u) == (uint32_t)(c_hi - c_lo);
+    last = atomicAdd(&p.counters[i], 1u) == (uint32_t)(p.tc_ksplit - 1);
   }
   if (!__shfl_sync(kFull, last, 0)) return;
   __threadfence();
@@ -1285,56 +1295,68 @@ __device__ void tc_boundary(const TileParams& p, int64_t i, int lane) {
     const int bc = idx >> 3, r = idx & 7;
     const int64_t orow = 8 * i + r;
     float sum = 0.f;
-    for (int64_t c = c_lo; c <= c_hi; ++c) {
-      const int64_t first_row = (p.n_tiles * c / ctas) / p.tiles_c;
-      const float* slot = p.partial + (2 * c + (i == first_row ? 0 : 1)) * 8 * kMaxTcRows;
-      sum += __ldcg(slot + bc * 8 + r);
-    }
+    for (int ks = 0; ks < p.tc_ksplit; ++ks) sum += __ldcg(tc_slot(p, ks, i) + bc * 8 + r);
     if (orow < p.rows) p.y[(int64_t)bc * p.rows + orow] = sum;
   }
   if (lane == 0) p.counters[i] = 0u;
 }
 
-// Decode warps (0 .. 15): warp w < teams R is slot r = w % R of team t = w / R.
+// 16 raw bytes of global memory, read once (not kept in L1).
+__device__ __forceinline__ uint4 ldg_stream128(const uint8_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// Decode warps (0 .. 29): warp w < teams R is slot r = w % R of team t = w / R.
+// A tile's lane lengths and streams come from the ring; its raw plane straight
+// from global memory, two 64-column groups ahead.  Warps 0 .. 15 also read the
+// accumulators back after each M-group.
 template <int CP, int CODE, int S>
 __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, const TcBars& tb,
                           const TcWork& wk, int warp, int lane) {
-  constexpr int kRaw = CP * 512;
   const WaitCtl wc = wait_ctl(p);
   const int R = p.tc_rows, TT = p.tc_teams;
   const bool decoder = warp < TT * R;
+  const bool epilogue = warp < kTcEpilogueWarps;
   const int t = warp / R, r = warp % R;
   const int g = lane >> 2, c = lane & 3;
   const uint32_t table = smem_u32(smem);
   const uint32_t ring = smem_u32(s.ring);
   const uint32_t limit = ring + (uint32_t)p.ring_bytes + kRingSlack;
   const uint32_t a_area = smem_u32(smem + p.tc_a_off);
-  const int64_t nj = decoder ? (p.tiles_c - t + TT - 1) / TT : 0;
+  const int64_t nj = decoder && t < wk.teams ? (wk.j_hi - wk.j_lo - t + TT - 1) / TT : 0;
   const uint32_t chunk_lo = ((uint32_t)(2 * c) ^ (uint32_t)g) << 4;
   const uint32_t chunk_hi = ((uint32_t)(2 * c + 1) ^ (uint32_t)g) << 4;
   uint32_t seq = 0;
   bool ok = true;
   for (int gi = 0; gi < wk.groups && ok; ++gi) {
-    const int64_t ig = wk.i0 + (int64_t)gi * R;
-    const int rg = (int)min((int64_t)R, wk.i1 + 1 - ig);
+    const int64_t ig = wk.i_lo + (int64_t)gi * R;
+    const int rg = (int)min((int64_t)R, wk.i_hi - ig);
     const int64_t i = ig + r;
     for (int64_t jj = 0; jj < nj && ok; ++jj) {
-      const int64_t j = t + jj * TT;
-      const int64_t v = i * p.tiles_c + j;
-      const bool present = r < rg && v >= wk.a && v < wk.b;
+      const int64_t j = wk.j_lo + t + jj * TT;
+      const bool present = r < rg;
       LaneDecoder<CODE, S> dec;
-      uint32_t chunk = 0, bw = 0;
+      const uint8_t* raw = nullptr;
+      uint4 rv0 = make_uint4(0u, 0u, 0u, 0u), rv1 = rv0;
+      uint32_t bw = 0;
       if (present) {
         const int64_t u = j * p.tiles_r + i;
+        raw = p.tiles + 16ull * __ldg(p.index + u);
+        rv0 = ldg_stream128(raw + lane * 16);  // groups 0 and 1, before the wait
+        if (CP > 1) rv1 = ldg_stream128(raw + 512 + lane * 16);
         bw = __ldg(p.tile_batch + u);
-        chunk = ring + __ldg(p.tile_ring + u);
-        if (!wait_issued(tb, bw & 0x0FFFFFFFu, wc) || !wait_batch(s, (int)(bw & 0x0FFFFFFFu), wc)) {
+        const uint32_t stage = ring + __ldg(p.tile_ring + u);
+        if (!wait_issued(tb, bw, wc) || !wait_batch(s, (int)bw, wc)) {
           ok = false;
           break;
         }
         uint32_t start[S];
-        lane_stream_starts<S>(chunk, kRaw, lane, start);
-        dec.init(chunk + kRaw + kLanes * S, start, limit, table);
+        lane_stream_starts<S>(stage, 0, lane, start);
+        dec.init(stage + kLanes * S, start, limit, table);
       }
       for (int m = 0; m < CP; ++m, ++seq) {
         const uint32_t st = seq & 1u, use = seq >> 1;
@@ -1347,7 +1369,9 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
             a_area + ((uint32_t)(2 * t + (int)st) * (uint32_t)R + (uint32_t)r) * kTcStageA +
             (uint32_t)g * 128u;
         if (present) {
-          const uint4 rv = lds128(chunk + m * 512 + lane * 16);
+          const uint4 rv = rv0;
+          rv0 = rv1;
+          if (m + 2 < CP) rv1 = ldg_stream128(raw + (m + 2) * 512 + lane * 16);
           uint32_t wv[8];
 #pragma unroll
           for (int k = 0; k < 8; k += 4) {
@@ -1358,24 +1382,21 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
           }
           sts128(arow + chunk_lo, wv[0], wv[1], wv[2], wv[3]);
           sts128(arow + chunk_hi, wv[4], wv[5], wv[6], wv[7]);
-        } else if (r < rg) {
-          // A row tile of the group outside this CTA's range for this column
-          // block: zeros, so its accumulator rows get nothing from it.
-          sts128(arow + chunk_lo, 0u, 0u, 0u, 0u);
-          sts128(arow + chunk_hi, 0u, 0u, 0u, 0u);
         }
+        // (A slot of a row past the group's last row tile keeps stale data:
+        // it only reaches accumulator rows that the epilogue skips.)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(&tb.sfull[2 * t + st]);
       }
       if (present && ok) {
         __syncwarp();
-        if (lane == 0) mbar_arrive_n(&s.empty[(bw & 0x0FFFFFFFu) % kSlots], 1u + (bw >> 28));
+        if (lane == 0) mbar_arrive(&s.empty[bw % kSlots]);
       }
     }
-    if (!ok) break;
-    // Epilogue of the group, by all 16 decode warps.
-    for (int tt = 0; tt < TT && ok; ++tt)
+    if (!ok || !epilogue) continue;
+    // Epilogue of the group, by warps 0 .. 15 (the others go on decoding).
+    for (int tt = 0; tt < wk.teams && ok; ++tt)
       ok = __all_sync(kFull, wait_bounded(&tb.accfull[tt], (uint32_t)gi & 1u, wc));
     if (!ok) break;
     tc_fence_after();
@@ -1389,18 +1410,13 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
     __threadfence();  // this warp's y and slot stores, before the arrival below
     __syncwarp();
     if (lane == 0) mbar_arrive(tb.accempty);
-    // Row tiles shared with other CTAs (at most the first and the last of the
-    // range): once every decode warp has stored its part (accempty completes
-    // this group's phase after all 16 arrivals), warp 0 delivers them.
-    if (warp == 0 && p.tiles_c > 1) {
+    // K split: once every epilogue warp has stored its slots (accempty
+    // completes this group's phase after their 16 arrivals), epilogue warp w
+    // delivers row tile ig + w.
+    if (p.tc_ksplit > 1) {
       ok = __all_sync(kFull, wait_bounded(tb.accempty, (uint32_t)gi & 1u, wc));
       if (!ok) break;
-      auto shared_row = [&](int64_t ii) {
-        return ii >= ig && ii < ig + rg &&
-               !(ii * p.tiles_c >= wk.a && (ii + 1) * p.tiles_c <= wk.b);
-      };
-      if (shared_row(wk.i0)) tc_boundary(p, wk.i0, lane);
-      if (wk.i1 != wk.i0 && shared_row(wk.i1)) tc_boundary(p, wk.i1, lane);
+      if (warp < rg) tc_reduce(p, ig + warp, lane);
     }
   }
   if (!ok && lane == 0) *tb.abort = 1u;
@@ -1410,25 +1426,30 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
 // K = 16 MMAs of every chunk once the team's decode warps have written it, and
 // commits their completion to the stage's barrier (and at the end of an
 // M-group to the team's accumulator barrier).  It serves the teams in turn
-// without blocking on any of them.
+// without blocking on any of them.  Its per-team counters live in shared
+// memory (tb.mma), so the kernel fits the 64 registers of 1024 threads.
 template <int CP>
 __device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* smem,
                        const TcBars& tb, const TcWork& wk) {
   const WaitCtl wc = wait_ctl(p);
-  const int R = p.tc_rows, TT = p.tc_teams, N = p.tc_n;
+  const int R = p.tc_rows, TT = p.tc_teams, N = p.tc_n, SB = p.tc_bstages;
   const uint32_t a_area = smem_u32(smem + p.tc_a_off), b_area = smem_u32(smem + p.tc_b_off);
+  const uint32_t bstage = (uint32_t)N * 128u;
   const uint32_t idesc = umma_idesc_bf16(128, N);
   const uint32_t tmem = *tb.tmem;
-  // Per team, in registers (the team loops are unrolled to kTcMaxTeams):
-  // chunks whose x was fetched (nx) and that were multiplied (nm), out of
-  // total; the within-group index of the next chunk to fetch (xw) and to
-  // multiply (mw), and the group of the latter (mg).  No divisions: CP is a
-  // power of two and the indices advance by one.
-  uint32_t nx[kTcMaxTeams], nm[kTcMaxTeams], total[kTcMaxTeams], per_group[kTcMaxTeams];
-  uint32_t xw[kTcMaxTeams], mw[kTcMaxTeams], mg[kTcMaxTeams];
-#pragma unroll
-  for (int t = 0; t < kTcMaxTeams; ++t) {
-    per_group[t] = t < TT ? (uint32_t)((p.tiles_c - t + TT - 1) / TT) * CP : 0u;
+  // Per team t: chunks whose x was fetched (nx) and that were multiplied (nm),
+  // out of total; the within-group index of the next chunk to fetch (xw) and
+  // to multiply (mw), the group of the latter (mg), and chunks per group.
+  uint32_t* nx = tb.mma;
+  uint32_t* nm = nx + kTcMaxTeams;
+  uint32_t* total = nm + kTcMaxTeams;
+  uint32_t* per_group = total + kTcMaxTeams;
+  uint32_t* xw = per_group + kTcMaxTeams;
+  uint32_t* mw = xw + kTcMaxTeams;
+  uint32_t* mg = mw + kTcMaxTeams;
+  for (int t = 0; t < TT; ++t) {
+    per_group[t] =
+        t < wk.teams ? (uint32_t)((wk.j_hi - wk.j_lo - t + TT - 1) / TT) * CP : 0u;
     total[t] = (uint32_t)wk.groups * per_group[t];
     nx[t] = nm[t] = xw[t] = mw[t] = mg[t] = 0;
   }
@@ -1436,45 +1457,52 @@ __device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* sm
   uint32_t idle = 0;
   for (;;) {
     bool done = true, moved = false;
-#pragma unroll
-    for (int t = 0; t < kTcMaxTeams; ++t) {
-      if (nm[t] >= total[t]) continue;
+    for (int t = 0; t < TT; ++t) {
+      uint32_t cm = nm[t], cx = nx[t];
+      const uint32_t tot = total[t];
+      if (cm >= tot) continue;
       done = false;
-      // x of chunk nx[t]: its stage is free once the MMAs two chunks back are done.
-      if (nx[t] < total[t] && nx[t] < nm[t] + 2) {
-        const uint32_t sx = nx[t] & 1u, use = nx[t] >> 1;
-        if (use == 0 || mbar_test_wait(&tb.sempty[2 * t + sx], (use - 1) & 1u)) {
-          const int64_t j = t + (int64_t)(xw[t] / CP) * TT;
-          const int m = (int)(xw[t] % CP);
-          mbar_expect_tx(&tb.xfull[2 * t + sx], (uint32_t)N * 128u);
-          tma_load_2d(b_area + (uint32_t)(2 * t + (int)sx) * kTcStageB, tmap,
-                      (int32_t)(j * CP * 64 + m * 64), 0, &tb.xfull[2 * t + sx]);
-          ++nx[t];
-          xw[t] = xw[t] + 1 == per_group[t] ? 0u : xw[t] + 1;
+      // x of chunk cx: its stage is free once the MMAs SB chunks back are done.
+      if (cx < tot && cx < cm + (uint32_t)SB) {
+        const uint32_t prev = cx - (uint32_t)SB;  // the chunk that last used the stage
+        if (cx < (uint32_t)SB ||
+            mbar_test_wait(&tb.sempty[2 * t + (int)(prev & 1u)], (prev >> 1) & 1u)) {
+          const uint32_t w = xw[t];
+          const int64_t j = wk.j_lo + t + (int64_t)(w / CP) * TT;
+          const int m = (int)(w % CP);
+          const uint32_t sx = cx % (uint32_t)SB;
+          mbar_expect_tx(&tb.xfull[2 * t + (int)sx], bstage);
+          tma_load_2d(b_area + (uint32_t)(t * SB + (int)sx) * bstage, tmap,
+                      (int32_t)(j * CP * 64 + m * 64), 0, &tb.xfull[2 * t + (int)sx]);
+          nx[t] = ++cx;
+          xw[t] = w + 1 == per_group[t] ? 0u : w + 1;
           moved = true;
         }
       }
-      // MMAs of chunk nm[t].
-      if (nm[t] < nx[t]) {
-        const uint32_t sm = nm[t] & 1u, ph = (nm[t] >> 1) & 1u;
-        if (mbar_test_wait(&tb.xfull[2 * t + sm], ph) && mbar_test_wait(&tb.sfull[2 * t + sm], ph) &&
-            (mw[t] != 0 || mg[t] == 0 || mbar_test_wait(tb.accempty, (mg[t] - 1) & 1u))) {
+      // MMAs of chunk cm.
+      if (cm < cx) {
+        const uint32_t sa = cm & 1u, ph = (cm >> 1) & 1u;
+        const uint32_t sx = cm % (uint32_t)SB, phx = (cm / (uint32_t)SB) & 1u;
+        const uint32_t w = mw[t], grp = mg[t];
+        if (mbar_test_wait(&tb.xfull[2 * t + (int)sx], phx) &&
+            mbar_test_wait(&tb.sfull[2 * t + (int)sa], ph) &&
+            (w != 0 || grp == 0 || mbar_test_wait(tb.accempty, (grp - 1) & 1u))) {
           tc_fence_after();
-          const uint32_t a0 = a_area + (uint32_t)(2 * t + (int)sm) * (uint32_t)R * kTcStageA;
-          const uint32_t b0 = b_area + (uint32_t)(2 * t + (int)sm) * kTcStageB;
+          const uint32_t a0 = a_area + (uint32_t)(2 * t + (int)sa) * (uint32_t)R * kTcStageA;
+          const uint32_t b0 = b_area + (uint32_t)(t * SB + (int)sx) * bstage;
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             umma_bf16(tmem + (uint32_t)(t * N), umma_desc_sw128(a0 + 32u * k),
-                      umma_desc_sw128(b0 + 32u * k), idesc, (mw[t] == 0 && k == 0) ? 0u : 1u);
-          umma_commit(&tb.sempty[2 * t + sm]);
-          if (mw[t] + 1 == per_group[t]) {
+                      umma_desc_sw128(b0 + 32u * k), idesc, (w == 0 && k == 0) ? 0u : 1u);
+          umma_commit(&tb.sempty[2 * t + (int)sa]);
+          if (w + 1 == per_group[t]) {
             umma_commit(&tb.accfull[t]);
             mw[t] = 0;
-            ++mg[t];
+            mg[t] = grp + 1;
           } else {
-            ++mw[t];
+            mw[t] = w + 1;
           }
-          ++nm[t];
+          nm[t] = cm + 1;
           moved = true;
         }
       }
@@ -1490,19 +1518,18 @@ __device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* sm
   }
   // Leave nothing in flight: x loads issued but not consumed, and the MMAs.
   const WaitCtl dc = drain_ctl(p);
-#pragma unroll
-  for (int t = 0; t < kTcMaxTeams; ++t) {
+  for (int t = 0; t < TT; ++t) {
     for (uint32_t k = nm[t]; k < nx[t]; ++k)
-      wait_bounded(&tb.xfull[2 * t + (int)(k & 1u)], (k >> 1) & 1u, dc);
+      wait_bounded(&tb.xfull[2 * t + (int)(k % (uint32_t)SB)], (k / (uint32_t)SB) & 1u, dc);
     if (nm[t] > 0)
       wait_bounded(&tb.sempty[2 * t + (int)((nm[t] - 1) & 1u)], ((nm[t] - 1) >> 1) & 1u, dc);
   }
 }
 
 // y[b][n] for up to kMaxTcRows rows b of x, every weight decoded once.
-// Warps 0..15 decode into the A stages and read the accumulators back, warp 16
-// allocates TMEM and issues x loads and MMAs, warp 17 moves the compressed
-// tiles into the ring (the same producer as the other kernels).
+// Warps 0..29 decode into the A stages (0..15 also read the accumulators
+// back), warp 30 allocates TMEM and issues x loads and MMAs, warp 31 moves the
+// compressed streams into the ring (the same producer as the other kernels).
 template <int CP, int CODE, int S>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemv_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap) {
@@ -1529,7 +1556,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&tb.sempty[k], 1);
     }
     for (int k = 0; k < kTcMaxTeams; ++k) mbar_init(&tb.accfull[k], 1);
-    mbar_init(tb.accempty, kTcDecodeWarps);
+    mbar_init(tb.accempty, kTcEpilogueWarps);
     *tb.abort = 0u;
     *tb.issued = 0u;
   }
@@ -1743,65 +1770,88 @@ cudaError_t launch_decompress(const TileParams& p, int tile_cols, int code,
   }
 }
 
-bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_chunk, uint64_t typical_chunk,
-              uint32_t table_bytes, int sm_count, size_t smem_limit, TcShape* out) {
-  const int64_t tiles = tiles_r * tiles_c;
-  int64_t ctas = tiles < sm_count ? tiles : sm_count;
-  if (ctas > (int64_t)kMaxCtas) ctas = kMaxCtas;
-  if (ctas < 1) ctas = 1;
-  const int64_t per_cta = (tiles + ctas - 1) / ctas;
-  // Row tiles a CTA touches: its tiles span at most this many rows.
-  int64_t rows_max = (per_cta + tiles_c - 1) / tiles_c + 1;
-  if (rows_max > tiles_r) rows_max = tiles_r;
-  if (rows_max > 16) rows_max = 16;
-  int bt = (int)((kBatchTarget + typical_chunk - 1) / (typical_chunk ? typical_chunk : 1));
-  if (bt < 2) bt = 2;
-  if (bt > 8) bt = 8;
+bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_streams, uint32_t table_bytes,
+              int n, int sm_count, size_t smem_limit, TcShape* out) {
+  int64_t cmax = sm_count < (int)kMaxCtas ? (int64_t)sm_count : (int64_t)kMaxCtas;
+  if (cmax < 1) cmax = 1;
+  int64_t ks_max = tc_max_ksplit(tiles_c);
+  if (ks_max > cmax) ks_max = cmax;
   const uint32_t bar_off = (uint32_t)xstage_offset(table_bytes);
+  const uint32_t a_off = (bar_off + kTcBarBytes + 1023u) / 1024u * 1024u;
+  const uint32_t bstage = (uint32_t)n * 128u;
+  // Candidates in order of preference: every decode warp's streams resident
+  // (full), fewest rounds, smallest split, two x stages, largest ring.
   bool found = false;
   TcShape best{};
-  int64_t best_rounds = 0, best_ring = 0;
-  for (int R = (int)rows_max; R >= 1; --R) {
-    int tmax = 16 / R;
-    if (tmax > tiles_c) tmax = (int)tiles_c;
-    if (tmax > kTcMaxTeams) tmax = kTcMaxTeams;
-    for (int TT = tmax; TT >= 1; --TT) {
-      const uint32_t a_off = (bar_off + kTcBarBytes + 1023u) / 1024u * 1024u;
-      const uint32_t b_off = a_off + (uint32_t)(2 * TT * R) * kTcStageA;
-      const size_t head = b_off + (size_t)(2 * TT) * kTcStageB;
-      const size_t ring_offset = (head + 127) / 128 * 128;
-      if (smem_limit < ring_offset + kRingSlack) continue;
-      size_t ring = smem_limit - ring_offset - kRingSlack;
-      const size_t cap = (size_t)per_cta * (size_t)max_chunk;
-      if (ring > cap) ring = cap;
-      ring = ring / 16 * 16;
-      // A team's run of R tiles plus two copies of worst-case chunks (no more
-      // than the CTA's tiles), and the last A stage's 16 KiB operand window,
-      // must fit.
-      int64_t need_tiles = (int64_t)R + 2 * bt;
-      if (need_tiles > per_cta) need_tiles = per_cta;
-      if (ring < (size_t)need_tiles * (size_t)max_chunk) continue;
-      if (ring_offset + ring + kRingSlack < (size_t)a_off + (size_t)(2 * TT * R - 1) * kTcStageA + 16384)
-        continue;
-      // Tile decodes on a decode warp's critical path: M-groups of the CTA's
-      // rows times rounds of column blocks per group.
-      const int64_t rounds = (rows_max + R - 1) / R * ((tiles_c + TT - 1) / TT);
-      if (!found || rounds < best_rounds || (rounds == best_rounds && (int64_t)ring > best_ring)) {
-        found = true;
-        best_rounds = rounds;
-        best_ring = (int64_t)ring;
-        best.rows = R;
-        best.teams = TT;
-        best.bar_off = bar_off;
-        best.a_off = a_off;
-        best.b_off = b_off;
-        best.s.ctas = (int)ctas;
-        best.s.table_bytes = table_bytes;
-        best.s.xstage_bytes = (uint32_t)(head - bar_off);
-        best.s.ring_offset = ring_offset;
-        best.s.ring_bytes = (int)ring;
-        best.s.batch_tiles = bt;
-        best.s.smem_bytes = ring_offset + ring + kRingSlack;
+  int64_t best_key[5] = {0, 0, 0, 0, 0};
+  for (int64_t KS = 1; KS <= ks_max; ++KS) {
+    int64_t row_ranges = cmax / KS;
+    if (row_ranges > tiles_r) row_ranges = tiles_r;
+    const int64_t ctas = row_ranges * KS;
+    const int64_t rows_c = (tiles_r + row_ranges - 1) / row_ranges;  // largest rectangle
+    const int64_t cols_c = (tiles_c + KS - 1) / KS;
+    const int64_t per_cta = rows_c * cols_c;
+    const int rows_max = rows_c < 16 ? (int)rows_c : 16;
+    for (int R = rows_max; R >= 1; --R) {
+      int tmax = kTcDecodeWarps / R;
+      if (tmax > cols_c) tmax = (int)cols_c;
+      if (tmax > kTcMaxTeams) tmax = kTcMaxTeams;
+      if (tmax > 512 / n) tmax = 512 / n;
+      for (int TT = tmax; TT >= 1; --TT) {
+        for (int SB = 2; SB >= 1; --SB) {
+          const uint32_t b_off = a_off + (uint32_t)(2 * TT * R) * kTcStageA;
+          const size_t head = b_off + (size_t)(TT * SB) * bstage;
+          const size_t ring_offset = (head + 127) / 128 * 128;
+          if (smem_limit < ring_offset + kRingSlack) continue;
+          size_t ring = smem_limit - ring_offset - kRingSlack;
+          const size_t cap = (size_t)per_cta * (size_t)max_streams;
+          if (ring > cap) ring = cap;
+          ring = ring / 16 * 16;
+          // Deadlock-free: a team's run of R single-tile copies, one more, and
+          // the wrap-around of a copy (no more than the CTA's tiles).
+          int64_t need = (int64_t)R + 2;
+          if (need > per_cta) need = per_cta;
+          if (ring < (size_t)need * (size_t)max_streams) continue;
+          // The last A stage's 16 KiB operand window stays inside shared
+          // memory: the allocation is padded to cover it when the ring ends
+          // earlier.
+          const size_t window_end =
+              (size_t)a_off + (size_t)(2 * TT * R - 1) * kTcStageA + 16384;
+          size_t smem_bytes = ring_offset + ring + kRingSlack;
+          if (smem_bytes < window_end) smem_bytes = window_end;
+          if (smem_bytes > smem_limit) continue;
+          int64_t warps_resident = (int64_t)TT * R + 2;
+          if (warps_resident > per_cta) warps_resident = per_cta;
+          const int64_t full = ring >= (size_t)warps_resident * (size_t)max_streams ? 1 : 0;
+          const int64_t rounds = (rows_c + R - 1) / R * ((cols_c + TT - 1) / TT);
+          // Larger is better: resident, then -rounds, -split, stages, ring.
+          const int64_t key[5] = {full, -rounds, -KS, SB, (int64_t)ring};
+          bool better = !found;
+          for (int k = 0; k < 5 && !better; ++k) {
+            if (key[k] != best_key[k]) {
+              better = key[k] > best_key[k];
+              break;
+            }
+          }
+          if (!better) continue;
+          found = true;
+          for (int k = 0; k < 5; ++k) best_key[k] = key[k];
+          best.rows = R;
+          best.teams = TT;
+          best.ksplit = (int)KS;
+          best.n = n;
+          best.bstages = SB;
+          best.bar_off = bar_off;
+          best.a_off = a_off;
+          best.b_off = b_off;
+          best.s.ctas = (int)ctas;
+          best.s.table_bytes = table_bytes;
+          best.s.xstage_bytes = (uint32_t)(head - bar_off);
+          best.s.ring_offset = ring_offset;
+          best.s.ring_bytes = (int)ring;
+          best.s.batch_tiles = 1;
+          best.s.smem_bytes = smem_bytes;
+        }
       }
     }
   }
@@ -1812,7 +1862,9 @@ bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_chunk, uint64_t typ
 cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols, int code,
                            const TcShape& s, cudaStream_t stream) {
   if (p.batch < 1 || p.batch > kMaxTcRows || p.tc_teams < 1 || p.tc_teams > kTcMaxTeams ||
-      p.tc_rows < 1 || p.tc_rows * p.tc_teams > kTcDecodeWarps)
+      p.tc_rows < 1 || p.tc_rows > 16 || p.tc_rows * p.tc_teams > kTcDecodeWarps ||
+      p.tc_ksplit < 1 || s.s.ctas % p.tc_ksplit != 0 ||
+      (p.tc_ksplit > 1 && p.tc_ksplit > tc_max_ksplit(p.tiles_c)))
     return cudaErrorInvalidValue;
   switch (tile_cols) {
     case 512: return code == kCodeRank ? launch_gemv_tc_t<8, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<8, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<8, kCode12>(p, tmap, s.s, stream);

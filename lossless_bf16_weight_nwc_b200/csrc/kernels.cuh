@@ -47,7 +47,8 @@ struct TileParams {
   const uint16_t* x;        // BF16 [batch x cols]
   float* y;                 // FP32 [batch x rows]
   int32_t batch;            // rows of x handled by this launch (<= kMaxPassRows)
-  float* partial;           // [tiles_c][batch][rows_pad] split-K partial sums
+  float* partial;           // split-K partial sums: [tiles_c][batch][rows_pad] (CUDA
+                            // cores), [ksplit][tiles_r][kMaxTcRows][8] (tensor cores)
   uint32_t* counters;       // [tiles_r] arrivals per row tile
   int64_t rows_pad;         // 8 * tiles_r
   // decompress
@@ -56,10 +57,13 @@ struct TileParams {
   uint32_t wait_limit;      // polls before a bounded wait gives up (0: default)
   int32_t streams;          // bit streams per lane and tile (1 or 2)
   // tensor-core kernel
-  const uint32_t* tile_batch;  // device: per tile, its batch | extra releases << 28
+  const uint32_t* index;       // device: chunk offsets (16-byte units), tiles + 1
+  const uint32_t* tile_batch;  // device: per tile, its copy's place in its CTA's schedule
+  int32_t tc_bstages;       // x stages per team (1 or 2)
   int32_t tc_rows;          // R: row tiles per M-group (rows of the MMA / 8)
   int32_t tc_teams;         // teams of R decode warps, each on its own column blocks
   int32_t tc_n;             // accumulator columns: rows of x padded to 16, 32 or 64
+  int32_t tc_ksplit;        // column ranges; gridDim.x is a multiple of it
   uint32_t tc_tmem_cols;    // TMEM columns allocated (power of two >= 32)
   uint32_t tc_bar_off, tc_a_off, tc_b_off;  // shared-memory offsets
 };
@@ -105,44 +109,62 @@ cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const Laun
 
 // ---- tensor-core (tcgen05) GEMV: decode once, multiply every row of x -----
 //
-// CTA c owns the tiles [T c / C, T (c + 1) / C) of the ROW-major tile order
-// v = i tiles_c + j (T tiles, C CTAs), so it owns whole row tiles except at
-// most one partial row tile at each end, and sums over K on chip.  Its row
+// The matrix's tile grid (tiles_r row tiles x tiles_c column blocks) is cut
+// into rectangles: K into ksplit column ranges, the rows into C / ksplit row
+// ranges; CTA c = rs ksplit + ks owns row range rs x column range ks.  Its row
 // tiles form M-groups of R (the MMA's M = 128 rows holds up to 16 row tiles);
-// `teams` teams of R decode warps take the column blocks j = t, t + teams, ...
-// of a group, each team accumulating into its own TMEM accumulator.
-constexpr int kTcDecodeWarps = 16;
-constexpr int kTcMmaWarp = 16;       // TMEM allocation, x loads (TMA), MMA issue
-constexpr int kTcProducerWarp = 17;  // bulk copies of the compressed tiles
-constexpr int kTcThreads = 18 * 32;
-constexpr uint32_t kTcBarBytes = 1024;                 // barriers, TMEM address, flags
-constexpr uint32_t kTcStageA = 1024;                   // one row tile: 8 x 64 BF16
-constexpr uint32_t kTcStageB = (uint32_t)kMaxTcRows * 128;  // 64 rows of x x 64 BF16
-constexpr int kTcMaxTeams = 8;                         // 8 accumulators of 64 columns
+// `teams` teams of R decode warps take the column blocks j_lo + t,
+// j_lo + t + teams, ... of a group, each team accumulating into its own TMEM
+// accumulator.  With ksplit = 1 a CTA owns whole rows and writes y; otherwise
+// each part writes its row tiles' sums to a slot of the scratch and the last
+// part to arrive adds the slots in order.  The ring holds only each tile's
+// lane lengths and streams (one bulk copy per tile); the decode warps read the
+// raw plane straight from global memory, so a tile held while it is decoded
+// costs about a quarter of its chunk.
+constexpr int kTcDecodeWarps = 30;
+constexpr int kTcEpilogueWarps = 16;  // 4 per TMEM lane quarter read the accumulators
+constexpr int kTcMmaWarp = 30;        // TMEM allocation, x loads (TMA), MMA issue
+constexpr int kTcProducerWarp = 31;   // bulk copies of the compressed streams
+constexpr int kTcThreads = 32 * 32;
+constexpr uint32_t kTcBarBytes = 2048;  // barriers, MMA-warp state, TMEM address, flags
+constexpr uint32_t kTcStageA = 1024;    // one row tile: 8 x 64 BF16
+constexpr int kTcMaxTeams = 15;
+// Accumulator widths (rows of x padded): one launch shape and schedule each.
+constexpr int kTcClasses = 3;
+constexpr int kTcColumns[kTcClasses] = {16, 32, 64};
+inline int tc_class(int rows_of_x) { return rows_of_x <= 16 ? 0 : rows_of_x <= 32 ? 1 : 2; }
 
 struct TcShape {
-  LaunchShape s;       // grid, ring and copies; s.xstage_bytes spans barriers, A and B
+  LaunchShape s;       // grid, ring and copies (batch_tiles 1); s.xstage_bytes spans barriers, A, B
   int rows;            // R
   int teams;
+  int ksplit;          // column ranges (s.ctas is a multiple of it)
+  int n;               // accumulator columns of the class
+  int bstages;         // x stages per team (1 or 2)
   uint32_t bar_off, a_off, b_off;  // shared-memory offsets
 };
-// Chooses R and the team count for a matrix of tiles_r x tiles_c tiles on a
-// device of sm_count SMs and smem_limit bytes of shared memory per block: the
-// fewest tile decodes on a decode warp's path (M-groups of the rows a CTA
-// touches x rounds of column blocks per group), then the largest ring, with
-// room in the ring
-// for a team's tiles plus two copies of worst-case chunks (so that a team never
-// waits for a tile that cannot be issued).  Returns false when nothing fits.
-bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_chunk, uint64_t typical_chunk,
-              uint32_t table_bytes, int sm_count, size_t smem_limit, TcShape* out);
-// The tensor-core kernel's schedule (layout in nwc_format.h) for shape s;
-// `out` receives sched_tc_bytes(tiles) bytes.
-void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c, const TcShape& s,
-                       uint8_t* out);
+// Chooses the K split, R, the team count and the x stages for a matrix of
+// tiles_r x tiles_c tiles and an accumulator of n columns on a device of
+// sm_count SMs and smem_limit bytes of shared memory per block: among the
+// layouts whose ring holds every decode warp's streams (max_streams bytes per
+// tile at most), the fewest tile decodes on a decode warp's path (M-groups x
+// rounds of column blocks of the largest rectangle), then the smallest split,
+// then two x stages, then the largest ring; else the layout with the most
+// decode warps whose ring still holds a team's tiles and two more (so that no
+// team waits for a tile that cannot be issued).  Returns false when nothing
+// fits.
+bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_streams, uint32_t table_bytes,
+              int n, int sm_count, size_t smem_limit, TcShape* out);
+// The tensor-core kernel's schedule (layout in nwc_format.h) for shape s:
+// one copy per tile of its lane lengths and streams (the chunk after its raw
+// plane of raw_bytes); `out` receives sched_tc_bytes(tiles) bytes.
+void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c,
+                       uint32_t raw_bytes, const TcShape& s, uint8_t* out);
 // tmap: the TMA descriptor of x (BF16 [rows of x][cols], box 64 columns x
 // tc_n rows, 128-byte swizzle).
 cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int tile_cols,
                            int code, const TcShape& s, cudaStream_t stream);
+
 cudaError_t launch_decompress(const TileParams& p, int tile_cols, int code,
                               const LaunchShape& s, cudaStream_t stream);
 // Row gather (embedding lookup) from the compressed matrix.

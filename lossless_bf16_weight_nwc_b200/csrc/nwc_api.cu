@@ -104,38 +104,44 @@ nwc_status write_schedule(nwc_handle_s* h, int cls, const nwc::LaunchShape& s,
   return NWC_OK;
 }
 
-uint64_t tc_class_off(const nwc_handle_s& h) {
-  return h.sched_off + (uint64_t)nwc::kStageClasses * nwc::sched_class_bytes((uint64_t)h.tiles);
+uint64_t tc_class_off(const nwc_handle_s& h, int cls) {
+  return h.sched_off + (uint64_t)nwc::kStageClasses * nwc::sched_class_bytes((uint64_t)h.tiles) +
+         (uint64_t)cls * nwc::sched_tc_bytes((uint64_t)h.tiles);
 }
 
-// Tensor-core launch shape for a handle on a device of `sms` SMs and `smem`
-// bytes of opt-in shared memory per block; false when it does not fit.
-bool tc_shape_on(const nwc_handle_s& h, int sms, size_t smem, nwc::TcShape* ts) {
-  const uint64_t typical = (h.blob_bytes - h.tiles_off) / (uint64_t)h.tiles;
-  return nwc::tc_shape(h.tiles_r, h.tiles_c, h.max_chunk, typical, table_bytes_of(h), sms, smem,
-                       ts);
+// Tensor-core launch shape of accumulator class cls for a handle on a device
+// of `sms` SMs and `smem` bytes of opt-in shared memory per block; false when
+// it does not fit.
+bool tc_shape_on(const nwc_handle_s& h, int sms, size_t smem, int cls, nwc::TcShape* ts) {
+  const uint64_t max_streams = h.max_chunk - nwc::raw_bytes(h.tile_cols);
+  return nwc::tc_shape(h.tiles_r, h.tiles_c, max_streams, table_bytes_of(h), nwc::kTcColumns[cls],
+                       sms, smem, ts);
 }
 
-bool same_tc_shape(const nwc_handle_s& h, const nwc::TcShape& t) {
-  return h.tc_rows == t.rows && h.tc_teams == t.teams && h.tc_ctas == t.s.ctas &&
-         h.tc_ring == t.s.ring_bytes && h.tc_bt == t.s.batch_tiles;
+bool same_tc_shape(const nwc_handle_s& h, int cls, const nwc::TcShape& t) {
+  return h.tc_rows[cls] == t.rows && h.tc_teams[cls] == t.teams && h.tc_ctas[cls] == t.s.ctas &&
+         h.tc_ring[cls] == t.s.ring_bytes && h.tc_bstages[cls] == t.bstages &&
+         h.tc_ksplit[cls] == t.ksplit;
 }
 
-void note_tc_schedule(nwc_handle_s* h, const nwc::TcShape& t) {
-  h->tc_rows = t.rows;
-  h->tc_teams = t.teams;
-  h->tc_ctas = t.s.ctas;
-  h->tc_ring = t.s.ring_bytes;
-  h->tc_bt = t.s.batch_tiles;
+void note_tc_schedule(nwc_handle_s* h, int cls, const nwc::TcShape& t) {
+  h->tc_rows[cls] = t.rows;
+  h->tc_teams[cls] = t.teams;
+  h->tc_ctas[cls] = t.s.ctas;
+  h->tc_ring[cls] = t.s.ring_bytes;
+  h->tc_bstages[cls] = t.bstages;
+  h->tc_ksplit[cls] = t.ksplit;
 }
 
-// Writes the tensor-core schedule for shape t into the device image on
+// Writes tensor-core schedule cls for shape t into the device image on
 // `stream`, or into `image` (a host copy of the device image) when given.
-nwc_status write_tc_schedule(nwc_handle_s* h, const nwc::TcShape& t, uint8_t* image,
+nwc_status write_tc_schedule(nwc_handle_s* h, int cls, const nwc::TcShape& t, uint8_t* image,
                              cudaStream_t stream) {
+  const uint32_t raw = nwc::raw_bytes(h->tile_cols);
   if (image) {
-    nwc::build_tc_schedule(h->index.data(), h->tiles_r, h->tiles_c, t, image + tc_class_off(*h));
-    note_tc_schedule(h, t);
+    nwc::build_tc_schedule(h->index.data(), h->tiles_r, h->tiles_c, raw, t,
+                           image + tc_class_off(*h, cls));
+    note_tc_schedule(h, cls, t);
     return NWC_OK;
   }
   std::vector<uint8_t> sched;
@@ -144,11 +150,11 @@ nwc_status write_tc_schedule(nwc_handle_s* h, const nwc::TcShape& t, uint8_t* im
   } catch (const std::bad_alloc&) {
     return NWC_ERR_NOMEM;
   }
-  nwc::build_tc_schedule(h->index.data(), h->tiles_r, h->tiles_c, t, sched.data());
-  if (cudaMemcpyAsync(h->d_base + tc_class_off(*h), sched.data(), sched.size(),
+  nwc::build_tc_schedule(h->index.data(), h->tiles_r, h->tiles_c, raw, t, sched.data());
+  if (cudaMemcpyAsync(h->d_base + tc_class_off(*h, cls), sched.data(), sched.size(),
                       cudaMemcpyHostToDevice, stream) != cudaSuccess)
     return NWC_ERR_CUDA;
-  note_tc_schedule(h, t);
+  note_tc_schedule(h, cls, t);
   return NWC_OK;
 }
 
@@ -227,7 +233,7 @@ uint64_t scratch_bytes_for(const nwc_handle_s& h, int32_t batch, bool tensor_cor
   if (h.tiles_c <= 1) return 0;
   const int b = batch < kChunkBatch ? batch : kChunkBatch;
   return round_up(4ull * (uint64_t)h.tiles_r, 256) +
-         (tensor_cores ? nwc::tc_partial_bytes((uint64_t)h.tiles_c)
+         (tensor_cores ? nwc::tc_partial_bytes((uint64_t)h.tiles_r, (uint64_t)h.tiles_c)
                        : nwc::split_partial_bytes((uint64_t)h.tiles_r, (uint64_t)h.tiles_c,
                                                   (uint64_t)b));
 }
@@ -273,8 +279,12 @@ nwc_status init_schedule(nwc_handle_s* h, uint8_t* image, cudaStream_t stream) {
     nwc::build_schedule(h->index.data(), h->tiles, s, image + class_off(*h, cls));
     note_schedule(h, cls, s);
   }
-  nwc::TcShape ts;
-  if (tc_shape_on(*h, sms, smem, &ts)) return write_tc_schedule(h, ts, image, stream);
+  for (int cls = 0; cls < nwc::kTcClasses; ++cls) {
+    nwc::TcShape ts;
+    if (!tc_shape_on(*h, sms, smem, cls, &ts)) continue;
+    st = write_tc_schedule(h, cls, ts, image, stream);
+    if (st != NWC_OK) return st;
+  }
   return NWC_OK;
 }
 
@@ -557,7 +567,8 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
 nwc_status nwc_gemv_scratch_bytes(nwc_handle_t h, int32_t batch, uint64_t* bytes) {
   if (!h || !bytes || batch < 1 || batch > 64) return NWC_ERR_INVALID_ARG;
   *bytes = scratch_bytes_for(*h, batch, batch >= h->tc_min_batch && h->tc_min_batch > 0 &&
-                                              h->tc_rows > 0 && (h->cols % 8) == 0);
+                                              h->tc_rows[nwc::tc_class(batch)] > 0 &&
+                                              (h->cols % 8) == 0);
   return NWC_OK;
 }
 
@@ -596,15 +607,12 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// Accumulator columns of the tensor-core kernel for `batch` rows of x.
-int tc_columns(int32_t batch) { return batch <= 16 ? 16 : batch <= 32 ? 32 : 64; }
-
 // Whether a GEMV of `batch` rows takes the tensor-core kernel: at or above the
 // handle's threshold, when its shape fits this device and x can be read by TMA
 // (16-byte aligned rows).
 bool use_tensor_cores(const nwc_handle_s& h, const uint16_t* d_x, int32_t batch) {
   return h.tc_min_batch > 0 && batch >= h.tc_min_batch && batch <= nwc::kMaxTcRows &&
-         h.tc_rows > 0 && (h.cols % 8) == 0 && aligned(d_x, 16);
+         h.tc_rows[nwc::tc_class(batch)] > 0 && (h.cols % 8) == 0 && aligned(d_x, 16);
 }
 
 // The tensor-core launch: one kernel for up to 64 rows of x, every weight
@@ -615,18 +623,19 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
   size_t smem;
   nwc_status st = current_device(&dev, &sms, &smem);
   if (st != NWC_OK) return st;
+  const int cls = nwc::tc_class(batch);
   nwc::TcShape ts;
-  if (!tc_shape_on(*h, sms, smem, &ts)) return NWC_ERR_UNSUPPORTED;
+  if (!tc_shape_on(*h, sms, smem, cls, &ts)) return NWC_ERR_UNSUPPORTED;
   {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!same_tc_shape(*h, ts)) {
-      st = write_tc_schedule(h, ts, nullptr, cs);
+    if (!same_tc_shape(*h, cls, ts)) {
+      st = write_tc_schedule(h, cls, ts, nullptr, cs);
       if (st != NWC_OK) return st;
     }
   }
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (!encode) return NWC_ERR_UNSUPPORTED;
-  const int n = tc_columns(batch);
+  const int n = nwc::kTcColumns[cls];
   CUtensorMap tmap;
   const cuuint64_t dims[2] = {(cuuint64_t)h->cols, (cuuint64_t)batch};
   const cuuint64_t strides[1] = {(cuuint64_t)h->cols * 2};
@@ -638,8 +647,9 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
     return NWC_ERR_UNSUPPORTED;
   nwc::TileParams p;
   std::memset(&p, 0, sizeof(p));
-  const uint8_t* sched = h->d_base + tc_class_off(*h);
+  const uint8_t* sched = h->d_base + tc_class_off(*h, cls);
   p.tiles = h->d_base + h->tiles_off;
+  p.index = reinterpret_cast<const uint32_t*>(h->d_base + h->index_off);
   p.sched_cta = reinterpret_cast<const uint32_t*>(sched);
   p.sched_batch = reinterpret_cast<const uint4*>(sched + nwc::sched_batch_off());
   p.tile_ring = reinterpret_cast<const uint32_t*>(sched + nwc::sched_tc_ring_off((uint64_t)h->tiles));
@@ -668,6 +678,8 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
   p.tc_rows = ts.rows;
   p.tc_teams = ts.teams;
   p.tc_n = n;
+  p.tc_bstages = ts.bstages;
+  p.tc_ksplit = ts.ksplit;
   uint32_t cols = 32;
   while (cols < (uint32_t)(ts.teams * n)) cols <<= 1;
   p.tc_tmem_cols = cols;
@@ -853,29 +865,35 @@ nwc_status nwc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t 
 }
 
 nwc_status nwc_tc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
-                                    uint64_t smem_limit, nwc_tc_schedule_info* info,
-                                    uint32_t* cta_batch, uint32_t* batch, uint32_t* tile_ring,
-                                    uint32_t* tile_batch) {
-  if (!blob || !info || info->struct_size < sizeof(nwc_tc_schedule_info) || sm_count < 1)
+                                    uint64_t smem_limit, int32_t rows_of_x,
+                                    nwc_tc_schedule_info* info, uint32_t* cta_batch,
+                                    uint32_t* batch, uint32_t* tile_ring, uint32_t* tile_batch) {
+  if (!blob || !info || info->struct_size < sizeof(nwc_tc_schedule_info) || sm_count < 1 ||
+      rows_of_x < 1 || rows_of_x > nwc::kMaxTcRows)
     return NWC_ERR_INVALID_ARG;
   nwc_handle_s h;
   nwc_status st = parse(static_cast<const uint8_t*>(blob), blob_bytes, blob_bytes, &h, nullptr);
   if (st != NWC_OK) return st;
   nwc::TcShape ts;
-  if (!tc_shape_on(h, sm_count, (size_t)smem_limit, &ts)) return NWC_ERR_UNSUPPORTED;
+  if (!tc_shape_on(h, sm_count, (size_t)smem_limit, nwc::tc_class(rows_of_x), &ts))
+    return NWC_ERR_UNSUPPORTED;
   std::vector<uint8_t> sched;
   try {
     sched.resize(nwc::sched_tc_bytes((uint64_t)h.tiles));
   } catch (const std::bad_alloc&) {
     return NWC_ERR_NOMEM;
   }
-  nwc::build_tc_schedule(h.index.data(), h.tiles_r, h.tiles_c, ts, sched.data());
+  nwc::build_tc_schedule(h.index.data(), h.tiles_r, h.tiles_c, nwc::raw_bytes(h.tile_cols), ts,
+                         sched.data());
   const uint32_t* cb = reinterpret_cast<const uint32_t*>(sched.data());
   info->ctas = ts.s.ctas;
   info->rows = ts.rows;
   info->teams = ts.teams;
   info->batch_tiles = ts.s.batch_tiles;
   info->ring_bytes = ts.s.ring_bytes;
+  info->n = ts.n;
+  info->x_stages = ts.bstages;
+  info->ksplit = ts.ksplit;
   info->tiles = h.tiles;
   info->batches = cb[ts.s.ctas];
   info->smem_bytes = ts.s.smem_bytes;

@@ -109,9 +109,11 @@ constexpr int kStageClasses = 2;
 constexpr uint64_t sched_class_bytes(uint64_t tiles) {
   return round_up(sched_tile_off(tiles) + 4ull * tiles, 256);
 }
-// The tensor-core kernel's schedule follows the class schedules.  Its CTAs
-// take their tiles in another order (row panels, see kernels.cuh), so a copy
-// may move a single tile; it adds, per tile, the batch that brings it:
+// The tensor-core kernel's schedules (one per accumulator width) follow the
+// class schedules.  Their CTAs take their tiles in another order (row panels,
+// see kernels.cuh) and a copy moves one tile's lane lengths and streams (the
+// raw plane is read from global memory); they add, per tile, the batch that
+// brings it:
 //   u32 cta_batch[kMaxCtas + 1] | u32x4 batch[tiles + kMaxCtas]
 //   | u32 tile_ring[tiles] | u32 tile_batch[tiles]
 // tile_batch = batch index | (extra releases << 28): a batch of fewer tiles
@@ -124,8 +126,11 @@ constexpr uint64_t sched_tc_tbatch_off(uint64_t tiles) { return sched_tc_ring_of
 constexpr uint64_t sched_tc_bytes(uint64_t tiles) {
   return round_up(sched_tc_tbatch_off(tiles) + 4ull * tiles, 256);
 }
+// One tensor-core schedule per accumulator width (16, 32, 64 columns): the x
+// stage, and with it the ring, scales with the rows of x.
+constexpr int kTcSchedClasses = 3;
 constexpr uint64_t sched_bytes(uint64_t tiles) {
-  return kStageClasses * sched_class_bytes(tiles) + sched_tc_bytes(tiles);
+  return kStageClasses * sched_class_bytes(tiles) + kTcSchedClasses * sched_tc_bytes(tiles);
 }
 
 // Rows of x one launch of the CUDA-core GEMV kernel handles (one 16-row
@@ -140,8 +145,10 @@ constexpr int kMaxTcRows = 64;
 //   u32 arrival counters [tiles_r] | pad to 256
 //   FP32 partial sums: the split-K partials of one CUDA-core launch
 //   [tiles_c][kMaxPassRows][8 tiles_r], or the tensor-core kernel's partial row
-//   tiles at CTA boundaries [2 kMaxCtas][8][kMaxTcRows], whichever is larger;
-//   none when the matrix has one column tile.
+//   tiles when it splits K into ksplit parts [ksplit][tiles_r][kMaxTcRows][8],
+//   whichever is larger; none when the matrix has one column tile.  The
+//   tensor-core split is at most tc_max_ksplit(tiles_c), which keeps its part
+//   no larger than the CUDA-core one.
 constexpr uint64_t kScratchCountersOff = 256;
 constexpr uint64_t scratch_partial_off(uint64_t tiles_r) {
   return kScratchCountersOff + round_up(4ull * tiles_r, 256);
@@ -149,11 +156,16 @@ constexpr uint64_t scratch_partial_off(uint64_t tiles_r) {
 constexpr uint64_t split_partial_bytes(uint64_t tiles_r, uint64_t tiles_c, uint64_t rows_of_x) {
   return tiles_c <= 1 ? 0 : 4ull * tiles_c * rows_of_x * 8ull * tiles_r;
 }
-constexpr uint64_t tc_partial_bytes(uint64_t tiles_c) {
-  return tiles_c <= 1 ? 0 : 4ull * 2ull * kMaxCtas * 8ull * (uint64_t)kMaxTcRows;
+constexpr int64_t tc_max_ksplit(int64_t tiles_c) { return tiles_c >= 8 ? tiles_c / 4 : 1; }
+constexpr uint64_t tc_partial_bytes(uint64_t tiles_r, uint64_t tiles_c) {
+  return tc_max_ksplit((int64_t)tiles_c) <= 1
+             ? 0
+             : 4ull * (uint64_t)tc_max_ksplit((int64_t)tiles_c) * tiles_r * 8ull *
+                   (uint64_t)kMaxTcRows;
 }
 constexpr uint64_t scratch_bytes(uint64_t tiles_r, uint64_t tiles_c) {
-  const uint64_t a = split_partial_bytes(tiles_r, tiles_c, kMaxPassRows), b = tc_partial_bytes(tiles_c);
+  const uint64_t a = split_partial_bytes(tiles_r, tiles_c, kMaxPassRows),
+                 b = tc_partial_bytes(tiles_r, tiles_c);
   return round_up(scratch_partial_off(tiles_r) + (a > b ? a : b), 256);
 }
 

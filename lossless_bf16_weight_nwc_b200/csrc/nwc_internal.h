@@ -48,9 +48,11 @@ struct nwc_handle_s {
   // class) was written for (0: none yet).
   int sched_ctas[nwc::kStageClasses] = {}, sched_ring[nwc::kStageClasses] = {},
       sched_tiles_per_batch[nwc::kStageClasses] = {};
-  // Shape the tensor-core kernel's schedule was written for (tc_rows 0: none),
-  // and the smallest batch that takes that kernel (0: never).
-  int tc_ctas = 0, tc_ring = 0, tc_bt = 0, tc_rows = 0, tc_teams = 0;
+  // Shape each tensor-core schedule (one per accumulator width) was written
+  // for (tc_rows 0: none), and the smallest batch that takes that kernel (0:
+  // never).
+  int tc_ctas[3] = {}, tc_ring[3] = {}, tc_bstages[3] = {}, tc_rows[3] = {}, tc_teams[3] = {},
+      tc_ksplit[3] = {};
   int32_t tc_min_batch = 16;
 };
 

@@ -66,15 +66,16 @@ void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s
 
 namespace nwc {
 
-// The tensor-core kernel's CTAs take their tiles in row panels (see
-// kernels.cuh): for each M-group of R row tiles, round by round, each team's
-// column block, its present row tiles in order.  Those are consecutive in the
-// blob (u = j tiles_r + i), so each team's run of a round is one or more
-// copies of at most batch_tiles tiles.  Copies are placed in the ring first in,
-// first out, as in build_schedule, with fewer than kSlots outstanding; the
-// kernel's consumers wait until a copy is issued before they poll its slot.
-void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c, const TcShape& ts,
-                       uint8_t* out) {
+// The tensor-core kernel's CTAs take their tiles by rectangles (see
+// kernels.cuh): CTA c = rs ksplit + ks owns row range rs and column range ks;
+// for each M-group of R row tiles, round by round, each team's column block,
+// its row tiles in order.  Each tile is one copy of its lane lengths and
+// streams (the chunk after its raw plane, which the kernel reads from global
+// memory).  Copies are placed in the ring first in, first out, as in
+// build_schedule, with fewer than kSlots outstanding; the kernel's consumers
+// wait until a copy is issued before they poll its slot.
+void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c,
+                       uint32_t raw_bytes, const TcShape& ts, uint8_t* out) {
   const int64_t tiles = tiles_r * tiles_c;
   std::memset(out, 0, sched_tc_bytes((uint64_t)tiles));
   uint32_t* cta_batch = reinterpret_cast<uint32_t*>(out);
@@ -82,55 +83,37 @@ void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c, 
   uint32_t* tile_ring = reinterpret_cast<uint32_t*>(out + sched_tc_ring_off((uint64_t)tiles));
   uint32_t* tile_batch = reinterpret_cast<uint32_t*>(out + sched_tc_tbatch_off((uint64_t)tiles));
   const LaunchShape& s = ts.s;
-  const int BT = s.batch_tiles, R = ts.rows, TT = ts.teams;
+  const int R = ts.rows, TT = ts.teams;
+  const int64_t KS = ts.ksplit, row_ranges = s.ctas / ts.ksplit;
   const uint64_t ring = (uint64_t)s.ring_bytes;
   const int64_t max_outstanding = kSlots - 16;
-  struct Run {
-    int64_t u0;
-    int n;
-  };
-  std::vector<Run> runs;
+  std::vector<int64_t> order;
   std::vector<uint64_t> vstart;
   uint32_t g = 0;  // batches of the CTAs before this one
   for (int c = 0; c < s.ctas; ++c) {
-    const int64_t a = tiles * c / s.ctas, b = tiles * (c + 1) / s.ctas;
-    const int64_t i0 = a / tiles_c, i1 = (b - 1) / tiles_c;
-    const int64_t groups = (i1 - i0 + R) / R;
-    runs.clear();
-    for (int64_t gi = 0; gi < groups; ++gi) {
-      const int64_t ig = i0 + gi * R;
-      const int64_t rg = std::min<int64_t>(R, i1 + 1 - ig);
-      for (int64_t rho = 0; rho * TT < tiles_c; ++rho) {
-        for (int t = 0; t < TT; ++t) {
-          const int64_t j = rho * TT + t;
-          if (j >= tiles_c) break;
-          int64_t r = 0;
-          while (r < rg) {
-            const int64_t v = (ig + r) * tiles_c + j;
-            if (v < a || v >= b) {
-              ++r;
-              continue;
-            }
-            const int64_t r0 = r;
-            while (r < rg && (ig + r) * tiles_c + j < b && (ig + r) * tiles_c + j >= a &&
-                   r - r0 < BT)
-              ++r;
-            runs.push_back(Run{j * tiles_r + ig + r0, (int)(r - r0)});
-          }
+    const int64_t ks = c % KS, rs = c / KS;
+    const int64_t i_lo = tiles_r * rs / row_ranges, i_hi = tiles_r * (rs + 1) / row_ranges;
+    const int64_t j_lo = tiles_c * ks / KS, j_hi = tiles_c * (ks + 1) / KS;
+    order.clear();
+    for (int64_t ig = i_lo; ig < i_hi; ig += R) {
+      const int64_t rg = std::min<int64_t>(R, i_hi - ig);
+      for (int64_t j0 = j_lo; j0 < j_hi; j0 += TT) {
+        for (int t = 0; t < TT && j0 + t < j_hi; ++t) {
+          for (int64_t r = 0; r < rg; ++r) order.push_back((j0 + t) * tiles_r + ig + r);
         }
       }
     }
     cta_batch[c] = g;
-    const int64_t nb = (int64_t)runs.size();
+    const int64_t nb = (int64_t)order.size();
     vstart.assign((size_t)nb, 0);
     uint64_t vhead = 0;
     int64_t oldest = 0;
     for (int64_t k = 0; k < nb; ++k) {
-      const Run& run = runs[(size_t)k];
-      const uint32_t c0 = index[run.u0], c1 = index[run.u0 + run.n];
+      const int64_t u = order[(size_t)k];
+      const uint32_t c0 = index[u] + raw_bytes / 16, c1 = index[u + 1];
       const uint64_t bytes = 16ull * (c1 - c0);
       uint64_t at = vhead;
-      if (at % ring + bytes > ring) at += ring - at % ring;  // a batch never wraps
+      if (at % ring + bytes > ring) at += ring - at % ring;  // a copy never wraps
       vstart[(size_t)k] = at;
       while (oldest < k && vstart[(size_t)oldest] + ring < at + bytes) ++oldest;
       int64_t need = oldest;
@@ -140,11 +123,8 @@ void build_tc_schedule(const uint32_t* index, int64_t tiles_r, int64_t tiles_c, 
       d[1] = (uint32_t)bytes;
       d[2] = (uint32_t)(at % ring);
       d[3] = (uint32_t)need;
-      for (int q = 0; q < run.n; ++q) {
-        const int64_t u = run.u0 + q;
-        tile_ring[u] = (uint32_t)(at % ring + 16ull * (index[u] - c0));
-        tile_batch[u] = (uint32_t)k | (q == 0 ? (uint32_t)(BT - run.n) << 28 : 0u);
-      }
+      tile_ring[u] = (uint32_t)(at % ring);
+      tile_batch[u] = (uint32_t)k;
       vhead = at + bytes;
     }
     g += (uint32_t)nb;

@@ -2,11 +2,14 @@
 
 The kernel decodes each tile once into shared memory and multiplies it with
 every row of x on the tensor cores ("Unweight", "Direct GPU Decompression").
-Its CTAs own row panels (whole row tiles except at most one shared row tile at
-each end), so these shapes cover: a single column tile, many column tiles, a
-CTA owning less than one row tile, ragged rows and columns (a partial last
-64-column chunk read by TMA past the end of x), every tile width, both code
-limits, and every accumulator width (16, 32, 64 columns).
+Its CTAs own rectangles of tiles (a row range x a column range; K is split
+into several column ranges when a CTA would otherwise own too few rows to
+keep its decode warps busy, and the parts' sums meet in scratch slots), so
+these shapes cover: a single column tile, many column tiles, a K split in two
+and in four with ragged row ranges, fewer row tiles than SMs, ragged rows and
+columns (a partial last 64-column chunk read by TMA past the end of x), every
+tile width, both code limits, and every accumulator width (16, 32, 64
+columns).
 
 The tolerance is the parity tests' (per output and overall L2) against the
 oracle's FP64 GEMV over the original BF16 weights.
@@ -46,7 +49,7 @@ def tc_gemv(lib, m, x):
 
 SHAPES = [((8, 512), 512), ((300, 2000), 512), ((1024, 1024), 512), ((77, 1032), 512),
           ((129, 296), 256), ((40, 200), 128), ((17, 136), 64), ((4100, 96), 512),
-          ((2048, 4096), 512), ((520, 14336), 512), ((96, 512), 512)]
+          ((2048, 4096), 512), ((520, 14336), 512), ((96, 512), 512), ((1000, 8192), 512)]
 
 
 @pytest.mark.parametrize("lmax", [0, 12])

@@ -48,7 +48,9 @@ def corrupt_need(image, sched_class_off, batch=1):
     image[at:at + 4] = torch.tensor([batch + 1], dtype=torch.int32).view(torch.uint8).to(image.device)
 
 
-def layout(lib, m):
+def layout(lib, m, rows_of_x):
+    """Offsets of the class-0 schedule and of the tensor-core schedule for
+    rows_of_x rows (one per accumulator width: 16, 32, 64 columns)."""
     info = lib.nwc_handle_info(m.handle)
     lmax = int(m.image[12:16].cpu().numpy().view(np.uint32)[0])
     tiles = (m.rows + 7) // 8 * ((m.cols + 511) // 512)
@@ -56,7 +58,9 @@ def layout(lib, m):
     sched = r256(r256(info["blob_bytes"]) + table)
     batch_off = (4 * (KSLOTS_CTAS + 1) + 15) // 16 * 16
     class_bytes = r256(batch_off + 16 * ((tiles + 1) // 2 + KSLOTS_CTAS) + 4 * tiles)
-    return sched, sched + 2 * class_bytes
+    tc_bytes = r256(batch_off + 16 * (tiles + KSLOTS_CTAS) + 8 * tiles)
+    tc_class = 0 if rows_of_x <= 16 else 1 if rows_of_x <= 32 else 2
+    return sched, sched + 2 * class_bytes + tc_class * tc_bytes
 
 
 @pytest.mark.parametrize("batch", [1, 32])
@@ -68,7 +72,7 @@ def test_bounded_wait_gives_up_and_device_recovers(lib, orc, batch):
     xt = to_bf16(x)
     launches, tc = lib.nwc_gemv_path(m.handle, xt, batch)
     assert tc == (batch >= 16)
-    class0, tc_off = layout(lib, m)
+    class0, tc_off = layout(lib, m, batch)
     torch.cuda.synchronize()
     corrupt_need(m.image, tc_off if tc else class0)
     y = torch.zeros((batch, spec.rows), dtype=torch.float32, device="cuda")

@@ -1,12 +1,15 @@
-"""The tensor-core kernel's launch schedule, checked on the CPU (no GPU).
+"""The tensor-core kernel's launch schedules, checked on the CPU (no GPU).
 
-The kernel's CTA c owns the tiles [T c / C, T (c + 1) / C) of the row-major tile
-order v = i tiles_c + j and walks them in M-groups of R row tiles, round by
-round, team by team (team t takes column blocks t, t + teams, ...), row by row.
-This test restates that walk independently and checks that the schedule
-brings exactly those tiles, in that order, in copies of consecutive chunks
-that never wrap the ring, never overwrite a copy still outstanding, keep fewer
-than 64 copies outstanding, and are released exactly batch_tiles times.
+The kernel splits K into ksplit column ranges and the row tiles into
+ctas / ksplit row ranges (part k of n over m items: [m k / n, m (k + 1) / n));
+CTA c = rs ksplit + ks owns row range rs x column range ks and walks it in
+M-groups of R row tiles, round by round, team by team (team t takes column
+blocks j_lo + t, j_lo + t + teams, ...), row by row.  This test restates that
+walk independently and checks that each schedule (one per accumulator width)
+brings exactly those tiles' lane lengths and streams (the chunk after its raw
+plane), in that order, one copy per tile, never wrapping the ring, never
+overwriting a copy still outstanding, keeping fewer than 64 copies
+outstanding, and that every tile belongs to exactly one CTA.
 """
 import numpy as np
 import pytest
@@ -36,25 +39,27 @@ def header(blob):
     return rows, cols, tile_cols, tiles_r, tiles_c, index
 
 
-def walk(tiles_r, tiles_c, ctas, R, TT):
-    """Per CTA, its present tiles (blob index u) in the kernel's order."""
-    T = tiles_r * tiles_c
+def walk(tiles_r, tiles_c, ctas, R, TT, KS):
+    """Per CTA, its tiles (blob index u) in the kernel's order."""
+    assert ctas % KS == 0
+    RS = ctas // KS
     out = []
     for c in range(ctas):
-        a, b = T * c // ctas, T * (c + 1) // ctas
-        i0, i1 = a // tiles_c, (b - 1) // tiles_c
+        ks, rs = c % KS, c // KS
+        i_lo, i_hi = tiles_r * rs // RS, tiles_r * (rs + 1) // RS
+        j_lo, j_hi = tiles_c * ks // KS, tiles_c * (ks + 1) // KS
         seq = []
-        for ig in range(i0, i1 + 1, R):
-            rg = min(R, i1 + 1 - ig)
-            for rho in range((tiles_c + TT - 1) // TT):
+        ig = i_lo
+        while ig < i_hi:
+            rg = min(R, i_hi - ig)
+            j0 = j_lo
+            while j0 < j_hi:
                 for t in range(TT):
-                    j = rho * TT + t
-                    if j >= tiles_c:
+                    if j0 + t >= j_hi:
                         break
-                    for r in range(rg):
-                        v = (ig + r) * tiles_c + j
-                        if a <= v < b:
-                            seq.append(j * tiles_r + ig + r)
+                    seq += [(j0 + t) * tiles_r + ig + r for r in range(rg)]
+                j0 += TT
+            ig += R
         out.append(seq)
     return out
 
@@ -66,68 +71,88 @@ CASES = [(8, 512, 512), (300, 2000, 512), (1024, 1024, 512), (77, 1032, 512), (1
 
 @pytest.mark.parametrize("rows,cols,tile_cols", CASES)
 @pytest.mark.parametrize("sms,smem", [(148, 232448), (132, 232448), (7, 232448), (148, 200000)])
-def test_tc_schedule_invariants(rows, cols, tile_cols, sms, smem):
+@pytest.mark.parametrize("rows_of_x", [1, 32, 64])
+def test_tc_schedule_invariants(rows, cols, tile_cols, sms, smem, rows_of_x):
     blob = blob_of(rows, cols, tile_cols)
     _, _, _, tiles_r, tiles_c, index = header(blob)
     try:
-        info, cta, bat, ring, tb = lib.nwc_tc_schedule_describe(blob, sms, smem)
+        info, cta, bat, ring, tb = lib.nwc_tc_schedule_describe(blob, sms, smem, rows_of_x)
     except lib.NwcError as e:
         assert e.status == 2                     # UNSUPPORTED: no layout fits
         return
     T = tiles_r * tiles_c
-    C, R, TT, BT = info["ctas"], info["rows"], info["teams"], info["batch_tiles"]
+    C, R, TT, N, SB = info["ctas"], info["rows"], info["teams"], info["n"], info["x_stages"]
+    KS = info["ksplit"]
     ring_bytes = info["ring_bytes"]
-    assert C == min(T, sms, 256) and info["tiles"] == T
-    assert 1 <= TT <= 8 and 1 <= R <= 16 and R * TT <= 16 and TT <= tiles_c
-    assert info["smem_bytes"] <= smem
+    raw = 8 * tile_cols
+    # The split stays within the scratch slots: at most tiles_c / 4 parts.
+    assert KS == 1 or 2 <= KS <= tiles_c // 4
+    assert C % KS == 0 and C // KS == min(tiles_r, min(sms, 256) // KS)
+    assert info["tiles"] == T and info["batch_tiles"] == 1
+    assert N == (16 if rows_of_x <= 16 else 32 if rows_of_x <= 32 else 64)
+    assert 1 <= TT <= 15 and 1 <= R <= 16 and R * TT <= 30 and TT * N <= 512
+    assert TT <= -(-tiles_c // KS)
+    assert SB in (1, 2) and info["smem_bytes"] <= smem
     assert info["a_offset"] % 1024 == 0 and info["b_offset"] % 1024 == 0
     assert info["b_offset"] == info["a_offset"] + 2 * TT * R * 1024
-    assert info["ring_offset"] >= info["b_offset"] + 2 * TT * 8192
-    chunk = 16 * np.diff(index)
-    per_cta = -(-T // C)
-    assert ring_bytes >= min(R + 2 * BT, per_cta) * chunk.max()
+    assert info["ring_offset"] >= info["b_offset"] + TT * SB * N * 128
+    streams = 16 * np.diff(index) - raw
+    per_cta = -(-tiles_r // (C // KS)) * -(-tiles_c // KS)
+    assert ring_bytes >= min(R + 2, per_cta) * streams.max()
     seen = np.zeros(T, dtype=np.int64)
-    for c, seq in enumerate(walk(tiles_r, tiles_c, C, R, TT)):
+    for c, seq in enumerate(walk(tiles_r, tiles_c, C, R, TT, KS)):
         b0, b1 = int(cta[c]), int(cta[c + 1])
-        order = []
+        assert b1 - b0 == len(seq)
         vstart = []
         vhead = 0
-        for k in range(b1 - b0):
+        for k, u in enumerate(seq):
             off16, nbytes, at, need = (int(v) for v in bat[b0 + k])
-            # consecutive chunks starting at chunk off16
-            u0 = int(np.searchsorted(index, off16))
-            assert index[u0] == off16
-            n = int(np.searchsorted(index, off16 + nbytes // 16)) - u0
-            assert 1 <= n <= BT and 16 * (index[u0 + n] - index[u0]) == nbytes
+            # the tile's lane lengths and streams: after its raw plane
+            assert off16 == index[u] + raw // 16 and nbytes == 16 * index[u + 1] - 16 * off16
             assert at % 16 == 0 and at + nbytes <= ring_bytes
             assert need <= k and need >= k - KMAX_OUTSTANDING + 1
-            # first in, first out: the copy's bytes overlap no copy issued
-            # after the released ones [0, need)
             pos = vhead if vhead % ring_bytes + nbytes <= ring_bytes else \
                 vhead + ring_bytes - vhead % ring_bytes
             assert pos % ring_bytes == at
-            for q in range(need, k):
-                assert vstart[q][0] + vstart[q][1] <= pos or pos + nbytes <= vstart[q][0] + ring_bytes
+            for q in range(need, k):                    # no overlap with outstanding copies
                 assert pos - vstart[q][0] < ring_bytes
+                assert vstart[q][0] + vstart[q][1] <= pos or pos + nbytes <= vstart[q][0] + ring_bytes
             vstart.append((pos, nbytes))
             vhead = pos + nbytes
-            for q in range(n):
-                u = u0 + q
-                order.append(u)
-                assert ring[u] == at + 16 * (index[u] - index[u0])
-                assert tb[u] & 0x0FFFFFFF == k
-                assert tb[u] >> 28 == (BT - n if q == 0 else 0)
-        assert order == seq, c
-        for u in seq:
+            assert ring[u] == at and tb[u] == k
             seen[u] += 1
     assert (seen == 1).all()
 
 
-def test_tc_shape_takes_the_fewest_rounds():
-    """A 4096 x 4096 matrix gives each of 148 CTAs 28 tiles over at most 5 row
-    tiles: one M-group of 5 rows with 3 teams takes 3 rounds of column blocks,
-    where 4 rows x 4 teams would take 2 groups x 2 rounds."""
-    info = lib.nwc_tc_schedule_describe(blob_of(4096, 4096))[0]
-    assert (info["rows"], info["teams"]) == (5, 3)
-    tall = lib.nwc_tc_schedule_describe(blob_of(20000, 1024))[0]
-    assert tall["rows"] * tall["teams"] >= 14
+def rounds(info, tiles_r, tiles_c):
+    KS, RS = info["ksplit"], info["ctas"] // info["ksplit"]
+    rows_c, cols_c = -(-tiles_r // RS), -(-tiles_c // KS)
+    return -(-rows_c // info["rows"]) * -(-cols_c // info["teams"])
+
+
+def test_tc_shape_takes_the_fewest_rounds_with_every_warp_resident():
+    """A 4096 x 4096 matrix (512 x 8 tiles) on 148 SMs: K split in two, 74 row
+    ranges of 6 or 7 row tiles x 4 column blocks, one M-group of 7 rows and 4
+    teams: every decode warp decodes one tile, with every warp's streams
+    resident.  Without the split, 4 rows x 8 column blocks would take two
+    rounds of at most 30 warps."""
+    blob = blob_of(4096, 4096)
+    _, _, _, _, _, index = header(blob)
+    streams = int((16 * np.diff(index) - 4096).max())
+    for rows_of_x in (1, 64):
+        info = lib.nwc_tc_schedule_describe(blob, rows_of_x=rows_of_x)[0]
+        assert (info["ksplit"], info["ctas"], info["rows"], info["teams"]) == (2, 148, 7, 4)
+        assert rounds(info, 512, 8) == 1
+        assert info["ring_bytes"] >= 28 * streams
+
+
+@pytest.mark.parametrize("rows,cols,best", [(14336, 4096, 4), (4096, 14336, 4), (1024, 4096, 1),
+                                            (20000, 1024, 2)])
+def test_tc_shape_rounds_meet_the_bound(rows, cols, best):
+    """The fewest rounds any rectangle split can give: at least the tiles of
+    the largest rectangle over 30 decode warps."""
+    blob = blob_of(rows, cols)
+    tiles_r, tiles_c = rows // 8, cols // 512
+    info = lib.nwc_tc_schedule_describe(blob, rows_of_x=64)[0]
+    assert rounds(info, tiles_r, tiles_c) == best
+    assert best >= -(-(tiles_r * tiles_c) // (148 * 30))
