@@ -356,7 +356,7 @@ typedef struct {
   int32_t ctas, rows, teams, batch_tiles, ring_bytes, n, x_stages;
   int64_t tiles, batches;
   uint64_t smem_bytes, a_offset, b_offset, ring_offset;
-  int32_t ksplit;
+  int32_t ksplit, a_stages;
 } nwc_tc_schedule_info;
 nwc_status nwc_tc_schedule_describe(const void* blob, uint64_t blob_bytes, int32_t sm_count,
                                     uint64_t smem_limit, int32_t rows_of_x,

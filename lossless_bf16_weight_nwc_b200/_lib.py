@@ -44,7 +44,7 @@ class nwc_tc_schedule_info(ctypes.Structure):
                 ("tiles", ctypes.c_int64), ("batches", ctypes.c_int64),
                 ("smem_bytes", ctypes.c_uint64), ("a_offset", ctypes.c_uint64),
                 ("b_offset", ctypes.c_uint64), ("ring_offset", ctypes.c_uint64),
-                ("ksplit", ctypes.c_int32)]
+                ("ksplit", ctypes.c_int32), ("a_stages", ctypes.c_int32)]
 
 
 NWC_CODE_PREFIX, NWC_CODE_RANK = 0, 1

@@ -1169,34 +1169,61 @@ __device__ __forceinline__ void tmem_load<16>(uint32_t taddr, float (&v)[16]) {
   for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(r[k]);
 }
 
-// Barriers, the MMA warp's state and flags of the tensor-core kernel (at
-// p.tc_bar_off).
+// Barriers, counters and flags of the tensor-core kernel (at p.tc_bar_off).
 struct TcBars {
-  uint64_t* xfull;    // [team][2]: x chunk of the stage landed (TMA bytes)
-  uint64_t* sfull;    // [team][2]: the team's R decode warps wrote the A stage
-  uint64_t* sempty;   // [team][2]: the MMAs that read the stage completed
+  uint64_t* xfull;    // [team][2]: the x chunk of the stage landed (TMA bytes)
+  uint64_t* sempty;   // [team][kTcMaxAStages]: the MMAs that read the A stage completed
   uint64_t* accfull;  // [team]: the team's accumulator holds its M-group sum
   uint64_t* accempty; // the epilogue warps have read the accumulators
   uint32_t* tmem;     // TMEM base address (tcgen05.alloc writes it)
-  volatile uint32_t* abort;   // a wait gave up: leave
-  volatile uint32_t* issued;  // batches the producer has issued so far
-  uint32_t* mma;      // [7][team]: the MMA warp's counters (see tc_mma)
+  volatile uint32_t* abort;     // a wait gave up: leave
+  volatile uint32_t* issued;    // copies the producer has issued so far
+  uint32_t* arrived;            // [team][kTcMaxAStages]: decode warps done with the stage
+  volatile uint32_t* mma_next;  // [team]: chunks whose MMAs have been issued
+  uint32_t* xs;                 // x loader: [3][team] fetched, next in group, per group
 };
 __device__ __forceinline__ TcBars tc_bars(uint8_t* smem, const TileParams& p) {
   TcBars b;
   b.xfull = reinterpret_cast<uint64_t*>(smem + p.tc_bar_off);
-  b.sfull = b.xfull + 2 * kTcMaxTeams;
-  b.sempty = b.sfull + 2 * kTcMaxTeams;
-  b.accfull = b.sempty + 2 * kTcMaxTeams;
+  b.sempty = b.xfull + 2 * kTcMaxTeams;
+  b.accfull = b.sempty + kTcMaxAStages * kTcMaxTeams;
   b.accempty = b.accfull + kTcMaxTeams;
   b.tmem = reinterpret_cast<uint32_t*>(b.accempty + 1);
   b.abort = b.tmem + 1;
   b.issued = b.tmem + 2;
-  b.mma = b.tmem + 4;
+  b.arrived = b.tmem + 4;
+  b.mma_next = b.arrived + kTcMaxAStages * kTcMaxTeams;
+  b.xs = const_cast<uint32_t*>(b.mma_next) + kTcMaxTeams;
   return b;
 }
-static_assert(8 * (7 * kTcMaxTeams + 1) + 16 + 4 * 7 * kTcMaxTeams <= (int)kTcBarBytes,
+static_assert(8 * ((2 + kTcMaxAStages + 1) * kTcMaxTeams + 1) + 16 +
+                      4 * (kTcMaxAStages + 1 + 3) * kTcMaxTeams <=
+                  (int)kTcBarBytes,
               "tensor-core barrier area");
+
+// CTA-scope ordered accesses to shared-memory words.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_cta(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "r"(smem_u32(p)), "r"(v)
+               : "memory");
+  return old;
+}
+__device__ __forceinline__ uint32_t ld_acquire_cta(const volatile uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
+               : "=r"(v)
+               : "r"(smem_u32(const_cast<const uint32_t*>(p)))
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_cta(volatile uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(
+                   smem_u32(const_cast<const uint32_t*>(p))),
+               "r"(v)
+               : "memory");
+}
 
 // A consumer polls batch k's slot only once the producer has issued batch k:
 // the schedule keeps fewer than kSlots batches outstanding, so the slot's
@@ -1310,15 +1337,58 @@ __device__ __forceinline__ uint4 ldg_stream128(const uint8_t* p) {
   return v;
 }
 
+// Issues the MMAs of chunk c of team t: the four K = 16 steps of A stage
+// c % astages against x stage c % bstages into the team's accumulator, their
+// completion committed to the A stage's barrier (and, for the group's last
+// chunk, to the team's accumulator barrier).  Called by lane 0 of the decode
+// warp that finished the chunk last.  A team's chunks are issued in order:
+// chunk c waits for chunk c - 1's issue (mma_next), so the accumulation order
+// is fixed.  w is the chunk's index within its M-group gi, per_group the
+// team's chunks per group.
+__device__ bool tc_issue(const TileParams& p, const TcBars& tb, uint32_t a_area, uint32_t b_area,
+                         int t, uint32_t c, uint32_t w, uint32_t per_group, int gi,
+                         const WaitCtl& wc) {
+  for (uint32_t it = 0; ld_acquire_cta(&tb.mma_next[t]) != c; ++it) {
+    if (it >= wc.limit || *tb.abort) {
+      atomicOr(wc.err, kErrTimeout);
+      return false;
+    }
+  }
+  const uint32_t SB = (uint32_t)p.tc_bstages, NA = (uint32_t)p.tc_astages;
+  const uint32_t sx = c % SB, st = c % NA;
+  if (!wait_bounded(&tb.xfull[2 * t + (int)sx], (c / SB) & 1u, wc)) return false;
+  // The group's first MMA overwrites the accumulator: the epilogue of the
+  // previous group must have read it.
+  if (w == 0 && gi > 0 && !wait_bounded(tb.accempty, (uint32_t)(gi - 1) & 1u, wc)) return false;
+  tc_fence_after();
+  const uint32_t N = (uint32_t)p.tc_n;
+  const uint32_t a0 = a_area + ((uint32_t)t * NA + st) * (uint32_t)p.tc_rows * kTcStageA;
+  const uint32_t b0 = b_area + ((uint32_t)t * SB + sx) * N * 128u;
+  const uint32_t idesc = umma_idesc_bf16(128, (int)N);
+  const uint32_t d = *tb.tmem + (uint32_t)t * N;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    umma_bf16(d, umma_desc_sw128(a0 + 32u * k), umma_desc_sw128(b0 + 32u * k), idesc,
+              (w == 0 && k == 0) ? 0u : 1u);
+  umma_commit(&tb.sempty[kTcMaxAStages * t + (int)st]);
+  if (w + 1 == per_group) umma_commit(&tb.accfull[t]);
+  tc_fence_before();
+  st_release_cta(&tb.mma_next[t], c + 1);
+  return true;
+}
+
 // Decode warps (0 .. 29): warp w < teams R is slot r = w % R of team t = w / R.
 // A tile's lane lengths and streams come from the ring; its raw plane straight
-// from global memory, two 64-column groups ahead.  Warps 0 .. 15 also read the
+// from global memory, two 64-column groups ahead.  Each warp writes its row
+// tile's 8 x 64 chunk into the team's A stage; the warp that completes a
+// chunk for the team issues its MMAs.  Warps 0 .. 15 also read the
 // accumulators back after each M-group.
 template <int CP, int CODE, int S>
 __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, const TcBars& tb,
                           const TcWork& wk, int warp, int lane) {
   const WaitCtl wc = wait_ctl(p);
   const int R = p.tc_rows, TT = p.tc_teams;
+  const uint32_t NA = (uint32_t)p.tc_astages;
   const bool decoder = warp < TT * R;
   const bool epilogue = warp < kTcEpilogueWarps;
   const int t = warp / R, r = warp % R;
@@ -1327,7 +1397,9 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
   const uint32_t ring = smem_u32(s.ring);
   const uint32_t limit = ring + (uint32_t)p.ring_bytes + kRingSlack;
   const uint32_t a_area = smem_u32(smem + p.tc_a_off);
+  const uint32_t b_area = smem_u32(smem + p.tc_b_off);
   const int64_t nj = decoder && t < wk.teams ? (wk.j_hi - wk.j_lo - t + TT - 1) / TT : 0;
+  const uint32_t per_group = (uint32_t)nj * CP;
   const uint32_t chunk_lo = ((uint32_t)(2 * c) ^ (uint32_t)g) << 4;
   const uint32_t chunk_hi = ((uint32_t)(2 * c + 1) ^ (uint32_t)g) << 4;
   uint32_t seq = 0;
@@ -1359,14 +1431,15 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
         dec.init(stage + kLanes * S, start, limit, table);
       }
       for (int m = 0; m < CP; ++m, ++seq) {
-        const uint32_t st = seq & 1u, use = seq >> 1;
-        if (use > 0 &&
-            !__all_sync(kFull, wait_bounded(&tb.sempty[2 * t + st], (use - 1) & 1u, wc))) {
+        const uint32_t st = seq % NA, use = seq / NA;
+        // The stage's previous chunk (seq - NA) must have been multiplied.
+        if (use > 0 && !__all_sync(kFull, wait_bounded(&tb.sempty[kTcMaxAStages * t + (int)st],
+                                                       (use - 1) & 1u, wc))) {
           ok = false;
           break;
         }
         const uint32_t arow =
-            a_area + ((uint32_t)(2 * t + (int)st) * (uint32_t)R + (uint32_t)r) * kTcStageA +
+            a_area + (((uint32_t)t * NA + st) * (uint32_t)R + (uint32_t)r) * kTcStageA +
             (uint32_t)g * 128u;
         if (present) {
           const uint4 rv = rv0;
@@ -1385,9 +1458,22 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
         }
         // (A slot of a row past the group's last row tile keeps stale data:
         // it only reaches accumulator rows that the epilogue skips.)
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();  // this lane's A writes, before the MMAs read them
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tb.sfull[2 * t + st]);
+        uint32_t issued_ok = 1u;
+        if (lane == 0) {
+          // The R-th arrival of this use of the stage completes the chunk.
+          const uint32_t before = atom_add_acq_rel_cta(&tb.arrived[kTcMaxAStages * t + (int)st], 1u);
+          if (before + 1u == (use + 1u) * (uint32_t)R)
+            issued_ok = tc_issue(p, tb, a_area, b_area, t, seq,
+                                 (uint32_t)jj * CP + (uint32_t)m, per_group, gi, wc)
+                            ? 1u
+                            : 0u;
+        }
+        if (!__shfl_sync(kFull, issued_ok, 0)) {
+          ok = false;
+          break;
+        }
       }
       if (present && ok) {
         __syncwarp();
@@ -1422,114 +1508,85 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
   if (!ok && lane == 0) *tb.abort = 1u;
 }
 
-// The MMA warp: lane 0 loads x (TMA) into each team's B stage, issues the four
-// K = 16 MMAs of every chunk once the team's decode warps have written it, and
-// commits their completion to the stage's barrier (and at the end of an
-// M-group to the team's accumulator barrier).  It serves the teams in turn
-// without blocking on any of them.  Its per-team counters live in shared
-// memory (tb.mma), so the kernel fits the 64 registers of 1024 threads.
+// The x loader (lane 0 of warp 30): brings each team's x chunks into its x
+// stages by TMA, in the team's chunk order, as soon as the stage's previous
+// chunk has been multiplied.  It serves the teams in turn without blocking on
+// any of them; its per-team counters live in shared memory (tb.xs).
 template <int CP>
-__device__ void tc_mma(const TileParams& p, const CUtensorMap* tmap, uint8_t* smem,
-                       const TcBars& tb, const TcWork& wk) {
+__device__ void tc_xload(const TileParams& p, const CUtensorMap* tmap, uint8_t* smem,
+                         const TcBars& tb, const TcWork& wk) {
   const WaitCtl wc = wait_ctl(p);
-  const int R = p.tc_rows, TT = p.tc_teams, N = p.tc_n, SB = p.tc_bstages;
-  const uint32_t a_area = smem_u32(smem + p.tc_a_off), b_area = smem_u32(smem + p.tc_b_off);
-  const uint32_t bstage = (uint32_t)N * 128u;
-  const uint32_t idesc = umma_idesc_bf16(128, N);
-  const uint32_t tmem = *tb.tmem;
-  // Per team t: chunks whose x was fetched (nx) and that were multiplied (nm),
-  // out of total; the within-group index of the next chunk to fetch (xw) and
-  // to multiply (mw), the group of the latter (mg), and chunks per group.
-  uint32_t* nx = tb.mma;
-  uint32_t* nm = nx + kTcMaxTeams;
-  uint32_t* total = nm + kTcMaxTeams;
-  uint32_t* per_group = total + kTcMaxTeams;
-  uint32_t* xw = per_group + kTcMaxTeams;
-  uint32_t* mw = xw + kTcMaxTeams;
-  uint32_t* mg = mw + kTcMaxTeams;
+  const int TT = p.tc_teams;
+  const uint32_t SB = (uint32_t)p.tc_bstages, NA = (uint32_t)p.tc_astages;
+  const uint32_t b_area = smem_u32(smem + p.tc_b_off);
+  const uint32_t bstage = (uint32_t)p.tc_n * 128u;
+  uint32_t* nx = tb.xs;                       // chunks fetched
+  uint32_t* xw = nx + kTcMaxTeams;            // within-group index of the next
+  uint32_t* per_group = xw + kTcMaxTeams;     // chunks per group
   for (int t = 0; t < TT; ++t) {
     per_group[t] =
         t < wk.teams ? (uint32_t)((wk.j_hi - wk.j_lo - t + TT - 1) / TT) * CP : 0u;
-    total[t] = (uint32_t)wk.groups * per_group[t];
-    nx[t] = nm[t] = xw[t] = mw[t] = mg[t] = 0;
+    nx[t] = xw[t] = 0;
   }
   wait_prerequisites();  // x may be written by the previous kernel on the stream
   uint32_t idle = 0;
   for (;;) {
     bool done = true, moved = false;
     for (int t = 0; t < TT; ++t) {
-      uint32_t cm = nm[t], cx = nx[t];
-      const uint32_t tot = total[t];
-      if (cm >= tot) continue;
+      const uint32_t cx = nx[t], tot = (uint32_t)wk.groups * per_group[t];
+      if (cx >= tot) continue;
       done = false;
-      // x of chunk cx: its stage is free once the MMAs SB chunks back are done.
-      if (cx < tot && cx < cm + (uint32_t)SB) {
-        const uint32_t prev = cx - (uint32_t)SB;  // the chunk that last used the stage
-        if (cx < (uint32_t)SB ||
-            mbar_test_wait(&tb.sempty[2 * t + (int)(prev & 1u)], (prev >> 1) & 1u)) {
-          const uint32_t w = xw[t];
-          const int64_t j = wk.j_lo + t + (int64_t)(w / CP) * TT;
-          const int m = (int)(w % CP);
-          const uint32_t sx = cx % (uint32_t)SB;
-          mbar_expect_tx(&tb.xfull[2 * t + (int)sx], bstage);
-          tma_load_2d(b_area + (uint32_t)(t * SB + (int)sx) * bstage, tmap,
-                      (int32_t)(j * CP * 64 + m * 64), 0, &tb.xfull[2 * t + (int)sx]);
-          nx[t] = ++cx;
-          xw[t] = w + 1 == per_group[t] ? 0u : w + 1;
-          moved = true;
-        }
+      // x stage cx % SB is free once chunk cx - SB (A stage (cx - SB) % NA)
+      // has been multiplied.
+      if (cx >= SB) {
+        const uint32_t prev = cx - SB;
+        if (!mbar_test_wait(&tb.sempty[kTcMaxAStages * t + (int)(prev % NA)], (prev / NA) & 1u))
+          continue;
       }
-      // MMAs of chunk cm.
-      if (cm < cx) {
-        const uint32_t sa = cm & 1u, ph = (cm >> 1) & 1u;
-        const uint32_t sx = cm % (uint32_t)SB, phx = (cm / (uint32_t)SB) & 1u;
-        const uint32_t w = mw[t], grp = mg[t];
-        if (mbar_test_wait(&tb.xfull[2 * t + (int)sx], phx) &&
-            mbar_test_wait(&tb.sfull[2 * t + (int)sa], ph) &&
-            (w != 0 || grp == 0 || mbar_test_wait(tb.accempty, (grp - 1) & 1u))) {
-          tc_fence_after();
-          const uint32_t a0 = a_area + (uint32_t)(2 * t + (int)sa) * (uint32_t)R * kTcStageA;
-          const uint32_t b0 = b_area + (uint32_t)(t * SB + (int)sx) * bstage;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma_bf16(tmem + (uint32_t)(t * N), umma_desc_sw128(a0 + 32u * k),
-                      umma_desc_sw128(b0 + 32u * k), idesc, (w == 0 && k == 0) ? 0u : 1u);
-          umma_commit(&tb.sempty[2 * t + (int)sa]);
-          if (w + 1 == per_group[t]) {
-            umma_commit(&tb.accfull[t]);
-            mw[t] = 0;
-            mg[t] = grp + 1;
-          } else {
-            mw[t] = w + 1;
-          }
-          nm[t] = cm + 1;
-          moved = true;
-        }
-      }
+      const uint32_t w = xw[t];
+      const int64_t j = wk.j_lo + t + (int64_t)(w / CP) * TT;
+      const int m = (int)(w % CP);
+      const uint32_t sx = cx % SB;
+      mbar_expect_tx(&tb.xfull[2 * t + (int)sx], bstage);
+      tma_load_2d(b_area + ((uint32_t)t * SB + sx) * bstage, tmap, (int32_t)(j * CP * 64 + m * 64),
+                  0, &tb.xfull[2 * t + (int)sx]);
+      nx[t] = cx + 1;
+      xw[t] = w + 1 == per_group[t] ? 0u : w + 1;
+      moved = true;
     }
     if (done) break;
     if (moved) {
       idle = 0;
     } else if (++idle >= wc.limit || *tb.abort) {
-      atomicOr(wc.err, kErrTimeout);
+      if (!*tb.abort) atomicOr(wc.err, kErrTimeout);
       *tb.abort = 1u;
       break;
     }
   }
-  // Leave nothing in flight: x loads issued but not consumed, and the MMAs.
+}
+
+// After every decode warp has left: wait (bounded) for the x loads that no MMA
+// consumed and for the MMAs issued, so that nothing writes this CTA's shared
+// memory or TMEM once it is released.  On the ordinary path every load was
+// consumed and the epilogue saw every MMA complete; this matters after a wait
+// gave up.
+__device__ void tc_drain(const TileParams& p, const TcBars& tb) {
   const WaitCtl dc = drain_ctl(p);
-  for (int t = 0; t < TT; ++t) {
-    for (uint32_t k = nm[t]; k < nx[t]; ++k)
-      wait_bounded(&tb.xfull[2 * t + (int)(k % (uint32_t)SB)], (k / (uint32_t)SB) & 1u, dc);
-    if (nm[t] > 0)
-      wait_bounded(&tb.sempty[2 * t + (int)((nm[t] - 1) & 1u)], ((nm[t] - 1) >> 1) & 1u, dc);
+  const uint32_t SB = (uint32_t)p.tc_bstages, NA = (uint32_t)p.tc_astages;
+  for (int t = 0; t < p.tc_teams; ++t) {
+    const uint32_t issued = ld_acquire_cta(&tb.mma_next[t]);
+    for (uint32_t k = issued; k < tb.xs[t]; ++k)
+      wait_bounded(&tb.xfull[2 * t + (int)(k % SB)], (k / SB) & 1u, dc);
+    for (uint32_t k = issued > NA ? issued - NA : 0u; k < issued; ++k)
+      wait_bounded(&tb.sempty[kTcMaxAStages * t + (int)(k % NA)], (k / NA) & 1u, dc);
   }
 }
 
 // y[b][n] for up to kMaxTcRows rows b of x, every weight decoded once.
-// Warps 0..29 decode into the A stages (0..15 also read the accumulators
-// back), warp 30 allocates TMEM and issues x loads and MMAs, warp 31 moves the
-// compressed streams into the ring (the same producer as the other kernels).
+// Warps 0..29 decode into the A stages and issue the MMAs (0..15 also read
+// the accumulators back), warp 30 allocates TMEM and loads x, warp 31 moves
+// the compressed streams into the ring (the same producer as the other
+// kernels).
 template <int CP, int CODE, int S>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemv_tc_kernel(const TileParams p, const __grid_constant__ CUtensorMap tmap) {
@@ -1550,12 +1607,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s.full[k], 1);
       mbar_init(&s.empty[k], (uint32_t)p.batch_tiles);
     }
-    for (int k = 0; k < 2 * kTcMaxTeams; ++k) {
-      mbar_init(&tb.xfull[k], 1);
-      mbar_init(&tb.sfull[k], (uint32_t)p.tc_rows);
+    for (int k = 0; k < 2 * kTcMaxTeams; ++k) mbar_init(&tb.xfull[k], 1);
+    for (int k = 0; k < kTcMaxAStages * kTcMaxTeams; ++k) {
       mbar_init(&tb.sempty[k], 1);
+      tb.arrived[k] = 0u;
     }
-    for (int k = 0; k < kTcMaxTeams; ++k) mbar_init(&tb.accfull[k], 1);
+    for (int k = 0; k < kTcMaxTeams; ++k) {
+      mbar_init(&tb.accfull[k], 1);
+      tb.mma_next[k] = 0u;
+      tb.xs[k] = 0u;
+    }
     mbar_init(tb.accempty, kTcEpilogueWarps);
     *tb.abort = 0u;
     *tb.issued = 0u;
@@ -1585,13 +1646,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     __syncwarp();
   } else if (lane == 0) {
-    tc_mma<CP>(p, &tmap, smem, tb, wk);
+    tc_xload<CP>(p, &tmap, smem, tb, wk);
   }
   __syncwarp();
-  // Teardown: every decode warp and the MMA warp, then TMEM goes back.
+  // Teardown: every decode warp and the x loader, then what is still in
+  // flight, then TMEM goes back.
   tc_fence_before();
   named_barrier_sync(3, (kTcDecodeWarps + 1) * 32);
   if (warp == kTcMmaWarp) {
+    if (lane == 0) tc_drain(p, tb);
+    __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*tb.tmem),
                  "r"(p.tc_tmem_cols)
@@ -1780,10 +1844,11 @@ bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_streams, uint32_t t
   const uint32_t a_off = (bar_off + kTcBarBytes + 1023u) / 1024u * 1024u;
   const uint32_t bstage = (uint32_t)n * 128u;
   // Candidates in order of preference: every decode warp's streams resident
-  // (full), fewest rounds, smallest split, two x stages, largest ring.
+  // (full), fewest rounds, smallest split, two x stages, three A stages,
+  // largest ring.
   bool found = false;
   TcShape best{};
-  int64_t best_key[5] = {0, 0, 0, 0, 0};
+  int64_t best_key[6] = {0, 0, 0, 0, 0, 0};
   for (int64_t KS = 1; KS <= ks_max; ++KS) {
     int64_t row_ranges = cmax / KS;
     if (row_ranges > tiles_r) row_ranges = tiles_r;
@@ -1799,58 +1864,61 @@ bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_streams, uint32_t t
       if (tmax > 512 / n) tmax = 512 / n;
       for (int TT = tmax; TT >= 1; --TT) {
         for (int SB = 2; SB >= 1; --SB) {
-          const uint32_t b_off = a_off + (uint32_t)(2 * TT * R) * kTcStageA;
-          const size_t head = b_off + (size_t)(TT * SB) * bstage;
-          const size_t ring_offset = (head + 127) / 128 * 128;
-          if (smem_limit < ring_offset + kRingSlack) continue;
-          size_t ring = smem_limit - ring_offset - kRingSlack;
-          const size_t cap = (size_t)per_cta * (size_t)max_streams;
-          if (ring > cap) ring = cap;
-          ring = ring / 16 * 16;
-          // Deadlock-free: a team's run of R single-tile copies, one more, and
-          // the wrap-around of a copy (no more than the CTA's tiles).
-          int64_t need = (int64_t)R + 2;
-          if (need > per_cta) need = per_cta;
-          if (ring < (size_t)need * (size_t)max_streams) continue;
-          // The last A stage's 16 KiB operand window stays inside shared
-          // memory: the allocation is padded to cover it when the ring ends
-          // earlier.
-          const size_t window_end =
-              (size_t)a_off + (size_t)(2 * TT * R - 1) * kTcStageA + 16384;
-          size_t smem_bytes = ring_offset + ring + kRingSlack;
-          if (smem_bytes < window_end) smem_bytes = window_end;
-          if (smem_bytes > smem_limit) continue;
-          int64_t warps_resident = (int64_t)TT * R + 2;
-          if (warps_resident > per_cta) warps_resident = per_cta;
-          const int64_t full = ring >= (size_t)warps_resident * (size_t)max_streams ? 1 : 0;
-          const int64_t rounds = (rows_c + R - 1) / R * ((cols_c + TT - 1) / TT);
-          // Larger is better: resident, then -rounds, -split, stages, ring.
-          const int64_t key[5] = {full, -rounds, -KS, SB, (int64_t)ring};
-          bool better = !found;
-          for (int k = 0; k < 5 && !better; ++k) {
-            if (key[k] != best_key[k]) {
-              better = key[k] > best_key[k];
-              break;
+          for (int NA = kTcMaxAStages; NA >= 2; --NA) {
+            const uint32_t b_off = a_off + (uint32_t)(NA * TT * R) * kTcStageA;
+            const size_t head = b_off + (size_t)(TT * SB) * bstage;
+            const size_t ring_offset = (head + 127) / 128 * 128;
+            if (smem_limit < ring_offset + kRingSlack) continue;
+            size_t ring = smem_limit - ring_offset - kRingSlack;
+            const size_t cap = (size_t)per_cta * (size_t)max_streams;
+            if (ring > cap) ring = cap;
+            ring = ring / 16 * 16;
+            // Deadlock-free: a team's run of R single-tile copies, one more,
+            // and the wrap-around of a copy (no more than the CTA's tiles).
+            int64_t need = (int64_t)R + 2;
+            if (need > per_cta) need = per_cta;
+            if (ring < (size_t)need * (size_t)max_streams) continue;
+            // The last A stage's 16 KiB operand window stays inside shared
+            // memory: the allocation is padded to cover it when the ring ends
+            // earlier.
+            const size_t window_end =
+                (size_t)a_off + (size_t)(NA * TT * R - 1) * kTcStageA + 16384;
+            size_t smem_bytes = ring_offset + ring + kRingSlack;
+            if (smem_bytes < window_end) smem_bytes = window_end;
+            if (smem_bytes > smem_limit) continue;
+            int64_t warps_resident = (int64_t)TT * R + 2;
+            if (warps_resident > per_cta) warps_resident = per_cta;
+            const int64_t full = ring >= (size_t)warps_resident * (size_t)max_streams ? 1 : 0;
+            const int64_t rounds = (rows_c + R - 1) / R * ((cols_c + TT - 1) / TT);
+            // Larger is better: resident, -rounds, -split, x stages, A stages, ring.
+            const int64_t key[6] = {full, -rounds, -KS, SB, NA, (int64_t)ring};
+            bool better = !found;
+            for (int k = 0; k < 6 && !better; ++k) {
+              if (key[k] != best_key[k]) {
+                better = key[k] > best_key[k];
+                break;
+              }
             }
+            if (!better) continue;
+            found = true;
+            for (int k = 0; k < 6; ++k) best_key[k] = key[k];
+            best.rows = R;
+            best.teams = TT;
+            best.ksplit = (int)KS;
+            best.n = n;
+            best.bstages = SB;
+            best.astages = NA;
+            best.bar_off = bar_off;
+            best.a_off = a_off;
+            best.b_off = b_off;
+            best.s.ctas = (int)ctas;
+            best.s.table_bytes = table_bytes;
+            best.s.xstage_bytes = (uint32_t)(head - bar_off);
+            best.s.ring_offset = ring_offset;
+            best.s.ring_bytes = (int)ring;
+            best.s.batch_tiles = 1;
+            best.s.smem_bytes = smem_bytes;
           }
-          if (!better) continue;
-          found = true;
-          for (int k = 0; k < 5; ++k) best_key[k] = key[k];
-          best.rows = R;
-          best.teams = TT;
-          best.ksplit = (int)KS;
-          best.n = n;
-          best.bstages = SB;
-          best.bar_off = bar_off;
-          best.a_off = a_off;
-          best.b_off = b_off;
-          best.s.ctas = (int)ctas;
-          best.s.table_bytes = table_bytes;
-          best.s.xstage_bytes = (uint32_t)(head - bar_off);
-          best.s.ring_offset = ring_offset;
-          best.s.ring_bytes = (int)ring;
-          best.s.batch_tiles = 1;
-          best.s.smem_bytes = smem_bytes;
         }
       }
     }
@@ -1863,7 +1931,9 @@ cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int til
                            const TcShape& s, cudaStream_t stream) {
   if (p.batch < 1 || p.batch > kMaxTcRows || p.tc_teams < 1 || p.tc_teams > kTcMaxTeams ||
       p.tc_rows < 1 || p.tc_rows > 16 || p.tc_rows * p.tc_teams > kTcDecodeWarps ||
-      p.tc_ksplit < 1 || s.s.ctas % p.tc_ksplit != 0 ||
+      p.tc_ksplit < 1 || s.s.ctas % p.tc_ksplit != 0 || p.tc_astages < 2 ||
+      p.tc_astages > kTcMaxAStages || p.tc_bstages < 1 || p.tc_bstages > 2 ||
+      p.tc_bstages > p.tc_astages ||
       (p.tc_ksplit > 1 && p.tc_ksplit > tc_max_ksplit(p.tiles_c)))
     return cudaErrorInvalidValue;
   switch (tile_cols) {

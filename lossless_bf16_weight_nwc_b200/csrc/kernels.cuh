@@ -60,6 +60,7 @@ struct TileParams {
   const uint32_t* index;       // device: chunk offsets (16-byte units), tiles + 1
   const uint32_t* tile_batch;  // device: per tile, its copy's place in its CTA's schedule
   int32_t tc_bstages;       // x stages per team (1 or 2)
+  int32_t tc_astages;       // A stages per team (2 or 3)
   int32_t tc_rows;          // R: row tiles per M-group (rows of the MMA / 8)
   int32_t tc_teams;         // teams of R decode warps, each on its own column blocks
   int32_t tc_n;             // accumulator columns: rows of x padded to 16, 32 or 64
@@ -123,12 +124,13 @@ cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const Laun
 // costs about a quarter of its chunk.
 constexpr int kTcDecodeWarps = 30;
 constexpr int kTcEpilogueWarps = 16;  // 4 per TMEM lane quarter read the accumulators
-constexpr int kTcMmaWarp = 30;        // TMEM allocation, x loads (TMA), MMA issue
+constexpr int kTcMmaWarp = 30;        // TMEM allocation and x loads (TMA)
 constexpr int kTcProducerWarp = 31;   // bulk copies of the compressed streams
 constexpr int kTcThreads = 32 * 32;
 constexpr uint32_t kTcBarBytes = 2048;  // barriers, MMA-warp state, TMEM address, flags
 constexpr uint32_t kTcStageA = 1024;    // one row tile: 8 x 64 BF16
 constexpr int kTcMaxTeams = 15;
+constexpr int kTcMaxAStages = 3;        // A stages per team (decoded 64-column chunks)
 // Accumulator widths (rows of x padded): one launch shape and schedule each.
 constexpr int kTcClasses = 3;
 constexpr int kTcColumns[kTcClasses] = {16, 32, 64};
@@ -141,6 +143,7 @@ struct TcShape {
   int ksplit;          // column ranges (s.ctas is a multiple of it)
   int n;               // accumulator columns of the class
   int bstages;         // x stages per team (1 or 2)
+  int astages;         // A stages per team (2 or 3)
   uint32_t bar_off, a_off, b_off;  // shared-memory offsets
 };
 // Chooses the K split, R, the team count and the x stages for a matrix of

@@ -121,7 +121,7 @@ bool tc_shape_on(const nwc_handle_s& h, int sms, size_t smem, int cls, nwc::TcSh
 bool same_tc_shape(const nwc_handle_s& h, int cls, const nwc::TcShape& t) {
   return h.tc_rows[cls] == t.rows && h.tc_teams[cls] == t.teams && h.tc_ctas[cls] == t.s.ctas &&
          h.tc_ring[cls] == t.s.ring_bytes && h.tc_bstages[cls] == t.bstages &&
-         h.tc_ksplit[cls] == t.ksplit;
+         h.tc_ksplit[cls] == t.ksplit && h.tc_astages[cls] == t.astages;
 }
 
 void note_tc_schedule(nwc_handle_s* h, int cls, const nwc::TcShape& t) {
@@ -131,6 +131,7 @@ void note_tc_schedule(nwc_handle_s* h, int cls, const nwc::TcShape& t) {
   h->tc_ring[cls] = t.s.ring_bytes;
   h->tc_bstages[cls] = t.bstages;
   h->tc_ksplit[cls] = t.ksplit;
+  h->tc_astages[cls] = t.astages;
 }
 
 // Writes tensor-core schedule cls for shape t into the device image on
@@ -680,6 +681,7 @@ nwc_status gemv_run_tc(nwc_handle_s* h, const uint16_t* d_x, float* d_y, int32_t
   p.tc_n = n;
   p.tc_bstages = ts.bstages;
   p.tc_ksplit = ts.ksplit;
+  p.tc_astages = ts.astages;
   uint32_t cols = 32;
   while (cols < (uint32_t)(ts.teams * n)) cols <<= 1;
   p.tc_tmem_cols = cols;
@@ -894,6 +896,7 @@ nwc_status nwc_tc_schedule_describe(const void* blob, uint64_t blob_bytes, int32
   info->n = ts.n;
   info->x_stages = ts.bstages;
   info->ksplit = ts.ksplit;
+  info->a_stages = ts.astages;
   info->tiles = h.tiles;
   info->batches = cb[ts.s.ctas];
   info->smem_bytes = ts.s.smem_bytes;

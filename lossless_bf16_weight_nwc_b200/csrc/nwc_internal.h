@@ -52,7 +52,7 @@ struct nwc_handle_s {
   // for (tc_rows 0: none), and the smallest batch that takes that kernel (0:
   // never).
   int tc_ctas[3] = {}, tc_ring[3] = {}, tc_bstages[3] = {}, tc_rows[3] = {}, tc_teams[3] = {},
-      tc_ksplit[3] = {};
+      tc_ksplit[3] = {}, tc_astages[3] = {};
   int32_t tc_min_batch = 16;
 };
 

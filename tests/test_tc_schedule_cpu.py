@@ -94,7 +94,9 @@ def test_tc_schedule_invariants(rows, cols, tile_cols, sms, smem, rows_of_x):
     assert TT <= -(-tiles_c // KS)
     assert SB in (1, 2) and info["smem_bytes"] <= smem
     assert info["a_offset"] % 1024 == 0 and info["b_offset"] % 1024 == 0
-    assert info["b_offset"] == info["a_offset"] + 2 * TT * R * 1024
+    NA = info["a_stages"]
+    assert SB <= NA <= 3
+    assert info["b_offset"] == info["a_offset"] + NA * TT * R * 1024
     assert info["ring_offset"] >= info["b_offset"] + TT * SB * N * 128
     streams = 16 * np.diff(index) - raw
     per_cta = -(-tiles_r // (C // KS)) * -(-tiles_c // KS)
