@@ -66,7 +66,7 @@ def parse_args():
                          "unary code (NWR1, 7 ranks)")
     ap.add_argument("--tc-min-batch", type=int, default=None,
                     help="smallest batch that takes the tensor-core kernel (default: the "
-                         "library's, 16; 0 = never)")
+                         "library's, 17; 0 = never)")
     ap.add_argument("--report", action="store_true",
                     help="the five configurations as a markdown table (not the headline line)")
     ap.add_argument("--report-json", default=None, help="with --report: every line, to this file")

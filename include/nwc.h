@@ -256,8 +256,11 @@ nwc_status nwc_gemv(nwc_handle_t handle, const uint16_t* d_x, float* d_y,
  * (up to 64) on the tcgen05 tensor cores, accumulating in TMEM ("Unweight",
  * "Direct GPU Decompression": decompress into shared memory, then the tensor
  * cores).  A GEMV takes the tensor-core kernel when batch >= the handle's
- * threshold (16 by default), cols is a multiple of 8, d_x is 16-byte aligned
- * and the kernel's shared-memory layout fits the device.
+ * threshold, cols is a multiple of 8, d_x is 16-byte aligned and the kernel's
+ * shared-memory layout fits the device.  The default threshold is 17: on
+ * B200 one CUDA-core launch of up to 16 rows is faster than the tensor-core
+ * kernel, whose per-chunk synchronization costs more than it saves until a
+ * second CUDA-core launch would be needed.
  * nwc_gemv_set_tc_min_batch sets the threshold: 1..64, or 0 for never.
  * Errors: INVALID_ARG. */
 nwc_status nwc_gemv_set_tc_min_batch(nwc_handle_t handle, int32_t min_batch);

@@ -40,6 +40,7 @@ namespace {
 
 constexpr int kRingSlack = 512;                  // readers may run past a chunk (corrupt data)
 constexpr int kTablePieces = 8;                  // bulk copies that bring in the decode table
+static_assert(kTablePieces <= 32, "one table piece per producer lane");
 constexpr int kMaxPairSteps = 32;                // two-step reads per tile (8 groups x 4)
 constexpr uint32_t kPairReadSpan = 12 + 4 * kMaxPairSteps + 4;  // bytes one tile's reader may touch
 static_assert(kPairReadSpan <= kRingSlack, "a clamped reader must stay inside the ring slack");
@@ -86,6 +87,10 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+// Hint: bring `bytes` (a multiple of 16) of global memory into L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -540,49 +545,63 @@ __device__ __forceinline__ Smem carve(uint8_t* smem, const TileParams& p) {
 // for releases and issues the copies.  The loop body is a handful of
 // instructions, so the copies go out as fast as the ring allows.
 __device__ void produce(const TileParams& p, uint8_t* smem, const Smem& s, const uint4* desc,
-                        int nb, int lane, volatile uint32_t* issued = nullptr) {
-  if (lane == 0) {
-    // The decode table in kTablePieces copies, each CTA starting at a different
-    // piece, so that the CTAs do not all ask the same L2 lines at once.
-    mbar_expect_tx(s.table_bar, p.table_bytes);
+                        int nb, int lane, volatile uint32_t* issued = nullptr,
+                        uint32_t raw_prefetch = 0) {
+  // The decode table in kTablePieces copies, one per lane, each CTA starting
+  // at a different piece, so that the CTAs do not all ask the same L2 lines at
+  // once.
+  if (lane == 0) mbar_expect_tx(s.table_bar, p.table_bytes);
+  __syncwarp();
+  if (lane < kTablePieces) {
     const uint32_t piece = p.table_bytes / kTablePieces;
-    for (int k = 0; k < kTablePieces; ++k) {
-      const uint32_t off = ((blockIdx.x + k) % kTablePieces) * piece;
-      bulk_load(smem + off, reinterpret_cast<const uint8_t*>(p.table) + off, piece, s.table_bar);
-    }
+    const uint32_t off = ((blockIdx.x + lane) % kTablePieces) * piece;
+    bulk_load(smem + off, reinterpret_cast<const uint8_t*>(p.table) + off, piece, s.table_bar);
   }
+  // Lane l holds the descriptor of copy base + l (and the next window's in
+  // dn).  Every copy from k on whose releases (`need`) lane 0 has already
+  // observed goes out at once, one per lane; otherwise lane 0 waits for the
+  // next release.  With raw_prefetch, each copy's tile also has the raw plane
+  // before its streams (raw_prefetch bytes) prefetched into L2.
   const WaitCtl wc = wait_ctl(p);
-  const uint4 none = make_uint4(0u, 0u, 0u, 0u);
-  uint4 cur = lane < nb ? __ldg(desc + lane) : none;
-  uint4 nxt = 32 + lane < nb ? __ldg(desc + 32 + lane) : none;
+  const uint4 none = make_uint4(0u, 0u, 0u, ~0u);
+  uint4 d = lane < nb ? __ldg(desc + lane) : none;
+  uint4 dn = 32 + lane < nb ? __ldg(desc + 32 + lane) : none;
   uint32_t released = 0;  // batches whose release lane 0 has observed
-  int k = 0;
-  for (; k < nb; ++k) {
-    const int l = k & 31;
-    if (l == 0 && k) {
-      cur = nxt;
-      nxt = k + 32 + lane < nb ? __ldg(desc + k + 32 + lane) : none;
+  int k = 0, base = 0;
+  uint32_t ok = 1;
+  while (k < nb) {
+    if (k >= base + 32) {
+      base += 32;
+      d = dn;
+      dn = base + 32 + lane < nb ? __ldg(desc + base + 32 + lane) : none;
     }
-    const uint32_t src = __shfl_sync(kFull, cur.x, l);
-    const uint32_t bytes = __shfl_sync(kFull, cur.y, l);
-    const uint32_t at = __shfl_sync(kFull, cur.z, l);
-    const uint32_t need = __shfl_sync(kFull, cur.w, l);
-    uint32_t ok = 1;
-    if (lane == 0) {
-      for (; released < need; ++released) {
-        if (!wait_bounded(&s.empty[released % kSlots], (released / kSlots) & 1u, wc)) {
-          ok = 0;
-          break;
+    const int off = k - base;
+    const uint32_t seen = __shfl_sync(kFull, released, 0);
+    const uint32_t ready =
+        __ballot_sync(kFull, lane >= off && base + lane < nb && d.w <= seen) >> off;
+    const int run = ready == (kFull >> off) ? 32 - off : __ffs(~ready) - 1;
+    if (run == 0) {  // copy k waits for the releases it needs, in order
+      const uint32_t need = __shfl_sync(kFull, d.w, off);
+      if (lane == 0) {
+        for (; released < need; ++released) {
+          if (!wait_bounded(&s.empty[released % kSlots], (released / kSlots) & 1u, wc)) {
+            ok = 0;
+            break;
+          }
         }
       }
-      if (ok) {
-        uint64_t* bar = &s.full[k % kSlots];
-        mbar_expect_tx(bar, bytes);  // arrive (release) + byte count
-        bulk_load(s.ring + at, p.tiles + 16ull * src, bytes, bar);
-        if (issued) *issued = (uint32_t)(k + 1);
-      }
+      if (!__shfl_sync(kFull, ok, 0)) break;
+      continue;
     }
-    if (!__shfl_sync(kFull, ok, 0)) break;
+    if (lane >= off && lane < off + run) {
+      if (raw_prefetch) bulk_prefetch_l2(p.tiles + 16ull * d.x - raw_prefetch, raw_prefetch);
+      uint64_t* bar = &s.full[(base + lane) % kSlots];
+      mbar_expect_tx(bar, d.y);  // arrive (release) + byte count
+      bulk_load(s.ring + d.z, p.tiles + 16ull * d.x, d.y, bar);
+    }
+    k += run;
+    __syncwarp();
+    if (lane == 0 && issued) *issued = (uint32_t)k;
   }
   // Leave no copy in flight: batches [0, k) were issued, and those more than
   // kSlots back have been released, hence landed.
@@ -1178,7 +1197,6 @@ struct TcBars {
   uint32_t* tmem;     // TMEM base address (tcgen05.alloc writes it)
   volatile uint32_t* abort;     // a wait gave up: leave
   volatile uint32_t* issued;    // copies the producer has issued so far
-  uint32_t* arrived;            // [team][kTcMaxAStages]: decode warps done with the stage
   volatile uint32_t* mma_next;  // [team]: chunks whose MMAs have been issued
   uint32_t* xs;                 // x loader: [3][team] fetched, next in group, per group
 };
@@ -1191,39 +1209,13 @@ __device__ __forceinline__ TcBars tc_bars(uint8_t* smem, const TileParams& p) {
   b.tmem = reinterpret_cast<uint32_t*>(b.accempty + 1);
   b.abort = b.tmem + 1;
   b.issued = b.tmem + 2;
-  b.arrived = b.tmem + 4;
-  b.mma_next = b.arrived + kTcMaxAStages * kTcMaxTeams;
+  b.mma_next = b.tmem + 4;
   b.xs = const_cast<uint32_t*>(b.mma_next) + kTcMaxTeams;
   return b;
 }
-static_assert(8 * ((2 + kTcMaxAStages + 1) * kTcMaxTeams + 1) + 16 +
-                      4 * (kTcMaxAStages + 1 + 3) * kTcMaxTeams <=
+static_assert(8 * ((2 + kTcMaxAStages + 1) * kTcMaxTeams + 1) + 16 + 4 * (1 + 3) * kTcMaxTeams <=
                   (int)kTcBarBytes,
               "tensor-core barrier area");
-
-// CTA-scope ordered accesses to shared-memory words.
-__device__ __forceinline__ uint32_t atom_add_acq_rel_cta(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
-               : "=r"(old)
-               : "r"(smem_u32(p)), "r"(v)
-               : "memory");
-  return old;
-}
-__device__ __forceinline__ uint32_t ld_acquire_cta(const volatile uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];"
-               : "=r"(v)
-               : "r"(smem_u32(const_cast<const uint32_t*>(p)))
-               : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_cta(volatile uint32_t* p, uint32_t v) {
-  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(
-                   smem_u32(const_cast<const uint32_t*>(p))),
-               "r"(v)
-               : "memory");
-}
 
 // A consumer polls batch k's slot only once the producer has issued batch k:
 // the schedule keeps fewer than kSlots batches outstanding, so the slot's
@@ -1337,52 +1329,62 @@ __device__ __forceinline__ uint4 ldg_stream128(const uint8_t* p) {
   return v;
 }
 
+// Waits (bounded) for `parity` of `bar`, or gives up at once when another
+// warp of the CTA already gave up.
+__device__ bool wait_or_abort(uint64_t* bar, uint32_t parity, const WaitCtl& w,
+                              volatile uint32_t* abort) {
+  for (uint32_t it = 0; it < w.limit; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (it >= 2) __nanosleep(64);  // a long wait leaves the issue slots to the decoders
+  }
+  atomicOr(w.err, kErrTimeout);
+  return false;
+}
+
 // Issues the MMAs of chunk c of team t: the four K = 16 steps of A stage
 // c % astages against x stage c % bstages into the team's accumulator, their
 // completion committed to the A stage's barrier (and, for the group's last
-// chunk, to the team's accumulator barrier).  Called by lane 0 of the decode
-// warp that finished the chunk last.  A team's chunks are issued in order:
-// chunk c waits for chunk c - 1's issue (mma_next), so the accumulation order
-// is fixed.  w is the chunk's index within its M-group gi, per_group the
-// team's chunks per group.
+// chunk, to the team's accumulator barrier).  Called by lane 0 of the team's
+// leader warp once the team's warps have written the chunk, so a team's
+// chunks are issued by one thread in order.  w is the chunk's index within its
+// M-group gi, per_group the team's chunks per group.
 __device__ bool tc_issue(const TileParams& p, const TcBars& tb, uint32_t a_area, uint32_t b_area,
-                         int t, uint32_t c, uint32_t w, uint32_t per_group, int gi,
+                         int t, uint32_t c, uint32_t st, uint32_t w, uint32_t per_group, int gi,
                          const WaitCtl& wc) {
-  for (uint32_t it = 0; ld_acquire_cta(&tb.mma_next[t]) != c; ++it) {
-    if (it >= wc.limit || *tb.abort) {
-      atomicOr(wc.err, kErrTimeout);
-      return false;
-    }
-  }
   const uint32_t SB = (uint32_t)p.tc_bstages, NA = (uint32_t)p.tc_astages;
-  const uint32_t sx = c % SB, st = c % NA;
-  if (!wait_bounded(&tb.xfull[2 * t + (int)sx], (c / SB) & 1u, wc)) return false;
+  // x stage and its phase parity (one or two stages).
+  const uint32_t sx = SB == 2u ? (c & 1u) : 0u, phx = SB == 2u ? ((c >> 1) & 1u) : (c & 1u);
+  if (!wait_or_abort(&tb.xfull[2 * t + (int)sx], phx, wc, tb.abort)) return false;
   // The group's first MMA overwrites the accumulator: the epilogue of the
   // previous group must have read it.
-  if (w == 0 && gi > 0 && !wait_bounded(tb.accempty, (uint32_t)(gi - 1) & 1u, wc)) return false;
+  if (w == 0 && gi > 0 && !wait_or_abort(tb.accempty, (uint32_t)(gi - 1) & 1u, wc, tb.abort))
+    return false;
   tc_fence_after();
   const uint32_t N = (uint32_t)p.tc_n;
   const uint32_t a0 = a_area + ((uint32_t)t * NA + st) * (uint32_t)p.tc_rows * kTcStageA;
   const uint32_t b0 = b_area + ((uint32_t)t * SB + sx) * N * 128u;
   const uint32_t idesc = umma_idesc_bf16(128, (int)N);
   const uint32_t d = *tb.tmem + (uint32_t)t * N;
+  // The next 16 columns start 32 bytes further: 2 in the descriptor's start
+  // field (address / 16, which stays below 2^14 inside shared memory).
+  const uint64_t da = umma_desc_sw128(a0), db = umma_desc_sw128(b0);
+  umma_bf16(d, da, db, idesc, w == 0 ? 0u : 1u);
 #pragma unroll
-  for (int k = 0; k < 4; ++k)
-    umma_bf16(d, umma_desc_sw128(a0 + 32u * k), umma_desc_sw128(b0 + 32u * k), idesc,
-              (w == 0 && k == 0) ? 0u : 1u);
+  for (int k = 1; k < 4; ++k) umma_bf16(d, da + 2u * k, db + 2u * k, idesc, 1u);
   umma_commit(&tb.sempty[kTcMaxAStages * t + (int)st]);
   if (w + 1 == per_group) umma_commit(&tb.accfull[t]);
-  tc_fence_before();
-  st_release_cta(&tb.mma_next[t], c + 1);
+  tb.mma_next[t] = c + 1;  // read by the teardown (after a CTA barrier)
   return true;
 }
 
 // Decode warps (0 .. 29): warp w < teams R is slot r = w % R of team t = w / R.
 // A tile's lane lengths and streams come from the ring; its raw plane straight
 // from global memory, two 64-column groups ahead.  Each warp writes its row
-// tile's 8 x 64 chunk into the team's A stage; the warp that completes a
-// chunk for the team issues its MMAs.  Warps 0 .. 15 also read the
-// accumulators back after each M-group.
+// tile's 8 x 64 chunk into the team's A stage; the team's leader (slot 0)
+// issues each chunk's MMAs once the whole team has passed the team's named
+// barrier (bar.sync by all R warps, once per chunk, in lockstep).
+// Warps 0 .. 15 also read the accumulators back after each M-group.
 template <int CP, int CODE, int S>
 __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, const TcBars& tb,
                           const TcWork& wk, int warp, int lane) {
@@ -1402,46 +1404,50 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
   const uint32_t per_group = (uint32_t)nj * CP;
   const uint32_t chunk_lo = ((uint32_t)(2 * c) ^ (uint32_t)g) << 4;
   const uint32_t chunk_hi = ((uint32_t)(2 * c + 1) ^ (uint32_t)g) << 4;
-  uint32_t seq = 0;
+  uint32_t seq = 0, st = 0, use = 0;  // chunk count, its A stage (seq % NA) and use (seq / NA)
   bool ok = true;
-  for (int gi = 0; gi < wk.groups && ok; ++gi) {
+  // The loops run to the end even after a wait gave up (ok false, abort set):
+  // every warp must pass its team's barrier as often as the others.
+  for (int gi = 0; gi < wk.groups; ++gi) {
     const int64_t ig = wk.i_lo + (int64_t)gi * R;
     const int rg = (int)min((int64_t)R, wk.i_hi - ig);
     const int64_t i = ig + r;
-    for (int64_t jj = 0; jj < nj && ok; ++jj) {
+    for (int64_t jj = 0; jj < nj; ++jj) {
       const int64_t j = wk.j_lo + t + jj * TT;
       const bool present = r < rg;
       LaneDecoder<CODE, S> dec;
       const uint8_t* raw = nullptr;
       uint4 rv0 = make_uint4(0u, 0u, 0u, 0u), rv1 = rv0;
       uint32_t bw = 0;
-      if (present) {
+      if (ok && present) {
         const int64_t u = j * p.tiles_r + i;
         raw = p.tiles + 16ull * __ldg(p.index + u);
         rv0 = ldg_stream128(raw + lane * 16);  // groups 0 and 1, before the wait
         if (CP > 1) rv1 = ldg_stream128(raw + 512 + lane * 16);
         bw = __ldg(p.tile_batch + u);
         const uint32_t stage = ring + __ldg(p.tile_ring + u);
-        if (!wait_issued(tb, bw, wc) || !wait_batch(s, (int)bw, wc)) {
-          ok = false;
-          break;
+        ok = __all_sync(kFull, wait_issued(tb, bw, wc) &&
+                                   wait_or_abort(&s.full[bw % kSlots], (bw / kSlots) & 1u, wc,
+                                                 tb.abort));
+        if (ok) {
+          uint32_t start[S];
+          lane_stream_starts<S>(stage, 0, lane, start);
+          dec.init(stage + kLanes * S, start, limit, table);
+        } else if (lane == 0) {
+          *tb.abort = 1u;
         }
-        uint32_t start[S];
-        lane_stream_starts<S>(stage, 0, lane, start);
-        dec.init(stage + kLanes * S, start, limit, table);
       }
-      for (int m = 0; m < CP; ++m, ++seq) {
-        const uint32_t st = seq % NA, use = seq / NA;
+      for (int m = 0; m < CP; ++m, ++seq, st = st + 1u == NA ? 0u : st + 1u, use += st == 0u) {
         // The stage's previous chunk (seq - NA) must have been multiplied.
-        if (use > 0 && !__all_sync(kFull, wait_bounded(&tb.sempty[kTcMaxAStages * t + (int)st],
-                                                       (use - 1) & 1u, wc))) {
-          ok = false;
-          break;
+        if (ok && use > 0) {
+          ok = __all_sync(kFull, wait_or_abort(&tb.sempty[kTcMaxAStages * t + (int)st],
+                                               (use - 1) & 1u, wc, tb.abort));
+          if (!ok && lane == 0) *tb.abort = 1u;
         }
         const uint32_t arow =
             a_area + (((uint32_t)t * NA + st) * (uint32_t)R + (uint32_t)r) * kTcStageA +
             (uint32_t)g * 128u;
-        if (present) {
+        if (ok && present) {
           const uint4 rv = rv0;
           rv0 = rv1;
           if (m + 2 < CP) rv1 = ldg_stream128(raw + (m + 2) * 512 + lane * 16);
@@ -1459,20 +1465,19 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
         // (A slot of a row past the group's last row tile keeps stale data:
         // it only reaches accumulator rows that the epilogue skips.)
         fence_proxy_async_smem();  // this lane's A writes, before the MMAs read them
-        __syncwarp();
-        uint32_t issued_ok = 1u;
-        if (lane == 0) {
-          // The R-th arrival of this use of the stage completes the chunk.
-          const uint32_t before = atom_add_acq_rel_cta(&tb.arrived[kTcMaxAStages * t + (int)st], 1u);
-          if (before + 1u == (use + 1u) * (uint32_t)R)
-            issued_ok = tc_issue(p, tb, a_area, b_area, t, seq,
+        // Every warp of the team passes the team's barrier (bar.sync, so no
+        // warp can lap it) once per chunk, whatever happened; after it the
+        // leader (r = 0) issues the chunk's MMAs.
+        named_barrier_sync(kTcTeamBarrier0 + t, R * 32);
+        if (r == 0) {
+          uint32_t issued_ok = 1u;
+          if (lane == 0 && ok && !*tb.abort)
+            issued_ok = tc_issue(p, tb, a_area, b_area, t, seq, st,
                                  (uint32_t)jj * CP + (uint32_t)m, per_group, gi, wc)
                             ? 1u
                             : 0u;
-        }
-        if (!__shfl_sync(kFull, issued_ok, 0)) {
-          ok = false;
-          break;
+          ok = ok && __shfl_sync(kFull, issued_ok, 0);
+          if (!ok && lane == 0) *tb.abort = 1u;
         }
       }
       if (present && ok) {
@@ -1483,8 +1488,11 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
     if (!ok || !epilogue) continue;
     // Epilogue of the group, by warps 0 .. 15 (the others go on decoding).
     for (int tt = 0; tt < wk.teams && ok; ++tt)
-      ok = __all_sync(kFull, wait_bounded(&tb.accfull[tt], (uint32_t)gi & 1u, wc));
-    if (!ok) break;
+      ok = __all_sync(kFull, wait_or_abort(&tb.accfull[tt], (uint32_t)gi & 1u, wc, tb.abort));
+    if (!ok) {
+      if (lane == 0) *tb.abort = 1u;
+      continue;
+    }
     tc_fence_after();
     const uint32_t tmem = *tb.tmem;
     switch (p.tc_n) {
@@ -1500,9 +1508,8 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
     // completes this group's phase after their 16 arrivals), epilogue warp w
     // delivers row tile ig + w.
     if (p.tc_ksplit > 1) {
-      ok = __all_sync(kFull, wait_bounded(tb.accempty, (uint32_t)gi & 1u, wc));
-      if (!ok) break;
-      if (warp < rg) tc_reduce(p, ig + warp, lane);
+      ok = __all_sync(kFull, wait_or_abort(tb.accempty, (uint32_t)gi & 1u, wc, tb.abort));
+      if (ok && warp < rg) tc_reduce(p, ig + warp, lane);
     }
   }
   if (!ok && lane == 0) *tb.abort = 1u;
@@ -1561,6 +1568,8 @@ __device__ void tc_xload(const TileParams& p, const CUtensorMap* tmap, uint8_t* 
       if (!*tb.abort) atomicOr(wc.err, kErrTimeout);
       *tb.abort = 1u;
       break;
+    } else {
+      __nanosleep(64);  // leave the issue slots to the decode warps
     }
   }
 }
@@ -1574,7 +1583,7 @@ __device__ void tc_drain(const TileParams& p, const TcBars& tb) {
   const WaitCtl dc = drain_ctl(p);
   const uint32_t SB = (uint32_t)p.tc_bstages, NA = (uint32_t)p.tc_astages;
   for (int t = 0; t < p.tc_teams; ++t) {
-    const uint32_t issued = ld_acquire_cta(&tb.mma_next[t]);
+    const uint32_t issued = tb.mma_next[t];
     for (uint32_t k = issued; k < tb.xs[t]; ++k)
       wait_bounded(&tb.xfull[2 * t + (int)(k % SB)], (k / SB) & 1u, dc);
     for (uint32_t k = issued > NA ? issued - NA : 0u; k < issued; ++k)
@@ -1608,10 +1617,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&s.empty[k], (uint32_t)p.batch_tiles);
     }
     for (int k = 0; k < 2 * kTcMaxTeams; ++k) mbar_init(&tb.xfull[k], 1);
-    for (int k = 0; k < kTcMaxAStages * kTcMaxTeams; ++k) {
-      mbar_init(&tb.sempty[k], 1);
-      tb.arrived[k] = 0u;
-    }
+    for (int k = 0; k < kTcMaxAStages * kTcMaxTeams; ++k) mbar_init(&tb.sempty[k], 1);
     for (int k = 0; k < kTcMaxTeams; ++k) {
       mbar_init(&tb.accfull[k], 1);
       tb.mma_next[k] = 0u;
@@ -1633,7 +1639,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   if (warp == kTcProducerWarp) {
     const uint32_t b0 = __ldg(p.sched_cta + blockIdx.x), b1 = __ldg(p.sched_cta + blockIdx.x + 1);
-    produce(p, smem, s, p.sched_batch + b0, (int)(b1 - b0), lane, tb.issued);
+    // Each copy brings a tile's streams; its raw plane (read by the decode
+    // warps from global memory) is prefetched into L2 at the same time.
+    produce(p, smem, s, p.sched_batch + b0, (int)(b1 - b0), lane, tb.issued, CP * 512u);
     return;
   }
   if (warp < kTcDecodeWarps) {
@@ -1652,9 +1660,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // Teardown: every decode warp and the x loader, then what is still in
   // flight, then TMEM goes back.
   tc_fence_before();
-  named_barrier_sync(3, (kTcDecodeWarps + 1) * 32);
+  named_barrier_sync(kTcTeardownBarrier, (kTcDecodeWarps + 1) * 32);
   if (warp == kTcMmaWarp) {
-    if (lane == 0) tc_drain(p, tb);
+    // On the ordinary path every x load was consumed and the epilogue saw
+    // every MMA complete; only after a wait gave up is there anything to wait
+    // for.
+    if (lane == 0 && *tb.abort) tc_drain(p, tb);
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(*tb.tmem),

@@ -129,7 +129,9 @@ constexpr int kTcProducerWarp = 31;   // bulk copies of the compressed streams
 constexpr int kTcThreads = 32 * 32;
 constexpr uint32_t kTcBarBytes = 2048;  // barriers, MMA-warp state, TMEM address, flags
 constexpr uint32_t kTcStageA = 1024;    // one row tile: 8 x 64 BF16
-constexpr int kTcMaxTeams = 15;
+constexpr int kTcMaxTeams = 14;
+constexpr int kTcTeamBarrier0 = 1;      // named barrier of team t: 1 + t
+constexpr int kTcTeardownBarrier = 15;
 constexpr int kTcMaxAStages = 3;        // A stages per team (decoded 64-column chunks)
 // Accumulator widths (rows of x padded): one launch shape and schedule each.
 constexpr int kTcClasses = 3;

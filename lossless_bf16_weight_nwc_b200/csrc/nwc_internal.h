@@ -53,7 +53,7 @@ struct nwc_handle_s {
   // never).
   int tc_ctas[3] = {}, tc_ring[3] = {}, tc_bstages[3] = {}, tc_rows[3] = {}, tc_teams[3] = {},
       tc_ksplit[3] = {}, tc_astages[3] = {};
-  int32_t tc_min_batch = 16;
+  int32_t tc_min_batch = 17;
 };
 
 namespace nwc {

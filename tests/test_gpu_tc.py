@@ -75,13 +75,13 @@ def test_tc_every_width(lib, orc, batch):
 
 
 def test_tc_deterministic_and_default_threshold(lib, orc):
-    """Reruns give the same bits; batches of 16 and more take the tensor-core
-    kernel by default, smaller ones the CUDA-core kernel, and both meet the
-    tolerance."""
+    """Reruns give the same bits; batches of 17 and more take the tensor-core
+    kernel by default, up to 16 the CUDA-core kernel (one launch), and both
+    meet the tolerance."""
     spec = synth.MatrixSpec("w", 2048, 4096, "normal", 0.02, 0)
     w = synth.matrix(spec, 8)
     m = lib.CompressedMatrix.compress(w)
-    for batch, want_tc in ((8, False), (16, True), (40, True)):
+    for batch, want_tc in ((8, False), (16, False), (17, True), (40, True)):
         x = synth.activations(8, batch, spec.cols)
         xt = to_bf16(x)
         launches, tc = lib.nwc_gemv_path(m.handle, xt, batch)
@@ -123,6 +123,7 @@ def test_tc_llama_shapes_full_size(lib, orc, batch):
         seen.add((spec.rows, spec.cols))
         w = synth.head_matrix(spec, wl.seed) if spec is head else synth.matrix(spec, wl.seed)
         m = lib.CompressedMatrix.compress(w)
+        lib.nwc_gemv_set_tc_min_batch(m.handle, 1)
         x = synth.activations(wl.seed, batch, spec.cols)
         xt = to_bf16(x)
         assert lib.nwc_gemv_path(m.handle, xt, batch) == (1, True)

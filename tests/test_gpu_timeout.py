@@ -71,7 +71,7 @@ def test_bounded_wait_gives_up_and_device_recovers(lib, orc, batch):
     m = lib.CompressedMatrix.compress(w)
     xt = to_bf16(x)
     launches, tc = lib.nwc_gemv_path(m.handle, xt, batch)
-    assert tc == (batch >= 16)
+    assert tc == (batch >= 17)
     class0, tc_off = layout(lib, m, batch)
     torch.cuda.synchronize()
     corrupt_need(m.image, tc_off if tc else class0)
@@ -91,7 +91,7 @@ def test_bounded_wait_gives_up_and_device_recovers(lib, orc, batch):
     # scratch); the GEMV that follows is ordinary.
     h2 = lib.nwc_handle_from_device(m.image, m.image.numel())
     try:
-        lib.nwc_gemv_set_tc_min_batch(h2, 16)
+        lib.nwc_gemv_set_tc_min_batch(h2, 17)
         y2 = torch.full((batch, spec.rows), float("nan"), dtype=torch.float32, device="cuda")
         lib.nwc_gemv(h2, xt, y2, batch)
         torch.cuda.synchronize()
