@@ -503,7 +503,12 @@ def run_stack(args) -> None:
         "device_image_bytes_per_token": image_bytes,
         "footprint_ratio": weight_bytes / image_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": None,
+                     "frac": achieved / hbm,
+                     "traffic": profile_traffic(args.workload, batch),
+                     "traffic_basis": "DRAM bytes per GEMV launch, averaged over a token's "
+                                      "launches (committed ncu summary, current kernel source "
+                                      "only; else null)",
+                     "algorithmic_bytes_per_launch": alg / launches,
                      "peak_source": f"{peak_src} hbm_gbs (copy)", "kernel": kernel,
                      "basis": "algorithmic bytes of the token's GEMVs / graph time per token",
                      "tokens_per_s_ceiling_at_peak": hbm * 1e9 / alg},
@@ -779,7 +784,8 @@ def run_report(args) -> None:
     peak, compression ratio, the uncompressed cuBLAS time and the kernel
     path."""
     rows = [("single_1024", 1), ("attn_4096_outliers", 1), ("attn_4096_outliers", 4),
-            ("mlp_pair_t5", 1), ("mlp_pair_t5", 2), ("mlp_pair_t5", 8),
+            ("attn_4096_outliers", 16), ("attn_4096_outliers", 64),
+            ("mlp_pair_t5", 1), ("mlp_pair_t5", 2), ("mlp_pair_t5", 8), ("mlp_pair_t5", 64),
             ("qwen3_4b_stack", 1), ("llama31_8b_stack", 1), ("llama31_8b_stack", 16),
             ("llama31_8b_stack", 64)]
     lines = []
@@ -794,6 +800,7 @@ def run_report(args) -> None:
         line = run_stack(a) if stack else run_matrix(a)
         lines.append(line)
         print(f"{workload} b{batch}: {line['ms_per_step'] * 1e3:.2f} us", file=sys.stderr, flush=True)
+    gather = gather_report()
     print("| workload | batch | µs per step | effective GB/s | compressed GB/s | fraction of HBM "
           "peak | ratio | cuBLAS BF16 µs | kernel |")
     print("|---|---|---|---|---|---|---|---|---|")
@@ -806,10 +813,71 @@ def run_report(args) -> None:
         print(f"| {workload} | {batch} | {us:.2f} | {line['value']:.0f} | "
               f"{comp / (us * 1e-6) / 1e9:.0f} | {rf['frac']:.3f} ({rf['peak_source']}) | "
               f"{line['compression_ratio']:.3f} | {cb_us:.2f} | {line.get('kernel_path')} |")
+    print()
+    print("| row gather from the 151936 x 2560 lm_head | µs per call (L2 flushed) |")
+    print("|---|---|")
+    for name, us in gather:
+        print(f"| {name} | {us:.2f} |")
     if args.report_json:
         with open(args.report_json, "w") as f:
             for line in lines:
                 f.write(json.dumps(line) + "\n")
+            f.write(json.dumps({"gather_report": dict(gather)}) + "\n")
+
+
+def gather_report(calls: int = 64) -> list:
+    """Embedding lookup from the compressed Qwen3-4B-shaped lm_head
+    (151936 x 2560, tied embedding): n random rows per call (n = 1, 8), against
+    one GEMV of the same stack's 4096 x 2560 q projection at batch 1.  Each
+    call is timed alone with CUDA events after a 256 MiB write that evicts L2,
+    with fresh row ids per call; the gathered rows are checked bit for bit."""
+    import torch
+
+    from lossless_bf16_weight_nwc_b200 import _lib, synth
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl, layer0, head, _ = synth.stack_parts("qwen3_4b_stack")
+    w_head = synth.head_matrix(head, wl.seed)
+    m_head = _lib.CompressedMatrix.compress(w_head, device=dev)
+    q = layer0[0]
+    w_q = synth.matrix(q, wl.seed)
+    m_q = _lib.CompressedMatrix.compress(w_q, device=dev)
+    x = torch.from_numpy(synth.activations(wl.seed, 1, q.cols).view(np.int16)).view(
+        torch.bfloat16).to(dev)
+    y = torch.empty((1, q.rows), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rng = np.random.default_rng(11)
+    out = []
+
+    def timed(fn):
+        for _ in range(3):
+            fn(0)
+        torch.cuda.synchronize()
+        durs = []
+        for i in range(calls):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn(i)
+            e1.record()
+            torch.cuda.synchronize()
+            durs.append(e0.elapsed_time(e1) * 1e3)
+        return statistics.median(durs)
+
+    for n in (1, 8):
+        ids = [torch.from_numpy(rng.integers(0, head.rows, n).astype(np.int32)).to(dev)
+               for _ in range(calls)]
+        got = m_head.gather_rows(ids[0])
+        assert np.array_equal(got.view(torch.int16).cpu().numpy().view(np.uint16),
+                              w_head[ids[0].cpu().numpy()]), "gather parity"
+        out.append((f"gather {n} row{'s' if n > 1 else ''}",
+                    timed(lambda i: m_head.gather_rows(ids[i]))))
+    out.append(("GEMV 4096 x 2560 (q projection), batch 1",
+                timed(lambda i: _lib.nwc_gemv(m_q.handle, x, y, 1))))
+    st, word = m_head.device_error()
+    assert st == 0, ("device error", st, word)
+    m_head.close()
+    m_q.close()
+    return out
 
 
 

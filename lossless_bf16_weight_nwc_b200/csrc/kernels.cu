@@ -109,6 +109,9 @@ __device__ __forceinline__ WaitCtl wait_ctl(const TileParams& p) {
 __device__ __forceinline__ WaitCtl drain_ctl(const TileParams& p) {
   return WaitCtl{p.err, p.wait_limit > kDefaultWaitLimit ? p.wait_limit : kDefaultWaitLimit};
 }
+__device__ __forceinline__ WaitCtl drain_ctl_default(uint32_t* err) {
+  return WaitCtl{err, kDefaultWaitLimit};
+}
 // Polls `bar` for `parity` at most w.limit times; on failure records a
 // timeout in the handle's error word.
 __device__ bool wait_bounded(uint64_t* bar, uint32_t parity, const WaitCtl& w) {
@@ -988,33 +991,48 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
 }
 
 // Row gather ("NWC", "How it works > Dequantization and embedding lookup": the
-// same decoder serves row lookups).  Persistent CTAs take the requested rows in
-// turn; each first copies the decode table into shared memory.  For a row, warp
-// w takes column blocks w, w + warps, ...: it stages the tile's lane lengths
-// and bit streams in shared memory with coalesced 16-byte loads, finds every
-// lane's stream start by a warp prefix sum, and the four lanes that own the
-// row's tile row (lane 4g + c owns row g) decode it with the GEMV's reader,
-// taking the raw plane straight from global memory.  Only the tiles of the
-// requested rows are read.
+// same decoder serves row lookups).  CTA i takes requested rows i, i + CTAs,
+// ...; for a row, warp w takes column blocks w, w + warps, ...  The decode
+// table arrives by bulk copy (lanes 0 .. 7 of warp 0 issue its pieces) while
+// every warp fetches its first tile: the chunk offsets, the raw plane
+// (straight into registers, all of it at once) and the lane lengths and
+// streams (into the warp's shared-memory stage with coalesced 16-byte loads).
+// A warp prefix sum gives every lane's stream start, and the four lanes that
+// own the row's tile row (lane 4g + c owns row g) decode it with the GEMV's
+// reader.  Only the tiles of the requested rows are read.
 constexpr int kGatherWarps = 8;
+constexpr uint32_t kGatherBarBytes = 16;  // table barrier, between table and stages
 
 template <int CP, int CODE, int S>
 __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams p) {
   extern __shared__ __align__(16) uint8_t gsm[];
   constexpr int kRaw = CP * 512;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (uint32_t o = 16 * threadIdx.x; o < p.table_bytes; o += 16 * blockDim.x)
-    *reinterpret_cast<uint4*>(gsm + o) =
-        __ldg(reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.table) + o));
+  uint64_t* tbar = reinterpret_cast<uint64_t*>(gsm + p.table_bytes);
+  if (threadIdx.x == 0) {
+    mbar_init(tbar, 1);
+    fence_barrier_init();
+  }
   __syncthreads();
+  if (warp == 0) {
+    if (lane == 0) mbar_expect_tx(tbar, p.table_bytes);
+    __syncwarp();
+    if (lane < kTablePieces) {
+      const uint32_t piece = p.table_bytes / kTablePieces;
+      const uint32_t off = ((blockIdx.x + lane) % kTablePieces) * piece;
+      bulk_load(gsm + off, reinterpret_cast<const uint8_t*>(p.table) + off, piece, tbar);
+    }
+  }
+  const WaitCtl wc{p.err, kDefaultWaitLimit};
   const uint32_t table = smem_u32(gsm);
-  uint8_t* stage = gsm + p.table_bytes + (size_t)warp * p.stage_bytes;
+  uint8_t* stage = gsm + p.table_bytes + kGatherBarBytes + (size_t)warp * p.stage_bytes;
   const uint32_t sbase = smem_u32(stage);
   const uint32_t limit = sbase + p.stage_bytes;
   const int g = lane >> 2, c = lane & 3;
   const bool vec = (p.cols % 8 == 0) && ((reinterpret_cast<uintptr_t>(p.out) & 15) == 0);
   uint32_t invalid = 0;
-  for (int64_t i = blockIdx.x; i < p.n; i += gridDim.x) {
+  bool have_table = false, ok = true;
+  for (int64_t i = blockIdx.x; i < p.n && ok; i += gridDim.x) {
     const int32_t row = __ldg(p.row_ids + i);
     if (row < 0 || row >= p.rows) {
       if (threadIdx.x == 0) atomicOr(p.err, kErrRange);
@@ -1025,24 +1043,48 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
       const int64_t u = j * p.tiles_r + row / kTileRows;
       const uint32_t c0 = __ldg(p.index + u), c1 = __ldg(p.index + u + 1);
       const uint8_t* chunk = p.tiles + 16ull * c0;
+      const bool mine = g == row % kTileRows;
+      uint4 rv[CP];
+      if (mine) {
+#pragma unroll
+        for (int m = 0; m < CP; ++m)
+          rv[m] = __ldg(reinterpret_cast<const uint4*>(chunk + m * 512 + lane * 16));
+      }
       // Lane lengths and streams: the chunk after its raw plane, clamped to the
       // stage (a corrupt index can misdecode but not overrun it).
       uint32_t bytes = 16u * (c1 - c0) > (uint32_t)kRaw ? 16u * (c1 - c0) - (uint32_t)kRaw : 0u;
       if (bytes > p.stage_bytes - kRingSlack) bytes = p.stage_bytes - kRingSlack;
       __syncwarp();
-      for (uint32_t o = 16 * lane; o < bytes; o += 16 * 32)
-        *reinterpret_cast<uint4*>(stage + o) = __ldg(reinterpret_cast<const uint4*>(chunk + kRaw + o));
+      {
+        uint4 sv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t o = 16u * lane + 512u * q;
+          if (o < bytes) sv[q] = __ldg(reinterpret_cast<const uint4*>(chunk + kRaw + o));
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t o = 16u * lane + 512u * q;
+          if (o < bytes) *reinterpret_cast<uint4*>(stage + o) = sv[q];
+        }
+        for (uint32_t o = 16u * lane + 2048u; o < bytes; o += 512u)
+          *reinterpret_cast<uint4*>(stage + o) = __ldg(reinterpret_cast<const uint4*>(chunk + kRaw + o));
+      }
       __syncwarp();
       uint32_t start[S];
       lane_stream_starts<S>(sbase, 0, lane, start);
-      if (g != row % kTileRows) continue;
+      if (!have_table) {
+        have_table = __all_sync(kFull, wait_bounded(tbar, 0, wc));
+        if (!have_table) {
+          ok = false;
+          break;
+        }
+      }
+      if (!mine) continue;
       LaneDecoder<CODE, S> dec;
       dec.init(sbase + kLanes * S, start, limit, table);
-      uint4 rv = __ldg(reinterpret_cast<const uint4*>(chunk + lane * 16));
-#pragma unroll 1
+#pragma unroll
       for (int m = 0; m < CP; ++m) {
-        const uint4 cur = rv;
-        if (m + 1 < CP) rv = __ldg(reinterpret_cast<const uint4*>(chunk + (m + 1) * 512 + lane * 16));
         uint32_t wv[8];
 #pragma unroll
         for (int r = 0; r < 8; r += 4) {
@@ -1051,7 +1093,7 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             invalid |= e[k];
-            wv[r + k] = assemble<CODE>(raw_pair_r(cur, r + k), e[k]);
+            wv[r + k] = assemble<CODE>(raw_pair_r(rv[m], r + k), e[k]);
           }
         }
         const int64_t col = j * (CP * 64) + m * 64 + 16 * c;
@@ -1071,6 +1113,9 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
     }
   }
   if (invalid & kEntryInvalid) atomicOr(p.err, kErrCorrupt);
+  // The table copy must have landed before the CTA's shared memory is
+  // released, also in a CTA that had no valid row to decode.
+  if (threadIdx.x == 0 && !have_table) wait_bounded(tbar, 0, drain_ctl_default(p.err));
 }
 
 // ---- tensor-core path: decode once into shared memory, tcgen05 MMA ---------
@@ -1979,7 +2024,8 @@ cudaError_t launch_gather(const GatherParams& g, int sm_count, cudaStream_t stre
   if (g.n < 1) return cudaErrorInvalidValue;
   const int64_t want = 2 * (int64_t)(sm_count > 0 ? sm_count : 1);
   const int ctas = (int)(g.n < want ? g.n : want);
-  const size_t smem = (size_t)g.table_bytes + (size_t)kGatherWarps * g.stage_bytes;
+  const size_t smem =
+      (size_t)g.table_bytes + kGatherBarBytes + (size_t)kGatherWarps * g.stage_bytes;
   const int code = g.code;
   switch (g.tile_cols) {
     case 512: return code == kCodeRank ? launch_gather_t<8, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<8, kCode14>(g, ctas, smem, stream) : launch_gather_t<8, kCode12>(g, ctas, smem, stream);
