@@ -173,51 +173,73 @@ class Tuner:
              reps: int = 50, retune: bool = False) -> Choice:
         """The fastest candidate for this matrix shape and batch on the current
         device (from the cache unless retune)."""
+        return self.tune_batches(w_host, [batch], candidates, reps, retune)[batch]
+
+    def tune_batches(self, w_host: np.ndarray, batches: Iterable[int],
+                     candidates: Iterable[Strategy] | None = None, reps: int = 50,
+                     retune: bool = False) -> dict:
+        """tune for several batches at once: each format is compressed once and
+        timed at every batch that is not cached yet.  Returns {batch: Choice}."""
         w_host = np.ascontiguousarray(w_host, dtype=np.uint16)
         if w_host.ndim != 2:
             raise ValueError("w_host: a 2-D matrix of BF16 bit patterns")
-        if not 1 <= batch <= 64:
+        batches = list(dict.fromkeys(int(b) for b in batches))
+        if not batches or not all(1 <= b <= 64 for b in batches):
             raise ValueError("batch: 1..64")
         rows, cols = w_host.shape
-        key = _key(self._name(), rows, cols, batch)
-        if not retune and key in self.cache:
-            return Choice.from_json(self.cache[key])
-        cands = validate_candidates(default_candidates(batch) if candidates is None
-                                    else candidates)
+        name = self._name()
+        out, todo = {}, []
+        for b in batches:
+            key = _key(name, rows, cols, b)
+            if not retune and key in self.cache:
+                out[b] = Choice.from_json(self.cache[key])
+            else:
+                todo.append(b)
+        if not todo:
+            return out
+        cands = {b: validate_candidates(default_candidates(b) if candidates is None
+                                        else candidates) for b in todo}
         compress = self._compress or self._compress_default
         timer = self._timer or time_gemv
         set_kernel = self._set_kernel or apply
-        x = self._activations(batch, cols)
-        timings, refused = {}, {}
+        xs = {b: self._activations(b, cols) for b in todo}
+        timings = {b: {} for b in todo}
+        refused = {}
         formats: dict[tuple, list[Strategy]] = {}
-        for s in cands:
-            formats.setdefault(s.format, []).append(s)
+        for b in todo:
+            for st in cands[b]:
+                formats.setdefault(st.format, [])
+                if st not in formats[st.format]:
+                    formats[st.format].append(st)
         for fmt, strategies in formats.items():
             try:
                 m = compress(w_host, strategies[0])
             except RuntimeError as e:  # e.g. a code limit too short for the matrix
-                for s in strategies:
-                    refused[s.key] = str(e)
+                for st in strategies:
+                    refused[st.key] = str(e)
                 continue
             try:
-                for s in strategies:
-                    set_kernel(m, s)
-                    timings[s.key] = float(timer(m, x, reps))
+                for b in todo:
+                    for st in strategies:
+                        if st in cands[b]:
+                            set_kernel(m, st)
+                            timings[b][st.key] = float(timer(m, xs[b], reps))
             finally:
                 close = getattr(m, "close", None)
                 if close:
                     close()
-        if not timings:
-            raise RuntimeError(f"no candidate could be compressed: {refused}")
-        timed = [s for s in cands if s.key in timings]
-        # Fastest; on a tie the earlier candidate (the simpler format first).
-        best = min(timed, key=lambda s: (timings[s.key], timed.index(s)))
-        choice = Choice(best, timings[best.key], timings)
-        self.cache[key] = choice.to_json()
+        for b in todo:
+            if not timings[b]:
+                raise RuntimeError(f"no candidate could be compressed: {refused}")
+            timed = [st for st in cands[b] if st.key in timings[b]]
+            # Fastest; on a tie the earlier candidate (the simpler format first).
+            best = min(timed, key=lambda st: (timings[b][st.key], timed.index(st)))
+            out[b] = Choice(best, timings[b][best.key], timings[b])
+            self.cache[_key(name, rows, cols, b)] = out[b].to_json()
         if self.path:
             with open(self.path, "w") as f:
                 json.dump(self.cache, f, indent=1, sort_keys=True)
-        return choice
+        return out
 
     def _activations(self, batch: int, cols: int):
         if self._make_x is not None:
@@ -254,8 +276,7 @@ def sweep(workloads, batches, path: str, reps: int = 30) -> dict:
                 continue
             seen.add((spec.rows, spec.cols))
             w = synth.head_matrix(spec, wl.seed) if spec is head else synth.matrix(spec, wl.seed)
-            for batch in batches:
-                c = tuner.tune(w, batch, reps=reps)
+            for batch, c in tuner.tune_batches(w, batches, reps=reps).items():
                 print(f"{name} {spec.rows}x{spec.cols} b{batch}: {c.strategy.key} "
                       f"{c.us_per_call:.2f} us", flush=True)
     return tuner.cache

@@ -112,3 +112,24 @@ def test_arguments_checked():
     with pytest.raises(ValueError):
         tuner(fake).tune(W.reshape(-1), 1)
     assert autotune.validate_candidates([A, A, C]) == [A, C]
+
+
+def test_several_batches_share_one_compression_per_format(tmp_path):
+    """tune_batches compresses each format once for all batches, times each
+    batch's candidates, and caches a choice per batch; batches already cached
+    are not timed again."""
+    fake = Fake(t_of((A, 30.0), (B, 21.5), (C, 25.0)))
+    t = tuner(fake, str(tmp_path / "tune.json"))
+    got = t.tune_batches(W, [1, 16], candidates=[A, B, C], reps=7)
+    assert sorted(fake.compressed) == sorted([A.format, C.format])
+    assert fake.closed == 2
+    assert got[1].strategy == B and got[16].strategy == B
+    assert set(got[1].timings) == {A.key, B.key, C.key}
+    fake.compressed.clear()
+    again = t.tune_batches(W, [1, 16, 4], candidates=[A, C], reps=7)
+    assert again[1] == got[1] and again[16] == got[16]
+    assert again[4].strategy == C and fake.compressed == [A.format, C.format]
+    with pytest.raises(ValueError):
+        t.tune_batches(W, [], reps=7)
+    with pytest.raises(ValueError):
+        t.tune_batches(W, [65], reps=7)
