@@ -87,9 +87,10 @@ typedef enum {
  * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512.
  * streams (a struct_size that ends before it means 1): bit streams per lane
  * and tile, each lane's symbol pairs dealt to its streams in turn (header
- * offset 60 holds streams - 1).  2 and 4 are a host-encoder-only layout for
- * now, with the prefix code only: nwc_plan_size reports device_bytes = 0 and
- * the calls that need a device image return UNSUPPORTED. */
+ * offset 60 holds streams - 1), with the prefix code only.  Every kernel
+ * reads 1 and 2 (a lane then follows two independent decode chains); 4 is a
+ * host-encoder-only layout: nwc_plan_size reports device_bytes = 0 and the
+ * calls that need a device image return UNSUPPORTED. */
 typedef struct {
   uint32_t struct_size;
   uint32_t lmax;
@@ -220,11 +221,13 @@ nwc_status nwc_gather_rows(nwc_handle_t handle, const int32_t* d_rows, int32_t n
                            uint16_t* d_out, nwc_stream_t stream);
 
 /* Bytes of split-K scratch one GEMV call of `batch` rows uses: u32 arrival
- * counters (one per 8 rows, padded to 256 bytes) and one FP32 partial sum per
- * (column tile, row of x in a launch, output row); 0 when the matrix has a
- * single column tile.  nwc_gemv takes them from the device image's scratch
- * area, nwc_gemv_noalloc from the library's static array.  The partials make
- * the reduction deterministic (fixed summation order). */
+ * counters (one per 8 rows, padded to 256 bytes) and FP32 partial sums: on the
+ * CUDA-core kernel one per (column tile, row of x in a launch, output row), on
+ * the tensor-core kernel one per (part of its K split, row of x up to 64,
+ * output row) when it splits K; 0 when the matrix has a single column tile.
+ * nwc_gemv takes them from the device image's scratch area, nwc_gemv_noalloc
+ * from the library's static array.  The partials make the reduction
+ * deterministic (fixed summation order). */
 nwc_status nwc_gemv_scratch_bytes(nwc_handle_t handle, int32_t batch, uint64_t* bytes);
 
 /* The fused decode-GEMV ("NWC", "How it works > Fused kernel": the matrix-vector

@@ -47,7 +47,8 @@ constexpr uint32_t kMagic = 0x3142574Eu;  // "NWB1"
 // number of ranks (1..7); its 256-byte lens area holds the ranked values of e
 // (R bytes in rank order, then zeros); its filler field the rank-0 value.  A
 // weight's code is its sign bit, then r zeros and a one for rank r < R, else R
-// zeros and the 7 bits of e.  Host encoder only: no kernel reads it yet.
+// zeros and the 7 bits of e.  Every kernel reads it (one stream per lane);
+// the device image holds a 256-byte rank table in place of the decode table.
 constexpr uint32_t kRankMagic = 0x3152574Eu;  // "NWR1"
 constexpr int kMaxRanks = 7;
 constexpr uint32_t kVersion = 1;
