@@ -4,7 +4,10 @@
 Default workload: the Llama-3.1-8B-shaped stack (32 layers of q, k, v, o, gate,
 up, down plus the lm_head, 7.5 G weights), the largest configuration that fits
 one GPU.  One step = one token: every GEMV of the stack, captured as one CUDA
-graph, with x and y resident in HBM and every layer larger than L2.  With a
+graph, with x and y resident in HBM and every layer larger than L2.  As the NWC
+page runs its models, the projections that read the same input are fused
+(q, k, v into one matrix, gate and up into another: 4 calls per layer);
+--no-fuse runs all 7.  With a
 single-matrix workload (--workload attn_4096_outliers, ...) one step is one
 nwc_gemv call, rotating over enough compressed copies that the weights never
 sit in L2 (126 MB).  Exactly --steps steps are timed; when they take less than
@@ -70,8 +73,15 @@ def parse_args():
     ap.add_argument("--report", action="store_true",
                     help="the five configurations as a markdown table (not the headline line)")
     ap.add_argument("--report-json", default=None, help="with --report: every line, to this file")
-    ap.add_argument("--fuse", action="store_true",
-                    help="stacks: q, k, v and gate, up each run as one stacked matrix")
+    ap.add_argument("--fuse", dest="fuse", action="store_true", default=True,
+                    help="stacks: q, k, v and gate, up each run as one stacked matrix (the "
+                         "default)")
+    ap.add_argument("--no-fuse", dest="fuse", action="store_false",
+                    help="stacks: every projection its own matrix and call")
+    ap.add_argument("--shard", action="store_true",
+                    help="one matrix split by output rows over the ranks (ShardedMatrix): "
+                         "each rank decodes its rows, then one NCCL all-gather of y per "
+                         "step (strong scaling); default: independent replicas")
     return ap.parse_args()
 
 
@@ -504,7 +514,8 @@ def run_stack(args) -> None:
         "footprint_ratio": weight_bytes / image_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm,
-                     "traffic": profile_traffic(args.workload, batch),
+                     "traffic": profile_traffic(args.workload + ("_fused" if args.fuse else ""),
+                                                batch),
                      "traffic_basis": "DRAM bytes per GEMV launch, averaged over a token's "
                                       "launches (committed ncu summary, current kernel source "
                                       "only; else null)",
@@ -768,7 +779,12 @@ def main():
     if args.report:
         run_report(args)
         return
-    line = run_stack(args) if args.workload in STACKS else run_matrix(args)
+    if args.shard:
+        if args.workload in STACKS:
+            raise SystemExit("--shard takes a single-matrix workload")
+        line = run_matrix_sharded(args)
+    else:
+        line = run_stack(args) if args.workload in STACKS else run_matrix(args)
     if line is not None:
         print(json.dumps(line))
     if int(os.environ.get("WORLD_SIZE", 1)) > 1:
@@ -777,21 +793,126 @@ def main():
             dist.destroy_process_group()
 
 
+def run_matrix_sharded(args):
+    """One matrix of the workload split by output rows over the job's ranks
+    (whole 8-row tile blocks, one code table per shard): a step is one GEMV of
+    each rank's rows plus one NCCL all-gather that leaves the whole y on every
+    rank.  Each rank rotates over enough device copies of its shard that the
+    weights never sit in L2.  Steps are launched eagerly (the gather is a
+    collective) and timed with CUDA events between barriers; the time is the
+    slowest rank's, and value counts the whole matrix once (strong scaling)."""
+    import torch
+
+    from lossless_bf16_weight_nwc_b200 import _lib, synth
+    from lossless_bf16_weight_nwc_b200.sharded import ShardedMatrix
+    rank, world = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.workload(args.workload)
+    spec = wl.matrices[0]
+    batch = args.batch
+    w = synth.matrix(spec, wl.seed)
+    x_host = synth.activations(wl.seed, batch, spec.cols)
+    sm = ShardedMatrix.compress(w, group=None, device=dev, streams=args.streams,
+                                code=CODES[args.code])
+    local = sm.local
+    image_bytes = local.compressed_bytes if local is not None else 0
+    copies = max(2, int(np.ceil(2.2 * L2_BYTES / max(image_bytes, 1)))) if local else 1
+    mats = [local]
+    if local is not None:
+        for _ in range(copies - 1):
+            m = _lib.CompressedMatrix(local.image.clone(), None, local.rows, local.cols,
+                                      local.blob_bytes)
+            m.handle = _lib.nwc_handle_from_device(m.image, m.image.numel())
+            mats.append(m)
+        if args.tc_min_batch is not None:
+            for m in mats:
+                _lib.nwc_gemv_set_tc_min_batch(m.handle, args.tc_min_batch)
+    x = torch.from_numpy(x_host.view(np.int16)).view(torch.bfloat16).to(dev)
+    y_local = torch.empty((batch, local.rows if local else 0), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        m = mats[i % len(mats)]
+        if m is None:
+            return sm.gemv(x)
+        return sm.gemv(x, local_gemv=lambda xx: (
+            _lib.nwc_gemv(m.handle, xx, y_local, batch, stream.cuda_stream), y_local)[1])
+
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    steps = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index) as clocks:
+        barrier(world)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i in range(steps):
+            y = step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / steps
+    parity_ok = True
+    if rank == 0:
+        import oracle
+        rows_chk = np.arange(0, spec.rows, max(1, spec.rows // 256))
+        y_ref = oracle.gemv(w[rows_chk], x_host)
+        y_gpu = y.double().cpu().numpy()[:, rows_chk]
+        wf = synth.bf16_bits_to_float(w[rows_chk]).astype(np.float64)
+        xf = synth.bf16_bits_to_float(x_host).astype(np.float64)
+        bound = 1e-2 * np.outer(np.linalg.norm(xf, axis=1), np.linalg.norm(wf, axis=1)) * 2.0 ** -8
+        parity_ok = bool((np.abs(y_gpu - y_ref) <= bound).all())
+    weight_bytes = 2.0 * spec.rows * spec.cols
+    peaks, peak_src = measured_peaks()
+    line = {
+        "metric": METRIC, "value": weight_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "matrix": f"{spec.rows}x{spec.cols}",
+                   "batch": batch, "parallelism": f"rows x{world} (ShardedMatrix) + all-gather of y",
+                   "rows_per_rank": [e - s for s, e in sm.ranges],
+                   "l2": f"inputs larger than L2: {copies} rotating copies of each shard",
+                   "launch": "eager (GEMV + NCCL all-gather per step)"},
+        "us_per_call": ms * 1e3,
+        "roofline": {"bound": "hbm", "achieved": image_bytes / (ms * 1e-3) / 1e9,
+                     "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                     "frac": image_bytes / (ms * 1e-3) / 1e9 / float(peaks["hbm_gbs"]),
+                     "traffic": None, "peak_source": f"{peak_src} hbm_gbs (copy)",
+                     "basis": "rank 0's compressed shard bytes / time per step (GEMV + gather)"},
+        "clocks": clocks.summary(),
+        "e2e": None,
+        "gpu_launches": steps,
+        "kernel_path": "gemv_tc_kernel" if local is not None and _lib.nwc_gemv_path(
+            local.handle, x, batch)[1] else "gemv_kernel",
+        "parity_spot_check": parity_ok,
+    }
+    for m in mats[1:]:
+        m.close()
+    sm.close()
+    return line if rank == 0 else None
+
+
 def run_report(args) -> None:
     """The five benchmark configurations in one run, as a markdown table
     (and every configuration's JSON line in --report-json when given): per
     call or per token, effective and compressed GB/s, fraction of the HBM
     peak, compression ratio, the uncompressed cuBLAS time and the kernel
     path."""
-    rows = [("single_1024", 1), ("attn_4096_outliers", 1), ("attn_4096_outliers", 4),
-            ("attn_4096_outliers", 16), ("attn_4096_outliers", 64),
-            ("mlp_pair_t5", 1), ("mlp_pair_t5", 2), ("mlp_pair_t5", 8), ("mlp_pair_t5", 64),
-            ("qwen3_4b_stack", 1), ("llama31_8b_stack", 1), ("llama31_8b_stack", 16),
-            ("llama31_8b_stack", 64)]
+    rows = [("single_1024", 1, None), ("attn_4096_outliers", 1, None),
+            ("attn_4096_outliers", 4, None), ("attn_4096_outliers", 16, None),
+            ("attn_4096_outliers", 64, None), ("mlp_pair_t5", 1, None), ("mlp_pair_t5", 2, None),
+            ("mlp_pair_t5", 8, None), ("mlp_pair_t5", 64, None),
+            ("qwen3_4b_stack", 1, False), ("qwen3_4b_stack", 1, True),
+            ("llama31_8b_stack", 1, False), ("llama31_8b_stack", 1, True),
+            ("llama31_8b_stack", 16, True), ("llama31_8b_stack", 64, True)]
     lines = []
-    for workload, batch in rows:
+    for workload, batch, fuse in rows:
         a = argparse.Namespace(**vars(args))
         a.workload, a.batch, a.report = workload, batch, False
+        if fuse is not None:
+            a.fuse = fuse
         a.no_cpu_baseline = True
         a.e2e_steps = 0
         stack = workload in STACKS
@@ -804,7 +925,9 @@ def run_report(args) -> None:
     print("| workload | batch | µs per step | effective GB/s | compressed GB/s | fraction of HBM "
           "peak | ratio | cuBLAS BF16 µs | kernel |")
     print("|---|---|---|---|---|---|---|---|---|")
-    for (workload, batch), line in zip(rows, lines):
+    for (workload, batch, fuse), line in zip(rows, lines):
+        if fuse is not None:
+            workload = f"{workload} ({'fused' if fuse else 'unfused'})"
         rf = line["roofline"]
         comp = line.get("compressed_bytes") or line.get("compressed_bytes_per_token")
         us = line["ms_per_step"] * 1e3

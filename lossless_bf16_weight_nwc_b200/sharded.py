@@ -82,6 +82,9 @@ class ShardedMatrix:
         gathered = torch.empty((self.world, batch, width), dtype=torch.float32, device=x.device)
         gather = self._gather or _all_gather
         gather(gathered, part, self.group)
+        if batch == 1 and all(e - s == width for s, e in self.ranges):
+            # One row of x and equal shards: the gathered rows are y, in order.
+            return gathered.view(1, self.world * width)
         return torch.cat([gathered[r, :, :e - s] for r, (s, e) in enumerate(self.ranges)], dim=1)
 
     def close(self) -> None:

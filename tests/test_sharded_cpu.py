@@ -63,7 +63,17 @@ def _rank_main(rank, world, port, out):
         xt = torch.zeros((3, 300))
         y = m.gemv(xt, local_gemv=lambda _: torch.from_numpy(oracle.gemv(m.local.part, x)).float())
         full = oracle.gemv(w, x).astype(np.float32)
-        out.put((rank, bool(np.array_equal(y.numpy(), full)), tuple(y.shape)))
+        # One row of x over equal shards (80 rows: 5 tile blocks each): the
+        # gathered buffer is y itself.
+        w1 = synth.matrix(synth.MatrixSpec("w1", 80, 300, "normal", 0.02, 0), 6)
+        x1 = synth.activations(6, 1, 300)
+        m1 = sharded.ShardedMatrix.compress(w1, compress=lambda part, device=None: Shard(part),
+                                            device="cpu")
+        y1 = m1.gemv(torch.zeros((1, 300)),
+                     local_gemv=lambda _: torch.from_numpy(oracle.gemv(m1.local.part, x1)).float())
+        full1 = oracle.gemv(w1, x1).astype(np.float32)
+        out.put((rank, bool(np.array_equal(y.numpy(), full)), tuple(y.shape),
+                 bool(np.array_equal(y1.numpy(), full1)), tuple(y1.shape)))
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -81,7 +91,7 @@ def test_two_gloo_ranks_gather_the_whole_y():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert results == [(0, True, (3, 77)), (1, True, (3, 77))]
+    assert results == [(0, True, (3, 77), True, (1, 80)), (1, True, (3, 77), True, (1, 80))]
 
 
 def test_single_process_needs_no_collective():
