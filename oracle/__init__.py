@@ -84,6 +84,11 @@ def _declare(h: ctypes.CDLL) -> ctypes.CDLL:
     h.orc_rank_encode.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, u8p,
                                   i64, c.POINTER(i64)]
     h.orc_rank_decode.argtypes = [u8p, i64, u16p, i64]
+    h.orc_escape_blob_size.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, c.c_int,
+                                       c.POINTER(i64)]
+    h.orc_escape_encode.argtypes = [u16p, i64, i64, c.c_int, c.c_int, c.c_int, c.c_int, u8p,
+                                    i64, c.POINTER(i64)]
+    h.orc_escape_decode.argtypes = [u8p, i64, u16p, i64]
     return h
 
 
@@ -305,4 +310,40 @@ def rank_decode(blob: np.ndarray) -> np.ndarray:
     out = np.zeros((rows, cols), dtype=np.uint16)
     _check(lib().orc_rank_decode(_ptr(blob, ctypes.c_uint8), blob.size,
                                  _ptr(out, ctypes.c_uint16), out.size), "rank_decode")
+    return out
+
+
+# ---- variant NWE1: rare exponents in verbatim runs -------------------------
+
+def escape_encode(w: np.ndarray, tile_cols: int = 512, lmax: int = 7, keep: int = 16,
+                  tile_rows: int = 8) -> np.ndarray:
+    """BF16 bit patterns [rows, cols] -> NWE1 blob (uint8 array): the `keep`
+    most frequent exponent bytes coded, runs of 64 holding another one verbatim."""
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, cols = w.shape
+    size = ctypes.c_int64()
+    _check(lib().orc_escape_blob_size(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows,
+                                      tile_cols, lmax, keep, ctypes.byref(size)),
+           "escape_blob_size")
+    blob = np.zeros(size.value, dtype=np.uint8)
+    got = ctypes.c_int64()
+    _check(lib().orc_escape_encode(_ptr(w, ctypes.c_uint16), rows, cols, tile_rows, tile_cols,
+                                   lmax, keep, _ptr(blob, ctypes.c_uint8), blob.size,
+                                   ctypes.byref(got)), "escape_encode")
+    assert got.value == blob.size
+    return blob
+
+
+def escape_decode(blob: np.ndarray) -> np.ndarray:
+    """NWE1 blob -> BF16 bit patterns [rows, cols]."""
+    blob = np.ascontiguousarray(blob, dtype=np.uint8)
+    if blob.size < 32:
+        raise OracleError(ORC_E_CORRUPT, "escape_decode")
+    rows = int.from_bytes(blob[16:24].tobytes(), "little")
+    cols = int.from_bytes(blob[24:32].tobytes(), "little")
+    if not (1 <= rows <= 1 << 32 and 1 <= cols <= 1 << 32) or rows * cols > 1 << 34:
+        raise OracleError(ORC_E_CORRUPT, "escape_decode")
+    out = np.zeros((rows, cols), dtype=np.uint16)
+    _check(lib().orc_escape_decode(_ptr(blob, ctypes.c_uint8), blob.size,
+                                   _ptr(out, ctypes.c_uint16), out.size), "escape_decode")
     return out

@@ -101,6 +101,46 @@
  * Readings where the v9 passage is silent: the sign bit comes first, a rank is
  * counted in zero bits ended by a one, the escape is the 7-bit field after R
  * zero bits, R = 7 by default.
+ *
+ * Variant "NWE1", rare exponents in verbatim runs ("Unweight", "Compressing
+ * BF16 Weights": the 16 most common exponents cover nearly all weights of a
+ * layer and are Huffman-coded; a row of 64 weights that holds any other
+ * exponent is stored verbatim, so the decoder branches once per run, not per
+ * weight):
+ *
+ *  1. Planes and filler as NWB1.
+ *  2. Kept symbols: the K most frequent exponent bytes over the real weights
+ *     and the fillers (largest count first, smaller symbol first on a tie;
+ *     K = min(keep, number present), keep = 16 by default).  The filler is
+ *     always kept.
+ *  3. Runs: in a tile, run (g, m) is row g and the columns 64 m .. 64 m + 63 of
+ *     the tile (64 consecutive weights of one matrix row; fillers past the
+ *     edge).  A run is escaped when one of its 64 exponent bytes is not kept.
+ *     It is the 16-symbol slice of lanes 4 g .. 4 g + 3 in group m.
+ *  4. Code: the optimal code limited to lmax bits over the counts of the
+ *     symbols of the runs that are not escaped, assigned canonically as in
+ *     NWB1 (all lengths 0 when every run is escaped).  So a run is escaped
+ *     exactly when it holds a symbol without a code.
+ *  5. Chunk of a tile:
+ *       raw    u8[8 * tile_cols], as NWB1 (every position, escaped or not)
+ *       flags  u8[16]: bit m of byte g set when run (g, m) is escaped; bits
+ *              m >= tile_cols / 64 and bytes 8 .. 15 zero
+ *       runs   u8[64 * n]: the exponent bytes of the tile's n escaped runs in
+ *              (g, m) order, each run's 64 bytes in column order (lane 4 g + c
+ *              finds its 16 at byte 16 c of the run)
+ *       lens   u8[32] and bits: as NWB1 with one stream per lane, the streams
+ *              holding the codes of the symbols of the runs not escaped only.
+ *     An escaped run costs 16 bits per weight (its raw bytes and its exponent
+ *     bytes), as a run stored verbatim does.
+ *
+ *   header differences from NWB1: magic 0x3145574E ("NWE1"); offset 60 holds
+ *   K; offset 96 the total code bits; offset 104 the number of escaped runs
+ *   (u64).  lens[256] as NWB1.
+ *
+ * Readings where the passage is silent: the run is aligned to 64 columns of
+ * the tile (so to 64 columns of the matrix), the exponent bytes of an escaped
+ * run sit in the chunk and its raw bytes stay in the raw plane (16 bits per
+ * weight either way), the kept set counts the fillers.
  */
 #include "nwc_oracle.h"
 
@@ -681,6 +721,323 @@ int decode_rank_impl(const uint8_t* blob, int64_t size, uint16_t* out, int64_t c
   return ORC_OK;
 }
 
+/* ---- Variant NWE1: rare exponents in verbatim runs ------------------------ */
+
+const uint32_t kEscMagic = 0x3145574Eu;
+
+/* The `keep` most frequent symbols (largest count first, smaller symbol on a
+ * tie) among those present.  Returns how many were kept. */
+int kept_symbols(const uint64_t cnt[256], int keep, bool kept[256]) {
+  std::vector<int> present;
+  for (int s = 0; s < 256; ++s) {
+    kept[s] = false;
+    if (cnt[s] > 0) present.push_back(s);
+  }
+  std::stable_sort(present.begin(), present.end(),
+                   [&](int x, int y) { return cnt[x] > cnt[y]; });
+  const int n = (int)std::min<size_t>(present.size(), (size_t)keep);
+  for (int q = 0; q < n; ++q) kept[present[(size_t)q]] = true;
+  return n;
+}
+
+/* Exponent byte and raw byte of tile element (r, c) of tile (i, j); the filler
+ * outside the matrix. */
+void tile_element(const uint16_t* w, int64_t rows, int64_t cols, int64_t i, int64_t j,
+                  int tile_rows, int tile_cols, int filler, int r, int c, uint8_t* s,
+                  uint8_t* rb) {
+  const int64_t row = i * tile_rows + r, col = j * tile_cols + c;
+  *s = (uint8_t)filler;
+  *rb = 0;
+  if (row < rows && col < cols) orc_plane_split(w[row * cols + col], s, rb);
+}
+
+int encode_escape_impl(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                       int tile_cols, int lmax, int keep, uint8_t* blob, int64_t cap,
+                       int64_t* size) {
+  if (!w || rows < 1 || cols < 1 || !size) return ORC_E_ARG;
+  if (!geometry_ok(tile_rows, tile_cols, lmax) || keep < 1 || keep > 256) return ORC_E_ARG;
+  const int64_t tiles_r = (rows + tile_rows - 1) / tile_rows;
+  const int64_t tiles_c = (cols + tile_cols - 1) / tile_cols;
+  const int64_t tiles = tiles_r * tiles_c;
+  const int groups = tile_cols / 64;
+  const int lane_syms = 2 * tile_rows * groups;
+  const int raw_bytes = tile_rows * tile_cols;
+
+  /* Step 2: histogram with the fillers, filler, kept symbols. */
+  uint64_t cnt[256];
+  orc_histogram(w, rows, cols, cnt);
+  const int filler = filler_symbol(cnt);
+  cnt[filler] += (uint64_t)(tiles_r * tile_rows) * (uint64_t)(tiles_c * tile_cols) -
+                 (uint64_t)rows * (uint64_t)cols;
+  bool kept[256];
+  const int K = kept_symbols(cnt, keep, kept);
+
+  /* Step 3: which runs are escaped; step 4: counts over the other runs. */
+  std::vector<uint8_t> escaped((size_t)(tiles * tile_rows * groups), 0);
+  uint64_t ccnt[256] = {};
+  uint64_t n_escaped = 0;
+  for (int64_t u = 0; u < tiles; ++u) {
+    const int64_t i = u % tiles_r, j = u / tiles_r;
+    for (int g = 0; g < tile_rows; ++g) {
+      for (int m = 0; m < groups; ++m) {
+        bool rare = false;
+        for (int c = 64 * m; c < 64 * m + 64; ++c) {
+          uint8_t s, rb;
+          tile_element(w, rows, cols, i, j, tile_rows, tile_cols, filler, g, c, &s, &rb);
+          if (!kept[s]) rare = true;
+        }
+        escaped[(size_t)((u * tile_rows + g) * groups + m)] = rare ? 1 : 0;
+        if (rare) {
+          ++n_escaped;
+          continue;
+        }
+        for (int c = 64 * m; c < 64 * m + 64; ++c) {
+          uint8_t s, rb;
+          tile_element(w, rows, cols, i, j, tile_rows, tile_cols, filler, g, c, &s, &rb);
+          ccnt[s] += 1;
+        }
+      }
+    }
+  }
+  uint8_t len[256] = {};
+  uint64_t any = 0;
+  for (int s = 0; s < 256; ++s) any += ccnt[s];
+  if (any) {
+    const int rc = orc_code_lengths(ccnt, lmax, len);
+    if (rc != ORC_OK) return rc;
+  }
+  uint32_t code[256];
+  orc_canonical_codes(len, code);
+  uint64_t coded_bits = 0;
+  for (int s = 0; s < 256; ++s) coded_bits += ccnt[s] * (uint64_t)len[s];
+
+  /* Step 5: the chunks. */
+  const uint64_t lens_off = kHeaderBytes;
+  const uint64_t index_off = lens_off + 256;
+  const uint64_t tiles_off = round_up(index_off + 4 * (uint64_t)(tiles + 1), 256);
+  std::vector<uint32_t> index((size_t)tiles + 1);
+  uint64_t area = 0;
+  for (int64_t u = 0; u < tiles; ++u) {
+    const int64_t i = u % tiles_r, j = u / tiles_r;
+    auto is_escaped = [&](int g, int m) {
+      return escaped[(size_t)((u * tile_rows + g) * groups + m)] != 0;
+    };
+    std::vector<uint8_t> raw((size_t)raw_bytes, 0);
+    std::vector<uint8_t> flags(16, 0);
+    std::vector<uint8_t> runs;
+    for (int g = 0; g < tile_rows; ++g) {
+      for (int m = 0; m < groups; ++m) {
+        if (!is_escaped(g, m)) continue;
+        flags[(size_t)g] |= (uint8_t)(1u << m);
+        for (int c = 64 * m; c < 64 * m + 64; ++c) {
+          uint8_t s, rb;
+          tile_element(w, rows, cols, i, j, tile_rows, tile_cols, filler, g, c, &s, &rb);
+          runs.push_back(s);
+        }
+      }
+    }
+    std::vector<uint8_t> seq; /* one entry per bit */
+    uint8_t lane_bytes[kLanes];
+    for (int t = 0; t < kLanes; ++t) {
+      std::vector<uint8_t> lb;
+      for (int k = 0; k < lane_syms; ++k) {
+        int r, c;
+        lane_symbol_position(t, k, &r, &c);
+        uint8_t s, rb;
+        tile_element(w, rows, cols, i, j, tile_rows, tile_cols, filler, r, c, &s, &rb);
+        raw[(size_t)raw_position(t, k)] = rb;
+        if (is_escaped(r, k / 16)) continue;
+        for (int b = len[s] - 1; b >= 0; --b) lb.push_back((uint8_t)((code[s] >> b) & 1u));
+      }
+      while (lb.size() % 8 != 0) lb.push_back(0);
+      lane_bytes[t] = (uint8_t)(lb.size() / 8);
+      seq.insert(seq.end(), lb.begin(), lb.end());
+    }
+    while (seq.size() % 128 != 0) seq.push_back(0);
+    std::vector<uint8_t> bits(seq.size() / 8, 0);
+    for (size_t b = 0; b < seq.size(); ++b) {
+      if (!seq[b]) continue;
+      const int bit = 31 - (int)(b % 32);
+      bits[(b / 32) * 4 + (size_t)(bit / 8)] |= (uint8_t)(1u << (bit % 8));
+    }
+    std::vector<uint8_t> chunk;
+    chunk.insert(chunk.end(), raw.begin(), raw.end());
+    chunk.insert(chunk.end(), flags.begin(), flags.end());
+    chunk.insert(chunk.end(), runs.begin(), runs.end());
+    chunk.insert(chunk.end(), lane_bytes, lane_bytes + kLanes);
+    chunk.insert(chunk.end(), bits.begin(), bits.end());
+    index[(size_t)u] = (uint32_t)(area / 16);
+    if (blob) {
+      if ((int64_t)(tiles_off + area + chunk.size()) > cap) return ORC_E_SPACE;
+      std::memcpy(blob + tiles_off + area, chunk.data(), chunk.size());
+    }
+    area += chunk.size();
+    if (area / 16 > 0xFFFFFFFFull) return ORC_E_ARG;
+  }
+  index[(size_t)tiles] = (uint32_t)(area / 16);
+  const uint64_t total = tiles_off + area;
+  *size = (int64_t)total;
+  if (!blob) return ORC_OK;
+  if ((int64_t)total > cap) return ORC_E_SPACE;
+  std::memset(blob, 0, (size_t)tiles_off);
+  put_u32(blob + 0, kEscMagic);
+  put_u32(blob + 4, kVersion);
+  put_u32(blob + 8, kHeaderBytes);
+  put_u32(blob + 12, (uint32_t)lmax);
+  put_u64(blob + 16, (uint64_t)rows);
+  put_u64(blob + 24, (uint64_t)cols);
+  put_u32(blob + 32, (uint32_t)tile_rows);
+  put_u32(blob + 36, (uint32_t)tile_cols);
+  put_u64(blob + 40, (uint64_t)tiles_r);
+  put_u64(blob + 48, (uint64_t)tiles_c);
+  put_u32(blob + 56, (uint32_t)filler);
+  put_u32(blob + 60, (uint32_t)K);
+  put_u64(blob + 64, lens_off);
+  put_u64(blob + 72, index_off);
+  put_u64(blob + 80, tiles_off);
+  put_u64(blob + 88, total);
+  put_u64(blob + 96, coded_bits);
+  put_u64(blob + 104, n_escaped);
+  std::memcpy(blob + lens_off, len, 256);
+  for (int64_t u = 0; u <= tiles; ++u) put_u32(blob + index_off + 4 * u, index[(size_t)u]);
+  return ORC_OK;
+}
+
+int decode_escape_impl(const uint8_t* blob, int64_t size, uint16_t* out, int64_t cap_elems) {
+  if (!blob || size < kHeaderBytes + 256) return ORC_E_CORRUPT;
+  if (get_u32(blob) != kEscMagic || get_u32(blob + 4) != kVersion ||
+      get_u32(blob + 8) != (uint32_t)kHeaderBytes)
+    return ORC_E_CORRUPT;
+  const int lmax = (int)get_u32(blob + 12);
+  const int64_t rows = (int64_t)get_u64(blob + 16), cols = (int64_t)get_u64(blob + 24);
+  const int tile_rows = (int)get_u32(blob + 32), tile_cols = (int)get_u32(blob + 36);
+  const int64_t tiles_r = (int64_t)get_u64(blob + 40), tiles_c = (int64_t)get_u64(blob + 48);
+  const int filler = (int)get_u32(blob + 56);
+  const int K = (int)get_u32(blob + 60);
+  const uint64_t lens_off = get_u64(blob + 64), index_off = get_u64(blob + 72);
+  const uint64_t tiles_off = get_u64(blob + 80), total = get_u64(blob + 88);
+  const uint64_t n_escaped = get_u64(blob + 104);
+  if (rows < 1 || cols < 1 || !geometry_ok(tile_rows, tile_cols, lmax)) return ORC_E_CORRUPT;
+  if (K < 1 || K > 256 || filler < 0 || filler > 255) return ORC_E_CORRUPT;
+  if (tiles_r != (rows + tile_rows - 1) / tile_rows ||
+      tiles_c != (cols + tile_cols - 1) / tile_cols)
+    return ORC_E_CORRUPT;
+  const int64_t tiles = tiles_r * tiles_c;
+  if (lens_off != (uint64_t)kHeaderBytes || index_off != lens_off + 256 ||
+      tiles_off != round_up(index_off + 4 * (uint64_t)(tiles + 1), 256) ||
+      total != (uint64_t)size)
+    return ORC_E_CORRUPT;
+  for (int q = 112; q < kHeaderBytes; ++q)
+    if (blob[q]) return ORC_E_CORRUPT;
+  /* The code: Kraft sum at most one, no more coded symbols than kept ones. */
+  uint8_t len[256];
+  std::memcpy(len, blob + lens_off, 256);
+  double kraft = 0.0;
+  int coded = 0;
+  for (int s = 0; s < 256; ++s) {
+    if (len[s] > lmax) return ORC_E_CORRUPT;
+    if (len[s]) {
+      kraft += 1.0 / (double)(1u << len[s]);
+      ++coded;
+    }
+  }
+  if (kraft > 1.0 || coded > K) return ORC_E_CORRUPT;
+  uint32_t code[256];
+  orc_canonical_codes(len, code);
+  std::vector<std::vector<int> > sym_of(13);
+  for (int l = 1; l <= 12; ++l) sym_of[(size_t)l].assign((size_t)1 << l, -1);
+  for (int s = 0; s < 256; ++s)
+    if (len[s]) sym_of[len[s]][code[s]] = s;
+  if (!out || cap_elems < rows * cols) return ORC_E_SPACE;
+
+  const int groups = tile_cols / 64;
+  const int lane_syms = 2 * tile_rows * groups;
+  const int raw_bytes = tile_rows * tile_cols;
+  const uint64_t area = (uint64_t)size - tiles_off;
+  uint64_t escaped_total = 0;
+  for (int64_t u = 0; u < tiles; ++u) {
+    const uint64_t c0 = 16ull * get_u32(blob + index_off + 4 * u);
+    const uint64_t c1 = 16ull * get_u32(blob + index_off + 4 * (u + 1));
+    if (c1 < c0 || c1 > area || c1 - c0 < (uint64_t)raw_bytes + 16 + kLanes)
+      return ORC_E_CORRUPT;
+    const uint8_t* chunk = blob + tiles_off + c0;
+    const uint8_t* raw = chunk;
+    const uint8_t* flags = chunk + raw_bytes;
+    /* Flags: only bits of real groups, bytes 8 .. 15 zero. */
+    for (int q = 0; q < 16; ++q) {
+      const unsigned allowed = q < tile_rows ? (1u << groups) - 1u : 0u;
+      if (flags[q] & ~allowed) return ORC_E_CORRUPT;
+    }
+    /* Place of every escaped run among the tile's runs, in (g, m) order. */
+    std::vector<int> run_at((size_t)(tile_rows * groups), -1);
+    int n = 0;
+    for (int g = 0; g < tile_rows; ++g)
+      for (int m = 0; m < groups; ++m)
+        if ((flags[g] >> m) & 1u) run_at[(size_t)(g * groups + m)] = n++;
+    escaped_total += (uint64_t)n;
+    const uint64_t head = (uint64_t)raw_bytes + 16 + 64ull * (uint64_t)n;
+    if (c1 - c0 < head + kLanes) return ORC_E_CORRUPT;
+    const uint8_t* runs = chunk + raw_bytes + 16;
+    const uint8_t* lane_bytes = chunk + head;
+    const uint8_t* bits = chunk + head + kLanes;
+    uint64_t stream_bytes = 0;
+    for (int t = 0; t < kLanes; ++t) stream_bytes += lane_bytes[t];
+    if (c1 - c0 != head + kLanes + round_up(stream_bytes, 16)) return ORC_E_CORRUPT;
+    /* An escaped run holds a symbol without a code (otherwise it would have
+     * been coded). */
+    for (int q = 0; q < n; ++q) {
+      bool rare = false;
+      for (int b = 0; b < 64; ++b) rare = rare || len[runs[64 * q + b]] == 0;
+      if (!rare) return ORC_E_CORRUPT;
+    }
+    auto bit_at = [&](uint64_t q) -> int {
+      const int b = 31 - (int)(q % 32);
+      return (bits[(q / 32) * 4 + (uint64_t)(b / 8)] >> (b % 8)) & 1;
+    };
+    const int64_t i = u % tiles_r, j = u / tiles_r;
+    uint64_t lane_start = 0;
+    for (int t = 0; t < kLanes; ++t) {
+      uint64_t pos = lane_start;
+      const uint64_t end = lane_start + 8ull * lane_bytes[t];
+      for (int k = 0; k < lane_syms; ++k) {
+        int r, c;
+        lane_symbol_position(t, k, &r, &c);
+        const int at = run_at[(size_t)(r * groups + k / 16)];
+        int s = -1;
+        if (at >= 0) {
+          /* Column c of the tile is byte c - 64 m of its run. */
+          s = runs[64 * at + (c - 64 * (k / 16))];
+        } else {
+          uint32_t v = 0;
+          int l = 0;
+          while (s < 0) {
+            if (pos >= end || l >= lmax) return ORC_E_CORRUPT;
+            v = (v << 1) | (uint32_t)bit_at(pos++);
+            ++l;
+            s = sym_of[(size_t)l][v];
+          }
+        }
+        const uint8_t rb = raw[raw_position(t, k)];
+        const int64_t row = i * tile_rows + r, col = j * tile_cols + c;
+        if (row < rows && col < cols) {
+          out[row * cols + col] = orc_plane_join((uint8_t)s, rb);
+        } else if (s != filler || rb != 0) {
+          return ORC_E_CORRUPT;
+        }
+      }
+      if (end - pos >= 8) return ORC_E_CORRUPT;
+      while (pos < end)
+        if (bit_at(pos++)) return ORC_E_CORRUPT;
+      lane_start = end;
+    }
+    for (uint64_t q = lane_start; q < 8 * round_up(stream_bytes, 16); ++q)
+      if (bit_at(q)) return ORC_E_CORRUPT;
+  }
+  if (escaped_total != n_escaped) return ORC_E_CORRUPT;
+  return ORC_OK;
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -886,6 +1243,22 @@ int orc_rank_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows
 
 int orc_rank_decode(const uint8_t* blob, int64_t size, uint16_t* w_out, int64_t cap_elems) {
   return decode_rank_impl(blob, size, w_out, cap_elems);
+}
+
+int orc_escape_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                         int tile_cols, int lmax, int keep, int64_t* size) {
+  return encode_escape_impl(w, rows, cols, tile_rows, tile_cols, lmax, keep, nullptr, 0, size);
+}
+
+int orc_escape_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                      int tile_cols, int lmax, int keep, uint8_t* blob, int64_t cap,
+                      int64_t* size) {
+  if (!blob) return ORC_E_ARG;
+  return encode_escape_impl(w, rows, cols, tile_rows, tile_cols, lmax, keep, blob, cap, size);
+}
+
+int orc_escape_decode(const uint8_t* blob, int64_t size, uint16_t* w_out, int64_t cap_elems) {
+  return decode_escape_impl(blob, size, w_out, cap_elems);
 }
 
 }  // extern "C"

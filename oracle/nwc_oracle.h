@@ -21,9 +21,10 @@
  *         "Fused kernel" (blocks of 8 rows x 512 columns, one bit stream per
  *         lane, padding for any shape).
  *
- * The formats these functions write and read ("NWB1", and the variant "NWR1"
- * of [NWC]'s ranked unary code) are stated field by field at the top of
- * nwc_oracle.cpp.  Status codes: 0 = OK, negative = error (see ORC_E_*).
+ * The formats these functions write and read ("NWB1", the variant "NWR1" of
+ * [NWC]'s ranked unary code and the variant "NWE1" of [UW]'s verbatim runs)
+ * are stated field by field at the top of nwc_oracle.cpp.  Status codes:
+ * 0 = OK, negative = error (see ORC_E_*).
  */
 #ifndef NWC_ORACLE_H
 #define NWC_ORACLE_H
@@ -99,6 +100,17 @@ int orc_rank_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_r
 int orc_rank_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
                     int tile_cols, int ranks, uint8_t* blob, int64_t cap, int64_t* size);
 int orc_rank_decode(const uint8_t* blob, int64_t size, uint16_t* w_out, int64_t cap_elems);
+
+/* Variant "NWE1" (stated at the top of nwc_oracle.cpp): [UW] "Compressing BF16
+ * Weights" — the `keep` most common exponent bytes are coded (limit lmax); a
+ * run of 64 weights of a row that holds any other exponent keeps its exponent
+ * bytes verbatim. */
+int orc_escape_blob_size(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                         int tile_cols, int lmax, int keep, int64_t* size);
+int orc_escape_encode(const uint16_t* w, int64_t rows, int64_t cols, int tile_rows,
+                      int tile_cols, int lmax, int keep, uint8_t* blob, int64_t cap,
+                      int64_t* size);
+int orc_escape_decode(const uint8_t* blob, int64_t size, uint16_t* w_out, int64_t cap_elems);
 
 #ifdef __cplusplus
 }
