@@ -64,9 +64,10 @@ def parse_args():
                     help="how y reaches the host in the end-to-end leg")
     ap.add_argument("--streams", type=int, default=1, choices=[1, 2],
                     help="bit streams per lane and tile of the compressed matrices")
-    ap.add_argument("--code", default="prefix", choices=["prefix", "rank"],
-                    help="exponent code: the length-limited prefix code (NWB1) or the ranked "
-                         "unary code (NWR1, 7 ranks)")
+    ap.add_argument("--code", default="prefix", choices=["prefix", "rank", "escape"],
+                    help="exponent code: the length-limited prefix code (NWB1), the ranked "
+                         "unary code (NWR1, 7 ranks) or the prefix code of the 16 most "
+                         "frequent exponents with verbatim runs for the rest (NWE1)")
     ap.add_argument("--tc-min-batch", type=int, default=None,
                     help="smallest batch that takes the tensor-core kernel (default: the "
                          "library's, 17; 0 = never)")
@@ -104,6 +105,12 @@ def kernel_source_hash() -> str:
             if code:
                 lines.append(code)
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
+def format_suffix(args) -> str:
+    """Key suffix of a non-default compressed format in the traffic summary."""
+    return ("" if args.code == "prefix" else f"_{args.code}") + \
+        ("" if args.streams == 1 else f"_s{args.streams}")
 
 
 def profile_traffic(workload: str, batch: int) -> float | None:
@@ -319,7 +326,7 @@ def run_reference(args) -> None:
 
 
 STACKS = ("qwen3_4b_stack", "llama31_8b_stack")
-CODES = {"prefix": 0, "rank": 1}    # nwc_opts.code
+CODES = {"prefix": 0, "rank": 1, "escape": 2}    # nwc_opts.code
 
 
 def run_stack(args) -> None:
@@ -514,8 +521,9 @@ def run_stack(args) -> None:
         "footprint_ratio": weight_bytes / image_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm,
-                     "traffic": profile_traffic(args.workload + ("_fused" if args.fuse else ""),
-                                                batch),
+                     "traffic": profile_traffic(
+                         args.workload + ("_fused" if args.fuse else "") + format_suffix(args),
+                         batch),
                      "traffic_basis": "DRAM bytes per GEMV launch, averaged over a token's "
                                       "launches (committed ncu summary, current kernel source "
                                       "only; else null)",
@@ -653,7 +661,7 @@ def run_matrix(args):
     hbm = float(peaks["hbm_gbs"])
     eff_gbs = replica_value(weight_bytes, world, ms_per_step)
     achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
-    traffic = profile_traffic(args.workload, batch)
+    traffic = profile_traffic(args.workload + format_suffix(args), batch)
 
     # End to end through the public API with host buffers: pinned x in, y out.
     e2e = None

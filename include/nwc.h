@@ -68,10 +68,18 @@ typedef enum {
   NWC_CODE_PREFIX = 0,
   /* "NWR1": exponent bits 14..8 ranked by count in a unary code with the sign
    * bit beside it and an escape ("NWC", "How it works > Prefix code instead of
-   * rANS", format v9); bits 7..0 raw.  Host encoder only for now: nwc_plan,
-   * nwc_plan_size (device_bytes = 0) and nwc_compress_host take it; the calls
-   * that need a device image return UNSUPPORTED. */
-  NWC_CODE_RANK = 1
+   * rANS", format v9); bits 7..0 raw; one stream per lane.  Every call takes
+   * it. */
+  NWC_CODE_RANK = 1,
+  /* "NWE1": the `keep` most frequent exponent bytes in the length-limited
+   * canonical prefix code; a run of 64 weights of a tile row (one row, one
+   * 64-column group) that holds any other exponent keeps its exponent bytes
+   * verbatim in the tile's chunk, beside a 16-byte flag field ("Unweight",
+   * "Compressing BF16 Weights": the 16 most common exponents cover nearly all
+   * weights; rare ones are stored with their whole row of 64, so the decoder
+   * branches once per run).  Sign and fraction raw; one stream per lane;
+   * lmax <= 7.  Every call takes it. */
+  NWC_CODE_ESCAPE = 2
 } nwc_code;
 
 /* Plan options.  Set struct_size = sizeof(nwc_opts); pass NULL for the defaults
@@ -84,13 +92,18 @@ typedef enum {
  * bits and every peek holds two complete codes; with 8..12 it peeks 12 bits and
  * takes a second lookup when a pair does not fit.
  * lmax, NWC_CODE_RANK: the number of ranks, 0 = 7, else in [1, 7].
+ * lmax, NWC_CODE_ESCAPE: 0 = 7, else in [1, 7] and at least ceil(log2(coded
+ * exponents)) (8..12 are a valid format that no kernel reads: UNSUPPORTED).
+ * keep (a struct_size that ends before it, or 0, means 16): NWC_CODE_ESCAPE's
+ * number of coded exponents, 1..256; ignored by the other codes.
  * tile_rows must be 8; tile_cols must be 64, 128, 256 or 512.
  * streams (a struct_size that ends before it means 1): bit streams per lane
  * and tile, each lane's symbol pairs dealt to its streams in turn (header
- * offset 60 holds streams - 1), with the prefix code only.  Every kernel
- * reads 1 and 2 (a lane then follows two independent decode chains); 4 is a
- * host-encoder-only layout: nwc_plan_size reports device_bytes = 0 and the
- * calls that need a device image return UNSUPPORTED. */
+ * offset 60 holds streams - 1), with NWC_CODE_PREFIX only (others:
+ * UNSUPPORTED).  Every kernel reads 1 and 2 (a lane then follows two
+ * independent decode chains); 4 is a host-encoder-only layout: nwc_plan_size
+ * reports device_bytes = 0 and the calls that need a device image return
+ * UNSUPPORTED. */
 typedef struct {
   uint32_t struct_size;
   uint32_t lmax;
@@ -99,6 +112,7 @@ typedef struct {
   uint32_t threads; /* host encoder threads; 0 = hardware concurrency */
   uint32_t code;    /* nwc_code */
   uint32_t streams; /* bit streams per lane and tile: 0 or 1, 2, 4 (see below) */
+  uint32_t keep;    /* NWC_CODE_ESCAPE: exponents coded, 0 = 16 (see below) */
 } nwc_opts;
 
 /* Library version: major * 10000 + minor * 100 + patch. */

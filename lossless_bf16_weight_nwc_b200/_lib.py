@@ -47,14 +47,14 @@ class nwc_tc_schedule_info(ctypes.Structure):
                 ("ksplit", ctypes.c_int32), ("a_stages", ctypes.c_int32)]
 
 
-NWC_CODE_PREFIX, NWC_CODE_RANK = 0, 1
+NWC_CODE_PREFIX, NWC_CODE_RANK, NWC_CODE_ESCAPE = 0, 1, 2
 
 
 class nwc_opts(ctypes.Structure):
     _fields_ = [("struct_size", ctypes.c_uint32), ("lmax", ctypes.c_uint32),
                 ("tile_rows", ctypes.c_uint32), ("tile_cols", ctypes.c_uint32),
                 ("threads", ctypes.c_uint32), ("code", ctypes.c_uint32),
-                ("streams", ctypes.c_uint32)]
+                ("streams", ctypes.c_uint32), ("keep", ctypes.c_uint32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -135,13 +135,14 @@ def nwc_version() -> int:
 
 
 def nwc_plan(w_host: np.ndarray, lmax: int = 0, tile_cols: int = 512, threads: int = 0,
-             code: int = NWC_CODE_PREFIX, streams: int = 1):
+             code: int = NWC_CODE_PREFIX, streams: int = 1, keep: int = 0):
     """code NWC_CODE_RANK: the ranked unary code, lmax = number of ranks (0 = 7);
-    streams 2 or 4: bit streams per lane (the kernels read 1 and 2; 4 is host
-    encoder only, nwc_compress_host)."""
+    code NWC_CODE_ESCAPE: the `keep` (0 = 16) most frequent exponents coded, runs
+    of 64 holding another one verbatim; streams 2 or 4: bit streams per lane
+    (the kernels read 1 and 2; 4 is host encoder only, nwc_compress_host)."""
     w = np.ascontiguousarray(w_host, dtype=np.uint16)
     rows, cols = w.shape
-    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads, code, streams)
+    opts = nwc_opts(ctypes.sizeof(nwc_opts), lmax, 8, tile_cols, threads, code, streams, keep)
     plan = ctypes.c_void_p()
     _check(LIB.nwc_plan(w.ctypes.data, rows, cols, ctypes.byref(opts), ctypes.byref(plan)),
            "nwc_plan")
@@ -345,13 +346,15 @@ class CompressedMatrix:
     @classmethod
     def compress(cls, w_host: np.ndarray, device="cuda", lmax: int = 0, tile_cols: int = 512,
                  threads: int = 0, stream=None, streams: int = 1,
-                 code: int = NWC_CODE_PREFIX) -> "CompressedMatrix":
+                 code: int = NWC_CODE_PREFIX, keep: int = 0) -> "CompressedMatrix":
         """streams: bit streams per lane and tile (1 or 2; with 2 a lane's
         decoder follows two independent streams).  code NWC_CODE_RANK: the
-        ranked unary code, lmax = its number of ranks (0 = 7)."""
+        ranked unary code, lmax = its number of ranks (0 = 7).  code
+        NWC_CODE_ESCAPE: the `keep` (0 = 16) most frequent exponents coded, a
+        run of 64 weights holding another one kept verbatim."""
         import torch
         plan = nwc_plan(w_host, lmax=lmax, tile_cols=tile_cols, threads=threads, streams=streams,
-                        code=code)
+                        code=code, keep=keep)
         try:
             dev_bytes, blob_bytes = nwc_plan_size(plan)
             image = torch.empty(dev_bytes, dtype=torch.uint8, device=device)
@@ -363,7 +366,8 @@ class CompressedMatrix:
 
     @classmethod
     def compress_fused(cls, parts, device="cuda", lmax: int = 0, tile_cols: int = 512,
-                       threads: int = 0, stream=None, streams: int = 1) -> "CompressedMatrix":
+                       threads: int = 0, stream=None, streams: int = 1,
+                       code: int = NWC_CODE_PREFIX, keep: int = 0) -> "CompressedMatrix":
         """Projections that read the same input (q, k, v; gate, up) held as one
         matrix: the parts' rows stacked in order under one code table, so that a
         call is one launch ("NWC — Neural Weight Compression", "Install": fuse
@@ -373,7 +377,8 @@ class CompressedMatrix:
         if not ws or any(w.ndim != 2 or w.shape[1] != ws[0].shape[1] for w in ws):
             raise ValueError("parts: one or more 2-D matrices with the same number of columns")
         m = cls.compress(np.concatenate(ws, axis=0), device=device, lmax=lmax,
-                         tile_cols=tile_cols, threads=threads, stream=stream, streams=streams)
+                         tile_cols=tile_cols, threads=threads, stream=stream, streams=streams,
+                         code=code, keep=keep)
         m.row_splits = [int(v) for v in np.cumsum([0] + [w.shape[0] for w in ws])]
         return m
 

@@ -10,7 +10,8 @@ workload.  Here a strategy is
   matrix), the code limit (7 bits, whose 14-bit table peek always holds two
   codes, or a longer limit), the bit streams per lane (1, or 2 so that a lane
   follows two independent decode chains) and the exponent code (the
-  length-limited prefix code, or the table-free ranked unary code);
+  length-limited prefix code, the table-free ranked unary code, or the prefix
+  code of the 16 most frequent exponents with verbatim runs for the rest);
 * the kernel, chosen per call: the CUDA-core kernel (mma.sync on the decoded
   registers, up to 16 rows of x per launch, the matrix decoded again for every
   16 rows) or the tensor-core kernel (tcgen05, each weight decoded once into
@@ -36,14 +37,15 @@ from typing import Callable, Iterable
 import numpy as np
 
 TILE_COLS = (64, 128, 256, 512)
-CODES = ("prefix", "rank")
+CODES = ("prefix", "rank", "escape")
 KERNELS = ("cuda", "tensor")
 
 
 @dataclasses.dataclass(frozen=True)
 class Strategy:
     tile_cols: int = 512
-    lmax: int = 0          # prefix: 0 = automatic (7 unless > 128 exponents); rank: ranks (0 = 7)
+    lmax: int = 0          # prefix: 0 = automatic (7 unless > 128 exponents); rank: ranks
+                           # (0 = 7); escape: 0 = 7, else 1..7
     streams: int = 1
     code: str = "prefix"
     kernel: str = "cuda"
@@ -62,7 +64,7 @@ def default_candidates(batch: int) -> list[Strategy]:
     (the tensor-core kernel for any batch; the CUDA-core one up to 16 rows of x
     per launch, so for larger batches only as a baseline)."""
     formats = [(512, 0, 1, "prefix"), (512, 0, 2, "prefix"), (256, 0, 1, "prefix"),
-               (512, 12, 1, "prefix"), (512, 0, 1, "rank")]
+               (512, 12, 1, "prefix"), (512, 0, 1, "rank"), (512, 0, 1, "escape")]
     kernels = ("cuda", "tensor") if batch >= 8 else ("cuda",)
     return [Strategy(*f, kernel=k) for f in formats for k in kernels]
 
@@ -97,10 +99,10 @@ def validate_candidates(candidates: Iterable[Strategy]) -> list[Strategy]:
             raise ValueError(f"code {s.code!r}: one of {CODES}")
         if s.kernel not in KERNELS:
             raise ValueError(f"kernel {s.kernel!r}: one of {KERNELS}")
-        if s.streams not in (1, 2) or (s.code == "rank" and s.streams != 1):
-            raise ValueError(f"streams {s.streams}: 1 or 2 (1 for the rank code)")
-        if not 0 <= s.lmax <= (7 if s.code == "rank" else 12):
-            raise ValueError(f"lmax {s.lmax}: 0 (automatic) or 1..12 (ranks: 1..7)")
+        if s.streams not in (1, 2) or (s.code != "prefix" and s.streams != 1):
+            raise ValueError(f"streams {s.streams}: 1 or 2 (1 for the rank and escape codes)")
+        if not 0 <= s.lmax <= (12 if s.code == "prefix" else 7):
+            raise ValueError(f"lmax {s.lmax}: 0 (automatic) or 1..12 (rank, escape: 1..7)")
         if s not in out:
             out.append(s)
     if not out:
@@ -251,10 +253,10 @@ class Tuner:
 
     @staticmethod
     def _compress_default(w_host, s: Strategy):
-        from ._lib import NWC_CODE_PREFIX, NWC_CODE_RANK, CompressedMatrix
+        from ._lib import NWC_CODE_ESCAPE, NWC_CODE_PREFIX, NWC_CODE_RANK, CompressedMatrix
+        code = {"prefix": NWC_CODE_PREFIX, "rank": NWC_CODE_RANK, "escape": NWC_CODE_ESCAPE}
         return CompressedMatrix.compress(w_host, tile_cols=s.tile_cols, lmax=s.lmax,
-                                         streams=s.streams,
-                                         code=NWC_CODE_RANK if s.code == "rank" else NWC_CODE_PREFIX)
+                                         streams=s.streams, code=code[s.code])
 
 
 def sweep(workloads, batches, path: str, reps: int = 30) -> dict:

@@ -18,6 +18,11 @@
 // code of "NWC", "Prefix code instead of rANS" (format v9): exponent bits
 // 14..8 ranked by count, the sign bit raw in the stream, bits 7..0 raw; step 4
 // is shared.
+// The variant NWE1 (plan_build_escape) follows "Unweight", "Compressing BF16
+// Weights": only the K most frequent exponents are coded (step 3 over the runs
+// that hold no other exponent); a run of 64 weights of a tile row that holds
+// another one keeps its exponent bytes verbatim in the chunk, and its symbols
+// leave the lane streams.
 #include <algorithm>
 #include <cstring>
 #include <functional>
@@ -75,7 +80,7 @@ inline void symbol_of(const nwc_plan_s& p, const TileView& v, int r, int c, uint
   const bool in = v.inside(r, c);
   const uint16_t x = in ? v.at(r, c) : 0;
   *raw = 0;
-  if (p.code_kind == 0) {
+  if (p.code_kind != 1) {
     uint8_t s = v.filler;
     if (in) {
       s = exponent_byte(x);
@@ -99,6 +104,40 @@ inline void symbol_of(const nwc_plan_s& p, const TileView& v, int r, int c, uint
 // streams: consecutive symbol pairs go to the lane's streams in turn.
 inline int stream_of(int t, int k, int S) { return t * S + (k / 2) % S; }
 
+// NWE1: whether run (row r, group m) of tile u is verbatim, and how many of
+// the tile's runs are.
+inline bool escaped(const nwc_plan_s& p, int64_t u, int r, int m) {
+  return (p.esc_flags[(size_t)(8 * u + r)] >> m) & 1u;
+}
+inline uint32_t escaped_runs(const nwc_plan_s& p, int64_t u) {
+  uint32_t n = 0;
+  for (int r = 0; r < kTileRows; ++r) n += (uint32_t)__builtin_popcount(p.esc_flags[(size_t)(8 * u + r)]);
+  return n;
+}
+
+// Exponent-byte histogram of the rows x cols weights, one partial per thread.
+void exponent_histogram(const uint16_t* w, int64_t rows, int64_t cols, unsigned nt,
+                        uint64_t cnt[256]) {
+  std::vector<std::vector<uint64_t>> part(nt, std::vector<uint64_t>(256, 0));
+  {
+    std::vector<std::thread> pool;
+    for (unsigned q = 0; q < nt; ++q) {
+      pool.emplace_back([&, q] {
+        const int64_t b = rows * q / nt, e = rows * (q + 1) / nt;
+        uint64_t* h = part[q].data();
+        for (int64_t r = b; r < e; ++r) {
+          const uint16_t* row = w + r * cols;
+          for (int64_t c = 0; c < cols; ++c) h[exponent_byte(row[c])] += 1;
+        }
+      });
+    }
+    for (auto& t : pool) t.join();
+  }
+  for (int s = 0; s < 256; ++s) cnt[s] = 0;
+  for (unsigned q = 0; q < nt; ++q)
+    for (int s = 0; s < 256; ++s) cnt[s] += part[q][s];
+}
+
 // Bits of each stream in tile u (kLanes * p.streams entries).
 void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t* bits) {
   const int64_t i = u % p.tiles_r, j = u / p.tiles_r;
@@ -110,7 +149,8 @@ void lane_bits(const nwc_plan_s& p, const uint16_t* w, int64_t u, uint32_t* bits
       const int t = 4 * r + (c % 64) / 16;  // lane t = 4 r + q owns row r, columns 16 q .. of a group
       const int k = 16 * (c / 64) + c % 16;  // the lane's symbol index
       const int sigma = stream_of(t, k, S);
-      if (p.code_kind == 0) {
+      if (p.code_kind == 2 && escaped(p, u, r, c / 64)) continue;
+      if (p.code_kind != 1) {
         const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
         bits[sigma] += p.len[s];
       } else {
@@ -267,26 +307,8 @@ int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows
   p->tiles_c = (cols + tile_cols - 1) / tile_cols;
   p->tiles = p->tiles_r * p->tiles_c;
 
-  // Histogram, one partial per thread.
-  const unsigned nt = p->threads;
-  std::vector<std::vector<uint64_t>> part(nt, std::vector<uint64_t>(256, 0));
-  {
-    std::vector<std::thread> pool;
-    for (unsigned q = 0; q < nt; ++q) {
-      pool.emplace_back([&, q] {
-        const int64_t b = rows * q / nt, e = rows * (q + 1) / nt;
-        uint64_t* h = part[q].data();
-        for (int64_t r = b; r < e; ++r) {
-          const uint16_t* row = w + r * cols;
-          for (int64_t c = 0; c < cols; ++c) h[exponent_byte(row[c])] += 1;
-        }
-      });
-    }
-    for (auto& t : pool) t.join();
-  }
-  uint64_t cnt[256] = {};
-  for (unsigned q = 0; q < nt; ++q)
-    for (int s = 0; s < 256; ++s) cnt[s] += part[q][s];
+  uint64_t cnt[256];
+  exponent_histogram(w, rows, cols, p->threads, cnt);
   uint32_t filler = 0;
   for (uint32_t s = 1; s < 256; ++s)
     if (cnt[s] > cnt[filler]) filler = s;
@@ -393,6 +415,104 @@ int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile
   return 0;
 }
 
+int plan_build_escape(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_cols,
+                      uint32_t lmax, uint32_t keep, uint32_t threads, nwc_plan_s* p) {
+  if (keep < 1 || keep > 256) return -1;
+  if (lmax == 0) lmax = kEscMaxLmax;
+  if (lmax > kEscMaxLmax) return -1;
+  p->code_kind = 2;
+  p->streams = 1;
+  p->rows = rows;
+  p->cols = cols;
+  p->tile_rows = kTileRows;
+  p->tile_cols = tile_cols;
+  p->lmax = lmax;
+  p->threads = hardware_threads(threads);
+  p->tiles_r = (rows + kTileRows - 1) / kTileRows;
+  p->tiles_c = (cols + tile_cols - 1) / tile_cols;
+  p->tiles = p->tiles_r * p->tiles_c;
+
+  // Histogram with the fillers; the filler is the most frequent exponent.
+  uint64_t cnt[256];
+  exponent_histogram(w, rows, cols, p->threads, cnt);
+  uint32_t filler = 0;
+  for (uint32_t s = 1; s < 256; ++s)
+    if (cnt[s] > cnt[filler]) filler = s;
+  p->filler = filler;
+  cnt[filler] += (uint64_t)(p->tiles_r * kTileRows) * (uint64_t)(p->tiles_c * tile_cols) -
+                 (uint64_t)rows * (uint64_t)cols;
+  // The kept exponents: the `keep` most frequent, smaller symbol first on a tie.
+  std::vector<int> present;
+  for (int s = 0; s < 256; ++s)
+    if (cnt[s]) present.push_back(s);
+  std::stable_sort(present.begin(), present.end(), [&](int a, int b) { return cnt[a] > cnt[b]; });
+  bool kept[256] = {};
+  p->keep = (uint32_t)std::min<size_t>(present.size(), keep);
+  for (uint32_t q = 0; q < p->keep; ++q) kept[present[q]] = true;
+
+  // Verbatim runs per tile, and the histogram of the other runs (one partial
+  // per part of the tiles).
+  const int groups = (int)(tile_cols / 64);
+  p->esc_flags.assign((size_t)(8 * p->tiles), 0);
+  const unsigned parts = (unsigned)std::min<int64_t>(p->threads, p->tiles);
+  std::vector<std::vector<uint64_t>> part(parts, std::vector<uint64_t>(256, 0));
+  std::vector<uint64_t> part_runs(parts, 0);
+  {
+    std::vector<std::thread> pool;
+    for (unsigned q = 0; q < parts; ++q) {
+      pool.emplace_back([&, q] {
+        const int64_t b = p->tiles * q / parts, e = p->tiles * (q + 1) / parts;
+        uint64_t* h = part[q].data();
+        for (int64_t u = b; u < e; ++u) {
+          const int64_t i = u % p->tiles_r, j = u / p->tiles_r;
+          TileView v{w, rows, cols, i * kTileRows, j * (int64_t)tile_cols, (uint8_t)filler};
+          for (int r = 0; r < kTileRows; ++r) {
+            for (int m = 0; m < groups; ++m) {
+              uint64_t run[256 / 64] = {};  // exponents present in the run
+              for (int c = 64 * m; c < 64 * m + 64; ++c) {
+                const uint8_t s = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
+                run[s / 64] |= 1ull << (s % 64);
+              }
+              bool rare = false;
+              for (int s = 0; s < 256 && !rare; ++s) rare = ((run[s / 64] >> (s % 64)) & 1u) && !kept[s];
+              if (rare) {
+                p->esc_flags[(size_t)(8 * u + r)] |= (uint8_t)(1u << m);
+                part_runs[q] += 1;
+                continue;
+              }
+              for (int c = 64 * m; c < 64 * m + 64; ++c)
+                h[v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler] += 1;
+            }
+          }
+        }
+      });
+    }
+    for (auto& t : pool) t.join();
+  }
+  uint64_t ccnt[256] = {};
+  p->n_escaped = 0;
+  for (unsigned q = 0; q < parts; ++q) {
+    for (int s = 0; s < 256; ++s) ccnt[s] += part[q][s];
+    p->n_escaped += part_runs[q];
+  }
+  uint64_t coded = 0;
+  for (int s = 0; s < 256; ++s) coded += ccnt[s];
+  std::memset(p->len, 0, sizeof(p->len));
+  if (coded && !code_lengths(ccnt, lmax, p->len)) return -1;
+  canonical_codes(p->len, p->code);
+  p->coded_bits = 0;
+  for (int s = 0; s < 256; ++s) p->coded_bits += ccnt[s] * p->len[s];
+  const int rc = plan_tiles(w, p);
+  if (rc != 0) return rc;
+  const ImageLayout L =
+      image_layout(p->blob_bytes, p->lmax, (uint64_t)p->tiles_r, (uint64_t)p->tiles_c);
+  p->table_off = L.table_off;
+  p->sched_off = L.sched_off;
+  p->scratch_off = L.scratch_off;
+  p->device_bytes = L.device_bytes;
+  return 0;
+}
+
 void build_rank_table(const uint8_t* ranked, uint32_t ranks, uint32_t* out) {
   std::memset(out, 0, kRankTableBytes);
   uint8_t bytes[8] = {};
@@ -411,8 +531,9 @@ int plan_tiles(const uint16_t* w, nwc_plan_s* p) {
     uint32_t bits[kLanes * kMaxStreams];
     for (int64_t u = b; u < e; ++u) {
       lane_bits(*p, w, u, bits);
-      const uint32_t bytes =
+      uint32_t bytes =
           raw_bytes(tile_cols) + n + (uint32_t)round_up(stream_bytes_of(bits, n), 16);
+      if (p->code_kind == 2) bytes += kEscFlagBytes + kEscRunBytes * escaped_runs(*p, u);
       chunk16[(size_t)u] = bytes / 16;
     }
   });
@@ -432,7 +553,7 @@ int plan_tiles(const uint16_t* w, nwc_plan_s* p) {
 void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
   BlobHeader h;
   std::memset(&h, 0, sizeof(h));
-  h.magic = p.code_kind == 0 ? kMagic : kRankMagic;
+  h.magic = p.code_kind == 0 ? kMagic : p.code_kind == 1 ? kRankMagic : kEscMagic;
   h.version = kVersion;
   h.header_bytes = kHeaderBytes;
   h.lmax = p.lmax;
@@ -443,15 +564,16 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
   h.tiles_r = (uint64_t)p.tiles_r;
   h.tiles_c = (uint64_t)p.tiles_c;
   h.filler = p.filler;
-  h.zero = p.streams - 1;  // streams per lane, S - 1
+  h.zero = p.code_kind == 2 ? p.keep : p.streams - 1;  // NWE1: K; else S - 1
   h.lens_off = kLensOffset;
   h.index_off = kIndexOffset;
   h.tiles_off = p.tiles_off;
   h.total_bytes = p.blob_bytes;
   h.coded_bits = p.coded_bits;
+  if (p.code_kind == 2) std::memcpy(h.pad, &p.n_escaped, 8);  // offset 104
   std::memset(blob, 0, p.tiles_off);
   std::memcpy(blob, &h, sizeof(h));
-  if (p.code_kind == 0)
+  if (p.code_kind != 1)
     std::memcpy(blob + kLensOffset, p.len, 256);
   else
     std::memcpy(blob + kLensOffset, p.rank_table, p.ranks);
@@ -468,10 +590,27 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
       TileView v{w, p.rows, p.cols, i * kTileRows, j * (int64_t)p.tile_cols, (uint8_t)p.filler};
       uint8_t* chunk = blob + p.tiles_off + 16ull * p.index[(size_t)u];
       const uint32_t chunk_bytes = 16u * (p.index[(size_t)u + 1] - p.index[(size_t)u]);
-      const uint32_t area = chunk_bytes - raw_n - nstreams;
+      const bool esc = p.code_kind == 2;
+      const uint32_t head =
+          raw_n + (esc ? kEscFlagBytes + kEscRunBytes * escaped_runs(p, u) : 0u);
+      const uint32_t area = chunk_bytes - head - nstreams;
       uint8_t* raw = chunk;
-      uint8_t* lane_len = chunk + raw_n;
-      uint8_t* words = chunk + raw_n + nstreams;
+      uint8_t* lane_len = chunk + head;
+      uint8_t* words = chunk + head + nstreams;
+      if (esc) {
+        // Flags, then the verbatim runs' exponent bytes in (row, group) order.
+        uint8_t* flags = chunk + raw_n;
+        std::memset(flags, 0, kEscFlagBytes);
+        uint8_t* run = flags + kEscFlagBytes;
+        for (int r = 0; r < kTileRows; ++r) {
+          flags[r] = p.esc_flags[(size_t)(8 * u + r)];
+          for (uint32_t g = 0; g < groups; ++g) {
+            if (!escaped(p, u, r, (int)g)) continue;
+            for (int c = (int)(64 * g); c < (int)(64 * g) + 64; ++c)
+              *run++ = v.inside(r, c) ? exponent_byte(v.at(r, c)) : v.filler;
+          }
+        }
+      }
       seq.assign(area, 0);
       uint32_t out = 0;
       for (int sigma = 0; sigma < (int)nstreams; ++sigma) {
@@ -493,6 +632,7 @@ void encode_blob(const nwc_plan_s& p, const uint16_t* w, uint8_t* blob) {
             uint8_t rb;
             symbol_of(p, v, r, c, &code, &len, &rb);
             raw[(k / 16) * 512 + 16 * t + (k % 16)] = rb;
+            if (esc && escaped(p, u, r, (int)g)) continue;  // verbatim: no bits
             accb = (accb << len) | code;
             nacc += len;
             while (nacc >= 8) {
@@ -521,10 +661,12 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   if (!blob || head_bytes < kHeaderBytes + 256 || head_bytes > bytes) return false;
   BlobHeader h;
   std::memcpy(&h, blob, sizeof(h));
-  const bool rank = h.magic == kRankMagic;
-  if ((h.magic != kMagic && !rank) || h.version != kVersion || h.header_bytes != kHeaderBytes)
+  const bool rank = h.magic == kRankMagic, esc = h.magic == kEscMagic;
+  if ((h.magic != kMagic && !rank && !esc) || h.version != kVersion ||
+      h.header_bytes != kHeaderBytes)
     return false;
-  const uint32_t lmax_cap = rank ? (uint32_t)kMaxRanks : (uint32_t)kMaxLmax;
+  const uint32_t lmax_cap =
+      rank ? (uint32_t)kMaxRanks : esc ? kEscMaxLmax : (uint32_t)kMaxLmax;
   if (h.lmax < 1 || h.lmax > lmax_cap || h.tile_rows != (uint32_t)kTileRows) return false;
   if (h.tile_cols < 64 || h.tile_cols > (uint32_t)kMaxTileCols || h.tile_cols % 64) return false;
   if (h.rows < 1 || h.cols < 1 || h.rows > (1ull << 40) || h.cols > (1ull << 40)) return false;
@@ -532,9 +674,10 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
     return false;
   if (h.lens_off != kLensOffset || h.index_off != kIndexOffset || h.filler > 255) return false;
   // The streams field holds S - 1 for S bit streams per lane (1 or 2 here;
-  // the ranked unary code has one).
-  if (h.zero + 1 > (rank ? 1u : kMaxDeviceStreams)) return false;
-  const uint32_t S = h.zero + 1;
+  // the ranked unary code has one); NWE1 has one and holds K there.
+  if (esc ? (h.zero < 1 || h.zero > 256) : h.zero + 1 > (rank ? 1u : kMaxDeviceStreams))
+    return false;
+  const uint32_t S = esc ? 1u : h.zero + 1;
   // Every tile has a 4-byte index entry inside the head, which bounds the tile
   // count before it is formed: no size computed from it below can wrap around.
   const uint64_t max_tiles = head_bytes / 4;
@@ -558,20 +701,28 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
     if (h.filler != lens[0]) return false;
   } else {
     double kraft = 0;
+    uint32_t coded = 0;
     for (int s = 0; s < 256; ++s) {
       if (lens[s] > h.lmax) return false;
-      if (lens[s]) kraft += 1.0 / double(1u << lens[s]);
+      if (lens[s]) {
+        kraft += 1.0 / double(1u << lens[s]);
+        ++coded;
+      }
     }
-    if (kraft > 1.0 || lens[h.filler] == 0) return false;
+    if (kraft > 1.0) return false;
+    // NWE1: no more codes than kept exponents (none at all when every run is
+    // verbatim, so the filler may have none); NWB1: the filler has a code.
+    if (esc ? coded > h.zero : lens[h.filler] == 0) return false;
   }
   auto index_at = [&](uint64_t u) {
     uint32_t v;
     std::memcpy(&v, blob + kIndexOffset + 4 * u, 4);
     return v;
   };
-  const uint64_t max_chunk =
-      rank ? max_rank_chunk_bytes(h.tile_cols, h.lmax) : max_chunk_bytes(h.tile_cols, h.lmax, S);
-  const uint64_t min_chunk = raw_bytes(h.tile_cols) + kLanes * S;
+  const uint64_t max_chunk = rank  ? max_rank_chunk_bytes(h.tile_cols, h.lmax)
+                             : esc ? max_escape_chunk_bytes(h.tile_cols, h.lmax)
+                                   : max_chunk_bytes(h.tile_cols, h.lmax, S);
+  const uint64_t min_chunk = raw_bytes(h.tile_cols) + kLanes * S + (esc ? kEscFlagBytes : 0u);
   uint64_t largest = 0;
   if (index_at(0) != 0) return false;
   uint32_t prev = 0;
@@ -589,7 +740,7 @@ bool parse_blob(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_ha
   hd->tile_cols = h.tile_cols;
   hd->lmax = h.lmax;
   hd->streams = S;
-  hd->code_kind = rank ? 1u : 0u;
+  hd->code_kind = rank ? 1u : esc ? 2u : 0u;
   hd->filler = h.filler;
   hd->tiles_r = (int64_t)h.tiles_r;
   hd->tiles_c = (int64_t)h.tiles_c;

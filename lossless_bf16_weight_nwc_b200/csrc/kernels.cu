@@ -30,6 +30,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels.cuh"
 #include "nwc_format.h"
@@ -393,6 +394,9 @@ struct StreamDecoder<kCode12> {
     br.refill();
   }
 };
+// NWE1 codes its kept exponents exactly as the 14-bit prefix code.
+template <>
+struct StreamDecoder<kCodeEsc> : StreamDecoder<kCode14> {};
 template <>
 struct StreamDecoder<kCodeRank> {
   RankReader r;
@@ -473,6 +477,54 @@ __device__ __forceinline__ void lane_stream_starts(uint32_t chunk, int raw, int 
     start[0] = incl - mine;
     start[1] = start[0] + len0;
   }
+}
+
+// Verbatim runs of an NWE1 tile ("Unweight", "Compressing BF16 Weights": a
+// run of 64 weights of a row holding a rare exponent is stored whole, so the
+// decoder branches once per run).  After the raw plane a chunk holds flags
+// u8[16] (bit m of byte g: run (row g, group m) is verbatim), the runs'
+// exponent bytes (64 each, in (g, m) order), then the lane lengths and
+// streams.  Lane 4 g + c reads bytes 16 c .. 16 c + 15 of its row's runs.
+struct EscRuns {
+  uint32_t mine;  // bit m: this lane's 16 symbols of group m are verbatim;
+                  // bit 31: the flag field is corrupt
+  uint32_t at;    // shared-memory address of its bytes in its next such run
+};
+constexpr uint32_t kEscCorrupt = 1u << 31;
+// flags: shared-memory address of the flag field of a tile of CP groups;
+// limit: end of the readable buffer.  Returns the offset of the lane lengths
+// from the flags.  A flag field that names a group past the tile, or more
+// runs than the buffer holds, is corrupt: the lane then decodes its streams
+// from just after the flags (a wrong result, but every read stays inside the
+// buffer, which holds at least the flags and the lane lengths).
+template <int CP>
+__device__ __forceinline__ uint32_t esc_runs(uint32_t flags, uint32_t limit, int lane,
+                                             EscRuns& er) {
+  const uint2 f = lds64(flags);
+  const int g = lane >> 2;
+  const uint32_t lo = g < 4 ? f.x : f.y;
+  const int sh = 8 * (g & 3);
+  const uint32_t before =
+      __popc(lo & ((1u << sh) - 1u)) + (g < 4 ? 0u : (uint32_t)__popc(f.x));
+  const uint32_t lens = kEscFlagBytes + kEscRunBytes * (uint32_t)(__popc(f.x) + __popc(f.y));
+  constexpr uint32_t kValid = 0x01010101u * ((1u << CP) - 1u);
+  if (((f.x | f.y) & ~kValid) != 0u || flags + lens + kLanes > limit) {
+    er.mine = kEscCorrupt;
+    er.at = flags;
+    return kEscFlagBytes;
+  }
+  er.mine = (lo >> sh) & 0xFFu;
+  er.at = flags + kEscFlagBytes + kEscRunBytes * before + 16u * (uint32_t)(lane & 3);
+  return lens;
+}
+// Table-entry form (exponent bytes at their BF16 positions, nothing else) of
+// pairs 4 q .. 4 q + 3 of a lane's 16 verbatim exponent bytes.
+__device__ __forceinline__ void esc_quad(const uint4& ev, int q, uint32_t (&e)[4]) {
+  const uint32_t a = q == 0 ? ev.x : ev.z, b = q == 0 ? ev.y : ev.w;
+  e[0] = __byte_perm(a, 0u, 0x4140u) << 7;
+  e[1] = __byte_perm(a, 0u, 0x4342u) << 7;
+  e[2] = __byte_perm(b, 0u, 0x4140u) << 7;
+  e[3] = __byte_perm(b, 0u, 0x4342u) << 7;
 }
 
 // A lane's decoder over its S bit streams: quad() yields the table entries of
@@ -676,10 +728,13 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
                                                  uint32_t xrow) {
   constexpr int kRaw = CP * 512;
   LaneDecoder<CODE, S> dec;
+  EscRuns er{0u, 0u};
   {
+    const uint32_t lens =
+        kRaw + (CODE == kCodeEsc ? esc_runs<CP>(chunk + kRaw, limit, lane, er) : 0u);
     uint32_t start[S];
-    lane_stream_starts<S>(chunk, kRaw, lane, start);
-    dec.init(chunk + kRaw + kLanes * S, start, limit, table);
+    lane_stream_starts<S>(chunk, lens, lane, start);
+    dec.init(chunk + lens + kLanes * S, start, limit, table);
   }
   const int g = lane >> 2, c = lane & 3;
   const int64_t cols = p.cols;
@@ -702,10 +757,20 @@ __device__ __forceinline__ void decode_gemv_tile(uint32_t chunk, uint32_t table,
 #pragma unroll 2
   for (int m = 0; m < CP; ++m) {
     const uint4 rv = lds128(chunk + m * 512 + lane * 16);
+    const bool esc = CODE == kCodeEsc && ((er.mine >> m) & 1u);
+    uint4 ev = make_uint4(0u, 0u, 0u, 0u);
+    if (esc) {
+      ev = lds128(er.at);
+      er.at += kEscRunBytes;
+    }
 #pragma unroll
     for (int s2 = 0; s2 < 4; s2 += 2) {
       uint32_t e[4];
-      dec.quad(table, e);  // pairs 2 s2 .. 2 s2 + 3: blocks s2 and s2 + 1
+      if (esc)
+        esc_quad(ev, s2 / 2, e);
+      else
+        dec.quad(table, e);  // pairs 2 s2 .. 2 s2 + 3: blocks s2 and s2 + 1
+      if (CODE == kCodeEsc) __syncwarp();  // the MMAs below are warp-wide
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int s = s2 + h;
@@ -946,11 +1011,15 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     if (!wait_batch(s, k, wc)) return;
     const int64_t i = pos.i, j = pos.j;
     LaneDecoder<CODE, S> dec;
+    EscRuns er{0u, 0u};
     {
+      const uint32_t lens =
+          kRaw + (CODE == kCodeEsc ? esc_runs<CP>(chunk + kRaw, limit, lane, er) : 0u);
       uint32_t start[S];
-      lane_stream_starts<S>(chunk, kRaw, lane, start);
-      dec.init(chunk + kRaw + kLanes * S, start, limit, table);
+      lane_stream_starts<S>(chunk, lens, lane, start);
+      dec.init(chunk + lens + kLanes * S, start, limit, table);
     }
+    if (er.mine & kEscCorrupt) invalid |= kEntryInvalid;
     // Lane L owns row L / 4 of the tile and 16 consecutive columns per group.
     const int64_t row = i * 8 + (lane >> 2);
     const bool row_in = row < p.rows;
@@ -959,11 +1028,20 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1) decompress_kernel(TileParams
     for (int g = 0; g < CP; ++g) {
       const uint4 rv = lds128(chunk + g * 512 + lane * 16);
       const int64_t col = j * (CP * 64) + g * 64 + 16 * (lane & 3);
+      const bool esc = CODE == kCodeEsc && ((er.mine >> g) & 1u);
+      uint4 ev = make_uint4(0u, 0u, 0u, 0u);
+      if (esc) {
+        ev = lds128(er.at);
+        er.at += kEscRunBytes;
+      }
       uint32_t wv[8];
 #pragma unroll
       for (int r = 0; r < 8; r += 4) {
         uint32_t e[4];
-        dec.quad(table, e);
+        if (esc)
+          esc_quad(ev, r / 4, e);
+        else
+          dec.quad(table, e);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           invalid |= e[k];
@@ -1071,8 +1149,11 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
           *reinterpret_cast<uint4*>(stage + o) = __ldg(reinterpret_cast<const uint4*>(chunk + kRaw + o));
       }
       __syncwarp();
+      EscRuns er{0u, 0u};
+      const uint32_t lens = CODE == kCodeEsc ? esc_runs<CP>(sbase, limit, lane, er) : 0u;
+      if (er.mine & kEscCorrupt) invalid |= kEntryInvalid;
       uint32_t start[S];
-      lane_stream_starts<S>(sbase, 0, lane, start);
+      lane_stream_starts<S>(sbase, lens, lane, start);
       if (!have_table) {
         have_table = __all_sync(kFull, wait_bounded(tbar, 0, wc));
         if (!have_table) {
@@ -1082,14 +1163,23 @@ __global__ void __launch_bounds__(kGatherWarps * 32) gather_kernel(GatherParams 
       }
       if (!mine) continue;
       LaneDecoder<CODE, S> dec;
-      dec.init(sbase + kLanes * S, start, limit, table);
+      dec.init(sbase + lens + kLanes * S, start, limit, table);
 #pragma unroll
       for (int m = 0; m < CP; ++m) {
+        const bool esc = CODE == kCodeEsc && ((er.mine >> m) & 1u);
+        uint4 ev = make_uint4(0u, 0u, 0u, 0u);
+        if (esc) {
+          ev = lds128(er.at);
+          er.at += kEscRunBytes;
+        }
         uint32_t wv[8];
 #pragma unroll
         for (int r = 0; r < 8; r += 4) {
           uint32_t e[4];
-          dec.quad(table, e);
+          if (esc)
+            esc_quad(ev, r / 4, e);
+          else
+            dec.quad(table, e);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             invalid |= e[k];
@@ -1461,6 +1551,7 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
       const int64_t j = wk.j_lo + t + jj * TT;
       const bool present = r < rg;
       LaneDecoder<CODE, S> dec;
+      EscRuns er{0u, 0u};
       const uint8_t* raw = nullptr;
       uint4 rv0 = make_uint4(0u, 0u, 0u, 0u), rv1 = rv0;
       uint32_t bw = 0;
@@ -1475,9 +1566,10 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
                                    wait_or_abort(&s.full[bw % kSlots], (bw / kSlots) & 1u, wc,
                                                  tb.abort));
         if (ok) {
+          const uint32_t lens = CODE == kCodeEsc ? esc_runs<CP>(stage, limit, lane, er) : 0u;
           uint32_t start[S];
-          lane_stream_starts<S>(stage, 0, lane, start);
-          dec.init(stage + kLanes * S, start, limit, table);
+          lane_stream_starts<S>(stage, lens, lane, start);
+          dec.init(stage + lens + kLanes * S, start, limit, table);
         } else if (lane == 0) {
           *tb.abort = 1u;
         }
@@ -1496,14 +1588,24 @@ __device__ void tc_decode(const TileParams& p, uint8_t* smem, const Smem& s, con
           const uint4 rv = rv0;
           rv0 = rv1;
           if (m + 2 < CP) rv1 = ldg_stream128(raw + (m + 2) * 512 + lane * 16);
+          const bool esc = CODE == kCodeEsc && ((er.mine >> m) & 1u);
+          uint4 ev = make_uint4(0u, 0u, 0u, 0u);
+          if (esc) {
+            ev = lds128(er.at);
+            er.at += kEscRunBytes;
+          }
           uint32_t wv[8];
 #pragma unroll
           for (int k = 0; k < 8; k += 4) {
             uint32_t e[4];
-            dec.quad(table, e);
+            if (esc)
+              esc_quad(ev, k / 4, e);
+            else
+              dec.quad(table, e);
 #pragma unroll
             for (int q = 0; q < 4; ++q) wv[k + q] = assemble<CODE>(raw_pair_r(rv, k + q), e[q]);
           }
+          if (CODE == kCodeEsc) __syncwarp();
           sts128(arow + chunk_lo, wv[0], wv[1], wv[2], wv[3]);
           sts128(arow + chunk_hi, wv[4], wv[5], wv[6], wv[7]);
         }
@@ -1775,7 +1877,7 @@ cudaError_t launch_gemv_s(const TileParams& p, const LaunchShape& s, cudaStream_
 
 template <int CP, int CODE>
 cudaError_t launch_gemv_cp(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
-  if constexpr (CODE == kCodeRank) {
+  if constexpr (CODE == kCodeRank || CODE == kCodeEsc) {
     return launch_gemv_s<CP, CODE, 1>(p, s, stream);
   } else {
     return p.streams == 2 ? launch_gemv_s<CP, CODE, 2>(p, s, stream)
@@ -1805,7 +1907,7 @@ cudaError_t launch_gemv_tc_s(const TileParams& p, const CUtensorMap& tmap, const
 template <int CP, int CODE>
 cudaError_t launch_gemv_tc_t(const TileParams& p, const CUtensorMap& tmap, const LaunchShape& s,
                              cudaStream_t stream) {
-  if constexpr (CODE == kCodeRank) {
+  if constexpr (CODE == kCodeRank || CODE == kCodeEsc) {
     return launch_gemv_tc_s<CP, CODE, 1>(p, tmap, s, stream);
   } else {
     return p.streams == 2 ? launch_gemv_tc_s<CP, CODE, 2>(p, tmap, s, stream)
@@ -1824,7 +1926,7 @@ cudaError_t launch_decompress_s(const TileParams& p, const LaunchShape& s, cudaS
 
 template <int CP, int CODE>
 cudaError_t launch_decompress_t(const TileParams& p, const LaunchShape& s, cudaStream_t stream) {
-  if constexpr (CODE == kCodeRank) {
+  if constexpr (CODE == kCodeRank || CODE == kCodeEsc) {
     return launch_decompress_s<CP, CODE, 1>(p, s, stream);
   } else {
     return p.streams == 2 ? launch_decompress_s<CP, CODE, 2>(p, s, stream)
@@ -1868,13 +1970,25 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
   return s;
 }
 
+// Calls f with std::integral_constant<int, code> for a runtime code.
+template <typename F>
+cudaError_t by_code(int code, F&& f) {
+  switch (code) {
+    case kCodeRank: return f(std::integral_constant<int, kCodeRank>{});
+    case kCodeEsc: return f(std::integral_constant<int, kCodeEsc>{});
+    case kCode14: return f(std::integral_constant<int, kCode14>{});
+    case kCode12: return f(std::integral_constant<int, kCode12>{});
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const LaunchShape& s,
                         cudaStream_t stream) {
   switch (tile_cols) {
-    case 512: return code == kCodeRank ? launch_gemv_cp<8, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<8, kCode14>(p, s, stream) : launch_gemv_cp<8, kCode12>(p, s, stream);
-    case 256: return code == kCodeRank ? launch_gemv_cp<4, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<4, kCode14>(p, s, stream) : launch_gemv_cp<4, kCode12>(p, s, stream);
-    case 128: return code == kCodeRank ? launch_gemv_cp<2, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<2, kCode14>(p, s, stream) : launch_gemv_cp<2, kCode12>(p, s, stream);
-    case 64: return code == kCodeRank ? launch_gemv_cp<1, kCodeRank>(p, s, stream) : code == kCode14 ? launch_gemv_cp<1, kCode14>(p, s, stream) : launch_gemv_cp<1, kCode12>(p, s, stream);
+    case 512: return by_code(code, [&](auto k) { return launch_gemv_cp<8, decltype(k)::value>(p, s, stream); });
+    case 256: return by_code(code, [&](auto k) { return launch_gemv_cp<4, decltype(k)::value>(p, s, stream); });
+    case 128: return by_code(code, [&](auto k) { return launch_gemv_cp<2, decltype(k)::value>(p, s, stream); });
+    case 64: return by_code(code, [&](auto k) { return launch_gemv_cp<1, decltype(k)::value>(p, s, stream); });
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1882,10 +1996,10 @@ cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const Laun
 cudaError_t launch_decompress(const TileParams& p, int tile_cols, int code,
                               const LaunchShape& s, cudaStream_t stream) {
   switch (tile_cols) {
-    case 512: return code == kCodeRank ? launch_decompress_t<8, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<8, kCode14>(p, s, stream) : launch_decompress_t<8, kCode12>(p, s, stream);
-    case 256: return code == kCodeRank ? launch_decompress_t<4, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<4, kCode14>(p, s, stream) : launch_decompress_t<4, kCode12>(p, s, stream);
-    case 128: return code == kCodeRank ? launch_decompress_t<2, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<2, kCode14>(p, s, stream) : launch_decompress_t<2, kCode12>(p, s, stream);
-    case 64: return code == kCodeRank ? launch_decompress_t<1, kCodeRank>(p, s, stream) : code == kCode14 ? launch_decompress_t<1, kCode14>(p, s, stream) : launch_decompress_t<1, kCode12>(p, s, stream);
+    case 512: return by_code(code, [&](auto k) { return launch_decompress_t<8, decltype(k)::value>(p, s, stream); });
+    case 256: return by_code(code, [&](auto k) { return launch_decompress_t<4, decltype(k)::value>(p, s, stream); });
+    case 128: return by_code(code, [&](auto k) { return launch_decompress_t<2, decltype(k)::value>(p, s, stream); });
+    case 64: return by_code(code, [&](auto k) { return launch_decompress_t<1, decltype(k)::value>(p, s, stream); });
     default: return cudaErrorInvalidValue;
   }
 }
@@ -1993,10 +2107,10 @@ cudaError_t launch_gemv_tc(const TileParams& p, const CUtensorMap& tmap, int til
       (p.tc_ksplit > 1 && p.tc_ksplit > tc_max_ksplit(p.tiles_c)))
     return cudaErrorInvalidValue;
   switch (tile_cols) {
-    case 512: return code == kCodeRank ? launch_gemv_tc_t<8, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<8, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<8, kCode12>(p, tmap, s.s, stream);
-    case 256: return code == kCodeRank ? launch_gemv_tc_t<4, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<4, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<4, kCode12>(p, tmap, s.s, stream);
-    case 128: return code == kCodeRank ? launch_gemv_tc_t<2, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<2, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<2, kCode12>(p, tmap, s.s, stream);
-    case 64: return code == kCodeRank ? launch_gemv_tc_t<1, kCodeRank>(p, tmap, s.s, stream) : code == kCode14 ? launch_gemv_tc_t<1, kCode14>(p, tmap, s.s, stream) : launch_gemv_tc_t<1, kCode12>(p, tmap, s.s, stream);
+    case 512: return by_code(code, [&](auto k) { return launch_gemv_tc_t<8, decltype(k)::value>(p, tmap, s.s, stream); });
+    case 256: return by_code(code, [&](auto k) { return launch_gemv_tc_t<4, decltype(k)::value>(p, tmap, s.s, stream); });
+    case 128: return by_code(code, [&](auto k) { return launch_gemv_tc_t<2, decltype(k)::value>(p, tmap, s.s, stream); });
+    case 64: return by_code(code, [&](auto k) { return launch_gemv_tc_t<1, decltype(k)::value>(p, tmap, s.s, stream); });
     default: return cudaErrorInvalidValue;
   }
 }
@@ -2012,7 +2126,7 @@ cudaError_t launch_gather_s(const GatherParams& g, int ctas, size_t smem, cudaSt
 
 template <int CP, int CODE>
 cudaError_t launch_gather_t(const GatherParams& g, int ctas, size_t smem, cudaStream_t stream) {
-  if constexpr (CODE == kCodeRank) {
+  if constexpr (CODE == kCodeRank || CODE == kCodeEsc) {
     return launch_gather_s<CP, CODE, 1>(g, ctas, smem, stream);
   } else {
     return g.streams == 2 ? launch_gather_s<CP, CODE, 2>(g, ctas, smem, stream)
@@ -2028,10 +2142,10 @@ cudaError_t launch_gather(const GatherParams& g, int sm_count, cudaStream_t stre
       (size_t)g.table_bytes + kGatherBarBytes + (size_t)kGatherWarps * g.stage_bytes;
   const int code = g.code;
   switch (g.tile_cols) {
-    case 512: return code == kCodeRank ? launch_gather_t<8, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<8, kCode14>(g, ctas, smem, stream) : launch_gather_t<8, kCode12>(g, ctas, smem, stream);
-    case 256: return code == kCodeRank ? launch_gather_t<4, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<4, kCode14>(g, ctas, smem, stream) : launch_gather_t<4, kCode12>(g, ctas, smem, stream);
-    case 128: return code == kCodeRank ? launch_gather_t<2, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<2, kCode14>(g, ctas, smem, stream) : launch_gather_t<2, kCode12>(g, ctas, smem, stream);
-    case 64: return code == kCodeRank ? launch_gather_t<1, kCodeRank>(g, ctas, smem, stream) : code == kCode14 ? launch_gather_t<1, kCode14>(g, ctas, smem, stream) : launch_gather_t<1, kCode12>(g, ctas, smem, stream);
+    case 512: return by_code(code, [&](auto k) { return launch_gather_t<8, decltype(k)::value>(g, ctas, smem, stream); });
+    case 256: return by_code(code, [&](auto k) { return launch_gather_t<4, decltype(k)::value>(g, ctas, smem, stream); });
+    case 128: return by_code(code, [&](auto k) { return launch_gather_t<2, decltype(k)::value>(g, ctas, smem, stream); });
+    case 64: return by_code(code, [&](auto k) { return launch_gather_t<1, decltype(k)::value>(g, ctas, smem, stream); });
     default: return cudaErrorInvalidValue;
   }
 }

@@ -27,8 +27,10 @@ constexpr uint32_t kErrLayout = 8u;    // shared memory not aligned as a kernel 
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
 
 // The exponent code a kernel reads: the prefix code through a 12-bit or a
-// 14-bit table peek, or the ranked unary code (variant NWR1, no table).
-constexpr int kCode12 = 0, kCode14 = 1, kCodeRank = 2;
+// 14-bit table peek, the ranked unary code (variant NWR1, no table), or the
+// prefix code through the 14-bit peek with runs of rare exponents stored
+// verbatim (variant NWE1).
+constexpr int kCode12 = 0, kCode14 = 1, kCodeRank = 2, kCodeEsc = 3;
 
 struct TileParams {
   const uint8_t* tiles;     // device: tile area of the blob
@@ -103,8 +105,8 @@ LaunchShape launch_shape(int64_t n_tiles, uint64_t max_chunk, uint64_t typical_c
 // sched_class_bytes(n_tiles) bytes (one class) laid out as nwc_format.h describes.
 void build_schedule(const uint32_t* index, int64_t n_tiles, const LaunchShape& s, uint8_t* out);
 
-// code: kCode12, kCode14 (lmax <= 7: two codes per table entry always) or
-// kCodeRank.
+// code: kCode12, kCode14 (lmax <= 7: two codes per table entry always),
+// kCodeRank or kCodeEsc.
 cudaError_t launch_gemv(const TileParams& p, int tile_cols, int code, const LaunchShape& s,
                         cudaStream_t stream);
 
@@ -180,7 +182,7 @@ struct GatherParams {
   uint32_t table_bytes;
   uint32_t stage_bytes;     // per warp: a tile's lane lengths and streams + slack
   int32_t streams;          // bit streams per lane and tile (1 or 2)
-  int32_t code;             // kCode12, kCode14 or kCodeRank
+  int32_t code;             // kCode12, kCode14, kCodeRank or kCodeEsc
   int32_t peek;             // table peek width (12 or 14)
   int32_t tile_cols;
   int64_t rows, cols, tiles_r, tiles_c;

@@ -55,7 +55,10 @@ nwc_status current_device(int* dev, int* sms, size_t* smem) {
 
 // The code kind the kernels read for a handle, and the table bytes a CTA loads.
 int code_of(const nwc_handle_s& h) {
-  return h.code_kind == 1 ? nwc::kCodeRank : h.lmax <= 7 ? nwc::kCode14 : nwc::kCode12;
+  return h.code_kind == 1   ? nwc::kCodeRank
+         : h.code_kind == 2 ? nwc::kCodeEsc
+         : h.lmax <= 7      ? nwc::kCode14
+                            : nwc::kCode12;
 }
 uint32_t table_bytes_of(const nwc_handle_s& h) {
   return nwc::device_table_bytes(h.lmax, h.code_kind == 1);
@@ -181,13 +184,18 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 // no C++ exception leaves the C ABI.
 nwc_status parse(const uint8_t* blob, uint64_t head_bytes, uint64_t bytes, nwc_handle_s* h,
                  const uint8_t** lens) {
-  // A well-defined layout that no kernel reads: NWB1 with 4 bit streams per
-  // lane (header offset 60 = S - 1).
+  // Well-defined layouts that no kernel reads: NWB1 with 4 bit streams per
+  // lane (header offset 60 = S - 1), NWE1 with lmax over 7.
   if (blob && head_bytes >= 64) {
     uint32_t magic, streams_m1;
     std::memcpy(&magic, blob, 4);
     std::memcpy(&streams_m1, blob + 60, 4);
     if (magic == nwc::kMagic && streams_m1 == 3) return NWC_ERR_UNSUPPORTED;
+    // NWE1 with codes longer than the kernels' 14-bit table allows.
+    uint32_t lmax;
+    std::memcpy(&lmax, blob + 12, 4);
+    if (magic == nwc::kEscMagic && lmax > nwc::kEscMaxLmax && lmax <= (uint32_t)nwc::kMaxLmax)
+      return NWC_ERR_UNSUPPORTED;
   }
   try {
     return nwc::parse_blob(blob, head_bytes, bytes, h, lens) ? NWC_OK : NWC_ERR_CORRUPT;
@@ -316,7 +324,7 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
   if (rows > (1ll << 40) || cols > (1ll << 40)) return NWC_ERR_INVALID_ARG;
   *out_plan = nullptr;
   uint32_t lmax = 0, tile_rows = 8, tile_cols = 512, threads = 0, code = NWC_CODE_PREFIX;
-  uint32_t streams = 1;
+  uint32_t streams = 1, keep = 16;
   if (opts) {
     if (opts->struct_size < offsetof(nwc_opts, code)) return NWC_ERR_INVALID_ARG;
     lmax = opts->lmax;
@@ -324,12 +332,17 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
     tile_cols = opts->tile_cols;
     threads = opts->threads;
     if (opts->struct_size >= offsetof(nwc_opts, streams)) code = opts->code;
-    if (opts->struct_size >= sizeof(nwc_opts) && opts->streams) streams = opts->streams;
+    if (opts->struct_size >= offsetof(nwc_opts, keep) && opts->streams) streams = opts->streams;
+    if (opts->struct_size >= sizeof(nwc_opts) && opts->keep) keep = opts->keep;
   }
-  if (code != NWC_CODE_PREFIX && code != NWC_CODE_RANK) return NWC_ERR_INVALID_ARG;
+  if (code != NWC_CODE_PREFIX && code != NWC_CODE_RANK && code != NWC_CODE_ESCAPE)
+    return NWC_ERR_INVALID_ARG;
   if (streams != 1 && streams != 2 && streams != 4) return NWC_ERR_INVALID_ARG;
-  if (code == NWC_CODE_RANK && streams != 1) return NWC_ERR_UNSUPPORTED;
+  if (code != NWC_CODE_PREFIX && streams != 1) return NWC_ERR_UNSUPPORTED;
   if (code == NWC_CODE_RANK && lmax > (uint32_t)nwc::kMaxRanks) return NWC_ERR_INVALID_ARG;
+  if (code == NWC_CODE_ESCAPE && keep > 256) return NWC_ERR_INVALID_ARG;
+  if (code == NWC_CODE_ESCAPE && lmax > nwc::kEscMaxLmax && lmax <= (uint32_t)nwc::kMaxLmax)
+    return NWC_ERR_UNSUPPORTED;
   if (lmax > (uint32_t)nwc::kMaxLmax) return NWC_ERR_INVALID_ARG;
   if (tile_rows != 8) return NWC_ERR_UNSUPPORTED;
   if (tile_cols != 64 && tile_cols != 128 && tile_cols != 256 && tile_cols != 512)
@@ -341,6 +354,8 @@ nwc_status nwc_plan(const uint16_t* w_host, int64_t rows, int64_t cols, const nw
     rc = code == NWC_CODE_RANK
              ? nwc::plan_build_rank(w_host, rows, cols, tile_cols, lmax ? lmax : nwc::kMaxRanks,
                                     threads, p)
+         : code == NWC_CODE_ESCAPE
+             ? nwc::plan_build_escape(w_host, rows, cols, tile_cols, lmax, keep, threads, p)
              : nwc::plan_build(w_host, rows, cols, tile_rows, tile_cols, lmax, threads, p,
                                streams);
   } catch (const std::bad_alloc&) {
@@ -483,7 +498,8 @@ nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes, nwc_handle_t* o
   if (cudaMemcpy(&hd, d_buf, sizeof(hd), cudaMemcpyDeviceToHost) != cudaSuccess)
     return NWC_ERR_CUDA;
   if (hd.magic == nwc::kMagic && hd.zero == 3) return NWC_ERR_UNSUPPORTED;
-  if ((hd.magic != nwc::kMagic && hd.magic != nwc::kRankMagic) || hd.total_bytes > d_bytes ||
+  if ((hd.magic != nwc::kMagic && hd.magic != nwc::kRankMagic && hd.magic != nwc::kEscMagic) ||
+      hd.total_bytes > d_bytes ||
       hd.tiles_off > hd.total_bytes ||
       hd.tiles_off < nwc::kIndexOffset)
     return NWC_ERR_CORRUPT;
@@ -545,9 +561,10 @@ nwc_status nwc_gather_rows(nwc_handle_t h, const int32_t* d_rows, int32_t n, uin
   g.table_bytes = table_bytes_of(*h);
   // Lane lengths and the longest streams a tile can hold, plus the readers'
   // slack.
-  const uint32_t max_chunk = h->code_kind == 1
-                                 ? nwc::max_rank_chunk_bytes(h->tile_cols, h->lmax)
-                                 : nwc::max_chunk_bytes(h->tile_cols, h->lmax, h->streams);
+  const uint32_t max_chunk = h->code_kind == 1   ? nwc::max_rank_chunk_bytes(h->tile_cols, h->lmax)
+                             : h->code_kind == 2 ? nwc::max_escape_chunk_bytes(h->tile_cols, h->lmax)
+                                                 : nwc::max_chunk_bytes(h->tile_cols, h->lmax,
+                                                                        h->streams);
   g.stage_bytes = max_chunk - nwc::raw_bytes(h->tile_cols) + 512;
   if ((size_t)g.table_bytes + 8ull * g.stage_bytes > smem) return NWC_ERR_UNSUPPORTED;
   g.peek = nwc::peek_bits(h->lmax);
@@ -585,7 +602,7 @@ nwc_status gemv_check(const nwc_handle_s* h, const uint16_t* d_x, const float* d
   if (!aligned(d_x, (h->cols & 1) ? 2 : 4) || !aligned(d_y, 4)) return NWC_ERR_INVALID_ARG;
   // A filler exponent of 255 (Inf/NaN) in padded columns would meet x = 0
   // (the ranked code's filler, e with raw byte 0, is always finite).
-  if (h->code_kind == 0 && h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0)
+  if (h->code_kind != 1 && h->filler == 255 && (h->cols % (int64_t)h->tile_cols) != 0)
     return NWC_ERR_UNSUPPORTED;
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return NWC_ERR_CUDA;

@@ -51,6 +51,22 @@ constexpr uint32_t kMagic = 0x3142574Eu;  // "NWB1"
 // the device image holds a 256-byte rank table in place of the decode table.
 constexpr uint32_t kRankMagic = 0x3152574Eu;  // "NWR1"
 constexpr int kMaxRanks = 7;
+// Variant "NWE1": rare exponents in verbatim runs ("Unweight", "Compressing
+// BF16 Weights": the most common exponents are Huffman-coded; a row of 64
+// weights holding any other exponent is stored whole).  NWB1's header, lens,
+// index and raw plane, with: the K most frequent exponent bytes kept (header
+// offset 60 holds K); run (g, m) of a tile = row g, columns 64 m .. 64 m + 63;
+// a run holding an exponent outside the kept set is verbatim; the code covers
+// the symbols of the other runs only (so a run is verbatim exactly when it
+// holds a symbol without a code).  A chunk is raw u8[8 tile_cols] | flags
+// u8[16] (bit m of byte g: run (g, m) verbatim) | the verbatim runs' exponent
+// bytes u8[64 n] in (g, m) order | lane lengths u8[32] | streams (one per lane,
+// the coded symbols only).  Header offset 104 holds the number of verbatim
+// runs (u64).  The kernels read it with lmax <= 7 (the 14-bit table).
+constexpr uint32_t kEscMagic = 0x3145574Eu;  // "NWE1"
+constexpr uint32_t kEscFlagBytes = 16;
+constexpr uint32_t kEscRunBytes = 64;
+constexpr uint32_t kEscMaxLmax = 7;
 constexpr uint32_t kVersion = 1;
 constexpr uint32_t kHeaderBytes = 128;
 constexpr uint32_t kLensOffset = 128;
@@ -204,6 +220,14 @@ constexpr uint32_t max_chunk_bytes(uint32_t tile_cols, uint32_t lmax, uint32_t s
                          ((2 * kTileRows * (tile_cols / 64) / streams * lmax + 7) / 8) +
                      15) /
                     16 * 16);
+}
+// Worst-case NWE1 chunk: every run either verbatim (64 bytes) or coded (4
+// lanes x 16 symbols of at most lmax bits), plus each lane's byte padding and
+// the 16-byte padding of the streams.
+constexpr uint32_t max_escape_chunk_bytes(uint32_t tile_cols, uint32_t lmax) {
+  return raw_bytes(tile_cols) + kEscFlagBytes + kLanes +
+         kTileRows * (tile_cols / 64) * (8 * lmax > kEscRunBytes ? 8 * lmax : kEscRunBytes) +
+         kLanes + 16;
 }
 // Bit streams per lane that the kernels read (1 or 2).
 constexpr uint32_t kMaxDeviceStreams = 2;

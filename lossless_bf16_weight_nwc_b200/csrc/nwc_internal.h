@@ -14,8 +14,12 @@ struct nwc_plan_s {
   uint32_t filler = 0;
   uint64_t coded_bits = 0;
   // Exponent code: 0 = canonical prefix code of bits 14..7 (NWB1), 1 = ranked
-  // unary code of bits 14..8 with the sign bit (NWR1).
+  // unary code of bits 14..8 with the sign bit (NWR1), 2 = the prefix code of
+  // the kept exponents with verbatim runs for the rest (NWE1).
   uint32_t code_kind = 0;
+  uint32_t keep = 0;                         // NWE1: K, the kept exponents
+  uint64_t n_escaped = 0;                    // NWE1: verbatim runs
+  std::vector<uint8_t> esc_flags;            // NWE1: 8 bytes a tile, bit m of byte g
   uint32_t streams = 1;                      // bit streams per lane and tile (1, 2, 4)
   uint32_t ranks = 0;                        // NWR1: R
   uint8_t rank_table[nwc::kMaxRanks] = {};   // NWR1: ranked values of e
@@ -36,7 +40,7 @@ struct nwc_handle_s {
   int64_t rows = 0, cols = 0;
   uint32_t tile_cols = 512, lmax = 7, filler = 0;
   uint32_t streams = 1;    // bit streams per lane and tile (1 or 2)
-  uint32_t code_kind = 0;  // 0: prefix code (NWB1), 1: ranked unary code (NWR1)
+  uint32_t code_kind = 0;  // 0: prefix code (NWB1), 1: ranked unary code (NWR1), 2: NWE1
   int64_t tiles_r = 0, tiles_c = 0, tiles = 0;
   uint64_t index_off = 0, tiles_off = 0, blob_bytes = 0, table_off = 0, sched_off = 0,
            scratch_off = 0;
@@ -64,10 +68,14 @@ namespace nwc {
 int plan_build(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_rows,
                uint32_t tile_cols, uint32_t lmax, uint32_t threads, nwc_plan_s* plan,
                uint32_t streams = 1);
-// The ranked unary code (NWR1) with `ranks` ranks (1..7); the plan has no
-// device image (device_bytes = 0).
+// The ranked unary code (NWR1) with `ranks` ranks (1..7).
 int plan_build_rank(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_cols,
                     uint32_t ranks, uint32_t threads, nwc_plan_s* plan);
+// The kept-exponent prefix code with verbatim runs (NWE1): the `keep` (1..256)
+// most frequent exponents coded with lengths <= lmax (0 = 7; at most 7, the
+// kernels' 14-bit table).
+int plan_build_escape(const uint16_t* w, int64_t rows, int64_t cols, uint32_t tile_cols,
+                      uint32_t lmax, uint32_t keep, uint32_t threads, nwc_plan_s* plan);
 void encode_blob(const nwc_plan_s& plan, const uint16_t* w, uint8_t* blob);
 bool code_lengths(const uint64_t cnt[256], uint32_t lmax, uint8_t len[256]);
 void canonical_codes(const uint8_t len[256], uint32_t code[256]);

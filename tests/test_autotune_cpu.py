@@ -92,7 +92,8 @@ def test_default_candidates_cover_the_kernels():
     large = autotune.default_candidates(16)
     assert {s.kernel for s in small} == {"cuda"}
     assert {s.kernel for s in large} == {"cuda", "tensor"}
-    assert {s.code for s in large} == {"prefix", "rank"} and {s.streams for s in large} == {1, 2}
+    assert {s.code for s in large} == {"prefix", "rank", "escape"}
+    assert {s.streams for s in large} == {1, 2}
     assert autotune.validate_candidates(large) == large
 
 
@@ -100,7 +101,8 @@ def test_arguments_checked():
     fake = Fake({})
     for bad in (Strategy(100), Strategy(512, 13), Strategy(512, 0, 3), Strategy(code="huffman"),
                 Strategy(kernel="cpu"), Strategy(streams=2, code="rank"),
-                Strategy(lmax=8, code="rank")):
+                Strategy(lmax=8, code="rank"), Strategy(streams=2, code="escape"),
+                Strategy(lmax=8, code="escape")):
         with pytest.raises(ValueError):
             tuner(fake).tune(W, 1, candidates=[bad])
     with pytest.raises(TypeError):

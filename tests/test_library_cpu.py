@@ -162,7 +162,7 @@ def test_plan_options_code_field(lib):
     import ctypes
     w = synth.matrix(synth.MatrixSpec("w", 16, 256, "normal", 0.02, 0), 1)
     with pytest.raises(lib.NwcError):
-        lib.nwc_plan(w, code=2)
+        lib.nwc_plan(w, code=3)
     with pytest.raises(lib.NwcError):                   # at most 7 ranks
         lib.nwc_plan(w, lmax=8, code=lib.NWC_CODE_RANK)
     # The options layout without `code` still means the prefix code.
