@@ -2013,9 +2013,10 @@ bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_streams, uint32_t t
   const uint32_t bar_off = (uint32_t)xstage_offset(table_bytes);
   const uint32_t a_off = (bar_off + kTcBarBytes + 1023u) / 1024u * 1024u;
   const uint32_t bstage = (uint32_t)n * 128u;
-  // Candidates in order of preference: every decode warp's streams resident
-  // (full), fewest rounds, smallest split, two x stages, three A stages,
-  // largest ring.
+  // Candidates in order of preference: two x stages (with one, a team's next x
+  // chunk can only be fetched once its last MMAs completed, which serialises
+  // the TMA latency with every chunk), every decode warp's streams resident
+  // (full), fewest rounds, smallest split, three A stages, largest ring.
   bool found = false;
   TcShape best{};
   int64_t best_key[6] = {0, 0, 0, 0, 0, 0};
@@ -2060,8 +2061,8 @@ bool tc_shape(int64_t tiles_r, int64_t tiles_c, uint64_t max_streams, uint32_t t
             if (warps_resident > per_cta) warps_resident = per_cta;
             const int64_t full = ring >= (size_t)warps_resident * (size_t)max_streams ? 1 : 0;
             const int64_t rounds = (rows_c + R - 1) / R * ((cols_c + TT - 1) / TT);
-            // Larger is better: resident, -rounds, -split, x stages, A stages, ring.
-            const int64_t key[6] = {full, -rounds, -KS, SB, NA, (int64_t)ring};
+            // Larger is better: x stages, resident, -rounds, -split, A stages, ring.
+            const int64_t key[6] = {SB, full, -rounds, -KS, NA, (int64_t)ring};
             bool better = !found;
             for (int k = 0; k < 6 && !better; ++k) {
               if (key[k] != best_key[k]) {

@@ -132,20 +132,27 @@ def rounds(info, tiles_r, tiles_c):
     return -(-rows_c // info["rows"]) * -(-cols_c // info["teams"])
 
 
-def test_tc_shape_takes_the_fewest_rounds_with_every_warp_resident():
-    """A 4096 x 4096 matrix (512 x 8 tiles) on 148 SMs: K split in two, 74 row
-    ranges of 6 or 7 row tiles x 4 column blocks, one M-group of 7 rows and 4
-    teams: every decode warp decodes one tile, with every warp's streams
-    resident.  Without the split, 4 rows x 8 column blocks would take two
-    rounds of at most 30 warps."""
+def test_tc_shape_prefers_two_x_stages_then_the_fewest_rounds():
+    """A 4096 x 4096 matrix (512 x 8 tiles) on 148 SMs.  With accumulators of
+    16 or 32 columns the x stages are small: two per team, K split in two, 74
+    row ranges of 6 or 7 row tiles x 4 column blocks, one M-group of 7 rows and
+    4 teams, every decode warp one tile with its streams resident.  At 64
+    columns two x stages per team take 64 KiB: they are kept (with one, a
+    team's next x chunk waits for its last MMAs), and the shape with every
+    warp's streams resident is then 4 teams of 4 rows without a split, in two
+    rounds."""
     blob = blob_of(4096, 4096)
     _, _, _, _, _, index = header(blob)
     streams = int((16 * np.diff(index) - 4096).max())
-    for rows_of_x in (1, 64):
+    for rows_of_x in (1, 17):
         info = lib.nwc_tc_schedule_describe(blob, rows_of_x=rows_of_x)[0]
         assert (info["ksplit"], info["ctas"], info["rows"], info["teams"]) == (2, 148, 7, 4)
-        assert rounds(info, 512, 8) == 1
+        assert info["x_stages"] == 2 and rounds(info, 512, 8) == 1
         assert info["ring_bytes"] >= 28 * streams
+    info = lib.nwc_tc_schedule_describe(blob, rows_of_x=64)[0]
+    assert (info["ksplit"], info["ctas"], info["rows"], info["teams"]) == (1, 148, 4, 4)
+    assert info["x_stages"] == 2 and rounds(info, 512, 8) == 2
+    assert info["ring_bytes"] >= 18 * streams
 
 
 @pytest.mark.parametrize("rows,cols,best", [(14336, 4096, 4), (4096, 14336, 4), (1024, 4096, 1),
