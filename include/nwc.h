@@ -165,7 +165,7 @@ nwc_status nwc_compress(nwc_plan_t plan, const uint16_t* w_host, void* d_buf,
                         nwc_handle_t* out_handle);
 
 /* Encode into a host buffer (>= host_blob_bytes).  The bytes are the
- * serialisable "NWB1" blob. */
+ * serialisable blob of the plan's code: "NWB1", "NWR1" or "NWE1". */
 nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob,
                              uint64_t blob_bytes);
 
@@ -175,15 +175,21 @@ nwc_status nwc_compress_host(nwc_plan_t plan, const uint16_t* w_host, void* blob
  * Errors: INVALID_ARG (null), CORRUPT (the blob does not parse: a header field
  * inconsistent with the others or with blob_bytes, code lengths over lmax or
  * not a prefix code, an index that is not increasing or whose chunk sizes fall
- * outside what the geometry allows), NOMEM (the host copy of the index). */
+ * outside what the geometry allows), UNSUPPORTED (a valid layout that no kernel
+ * reads, as nwc_upload_blob), NOMEM (the host copy of the index). */
 nwc_status nwc_blob_device_bytes(const void* blob, uint64_t blob_bytes,
                                  uint64_t* device_bytes);
 
-/* Validate a host blob, upload it into d_buf, and build its decode table and
- * launch schedule for the current device.  The call is synchronous: it returns
- * after the copies finish.
+/* Validate a host blob ("NWB1", "NWR1" or "NWE1"), upload it into d_buf, and
+ * build its decode table and launch schedule for the current device.  The call
+ * is synchronous: it returns after the copies finish.
  * Errors: CORRUPT (header, code lengths or index do not parse, as for
- * nwc_blob_device_bytes), INVALID_ARG, NOMEM, CUDA. */
+ * nwc_blob_device_bytes), UNSUPPORTED (a valid layout no kernel reads: NWB1
+ * with 4 streams per lane, NWE1 with lmax over 7), INVALID_ARG, NOMEM, CUDA.
+ * The tile area is not read on the host: a corrupt chunk (a stream without a
+ * valid code, an NWE1 flag field naming a group past the tile or more runs than
+ * the chunk holds) is found by the kernels, which stay inside their buffers and
+ * set the handle's corrupt bit (nwc_get_device_error). */
 nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
                            uint64_t d_bytes, nwc_stream_t stream,
                            nwc_handle_t* out_handle);
@@ -192,8 +198,8 @@ nwc_status nwc_upload_blob(const void* blob, uint64_t blob_bytes, void* d_buf,
  * nwc_compress or nwc_upload_blob, possibly copied elsewhere).  The call is
  * synchronous: it reads the header, code lengths and index back to the host,
  * then rewrites the image's launch-schedule area for the current device (the
- * blob and the decode table are not written).
- * Errors: CORRUPT, INVALID_ARG, NOMEM, CUDA. */
+ * blob and the decode table are not written).  Any of the three formats.
+ * Errors: CORRUPT, UNSUPPORTED (as nwc_upload_blob), INVALID_ARG, NOMEM, CUDA. */
 nwc_status nwc_handle_from_device(void* d_buf, uint64_t d_bytes,
                                   nwc_handle_t* out_handle);
 
