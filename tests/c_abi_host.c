@@ -3,8 +3,8 @@
  * must be able to plan, encode and inspect a matrix through the ABI alone.
  *
  * Usage: c_abi_host OUT_PREFIX
- * Writes OUT_PREFIX.nwb1 (prefix code) and OUT_PREFIX.nwr1 (ranked unary code)
- * for the 24 x 200 matrix w[i][j] = 0x3C00 + (37 i + 11 j) % 1024 (BF16 bit
+ * Writes OUT_PREFIX.nwb1 (prefix code), OUT_PREFIX.nwr1 (ranked unary code)
+ * and OUT_PREFIX.nwe1 (verbatim runs for rare exponents) for the 24 x 200 matrix w[i][j] = 0x3C00 + (37 i + 11 j) % 1024 (BF16 bit
  * patterns), and prints one "key value" line per checked quantity. */
 #include <stdio.h>
 #include <stdlib.h>
@@ -90,6 +90,18 @@ int main(int argc, char** argv) {
   snprintf(path, sizeof path, "%s.nwr1", argv[1]);
   if (encode(w, &opts, path, &dev)) return 1;
   printf("nwr1_device_bytes %llu\n", (unsigned long long)dev);
+
+  /* Verbatim runs for rare exponents: 4 kept exponents, 128-column tiles. */
+  memset(&opts, 0, sizeof opts);
+  opts.struct_size = sizeof opts;
+  opts.tile_rows = 8;
+  opts.tile_cols = 128;
+  opts.threads = 2;
+  opts.code = NWC_CODE_ESCAPE;
+  opts.keep = 4;
+  snprintf(path, sizeof path, "%s.nwe1", argv[1]);
+  if (encode(w, &opts, path, &dev)) return 1;
+  printf("nwe1_device_bytes %llu\n", (unsigned long long)dev);
 
   /* Argument errors come back as status codes. */
   nwc_plan_t plan = NULL;

@@ -40,6 +40,10 @@ def test_c_caller_matches_oracle(c_program, orc):
     nwr1 = np.fromfile(prefix + ".nwr1", dtype=np.uint8)
     assert np.array_equal(nwb1, orc.encode(w, lmax=7))
     assert np.array_equal(nwr1, orc.rank_encode(w, tile_cols=64, ranks=3))
+    nwe1 = np.fromfile(prefix + ".nwe1", dtype=np.uint8)
+    assert np.array_equal(nwe1, orc.escape_encode(w, tile_cols=128, lmax=7, keep=4))
+    assert int.from_bytes(nwe1[104:112].tobytes(), "little") > 0      # some runs verbatim
+    assert int(vals["nwe1_device_bytes"]) > nwe1.size + 65536         # blob, table, schedules
     assert int(vals["nwb1_device_bytes"]) == int(vals["blob_device_bytes"]) > nwb1.size
     assert int(vals["schedule_tiles"]) == 3 and int(vals["schedule_ctas"]) == 3
     assert int(vals["corrupt_status"]) == 4          # NWC_ERR_CORRUPT
