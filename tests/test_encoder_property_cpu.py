@@ -1,7 +1,7 @@
 """Property tests (hypothesis, CPU): for random shapes, tile widths, code
 limits, rank counts, streams per lane and bit patterns -- NaN payloads, infinities, signed zeros
 and subnormals included -- the library's host encoder writes exactly the
-oracle's bytes for both codes, the oracle decodes them back to the input, and
+oracle's bytes for every code, the oracle decodes them back to the input, and
 the library's size and schedule checks accept them."""
 import numpy as np
 import pytest
@@ -77,3 +77,29 @@ def test_rank_code_matches_oracle(lib, orc, w, tile_cols, ranks, threads):
         lib.nwc_plan_destroy(plan)
     assert np.array_equal(blob, orc.rank_encode(w, tile_cols=tile_cols, ranks=ranks or 7))
     assert np.array_equal(orc.rank_decode(blob), w)
+
+
+@settings(max_examples=150, deadline=None, suppress_health_check=[HealthCheck.too_slow])
+@given(w=matrices(), tile_cols=st.sampled_from([64, 128, 256, 512]),
+       keep=st.sampled_from([1, 2, 5, 16, 64, 128, 256]), lmax=st.sampled_from([0, 5, 7]),
+       threads=st.integers(1, 4))
+def test_escape_code_matches_oracle(lib, orc, w, tile_cols, keep, lmax, threads):
+    """The verbatim-run format (NWE1): the library's bytes are the oracle's, or
+    both refuse (more coded exponents than lmax bits admit)."""
+    try:
+        ref = orc.escape_encode(w, tile_cols=tile_cols, lmax=lmax or 7, keep=keep)
+    except orc.OracleError:
+        with pytest.raises(lib.NwcError):
+            lib.nwc_plan(w, lmax=lmax, tile_cols=tile_cols, threads=threads,
+                         code=lib.NWC_CODE_ESCAPE, keep=keep)
+        return
+    plan = lib.nwc_plan(w, lmax=lmax, tile_cols=tile_cols, threads=threads,
+                        code=lib.NWC_CODE_ESCAPE, keep=keep)
+    try:
+        blob = lib.nwc_compress_host(plan, w)
+        dev_bytes, _ = lib.nwc_plan_size(plan)
+    finally:
+        lib.nwc_plan_destroy(plan)
+    assert np.array_equal(blob, ref)
+    assert np.array_equal(orc.escape_decode(blob), w)
+    assert lib.nwc_blob_device_bytes(blob) == dev_bytes
