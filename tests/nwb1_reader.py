@@ -1,5 +1,6 @@
 """A second, pure-Python reader of the NWB1 blob format (test helper), with 1,
-2 or 4 bit streams per lane.
+2 or 4 bit streams per lane, and of its variant NWE1 (verbatim runs for rare
+exponents).
 
 Written from the format statement alone, in a different language and style
 from the oracle's C++ decoder, so that the encoder is checked against the
@@ -14,9 +15,10 @@ def parse(blob: bytes):
     (magic, version, hdr, lmax, rows, cols, tile_rows, tile_cols, tiles_r, tiles_c,
      filler, zero, lens_off, index_off, tiles_off, total, coded_bits) = struct.unpack_from(
         "<IIIIQQIIQQIIQQQQQ", b, 0)
-    assert magic == 0x3142574E and version == 1 and hdr == 128, "header"
+    assert magic in (0x3142574E, 0x3145574E) and version == 1 and hdr == 128, "header"
     assert total == len(b), "total bytes"
-    streams = zero + 1              # bit streams per lane and tile
+    verbatim = magic == 0x3145574E  # NWE1: offset 60 holds the kept exponents
+    streams = 1 if verbatim else zero + 1   # bit streams per lane and tile
     assert streams in (1, 2, 4), "streams per lane"
     lens = list(b[lens_off:lens_off + 256])
     n_tiles = tiles_r * tiles_c
@@ -24,7 +26,8 @@ def parse(blob: bytes):
     return dict(lmax=lmax, rows=rows, cols=cols, tile_rows=tile_rows, tile_cols=tile_cols,
                 tiles_r=tiles_r, tiles_c=tiles_c, filler=filler, lens=lens,
                 index=index, tiles_off=tiles_off, total=total, coded_bits=coded_bits,
-                streams=streams)
+                streams=streams, verbatim=verbatim, kept=zero if verbatim else None,
+                verbatim_runs=struct.unpack_from("<Q", b, 104)[0] if verbatim else None)
 
 
 def codebook(lens):
@@ -60,8 +63,19 @@ def decode(blob: bytes) -> np.ndarray:
         c0 = h["tiles_off"] + 16 * h["index"][u]
         c1 = h["tiles_off"] + 16 * h["index"][u + 1]
         raw = b[c0:c0 + tr * tc]
-        lane_len = b[c0 + tr * tc:c0 + tr * tc + n_streams]
-        bits = sequence_bits(b[c0 + tr * tc + n_streams:c1])
+        head = c0 + tr * tc
+        runs = {}                   # NWE1: (row, group) -> its 64 verbatim exponent bytes
+        if h["verbatim"]:
+            flags = b[head:head + 16]
+            at = head + 16
+            for r in range(tr):
+                for m in range(tc // 64):
+                    if flags[r] >> m & 1:
+                        runs[(r, m)] = b[at:at + 64]
+                        at += 64
+            head = at
+        lane_len = b[head:head + n_streams]
+        bits = sequence_bits(b[head + n_streams:c1])
         start = 0
         for sigma in range(n_streams):
             # Stream sigma: lane sigma // S, the lane's symbol pairs q with q % S == sigma % S.
@@ -70,15 +84,18 @@ def decode(blob: bytes) -> np.ndarray:
             start += 8 * lane_len[sigma]
             p = 0
             for k in [k for k in range(per_lane) if (k // 2) % S == sigma % S]:
-                q = p + 1
-                while s[p:q] not in book:
-                    q += 1
-                    assert q - p <= h["lmax"], "no code"
-                sym = book[s[p:q]]
-                p = q
-                rb = raw[(k // 16) * 512 + 16 * t + k % 16]
                 r = t // 4
                 c = 64 * (k // 16) + 16 * (t % 4) + k % 16
+                if (r, k // 16) in runs:
+                    sym = runs[(r, k // 16)][c - 64 * (k // 16)]
+                else:
+                    q = p + 1
+                    while s[p:q] not in book:
+                        q += 1
+                        assert q - p <= h["lmax"], "no code"
+                    sym = book[s[p:q]]
+                    p = q
+                rb = raw[(k // 16) * 512 + 16 * t + k % 16]
                 row, col = i * tr + r, j * tc + c
                 if row < rows and col < cols:
                     out[row, col] = ((rb >> 7) << 15) | (sym << 7) | (rb & 0x7F)

@@ -9,6 +9,7 @@ holding any other exponent stored verbatim):
   from the format statement (not from the oracle's code);
 * the bits per weight equal the costing of the format-variant study;
 * a matrix whose every run is escaped has the closed-form size;
+* an independent pure-Python reader (tests/nwb1_reader.py) decodes the blobs;
 * round trip over all 65,536 BF16 patterns, odd shapes, every tile width and
   kept count, and the workload generators;
 * blobs that break the format are refused;
@@ -199,6 +200,21 @@ def test_bits_per_weight_match_the_variant_costing(orc, name):
         esc = _u64(blob, 104)
         bits = _u64(blob, 96) + 8 * (n - 64 * esc) + 16 * 64 * esc + runs
         assert bits / n == pytest.approx(escape_rows_cost(orc, w, lmax=lmax), rel=1e-12)
+
+
+@pytest.mark.parametrize("shape,tile_cols,keep", [((9, 65), 64, 2), ((40, 300), 128, 4),
+                                                   ((16, 1030), 512, 6), ((8, 256), 256, 1)])
+def test_independent_reader_decodes_oracle_blobs(orc, shape, tile_cols, keep):
+    """The pure-Python reader (tests/nwb1_reader.py), written from the format
+    statement, reads the oracle's NWE1 blobs back to the input: the encoder is
+    checked against the format, not only against the oracle's own decoder."""
+    import nwb1_reader
+    rng = np.random.default_rng(sum(shape) + keep)
+    w = synth.to_bf16_bits(rng.standard_t(2, size=shape) * 0.02)
+    blob = orc.escape_encode(w, tile_cols=tile_cols, lmax=7, keep=keep)
+    h = nwb1_reader.parse(blob.tobytes())
+    assert h["verbatim"] and h["kept"] == keep and h["verbatim_runs"] > 0
+    assert np.array_equal(nwb1_reader.decode(blob.tobytes()), w)
 
 
 def test_all_runs_escaped_closed_form(orc):
