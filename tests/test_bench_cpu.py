@@ -71,3 +71,19 @@ def test_traffic_summary_used_only_for_the_kernel_code_it_was_taken_on(tmp_path,
             assert got == pytest.approx(entry["dram_bytes_per_launch"])
         else:
             assert got is None
+
+
+def test_traffic_key_names_the_compressed_format():
+    """The default format has no suffix; another code or stream count has its own
+    key, so a line for one format never reports another format's traffic."""
+    import argparse
+    ns = lambda **kw: argparse.Namespace(**{"code": "prefix", "streams": 1, **kw})  # noqa: E731
+    assert bench.format_suffix(ns()) == ""
+    assert bench.format_suffix(ns(code="escape")) == "_escape"
+    assert bench.format_suffix(ns(code="rank", streams=1)) == "_rank"
+    assert bench.format_suffix(ns(streams=2)) == "_s2"
+    with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+        data = json.load(f)
+    assert "attn_4096_outliers_escape/b1" in data
+    assert data["attn_4096_outliers_escape/b1"]["dram_bytes_per_launch"] != \
+        data["attn_4096_outliers/b1"]["dram_bytes_per_launch"]
