@@ -68,6 +68,10 @@ def parse_args():
                     help="exponent code: the length-limited prefix code (NWB1), the ranked "
                          "unary code (NWR1, 7 ranks) or the prefix code of the 16 most "
                          "frequent exponents with verbatim runs for the rest (NWE1)")
+    ap.add_argument("--lmax", type=int, default=0,
+                    help="code length limit of the compressed matrices (0: the library's "
+                         "automatic choice, 7 unless a matrix has more than 128 exponents; "
+                         "8..12 take the 16 KiB table of 12-bit peeks)")
     ap.add_argument("--tc-min-batch", type=int, default=None,
                     help="smallest batch that takes the tensor-core kernel (default: the "
                          "library's, 17; 0 = never)")
@@ -110,7 +114,8 @@ def kernel_source_hash() -> str:
 def format_suffix(args) -> str:
     """Key suffix of a non-default compressed format in the traffic summary."""
     return ("" if args.code == "prefix" else f"_{args.code}") + \
-        ("" if args.streams == 1 else f"_s{args.streams}")
+        ("" if args.streams == 1 else f"_s{args.streams}") + \
+        ("" if not getattr(args, "lmax", 0) else f"_l{args.lmax}")
 
 
 def profile_traffic(workload: str, batch: int) -> float | None:
@@ -359,7 +364,7 @@ def run_stack(args) -> None:
                            else synth.stacked_matrix(parts_of[sp.name], wl.seed))
         comp[sp.name] = _lib.CompressedMatrix.compress(host_w[sp.name], device=dev,
                                                        streams=args.streams,
-                                                       code=CODES[args.code])
+                                                       code=CODES[args.code], lmax=args.lmax)
     sets = [{sp.name: comp[sp.name] for sp in layer0}]
     second = {}
     for sp in layer0:
@@ -508,7 +513,7 @@ def run_stack(args) -> None:
                    f"({n_layers} layers x {len(layer0)} + lm_head), one CUDA graph",
                    "layer": [f"{g} {sp.rows}x{sp.cols}" for (g, _), sp in zip(units, layer0)],
                    "fused": bool(args.fuse), "streams_per_lane": args.streams,
-                   "code": args.code,
+                   "code": args.code, "lmax": args.lmax,
                    "weights": "layer 0 generated, two device copies alternating over the layers; "
                               f"lm_head = its first {synth.HEAD_BLOCK_ROWS} rows repeated",
                    "l2": "inputs larger than L2: every layer is larger than L2",
@@ -559,7 +564,7 @@ def run_matrix(args):
     w = synth.matrix(spec, wl.seed)
     x_host = synth.activations(wl.seed, batch, spec.cols)
     first = _lib.CompressedMatrix.compress(w, device=dev, streams=args.streams,
-                                           code=CODES[args.code])
+                                           code=CODES[args.code], lmax=args.lmax)
     image_bytes = first.compressed_bytes   # blob, table and schedules (no scratch)
     copies = max(2, int(np.ceil(2.2 * L2_BYTES / image_bytes)))
     copies = min(copies, args.steps) if args.steps >= 2 else copies
@@ -739,7 +744,7 @@ def run_matrix(args):
         "data": "synthetic",
         "config": {"workload": args.workload, "matrix": f"{spec.rows}x{spec.cols}",
                    "batch": batch, "values": spec.kind, "streams_per_lane": args.streams,
-                   "code": args.code,
+                   "code": args.code, "lmax": args.lmax,
                    "l2": f"inputs larger than L2: {copies} rotating compressed copies "
                          f"({copies * image_bytes / 2**20:.0f} MiB)",
                    "launch": "CUDA graph replay", "parallelism": f"replicas x{world}"},
@@ -821,7 +826,7 @@ def run_matrix_sharded(args):
     w = synth.matrix(spec, wl.seed)
     x_host = synth.activations(wl.seed, batch, spec.cols)
     sm = ShardedMatrix.compress(w, group=None, device=dev, streams=args.streams,
-                                code=CODES[args.code])
+                                code=CODES[args.code], lmax=args.lmax)
     local = sm.local
     image_bytes = local.compressed_bytes if local is not None else 0
     copies = max(2, int(np.ceil(2.2 * L2_BYTES / max(image_bytes, 1)))) if local else 1
